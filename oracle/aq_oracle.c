@@ -1,0 +1,348 @@
+/*
+ * Oracle for group-wise affine weight-only quantization and the quantized
+ * matmul that consumes it.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, obviously correct
+ * CPU statement of what the CUDA library computes.  Only the test suite, the
+ * smoke check and the CPU-baseline leg of the benchmark may load it.  It shares
+ * no code, header, table or helper with the CUDA path, and it never calls it.
+ *
+ * What it follows (page titles and sections of the source pages):
+ *  - "Quantizing a Model for MLX", section "What MLX quantization stores":
+ *    weights are cut into contiguous groups; each group has its own scale and
+ *    offset, stored in fp16 beside the integer codes, which are packed several
+ *    to a machine word.
+ *  - "metalworking — MLX Quantization", section "Mechanics": each group of
+ *    32/64/128 values along a row stores one scale, one bias and 2..8-bit
+ *    codes, with w ~= code * scale + bias.
+ *  - "anllm Tutorial 10: Quantization", section 3 "Packing Multiple Weights into
+ *    One Word": code j of a word sits at bit shift bits*j (shift, then mask);
+ *    dequantization is values * scales + biases with the group's scale and
+ *    bias repeated over its group_size values (section 2 "Group Quantization":
+ *    groups run along in_features, i.e. along K within one output row).
+ *  - Same tutorial, section 5 "Quantized Matrix Multiply": y = x @ W^T, and the
+ *    fused product equals dequantize-then-multiply.
+ *
+ * Readings where the pages are silent (each is also listed in the design notes):
+ *  - scale = (max - min) / (2^bits - 1) and bias = min, both computed in fp32
+ *    and rounded to fp16 (round to nearest, ties to even, subnormals kept).
+ *  - codes are computed from the STORED (fp16) scale and bias:
+ *        q = clamp(rint_even(fp32(fp32(w - bias16) / scale16)), 0, 2^bits - 1)
+ *    with IEEE correctly rounded fp32 subtraction and division.
+ *    A group whose fp16 scale is zero gets all codes 0.
+ *  - 3-bit codes form one contiguous LSB-first bitstream per row (32 codes in
+ *    3 words); every row starts on a word boundary.
+ *  - dequantized value: fp32(q * scale16 + bias16) with a single rounding (the
+ *    exact product-sum fits in fp64, so it is formed there and rounded once),
+ *    then rounded to bf16 for the bf16 output.
+ *  - matmul reference: y[m][n] = sum_k x[m][k] * (q*scale16 + bias16), exact
+ *    terms summed in fp64.
+ *
+ * Parity status: every function here is pinned by the not-gpu tests (closed
+ * forms from the pages, hand-derived fixtures, brute force, an independent
+ * NumPy implementation); none is "parity unpinned".
+ *
+ * Build: gcc -O2 -fno-fast-math -ffp-contract=off -fopenmp -shared -fPIC.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+
+/* ------------------------------------------------------------------------ */
+/* IEEE binary16 / bfloat16 rounding written out from the format definitions */
+/* ------------------------------------------------------------------------ */
+
+/* Round a finite double to the nearest value with `mant_bits` fraction bits
+ * and minimum normal exponent `emin` (ties to even), returning the rounded
+ * value as a double.  Values below 2^emin are rounded on the subnormal grid
+ * 2^(emin - mant_bits).  rint() runs in the default round-to-nearest-even mode. */
+static double round_to_format(double v, int mant_bits, int emin)
+{
+    if (v == 0.0 || !isfinite(v)) return v;
+    double a = fabs(v);
+    int ex;
+    frexp(a, &ex);          /* a = f * 2^ex with f in [0.5, 1) */
+    int e = ex - 1;         /* a in [2^e, 2^(e+1)) */
+    if (e < emin) e = emin; /* subnormal range shares the quantum of 2^emin */
+    double quantum = ldexp(1.0, e - mant_bits);
+    double r = rint(a / quantum) * quantum; /* a/quantum is exact (power of 2) */
+    return copysign(r, v);
+}
+
+/* fp16 bit pattern of the nearest binary16 value to v (v exactly a float). */
+static uint16_t f16_bits_from_double(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v)) return 0x7e00u;
+    double r = fabs(round_to_format(v, 10, -14));
+    if (isinf(v) || r >= 65536.0) return sign | 0x7c00u; /* overflow -> inf */
+    if (r == 0.0) return sign;
+    int ex;
+    frexp(r, &ex);
+    int e = ex - 1;
+    if (e < -14) { /* subnormal: value = m * 2^-24 */
+        uint16_t m = (uint16_t)ldexp(r, 24);
+        return sign | m;
+    }
+    uint16_t mant = (uint16_t)(ldexp(r, 10 - e) - 1024.0);
+    return sign | (uint16_t)((e + 15) << 10) | mant;
+}
+
+static double f16_value(uint16_t h)
+{
+    int sign = (h >> 15) & 1, exp = (h >> 10) & 0x1f, mant = h & 0x3ff;
+    double v;
+    if (exp == 0)
+        v = ldexp((double)mant, -24);
+    else if (exp == 31)
+        v = mant ? NAN : INFINITY;
+    else
+        v = ldexp(1024.0 + mant, exp - 25);
+    return sign ? -v : v;
+}
+
+/* bf16 bit pattern of the nearest bfloat16 value to v. */
+static uint16_t bf16_bits_from_double(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v)) return 0x7fc0u;
+    double r = fabs(round_to_format(v, 7, -126));
+    if (isinf(v) || r >= ldexp(1.0, 128)) return sign | 0x7f80u;
+    if (r == 0.0) return sign;
+    int ex;
+    frexp(r, &ex);
+    int e = ex - 1;
+    if (e < -126) {
+        uint16_t m = (uint16_t)ldexp(r, 133);
+        return sign | m;
+    }
+    uint16_t mant = (uint16_t)(ldexp(r, 7 - e) - 128.0);
+    return sign | (uint16_t)((e + 127) << 7) | mant;
+}
+
+static double bf16_value(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Exposed for the pins: element-wise conversions. */
+void oracle_f16_round(const float *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = f16_bits_from_double((double)in[i]);
+}
+
+void oracle_bf16_round(const float *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = bf16_bits_from_double((double)in[i]);
+}
+
+void oracle_f16_to_double(const uint16_t *in, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = f16_value(in[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Argument checks shared by the entry points of this file                  */
+/* ------------------------------------------------------------------------ */
+
+static int bad_shape(int64_t N, int64_t K, int G, int bits)
+{
+    if (N <= 0 || K <= 0) return 1;
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) return 1;
+    if (!(G == 32 || G == 64 || G == 128)) return 1;
+    if (K % G != 0) return 1;
+    return 0;
+}
+
+/* Words per packed row: K codes of `bits` bits, LSB-first bitstream. */
+static int64_t row_words(int64_t K, int bits) { return K * bits / 32; }
+
+/* ------------------------------------------------------------------------ */
+/* Quantize: per group min/max, fp16 scale and bias, codes, packing          */
+/* ------------------------------------------------------------------------ */
+
+/* Put code q of element k into row n's bitstream: bits [k*bits, k*bits+bits). */
+static void put_code(uint32_t *row, int64_t k, int bits, uint32_t q)
+{
+    for (int t = 0; t < bits; t++) {
+        int64_t bit = k * bits + t;
+        if ((q >> t) & 1u) row[bit / 32] |= (1u << (bit % 32));
+    }
+}
+
+static uint32_t get_code(const uint32_t *row, int64_t k, int bits)
+{
+    uint32_t q = 0;
+    for (int t = 0; t < bits; t++) {
+        int64_t bit = k * bits + t;
+        q |= ((row[bit / 32] >> (bit % 32)) & 1u) << t;
+    }
+    return q;
+}
+
+int oracle_quantize(const float *w, int64_t N, int64_t K, int G, int bits,
+                    uint32_t *packed, uint16_t *scales, uint16_t *biases)
+{
+    if (!w || !packed || !scales || !biases || bad_shape(N, K, G, bits)) return ORACLE_BAD_ARG;
+    const int64_t P = row_words(K, bits), Gn = K / G;
+    const uint32_t qmax = (1u << bits) - 1u;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        const float *wr = w + n * K;
+        uint32_t *pr = packed + n * P;
+        for (int64_t j = 0; j < P; j++) pr[j] = 0u;
+        for (int64_t g = 0; g < Gn; g++) {
+            /* group = G contiguous elements of row n along K */
+            float mn = wr[g * G], mx = wr[g * G];
+            for (int64_t i = 1; i < G; i++) {
+                float v = wr[g * G + i];
+                if (v < mn) mn = v;
+                if (v > mx) mx = v;
+            }
+            float d = mx - mn;                 /* fp32 subtraction */
+            float s32 = d / (float)qmax;       /* fp32 IEEE division */
+            uint16_t s16 = f16_bits_from_double((double)s32);
+            uint16_t b16 = f16_bits_from_double((double)mn);
+            scales[n * Gn + g] = s16;
+            biases[n * Gn + g] = b16;
+            float sf = (float)f16_value(s16), bf = (float)f16_value(b16);
+            for (int64_t i = 0; i < G; i++) {
+                int64_t k = g * G + i;
+                uint32_t q = 0;
+                if (sf != 0.0f) {
+                    float t = (wr[k] - bf) / sf;   /* fp32 sub, fp32 div */
+                    float r = rintf(t);            /* ties to even */
+                    if (r < 0.0f) r = 0.0f;
+                    if (r > (float)qmax) r = (float)qmax;
+                    q = (uint32_t)r;
+                }
+                put_code(pr, k, bits, q);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Codes as bytes [N, K], read back bit by bit from the packed bitstream. */
+int oracle_unpack_codes(const uint32_t *packed, int64_t N, int64_t K, int bits, uint8_t *codes)
+{
+    if (!packed || !codes || N <= 0 || K <= 0) return ORACLE_BAD_ARG;
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8) || (K * bits) % 32 != 0) return ORACLE_BAD_ARG;
+    const int64_t P = row_words(K, bits);
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) codes[n * K + k] = (uint8_t)get_code(packed + n * P, k, bits);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dequantize                                                               */
+/* ------------------------------------------------------------------------ */
+
+/* Exact q*scale + bias (fits in fp64: q has <= 8 bits, scale and bias are fp16). */
+static double exact_value(const uint32_t *prow, const uint16_t *srow, const uint16_t *brow,
+                          int64_t k, int G, int bits)
+{
+    uint32_t q = get_code(prow, k, bits);
+    return (double)q * f16_value(srow[k / G]) + f16_value(brow[k / G]);
+}
+
+int oracle_dequantize_f32(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                          int64_t N, int64_t K, int G, int bits, float *out)
+{
+    if (!packed || !scales || !biases || !out || bad_shape(N, K, G, bits)) return ORACLE_BAD_ARG;
+    const int64_t P = row_words(K, bits), Gn = K / G;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++)
+            out[n * K + k] = (float)exact_value(packed + n * P, scales + n * Gn, biases + n * Gn, k, G, bits);
+    return ORACLE_OK;
+}
+
+int oracle_dequantize_bf16(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                           int64_t N, int64_t K, int G, int bits, uint16_t *out)
+{
+    if (!packed || !scales || !biases || !out || bad_shape(N, K, G, bits)) return ORACLE_BAD_ARG;
+    const int64_t P = row_words(K, bits), Gn = K / G;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) {
+            float v = (float)exact_value(packed + n * P, scales + n * Gn, biases + n * Gn, k, G, bits);
+            out[n * K + k] = bf16_bits_from_double((double)v);
+        }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantized matmul reference: y = x @ dequant(W)^T in fp64                  */
+/* ------------------------------------------------------------------------ */
+
+/* y[i][j] for the requested rows m_idx[i] of x and rows n_idx[j] of W
+ * (output columns); the full product is m_idx = 0..M-1, n_idx = 0..N-1. */
+int oracle_matmul_sampled(const uint16_t *x_bf16, int64_t M, int64_t K,
+                          const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                          int64_t N, int G, int bits,
+                          const int64_t *m_idx, int64_t nm, const int64_t *n_idx, int64_t nn,
+                          double *y)
+{
+    if (!x_bf16 || !packed || !scales || !biases || !m_idx || !n_idx || !y) return ORACLE_BAD_ARG;
+    if (M <= 0 || bad_shape(N, K, G, bits) || nm < 0 || nn < 0) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < nm; i++) if (m_idx[i] < 0 || m_idx[i] >= M) return ORACLE_BAD_ARG;
+    for (int64_t j = 0; j < nn; j++) if (n_idx[j] < 0 || n_idx[j] >= N) return ORACLE_BAD_ARG;
+    const int64_t P = row_words(K, bits), Gn = K / G;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t j = 0; j < nn; j++) {
+        const int64_t n = n_idx[j];
+        const uint32_t *prow = packed + n * P;
+        const uint16_t *srow = scales + n * Gn, *brow = biases + n * Gn;
+        for (int64_t i = 0; i < nm; i++) {
+            const uint16_t *xr = x_bf16 + m_idx[i] * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += bf16_value(xr[k]) * exact_value(prow, srow, brow, k, G, bits);
+            y[i * nn + j] = acc;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Full product y[M][N]. */
+int oracle_matmul(const uint16_t *x_bf16, int64_t M, int64_t K,
+                  const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                  int64_t N, int G, int bits, double *y)
+{
+    if (!x_bf16 || !packed || !scales || !biases || !y) return ORACLE_BAD_ARG;
+    if (M <= 0 || bad_shape(N, K, G, bits)) return ORACLE_BAD_ARG;
+    const int64_t P = row_words(K, bits), Gn = K / G;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; n++) {
+        const uint32_t *prow = packed + n * P;
+        const uint16_t *srow = scales + n * Gn, *brow = biases + n * Gn;
+        for (int64_t m = 0; m < M; m++) {
+            const uint16_t *xr = x_bf16 + m * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += bf16_value(xr[k]) * exact_value(prow, srow, brow, k, G, bits);
+            y[m * N + n] = acc;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Number of threads the parallel loops above use. */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,398 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+Each check ties the oracle to something the pages or the mathematics fix:
+hand-derived groups (tests/golden/hand_groups.json), storage figures printed on
+the pages (tests/golden/storage_arithmetic.json), the shift/mask unpack printed
+in anllm 'Tutorial 10: Quantization' section 3, an independent NumPy quantizer,
+IEEE conversions from NumPy/PyTorch, brute-force fp64 matmul, closed forms and
+invariants.  ``test_planted_mistakes_are_caught`` rebuilds the oracle with
+plausible mistakes planted in it and checks that the pins reject each one.
+"""
+import json
+import os
+import re
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from pins import (affine_values_f64, bitwise_pack, bitwise_unpack, numpy_quantize, page_pack,
+                  page_unpack)
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+BITS = (2, 3, 4, 8)
+GROUPS = (32, 64, 128)
+
+
+def _hand_groups():
+    with open(os.path.join(GOLDEN, "hand_groups.json")) as f:
+        return json.load(f)["groups"]
+
+
+def _storage():
+    with open(os.path.join(GOLDEN, "storage_arithmetic.json")) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# IEEE conversions
+# --------------------------------------------------------------------------
+
+def _conversion_probe_values():
+    rng = np.random.default_rng(7)
+    parts = [rng.normal(0, 1, 4000), rng.normal(0, 1e-5, 2000), rng.normal(0, 1e-7, 2000),
+             rng.normal(0, 3e4, 1000), rng.uniform(-70000, 70000, 1000)]
+    # exact ties on the fp16 grid: 1 + (2j+1)*2^-11, and ties in the subnormal range
+    j = np.arange(0, 200)
+    parts.append(1.0 + (2 * j + 1) * 2.0 ** -11)
+    parts.append((2 * j + 1) * 2.0 ** -25)
+    parts.append(np.array([0.0, -0.0, 65504.0, 65519.0, 65520.0, -65520.0, 2.0 ** -24, 2.0 ** -25,
+                           3 * 2.0 ** -26, 6.1035156e-05, 6.097555e-05]))
+    return np.concatenate(parts).astype(np.float32)
+
+
+def test_f16_rounding_matches_numpy():
+    v = _conversion_probe_values()
+    ours = oracle.f16_round(v)
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_f16_decode_matches_numpy():
+    h = np.arange(0, 65536, dtype=np.uint32).astype(np.uint16)
+    finite = (h & 0x7C00) != 0x7C00
+    ours = oracle.f16_to_double(h[finite])
+    ref = h[finite].view(np.float16).astype(np.float64)
+    assert np.array_equal(ours, ref)
+
+
+def test_bf16_rounding_matches_torch():
+    v = _conversion_probe_values()
+    extra = (1.0 + (2 * np.arange(100) + 1) * 2.0 ** -8).astype(np.float32)  # bf16 ties
+    v = np.concatenate([v, extra, np.array([1e-40, -1e-39, 3e38], dtype=np.float32)])
+    ours = oracle.bf16_round(v)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# --------------------------------------------------------------------------
+# Hand-derived groups
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("g", _hand_groups(), ids=lambda g: g["name"])
+def test_hand_group(g):
+    w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+    bits, G = g["bits"], g["G"]
+    packed, scales, biases = oracle.quantize(w, G, bits)
+    assert scales[0, 0] == int(g["scale_f16"], 16), hex(scales[0, 0])
+    assert biases[0, 0] == int(g["bias_f16"], 16), hex(biases[0, 0])
+    assert [hex(x) for x in packed[0]] == [hex(int(x, 16)) for x in g["packed"]]
+    codes = oracle.unpack_codes(packed, w.shape[1], bits)
+    assert codes[0].tolist() == g["codes"]
+    # the independent NumPy statement agrees with the hand derivation too
+    p2, s2, b2, q2 = numpy_quantize(w, G, bits)
+    assert np.array_equal(p2, packed) and q2[0].tolist() == g["codes"]
+    # dequantize: q*scale + bias exactly (all hand groups are exact in fp32)
+    deq = oracle.dequantize_f32(packed, scales, biases, w.shape[1], G, bits)
+    expect = affine_values_f64(np.array([g["codes"]]), scales, biases, G).astype(np.float32)
+    assert np.array_equal(deq, expect)
+
+
+def test_hand_group_exact_reconstruction():
+    """Groups on an exact grid come back exactly (the 4-bit grid, 2-bit, 3-bit, 8-bit cases)."""
+    for g in _hand_groups():
+        if g["name"] not in ("2bit_pattern", "3bit_bitstream_straddle", "8bit_bytes"):
+            continue
+        w = np.array([float(s) for s in g["w"]], dtype=np.float32)[None, :]
+        p, s, b = oracle.quantize(w, g["G"], g["bits"])
+        assert np.array_equal(oracle.dequantize_f32(p, s, b, w.shape[1], g["G"], g["bits"]), w)
+
+
+# --------------------------------------------------------------------------
+# Storage arithmetic printed on the pages
+# --------------------------------------------------------------------------
+
+def _packed_bytes(N, K, G, bits):
+    p, s, b = (np.zeros((N, K * bits // 32), np.uint32), np.zeros((N, K // G), np.uint16),
+               np.zeros((N, K // G), np.uint16))
+    return p.nbytes + s.nbytes + b.nbytes
+
+
+def test_oracle_storage_matches_printed_figures():
+    st = _storage()
+    w = synth.weights(64, 64, seed=3, outliers=False)
+    p, s, b = oracle.quantize(w, 64, 4)
+    nbytes = p.nbytes + s.nbytes + b.nbytes
+    assert nbytes * 8 / w.size == st["bits_per_weight_4bit_G64"]["value"]
+    assert nbytes / w.size == st["bytes_per_param_4bit_G64"]["value"]
+    r = 2.0 / (nbytes / w.size)
+    assert abs(r - st["fp16_to_4bit_ratio"]["value"]) <= st["fp16_to_4bit_ratio"]["printed_precision"]
+    params = st["llama_3_3_70b_prediction"]["params"]
+    assert params * nbytes // w.size == st["llama_3_3_70b_prediction"]["bytes"]
+    assert 4096 * 14336 * 2 == st["linear_4096x14336_bf16_bytes"]["value"]
+    assert st["linear_4096x14336_bf16_bytes"]["value"] / 2 ** 20 == 112.0
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("G", GROUPS)
+def test_oracle_array_sizes_follow_formula(bits, G):
+    N, K = 3, 256
+    p, s, b = oracle.quantize(synth.weights(N, K, seed=1), G, bits)
+    assert p.nbytes + s.nbytes + b.nbytes == N * K * bits // 8 + 4 * N * K // G
+
+
+# --------------------------------------------------------------------------
+# Independent NumPy quantizer, page unpack, brute-force bitstream
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("G", GROUPS)
+def test_oracle_quantize_matches_numpy(bits, G):
+    w = synth.weights(48, 512, seed=100 + bits * 10 + G)
+    p, s, b = oracle.quantize(w, G, bits)
+    p2, s2, b2, q2 = numpy_quantize(w, G, bits)
+    assert np.array_equal(s, s2)
+    assert np.array_equal(b, b2)
+    assert np.array_equal(p, p2)
+
+
+def test_oracle_quantize_tiny_workload_matches_numpy():
+    c = synth.case("tiny")
+    w = synth.weights(c.N, c.K, c.w_seed, c.outliers)
+    p, s, b = oracle.quantize(w, c.G, c.bits)
+    p2, s2, b2, _ = numpy_quantize(w, c.G, c.bits)
+    assert np.array_equal(p, p2) and np.array_equal(s, s2) and np.array_equal(b, b2)
+
+
+@pytest.mark.parametrize("bits", (2, 4, 8))
+def test_page_shift_mask_unpack_round_trips(bits):
+    w = synth.weights(16, 256, seed=5)
+    p, s, b = oracle.quantize(w, 64, bits)
+    codes = page_unpack(p, bits)
+    assert np.array_equal(codes, oracle.unpack_codes(p, 256, bits))
+    assert np.array_equal(page_pack(codes, bits), p)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_bitstream_brute_force(bits):
+    w = synth.weights(8, 384, seed=9)
+    p, _, _ = oracle.quantize(w, 128, bits)
+    codes = bitwise_unpack(p, 384, bits)
+    assert np.array_equal(codes, oracle.unpack_codes(p, 384, bits))
+    assert np.array_equal(bitwise_pack(codes, bits), p)
+
+
+def test_3bit_packs_32_codes_in_3_words():
+    w = synth.weights(2, 64, seed=4)
+    p, _, _ = oracle.quantize(w, 32, 3)
+    assert p.shape == (2, 6)
+
+
+# --------------------------------------------------------------------------
+# Invariants: extreme codes, range, round-trip error bound
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("G", GROUPS)
+def test_codes_extremes_and_error_bound(bits, G):
+    N, K = 32, 1024
+    w = synth.weights(N, K, seed=200 + bits + G)
+    p, s, b = oracle.quantize(w, G, bits)
+    q = oracle.unpack_codes(p, K, bits).reshape(N, K // G, G)
+    qmax = (1 << bits) - 1
+    assert q.max() <= qmax
+    wg = w.reshape(N, K // G, G)
+    s64 = s.view(np.float16).astype(np.float64)
+    assert (s64 > 0).all()
+    # code 0 at the group minimum, 2^bits - 1 at the group maximum
+    amin = wg.argmin(axis=-1)
+    amax = wg.argmax(axis=-1)
+    assert (np.take_along_axis(q, amin[..., None], -1) == 0).all()
+    assert (np.take_along_axis(q, amax[..., None], -1) == qmax).all()
+    # |w - (q*s + b)| <= s*(1/2 + 2^(bits-23)): half a step plus the fp32 rounding of the quotient
+    wr = affine_values_f64(q.reshape(N, K), s, b, G).reshape(N, K // G, G)
+    err = np.abs(wg.astype(np.float64) - wr)
+    bound = s64[..., None] * (0.5 + 2.0 ** (bits - 23))
+    assert (err <= bound).all(), float((err / bound).max())
+
+
+def test_degenerate_groups_reconstruct_the_bias():
+    w = np.full((2, 128), 0.0123, dtype=np.float32)
+    w[1, :64] = -3.5
+    p, s, b = oracle.quantize(w, 64, 4)
+    assert (s == 0).all() and (p == 0).all()
+    d = oracle.dequantize_f32(p, s, b, 128, 64, 4)
+    assert np.array_equal(d, b.view(np.float16).astype(np.float32).repeat(64, axis=1))
+
+
+# --------------------------------------------------------------------------
+# Dequantize
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", BITS)
+def test_dequantize_matches_exact_affine_values(bits):
+    N, K, G = 16, 512, 64
+    w = synth.weights(N, K, seed=31)
+    p, s, b = oracle.quantize(w, G, bits)
+    codes = bitwise_unpack(p, K, bits)
+    exact = affine_values_f64(codes, s, b, G)
+    f32 = oracle.dequantize_f32(p, s, b, K, G, bits)
+    assert np.array_equal(f32, exact.astype(np.float32))  # one rounding, fp64 -> fp32 (RNE)
+    bf = oracle.dequantize_bf16(p, s, b, K, G, bits)
+    ref = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf, ref)
+
+
+# --------------------------------------------------------------------------
+# Matmul: brute force, closed form, sampled == full
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M", (1, 3, 8))
+def test_matmul_equals_dequantize_then_matmul(bits, M):
+    """anllm Tutorial 10, section 5: the fused product equals dequantize-then-multiply."""
+    N, K, G = 40, 256, 32
+    w = synth.weights(N, K, seed=41 + bits)
+    x = synth.activations(M, K, seed=42)
+    p, s, b = oracle.quantize(w, G, bits)
+    codes = page_unpack(p, bits) if bits != 3 else bitwise_unpack(p, K, bits)
+    w_full = affine_values_f64(codes, s, b, G)
+    y_ref = x.to(torch.float64).numpy() @ w_full.T
+    y = oracle.matmul(synth.bf16_bits(x), p, s, b, G, bits)
+    assert y.shape == (M, N)
+    np.testing.assert_allclose(y, y_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_matmul_all_zero_codes_closed_form():
+    """All codes 0: y[m, n] = sum_g bias[n, g] * sum_{k in g} x[m, k]."""
+    M, N, K, G = 4, 24, 512, 128
+    rng = np.random.default_rng(0)
+    p = np.zeros((N, K * 4 // 32), np.uint32)
+    s = rng.normal(0, 0.01, (N, K // G)).astype(np.float16).view(np.uint16)
+    b = rng.normal(0, 0.1, (N, K // G)).astype(np.float16).view(np.uint16)
+    x = synth.activations(M, K, seed=5)
+    xs = x.to(torch.float64).numpy().reshape(M, K // G, G).sum(-1)  # [M, Gn]
+    y_cf = xs @ b.view(np.float16).astype(np.float64).T
+    y = oracle.matmul(synth.bf16_bits(x), p, s, b, G, 4)
+    np.testing.assert_allclose(y, y_cf, rtol=1e-12, atol=1e-12)
+
+
+def test_matmul_one_hot_activation_selects_dequantized_column():
+    N, K, G, bits = 16, 256, 64, 4
+    w = synth.weights(N, K, seed=8)
+    p, s, b = oracle.quantize(w, G, bits)
+    x = torch.zeros(1, K, dtype=torch.bfloat16)
+    x[0, 77] = 1.0
+    y = oracle.matmul(synth.bf16_bits(x), p, s, b, G, bits)
+    col = oracle.dequantize_f32(p, s, b, K, G, bits)[:, 77]
+    assert np.array_equal(y[0].astype(np.float32), col)
+
+
+def test_matmul_sampled_equals_full():
+    M, N, K, G, bits = 5, 30, 256, 64, 3
+    w = synth.weights(N, K, seed=12)
+    x = synth.activations(M, K, seed=13)
+    p, s, b = oracle.quantize(w, G, bits)
+    full = oracle.matmul(synth.bf16_bits(x), p, s, b, G, bits)
+    mi, ni = np.array([4, 0, 2]), np.array([29, 3, 3, 17])
+    samp = oracle.matmul_sampled(synth.bf16_bits(x), p, s, b, G, bits, mi, ni)
+    assert np.array_equal(samp, full[np.ix_(mi, ni)])
+
+
+def test_tolerance_rule():
+    y_ref = np.array([1.0, -2.0, 0.0, 3.0])
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    ok, worst = oracle.tolerance_ok(y_ref + 8e-3 * (np.abs(y_ref) + rms) * 0.999, y_ref)
+    assert ok and worst < 1.0
+    ok, worst = oracle.tolerance_ok(y_ref + 8e-3 * (np.abs(y_ref) + rms) * 1.01, y_ref)
+    assert not ok
+
+
+def test_oracle_rejects_bad_arguments():
+    w = np.zeros((2, 96), np.float32)
+    with pytest.raises(ValueError):
+        oracle.quantize(w, 64, 4)      # K % G != 0
+    with pytest.raises(ValueError):
+        oracle.quantize(w[:, :64], 64, 5)   # unsupported bits
+    with pytest.raises(ValueError):
+        oracle.quantize(w[:, :64], 16, 4)   # unsupported group size
+
+
+# --------------------------------------------------------------------------
+# Planted mistakes: each must be rejected by at least one pin above
+# --------------------------------------------------------------------------
+
+MUTATIONS = {
+    "bias_dropped": ("return (double)q * f16_value(srow[k / G]) + f16_value(brow[k / G]);",
+                     "return (double)q * f16_value(srow[k / G]);"),
+    "bias_sign": ("return (double)q * f16_value(srow[k / G]) + f16_value(brow[k / G]);",
+                  "return (double)q * f16_value(srow[k / G]) - f16_value(brow[k / G]);"),
+    "ties_away": ("float r = rintf(t);", "float r = roundf(t);"),
+    "fp32_scale_for_codes": ("float t = (wr[k] - bf) / sf;", "float t = (wr[k] - mn) / s32;"),
+    "msb_first_packing": ("if ((q >> t) & 1u) row[bit / 32] |= (1u << (bit % 32));",
+                          "if ((q >> t) & 1u) row[bit / 32] |= (1u << (31 - bit % 32));"),
+    "group_index_off_by_one": ("uint32_t q = get_code(prow, k, bits);\n    return (double)q * f16_value(srow[k / G])",
+                               "uint32_t q = get_code(prow, k, bits);\n    return (double)q * f16_value(srow[(k + 1) / G])"),
+    "transposed_x_index": ("const uint16_t *xr = x_bf16 + m * K;", "const uint16_t *xr = x_bf16 + (M - 1 - m) * K;"),
+    "scale_divides_by_2pow_bits": ("float s32 = d / (float)qmax;", "float s32 = d / (float)(qmax + 1u);"),
+}
+
+
+def _pins_pass(o: "oracle.Oracle") -> bool:
+    """A compact run of the pins above against an arbitrary oracle build."""
+    try:
+        for g in _hand_groups():
+            w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+            p, s, b = o.quantize(w, g["G"], g["bits"])
+            if s[0, 0] != int(g["scale_f16"], 16) or b[0, 0] != int(g["bias_f16"], 16):
+                return False
+            if [int(x) for x in p[0]] != [int(x, 16) for x in g["packed"]]:
+                return False
+            deq = o.dequantize_f32(p, s, b, w.shape[1], g["G"], g["bits"])
+            if not np.array_equal(deq, affine_values_f64(np.array([g["codes"]]), s, b, g["G"]).astype(np.float32)):
+                return False
+        for bits in BITS:
+            N, K, G = 8, 256, 32
+            w = synth.weights(N, K, seed=41 + bits)
+            x = synth.activations(3, K, seed=42)
+            p, s, b = o.quantize(w, G, bits)
+            p2, s2, b2, _ = numpy_quantize(w, G, bits)
+            if not (np.array_equal(p, p2) and np.array_equal(s, s2) and np.array_equal(b, b2)):
+                return False
+            codes = bitwise_unpack(p, K, bits)
+            y_ref = x.to(torch.float64).numpy() @ affine_values_f64(codes, s, b, G).T
+            y = o.matmul(synth.bf16_bits(x), p, s, b, G, bits)
+            if not np.allclose(y, y_ref, rtol=1e-12, atol=1e-12):
+                return False
+        return True
+    except ValueError:
+        return False
+
+
+def _build_variant(tmp_path, name, old, new):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "aq_oracle.c")).read()
+    assert src.count(old) == 1, f"mutation {name}: anchor not found exactly once"
+    d = tmp_path / name
+    d.mkdir()
+    (d / "aq_oracle.c").write_text(src.replace(old, new))
+    lib = d / "liboracle.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, str(d / "aq_oracle.c"), "-o", str(lib), "-lm"])
+    return oracle.Oracle(str(lib))
+
+
+def test_unmutated_oracle_passes_compact_pins():
+    assert _pins_pass(oracle.default())
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistakes_are_caught(tmp_path, name):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    old, new = MUTATIONS[name]
+    variant = _build_variant(tmp_path, name, old, new)
+    assert not _pins_pass(variant), f"planted mistake '{name}' was not caught by the pins"
