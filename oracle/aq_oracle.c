@@ -26,6 +26,8 @@
  * Readings where the pages are silent (each is also listed in the design notes):
  *  - scale = (max - min) / (2^bits - 1) and bias = min, both computed in fp32
  *    and rounded to fp16 (round to nearest, ties to even, subnormals kept).
+ *    A group extreme equal to zero is taken as +0.0 (the sign of a zero min or
+ *    max is not a property of the set of values).
  *  - codes are computed from the STORED (fp16) scale and bias:
  *        q = clamp(rint_even(fp32(fp32(w - bias16) / scale16)), 0, 2^bits - 1)
  *    with IEEE correctly rounded fp32 subtraction and division.
@@ -208,6 +210,9 @@ int oracle_quantize(const float *w, int64_t N, int64_t K, int G, int bits,
                 if (v < mn) mn = v;
                 if (v > mx) mx = v;
             }
+            /* -0.0 and +0.0 are the same number: a zero extreme is taken as +0.0 */
+            if (mn == 0.0f) mn = 0.0f;
+            if (mx == 0.0f) mx = 0.0f;
             float d = mx - mn;                 /* fp32 subtraction */
             float s32 = d / (float)qmax;       /* fp32 IEEE division */
             uint16_t s16 = f16_bits_from_double((double)s32);

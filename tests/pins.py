@@ -61,6 +61,8 @@ def numpy_quantize(w: np.ndarray, G: int, bits: int):
     wg = w.reshape(N, K // G, G)
     mn = wg.min(axis=-1)
     mx = wg.max(axis=-1)
+    mn = np.where(mn == 0, np.float32(0.0), mn).astype(np.float32)   # zero extremes taken as +0.0
+    mx = np.where(mx == 0, np.float32(0.0), mx).astype(np.float32)
     d = (mx - mn).astype(np.float32)
     s32 = (d / np.float32(qmax)).astype(np.float32)
     s16 = s32.astype(np.float16)
