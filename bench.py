@@ -1,0 +1,486 @@
+"""Benchmark of the quantized-matmul hot path on B200.
+
+Headline (``metric``): weight GB/s of the 4-bit G=64 QMV kernel at M=1 on the
+decode workload: one "step" is a decode pass through three Llama-3-8B-shaped
+linears, (K, N) = (4096, 4096), (4096, 14336), (14336, 4096), each a
+``aq_matmul`` of one bf16 activation row against affine 4-bit G=64 weights.
+value = packed weight + scale + bias bytes of a step / step time, summed over
+ranks (weak scaling: every rank runs its own copy of the workload).
+
+Also measured in the same run (``sections``): QMM prefill TFLOP/s (M = 8192,
+K = 4096, N = 14336, the tensor-core kernel), the M = 1..8 QMV curve, and the
+quantize / dequantize kernels.  Inputs are synthetic (seeded; shapes of the
+models the pages measure on), resident in HBM before timing; weight sets are
+rotated so every timed launch reads HBM (working set > 126 MB L2).
+
+``--impl reference`` times the CPU oracle (the plain C statement of the method)
+on the host cores for the same metric: see ``oracle/``.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+DECODE_SHAPES = [(4096, 4096), (4096, 14336), (14336, 4096)]  # (K, N)
+G, BITS = 64, 4
+METRIC = "4-bit G64 QMV weight GB/s (% of HBM peak) at M=1; QMM prefill TFLOP/s"
+WORKLOAD = ("decode step: QMV M=1 over Llama-3-8B linears (K,N) = (4096,4096), (4096,14336), (14336,4096); "
+            "affine 4-bit G=64; W ~ N(0,0.02) with 0.1% x10 outliers; x ~ N(0,1) bf16")
+
+
+def weight_bytes(K, N, g=G, bits=BITS):
+    return N * K * bits // 8 + 4 * N * K // g
+
+
+STEP_BYTES = sum(weight_bytes(K, N) for K, N in DECODE_SHAPES)
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("common.cuh", "qmv.cu", "qmm.cu", "quantize.cu", "aq_api.cu"):
+        h.update(open(os.path.join(ROOT, "weight_only_group_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(name):
+    """DRAM bytes per unit for a kernel from a committed ncu summary, if the kernel
+    sources have not changed since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "counters.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(name)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_unit")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.index = str(device_index)
+        try:  # the GPU's UUID identifies it for nvidia-smi regardless of CUDA_VISIBLE_DEVICES
+            import torch
+            self.index = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.path = os.path.join("/tmp", f"aq_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our implementation
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import weight_only_group_b200 as aq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+
+    def barrier():
+        if dist is not None:
+            dist.barrier(device_ids=[local_rank])
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = read_peaks()
+    stream = torch.cuda.Stream(dev)
+
+    # -- resident inputs: weight sets rotated so the working set exceeds L2
+    copies = max(2, -(-2 * L2_BYTES // STEP_BYTES) + 1)
+    sets = []
+    for ci in range(copies):
+        layer = []
+        for si, (K, N) in enumerate(DECODE_SHAPES):
+            seed = 1000 + 100 * 2 + si
+            if ci == 0:
+                w = torch.from_numpy(synth.weights(N, K, seed)).to(dev)
+                p, s, b = aq.aq_quantize(w, G, BITS)
+                del w
+            else:
+                p, s, b = (t.clone() for t in sets[0][si][:3])
+            x = synth.activations(1, K, seed + 1).to(dev)
+            y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+            layer.append((p, s, b, x, y))
+        sets.append(layer)
+    torch.cuda.synchronize()
+
+    def step(layer):
+        for (p, s, b, x, y) in layer:
+            aq.aq_matmul(x, p, s, b, G, BITS, out=y)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            for layer in sets:
+                step(layer)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for layer in sets:
+            step(layer)
+    reps_w = max(1, -(-args.warmup // copies))
+    reps = max(1, -(-args.steps // copies))
+    steps = reps * copies
+    for _ in range(reps_w):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms)
+    clocks = clk.summary()
+    value = STEP_BYTES * steps * world / (ms_max * 1e-3) / 1e9
+    ms_per_step = ms_max / steps
+    achieved = STEP_BYTES / (ms / steps * 1e-3) / 1e9  # this rank's kernel-only GB/s (the step is 3 QMV launches)
+    traffic = recorded_traffic("qmv_decode_step")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "peak_source": peaks["source"], "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
+                "kernel": "qmv_kernel<4,1> (3 launches per step)",
+                "algorithmic_bytes_per_step": STEP_BYTES}
+    del graph
+
+    # -- end to end through the public API with host buffers (pinned), per step:
+    #    H2D of each linear's x, aq_matmul, D2H of each y, read on the host
+    e2e_steps = min(steps, args.e2e_steps)
+    hx = [synth.activations(1, K, 7).pin_memory() for K, N in DECODE_SHAPES]
+    hy = [torch.empty((1, N), dtype=torch.bfloat16).pin_memory() for K, N in DECODE_SHAPES]
+    h2d = sum(t.numel() * 2 for t in hx)
+    d2h = sum(t.numel() * 2 for t in hy)
+
+    def e2e_step(layer):
+        for (p, s, b, x, y), xh, yh in zip(layer, hx, hy):
+            x.copy_(xh, non_blocking=True)
+            aq.aq_matmul(x, p, s, b, G, BITS, out=y)
+            yh.copy_(y, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return float(hy[-1][0, 0])
+
+    with torch.cuda.stream(stream):
+        for i in range(20):
+            e2e_step(sets[i % copies])
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(sets[i % copies])
+        f1.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e = {"value": round(STEP_BYTES * e2e_steps * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+           "ms_per_step": round(e2e_ms / e2e_steps, 5)}
+    del sets
+    torch.cuda.empty_cache()
+
+    sections = {}
+    if not args.no_sections:
+        sections = measure_sections(args, aq, torch, dev, stream, peaks)
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": reps_w * copies, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; shapes of Llama-3-8B linears; no checkpoints)",
+            "config": {"workload": WORKLOAD, "M": 1, "bits": BITS, "G": G, "shapes_KN": DECODE_SHAPES,
+                       "parallelism": f"replicas x{world} (no data-path collective)",
+                       "l2": f"rotating {copies} resident weight sets ({copies * STEP_BYTES / 2**20:.0f} MiB > "
+                             f"126 MiB L2); step replayed from a CUDA graph"},
+            "pct_of_hbm_peak": round(value / world / peaks["hbm_gbs"] * 100, 2),
+            "roofline": roofline, "e2e": e2e, "gpu_launches": steps * len(DECODE_SHAPES),
+            "clocks": clocks, "sections": sections}
+    return line
+
+
+def timed_graph(torch, stream, fn, reps_inner, reps_outer):
+    """Capture reps_inner calls of fn into a graph; time reps_outer replays; ms per call."""
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn(0)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(reps_inner):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps_outer):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / (reps_inner * reps_outer)
+
+
+def measure_sections(args, aq, torch, dev, stream, peaks):
+    out = {}
+    # ---- QMM prefill: M = 8192, K = 4096, N = 14336 (the tensor-core kernel)
+    M, K, N = 8192, 4096, 14336
+    w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 5 + 4)).to(dev)
+    p, s, b = aq.aq_quantize(w, G, BITS)
+    del w
+    x = synth.activations(M, K, 7).to(dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, p, s, b, G, BITS, out=y), 2, max(2, args.qmm_reps))
+    flops = 2.0 * M * N * K
+    tf = flops / (ms * 1e-3) / 1e12
+    out["qmm_prefill"] = {"value": round(tf, 1), "unit": "TFLOP/s", "M": M, "K": K, "N": N, "bits": BITS, "G": G,
+                          "ms": round(ms, 4), "kernel": "qmm_kernel<4,256> (tcgen05, A=dequantized W in TMEM)",
+                          "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                                       "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                                       "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
+                                       "frac_of_burst": round(tf / peaks["bf16_tflops"], 4),
+                                       "traffic": recorded_traffic("qmm_prefill")}}
+    del p, s, b, x, y
+    torch.cuda.empty_cache()
+
+    # ---- QMV small-M curve on K=4096, N=14336 (rotating weight copies)
+    K, N = 4096, 14336
+    w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 3)).to(dev)
+    base = aq.aq_quantize(w, G, BITS)
+    del w
+    wb = weight_bytes(K, N)
+    copies = max(2, -(-2 * L2_BYTES // wb) + 1)
+    ws = [base] + [tuple(t.clone() for t in base) for _ in range(copies - 1)]
+    curve = {}
+    for M in (1, 2, 3, 4, 5, 6, 8):
+        x = synth.activations(M, K, 11).to(dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, *ws[i % copies], G, BITS, out=y), copies * 8, 50)
+        curve[str(M)] = {"us": round(ms * 1e3, 3), "weight_GBps": round(wb / (ms * 1e-3) / 1e9, 1),
+                         "kernel": ["qmv", "qmm"][aq.aq_dispatch(M, N, K, G, BITS) - 1]}
+    out["qmv_small_m"] = {"K": K, "N": N, "bits": BITS, "G": G, "curve": curve}
+    del ws, base
+    torch.cuda.empty_cache()
+
+    # ---- bits x group sweep at M=1 on K=8192, N=28672 (one point per bits, G=64 and the 4-bit G sweep)
+    K, N = 8192, 28672
+    w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 4)).to(dev)
+    sweep = {}
+    x = synth.activations(1, K, 13).to(dev)
+    y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+    for bits in (2, 3, 4, 8):
+        for g in ((32, 64, 128) if bits == 4 else (64,)):
+            q = aq.aq_quantize(w, g, bits)
+            wb = weight_bytes(K, N, g, bits)
+            copies = max(2, -(-2 * L2_BYTES // wb) + 1)
+            qs = [q] + [tuple(t.clone() for t in q) for _ in range(copies - 1)]
+            ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, *qs[i % copies], g, bits, out=y), copies * 4,
+                             20)
+            sweep[f"b{bits}_G{g}"] = {"us": round(ms * 1e3, 2), "weight_GBps": round(wb / (ms * 1e-3) / 1e9, 1)}
+            del qs, q
+            torch.cuda.empty_cache()
+    out["qmv_bits_group_sweep"] = {"K": K, "N": N, "M": 1, "points": sweep}
+
+    # ---- quantize and dequantize (bytes: read W fp32 + write packed/scales/biases; read packed + write bf16)
+    p, s, b = aq.aq_quantize(w, G, BITS)
+    ms_q = timed_graph(torch, stream, lambda i: aq.aq_quantize(w, G, BITS), 1, 10)
+    qbytes = N * K * 4 + weight_bytes(K, N)
+    dq = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    ms_d = timed_graph(torch, stream, lambda i: aq.aq_dequantize(p, s, b, K, G, BITS, out=dq), 1, 10)
+    dbytes = weight_bytes(K, N) + N * K * 2
+    out["quantize"] = {"K": K, "N": N, "bits": BITS, "G": G, "ms": round(ms_q, 4),
+                       "GBps": round(qbytes / (ms_q * 1e-3) / 1e9, 1),
+                       "frac_hbm": round(qbytes / (ms_q * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    out["dequantize_bf16"] = {"K": K, "N": N, "bits": BITS, "G": G, "ms": round(ms_d, 4),
+                              "GBps": round(dbytes / (ms_d * 1e-3) / 1e9, 1),
+                              "frac_hbm": round(dbytes / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+def oracle_decode_inputs():
+    import oracle
+    ins = []
+    for si, (K, N) in enumerate(DECODE_SHAPES):
+        seed = 1000 + 100 * 2 + si
+        p, s, b = oracle.quantize(synth.weights(N, K, seed), G, BITS)
+        ins.append((synth.bf16_bits(synth.activations(1, K, seed + 1)), p, s, b))
+    return ins
+
+
+def time_oracle(ins, steps, budget_s):
+    """Time decode steps of the oracle (plain C, fp64) on the host cores: at
+    most `steps` steps and about budget_s seconds.  Returns (GB/s, steps, s)."""
+    import oracle
+    t0 = time.perf_counter()
+    done = 0
+    while done < steps:
+        for (xb, p, s, b) in ins:
+            oracle.matmul(xb, p, s, b, G, BITS)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return STEP_BYTES * done / dt / 1e9, done, dt
+
+
+def cpu_baseline(budget_s):
+    import oracle
+    ins = oracle_decode_inputs()
+    time_oracle(ins, 1, 0)  # warm
+    gbs, done, dt = time_oracle(ins, 10 ** 6, budget_s)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{done} full decode steps (all three linears at M=1) in {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    ins = oracle_decode_inputs()
+    time_oracle(ins, max(1, args.warmup // 1000), 5.0)
+    gbs, done, dt = time_oracle(ins, max(1, args.ref_steps), args.ref_budget)
+    cores = oracle.num_threads()
+    return {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": done, "warmup": 1, "ms_per_step": round(dt / done * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; shapes of Llama-3-8B linears; no checkpoints)",
+            "config": {"workload": WORKLOAD, "M": 1, "bits": BITS, "G": G, "shapes_KN": DECODE_SHAPES,
+                       "parallelism": "host cores (OpenMP)"},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{done} full decode steps in {dt:.1f} s"},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--qmm-reps", type=int, default=20)
+    ap.add_argument("--no-sections", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-steps", type=int, default=30)
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    pg = False
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        pg = True
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+            print(json.dumps(line), flush=True)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,129 @@
+/*
+ * aq.h — C ABI of a B200 (sm_100a) library for group-wise affine weight-only
+ * quantization and the quantized matmul that consumes it.
+ *
+ * The method (sources: metalworking "MLX Quantization", section "Mechanics";
+ * "Quantizing a Model for MLX", section "What MLX quantization stores"; anllm
+ * "Tutorial 10: Quantization", sections 2-5):
+ *   W[N,K] is cut along K into groups of G = 32, 64 or 128 consecutive values
+ *   of one row.  Each group stores one fp16 scale, one fp16 bias and 2/3/4/8-bit
+ *   unsigned codes, so that  w ~= code * scale + bias.
+ *     scale = fp16((max - min) / (2^bits - 1))   (fp32 arithmetic, RNE)
+ *     bias  = fp16(min)
+ *     code  = clamp(rint_even(fp32(fp32(w - bias) / scale)), 0, 2^bits - 1)
+ *             computed from the stored fp16 scale and bias; code 0 when scale == 0.
+ *   Codes of one row form an LSB-first bitstream: code k occupies bits
+ *   [k*bits, k*bits + bits) of the row, and word j holds bits [32j, 32j + 32).
+ *   For bits = 2/4/8 this is "(word >> bits*j) & mask" (Tutorial 10, section 3);
+ *   for bits = 3 a code may straddle two words (32 codes per 3 words).
+ *
+ * Types: fp16 and bf16 values travel as their 16-bit patterns (uint16_t).
+ * Layouts: every array is row-major and contiguous.
+ *   w        fp32      [N, K]
+ *   packed   uint32    [N, K*bits/32]
+ *   scales   fp16 bits [N, K/G]
+ *   biases   fp16 bits [N, K/G]
+ *   x        bf16 bits [M, K]
+ *   y        bf16 bits [M, N]       y = x @ dequant(W)^T
+ * Ownership: every pointer argument is DEVICE memory, allocated, owned and freed
+ * by the caller; the library allocates no device memory and needs no workspace.
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ * stream); outputs are valid once the stream reaches the call.
+ * Errors: arguments are validated synchronously, before anything is launched;
+ * a rejected call launches nothing and returns a non-zero status.  Nothing is
+ * thrown across the ABI and no kernel traps.
+ */
+#ifndef AQ_H_
+#define AQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *aq_stream_t;
+
+typedef enum {
+  AQ_OK = 0,
+  AQ_ERR_INVALID_ARG = 1, /* null pointer, N/M/K <= 0, K % G != 0, size overflow */
+  AQ_ERR_UNSUPPORTED = 2, /* bits not in {2,3,4,8}, G not in {32,64,128}, shape outside a forced kernel's range,
+                             or a device that is not sm_100 */
+  AQ_ERR_ALIGNMENT = 3,   /* a pointer not 16-byte aligned */
+  AQ_ERR_CUDA = 4,        /* a CUDA runtime error at launch (see aq_last_cuda_error) */
+  AQ_ERR_DEVICE_FAULT = 5 /* a kernel recorded a bounded-wait timeout (see aq_device_fault) */
+} aq_status;
+
+/* Kernel choice for aq_matmul_with (aq_matmul always uses AQ_KERNEL_AUTO). */
+typedef enum {
+  AQ_KERNEL_AUTO = 0, /* host-side per-shape dispatch (see aq_dispatch) */
+  AQ_KERNEL_QMV = 1,  /* CUDA-core streaming kernel, M <= 8 */
+  AQ_KERNEL_QMM = 2   /* tcgen05 / TMEM tensor-core kernel, any M */
+} aq_kernel;
+
+/* Words of the packed code array: N*K*bits/32 (0 if the arguments are invalid). */
+size_t aq_packed_words(int64_t N, int64_t K, int bits);
+
+/* Bytes of codes + scales + biases: N*K*bits/8 + 4*N*K/G (0 if invalid).
+ * At bits=4, G=64 this is 4.5 bits per weight ("Quantizing a Model for MLX",
+ * section "What MLX quantization stores"). */
+size_t aq_packed_bytes(int64_t N, int64_t K, int G, int bits);
+
+/* Quantize fp32 W[N,K] into packed codes, fp16 scales and fp16 biases.
+ * Source: metalworking "MLX Quantization", section "Mechanics" (mx.quantize);
+ * "Quantizing a Model for MLX", section "What MLX quantization stores".
+ * Results are bit-exact with the definition in this header. */
+aq_status aq_quantize(const float *w, int64_t N, int64_t K, int G, int bits,
+                      uint32_t *packed, uint16_t *scales, uint16_t *biases, aq_stream_t stream);
+
+/* Dequantize to bf16: w_out[n,k] = bf16_rn(fp32_rn(code*scale + bias)) (a single
+ * fp32 rounding of the exact value, then RNE to bf16).
+ * Source: anllm "Tutorial 10: Quantization", sections 3 and 7 (dequantize, then
+ * astype(bfloat16)). */
+aq_status aq_dequantize(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                        int64_t N, int64_t K, int G, int bits, uint16_t *w_out_bf16, aq_stream_t stream);
+
+/* Same as aq_dequantize with fp32 output fp32_rn(code*scale + bias). */
+aq_status aq_dequantize_f32(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                            int64_t N, int64_t K, int G, int bits, float *w_out, aq_stream_t stream);
+
+/* Quantized matmul y[M,N] = x[M,K] @ dequant(W)^T, fp32 accumulation, bf16 (RNE)
+ * output, without materialising dequant(W) in global memory.
+ * Source: anllm "Tutorial 10: Quantization", section 5, approach 2
+ * (mx.quantized_matmul(..., transpose=True)); metalworking "MLX Quantization",
+ * section "Mechanics" (QMV for decode, QMM for prefill, host-side per-shape
+ * dispatch).  Accuracy: |y - y_ref| <= 8e-3 * (|y_ref| + rms(y_ref)) against the
+ * exact product. */
+aq_status aq_matmul(const uint16_t *x_bf16, int64_t M, int64_t K,
+                    const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                    int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
+
+/* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV returns AQ_ERR_UNSUPPORTED
+ * when M > 8 or its shared-memory staging of x does not fit; AQ_KERNEL_QMM
+ * returns AQ_ERR_UNSUPPORTED when K*bits is not a multiple of 128. */
+aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x_bf16, int64_t M, int64_t K,
+                         const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                         int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
+
+/* The kernel aq_matmul would run for this shape (host logic only; no GPU needed),
+ * or -1 if the arguments would be rejected. */
+int aq_dispatch(int64_t M, int64_t N, int64_t K, int G, int bits);
+
+/* Human-readable name of a status code (static storage). */
+const char *aq_status_string(aq_status status);
+
+/* The last CUDA error code seen by this library on the calling thread (0 if none). */
+int aq_last_cuda_error(void);
+
+/* Reads and clears the device-side fault word of the current device: non-zero
+ * when a kernel gave up a bounded wait (an mbarrier that never completed) and
+ * returned early; its output is then invalid.  Synchronizes the device. */
+aq_status aq_device_fault(uint32_t *fault_word);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQ_H_ */

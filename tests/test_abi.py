@@ -1,0 +1,141 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and its host-side logic (sizes, dispatch, validation) holds.
+
+Calls here are either host-only (sizes, dispatch, status strings) or rejected
+by argument validation before any CUDA call is made, so they run on a machine
+without a GPU.
+"""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+import weight_only_group_b200 as aq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "aq.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden", "storage_arithmetic.json")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    if not os.path.exists(aq.LIB_PATH):
+        from weight_only_group_b200 import build
+        build.build()
+    return aq.lib()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(aq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for must in ("aq_quantize", "aq_dequantize", "aq_matmul", "aq_packed_bytes", "aq_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = aq.lib()
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_packed_bytes_match_printed_storage_figures():
+    st = json.load(open(GOLDEN))
+    # 4.5 bits / weight and 0.5625 bytes / parameter at bits=4, G=64
+    assert aq.aq_packed_bytes(64, 64, 64, 4) * 8 / (64 * 64) == st["bits_per_weight_4bit_G64"]["value"]
+    assert aq.aq_packed_bytes(4096, 14336, 64, 4) / (4096 * 14336) == st["bytes_per_param_4bit_G64"]["value"]
+    # the 70B prediction: N*K = 70,553,706,496 parameters (K = 64 divides it)
+    p = st["llama_3_3_70b_prediction"]["params"]
+    assert p % 64 == 0
+    assert aq.aq_packed_bytes(p // 64, 64, 64, 4) == st["llama_3_3_70b_prediction"]["bytes"]
+    r = st["linear_4096x14336_bf16_bytes"]["value"] / aq.aq_packed_bytes(4096, 14336, 64, 4)
+    assert abs(r - st["fp16_to_4bit_ratio"]["value"]) <= st["fp16_to_4bit_ratio"]["printed_precision"]
+
+
+@pytest.mark.parametrize("bits", (2, 3, 4, 8))
+@pytest.mark.parametrize("G", (32, 64, 128))
+def test_packed_sizes_formula(bits, G):
+    N, K = 37, 4 * 128
+    assert aq.aq_packed_words(N, K, bits) == N * K * bits // 32
+    assert aq.aq_packed_bytes(N, K, G, bits) == N * K * bits // 8 + 4 * N * K // G
+
+
+def test_packed_sizes_reject_invalid():
+    assert aq.aq_packed_bytes(4, 96, 64, 4) == 0      # K % G != 0
+    assert aq.aq_packed_bytes(4, 64, 16, 4) == 0      # G unsupported
+    assert aq.aq_packed_bytes(4, 64, 64, 5) == 0      # bits unsupported
+    assert aq.aq_packed_bytes(0, 64, 64, 4) == 0
+    assert aq.aq_packed_words(4, 64, 6) == 0
+
+
+def test_dispatch_rule():
+    # decode shapes -> QMV, prefill shapes -> QMM (the tensor-core kernel)
+    for M in range(1, 9):
+        assert aq.aq_dispatch(M, 14336, 4096, 64, 4) == aq.AQ_KERNEL_QMV
+    assert aq.aq_dispatch(1, 4096, 14336, 64, 4) == aq.AQ_KERNEL_QMV
+    assert aq.aq_dispatch(1, 28672, 8192, 32, 3) == aq.AQ_KERNEL_QMV
+    for M in (9, 64, 512, 8192):
+        assert aq.aq_dispatch(M, 14336, 4096, 64, 4) == aq.AQ_KERNEL_QMM
+    # x staging for QMV would not fit shared memory: QMM takes it
+    assert aq.aq_dispatch(8, 4096, 14336, 64, 4) == aq.AQ_KERNEL_QMM
+    # invalid shapes
+    assert aq.aq_dispatch(0, 4096, 4096, 64, 4) == -1
+    assert aq.aq_dispatch(1, 4096, 4000, 64, 4) == -1
+    assert aq.aq_dispatch(1, 4096, 4096, 64, 7) == -1
+
+
+def test_status_strings():
+    for s in range(6):
+        assert aq.aq_status_string(s)
+    assert "unknown" in aq.aq_status_string(99)
+
+
+# Fake device pointers: every call below is rejected by host-side validation
+# before any CUDA call, so nothing is dereferenced.
+A = 0x10000  # 16-byte aligned
+U = 0x10004  # misaligned
+
+
+def _q(w=A, N=4, K=64, G=64, bits=4, p=A, s=A, b=A):
+    return aq.lib().aq_quantize(w, N, K, G, bits, p, s, b, None)
+
+
+def test_quantize_validation():
+    assert _q(bits=5) == aq.AQ_ERR_UNSUPPORTED
+    assert _q(G=16) == aq.AQ_ERR_UNSUPPORTED
+    assert _q(K=96) == aq.AQ_ERR_INVALID_ARG
+    assert _q(N=0) == aq.AQ_ERR_INVALID_ARG
+    assert _q(K=-64) == aq.AQ_ERR_INVALID_ARG
+    assert _q(w=0) == aq.AQ_ERR_INVALID_ARG
+    assert _q(p=0) == aq.AQ_ERR_INVALID_ARG
+    assert _q(w=U) == aq.AQ_ERR_ALIGNMENT
+    assert _q(s=U) == aq.AQ_ERR_ALIGNMENT
+
+
+def test_matmul_validation():
+    L = aq.lib()
+    call = lambda k=0, x=A, M=1, K=64, N=8, G=64, bits=4, y=A: L.aq_matmul_with(k, x, M, K, A, A, A, N, G, bits, y,
+                                                                                 None)
+    assert call(bits=1) == aq.AQ_ERR_UNSUPPORTED
+    assert call(M=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(x=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(y=U) == aq.AQ_ERR_ALIGNMENT
+    assert call(k=7) == aq.AQ_ERR_INVALID_ARG
+    # QMV forced beyond its range
+    assert call(k=aq.AQ_KERNEL_QMV, M=9) == aq.AQ_ERR_UNSUPPORTED
+    # QMM needs a 16-byte packed row pitch: K*bits % 128 == 0 (K=96, 3 bits: 288 bits)
+    assert call(k=aq.AQ_KERNEL_QMM, M=64, K=96, G=32, bits=3) == aq.AQ_ERR_UNSUPPORTED
+    assert L.aq_dequantize(A, A, A, 4, 64, 64, 4, U, None) == aq.AQ_ERR_ALIGNMENT
+    assert L.aq_dequantize_f32(A, A, A, 4, 64, 64, 9, A, None) == aq.AQ_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        aq.aq_quantize(torch.zeros(4, 64), 64, 4)

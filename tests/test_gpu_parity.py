@@ -1,0 +1,240 @@
+"""GPU parity: the CUDA library, called through its C ABI (via the binding),
+against the CPU oracle on the same seeded inputs.
+
+Bars: packed codes, scales, biases and dequantized values bit-exact; the
+quantized matmul within |y - y_ref| <= 8e-3 * (|y_ref| + rms(y_ref)) of the
+exact fp64 product.  Sizes cover the five workloads (full size; the prefill
+QMM checks a seeded sample of token rows against the oracle, every column),
+plus ragged and degenerate shapes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from cases import activations_bits, quantized, sample_rows, weights
+
+pytestmark = pytest.mark.gpu
+
+aq = pytest.importorskip("weight_only_group_b200")
+RTOL = 8e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    aq.lib()
+    yield
+    assert aq.aq_device_fault() == 0
+
+
+def _gpu_quantize(w: np.ndarray, G: int, bits: int):
+    p, s, b = aq.aq_quantize(torch.from_numpy(w).cuda(), G, bits)
+    torch.cuda.synchronize()
+    return p, s, b
+
+
+def _u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def _u16(t):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def _to_gpu(p, s, b):
+    return (torch.from_numpy(p.view(np.int32)).cuda(), torch.from_numpy(s.view(np.float16)).cuda(),
+            torch.from_numpy(b.view(np.float16)).cuda())
+
+
+def _x_gpu(xbits: np.ndarray):
+    return torch.from_numpy(xbits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _assert_close(y_gpu: torch.Tensor, y_ref: np.ndarray, what: str, rms=None):
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    ok, worst = oracle.tolerance_ok(y, y_ref, RTOL, rms)
+    assert ok, f"{what}: worst |y-y_ref| / (8e-3 (|y_ref| + rms)) = {worst:.3f}"
+    return worst
+
+
+# ----------------------------------------------------------------------------- quantize / dequantize
+
+QUANT_CASES = [(c.N, c.K, c.w_seed, c.outliers, c.G, c.bits) for wl in synth.WORKLOADS[:2] for c in wl.cases]
+SWEEP = [(c.N, c.K, c.w_seed, c.outliers, c.G, c.bits) for c in synth.WORKLOADS[3].cases]
+EDGE_QUANT = [
+    (1, 32, 11, False, 32, 4), (3, 96, 12, True, 32, 3), (129, 128, 13, True, 128, 2),
+    (7, 192, 14, True, 64, 8), (33, 4096, 15, True, 128, 3), (5, 2048, 16, False, 32, 2),
+]
+
+
+@pytest.mark.parametrize("N,K,seed,outl,G,bits", QUANT_CASES + EDGE_QUANT)
+def test_quantize_dequantize_bitexact(N, K, seed, outl, G, bits):
+    w = weights(N, K, seed, outl)
+    p_ref, s_ref, b_ref = quantized(N, K, seed, outl, G, bits)
+    p, s, b = _gpu_quantize(w, G, bits)
+    assert np.array_equal(_u16(s), s_ref)
+    assert np.array_equal(_u16(b), b_ref)
+    assert np.array_equal(_u32(p), p_ref)
+    d = aq.aq_dequantize(p, s, b, K, G, bits)
+    assert np.array_equal(_u16(d), oracle.dequantize_bf16(p_ref, s_ref, b_ref, K, G, bits))
+    f = aq.aq_dequantize_f32(p, s, b, K, G, bits)
+    assert np.array_equal(f.cpu().numpy(), oracle.dequantize_f32(p_ref, s_ref, b_ref, K, G, bits))
+
+
+@pytest.mark.parametrize("N,K,seed,outl,G,bits", SWEEP, ids=[f"b{c[5]}G{c[4]}" for c in SWEEP])
+def test_quantize_sweep_full_size_bitexact(N, K, seed, outl, G, bits):
+    w = weights(N, K, seed, outl)
+    p_ref, s_ref, b_ref = quantized(N, K, seed, outl, G, bits)
+    p, s, b = _gpu_quantize(w, G, bits)
+    assert np.array_equal(_u16(s), s_ref)
+    assert np.array_equal(_u16(b), b_ref)
+    assert np.array_equal(_u32(p), p_ref)
+
+
+def test_quantize_special_values():
+    """Degenerate groups, signed zeros, a subnormal fp16 scale, large magnitudes."""
+    rng = np.random.default_rng(3)
+    w = rng.normal(0, 0.02, (8, 256)).astype(np.float32)
+    w[0, :64] = 0.25                                     # constant group: scale 0, codes 0
+    w[1, :64] = 0.0
+    w[1, 3] = -0.0                                       # signed zeros in a zero group
+    w[2, :64] = np.arange(64, dtype=np.float32) * 2.0 ** -24 / 4  # range below one fp16 ulp of 1
+    w[3, :64] = rng.normal(0, 1e4, 64).astype(np.float32)          # large values
+    w[4, :] = -np.abs(w[4, :])                                     # all-negative row
+    w[5, 64:128] = np.float32(-0.0)
+    w[5, 70] = 1.0
+    for G in (32, 64, 128):
+        for bits in (2, 3, 4, 8):
+            p_ref, s_ref, b_ref = oracle.quantize(w, G, bits)
+            p, s, b = _gpu_quantize(w, G, bits)
+            assert np.array_equal(_u16(s), s_ref), (G, bits)
+            assert np.array_equal(_u16(b), b_ref), (G, bits)
+            assert np.array_equal(_u32(p), p_ref), (G, bits)
+            d = aq.aq_dequantize_f32(p, s, b, 256, G, bits)
+            assert np.array_equal(d.cpu().numpy(), oracle.dequantize_f32(p_ref, s_ref, b_ref, 256, G, bits))
+
+
+# ----------------------------------------------------------------------------- QMV (decode)
+
+def _matmul_case(M, K, N, bits, G, seed, kernel, outl=True, full=True, n_rows=48):
+    p_ref, s_ref, b_ref = quantized(N, K, seed, outl, G, bits)
+    xb = activations_bits(M, K, seed + 1)
+    pg, sg, bg = _to_gpu(p_ref, s_ref, b_ref)
+    y = aq.aq_matmul_with(kernel, _x_gpu(xb), pg, sg, bg, G, bits)
+    torch.cuda.synchronize()
+    if full:
+        y_ref = oracle.matmul(xb, p_ref, s_ref, b_ref, G, bits)
+        return _assert_close(y, y_ref, f"{kernel} M={M} K={K} N={N} b={bits} G={G}"), y
+    rows = sample_rows(M, n_rows, seed)
+    y_ref = oracle.matmul_sampled(xb, p_ref, s_ref, b_ref, G, bits, rows, np.arange(N))
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    return _assert_close(y[torch.from_numpy(rows).cuda()], y_ref, f"{kernel} M={M} K={K} N={N} (sampled)", rms), y
+
+
+@pytest.mark.parametrize("c", [c for c in synth.WORKLOADS[0].cases + synth.WORKLOADS[1].cases],
+                         ids=lambda c: c.name)
+def test_qmv_decode_workloads(c):
+    _matmul_case(c.M, c.K, c.N, c.bits, c.G, c.w_seed, "auto", c.outliers)
+    assert aq.aq_dispatch(c.M, c.N, c.K, c.G, c.bits) == aq.AQ_KERNEL_QMV
+
+
+@pytest.mark.parametrize("c", synth.WORKLOADS[2].cases, ids=lambda c: c.name)
+def test_qmv_small_m(c):
+    _matmul_case(c.M, c.K, c.N, c.bits, c.G, c.w_seed, "qmv", c.outliers)
+
+
+@pytest.mark.parametrize("c", synth.WORKLOADS[3].cases, ids=lambda c: c.name)
+def test_qmv_bits_group_sweep(c):
+    _matmul_case(c.M, c.K, c.N, c.bits, c.G, c.w_seed, "qmv", c.outliers)
+
+
+@pytest.mark.parametrize("M", (1, 2, 3, 5, 7, 8))
+@pytest.mark.parametrize("bits", (2, 3, 4, 8))
+@pytest.mark.parametrize("K,N,G", [(32, 1, 32), (96, 3, 32), (128, 37, 64), (640, 129, 128), (1024, 250, 64)])
+def test_qmv_ragged_and_tiny(M, bits, K, N, G):
+    _matmul_case(M, K, N, bits, G, 7000 + K + N, "qmv")
+
+
+def test_qmv_all_zero_codes_closed_form():
+    """All codes 0: y[m, n] = sum_g bias[n, g] * sum_{k in g} x[m, k]."""
+    M, N, K, G = 3, 77, 512, 64
+    rng = np.random.default_rng(1)
+    p = np.zeros((N, K * 4 // 32), np.uint32)
+    s = rng.normal(0, 0.01, (N, K // G)).astype(np.float16).view(np.uint16)
+    b = rng.normal(0, 0.1, (N, K // G)).astype(np.float16).view(np.uint16)
+    xb = activations_bits(M, K, 5)
+    x64 = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).double().numpy()
+    y_cf = x64.reshape(M, K // G, G).sum(-1) @ b.view(np.float16).astype(np.float64).T
+    y = aq.aq_matmul_with("qmv", _x_gpu(xb), *_to_gpu(p, s, b), G, 4)
+    _assert_close(y, y_cf, "zero codes")
+
+
+# ----------------------------------------------------------------------------- QMM (prefill, tcgen05)
+
+@pytest.mark.parametrize("c", synth.WORKLOADS[4].cases, ids=lambda c: c.name)
+def test_qmm_prefill_workloads(c):
+    _matmul_case(c.M, c.K, c.N, c.bits, c.G, c.w_seed, "auto", c.outliers, full=False, n_rows=40)
+    assert aq.aq_dispatch(c.M, c.N, c.K, c.G, c.bits) == aq.AQ_KERNEL_QMM
+
+
+@pytest.mark.parametrize("bits", (2, 3, 4, 8))
+@pytest.mark.parametrize("G", (32, 64, 128))
+def test_qmm_bits_groups(bits, G):
+    _matmul_case(300, 1024, 384, bits, G, 8100 + bits * 10 + G, "qmm")
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 128, 128), (9, 256, 130), (64, 512, 256), (65, 384, 200),
+                                   (129, 640, 129), (256, 1024, 1000), (257, 128, 384), (700, 2048, 300)])
+def test_qmm_ragged(M, K, N):
+    _matmul_case(M, K, N, 4, 64 if K % 64 == 0 else 32, 9000 + M + N, "qmm")
+
+
+def test_qmm_matches_dequantize_then_matmul():
+    """The fused product equals dequantize-then-multiply (anllm Tutorial 10, section 5):
+    the kernel's weights are exactly aq_dequantize's bf16 values, so a torch fp32
+    matmul of those values agrees to fp32 summation-order error."""
+    M, K, N, G, bits = 512, 4096, 1024, 64, 4
+    p_ref, s_ref, b_ref = quantized(N, K, 424, True, G, bits)
+    pg, sg, bg = _to_gpu(p_ref, s_ref, b_ref)
+    x = _x_gpu(activations_bits(M, K, 425))
+    y = aq.aq_matmul_with("qmm", x, pg, sg, bg, G, bits).float()
+    wd = aq.aq_dequantize(pg, sg, bg, K, G, bits).float()
+    y_ref = x.float() @ wd.T
+    err = (y - y_ref).abs() / (y_ref.abs() + y_ref.pow(2).mean().sqrt())
+    assert float(err.max()) < 2 ** -7  # bf16 output rounding plus fp32 order
+
+
+def test_kernels_agree_on_small_m():
+    M, K, N, G, bits = 8, 4096, 2048, 64, 4
+    w1, _ = _matmul_case(M, K, N, bits, G, 555, "qmv")
+    w2, _ = _matmul_case(M, K, N, bits, G, 555, "qmm")
+    assert w1 <= 1.0 and w2 <= 1.0
+
+
+def test_auto_equals_dispatched_kernel_and_is_deterministic():
+    for M in (1, 4, 600):
+        K, N, G, bits = 4096, 1536, 64, 4
+        p_ref, s_ref, b_ref = quantized(N, K, 77, True, G, bits)
+        pg, sg, bg = _to_gpu(p_ref, s_ref, b_ref)
+        x = _x_gpu(activations_bits(M, K, 78))
+        kern = {aq.AQ_KERNEL_QMV: "qmv", aq.AQ_KERNEL_QMM: "qmm"}[aq.aq_dispatch(M, N, K, G, bits)]
+        y1 = aq.aq_matmul(x, pg, sg, bg, G, bits)
+        y2 = aq.aq_matmul_with(kern, x, pg, sg, bg, G, bits)
+        y3 = aq.aq_matmul(x, pg, sg, bg, G, bits)
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+        assert torch.equal(y1.view(torch.int16), y3.view(torch.int16))
+
+
+def test_rejects_misaligned_device_pointer():
+    x = torch.zeros(1, 65, dtype=torch.bfloat16, device="cuda")[:, 1:]  # 2-byte offset
+    p, s, b = _gpu_quantize(np.zeros((8, 64), np.float32), 64, 4)
+    with pytest.raises(aq.AqError) as e:
+        aq.lib()
+        rc = aq.lib().aq_matmul(x.data_ptr(), 1, 64, p.data_ptr(), s.data_ptr(), b.data_ptr(), 8, 64, 4,
+                                torch.empty(1, 8, dtype=torch.bfloat16, device="cuda").data_ptr(), None)
+        aq._check(rc, "aq_matmul")
+    assert e.value.status == aq.AQ_ERR_ALIGNMENT

@@ -1,0 +1,202 @@
+"""Python binding of the aq C ABI (include/aq.h), a B200 (sm_100a) library for
+group-wise affine weight-only quantization and the quantized matmul.
+
+This module only marshals arguments: it checks tensor dtypes/shapes/devices,
+allocates outputs with PyTorch, and passes raw device pointers and the current
+CUDA stream to ``libaq.so``.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and importing the
+binding fails loudly when the library has not been built
+(``python -m weight_only_group_b200.build``).
+
+Names mirror the C entry points: ``aq_quantize``, ``aq_dequantize``,
+``aq_dequantize_f32``, ``aq_matmul``, ``aq_matmul_with``, ``aq_dispatch``,
+``aq_packed_words``, ``aq_packed_bytes``, ``aq_status_string``,
+``aq_device_fault``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libaq.so")
+
+AQ_OK = 0
+AQ_ERR_INVALID_ARG = 1
+AQ_ERR_UNSUPPORTED = 2
+AQ_ERR_ALIGNMENT = 3
+AQ_ERR_CUDA = 4
+AQ_ERR_DEVICE_FAULT = 5
+
+AQ_KERNEL_AUTO = 0
+AQ_KERNEL_QMV = 1
+AQ_KERNEL_QMM = 2
+KERNELS = {"auto": AQ_KERNEL_AUTO, "qmv": AQ_KERNEL_QMV, "qmm": AQ_KERNEL_QMM}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {aq_status_string(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libaq.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is not built: run `python -m weight_only_group_b200.build` "
+                                  "(the CUDA library is required; there is no fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            i64, i32, vp, u64 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+            L.aq_packed_words.argtypes = [i64, i64, i32]
+            L.aq_packed_words.restype = u64
+            L.aq_packed_bytes.argtypes = [i64, i64, i32, i32]
+            L.aq_packed_bytes.restype = u64
+            L.aq_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
+            L.aq_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
+            L.aq_dequantize_f32.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
+            L.aq_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
+            L.aq_matmul_with.argtypes = [i32, vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
+            L.aq_dispatch.argtypes = [i64, i64, i64, i32, i32]
+            L.aq_dispatch.restype = i32
+            L.aq_status_string.argtypes = [i32]
+            L.aq_status_string.restype = ctypes.c_char_p
+            L.aq_last_cuda_error.restype = i32
+            L.aq_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+            for f in ("aq_quantize", "aq_dequantize", "aq_dequantize_f32", "aq_matmul", "aq_matmul_with",
+                      "aq_device_fault"):
+                getattr(L, f).restype = i32
+            _lib = L
+    return _lib
+
+
+# ----------------------------------------------------------------------------- host-only calls
+
+def aq_packed_words(N: int, K: int, bits: int) -> int:
+    return int(lib().aq_packed_words(N, K, bits))
+
+
+def aq_packed_bytes(N: int, K: int, G: int, bits: int) -> int:
+    return int(lib().aq_packed_bytes(N, K, G, bits))
+
+
+def aq_dispatch(M: int, N: int, K: int, G: int, bits: int) -> int:
+    return int(lib().aq_dispatch(M, N, K, G, bits))
+
+
+def aq_status_string(status: int) -> str:
+    return lib().aq_status_string(status).decode()
+
+
+def aq_last_cuda_error() -> int:
+    return int(lib().aq_last_cuda_error())
+
+
+# ----------------------------------------------------------------------------- device calls
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtypes, ndim: int = 2) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor")
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != AQ_OK:
+        raise AqError(rc, what)
+
+
+_WORD = (torch.int32, torch.uint32)
+_HALF = (torch.float16, torch.int16, torch.uint16)
+
+
+def aq_quantize(w: torch.Tensor, G: int, bits: int):
+    """w fp32 [N, K] on the GPU -> (packed int32 [N, K*bits/32], scales fp16 [N, K/G], biases fp16 [N, K/G])."""
+    _need(w, "w", (torch.float32,))
+    N, K = w.shape
+    packed = torch.empty((N, K * bits // 32), dtype=torch.int32, device=w.device)
+    scales = torch.empty((N, max(K // G, 1)), dtype=torch.float16, device=w.device)
+    biases = torch.empty_like(scales)
+    with torch.cuda.device(w.device):
+        rc = lib().aq_quantize(w.data_ptr(), N, K, G, bits, packed.data_ptr(), scales.data_ptr(),
+                               biases.data_ptr(), _stream(w))
+    _check(rc, "aq_quantize")
+    return packed, scales, biases
+
+
+def _qw(packed, scales, biases):
+    _need(packed, "packed", _WORD)
+    _need(scales, "scales", _HALF)
+    _need(biases, "biases", _HALF)
+    if scales.shape != biases.shape or packed.shape[0] != scales.shape[0]:
+        raise ValueError("packed, scales and biases disagree on N")
+    return packed.shape[0]
+
+
+def aq_dequantize(packed, scales, biases, K: int, G: int, bits: int, out: torch.Tensor | None = None):
+    """-> bf16 [N, K] = bf16_rn(fp32_rn(code*scale + bias))."""
+    N = _qw(packed, scales, biases)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
+    _need(out, "out", (torch.bfloat16,))
+    with torch.cuda.device(packed.device):
+        rc = lib().aq_dequantize(packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, K, G, bits,
+                                 out.data_ptr(), _stream(packed))
+    _check(rc, "aq_dequantize")
+    return out
+
+
+def aq_dequantize_f32(packed, scales, biases, K: int, G: int, bits: int, out: torch.Tensor | None = None):
+    """-> fp32 [N, K] = fp32_rn(code*scale + bias)."""
+    N = _qw(packed, scales, biases)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float32, device=packed.device)
+    _need(out, "out", (torch.float32,))
+    with torch.cuda.device(packed.device):
+        rc = lib().aq_dequantize_f32(packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, K, G, bits,
+                                     out.data_ptr(), _stream(packed))
+    _check(rc, "aq_dequantize_f32")
+    return out
+
+
+def aq_matmul_with(kernel, x, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None):
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T with an explicit kernel ("auto", "qmv", "qmm")."""
+    k = KERNELS[kernel] if isinstance(kernel, str) else int(kernel)
+    _need(x, "x", (torch.bfloat16,))
+    N = _qw(packed, scales, biases)
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16,))
+    with torch.cuda.device(x.device):
+        rc = lib().aq_matmul_with(k, x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(),
+                                  biases.data_ptr(), N, G, bits, out.data_ptr(), _stream(x))
+    _check(rc, "aq_matmul")
+    return out
+
+
+def aq_matmul(x, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None):
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T, kernel chosen per shape by the library."""
+    return aq_matmul_with(AQ_KERNEL_AUTO, x, packed, scales, biases, G, bits, out)
+
+
+def aq_device_fault() -> int:
+    """Read and clear the device fault word (non-zero: a kernel gave up a bounded wait)."""
+    w = ctypes.c_uint32(0)
+    _check(lib().aq_device_fault(ctypes.byref(w)), "aq_device_fault")
+    return int(w.value)

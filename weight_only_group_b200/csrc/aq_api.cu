@@ -1,0 +1,176 @@
+// C ABI entry points: argument validation, per-shape dispatch, launches.
+// Method and layouts: see include/aq.h.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace aq {
+cudaError_t launch_quantize(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed,
+                            uint16_t *scales, uint16_t *biases, cudaStream_t s);
+cudaError_t launch_dequantize(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                              int64_t N, int64_t K, int G, int bits, void *out, bool bf16_out, cudaStream_t s);
+cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
+size_t qmv_required_smem(int64_t M, int64_t K);
+cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
+bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits);
+cudaError_t read_and_clear_fault(uint32_t *word);
+}  // namespace aq
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+// Largest dynamic shared memory a CTA may use on sm_100 (227 KB).
+constexpr size_t kMaxSmemPerBlock = 227 * 1024;
+// Upper bound of N, K (kernels index rows and columns with 32-bit ints).
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+bool valid_bits(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 8; }
+bool valid_group(int G) { return G == 32 || G == 64 || G == 128; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape validation shared by all entry points: AQ_OK, or the status to return.
+aq_status check_shape(int64_t N, int64_t K, int G, int bits) {
+  if (N <= 0 || K <= 0 || N > kMaxDim || K > kMaxDim) return AQ_ERR_INVALID_ARG;
+  if (!valid_bits(bits) || !valid_group(G)) return AQ_ERR_UNSUPPORTED;
+  if (K % G != 0) return AQ_ERR_INVALID_ARG;
+  // N*K elements must fit comfortably in int64 arithmetic (bytes of fp32 W).
+  if (N > (int64_t(1) << 62) / (4 * K)) return AQ_ERR_INVALID_ARG;
+  return AQ_OK;
+}
+
+aq_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return AQ_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return AQ_ERR_CUDA;
+}
+
+// The kernels are built for sm_100a only.  Checked once per device.
+aq_status check_device() {
+  static std::mutex mu;
+  static int checked[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return from_cuda(e);
+  if (dev < 0 || dev >= 64) return AQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (checked[dev] == 0) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return from_cuda(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return from_cuda(e);
+    checked[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return checked[dev] == 1 ? AQ_OK : AQ_ERR_UNSUPPORTED;
+}
+
+bool qmv_fits(int64_t M, int64_t K) { return M >= 1 && M <= 8 && aq::qmv_required_smem(M, K) <= kMaxSmemPerBlock; }
+
+}  // namespace
+
+extern "C" {
+
+size_t aq_packed_words(int64_t N, int64_t K, int bits) {
+  if (N <= 0 || K <= 0 || !valid_bits(bits) || K % 32 != 0) return 0;
+  if (N > (int64_t(1) << 62) / K) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K) * static_cast<size_t>(bits) / 32;
+}
+
+size_t aq_packed_bytes(int64_t N, int64_t K, int G, int bits) {
+  if (check_shape(N, K, G, bits) != AQ_OK) return 0;
+  const size_t nk = static_cast<size_t>(N) * static_cast<size_t>(K);
+  return nk * static_cast<size_t>(bits) / 8 + 4 * nk / static_cast<size_t>(G);
+}
+
+const char *aq_status_string(aq_status status) {
+  switch (status) {
+    case AQ_OK: return "ok";
+    case AQ_ERR_INVALID_ARG: return "invalid argument";
+    case AQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case AQ_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case AQ_ERR_CUDA: return "CUDA error";
+    case AQ_ERR_DEVICE_FAULT: return "device fault (bounded wait expired)";
+  }
+  return "unknown status";
+}
+
+int aq_last_cuda_error(void) { return t_last_cuda_error; }
+
+aq_status aq_quantize(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed, uint16_t *scales,
+                      uint16_t *biases, aq_stream_t stream) {
+  aq_status st = check_shape(N, K, G, bits);
+  if (st != AQ_OK) return st;
+  if (!w || !packed || !scales || !biases) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(packed) || !aligned16(scales) || !aligned16(biases)) return AQ_ERR_ALIGNMENT;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_quantize(w, N, K, G, bits, packed, scales, biases, stream));
+}
+
+static aq_status dequantize_common(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                                   int64_t N, int64_t K, int G, int bits, void *out, bool bf16, aq_stream_t stream) {
+  aq_status st = check_shape(N, K, G, bits);
+  if (st != AQ_OK) return st;
+  if (!packed || !scales || !biases || !out) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(scales) || !aligned16(biases) || !aligned16(out)) return AQ_ERR_ALIGNMENT;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_dequantize(packed, scales, biases, N, K, G, bits, out, bf16, stream));
+}
+
+aq_status aq_dequantize(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases, int64_t N,
+                        int64_t K, int G, int bits, uint16_t *w_out_bf16, aq_stream_t stream) {
+  return dequantize_common(packed, scales, biases, N, K, G, bits, w_out_bf16, true, stream);
+}
+
+aq_status aq_dequantize_f32(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases, int64_t N,
+                            int64_t K, int G, int bits, float *w_out, aq_stream_t stream) {
+  return dequantize_common(packed, scales, biases, N, K, G, bits, w_out, false, stream);
+}
+
+int aq_dispatch(int64_t M, int64_t N, int64_t K, int G, int bits) {
+  if (M <= 0 || M > kMaxDim || check_shape(N, K, G, bits) != AQ_OK) return -1;
+  if (qmv_fits(M, K)) return AQ_KERNEL_QMV;
+  if (aq::qmm_supports(M, N, K, G, bits)) return AQ_KERNEL_QMM;
+  return -1;
+}
+
+aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                         const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
+                         aq_stream_t stream) {
+  aq_status st = check_shape(N, K, G, bits);
+  if (st != AQ_OK) return st;
+  if (M <= 0 || M > kMaxDim) return AQ_ERR_INVALID_ARG;
+  if (!x || !packed || !scales || !biases || !y) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(biases) || !aligned16(y))
+    return AQ_ERR_ALIGNMENT;
+  if (kernel == AQ_KERNEL_AUTO) {
+    const int k = aq_dispatch(M, N, K, G, bits);
+    if (k < 0) return AQ_ERR_UNSUPPORTED;
+    kernel = static_cast<aq_kernel>(k);
+  }
+  if (kernel == AQ_KERNEL_QMV) {
+    if (!qmv_fits(M, K)) return AQ_ERR_UNSUPPORTED;
+    if ((st = check_device()) != AQ_OK) return st;
+    return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, stream));
+  }
+  if (kernel == AQ_KERNEL_QMM) {
+    if (!aq::qmm_supports(M, N, K, G, bits)) return AQ_ERR_UNSUPPORTED;
+    if ((st = check_device()) != AQ_OK) return st;
+    return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, stream));
+  }
+  return AQ_ERR_INVALID_ARG;
+}
+
+aq_status aq_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                    const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, aq_stream_t stream) {
+  return aq_matmul_with(AQ_KERNEL_AUTO, x, M, K, packed, scales, biases, N, G, bits, y, stream);
+}
+
+aq_status aq_device_fault(uint32_t *fault_word) {
+  if (!fault_word) return AQ_ERR_INVALID_ARG;
+  return from_cuda(aq::read_and_clear_fault(fault_word));
+}
+
+}  // extern "C"

@@ -1,0 +1,168 @@
+// Shared device helpers of the CUDA path (sm_100a only).  Nothing here is
+// shared with, or derived from, the CPU oracle.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/aq.h"
+
+#define AQ_DEVICE __device__ __forceinline__
+
+namespace aq {
+
+// Bits of the device-side fault word (defined next to the only kernel with
+// waits): set, never trapped, when a bounded wait gives up.
+enum : uint32_t {
+  kFaultMmaWait = 1u << 0,      // MMA issuer gave up waiting for operands
+  kFaultProducerWait = 1u << 1, // TMA producer gave up waiting for a free stage
+  kFaultDequantWait = 1u << 2,  // dequant warps gave up waiting for packed data / a free A stage
+  kFaultEpilogueWait = 1u << 3, // epilogue gave up waiting for the accumulator
+};
+
+// Upper bound of any spin on an mbarrier, in SM clock cycles (~1 s at 2 GHz).
+constexpr long long kWaitCycles = 2000000000LL;
+
+// ---------------------------------------------------------------------------
+// Loads
+// ---------------------------------------------------------------------------
+AQ_DEVICE uint4 ldg_stream16(const void *p) {  // read-once stream: skip L1
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+AQ_DEVICE uint4 ldg_nc16(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+AQ_DEVICE uint2 ldg_nc8(const void *p) {
+  uint2 v;
+  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+AQ_DEVICE uint32_t ldg_nc4(const void *p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+AQ_DEVICE uint16_t ldg_nc2(const void *p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+AQ_DEVICE float half_bits_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+AQ_DEVICE float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+AQ_DEVICE uint32_t smem_u32(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+// Packed fp32x2 FMA (sm_100): d = a * b + c on both halves.
+AQ_DEVICE float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long A = *reinterpret_cast<unsigned long long *>(&a);
+  unsigned long long B = *reinterpret_cast<unsigned long long *>(&b);
+  unsigned long long C = *reinterpret_cast<unsigned long long *>(&c);
+  unsigned long long D;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(D) : "l"(A), "l"(B), "l"(C));
+  return *reinterpret_cast<float2 *>(&D);
+}
+AQ_DEVICE float2 fadd2(float2 a, float2 b) {
+  unsigned long long A = *reinterpret_cast<unsigned long long *>(&a);
+  unsigned long long B = *reinterpret_cast<unsigned long long *>(&b);
+  unsigned long long D;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
+  return *reinterpret_cast<float2 *>(&D);
+}
+
+// ---------------------------------------------------------------------------
+// Code extraction into "magic" floats.
+//
+// A code field of `bits` bits is moved, by a rotation of its 32-bit word by a
+// multiple of 8, to a position p inside the fp32 mantissa and OR-ed with the
+// exponent of 1.0, giving the float f = 1 + q * 2^(p-23) exactly.  p is chosen
+// in [16-bits, 23-bits] so the field's top bit lies at 15..22.  The consumer
+// recovers q*x as x*2^(23-p)*f - x*2^(23-p); the 2^(23-p) factor is folded
+// into pre-scaled activations, so all products of one chunk accumulate in one
+// register.  Rotations by multiples of 8 are shared by the fields of a word.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kOne = 0x3F800000u;
+
+struct FieldPlace {
+  int word;      // word of the chunk holding the field's first bit
+  int off;       // bit offset of the field in that word
+  int rot;       // left rotation applied (0/8/16/24), or -1 if the field straddles two words
+  int p;         // mantissa bit where the field lands
+};
+
+__host__ __device__ constexpr int field_pmin(int bits) { return 16 - bits; }
+__host__ __device__ constexpr int field_pmax(int bits) { return 23 - bits; }
+
+__host__ __device__ constexpr FieldPlace field_place(int bits, int j) {
+  const int bp = j * bits, word = bp / 32, off = bp % 32;
+  if (off + bits > 32) return FieldPlace{word, off, -1, field_pmax(bits)};
+  if (bits == 8) return FieldPlace{word, off, 0, 8};  // byte permute, see extract_magic
+  for (int r = 0; r < 32; r += 8) {
+    const int p = (off + r) % 32;
+    if (p >= field_pmin(bits) && p <= field_pmax(bits)) return FieldPlace{word, off, r, p};
+  }
+  return FieldPlace{word, off, -2, 0};  // unreachable for bits in {2,3,4}
+}
+
+// 2^(23 - p) for code j of a 32-code chunk.
+__host__ __device__ constexpr float field_factor(int bits, int j) {
+  const int e = 23 - field_place(bits, j).p;
+  float f = 1.0f;
+  for (int i = 0; i < e; ++i) f *= 2.0f;
+  return f;
+}
+
+// Magic float bits for code J (0..31) of a chunk held in w[0..BITS-1].
+template <int BITS, int J>
+AQ_DEVICE uint32_t extract_magic(const uint32_t (&w)[BITS]) {
+  constexpr FieldPlace fp = field_place(BITS, J);
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  if constexpr (BITS == 8) {
+    // bytes of the result: [0x00, code, 0x80, 0x3F] -> 1 + code * 2^-15
+    constexpr uint32_t sel = 0x7604u | (uint32_t(fp.off / 8) << 4);
+    return __byte_perm(w[fp.word], kOne, sel);
+  } else if constexpr (fp.rot < 0) {
+    const uint32_t v = __funnelshift_r(w[fp.word], w[fp.word + 1], fp.off);
+    return ((v << fp.p) & (mask << fp.p)) | kOne;
+  } else {
+    const uint32_t v = fp.rot ? __funnelshift_l(w[fp.word], w[fp.word], fp.rot) : w[fp.word];
+    return (v & (mask << fp.p)) | kOne;
+  }
+}
+
+// Code J as an exact small integer (for the quantize/dequantize kernels).
+template <int BITS, int J>
+AQ_DEVICE uint32_t extract_code(const uint32_t (&w)[BITS]) {
+  constexpr int bp = J * BITS, word = bp / 32, off = bp % 32;
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  if constexpr (off + BITS <= 32) {
+    return (w[word] >> off) & mask;
+  } else {
+    return __funnelshift_r(w[word], w[word + 1], off) & mask;
+  }
+}
+
+template <int N>
+struct Int {
+  static constexpr int value = N;
+};
+
+template <int Begin, int End, class F>
+AQ_DEVICE void static_for(F &&f) {
+  if constexpr (Begin < End) {
+    f(Int<Begin>{});
+    static_for<Begin + 1, End>(f);
+  }
+}
+
+}  // namespace aq

@@ -1,0 +1,489 @@
+// QMM: quantized matrix x matrix for prefill on the 5th-generation tensor
+// cores (tcgen05 + tensor memory), sm_100a.
+//
+// Method: metalworking "MLX Quantization", section "Mechanics": QMM is the
+// prefill/batch case: dequantize weight tiles on chip, then a tiled GEMM
+// against them; "One trap for intuition": dequantize on every use, never a
+// cached fp16 copy.  anllm "Tutorial 10: Quantization", section 5: the fused
+// product equals dequantize-then-multiply; here every dequantized weight is
+// bf16_rn(fp32_rn(q*scale + bias)), exactly the value aq_dequantize writes, and
+// the products are accumulated in fp32.
+//
+// B200 design ("swap AB": weights are the MMA's A operand, tokens its N):
+//  * CTA tile: 128 rows of W (MMA M = 128, one TMEM lane per row) x BN tokens
+//    (MMA N = BN <= 256); persistent CTAs walk the tiles, token tiles fastest.
+//  * Warp 0 (one lane): TMA producer.  Per K block it loads the x tile
+//    [BN tokens x BK] (bf16, 128-byte swizzle, the canonical K-major UMMA
+//    layout) and the packed W tile [128 rows x BK*bits/32 words] into a ring
+//    of shared-memory stages, completing on the stage's mbarrier.
+//  * Warps 4..11 (two per TMEM lane quadrant): dequantize.  Thread (quadrant,
+//    lane) owns W row 32*quadrant+lane and one half of the K block: it reads
+//    its packed words from shared memory, turns codes into bf16 weights in
+//    registers and writes them with tcgen05.st straight into a TMEM stage
+//    that the MMA reads as operand A (no swizzled shared-memory round trip).
+//  * Warp 1 (one lane): issues tcgen05.mma.kind::f16 (A from TMEM, B from
+//    shared memory, fp32 accumulator of 128 x BN in TMEM) and tcgen05.commit
+//    to release stages; warp 1 also owns the TMEM allocation.
+//  * Epilogue: the dequant warps read the accumulator with tcgen05.ld and
+//    store bf16 (RNE) y[m, n] (a warp writes 32 consecutive n per token).
+//  * Every mbarrier wait is bounded; on expiry the kernel records a bit in a
+//    device fault word, stops issuing work and exits cleanly.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace aq {
+
+__device__ uint32_t g_fault_word = 0;
+
+namespace qmm {
+
+constexpr int kThreads = 384;     // 12 warps
+constexpr int kDequantWarp0 = 4;  // warps 4..11 dequantize + epilogue
+constexpr int kTmemCols = 512;
+constexpr int kAccCol = 0;        // accumulator columns [0, BN); A stages follow from column BN
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+AQ_DEVICE void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+AQ_DEVICE void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+AQ_DEVICE void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+AQ_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: true once the phase of the given parity completed, false on
+// timeout or when another role already aborted (the fault bit is recorded).
+AQ_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t fault_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(&g_fault_word, fault_bit);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+AQ_DEVICE void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+AQ_DEVICE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+AQ_DEVICE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+AQ_DEVICE void tc_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate)
+AQ_DEVICE void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+AQ_DEVICE void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+AQ_DEVICE void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+AQ_DEVICE void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+AQ_DEVICE void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row atoms of
+// 1024 bytes (stride byte offset 1024), descriptor version 1 (sm_100).
+AQ_DEVICE uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);      // start address
+  d |= static_cast<uint64_t>(1u) << 16;                        // leading byte offset (unused with swizzle)
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;                // stride byte offset
+  d |= static_cast<uint64_t>(1u) << 46;                        // version
+  d |= static_cast<uint64_t>(2u) << 61;                        // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major, M = 128, N = bn.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int bn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Tile configuration
+// ---------------------------------------------------------------------------
+template <int BITS, int BN>
+struct Cfg {
+  static constexpr int BK = (BITS == 3) ? 128 : 64;         // K per stage (elements)
+  static constexpr int BKW = BK * BITS / 32;                // packed words per W row per stage
+  static constexpr int X_BYTES = BN * BK * 2;               // x tile bytes
+  static constexpr int W_BYTES = 128 * BKW * 4;             // packed W tile bytes
+  static constexpr int STAGE_BYTES = ((X_BYTES + W_BYTES + 1023) / 1024) * 1024;
+  static constexpr int SMEM_BUDGET = 225 * 1024;
+  static constexpr int A_COLS = BK / 2;                     // TMEM columns per A stage (2 bf16 per column)
+  static constexpr int A_COL0 = BN;                         // first TMEM column of the A stages
+  static constexpr int STAGES = std::min(std::min(6, SMEM_BUDGET / STAGE_BYTES), (kTmemCols - A_COL0) / A_COLS);
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(STAGES >= 2, "not enough shared memory for two stages");
+  static_assert(A_COL0 + STAGES * A_COLS <= kTmemCols, "TMEM budget");
+  static_assert(BN <= 256 && BN % 16 == 0, "MMA N");
+};
+
+struct Params {
+  const __half *scales;
+  const __half *biases;
+  __nv_bfloat16 *y;
+  int M, N, K, G, Gn;
+  int m_tiles, n_tiles;
+};
+
+template <int BITS, int BN>
+__global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant__ CUtensorMap x_map,
+                                                          const __grid_constant__ CUtensorMap w_map, Params prm) {
+  using C = Cfg<BITS, BN>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES);
+  uint64_t *empty = full + S;
+  uint64_t *a_full = empty + S;
+  uint64_t *acc_full = a_full + S;
+  uint64_t *acc_empty = acc_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total_tiles = prm.m_tiles * prm.n_tiles;
+  const int KB = (prm.K + C::BK - 1) / C::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&a_full[s], 8);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&x_map)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&w_map)) : "memory");
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % prm.m_tiles) * BN;
+        const int n0 = (tile / prm.m_tiles) * 128;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t r = it / S;
+          if (r >= 1 && !(ok = mbar_wait(&empty[s], (r - 1) & 1, abort_flag, kFaultProducerWait))) break;
+          uint8_t *xs = smem + s * C::STAGE_BYTES;
+          uint8_t *ws = xs + C::X_BYTES;
+          mbar_arrive_expect_tx(&full[s], C::X_BYTES + C::W_BYTES);
+#pragma unroll
+          for (int a = 0; a < C::BK / 64; ++a) tma_load_2d(xs + a * BN * 128, &x_map, &full[s], kb * C::BK + a * 64, m0);
+          tma_load_2d(ws, &w_map, &full[s], kb * C::BKW, n0);
+        }
+      }
+      // drain: wait (bounded) until every issued load has landed
+      const uint32_t issued = it;
+      for (uint32_t j = (issued > static_cast<uint32_t>(S) ? issued - S : 0); j < issued; ++j) {
+        mbar_wait(&full[j % S], (j / S) & 1, abort_flag, kFaultProducerWait);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BN);
+      uint32_t it = 0, t = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t) {
+        if (t >= 1 && !(ok = mbar_wait(acc_empty, (t - 1) & 1, abort_flag, kFaultMmaWait))) break;
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t r = it / S;
+          if (!(ok = mbar_wait(&full[s], r & 1, abort_flag, kFaultMmaWait))) break;
+          if (!(ok = mbar_wait(&a_full[s], r & 1, abort_flag, kFaultMmaWait))) break;
+          tc_fence_after();
+          const uint32_t xs_addr = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t a_tmem = tmem_base + C::A_COL0 + s * C::A_COLS;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            // K = 16 slice kk: 32 bytes into a 128-byte swizzle row; a new atom column every 64 elements
+            const uint32_t b_addr = xs_addr + (kk / 4) * BN * 128 + (kk % 4) * 32;
+            tc_mma_ts(tmem_base + kAccCol, a_tmem + kk * 8, sw128_kmajor_desc(b_addr), idesc,
+                      (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        if (ok) tc_commit(acc_full);
+      }
+      // drain: the last commits must have landed before TMEM is released
+      if (it > 0) mbar_wait(&empty[(it - 1) % S], ((it - 1) / S) & 1, abort_flag, kFaultMmaWait);
+    }
+  } else if (warp >= kDequantWarp0) {
+    // ------------------------------------------------------------------ dequant + epilogue
+    const int q = warp & 3;                 // TMEM lane quadrant
+    const int h = (warp - kDequantWarp0) >> 2;  // which half of the K block
+    const int row = q * 32 + lane;          // W row within the tile == TMEM lane
+    constexpr int HALF = C::BK / 2;         // elements per thread per K block
+    constexpr int CH = HALF / 32;           // 32-code chunks per thread per K block
+    uint32_t it = 0, t = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t) {
+      const int m0 = (tile % prm.m_tiles) * BN;
+      const int n0 = (tile / prm.m_tiles) * 128;
+      const int n = n0 + row;
+      const bool row_ok = n < prm.N;
+      const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t r = it / S;
+        // scales/biases of this thread's chunks (loaded before the waits)
+        float sc[CH], bi[CH];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int k = kb * C::BK + h * HALF + c * 32;
+          const int g = k / prm.G;
+          const bool in = row_ok && g < prm.Gn;
+          sc[c] = in ? half_bits_to_float(ldg_nc2(prm.scales + g_row + g)) : 0.0f;
+          bi[c] = in ? half_bits_to_float(ldg_nc2(prm.biases + g_row + g)) : 0.0f;
+        }
+        if (!(ok = mbar_wait(&full[s], r & 1, abort_flag, kFaultDequantWait))) break;
+        if (r >= 1 && !(ok = mbar_wait(&empty[s], (r - 1) & 1, abort_flag, kFaultDequantWait))) break;
+        __syncwarp();  // lanes leave the spin at different times; tcgen05.st needs the whole warp
+        const uint32_t *ws = reinterpret_cast<const uint32_t *>(smem + s * C::STAGE_BYTES + C::X_BYTES);
+        const uint32_t *wrow = ws + row * C::BKW + h * (HALF * BITS / 32);
+        const uint32_t a_tmem = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::A_COL0 + s * C::A_COLS;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          uint32_t w[BITS];
+#pragma unroll
+          for (int i = 0; i < BITS; ++i) w[i] = wrow[c * BITS + i];
+          uint32_t packed_cols[16];
+          static_for<0, 16>([&](auto P) {
+            constexpr int j = 2 * P.value;
+            const float2 f = make_float2(__uint_as_float(extract_magic<BITS, j>(w)),
+                                         __uint_as_float(extract_magic<BITS, j + 1>(w)));
+            const float2 u = fadd2(f, make_float2(-1.0f, -1.0f));      // q * 2^(p-23), exact
+            constexpr float f0 = field_factor(BITS, j), f1 = field_factor(BITS, j + 1);
+            const float2 sp = make_float2(sc[c] * f0, sc[c] * f1);  // exact: powers of two
+            const float2 v = ffma2(u, sp, make_float2(bi[c], bi[c]));  // fp32_rn(q*s + b)
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v.x, v.y);
+            packed_cols[P.value] = *reinterpret_cast<uint32_t *>(&b2);
+          });
+          tmem_st16(a_tmem + h * (HALF / 2) + c * 16, packed_cols);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[s]);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------------- epilogue
+      if (!(ok = mbar_wait(acc_full, t & 1, abort_flag, kFaultEpilogueWait))) break;
+      __syncwarp();
+      tc_fence_after();
+      constexpr int COLS = BN / 2;  // accumulator columns handled by this warp
+#pragma unroll 1
+      for (int c0 = 0; c0 < COLS; c0 += 32) {
+        uint32_t v[32];
+        const int col = h * COLS + c0;
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + col, v);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int m = m0 + col + i;
+            if (m < prm.M) prm.y[static_cast<int64_t>(m) * prm.N + n] = __float2bfloat16_rn(__uint_as_float(v[i]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+template <int BITS, int BN>
+cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                     const uint16_t *biases, int64_t N, int G, uint16_t *y, cudaStream_t stream) {
+  using C = Cfg<BITS, BN>;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap x_map, w_map;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(BN)};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const int64_t P = K * BITS / 32;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(P) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(C::BKW), 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(packed), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  Params prm;
+  prm.scales = reinterpret_cast<const __half *>(scales);
+  prm.biases = reinterpret_cast<const __half *>(biases);
+  prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  prm.M = static_cast<int>(M);
+  prm.N = static_cast<int>(N);
+  prm.K = static_cast<int>(K);
+  prm.G = G;
+  prm.Gn = static_cast<int>(K / G);
+  prm.m_tiles = static_cast<int>((M + BN - 1) / BN);
+  prm.n_tiles = static_cast<int>((N + 127) / 128);
+
+  auto kern = qmm_kernel<BITS, BN>;
+  static thread_local int cached_dev = -1;
+  static thread_local int sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
+      return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, prm);
+  return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                        const uint16_t *biases, int64_t N, int G, uint16_t *y, cudaStream_t s) {
+  if (M <= 64) return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, s);
+  if (M <= 128) return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, s);
+  return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, s);
+}
+
+}  // namespace qmm
+
+bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits) {
+  (void)G;
+  if (M <= 0 || N <= 0 || K <= 0) return false;
+  // TMA: the packed row pitch must be a multiple of 16 bytes.
+  if ((K * bits) % 128 != 0) return false;
+  return true;
+}
+
+cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s) {
+  switch (bits) {
+    case 2: return qmm::launch_bits<2>(x, M, K, packed, scales, biases, N, G, y, s);
+    case 3: return qmm::launch_bits<3>(x, M, K, packed, scales, biases, N, G, y, s);
+    case 4: return qmm::launch_bits<4>(x, M, K, packed, scales, biases, N, G, y, s);
+    default: return qmm::launch_bits<8>(x, M, K, packed, scales, biases, N, G, y, s);
+  }
+}
+
+cudaError_t read_and_clear_fault(uint32_t *word) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemcpyFromSymbol(word, g_fault_word, sizeof(uint32_t))) != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_fault_word, &zero, sizeof(uint32_t));
+}
+
+}  // namespace aq
