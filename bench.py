@@ -137,6 +137,41 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- ranks (host plumbing only)
+
+def _dist():
+    try:
+        import torch.distributed as dist
+    except ImportError:
+        return None
+    return dist if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1 else None
+
+
+def rank_barrier(device=None):
+    dist = _dist()
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def reduce_max(v, device=None):
+    """Max of a per-rank scalar over all ranks (identity on one rank)."""
+    dist = _dist()
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(bytes_per_step, steps_per_rank, world, ms_max):
+    """Whole-job throughput: the bytes all ranks processed over the slowest rank's time."""
+    return bytes_per_step * steps_per_rank * world / (ms_max * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- our implementation
 
 def run_ours(args, rank, world, local_rank):
@@ -145,21 +180,12 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist_mod
-        dist = dist_mod
 
     def barrier():
-        if dist is not None:
-            dist.barrier(device_ids=[local_rank])
+        rank_barrier(dev)
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dev)
 
     peaks = read_peaks()
     stream = torch.cuda.Stream(dev)
@@ -217,7 +243,7 @@ def run_ours(args, rank, world, local_rank):
     ms = e0.elapsed_time(e1)
     ms_max = max_over_ranks(ms)
     clocks = clk.summary()
-    value = STEP_BYTES * steps * world / (ms_max * 1e-3) / 1e9
+    value = aggregate_gbs(STEP_BYTES, steps, world, ms_max)
     ms_per_step = ms_max / steps
     achieved = STEP_BYTES / (ms / steps * 1e-3) / 1e9  # this rank's kernel-only GB/s (the step is 3 QMV launches)
     traffic = recorded_traffic("qmv_decode_step")
@@ -263,7 +289,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.empty_cache()
 
     sections = {}
-    if not args.no_sections:
+    if args.sections != "none":
         sections = measure_sections(args, aq, torch, dev, stream, peaks)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps,
@@ -305,6 +331,18 @@ def timed_graph(torch, stream, fn, reps_inner, reps_outer):
 
 def measure_sections(args, aq, torch, dev, stream, peaks):
     out = {}
+    want = set(args.sections.split(",")) if args.sections != "all" else {"qmm", "curve", "sweep", "quant"}
+    if "qmm" in want:
+        out.update(section_qmm(args, aq, torch, dev, stream, peaks))
+    if "curve" in want:
+        out.update(section_curve(args, aq, torch, dev, stream, peaks))
+    if "sweep" in want or "quant" in want:
+        out.update(section_sweep_quant(args, aq, torch, dev, stream, peaks, want))
+    return out
+
+
+def section_qmm(args, aq, torch, dev, stream, peaks):
+    out = {}
     # ---- QMM prefill: M = 8192, K = 4096, N = 14336 (the tensor-core kernel)
     M, K, N = 8192, 4096, 14336
     w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 5 + 4)).to(dev)
@@ -324,7 +362,11 @@ def measure_sections(args, aq, torch, dev, stream, peaks):
                                        "traffic": recorded_traffic("qmm_prefill")}}
     del p, s, b, x, y
     torch.cuda.empty_cache()
+    return out
 
+
+def section_curve(args, aq, torch, dev, stream, peaks):
+    out = {}
     # ---- QMV small-M curve on K=4096, N=14336 (rotating weight copies)
     K, N = 4096, 14336
     w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 3)).to(dev)
@@ -343,14 +385,18 @@ def measure_sections(args, aq, torch, dev, stream, peaks):
     out["qmv_small_m"] = {"K": K, "N": N, "bits": BITS, "G": G, "curve": curve}
     del ws, base
     torch.cuda.empty_cache()
+    return out
 
+
+def section_sweep_quant(args, aq, torch, dev, stream, peaks, want):
+    out = {}
     # ---- bits x group sweep at M=1 on K=8192, N=28672 (one point per bits, G=64 and the 4-bit G sweep)
     K, N = 8192, 28672
     w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 4)).to(dev)
     sweep = {}
     x = synth.activations(1, K, 13).to(dev)
     y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
-    for bits in (2, 3, 4, 8):
+    for bits in ((2, 3, 4, 8) if "sweep" in want else ()):
         for g in ((32, 64, 128) if bits == 4 else (64,)):
             q = aq.aq_quantize(w, g, bits)
             wb = weight_bytes(K, N, g, bits)
@@ -361,7 +407,10 @@ def measure_sections(args, aq, torch, dev, stream, peaks):
             sweep[f"b{bits}_G{g}"] = {"us": round(ms * 1e3, 2), "weight_GBps": round(wb / (ms * 1e-3) / 1e9, 1)}
             del qs, q
             torch.cuda.empty_cache()
-    out["qmv_bits_group_sweep"] = {"K": K, "N": N, "M": 1, "points": sweep}
+    if sweep:
+        out["qmv_bits_group_sweep"] = {"K": K, "N": N, "M": 1, "points": sweep}
+    if "quant" not in want:
+        return out
 
     # ---- quantize and dequantize (bytes: read W fp32 + write packed/scales/biases; read packed + write bf16)
     p, s, b = aq.aq_quantize(w, G, BITS)
@@ -443,7 +492,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--qmm-reps", type=int, default=20)
-    ap.add_argument("--no-sections", action="store_true")
+    ap.add_argument("--sections", default="all",
+                    help="all | none | comma list of qmm,curve,sweep,quant (secondary measurements)")
+    ap.add_argument("--no-sections", dest="sections", action="store_const", const="none")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-steps", type=int, default=30)
     ap.add_argument("--ref-budget", type=float, default=60.0)

@@ -26,7 +26,10 @@
  *   x        bf16 bits [M, K]
  *   y        bf16 bits [M, N]       y = x @ dequant(W)^T
  * Ownership: every pointer argument is DEVICE memory, allocated, owned and freed
- * by the caller; the library allocates no device memory and needs no workspace.
+ * by the caller.  Only the tensor-core matmul path (large M) needs temporary
+ * device memory (a workspace: the activations converted to fp16); aq_matmul and
+ * aq_matmul_with take it from CUDA's stream-ordered allocator (cudaMallocAsync /
+ * cudaFreeAsync on `stream`), aq_matmul_ws takes it from the caller.
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  * stream); outputs are valid once the stream reaches the call.
  * Errors: arguments are validated synchronously, before anything is launched;
@@ -95,10 +98,26 @@ aq_status aq_dequantize_f32(const uint32_t *packed, const uint16_t *scales, cons
  * (mx.quantized_matmul(..., transpose=True)); metalworking "MLX Quantization",
  * section "Mechanics" (QMV for decode, QMM for prefill, host-side per-shape
  * dispatch).  Accuracy: |y - y_ref| <= 8e-3 * (|y_ref| + rms(y_ref)) against the
- * exact product. */
+ * exact product.  Kernels: QMV (CUDA cores, fp32 arithmetic on the exact codes)
+ * for M <= 8; QMM (tensor cores) otherwise, on fp16 operands: weights
+ * fp16_rn(fp32_rn(code*scale + bias)), activations scaled per row by an exact
+ * power of two into fp16, fp32 accumulation. */
 aq_status aq_matmul(const uint16_t *x_bf16, int64_t M, int64_t K,
                     const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                     int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
+
+/* Bytes of workspace aq_matmul_ws needs for this shape (0 when the dispatched
+ * kernel needs none, or when the arguments would be rejected).  Host only. */
+size_t aq_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K, int G, int bits);
+
+/* aq_matmul with caller-provided workspace: `workspace` is device memory of at
+ * least aq_matmul_workspace_bytes(M, N, K, G, bits) bytes, 16-byte aligned,
+ * not used by any other call in flight (NULL is allowed when that size is 0).
+ * Too small or NULL when needed -> AQ_ERR_INVALID_ARG. */
+aq_status aq_matmul_ws(const uint16_t *x_bf16, int64_t M, int64_t K,
+                       const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                       int64_t N, int G, int bits, uint16_t *y_bf16, void *workspace, size_t workspace_bytes,
+                       aq_stream_t stream);
 
 /* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV returns AQ_ERR_UNSUPPORTED
  * when M > 8 or its shared-memory staging of x does not fit; AQ_KERNEL_QMM

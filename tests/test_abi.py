@@ -139,3 +139,18 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         aq.aq_quantize(torch.zeros(4, 64), 64, 4)
+
+
+def test_workspace_size_rule():
+    assert aq.aq_matmul_workspace_bytes(1, 4096, 4096, 64, 4) == 0          # QMV: none
+    need = aq.aq_matmul_workspace_bytes(512, 4096, 4096, 64, 4)            # QMM: fp16 x + row scales
+    assert need >= 512 * 4096 * 2 + 512 * 4
+    assert aq.aq_matmul_workspace_bytes(512, 4096, 4000, 64, 4) == 0       # rejected shape
+
+
+def test_workspace_validation():
+    L = aq.lib()
+    # a QMM shape with no workspace -> invalid argument, before any CUDA call
+    assert L.aq_matmul_ws(A, 512, 4096, A, A, A, 64, 64, 4, A, None, 0, None) == aq.AQ_ERR_INVALID_ARG
+    assert L.aq_matmul_ws(A, 512, 4096, A, A, A, 64, 64, 4, A, A, 16, None) == aq.AQ_ERR_INVALID_ARG
+    assert L.aq_matmul_ws(A, 512, 4096, A, A, A, 64, 64, 4, A, U, 1 << 30, None) == aq.AQ_ERR_ALIGNMENT

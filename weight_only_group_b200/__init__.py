@@ -10,8 +10,8 @@ binding fails loudly when the library has not been built
 
 Names mirror the C entry points: ``aq_quantize``, ``aq_dequantize``,
 ``aq_dequantize_f32``, ``aq_matmul``, ``aq_matmul_with``, ``aq_dispatch``,
-``aq_packed_words``, ``aq_packed_bytes``, ``aq_status_string``,
-``aq_device_fault``.
+``aq_matmul_ws``, ``aq_matmul_workspace_bytes``, ``aq_packed_words``,
+``aq_packed_bytes``, ``aq_status_string``, ``aq_device_fault``.
 """
 from __future__ import annotations
 
@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
             L.aq_dequantize_f32.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
             L.aq_matmul_with.argtypes = [i32, vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
+            L.aq_matmul_ws.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, u64, vp]
+            L.aq_matmul_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
+            L.aq_matmul_workspace_bytes.restype = u64
             L.aq_dispatch.argtypes = [i64, i64, i64, i32, i32]
             L.aq_dispatch.restype = i32
             L.aq_status_string.argtypes = [i32]
@@ -71,7 +74,7 @@ def lib() -> ctypes.CDLL:
             L.aq_last_cuda_error.restype = i32
             L.aq_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
             for f in ("aq_quantize", "aq_dequantize", "aq_dequantize_f32", "aq_matmul", "aq_matmul_with",
-                      "aq_device_fault"):
+                      "aq_matmul_ws", "aq_device_fault"):
                 getattr(L, f).restype = i32
             _lib = L
     return _lib
@@ -89,6 +92,10 @@ def aq_packed_bytes(N: int, K: int, G: int, bits: int) -> int:
 
 def aq_dispatch(M: int, N: int, K: int, G: int, bits: int) -> int:
     return int(lib().aq_dispatch(M, N, K, G, bits))
+
+
+def aq_matmul_workspace_bytes(M: int, N: int, K: int, G: int, bits: int) -> int:
+    return int(lib().aq_matmul_workspace_bytes(M, N, K, G, bits))
 
 
 def aq_status_string(status: int) -> str:
@@ -193,6 +200,28 @@ def aq_matmul_with(kernel, x, packed, scales, biases, G: int, bits: int, out: to
 def aq_matmul(x, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None):
     """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T, kernel chosen per shape by the library."""
     return aq_matmul_with(AQ_KERNEL_AUTO, x, packed, scales, biases, G, bits, out)
+
+
+def aq_matmul_ws(x, packed, scales, biases, G: int, bits: int, workspace: torch.Tensor | None,
+                 out: torch.Tensor | None = None):
+    """aq_matmul with a caller-owned workspace (a CUDA tensor of at least
+    aq_matmul_workspace_bytes(...) bytes; None when that size is 0)."""
+    _need(x, "x", (torch.bfloat16,))
+    N = _qw(packed, scales, biases)
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16,))
+    wp, wb = 0, 0
+    if workspace is not None:
+        if workspace.device.type != "cuda" or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        wp, wb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    with torch.cuda.device(x.device):
+        rc = lib().aq_matmul_ws(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, G,
+                                bits, out.data_ptr(), wp, wb, _stream(x))
+    _check(rc, "aq_matmul_ws")
+    return out
 
 
 def aq_device_fault() -> int:

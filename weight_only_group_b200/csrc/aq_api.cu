@@ -12,8 +12,11 @@ cudaError_t launch_dequantize(const uint32_t *packed, const uint16_t *scales, co
 cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
 size_t qmv_required_smem(int64_t M, int64_t K);
+bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
+cudaError_t read_and_clear_qmv_fault(uint32_t *word);
 cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s);
+size_t qmm_workspace_bytes(int64_t M, int64_t K);
 bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t read_and_clear_fault(uint32_t *word);
 }  // namespace aq
@@ -67,7 +70,7 @@ aq_status check_device() {
   return checked[dev] == 1 ? AQ_OK : AQ_ERR_UNSUPPORTED;
 }
 
-bool qmv_fits(int64_t M, int64_t K) { return M >= 1 && M <= 8 && aq::qmv_required_smem(M, K) <= kMaxSmemPerBlock; }
+bool qmv_fits(int64_t M, int64_t N, int64_t K, int G, int bits) { return aq::qmv_supported(M, N, K, G, bits); }
 
 }  // namespace
 
@@ -131,14 +134,15 @@ aq_status aq_dequantize_f32(const uint32_t *packed, const uint16_t *scales, cons
 
 int aq_dispatch(int64_t M, int64_t N, int64_t K, int G, int bits) {
   if (M <= 0 || M > kMaxDim || check_shape(N, K, G, bits) != AQ_OK) return -1;
-  if (qmv_fits(M, K)) return AQ_KERNEL_QMV;
+  if (qmv_fits(M, N, K, G, bits)) return AQ_KERNEL_QMV;
   if (aq::qmm_supports(M, N, K, G, bits)) return AQ_KERNEL_QMM;
   return -1;
 }
 
-aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
-                         const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
-                         aq_stream_t stream) {
+// Validation and kernel choice shared by the matmul entry points.
+static aq_status matmul_prepare(aq_kernel &kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                                const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits,
+                                const uint16_t *y) {
   aq_status st = check_shape(N, K, G, bits);
   if (st != AQ_OK) return st;
   if (M <= 0 || M > kMaxDim) return AQ_ERR_INVALID_ARG;
@@ -150,17 +154,60 @@ aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t
     if (k < 0) return AQ_ERR_UNSUPPORTED;
     kernel = static_cast<aq_kernel>(k);
   }
-  if (kernel == AQ_KERNEL_QMV) {
-    if (!qmv_fits(M, K)) return AQ_ERR_UNSUPPORTED;
-    if ((st = check_device()) != AQ_OK) return st;
-    return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, stream));
-  }
-  if (kernel == AQ_KERNEL_QMM) {
-    if (!aq::qmm_supports(M, N, K, G, bits)) return AQ_ERR_UNSUPPORTED;
-    if ((st = check_device()) != AQ_OK) return st;
-    return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, stream));
-  }
+  if (kernel == AQ_KERNEL_QMV) return qmv_fits(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
+  if (kernel == AQ_KERNEL_QMM) return aq::qmm_supports(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
   return AQ_ERR_INVALID_ARG;
+}
+
+static size_t workspace_for(aq_kernel kernel, int64_t M, int64_t K) {
+  return kernel == AQ_KERNEL_QMM ? aq::qmm_workspace_bytes(M, K) : 0;
+}
+
+static aq_status matmul_run(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                            const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
+                            void *ws, aq_stream_t stream) {
+  aq_status st = check_device();
+  if (st != AQ_OK) return st;
+  if (kernel == AQ_KERNEL_QMV) return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, stream));
+  return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, ws, stream));
+}
+
+size_t aq_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K, int G, int bits) {
+  const int k = aq_dispatch(M, N, K, G, bits);
+  if (k < 0) return 0;
+  return workspace_for(static_cast<aq_kernel>(k), M, K);
+}
+
+aq_status aq_matmul_ws(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *workspace,
+                       size_t workspace_bytes, aq_stream_t stream) {
+  aq_kernel kernel = AQ_KERNEL_AUTO;
+  aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
+  if (st != AQ_OK) return st;
+  const size_t need = workspace_for(kernel, M, K);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return AQ_ERR_ALIGNMENT;
+  }
+  return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, workspace, stream);
+}
+
+aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                         const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
+                         aq_stream_t stream) {
+  aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
+  if (st != AQ_OK) return st;
+  const size_t need = workspace_for(kernel, M, K);
+  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream);
+  if ((st = check_device()) != AQ_OK) return st;
+  // workspace from the stream-ordered allocator, released on the same stream
+  void *ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, need, stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  st = matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, ws, stream);
+  e = cudaFreeAsync(ws, stream);
+  if (st == AQ_OK && e != cudaSuccess) st = from_cuda(e);
+  return st;
 }
 
 aq_status aq_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
@@ -170,7 +217,12 @@ aq_status aq_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pac
 
 aq_status aq_device_fault(uint32_t *fault_word) {
   if (!fault_word) return AQ_ERR_INVALID_ARG;
-  return from_cuda(aq::read_and_clear_fault(fault_word));
+  uint32_t a = 0, b = 0;
+  aq_status st = from_cuda(aq::read_and_clear_fault(&a));
+  if (st != AQ_OK) return st;
+  st = from_cuda(aq::read_and_clear_qmv_fault(&b));
+  *fault_word = a | b;
+  return st;
 }
 
 }  // extern "C"

@@ -20,6 +20,7 @@ enum : uint32_t {
   kFaultProducerWait = 1u << 1, // TMA producer gave up waiting for a free stage
   kFaultDequantWait = 1u << 2,  // dequant warps gave up waiting for packed data / a free A stage
   kFaultEpilogueWait = 1u << 3, // epilogue gave up waiting for the accumulator
+  kFaultQmvWait = 1u << 4,      // QMV gave up waiting for a weight stage
 };
 
 // Upper bound of any spin on an mbarrier, in SM clock cycles (~1 s at 2 GHz).
@@ -63,21 +64,61 @@ AQ_DEVICE float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16)
 
 AQ_DEVICE uint32_t smem_u32(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
-// Packed fp32x2 FMA (sm_100): d = a * b + c on both halves.
-AQ_DEVICE float2 ffma2(float2 a, float2 b, float2 c) {
-  unsigned long long A = *reinterpret_cast<unsigned long long *>(&a);
-  unsigned long long B = *reinterpret_cast<unsigned long long *>(&b);
-  unsigned long long C = *reinterpret_cast<unsigned long long *>(&c);
-  unsigned long long D;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(D) : "l"(A), "l"(B), "l"(C));
-  return *reinterpret_cast<float2 *>(&D);
+// Packed fp32x2 arithmetic (sm_100 builtins): two FMAs / adds per instruction.
+AQ_DEVICE float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+AQ_DEVICE float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// ---------------------------------------------------------------------------
+// mbarrier / bulk-copy helpers (shared memory addresses as 32-bit)
+// ---------------------------------------------------------------------------
+AQ_DEVICE void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
-AQ_DEVICE float2 fadd2(float2 a, float2 b) {
-  unsigned long long A = *reinterpret_cast<unsigned long long *>(&a);
-  unsigned long long B = *reinterpret_cast<unsigned long long *>(&b);
-  unsigned long long D;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
-  return *reinterpret_cast<float2 *>(&D);
+AQ_DEVICE void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+AQ_DEVICE void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+AQ_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: true once the phase with the given parity has completed; false
+// on timeout (the fault bit is OR-ed into *fault and *abort_flag is raised) or
+// when another thread of the CTA has already raised *abort_flag.
+AQ_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *fault,
+                         uint32_t fault_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(fault, fault_bit);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+AQ_DEVICE void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// 1-D bulk copy global -> shared, completing on an mbarrier (16-byte aligned, size % 16 == 0).
+AQ_DEVICE void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -5,27 +5,34 @@
 // prefill/batch case: dequantize weight tiles on chip, then a tiled GEMM
 // against them; "One trap for intuition": dequantize on every use, never a
 // cached fp16 copy.  anllm "Tutorial 10: Quantization", section 5: the fused
-// product equals dequantize-then-multiply; here every dequantized weight is
-// bf16_rn(fp32_rn(q*scale + bias)), exactly the value aq_dequantize writes, and
-// the products are accumulated in fp32.
+// product equals dequantize-then-multiply.
+//
+// Precision: both MMA operands are fp16 (11-bit significands).  Dequantized
+// weights are fp16_rn(fp32_rn(q*scale + bias)); bf16 (8 bits) is not enough:
+// in groups stretched by an outlier the bf16 rounding of every weight adds up
+// past the matmul tolerance.  Activations are carried as fp16 after an exact
+// power-of-two scaling of each token row (x = 2^e * x16, the row maximum of
+// x16 in [2^14, 2^15)), done by a small pre-pass into workspace memory; the
+// epilogue multiplies the fp32 accumulator by 2^e.
 //
 // B200 design ("swap AB": weights are the MMA's A operand, tokens its N):
 //  * CTA tile: 128 rows of W (MMA M = 128, one TMEM lane per row) x BN tokens
 //    (MMA N = BN <= 256); persistent CTAs walk the tiles, token tiles fastest.
-//  * Warp 0 (one lane): TMA producer.  Per K block it loads the x tile
-//    [BN tokens x BK] (bf16, 128-byte swizzle, the canonical K-major UMMA
+//  * Warp 0 (one lane): TMA producer.  Per K block it loads the x16 tile
+//    [BN tokens x BK] (fp16, 128-byte swizzle, the canonical K-major UMMA
 //    layout) and the packed W tile [128 rows x BK*bits/32 words] into a ring
 //    of shared-memory stages, completing on the stage's mbarrier.
 //  * Warps 4..11 (two per TMEM lane quadrant): dequantize.  Thread (quadrant,
 //    lane) owns W row 32*quadrant+lane and one half of the K block: it reads
-//    its packed words from shared memory, turns codes into bf16 weights in
+//    its packed words from shared memory, turns codes into fp16 weights in
 //    registers and writes them with tcgen05.st straight into a TMEM stage
 //    that the MMA reads as operand A (no swizzled shared-memory round trip).
-//  * Warp 1 (one lane): issues tcgen05.mma.kind::f16 (A from TMEM, B from
+//  * Warp 1 (one lane): issues tcgen05.mma.kind::f16 (fp16 A from TMEM, fp16 B from
 //    shared memory, fp32 accumulator of 128 x BN in TMEM) and tcgen05.commit
 //    to release stages; warp 1 also owns the TMEM allocation.
-//  * Epilogue: the dequant warps read the accumulator with tcgen05.ld and
-//    store bf16 (RNE) y[m, n] (a warp writes 32 consecutive n per token).
+//  * Epilogue: the dequant warps read the accumulator with tcgen05.ld, scale
+//    by 2^e of the token row and store bf16 (RNE) y[m, n] (a warp writes 32
+//    consecutive n per token).
 //  * Every mbarrier wait is bounded; on expiry the kernel records a bit in a
 //    device fault word, stops issuing work and exits cleanly.
 #include <cuda.h>
@@ -50,41 +57,9 @@ constexpr int kAccCol = 0;        // accumulator columns [0, BN); A stages follo
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
-AQ_DEVICE void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-AQ_DEVICE void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-AQ_DEVICE void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-AQ_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: true once the phase of the given parity completed, false on
-// timeout or when another role already aborted (the fault bit is recorded).
+// Bounded wait on this kernel's fault word.
 AQ_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t fault_bit) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      atomicOr(&g_fault_word, fault_bit);
-      *abort_flag = 1;
-      return false;
-    }
-  }
+  return aq::mbar_wait(bar, parity, abort_flag, &g_fault_word, fault_bit);
 }
 
 AQ_DEVICE void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
@@ -148,9 +123,11 @@ AQ_DEVICE uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major, M = 128, N = bn.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int bn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+// Instruction descriptor: kind::f16 with A = B = fp16 (format 0), D = f32
+// (format 1), both K-major, M = 128, N = bn.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int bn) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(bn >> 3) << 17) |
+         (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
 // ---------------------------------------------------------------------------
@@ -176,6 +153,7 @@ struct Cfg {
 struct Params {
   const __half *scales;
   const __half *biases;
+  const float *row_scale;  // per token row: x[m,:] = row_scale[m] * x16[m,:] exactly
   __nv_bfloat16 *y;
   int M, N, K, G, Gn;
   int m_tiles, n_tiles;
@@ -209,8 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
     *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    fence_barrier_init();
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -254,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BN);
+      constexpr uint32_t idesc = idesc_f16_f32(BN);
       uint32_t it = 0, t = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t) {
@@ -330,8 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
             constexpr float f0 = field_factor(BITS, j), f1 = field_factor(BITS, j + 1);
             const float2 sp = make_float2(sc[c] * f0, sc[c] * f1);  // exact: powers of two
             const float2 v = ffma2(u, sp, make_float2(bi[c], bi[c]));  // fp32_rn(q*s + b)
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(v.x, v.y);
-            packed_cols[P.value] = *reinterpret_cast<uint32_t *>(&b2);
+            __half2 h2 = __floats2half2_rn(v.x, v.y);
+            packed_cols[P.value] = *reinterpret_cast<uint32_t *>(&h2);
           });
           tmem_st16(a_tmem + h * (HALF / 2) + c * 16, packed_cols);
         }
@@ -356,7 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int m = m0 + col + i;
-            if (m < prm.M) prm.y[static_cast<int64_t>(m) * prm.N + n] = __float2bfloat16_rn(__uint_as_float(v[i]));
+            if (m < prm.M)
+              prm.y[static_cast<int64_t>(m) * prm.N + n] =
+                  __float2bfloat16_rn(__uint_as_float(v[i]) * __ldg(prm.row_scale + m));
           }
         }
       }
@@ -373,6 +352,66 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                  : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Pre-pass: x bf16 [M, K] -> x16 fp16 [M, K] and row_scale[M], with
+// x[m, k] = row_scale[m] * x16[m, k] exactly for every x16 that is a normal
+// fp16 value.  row_scale[m] = 2^e with e = floor(log2(max_k |x[m, k]|)) - 14,
+// so the row maximum of x16 lies in [2^14, 2^15) (far from fp16 overflow).
+// One CTA per row; two vectorized passes over the row (the second hits L2).
+// ---------------------------------------------------------------------------
+constexpr int kPrepThreads = 256;
+
+__global__ void __launch_bounds__(kPrepThreads) x_to_f16_rows_kernel(const __nv_bfloat16 *__restrict__ x, int K,
+                                                                     __half *__restrict__ x16,
+                                                                     float *__restrict__ row_scale) {
+  __shared__ float red[kPrepThreads / 32];
+  const int64_t m = blockIdx.x;
+  const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K);
+  const int n8 = K / 8;
+  float amax = 0.0f;
+  for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
+    const uint4 v = ldg_nc16(src + i);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(u[h] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(u[h] & 0xFFFF0000u)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < kPrepThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+  // exponent of amax (bf16 values are never fp32-subnormal-only: 8-bit exponent kept)
+  int e = 0;
+  if (amax > 0.0f) e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14;
+  // 2^-e and 2^e as exact fp32 powers of two (|e| <= 141 needs two factors)
+  const float down_a = __uint_as_float(static_cast<uint32_t>(127 - e / 2) << 23);
+  const float down_b = __uint_as_float(static_cast<uint32_t>(127 - (e - e / 2)) << 23);
+  if (threadIdx.x == 0) {
+    const float up_a = __uint_as_float(static_cast<uint32_t>(127 + e / 2) << 23);
+    const float up_b = __uint_as_float(static_cast<uint32_t>(127 + (e - e / 2)) << 23);
+    row_scale[m] = up_a * up_b;
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(x16 + m * K);
+  for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
+    const uint4 v = ldg_nc16(src + i);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float lo = __uint_as_float(u[h] << 16) * down_a * down_b;
+      const float hi = __uint_as_float(u[h] & 0xFFFF0000u) * down_a * down_b;
+      __half2 p = __floats2half2_rn(lo, hi);
+      o[h] = *reinterpret_cast<uint32_t *>(&p);
+    }
+    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -394,17 +433,23 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int BITS, int BN>
 cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                     const uint16_t *biases, int64_t N, int G, uint16_t *y, cudaStream_t stream) {
+                     const uint16_t *biases, int64_t N, int G, uint16_t *y, void *workspace, cudaStream_t stream) {
   using C = Cfg<BITS, BN>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
+  __half *x16 = reinterpret_cast<__half *>(workspace);
+  float *row_scale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + ((M * K * 2 + 255) / 256) * 256);
+  x_to_f16_rows_kernel<<<static_cast<unsigned>(M), kPrepThreads, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
   CUtensorMap x_map, w_map;
   {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
     cuuint32_t box[2] = {64, static_cast<cuuint32_t>(BN)};
     cuuint32_t estr[2] = {1, 1};
-    if (fn(&x_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
+    if (fn(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
@@ -423,6 +468,7 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
   Params prm;
   prm.scales = reinterpret_cast<const __half *>(scales);
   prm.biases = reinterpret_cast<const __half *>(biases);
+  prm.row_scale = row_scale;
   prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
   prm.M = static_cast<int>(M);
   prm.N = static_cast<int>(N);
@@ -452,10 +498,10 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
 
 template <int BITS>
 cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                        const uint16_t *biases, int64_t N, int G, uint16_t *y, cudaStream_t s) {
-  if (M <= 64) return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, s);
-  if (M <= 128) return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, s);
-  return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, s);
+                        const uint16_t *biases, int64_t N, int G, uint16_t *y, void *ws, cudaStream_t s) {
+  if (M <= 64) return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+  if (M <= 128) return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+  return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
 }
 
 }  // namespace qmm
@@ -468,13 +514,18 @@ bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits) {
   return true;
 }
 
+// Workspace of the QMM path: x16 (fp16 [M, K], 256-byte padded) + row_scale (fp32 [M]).
+size_t qmm_workspace_bytes(int64_t M, int64_t K) {
+  return static_cast<size_t>((M * K * 2 + 255) / 256 * 256) + static_cast<size_t>((M * 4 + 255) / 256 * 256);
+}
+
 cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s) {
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s) {
   switch (bits) {
-    case 2: return qmm::launch_bits<2>(x, M, K, packed, scales, biases, N, G, y, s);
-    case 3: return qmm::launch_bits<3>(x, M, K, packed, scales, biases, N, G, y, s);
-    case 4: return qmm::launch_bits<4>(x, M, K, packed, scales, biases, N, G, y, s);
-    default: return qmm::launch_bits<8>(x, M, K, packed, scales, biases, N, G, y, s);
+    case 2: return qmm::launch_bits<2>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case 3: return qmm::launch_bits<3>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case 4: return qmm::launch_bits<4>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    default: return qmm::launch_bits<8>(x, M, K, packed, scales, biases, N, G, y, ws, s);
   }
 }
 

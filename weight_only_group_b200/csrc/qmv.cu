@@ -219,6 +219,335 @@ __global__ void __launch_bounds__(kQmvThreads) qmv_kernel(const __nv_bfloat16 *_
   }
 }
 
+// ===========================================================================
+// Streaming QMV: the kernel used whenever rows of packed words and of
+// scales/biases start on 16-byte boundaries (K*bits % 128 == 0, (K/G) % 8 == 0).
+//
+//  * One persistent CTA per SM owns a contiguous, balanced range of rows
+//    (N / #CTAs +- 1), so every SM streams the same number of bytes.
+//  * Thread 0 streams the CTA's rows through a ring of shared-memory stages
+//    with 1-D bulk copies (cp.async.bulk, completion on mbarriers): a stage is
+//    RS consecutive rows of packed words, scales and biases, each one
+//    contiguous range of global memory.  All of a CTA's stages are in flight
+//    from the start when the ring is deep enough.
+//  * Threads are laid out as Tr row lanes x Tk group slots.  Thread (rl, gs)
+//    handles group slots gs, gs+Tk, ... of rows rl, rl+Tr, ... (RT rows per
+//    stage), so activations are read once per RT rows and the scale/bias fold
+//    runs once per group.
+//  * Row sums: warp reduce-scatter, then a cross-warp sum in shared memory.
+// ===========================================================================
+__device__ uint32_t g_qmv_fault = 0;
+
+constexpr int kStreamMaxThreads = 512;
+
+struct QmvStreamArgs {
+  const __nv_bfloat16 *x;
+  const uint32_t *packed;
+  const __half *scales;
+  const __half *biases;
+  __nv_bfloat16 *y;
+  int N, K, Gn;
+  int Tk, Tr;         // threads per row lane (multiple of 32), row lanes
+  int RS, NS;         // rows per stage, stages in the ring
+  int stage_bytes;    // bytes of one stage (16-aligned)
+  int sc_off, bi_off; // byte offsets of scales and biases inside a stage
+};
+
+// Reduce-scatter of NV values across a warp: afterwards lane l holds the warp
+// total of value (l >> (5 - log2(NVP))) (NVP = NV rounded up to a power of 2).
+template <int NV>
+struct RsInfo {
+  static constexpr int NVP = NV <= 1 ? 1 : NV <= 2 ? 2 : NV <= 4 ? 4 : NV <= 8 ? 8 : NV <= 16 ? 16 : 32;
+  static constexpr int LOG = NVP == 1 ? 0 : NVP == 2 ? 1 : NVP == 4 ? 2 : NVP == 8 ? 3 : NVP == 16 ? 4 : 5;
+};
+template <int NV>
+AQ_DEVICE float warp_reduce_scatter(float (&v)[RsInfo<NV>::NVP], int lane) {
+  constexpr int NVP = RsInfo<NV>::NVP;
+  int cnt = NVP;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (cnt > 1) {
+      const int half = cnt / 2;
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < NVP / 2; ++i) {
+        if (i < half) {
+          const float send = up ? v[i] : v[i + half];
+          const float keep = up ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      cnt = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+  return v[0];
+}
+
+template <int BITS, int CPT, int M, int RT>
+__global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const QmvStreamArgs a) {
+  constexpr int G = CPT * 32;
+  constexpr int GP = G + 4;          // padded floats per group of staged x
+  constexpr int WPG = CPT * BITS;    // packed words per group
+  constexpr int NV = RT * M;
+  constexpr int NVP = RsInfo<NV>::NVP;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t *ring = smem_raw;
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + a.NS * a.stage_bytes);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(full + a.NS);
+  float *xs = reinterpret_cast<float *>(full + a.NS + 2);             // [M][Gn][GP]
+  float2 *tab = reinterpret_cast<float2 *>(xs + M * a.Gn * GP);        // [M][Gn]  (sum x', sum x)
+  float *red = reinterpret_cast<float *>(tab + M * a.Gn);              // [2][warps][32]
+  float *fac = red + 2 * (kStreamMaxThreads / 32) * 32;               // [32]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthreads = a.Tk * a.Tr;
+  const int P = (a.K / 32) * BITS;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * a.N / gridDim.x;
+  const int64_t r1 = static_cast<int64_t>(blockIdx.x + 1) * a.N / gridDim.x;
+  const int nst = static_cast<int>((r1 - r0 + a.RS - 1) / a.RS);
+  const uint32_t row_w_bytes = static_cast<uint32_t>(P) * 4, row_s_bytes = static_cast<uint32_t>(a.Gn) * 2;
+
+  auto issue = [&](int st) {  // thread 0 only
+    const int s = st % a.NS;
+    const int64_t rb = r0 + static_cast<int64_t>(st) * a.RS;
+    const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(a.RS), r1 - rb));
+    uint8_t *dst = ring + s * a.stage_bytes;
+    mbar_arrive_expect_tx(&full[s], rows * (row_w_bytes + 2 * row_s_bytes));
+    bulk_g2s(dst, a.packed + rb * P, rows * row_w_bytes, &full[s]);
+    bulk_g2s(dst + a.sc_off, a.scales + rb * a.Gn, rows * row_s_bytes, &full[s]);
+    bulk_g2s(dst + a.bi_off, a.biases + rb * a.Gn, rows * row_s_bytes, &full[s]);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < a.NS; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    for (int st = 0; st < min(nst, a.NS); ++st) issue(st);
+  }
+  if (tid < 32) fac[tid] = field_factor(BITS, tid);
+  __syncthreads();
+
+  // ---- stage x' = x * 2^(23-p) per group (padded) and per-group sums
+  {
+    constexpr int PPG = G / 8;  // 8-element pieces per group (4, 8 or 16 adjacent lanes)
+    const int per_row = a.K >> 3;
+    const int total = M * per_row;
+    const int total_padded = (total + nthreads - 1) / nthreads * nthreads;
+    for (int i0 = 0; i0 < total_padded; i0 += nthreads) {
+      const int i = i0 + tid;
+      const bool act = i < total;
+      const int ii = act ? i : 0;
+      const int m = ii / per_row, piece = ii - m * per_row;
+      const int g = piece / PPG, j0 = (piece % PPG) * 8;  // element offset inside the group
+      const uint4 v = ldg_nc16(a.x + static_cast<int64_t>(m) * a.K + piece * 8);
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+      float xp[8];
+      float sp = 0.0f, sx = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float xv = bf16_bits_to_float(e & 1 ? (u[e >> 1] >> 16) : (u[e >> 1] & 0xFFFFu));
+        xp[e] = xv * fac[(j0 + e) & 31];
+        sx += xv;
+        sp += xp[e];
+      }
+      if (act) {
+        float4 *dst = reinterpret_cast<float4 *>(xs + (m * a.Gn + g) * GP + j0);
+        dst[0] = make_float4(xp[0], xp[1], xp[2], xp[3]);
+        dst[1] = make_float4(xp[4], xp[5], xp[6], xp[7]);
+      }
+#pragma unroll
+      for (int o = 1; o < PPG; o <<= 1) {
+        sp += __shfl_xor_sync(0xffffffffu, sp, o);
+        sx += __shfl_xor_sync(0xffffffffu, sx, o);
+      }
+      if (act && j0 == 0) tab[m * a.Gn + g] = make_float2(sp, sx);
+    }
+  }
+  __syncthreads();
+
+  const int rl = tid / a.Tk, gs0 = tid - rl * a.Tk;
+  const bool worker = tid < nthreads;
+  bool ok = true;
+  int st = 0;
+  for (; st < nst; ++st) {
+    const int s = st % a.NS;
+    ok = mbar_wait(&full[s], (st / a.NS) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait);
+    if (!ok) break;
+    const uint32_t *wst = reinterpret_cast<const uint32_t *>(ring + s * a.stage_bytes);
+    const __half *sst = reinterpret_cast<const __half *>(ring + s * a.stage_bytes + a.sc_off);
+    const __half *bst = reinterpret_cast<const __half *>(ring + s * a.stage_bytes + a.bi_off);
+    float acc[NVP];
+#pragma unroll
+    for (int v = 0; v < NVP; ++v) acc[v] = 0.0f;
+    if (worker) {
+      for (int gs = gs0; gs < a.Gn; gs += a.Tk) {
+        float sc[RT], bi[RT];
+        float2 A[RT][M];
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          const int lr = rl + a.Tr * r;
+          sc[r] = __half2float(sst[lr * a.Gn + gs]);
+          bi[r] = __half2float(bst[lr * a.Gn + gs]);
+#pragma unroll
+          for (int m = 0; m < M; ++m) A[r][m] = make_float2(0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+          uint32_t w[RT][BITS];
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            const uint32_t *src = wst + (rl + a.Tr * r) * P + gs * WPG + c * BITS;
+            if constexpr (BITS == 4) {
+              const uint4 q = *reinterpret_cast<const uint4 *>(src);
+              w[r][0] = q.x; w[r][1] = q.y; w[r][2] = q.z; w[r][3] = q.w;
+            } else if constexpr (BITS == 8) {
+              const uint4 q0 = reinterpret_cast<const uint4 *>(src)[0];
+              const uint4 q1 = reinterpret_cast<const uint4 *>(src)[1];
+              w[r][0] = q0.x; w[r][1] = q0.y; w[r][2] = q0.z; w[r][3] = q0.w;
+              w[r][4] = q1.x; w[r][5] = q1.y; w[r][6] = q1.z; w[r][7] = q1.w;
+            } else if constexpr (BITS == 2) {
+              const uint2 q = *reinterpret_cast<const uint2 *>(src);
+              w[r][0] = q.x; w[r][1] = q.y;
+            } else {
+#pragma unroll
+              for (int i = 0; i < BITS; ++i) w[r][i] = src[i];
+            }
+          }
+          const float *xc = xs + gs * GP + c * 32;
+          static_for<0, 8>([&](auto Q) {
+            constexpr int j = 4 * Q.value;
+            float4 xq[M];
+#pragma unroll
+            for (int m = 0; m < M; ++m) xq[m] = *reinterpret_cast<const float4 *>(xc + m * a.Gn * GP + j);
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+              const float2 f01 = make_float2(__uint_as_float(extract_magic<BITS, j + 0>(w[r])),
+                                             __uint_as_float(extract_magic<BITS, j + 1>(w[r])));
+              const float2 f23 = make_float2(__uint_as_float(extract_magic<BITS, j + 2>(w[r])),
+                                             __uint_as_float(extract_magic<BITS, j + 3>(w[r])));
+#pragma unroll
+              for (int m = 0; m < M; ++m) {
+                A[r][m] = ffma2(make_float2(xq[m].x, xq[m].y), f01, A[r][m]);
+                A[r][m] = ffma2(make_float2(xq[m].z, xq[m].w), f23, A[r][m]);
+              }
+            }
+          });
+        }
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const float2 t = tab[m * a.Gn + gs];
+#pragma unroll
+          for (int r = 0; r < RT; ++r) {
+            const float sxq = (A[r][m].x + A[r][m].y) - t.x;  // sum of x*q over the group
+            acc[r * M + m] = fmaf(sc[r], sxq, fmaf(bi[r], t.y, acc[r * M + m]));
+          }
+        }
+      }
+    }
+    warp_reduce_scatter<NV>(acc, lane);
+    float *rb = red + (st & 1) * (kStreamMaxThreads / 32) * 32;
+    {
+      constexpr int SH = 5 - RsInfo<NV>::LOG;
+      const int vi = lane >> SH;
+      if ((lane & ((1 << SH) - 1)) == 0 && vi < NV) rb[warp * 32 + vi] = acc[0];
+    }
+    __syncthreads();  // stage s fully read; partial sums visible
+    if (tid == 0 && st + a.NS < nst) issue(st + a.NS);
+    {
+      const int64_t rbase = r0 + static_cast<int64_t>(st) * a.RS;
+      const int rows = static_cast<int>(min(static_cast<int64_t>(a.RS), r1 - rbase));
+      const int wpr = a.Tk / 32;  // warps per row lane
+      for (int t = tid; t < rows * M; t += blockDim.x) {
+        const int lr = t / M, m = t - lr * M;
+        const int r = lr / a.Tr, l = lr - r * a.Tr;
+        float sum = 0.0f;
+        for (int j = 0; j < wpr; ++j) sum += rb[(l * wpr + j) * 32 + r * M + m];
+        a.y[static_cast<int64_t>(m) * a.N + rbase + lr] = __float2bfloat16_rn(sum);
+      }
+    }
+  }
+  // on an aborted wait: let the copies this CTA issued land before exiting (bounded)
+  if (!ok && tid == 0) {
+    for (int j = st; j < min(nst, st + a.NS); ++j)
+      mbar_wait(&full[j % a.NS], (j / a.NS) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait);
+  }
+}
+
+struct StreamPlan {
+  int Tk, Tr, RS, NS, stage_bytes, sc_off, bi_off, threads, grid;
+  size_t smem;
+};
+
+template <int BITS, int CPT, int M, int RT>
+static cudaError_t qmv_stream_launch(const uint16_t *x, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                                     const uint16_t *biases, int64_t N, uint16_t *y, cudaStream_t stream,
+                                     const StreamPlan &pl) {
+  auto kern = qmv_stream_kernel<BITS, CPT, M, RT>;
+  static thread_local int cached_dev = -1;
+  static thread_local size_t cached_smem = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev || pl.smem > cached_smem) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pl.smem))) !=
+        cudaSuccess)
+      return e;
+    cached_dev = dev;
+    cached_smem = pl.smem;
+  }
+  QmvStreamArgs a;
+  a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  a.packed = packed;
+  a.scales = reinterpret_cast<const __half *>(scales);
+  a.biases = reinterpret_cast<const __half *>(biases);
+  a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.Gn = static_cast<int>(K / (CPT * 32));
+  a.Tk = pl.Tk;
+  a.Tr = pl.Tr;
+  a.RS = pl.RS;
+  a.NS = pl.NS;
+  a.stage_bytes = pl.stage_bytes;
+  a.sc_off = pl.sc_off;
+  a.bi_off = pl.bi_off;
+  kern<<<pl.grid, pl.threads, pl.smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int M>
+struct StreamRows {
+  static constexpr int value = (M <= 2) ? 4 : 2;
+};
+
+// Host plan of the streaming kernel, or false if the shape cannot use it.
+static bool plan_stream(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, StreamPlan &pl) {
+  if ((K * bits) % 128 != 0) return false;  // packed rows 16-byte aligned
+  const int64_t Gn = K / G;
+  if (Gn % 8 != 0) return false;            // scale/bias rows 16-byte aligned
+  const int RT = (M <= 2) ? 4 : 2;
+  int Tk = static_cast<int>(std::min<int64_t>((Gn + 31) / 32 * 32, kStreamMaxThreads));
+  int Tr = std::max(1, 256 / Tk);
+  pl.Tk = Tk;
+  pl.Tr = Tr;
+  pl.threads = Tk * Tr;
+  pl.RS = Tr * RT;
+  const int64_t wb = K * bits / 8, sb = Gn * 2;
+  auto al16 = [](int64_t v) { return (v + 15) / 16 * 16; };
+  pl.sc_off = static_cast<int>(al16(pl.RS * wb));
+  pl.bi_off = static_cast<int>(pl.sc_off + al16(pl.RS * sb));
+  pl.stage_bytes = static_cast<int>((pl.bi_off + al16(pl.RS * sb) + 127) / 128 * 128);
+  const size_t fixed = 16 * 8 /*barriers*/ + 16 + static_cast<size_t>(M) * Gn * (G + 4) * 4 +
+                       static_cast<size_t>(M) * Gn * 8 + 2 * (kStreamMaxThreads / 32) * 32 * 4 + 32 * 4 + 128;
+  const size_t budget = 227 * 1024;
+  if (fixed + 2 * static_cast<size_t>(pl.stage_bytes) > budget) return false;
+  pl.NS = static_cast<int>(std::min<size_t>(8, (budget - fixed) / pl.stage_bytes));
+  pl.smem = fixed + static_cast<size_t>(pl.NS) * pl.stage_bytes;
+  pl.grid = static_cast<int>(std::min<int64_t>(sms, N));
+  return true;
+}
+
 struct QmvLaunchInfo {
   int blocks_per_sm = 0;
   int sms = 0;
@@ -260,10 +589,42 @@ static cudaError_t qmv_launch_t(const uint16_t *x, int64_t K, const uint32_t *pa
   return cudaGetLastError();
 }
 
+template <int BITS, int CPT>
+static cudaError_t qmv_stream_m(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                                const uint16_t *scales, const uint16_t *biases, int64_t N, uint16_t *y, cudaStream_t s,
+                                const StreamPlan &pl) {
+  switch (M) {
+    case 1: return qmv_stream_launch<BITS, CPT, 1, StreamRows<1>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 2: return qmv_stream_launch<BITS, CPT, 2, StreamRows<2>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 3: return qmv_stream_launch<BITS, CPT, 3, StreamRows<3>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 4: return qmv_stream_launch<BITS, CPT, 4, StreamRows<4>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 5: return qmv_stream_launch<BITS, CPT, 5, StreamRows<5>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 6: return qmv_stream_launch<BITS, CPT, 6, StreamRows<6>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 7: return qmv_stream_launch<BITS, CPT, 7, StreamRows<7>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    default: return qmv_stream_launch<BITS, CPT, 8, StreamRows<8>::value>(x, K, packed, scales, biases, N, y, s, pl);
+  }
+}
+
 template <int BITS>
 static cudaError_t qmv_launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                                    const uint16_t *scales, const uint16_t *biases, int64_t N, int G, uint16_t *y,
                                    cudaStream_t s) {
+  static thread_local int cached_dev = -1, sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  StreamPlan pl;
+  if (plan_stream(M, N, K, G, BITS, sms, pl)) {
+    switch (G) {
+      case 32: return qmv_stream_m<BITS, 1>(x, M, K, packed, scales, biases, N, y, s, pl);
+      case 64: return qmv_stream_m<BITS, 2>(x, M, K, packed, scales, biases, N, y, s, pl);
+      default: return qmv_stream_m<BITS, 4>(x, M, K, packed, scales, biases, N, y, s, pl);
+    }
+  }
   switch (M) {
     case 1: return qmv_launch_t<BITS, 1>(x, K, packed, scales, biases, N, G, y, s);
     case 2: return qmv_launch_t<BITS, 2>(x, K, packed, scales, biases, N, G, y, s);
@@ -277,6 +638,20 @@ static cudaError_t qmv_launch_bits(const uint16_t *x, int64_t M, int64_t K, cons
 }
 
 size_t qmv_required_smem(int64_t M, int64_t K) { return qmv_smem_bytes(static_cast<int>(M), static_cast<int>(K)); }
+
+bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits) {
+  if (M < 1 || M > 8) return false;
+  StreamPlan pl;
+  if (plan_stream(M, N, K, G, bits, 148, pl)) return true;
+  return qmv_smem_bytes(static_cast<int>(M), static_cast<int>(K)) <= 227 * 1024;
+}
+
+cudaError_t read_and_clear_qmv_fault(uint32_t *word) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_qmv_fault, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_qmv_fault, &zero, sizeof(uint32_t));
+}
 
 cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s) {
