@@ -285,6 +285,12 @@ AQ_DEVICE float warp_reduce_scatter(float (&v)[RsInfo<NV>::NVP], int lane) {
   return v[0];
 }
 
+// Byte offset of the staged activations: after the stage ring, its mbarriers
+// and the abort flag, rounded up to 128 bytes (the array is read as float4).
+__host__ __device__ inline int stream_xs_offset(int NS, int stage_bytes) {
+  return (NS * stage_bytes + 8 * NS + 16 + 127) / 128 * 128;
+}
+
 template <int BITS, int CPT, int M, int RT>
 __global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const QmvStreamArgs a) {
   constexpr int G = CPT * 32;
@@ -296,7 +302,7 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const 
   uint8_t *ring = smem_raw;
   uint64_t *full = reinterpret_cast<uint64_t *>(ring + a.NS * a.stage_bytes);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(full + a.NS);
-  float *xs = reinterpret_cast<float *>(full + a.NS + 2);             // [M][Gn][GP]
+  float *xs = reinterpret_cast<float *>(smem_raw + stream_xs_offset(a.NS, a.stage_bytes));  // [M][Gn][GP], 128-aligned
   float2 *tab = reinterpret_cast<float2 *>(xs + M * a.Gn * GP);        // [M][Gn]  (sum x', sum x)
   float *red = reinterpret_cast<float *>(tab + M * a.Gn);              // [2][warps][32]
   float *fac = red + 2 * (kStreamMaxThreads / 32) * 32;               // [32]
@@ -538,12 +544,16 @@ static bool plan_stream(int64_t M, int64_t N, int64_t K, int G, int bits, int sm
   pl.sc_off = static_cast<int>(al16(pl.RS * wb));
   pl.bi_off = static_cast<int>(pl.sc_off + al16(pl.RS * sb));
   pl.stage_bytes = static_cast<int>((pl.bi_off + al16(pl.RS * sb) + 127) / 128 * 128);
-  const size_t fixed = 16 * 8 /*barriers*/ + 16 + static_cast<size_t>(M) * Gn * (G + 4) * 4 +
-                       static_cast<size_t>(M) * Gn * 8 + 2 * (kStreamMaxThreads / 32) * 32 * 4 + 32 * 4 + 128;
+  // after the ring: mbarriers + flag (<= 8*8 + 16 bytes, padded to 128), then x', tables, reductions, factors
+  const size_t tail = static_cast<size_t>(M) * Gn * (G + 4) * 4 + static_cast<size_t>(M) * Gn * 8 +
+                      2 * (kStreamMaxThreads / 32) * 32 * 4 + 32 * 4;
   const size_t budget = 227 * 1024;
-  if (fixed + 2 * static_cast<size_t>(pl.stage_bytes) > budget) return false;
-  pl.NS = static_cast<int>(std::min<size_t>(8, (budget - fixed) / pl.stage_bytes));
-  pl.smem = fixed + static_cast<size_t>(pl.NS) * pl.stage_bytes;
+  auto total = [&](int ns) { return static_cast<size_t>(stream_xs_offset(ns, pl.stage_bytes)) + tail; };
+  if (total(2) > budget) return false;
+  int ns = 2;
+  while (ns < 8 && total(ns + 1) <= budget) ++ns;
+  pl.NS = ns;
+  pl.smem = total(ns);
   pl.grid = static_cast<int>(std::min<int64_t>(sms, N));
   return true;
 }
