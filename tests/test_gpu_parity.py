@@ -207,8 +207,8 @@ def test_qmm_matches_dequantize_then_matmul():
     y = aq.aq_matmul_with("qmm", x, pg, sg, bg, G, bits).float()
     w16 = aq.aq_dequantize_f32(pg, sg, bg, K, G, bits).half().float()
     y_ref = x.float() @ w16.T
-    err = (y - y_ref).abs() / (y_ref.abs() + 1e-3 * y_ref.pow(2).mean().sqrt())
-    assert float(err.max()) < 2 ** -8 + 1e-4  # bf16 output rounding plus fp32 order
+    err = (y - y_ref).abs() / (y_ref.abs() + 1e-2 * y_ref.pow(2).mean().sqrt())
+    assert float(err.max()) < 2 ** -8  # bf16 output rounding (<= 2^-9 |y|) plus fp32 summation order
 
 
 def test_qmm_workspace_entry_point_matches():

@@ -163,6 +163,14 @@ __host__ __device__ constexpr float field_factor(int bits, int j) {
   return f;
 }
 
+// (a & b) | c as one three-input logic operation (truth table 0xEA).
+template <uint32_t B>
+AQ_DEVICE uint32_t lop3_and_or(uint32_t a, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(B), "r"(c));
+  return d;
+}
+
 // Magic float bits for code J (0..31) of a chunk held in w[0..BITS-1].
 template <int BITS, int J>
 AQ_DEVICE uint32_t extract_magic(const uint32_t (&w)[BITS]) {
@@ -174,10 +182,10 @@ AQ_DEVICE uint32_t extract_magic(const uint32_t (&w)[BITS]) {
     return __byte_perm(w[fp.word], kOne, sel);
   } else if constexpr (fp.rot < 0) {
     const uint32_t v = __funnelshift_r(w[fp.word], w[fp.word + 1], fp.off);
-    return ((v << fp.p) & (mask << fp.p)) | kOne;
+    return lop3_and_or<(mask << fp.p)>(v << fp.p, kOne);
   } else {
     const uint32_t v = fp.rot ? __funnelshift_l(w[fp.word], w[fp.word], fp.rot) : w[fp.word];
-    return (v & (mask << fp.p)) | kOne;
+    return lop3_and_or<(mask << fp.p)>(v, kOne);
   }
 }
 

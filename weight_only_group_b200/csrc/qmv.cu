@@ -225,20 +225,21 @@ __global__ void __launch_bounds__(kQmvThreads) qmv_kernel(const __nv_bfloat16 *_
 //
 //  * One persistent CTA per SM owns a contiguous, balanced range of rows
 //    (N / #CTAs +- 1), so every SM streams the same number of bytes.
-//  * Thread 0 streams the CTA's rows through a ring of shared-memory stages
-//    with 1-D bulk copies (cp.async.bulk, completion on mbarriers): a stage is
-//    RS consecutive rows of packed words, scales and biases, each one
-//    contiguous range of global memory.  All of a CTA's stages are in flight
-//    from the start when the ring is deep enough.
-//  * Threads are laid out as Tr row lanes x Tk group slots.  Thread (rl, gs)
-//    handles group slots gs, gs+Tk, ... of rows rl, rl+Tr, ... (RT rows per
-//    stage), so activations are read once per RT rows and the scale/bias fold
-//    runs once per group.
-//  * Row sums: warp reduce-scatter, then a cross-warp sum in shared memory.
+//  * Warp 0 is the producer: one lane streams the CTA's rows through a ring
+//    of shared-memory stages with 1-D bulk copies (cp.async.bulk, completion
+//    on "full" mbarriers).  A stage is W*RT consecutive rows of packed words,
+//    scales and biases: three contiguous ranges of global memory.
+//  * Warps 1..W are consumers.  Consumer warp c owns rows c*RT .. c*RT+RT-1
+//    of every stage and the whole K of each: lanes stride over the groups of
+//    the row, so each group's scale/bias fold happens once, activations are
+//    read once per RT rows, and a row's sum needs only a warp shuffle
+//    reduction.  A consumer releases a stage by arriving on its "empty"
+//    mbarrier; there is no CTA-wide barrier after the prologue, so a warp
+//    runs ahead as soon as its next stage has landed.
 // ===========================================================================
 __device__ uint32_t g_qmv_fault = 0;
 
-constexpr int kStreamMaxThreads = 512;
+constexpr int kRowsMaxThreads = 416;  // producer warp + up to 12 consumer warps
 
 struct QmvStreamArgs {
   const __nv_bfloat16 *x;
@@ -247,78 +248,45 @@ struct QmvStreamArgs {
   const __half *biases;
   __nv_bfloat16 *y;
   int N, K, Gn;
-  int Tk, Tr;         // threads per row lane (multiple of 32), row lanes
-  int RS, NS;         // rows per stage, stages in the ring
-  int stage_bytes;    // bytes of one stage (16-aligned)
+  int W;              // consumer warps
+  int NS;             // stages in the ring
+  int stage_bytes;    // bytes of one stage (128-aligned)
   int sc_off, bi_off; // byte offsets of scales and biases inside a stage
 };
 
-// Reduce-scatter of NV values across a warp: afterwards lane l holds the warp
-// total of value (l >> (5 - log2(NVP))) (NVP = NV rounded up to a power of 2).
-template <int NV>
-struct RsInfo {
-  static constexpr int NVP = NV <= 1 ? 1 : NV <= 2 ? 2 : NV <= 4 ? 4 : NV <= 8 ? 8 : NV <= 16 ? 16 : 32;
-  static constexpr int LOG = NVP == 1 ? 0 : NVP == 2 ? 1 : NVP == 4 ? 2 : NVP == 8 ? 3 : NVP == 16 ? 4 : 5;
-};
-template <int NV>
-AQ_DEVICE float warp_reduce_scatter(float (&v)[RsInfo<NV>::NVP], int lane) {
-  constexpr int NVP = RsInfo<NV>::NVP;
-  int cnt = NVP;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    if (cnt > 1) {
-      const int half = cnt / 2;
-      const bool up = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < NVP / 2; ++i) {
-        if (i < half) {
-          const float send = up ? v[i] : v[i + half];
-          const float keep = up ? v[i + half] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      cnt = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
-    }
-  }
-  return v[0];
-}
-
-// Byte offset of the staged activations: after the stage ring, its mbarriers
-// and the abort flag, rounded up to 128 bytes (the array is read as float4).
+// Byte offset of the staged activations: after the stage ring, its 2*NS
+// mbarriers and the abort flag, rounded up to 128 bytes (read as float4).
 __host__ __device__ inline int stream_xs_offset(int NS, int stage_bytes) {
-  return (NS * stage_bytes + 8 * NS + 16 + 127) / 128 * 128;
+  return (NS * stage_bytes + 16 * NS + 16 + 127) / 128 * 128;
 }
 
 template <int BITS, int CPT, int M, int RT>
-__global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const QmvStreamArgs a) {
+__global__ void __launch_bounds__(kRowsMaxThreads, 1) qmv_stream_kernel(const QmvStreamArgs a) {
   constexpr int G = CPT * 32;
   constexpr int GP = G + 4;          // padded floats per group of staged x
   constexpr int WPG = CPT * BITS;    // packed words per group
-  constexpr int NV = RT * M;
-  constexpr int NVP = RsInfo<NV>::NVP;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t *ring = smem_raw;
   uint64_t *full = reinterpret_cast<uint64_t *>(ring + a.NS * a.stage_bytes);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(full + a.NS);
-  float *xs = reinterpret_cast<float *>(smem_raw + stream_xs_offset(a.NS, a.stage_bytes));  // [M][Gn][GP], 128-aligned
-  float2 *tab = reinterpret_cast<float2 *>(xs + M * a.Gn * GP);        // [M][Gn]  (sum x', sum x)
-  float *red = reinterpret_cast<float *>(tab + M * a.Gn);              // [2][warps][32]
-  float *fac = red + 2 * (kStreamMaxThreads / 32) * 32;               // [32]
+  uint64_t *empty = full + a.NS;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + a.NS);
+  float *xs = reinterpret_cast<float *>(smem_raw + stream_xs_offset(a.NS, a.stage_bytes));  // [M][Gn][GP]
+  float2 *tab = reinterpret_cast<float2 *>(xs + M * a.Gn * GP);  // [M][Gn]: (sum x', sum x)
+  float *fac = reinterpret_cast<float *>(tab + M * a.Gn);        // [32]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nthreads = a.Tk * a.Tr;
+  const int nthreads = blockDim.x;
+  const int RSt = a.W * RT;  // rows per stage
   const int P = (a.K / 32) * BITS;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * a.N / gridDim.x;
   const int64_t r1 = static_cast<int64_t>(blockIdx.x + 1) * a.N / gridDim.x;
-  const int nst = static_cast<int>((r1 - r0 + a.RS - 1) / a.RS);
+  const int nst = static_cast<int>((r1 - r0 + RSt - 1) / RSt);
   const uint32_t row_w_bytes = static_cast<uint32_t>(P) * 4, row_s_bytes = static_cast<uint32_t>(a.Gn) * 2;
 
-  auto issue = [&](int st) {  // thread 0 only
+  auto issue = [&](int st) {  // one lane of the producer warp
     const int s = st % a.NS;
-    const int64_t rb = r0 + static_cast<int64_t>(st) * a.RS;
-    const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(a.RS), r1 - rb));
+    const int64_t rb = r0 + static_cast<int64_t>(st) * RSt;
+    const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(RSt), r1 - rb));
     uint8_t *dst = ring + s * a.stage_bytes;
     mbar_arrive_expect_tx(&full[s], rows * (row_w_bytes + 2 * row_s_bytes));
     bulk_g2s(dst, a.packed + rb * P, rows * row_w_bytes, &full[s]);
@@ -326,7 +294,10 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const 
     bulk_g2s(dst + a.bi_off, a.biases + rb * a.Gn, rows * row_s_bytes, &full[s]);
   };
   if (tid == 0) {
-    for (int s = 0; s < a.NS; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < a.NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], a.W);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     for (int st = 0; st < min(nst, a.NS); ++st) issue(st);
@@ -334,7 +305,7 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const 
   if (tid < 32) fac[tid] = field_factor(BITS, tid);
   __syncthreads();
 
-  // ---- stage x' = x * 2^(23-p) per group (padded) and per-group sums
+  // ---- stage x' = x * 2^(23-p) per group (padded) and per-group sums (all threads)
   {
     constexpr int PPG = G / 8;  // 8-element pieces per group (4, 8 or 16 adjacent lanes)
     const int per_row = a.K >> 3;
@@ -372,29 +343,51 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const 
   }
   __syncthreads();
 
-  const int rl = tid / a.Tk, gs0 = tid - rl * a.Tk;
-  const bool worker = tid < nthreads;
-  bool ok = true;
-  int st = 0;
-  for (; st < nst; ++st) {
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      int st = a.NS;
+      for (; st < nst; ++st) {
+        const int s = st % a.NS;
+        if (!(ok = mbar_wait(&empty[s], ((st / a.NS) - 1) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait))) break;
+        issue(st);
+      }
+      if (!ok) {  // let the copies already issued land before the CTA exits (bounded)
+        for (int j = max(0, st - a.NS); j < st; ++j)
+          mbar_wait(&full[j % a.NS], (j / a.NS) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int cw = warp - 1;
+  for (int st = 0; st < nst; ++st) {
     const int s = st % a.NS;
-    ok = mbar_wait(&full[s], (st / a.NS) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait);
-    if (!ok) break;
-    const uint32_t *wst = reinterpret_cast<const uint32_t *>(ring + s * a.stage_bytes);
-    const __half *sst = reinterpret_cast<const __half *>(ring + s * a.stage_bytes + a.sc_off);
-    const __half *bst = reinterpret_cast<const __half *>(ring + s * a.stage_bytes + a.bi_off);
-    float acc[NVP];
+    if (!mbar_wait(&full[s], (st / a.NS) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait)) break;
+    const int64_t rb = r0 + static_cast<int64_t>(st) * RSt;
+    const int rows_here = static_cast<int>(min(static_cast<int64_t>(RSt), r1 - rb));
+    const int lr0 = cw * RT;
+    if (lr0 < rows_here) {
+      const uint32_t *wst = reinterpret_cast<const uint32_t *>(ring + s * a.stage_bytes);
+      const __half *sst = reinterpret_cast<const __half *>(ring + s * a.stage_bytes + a.sc_off);
+      const __half *bst = reinterpret_cast<const __half *>(ring + s * a.stage_bytes + a.bi_off);
+      int lrow[RT];
 #pragma unroll
-    for (int v = 0; v < NVP; ++v) acc[v] = 0.0f;
-    if (worker) {
-      for (int gs = gs0; gs < a.Gn; gs += a.Tk) {
+      for (int r = 0; r < RT; ++r) lrow[r] = min(lr0 + r, rows_here - 1);
+      float acc[RT][M];
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
+      for (int gs = lane; gs < a.Gn; gs += 32) {
         float sc[RT], bi[RT];
         float2 A[RT][M];
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-          const int lr = rl + a.Tr * r;
-          sc[r] = __half2float(sst[lr * a.Gn + gs]);
-          bi[r] = __half2float(bst[lr * a.Gn + gs]);
+          sc[r] = __half2float(sst[lrow[r] * a.Gn + gs]);
+          bi[r] = __half2float(bst[lrow[r] * a.Gn + gs]);
 #pragma unroll
           for (int m = 0; m < M; ++m) A[r][m] = make_float2(0.0f, 0.0f);
         }
@@ -403,7 +396,7 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const 
           uint32_t w[RT][BITS];
 #pragma unroll
           for (int r = 0; r < RT; ++r) {
-            const uint32_t *src = wst + (rl + a.Tr * r) * P + gs * WPG + c * BITS;
+            const uint32_t *src = wst + lrow[r] * P + gs * WPG + c * BITS;
             if constexpr (BITS == 4) {
               const uint4 q = *reinterpret_cast<const uint4 *>(src);
               w[r][0] = q.x; w[r][1] = q.y; w[r][2] = q.z; w[r][3] = q.w;
@@ -446,42 +439,35 @@ __global__ void __launch_bounds__(kStreamMaxThreads, 1) qmv_stream_kernel(const 
 #pragma unroll
           for (int r = 0; r < RT; ++r) {
             const float sxq = (A[r][m].x + A[r][m].y) - t.x;  // sum of x*q over the group
-            acc[r * M + m] = fmaf(sc[r], sxq, fmaf(bi[r], t.y, acc[r * M + m]));
+            acc[r][m] = fmaf(sc[r], sxq, fmaf(bi[r], t.y, acc[r][m]));
           }
         }
       }
-    }
-    warp_reduce_scatter<NV>(acc, lane);
-    float *rb = red + (st & 1) * (kStreamMaxThreads / 32) * 32;
-    {
-      constexpr int SH = 5 - RsInfo<NV>::LOG;
-      const int vi = lane >> SH;
-      if ((lane & ((1 << SH) - 1)) == 0 && vi < NV) rb[warp * 32 + vi] = acc[0];
-    }
-    __syncthreads();  // stage s fully read; partial sums visible
-    if (tid == 0 && st + a.NS < nst) issue(st + a.NS);
-    {
-      const int64_t rbase = r0 + static_cast<int64_t>(st) * a.RS;
-      const int rows = static_cast<int>(min(static_cast<int64_t>(a.RS), r1 - rbase));
-      const int wpr = a.Tk / 32;  // warps per row lane
-      for (int t = tid; t < rows * M; t += blockDim.x) {
-        const int lr = t / M, m = t - lr * M;
-        const int r = lr / a.Tr, l = lr - r * a.Tr;
-        float sum = 0.0f;
-        for (int j = 0; j < wpr; ++j) sum += rb[(l * wpr + j) * 32 + r * M + m];
-        a.y[static_cast<int64_t>(m) * a.N + rbase + lr] = __float2bfloat16_rn(sum);
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          float v = acc[r][m];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          acc[r][m] = v;
+        }
+      if (lane == 0) {
+#pragma unroll
+        for (int r = 0; r < RT; ++r)
+          if (lr0 + r < rows_here)
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+              a.y[static_cast<int64_t>(m) * a.N + rb + lr0 + r] = __float2bfloat16_rn(acc[r][m]);
       }
     }
-  }
-  // on an aborted wait: let the copies this CTA issued land before exiting (bounded)
-  if (!ok && tid == 0) {
-    for (int j = st; j < min(nst, st + a.NS); ++j)
-      mbar_wait(&full[j % a.NS], (j / a.NS) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 
 struct StreamPlan {
-  int Tk, Tr, RS, NS, stage_bytes, sc_off, bi_off, threads, grid;
+  int W, NS, stage_bytes, sc_off, bi_off, threads, grid;
   size_t smem;
 };
 
@@ -511,9 +497,7 @@ static cudaError_t qmv_stream_launch(const uint16_t *x, int64_t K, const uint32_
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
   a.Gn = static_cast<int>(K / (CPT * 32));
-  a.Tk = pl.Tk;
-  a.Tr = pl.Tr;
-  a.RS = pl.RS;
+  a.W = pl.W;
   a.NS = pl.NS;
   a.stage_bytes = pl.stage_bytes;
   a.sc_off = pl.sc_off;
@@ -522,9 +506,12 @@ static cudaError_t qmv_stream_launch(const uint16_t *x, int64_t K, const uint32_
   return cudaGetLastError();
 }
 
-template <int M>
+// Rows per consumer warp per stage: 2 shares each activation read between two
+// rows; wide codes (8-bit) and M > 4 keep one row to stay within registers.
+__host__ __device__ constexpr int stream_rows(int bits, int64_t M) { return (M <= 4 && bits != 8) ? 2 : 1; }
+template <int BITS, int M>
 struct StreamRows {
-  static constexpr int value = (M <= 2) ? 4 : 2;
+  static constexpr int value = stream_rows(BITS, M);
 };
 
 // Host plan of the streaming kernel, or false if the shape cannot use it.
@@ -532,30 +519,34 @@ static bool plan_stream(int64_t M, int64_t N, int64_t K, int G, int bits, int sm
   if ((K * bits) % 128 != 0) return false;  // packed rows 16-byte aligned
   const int64_t Gn = K / G;
   if (Gn % 8 != 0) return false;            // scale/bias rows 16-byte aligned
-  const int RT = (M <= 2) ? 4 : 2;
-  int Tk = static_cast<int>(std::min<int64_t>((Gn + 31) / 32 * 32, kStreamMaxThreads));
-  int Tr = std::max(1, 256 / Tk);
-  pl.Tk = Tk;
-  pl.Tr = Tr;
-  pl.threads = Tk * Tr;
-  pl.RS = Tr * RT;
+  const int RT = stream_rows(bits, M);
   const int64_t wb = K * bits / 8, sb = Gn * 2;
   auto al16 = [](int64_t v) { return (v + 15) / 16 * 16; };
-  pl.sc_off = static_cast<int>(al16(pl.RS * wb));
-  pl.bi_off = static_cast<int>(pl.sc_off + al16(pl.RS * sb));
-  pl.stage_bytes = static_cast<int>((pl.bi_off + al16(pl.RS * sb) + 127) / 128 * 128);
-  // after the ring: mbarriers + flag (<= 8*8 + 16 bytes, padded to 128), then x', tables, reductions, factors
-  const size_t tail = static_cast<size_t>(M) * Gn * (G + 4) * 4 + static_cast<size_t>(M) * Gn * 8 +
-                      2 * (kStreamMaxThreads / 32) * 32 * 4 + 32 * 4;
+  const size_t tail = static_cast<size_t>(M) * Gn * (G + 4) * 4 + static_cast<size_t>(M) * Gn * 8 + 32 * 4;
   const size_t budget = 227 * 1024;
-  auto total = [&](int ns) { return static_cast<size_t>(stream_xs_offset(ns, pl.stage_bytes)) + tail; };
-  if (total(2) > budget) return false;
-  int ns = 2;
-  while (ns < 8 && total(ns + 1) <= budget) ++ns;
-  pl.NS = ns;
-  pl.smem = total(ns);
-  pl.grid = static_cast<int>(std::min<int64_t>(sms, N));
-  return true;
+  // the most consumer warps (<= 12) whose ring of >= 2 stages fits next to the staged activations
+  for (int W = 12; W >= 1; --W) {
+    const int RSt = W * RT;
+    const int sc_off = static_cast<int>(al16(RSt * wb));
+    const int bi_off = static_cast<int>(sc_off + al16(RSt * sb));
+    const int stage_bytes = static_cast<int>((bi_off + al16(RSt * sb) + 127) / 128 * 128);
+    auto total = [&](int ns) { return static_cast<size_t>(stream_xs_offset(ns, stage_bytes)) + tail; };
+    if (total(2) > budget) continue;
+    int ns = 2;
+    while (ns < 8 && total(ns + 1) <= budget) ++ns;
+    // keep at least 3 stages in flight when a smaller stage allows it
+    if (ns < 3 && W > 4) continue;
+    pl.W = W;
+    pl.NS = ns;
+    pl.stage_bytes = stage_bytes;
+    pl.sc_off = sc_off;
+    pl.bi_off = bi_off;
+    pl.threads = 32 * (W + 1);
+    pl.smem = total(ns);
+    pl.grid = static_cast<int>(std::min<int64_t>(sms, N));
+    return true;
+  }
+  return false;
 }
 
 struct QmvLaunchInfo {
@@ -604,14 +595,14 @@ static cudaError_t qmv_stream_m(const uint16_t *x, int64_t M, int64_t K, const u
                                 const uint16_t *scales, const uint16_t *biases, int64_t N, uint16_t *y, cudaStream_t s,
                                 const StreamPlan &pl) {
   switch (M) {
-    case 1: return qmv_stream_launch<BITS, CPT, 1, StreamRows<1>::value>(x, K, packed, scales, biases, N, y, s, pl);
-    case 2: return qmv_stream_launch<BITS, CPT, 2, StreamRows<2>::value>(x, K, packed, scales, biases, N, y, s, pl);
-    case 3: return qmv_stream_launch<BITS, CPT, 3, StreamRows<3>::value>(x, K, packed, scales, biases, N, y, s, pl);
-    case 4: return qmv_stream_launch<BITS, CPT, 4, StreamRows<4>::value>(x, K, packed, scales, biases, N, y, s, pl);
-    case 5: return qmv_stream_launch<BITS, CPT, 5, StreamRows<5>::value>(x, K, packed, scales, biases, N, y, s, pl);
-    case 6: return qmv_stream_launch<BITS, CPT, 6, StreamRows<6>::value>(x, K, packed, scales, biases, N, y, s, pl);
-    case 7: return qmv_stream_launch<BITS, CPT, 7, StreamRows<7>::value>(x, K, packed, scales, biases, N, y, s, pl);
-    default: return qmv_stream_launch<BITS, CPT, 8, StreamRows<8>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 1: return qmv_stream_launch<BITS, CPT, 1, StreamRows<BITS, 1>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 2: return qmv_stream_launch<BITS, CPT, 2, StreamRows<BITS, 2>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 3: return qmv_stream_launch<BITS, CPT, 3, StreamRows<BITS, 3>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 4: return qmv_stream_launch<BITS, CPT, 4, StreamRows<BITS, 4>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 5: return qmv_stream_launch<BITS, CPT, 5, StreamRows<BITS, 5>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 6: return qmv_stream_launch<BITS, CPT, 6, StreamRows<BITS, 6>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    case 7: return qmv_stream_launch<BITS, CPT, 7, StreamRows<BITS, 7>::value>(x, K, packed, scales, biases, N, y, s, pl);
+    default: return qmv_stream_launch<BITS, CPT, 8, StreamRows<BITS, 8>::value>(x, K, packed, scales, biases, N, y, s, pl);
   }
 }
 
