@@ -119,6 +119,33 @@ aq_status aq_matmul_ws(const uint16_t *x_bf16, int64_t M, int64_t K,
                        int64_t N, int G, int bits, uint16_t *y_bf16, void *workspace, size_t workspace_bytes,
                        aq_stream_t stream);
 
+/* Size of the fixed device workspace behind aq_matmul_qmm_static: 80 MiB.  A
+ * call needs 2*M*K + 4*M bytes (each term rounded up to 256; the fp16
+ * activations and their row scales), so for example M = 8192 with K = 4096, or
+ * M = 2048 with K = 14336, fit. */
+#define AQ_QMM_STATIC_WORKSPACE_BYTES (80u * 1024u * 1024u)
+
+/* The tensor-core matmul (AQ_KERNEL_QMM) without any allocation: its workspace
+ * is a fixed device array compiled into this library (every GPU that loads the
+ * library holds AQ_QMM_STATIC_WORKSPACE_BYTES of it until the process exits)
+ * instead of cudaMallocAsync or caller memory.  No counterpart on the pages: it
+ * exists for callers that cannot allocate device memory at call time, e.g. work
+ * captured into graphs whose launch path rejects memory-allocation nodes, or
+ * runtimes that reserve the whole device up front and forbid later cudaMalloc.
+ * Same arguments, layouts and result as aq_matmul_with(AQ_KERNEL_QMM, ...).
+ * Errors: shapes whose workspace (aq_matmul_workspace_bytes for a QMM shape)
+ * exceeds AQ_QMM_STATIC_WORKSPACE_BYTES -> AQ_ERR_UNSUPPORTED, checked before
+ * anything is launched; otherwise as aq_matmul_with.
+ * The first call on each device looks up the array's device address (which may
+ * load the module): make that first call before any stream capture.
+ * Every call shares the one array per device, so calls that can overlap on the
+ * GPU (different streams, or graphs replayed concurrently) race on it; serialize
+ * them.  The array keeps the last call's contents; nothing in it needs to start
+ * at zero (each call writes all of it that it reads). */
+aq_status aq_matmul_qmm_static(const uint16_t *x_bf16, int64_t M, int64_t K,
+                               const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                               int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
+
 /* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV returns AQ_ERR_UNSUPPORTED
  * when M > 8 or its shared-memory staging of x does not fit; AQ_KERNEL_QMM
  * returns AQ_ERR_UNSUPPORTED when K*bits is not a multiple of 128. */
