@@ -150,6 +150,79 @@ struct Cfg {
   static_assert(BN <= 256 && BN % 16 == 0, "MMA N");
 };
 
+// ---------------------------------------------------------------------------
+// Dequantization of one 32-code chunk into 16 TMEM columns of fp16 pairs.
+//
+// Bits 2, 4 and 8: codes become exact fp16 values 1024 + q by OR-ing them into
+// the mantissa of 1024.0 (one logic op or byte permute per two codes), then
+// q = (1024 + q) - 1024 and w = q*scale + bias with packed fp16 arithmetic:
+// one rounding, w = fp16_rn(q*scale + bias).  The two codes of a pair are
+// (j, j+4) of a word for 4-bit and (j, j+8) for 2-bit, so the chunk's K order
+// is interleaved in blocks of 8 (resp. 16) elements; the activation pre-pass
+// writes x16 in the same order (kx_perm below), which leaves the product
+// unchanged.  8-bit pairs are adjacent bytes (natural order).  3-bit codes go
+// through fp32 (exact q via the mantissa trick, one fp32 FMA, then RNE to fp16).
+// ---------------------------------------------------------------------------
+template <int BITS>
+AQ_DEVICE void dequant_chunk_f16(const uint32_t (&w)[BITS], uint16_t sc_bits, uint16_t bi_bits,
+                                 uint32_t (&cols)[16]) {
+  if constexpr (BITS == 4 || BITS == 2) {
+    constexpr int PER_WORD = 32 / BITS / 2;  // pairs per word: 4 (4-bit) or 8 (2-bit)
+    constexpr uint32_t LO = (1u << BITS) - 1u;
+    constexpr uint32_t MASK = LO | (LO << 16);
+    const __half2 s2 = __half2half2(__ushort_as_half(sc_bits));
+    const __half2 b2 = __half2half2(__ushort_as_half(bi_bits));
+    const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
+    const uint32_t magic = 0x64006400u;
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) {
+#pragma unroll
+      for (int j = 0; j < PER_WORD; ++j) {
+        const uint32_t v = lop3_and_or<MASK>(j ? (w[i] >> (BITS * j)) : w[i], magic);
+        __half2 h = *reinterpret_cast<const __half2 *>(&v);
+        h = __hfma2(__hsub2(h, k1024), s2, b2);
+        cols[PER_WORD * i + j] = *reinterpret_cast<uint32_t *>(&h);
+      }
+    }
+  } else if constexpr (BITS == 8) {
+    const __half2 s2 = __half2half2(__ushort_as_half(sc_bits));
+    const __half2 b2 = __half2half2(__ushort_as_half(bi_bits));
+    const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
+    const uint32_t magic = 0x64646464u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // bytes of the result: [code0, 0x64, code1, 0x64] -> (1024 + code0, 1024 + code1)
+      const uint32_t v0 = __byte_perm(w[i], magic, 0x5140u);
+      const uint32_t v1 = __byte_perm(w[i], magic, 0x5342u);
+      __half2 h0 = *reinterpret_cast<const __half2 *>(&v0);
+      __half2 h1 = *reinterpret_cast<const __half2 *>(&v1);
+      h0 = __hfma2(__hsub2(h0, k1024), s2, b2);
+      h1 = __hfma2(__hsub2(h1, k1024), s2, b2);
+      cols[2 * i] = *reinterpret_cast<uint32_t *>(&h0);
+      cols[2 * i + 1] = *reinterpret_cast<uint32_t *>(&h1);
+    }
+  } else {
+    const float scf = half_bits_to_float(sc_bits), bif = half_bits_to_float(bi_bits);
+    static_for<0, 16>([&](auto P) {
+      constexpr int j = 2 * P.value;
+      const float2 f = make_float2(__uint_as_float(extract_magic<BITS, j>(w)),
+                                   __uint_as_float(extract_magic<BITS, j + 1>(w)));
+      const float2 u = fadd2(f, make_float2(-1.0f, -1.0f));  // q * 2^(p-23), exact
+      constexpr float f0 = field_factor(BITS, j), f1 = field_factor(BITS, j + 1);
+      const float2 v = ffma2(u, make_float2(scf * f0, scf * f1), make_float2(bif, bif));  // fp32_rn(q*s + b)
+      __half2 h2 = __floats2half2_rn(v.x, v.y);
+      cols[P.value] = *reinterpret_cast<uint32_t *>(&h2);
+    });
+  }
+}
+
+// K order of x16 inside each block of 8 (4-bit) or 16 (2-bit) elements: slot t
+// holds element kx_perm(t) of the block, matching the pairs of dequant_chunk_f16.
+__host__ __device__ constexpr int kx_block(int bits) { return bits == 4 ? 8 : bits == 2 ? 16 : 1; }
+__host__ __device__ constexpr int kx_perm(int bits, int t) {
+  return kx_block(bits) == 1 ? t : (t % 2) * (kx_block(bits) / 2) + t / 2;
+}
+
 struct Params {
   const __half *scales;
   const __half *biases;
@@ -274,19 +347,30 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
       const int n = n0 + row;
       const bool row_ok = n < prm.N;
       const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
-      for (int kb = 0; kb < KB; ++kb, ++it) {
-        const int s = it % S;
-        const uint32_t r = it / S;
-        // scales/biases of this thread's chunks (loaded before the waits)
-        float sc[CH], bi[CH];
+      // scales/biases (fp16 bits) of this thread's chunks, prefetched two K blocks ahead
+      auto load_sb = [&](int kb, uint16_t (&sc)[CH], uint16_t (&bi)[CH]) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
           const int k = kb * C::BK + h * HALF + c * 32;
           const int g = k / prm.G;
-          const bool in = row_ok && g < prm.Gn;
-          sc[c] = in ? half_bits_to_float(ldg_nc2(prm.scales + g_row + g)) : 0.0f;
-          bi[c] = in ? half_bits_to_float(ldg_nc2(prm.biases + g_row + g)) : 0.0f;
+          const bool in = row_ok && kb < KB && g < prm.Gn;
+          sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
+          bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
         }
+      };
+      uint16_t sc_pf[2][CH], bi_pf[2][CH];
+      load_sb(0, sc_pf[0], bi_pf[0]);
+      load_sb(1, sc_pf[1], bi_pf[1]);
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t r = it / S;
+        uint16_t sc[CH], bi[CH];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          sc[c] = sc_pf[kb & 1][c];
+          bi[c] = bi_pf[kb & 1][c];
+        }
+        load_sb(kb + 2, sc_pf[kb & 1], bi_pf[kb & 1]);
         if (!(ok = mbar_wait(&full[s], r & 1, abort_flag, kFaultDequantWait))) break;
         if (r >= 1 && !(ok = mbar_wait(&empty[s], (r - 1) & 1, abort_flag, kFaultDequantWait))) break;
         __syncwarp();  // lanes leave the spin at different times; tcgen05.st needs the whole warp
@@ -299,17 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
 #pragma unroll
           for (int i = 0; i < BITS; ++i) w[i] = wrow[c * BITS + i];
           uint32_t packed_cols[16];
-          static_for<0, 16>([&](auto P) {
-            constexpr int j = 2 * P.value;
-            const float2 f = make_float2(__uint_as_float(extract_magic<BITS, j>(w)),
-                                         __uint_as_float(extract_magic<BITS, j + 1>(w)));
-            const float2 u = fadd2(f, make_float2(-1.0f, -1.0f));      // q * 2^(p-23), exact
-            constexpr float f0 = field_factor(BITS, j), f1 = field_factor(BITS, j + 1);
-            const float2 sp = make_float2(sc[c] * f0, sc[c] * f1);  // exact: powers of two
-            const float2 v = ffma2(u, sp, make_float2(bi[c], bi[c]));  // fp32_rn(q*s + b)
-            __half2 h2 = __floats2half2_rn(v.x, v.y);
-            packed_cols[P.value] = *reinterpret_cast<uint32_t *>(&h2);
-          });
+          dequant_chunk_f16<BITS>(w, sc[c], bi[c], packed_cols);
           tmem_st16(a_tmem + h * (HALF / 2) + c * 16, packed_cols);
         }
         tmem_st_wait();
@@ -364,21 +438,22 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
 // ---------------------------------------------------------------------------
 constexpr int kPrepThreads = 256;
 
+template <int BITS>
 __global__ void __launch_bounds__(kPrepThreads) x_to_f16_rows_kernel(const __nv_bfloat16 *__restrict__ x, int K,
                                                                      __half *__restrict__ x16,
                                                                      float *__restrict__ row_scale) {
   __shared__ float red[kPrepThreads / 32];
   const int64_t m = blockIdx.x;
   const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K);
-  const int n8 = K / 8;
+  const int n16 = K / 16;  // 16-element steps (K is a multiple of 32)
   float amax = 0.0f;
-  for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
+  for (int i = threadIdx.x; i < 2 * n16; i += kPrepThreads) {
     const uint4 v = ldg_nc16(src + i);
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      amax = fmaxf(amax, fabsf(__uint_as_float(u[h] << 16)));
-      amax = fmaxf(amax, fabsf(__uint_as_float(u[h] & 0xFFFF0000u)));
+    for (int hh = 0; hh < 4; ++hh) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(u[hh] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(u[hh] & 0xFFFF0000u)));
     }
   }
 #pragma unroll
@@ -388,7 +463,7 @@ __global__ void __launch_bounds__(kPrepThreads) x_to_f16_rows_kernel(const __nv_
   amax = red[0];
 #pragma unroll
   for (int w = 1; w < kPrepThreads / 32; ++w) amax = fmaxf(amax, red[w]);
-  // exponent of amax (bf16 values are never fp32-subnormal-only: 8-bit exponent kept)
+  // exponent of amax (bf16 keeps fp32's 8-bit exponent, so this is exact)
   int e = 0;
   if (amax > 0.0f) e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14;
   // 2^-e and 2^e as exact fp32 powers of two (|e| <= 141 needs two factors)
@@ -400,18 +475,25 @@ __global__ void __launch_bounds__(kPrepThreads) x_to_f16_rows_kernel(const __nv_
     row_scale[m] = up_a * up_b;
   }
   uint4 *dst = reinterpret_cast<uint4 *>(x16 + m * K);
-  for (int i = threadIdx.x; i < n8; i += kPrepThreads) {
-    const uint4 v = ldg_nc16(src + i);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+  for (int i = threadIdx.x; i < n16; i += kPrepThreads) {
+    const uint4 v0 = ldg_nc16(src + 2 * i), v1 = ldg_nc16(src + 2 * i + 1);
+    const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float lo = __uint_as_float(u[h] << 16) * down_a * down_b;
-      const float hi = __uint_as_float(u[h] & 0xFFFF0000u) * down_a * down_b;
-      __half2 p = __floats2half2_rn(lo, hi);
-      o[h] = *reinterpret_cast<uint32_t *>(&p);
+    for (int e2 = 0; e2 < 16; ++e2)
+      f[e2] = __uint_as_float(e2 & 1 ? (u[e2 >> 1] & 0xFFFF0000u) : (u[e2 >> 1] << 16)) * down_a * down_b;
+    uint32_t o[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      constexpr int B = kx_block(BITS);
+      const int e0 = (B == 16) ? kx_perm(BITS, 2 * t) : (B == 8 ? (2 * t >= 8 ? 8 : 0) + kx_perm(BITS, (2 * t) % 8) : 2 * t);
+      const int e1 = (B == 16) ? kx_perm(BITS, 2 * t + 1)
+                               : (B == 8 ? (2 * t + 1 >= 8 ? 8 : 0) + kx_perm(BITS, (2 * t + 1) % 8) : 2 * t + 1);
+      __half2 p = __floats2half2_rn(f[e0], f[e1]);
+      o[t] = *reinterpret_cast<uint32_t *>(&p);
     }
-    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -439,7 +521,7 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
   if (!fn) return cudaErrorNotSupported;
   __half *x16 = reinterpret_cast<__half *>(workspace);
   float *row_scale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + ((M * K * 2 + 255) / 256) * 256);
-  x_to_f16_rows_kernel<<<static_cast<unsigned>(M), kPrepThreads, 0, stream>>>(
+  x_to_f16_rows_kernel<BITS><<<static_cast<unsigned>(M), kPrepThreads, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale);
   cudaError_t pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;
