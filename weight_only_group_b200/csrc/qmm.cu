@@ -23,7 +23,9 @@
 //    layout) and the packed W tile [128 rows x BK*bits/32 words] into a ring
 //    of shared-memory stages, completing on the stage's mbarrier.
 //  * Warps 4..11 (two per TMEM lane quadrant): dequantize.  Thread (quadrant,
-//    lane) owns W row 32*quadrant+lane and one half of the K block: it reads
+//    lane) owns W row 32*quadrant+lane; the quadrant's two warps take
+//    alternate K blocks (each warp a whole block, so it has two MMA blocks of
+//    time per block of dequantization): it reads
 //    its packed words from shared memory, turns codes into fp16 weights in
 //    registers and writes them with tcgen05.st straight into a TMEM stage
 //    that the MMA reads as operand A (no swizzled shared-memory round trip).
@@ -167,22 +169,37 @@ template <int BITS>
 AQ_DEVICE void dequant_chunk_f16(const uint32_t (&w)[BITS], uint16_t sc_bits, uint16_t bi_bits,
                                  uint32_t (&cols)[16]) {
   if constexpr (BITS == 4 || BITS == 2) {
+    // Pair j of a word holds codes j and j + PER_WORD.  Pairs 0..PER_WORD/2-1
+    // are masked in place from the word (codes at bit offset BITS*j inside each
+    // 16-bit half) and the rest from the word shifted right by 8, so one shift
+    // per word suffices.  A code at offset BITS*j' inside the half reads as
+    // 1024 + q*2^(BITS*j'); q = h*2^-(BITS*j') - 1024*2^-(BITS*j') exactly.
     constexpr int PER_WORD = 32 / BITS / 2;  // pairs per word: 4 (4-bit) or 8 (2-bit)
+    constexpr int IN_BYTE = PER_WORD / 2;    // pairs per shifted copy: 2 or 4
     constexpr uint32_t LO = (1u << BITS) - 1u;
-    constexpr uint32_t MASK = LO | (LO << 16);
     const __half2 s2 = __half2half2(__ushort_as_half(sc_bits));
     const __half2 b2 = __half2half2(__ushort_as_half(bi_bits));
-    const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));
     const uint32_t magic = 0x64006400u;
 #pragma unroll
     for (int i = 0; i < BITS; ++i) {
-#pragma unroll
-      for (int j = 0; j < PER_WORD; ++j) {
-        const uint32_t v = lop3_and_or<MASK>(j ? (w[i] >> (BITS * j)) : w[i], magic);
+      const uint32_t src[2] = {w[i], w[i] >> 8};
+      static_for<0, PER_WORD>([&](auto J) {
+        constexpr int j = J.value;
+        constexpr int jj = j % IN_BYTE;  // position inside the byte
+        constexpr uint32_t MASK = (LO | (LO << 16)) << (BITS * jj);
+        const uint32_t v = lop3_and_or<MASK>(src[j / IN_BYTE], magic);
         __half2 h = *reinterpret_cast<const __half2 *>(&v);
-        h = __hfma2(__hsub2(h, k1024), s2, b2);
+        if constexpr (jj == 0) {
+          h = __hsub2(h, __half2half2(__ushort_as_half(0x6400)));  // - 1024
+        } else {
+          // h * 2^-(BITS*jj) - 1024 * 2^-(BITS*jj): both constants exact in fp16
+          constexpr unsigned short INV = static_cast<unsigned short>((15 - BITS * jj) << 10);
+          constexpr unsigned short OFF = static_cast<unsigned short>(0x8000u | ((25 - BITS * jj) << 10));
+          h = __hfma2(h, __half2half2(__ushort_as_half(INV)), __half2half2(__ushort_as_half(OFF)));
+        }
+        h = __hfma2(h, s2, b2);
         cols[PER_WORD * i + j] = *reinterpret_cast<uint32_t *>(&h);
-      }
+      });
     }
   } else if constexpr (BITS == 8) {
     const __half2 s2 = __half2half2(__ushort_as_half(sc_bits));
@@ -255,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&a_full[s], 8);
+      mbar_init(&a_full[s], 4);  // one warp per TMEM lane quadrant fills a K block
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
@@ -334,57 +351,68 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
     }
   } else if (warp >= kDequantWarp0) {
     // ------------------------------------------------------------------ dequant + epilogue
-    const int q = warp & 3;                 // TMEM lane quadrant
-    const int h = (warp - kDequantWarp0) >> 2;  // which half of the K block
-    const int row = q * 32 + lane;          // W row within the tile == TMEM lane
-    constexpr int HALF = C::BK / 2;         // elements per thread per K block
-    constexpr int CH = HALF / 32;           // 32-code chunks per thread per K block
-    uint32_t it = 0, t = 0;
+    const int q = warp & 3;                     // TMEM lane quadrant
+    const int h = (warp - kDequantWarp0) >> 2;  // the two warps of a quadrant alternate K blocks
+    const int row = q * 32 + lane;              // W row within the tile == TMEM lane
+    constexpr int CH = C::BK / 32;              // 32-code chunks per thread per K block
+    uint32_t it0 = 0, t = 0;                    // stage counter at the start of the tile
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t) {
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t, it0 += KB) {
       const int m0 = (tile % prm.m_tiles) * BN;
       const int n0 = (tile / prm.m_tiles) * 128;
       const int n = n0 + row;
       const bool row_ok = n < prm.N;
       const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
-      // scales/biases (fp16 bits) of this thread's chunks, prefetched two K blocks ahead
+      // scales/biases (fp16 bits) of this thread's chunks, prefetched for this
+      // warp's next two K blocks
       auto load_sb = [&](int kb, uint16_t (&sc)[CH], uint16_t (&bi)[CH]) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          const int k = kb * C::BK + h * HALF + c * 32;
-          const int g = k / prm.G;
+          const int g = (kb * C::BK + c * 32) / prm.G;
           const bool in = row_ok && kb < KB && g < prm.Gn;
           sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
           bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
         }
       };
       uint16_t sc_pf[2][CH], bi_pf[2][CH];
-      load_sb(0, sc_pf[0], bi_pf[0]);
-      load_sb(1, sc_pf[1], bi_pf[1]);
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      load_sb(h, sc_pf[0], bi_pf[0]);
+      load_sb(h + 2, sc_pf[1], bi_pf[1]);
+      int slot = 0;
+      for (int kb = h; kb < KB; kb += 2, slot ^= 1) {
+        const uint32_t it = it0 + kb;
         const int s = it % S;
         const uint32_t r = it / S;
         uint16_t sc[CH], bi[CH];
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          sc[c] = sc_pf[kb & 1][c];
-          bi[c] = bi_pf[kb & 1][c];
+          sc[c] = sc_pf[slot][c];
+          bi[c] = bi_pf[slot][c];
         }
-        load_sb(kb + 2, sc_pf[kb & 1], bi_pf[kb & 1]);
+        load_sb(kb + 4, sc_pf[slot], bi_pf[slot]);
         if (!(ok = mbar_wait(&full[s], r & 1, abort_flag, kFaultDequantWait))) break;
         if (r >= 1 && !(ok = mbar_wait(&empty[s], (r - 1) & 1, abort_flag, kFaultDequantWait))) break;
         __syncwarp();  // lanes leave the spin at different times; tcgen05.st needs the whole warp
-        const uint32_t *ws = reinterpret_cast<const uint32_t *>(smem + s * C::STAGE_BYTES + C::X_BYTES);
-        const uint32_t *wrow = ws + row * C::BKW + h * (HALF * BITS / 32);
+        const uint32_t *wrow =
+            reinterpret_cast<const uint32_t *>(smem + s * C::STAGE_BYTES + C::X_BYTES) + row * C::BKW;
         const uint32_t a_tmem = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::A_COL0 + s * C::A_COLS;
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
           uint32_t w[BITS];
+          if constexpr (BITS == 4) {
+            const uint4 v4 = *reinterpret_cast<const uint4 *>(wrow + c * 4);
+            w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+          } else if constexpr (BITS == 8) {
+            const uint4 a4 = reinterpret_cast<const uint4 *>(wrow + c * 8)[0];
+            const uint4 b4 = reinterpret_cast<const uint4 *>(wrow + c * 8)[1];
+            w[0] = a4.x; w[1] = a4.y; w[2] = a4.z; w[3] = a4.w;
+            w[4] = b4.x; w[5] = b4.y; w[6] = b4.z; w[7] = b4.w;
+          } else {
 #pragma unroll
-          for (int i = 0; i < BITS; ++i) w[i] = wrow[c * BITS + i];
+            for (int i = 0; i < BITS; ++i) w[i] = wrow[c * BITS + i];
+          }
           uint32_t packed_cols[16];
           dequant_chunk_f16<BITS>(w, sc[c], bi[c], packed_cols);
-          tmem_st16(a_tmem + h * (HALF / 2) + c * 16, packed_cols);
+          tmem_st16(a_tmem + c * 16, packed_cols);
         }
         tmem_st_wait();
         tc_fence_before();
