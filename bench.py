@@ -250,7 +250,7 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "peak_source": peaks["source"], "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
-                "kernel": "qmv_kernel<4,1> (3 launches per step)",
+                "kernel": "qmv_tc_kernel<bits=4,G=64,MP=1> (mma.sync m16n8k16 on exact fp16 codes; 3 launches per step)",
                 "algorithmic_bytes_per_step": STEP_BYTES}
     del graph
 
@@ -294,7 +294,7 @@ def run_ours(args, rank, world, local_rank):
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps,
             "warmup": reps_w * copies, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic (seeded; shapes of Llama-3-8B linears; no checkpoints)",
             "config": {"workload": WORKLOAD, "M": 1, "bits": BITS, "G": G, "shapes_KN": DECODE_SHAPES,
                        "parallelism": f"replicas x{world} (no data-path collective)",

@@ -159,6 +159,36 @@ def test_qmv_ragged_and_tiny(M, bits, K, N, G):
     _matmul_case(M, K, N, bits, G, 7000 + K + N, "qmv")
 
 
+# The tensor-core QMV (K a multiple of 8 groups): every bits x G x token count,
+# several K chunks per row, and a last row tile of one or two rows in each CTA.
+@pytest.mark.parametrize("M", (1, 2, 3, 4, 5, 8))
+@pytest.mark.parametrize("bits", (2, 4, 8))
+@pytest.mark.parametrize("G", (32, 64, 128))
+def test_qmv_tensor_core_tiles(M, bits, G):
+    K, N = 48 * G, 2600
+    _matmul_case(M, K, N, bits, G, 9100 + G + bits, "qmv")
+
+
+def test_qmv_extreme_activation_rows():
+    """Rows far outside fp16 range, a row of tiny values, an all-zero row and a
+    single 3e38 element: the per-group power-of-two scaling keeps them exact in
+    fp16 and the fold stays inside the fp32 range."""
+    M, K, N, G, bits = 4, 4096, 512, 64, 4
+    p_ref, s_ref, b_ref = quantized(N, K, 435, True, G, bits)
+    x = torch.from_numpy(activations_bits(M, K, 436).view(np.int16)).view(torch.bfloat16).float()
+    x[0] *= 2.0 ** 40
+    x[1] *= 2.0 ** -60
+    x[2] = 0.0
+    x[3, 5] = 3.0e38
+    xb = x.to(torch.bfloat16)
+    y = aq.aq_matmul_with("qmv", xb.cuda(), *_to_gpu(p_ref, s_ref, b_ref), G, bits)
+    y_ref = oracle.matmul(synth.bf16_bits(xb), p_ref, s_ref, b_ref, G, bits)
+    y = y.float().cpu().numpy().astype(np.float64)
+    for m in range(M):
+        ok, worst = oracle.tolerance_ok(y[m], y_ref[m], RTOL)
+        assert ok, (m, worst)
+
+
 def test_qmv_all_zero_codes_closed_form():
     """All codes 0: y[m, n] = sum_g bias[n, g] * sum_{k in g} x[m, k]."""
     M, N, K, G = 3, 77, 512, 64

@@ -14,6 +14,7 @@ cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
 size_t qmv_required_smem(int64_t M, int64_t K);
 bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t read_and_clear_qmv_fault(uint32_t *word);
+cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word);
 cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s);
 size_t qmm_workspace_bytes(int64_t M, int64_t K);
@@ -217,11 +218,13 @@ aq_status aq_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pac
 
 aq_status aq_device_fault(uint32_t *fault_word) {
   if (!fault_word) return AQ_ERR_INVALID_ARG;
-  uint32_t a = 0, b = 0;
+  uint32_t a = 0, b = 0, c = 0;
   aq_status st = from_cuda(aq::read_and_clear_fault(&a));
   if (st != AQ_OK) return st;
   st = from_cuda(aq::read_and_clear_qmv_fault(&b));
-  *fault_word = a | b;
+  if (st != AQ_OK) return st;
+  st = from_cuda(aq::read_and_clear_qmv_tc_fault(&c));
+  *fault_word = a | b | c;
   return st;
 }
 

@@ -2,6 +2,7 @@
 // shared with, or derived from, the CPU oracle.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -109,6 +110,16 @@ AQ_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_fla
     }
   }
 }
+// Bounded wait used while shutting down after an abort: it ignores the abort
+// flag (the point is to let copies or MMAs already issued complete before the
+// CTA exits or frees what they write to) and gives up after kWaitCycles.
+AQ_DEVICE bool mbar_drain(uint64_t *bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
 AQ_DEVICE void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -119,6 +130,16 @@ AQ_DEVICE void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *ba
                    smem_u32(dst)),
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
+}
+
+// 2-D tiled TMA load global -> shared (no multicast), completing on an
+// mbarrier; c0 is the innermost coordinate, c0 * element size % 16 == 0.
+AQ_DEVICE void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ---------------------------------------------------------------------------

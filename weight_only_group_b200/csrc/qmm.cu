@@ -64,13 +64,6 @@ AQ_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_fla
   return aq::mbar_wait(bar, parity, abort_flag, &g_fault_word, fault_bit);
 }
 
-AQ_DEVICE void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
-}
 
 AQ_DEVICE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 AQ_DEVICE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -315,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
       // drain: wait (bounded) until every issued load has landed
       const uint32_t issued = it;
       for (uint32_t j = (issued > static_cast<uint32_t>(S) ? issued - S : 0); j < issued; ++j) {
-        mbar_wait(&full[j % S], (j / S) & 1, abort_flag, kFaultProducerWait);
+        mbar_drain(&full[j % S], (j / S) & 1);
       }
     }
   } else if (warp == 1) {
@@ -347,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
         if (ok) tc_commit(acc_full);
       }
       // drain: the last commits must have landed before TMEM is released
-      if (it > 0) mbar_wait(&empty[(it - 1) % S], ((it - 1) / S) & 1, abort_flag, kFaultMmaWait);
+      if (it > 0) mbar_drain(&empty[(it - 1) % S], ((it - 1) / S) & 1);
     }
   } else if (warp >= kDequantWarp0) {
     // ------------------------------------------------------------------ dequant + epilogue

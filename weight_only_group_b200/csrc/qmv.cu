@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kRowsMaxThreads, 1) qmv_stream_kernel(const Qm
       }
       if (!ok) {  // let the copies already issued land before the CTA exits (bounded)
         for (int j = max(0, st - a.NS); j < st; ++j)
-          mbar_wait(&full[j % a.NS], (j / a.NS) & 1, abort_flag, &g_qmv_fault, kFaultQmvWait);
+          mbar_drain(&full[j % a.NS], (j / a.NS) & 1);
       }
     }
     return;
@@ -638,10 +638,15 @@ static cudaError_t qmv_launch_bits(const uint16_t *x, int64_t M, int64_t K, cons
   }
 }
 
+bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
+cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                          const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
+
 size_t qmv_required_smem(int64_t M, int64_t K) { return qmv_smem_bytes(static_cast<int>(M), static_cast<int>(K)); }
 
 bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits) {
   if (M < 1 || M > 8) return false;
+  if (qmv_tc_supported(M, N, K, G, bits)) return true;
   StreamPlan pl;
   if (plan_stream(M, N, K, G, bits, 148, pl)) return true;
   return qmv_smem_bytes(static_cast<int>(M), static_cast<int>(K)) <= 227 * 1024;
@@ -656,6 +661,7 @@ cudaError_t read_and_clear_qmv_fault(uint32_t *word) {
 
 cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s) {
+  if (qmv_tc_supported(M, N, K, G, bits)) return launch_qmv_tc(x, M, K, packed, scales, biases, N, G, bits, y, s);
   switch (bits) {
     case 2: return qmv_launch_bits<2>(x, M, K, packed, scales, biases, N, G, y, s);
     case 3: return qmv_launch_bits<3>(x, M, K, packed, scales, biases, N, G, y, s);

@@ -1,0 +1,738 @@
+// QMV on the tensor cores: y[M,N] = x[M,K] . dequant(W)^T for decode, M = 1..8
+// activation rows, W never materialised.
+//
+// Method: metalworking "MLX Quantization", section "Mechanics" (QMV streams
+// each weight once per decode step and dequantizes on the fly; multi-token
+// decode, M = 3..6, must still read W once) and anllm "Tutorial 10:
+// Quantization", section 5 (y = x @ W^T on the packed weights).  Per group g of
+// a row: y += s_g * sum_k q_k x_k + b_g * sum_k x_k.
+//
+// Why the tensor cores on a bandwidth-bound product: on the CUDA cores, code
+// extraction plus one FMA per weight and activation reads from shared memory
+// took longer than streaming the weights at B200's HBM rate (measured: the
+// arithmetic of a 14336x4096 4-bit call alone ran 1.4x longer than its copies
+// alone).  Here the arithmetic per weight is half a logic op: codes become
+// exact fp16 values 1024 + c two at a time (one LOP3 or PRMT), straight into
+// the A registers of mma.sync m16n8k16 (fp32 accumulate); the tensor core does
+// the multiply-adds.  mma.sync rather than tcgen05: its B operand sits in
+// registers, so the per-lane zero masking below costs one select per group,
+// while a shared-memory B operand would need eight zero-padded copies of x.
+//
+// Layout of the arithmetic:
+//  * MMA rows = 16 rows of W (a tile); MMA K = 16 codes of one group (codes
+//    are permuted inside the group so each lane's A registers come from its
+//    own packed words; the activations are staged in the same permutation).
+//    A field sitting 4*j bits (4-bit) or 2*j bits (2-bit) up in its 16-bit
+//    half reads as 1024 + 2^(bits*j) q, so its activation is staged times
+//    2^(-bits*j).
+//  * MMA columns: with MP = M rounded up to a power of two, column n is token
+//    n / (8/MP) and group slot n % (8/MP).  A lane reads the real activations
+//    only while the current group's slot is its column's slot, and zeros
+//    otherwise, so one accumulator holds 8/MP groups side by side and is
+//    folded once per 8/MP groups:
+//        y += s * 2^-e * (D - 1024 * sum B) + b * sum x
+//    where B = x * 2^e (* 2^(-bits*j)) in fp16 and 2^e is a power of two
+//    that puts the group's largest |x| in [2^14, 2^15): bf16 values scaled so
+//    are exact in fp16, and every product is exact in fp32.
+//  * Streaming: a producer warp copies (16-row tile, K chunk) stages into a
+//    shared-memory ring: three 2-D TMA boxes (codes, scales, biases; 64-bit
+//    elements, box rows padded so that the lanes of one shared-memory read hit
+//    distinct banks).  A CTA owns >= 16 rows; its last tile is moved up to end
+//    on its last row, so it repeats a few rows just read (L2 hits, masked out
+//    of the output) and never reads another CTA's rows.  The activations
+//    arrive by one bulk copy per token and are converted in place.
+//    Consumer warps (a divisor of the ring depth: one warp per slot) take
+//    whole stages round-robin.  The chunks of one tile are
+//    summed in chunk order through shared memory by the warp that handled the
+//    last chunk (deterministic), then stored as bf16 (RNE).
+//  * Every wait is bounded; a timeout sets a bit of g_qmv_tc_fault.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace aq {
+
+__device__ uint32_t g_qmv_tc_fault = 0;
+
+namespace qmm {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();  // driver entry point, resolved once (qmm.cu)
+}
+
+namespace tc {
+
+constexpr int kRows = 16;           // rows of W per tile (the MMA's M)
+constexpr int kMaxConsumers = 12;   // consumer warps per CTA at most
+constexpr int kRedBufs = 2;         // tiles whose chunk partials can be in flight
+constexpr int kMaxStages = 16;
+constexpr int kStageTarget = 16 * 1024;  // packed bytes of one stage we aim for (<= 1 KB per row)
+constexpr int kAcc = 4;                  // independent accumulator chains per warp
+constexpr uint32_t kMagic2 = 0x64006400u;  // fp16 pair (1024, 1024)
+
+__host__ __device__ constexpr int pow2_tokens(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+
+// Packed words of one group row that one lane reads, and the first of them.
+template <int BITS, int G>
+struct LaneWords {
+  static constexpr int count = BITS == 4 ? G / 32 : BITS == 8 ? G / 16 : (G >= 64 ? G / 64 : 1);
+  AQ_DEVICE static int first(int t) { return (BITS == 2 && G == 32) ? (t >> 1) : t * count; }
+};
+
+// Activations one lane stages per group: a run of consecutive elements
+// starting at span_start(t); element span_index(...) of that run pairs with
+// half hf of A pair (m2, lohi) of the lane's 16-byte unit c.
+template <int BITS, int G>
+struct LaneSpan {
+  static constexpr int length = (BITS == 2 && G == 32) ? 16 : G / 4;
+  AQ_DEVICE static int start(int t) { return (BITS == 2 && G == 32) ? 16 * (t >> 1) : t * (G / 4); }
+  // hh: which half of the shared word a lane of a 2-bit, G = 32 pair owns (t & 1)
+  __host__ __device__ static constexpr int index(int c, int m2, int lohi, int hf, int hh) {
+    return BITS == 4   ? 8 * c + 2 * m2 + lohi + 4 * hf
+           : BITS == 8 ? 4 * (2 * c + m2) + lohi + 2 * hf
+           : G >= 64   ? 16 * (c >> 1) + 4 * (c & 1) + 2 * m2 + lohi + 8 * hf
+                       : 4 * hh + 2 * m2 + lohi + 8 * hf;
+  }
+  // the field of that element sits 2^shift above the bottom of its fp16 mantissa
+  __host__ __device__ static constexpr int shift(int m2, int lohi) {
+    return BITS == 4 ? 4 * lohi : BITS == 2 ? 2 * (2 * m2 + lohi) : 0;
+  }
+};
+
+template <int N>
+AQ_DEVICE void lds_words(const uint8_t *p, uint32_t (&w)[N]) {
+  if constexpr (N == 1) {
+    w[0] = *reinterpret_cast<const uint32_t *>(p);
+  } else if constexpr (N == 2) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint4 v = reinterpret_cast<const uint4 *>(p)[i];
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  }
+}
+
+// fp16 pairs (1024 + c_lo, 1024 + c_hi) of unit C from one row's lane words:
+// p[m2][lohi] feeds MMA 2C + m2, A register "k 2t..2t+1" (lohi 0) or
+// "k 2t+8..2t+9" (lohi 1).
+template <int BITS, int G, int C>
+AQ_DEVICE void unit_pairs(const uint32_t (&w)[LaneWords<BITS, G>::count], int t, uint32_t (&p)[2][2]) {
+  if constexpr (BITS == 4) {
+    const uint32_t v0 = w[C], v1 = w[C] >> 8;
+    p[0][0] = lop3_and_or<0x000F000Fu>(v0, kMagic2);
+    p[0][1] = lop3_and_or<0x00F000F0u>(v0, kMagic2);
+    p[1][0] = lop3_and_or<0x000F000Fu>(v1, kMagic2);
+    p[1][1] = lop3_and_or<0x00F000F0u>(v1, kMagic2);
+  } else if constexpr (BITS == 2) {
+    uint32_t v;
+    if constexpr (G == 32) {
+      v = w[0] >> ((t & 1) * 8);
+    } else {
+      v = (C & 1) ? (w[C >> 1] >> 8) : w[C >> 1];
+    }
+    p[0][0] = lop3_and_or<0x00030003u>(v, kMagic2);
+    p[0][1] = lop3_and_or<0x000C000Cu>(v, kMagic2);
+    p[1][0] = lop3_and_or<0x00300030u>(v, kMagic2);
+    p[1][1] = lop3_and_or<0x00C000C0u>(v, kMagic2);
+  } else {
+    p[0][0] = __byte_perm(w[2 * C], 0x64646464u, 0x4240);
+    p[0][1] = __byte_perm(w[2 * C], 0x64646464u, 0x4341);
+    p[1][0] = __byte_perm(w[2 * C + 1], 0x64646464u, 0x4240);
+    p[1][1] = __byte_perm(w[2 * C + 1], 0x64646464u, 0x4341);
+  }
+}
+
+AQ_DEVICE void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                        uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Bounded spin until *ctr >= target (shared-memory counter written by other
+// warps of the CTA); false on timeout (fault bit set, abort raised) or abort.
+AQ_DEVICE bool spin_until_at_least(int *ctr, int target, volatile int *abort_flag) {
+  volatile int *c = ctr;
+  if (*c >= target) return true;
+  const long long t0 = clock64();
+  while (*c < target) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(&g_qmv_tc_fault, kFaultQmvWait);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
+struct Args {
+  const __nv_bfloat16 *x;
+  const uint32_t *packed;
+  const __half *scales, *biases;
+  __nv_bfloat16 *y;
+  int M, N, K, Gn;
+  int W, NS;                 // consumer warps, ring stages
+  int Kc, nch;               // K chunk of a stage, chunks per row
+  int pitch_w, pitch_s;      // bytes per row of codes / of scales (biases) in a stage
+  int s_off, b_off, stage_bytes;
+  int xs_off, tok_stride;    // staged activations: token m at xs_off + m * tok_stride
+  int zero_off, zero_stride; // two zero blocks
+  int tab_off, red_off, bar_off;
+  int w_box_x, sb_box_x;     // TMA x coordinate step of one chunk (64-bit elements)
+};
+
+template <int BITS, int G, int MP>
+__global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(const __grid_constant__ Args a, const __grid_constant__ CUtensorMap wmap,
+                                                                  const __grid_constant__ CUtensorMap smap,
+                                                                  const __grid_constant__ CUtensorMap bmap) {
+  constexpr int GS = 8 / MP;                     // groups side by side in one accumulator
+  constexpr int U = G / 32;                      // 16-byte activation units (two MMAs) per lane per group
+  constexpr int NWD = LaneWords<BITS, G>::count;
+  constexpr int GBYTES = G * BITS / 8;           // packed bytes of one group row
+  constexpr int SL = LaneSpan<BITS, G>::length;
+  constexpr int NACC = kAcc;
+  using Span = LaneSpan<BITS, G>;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t *ring = smem;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.bar_off);
+  uint64_t *empty = full + a.NS;
+  uint64_t *xbar = empty + a.NS;
+  // chunk partials of a tile: red_ready[b] counts partials written into buffer
+  // b, red_done[b] the tiles summed out of it (monotonic, so a waiter can never
+  // mistake an older round for the one it needs)
+  int *red_ready = reinterpret_cast<int *>(xbar + 1);
+  int *red_done = red_ready + kRedBufs;
+  volatile int *abort_flag = red_done + kRedBufs;
+  uint8_t *xs = smem + a.xs_off;
+  uint8_t *zero = smem + a.zero_off;
+  float4 *tab = reinterpret_cast<float4 *>(smem + a.tab_off);  // [MP][Gn]: (1024 sum B, sum x, 2^-e_lo, 2^-e_hi)
+  float *red = reinterpret_cast<float *>(smem + a.red_off);    // [kRedBufs][nch][16][MP]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * a.N / gridDim.x;
+  const int64_t r1 = static_cast<int64_t>(blockIdx.x + 1) * a.N / gridDim.x;
+  const int tiles = static_cast<int>((r1 - r0 + kRows - 1) / kRows);
+  const int nst = tiles * a.nch;
+  const int gpc = a.Kc / G;  // groups per chunk
+
+  // One stage: rows of codes, scales and biases of (tile, chunk); whole producer warp.
+  // First W row of tile T.  A CTA owns >= 16 rows, so its last tile is moved
+  // up to end at r1: its first rows repeat rows of the tile before (read again
+  // from L2, not stored twice) and every stage is three whole TMA boxes.
+  auto tile_base = [&](int T) { return min(r0 + static_cast<int64_t>(T) * kRows, r1 - kRows); };
+  // One stage: 16 rows of codes, scales and biases of (tile, chunk); one lane.
+  auto issue = [&](int st) {
+    const int s = st % a.NS;
+    const int T = st / a.nch, ch = st - T * a.nch;
+    const int rb = static_cast<int>(tile_base(T));
+    uint8_t *dst = ring + static_cast<size_t>(s) * a.stage_bytes;
+    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRows * (a.pitch_w + 2 * a.pitch_s)));
+    tma_load_2d(dst, &wmap, &full[s], ch * a.w_box_x, rb);
+    tma_load_2d(dst + a.s_off, &smap, &full[s], ch * a.sb_box_x, rb);
+    tma_load_2d(dst + a.b_off, &bmap, &full[s], ch * a.sb_box_x, rb);
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < a.NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < kRedBufs; ++b) red_ready[b] = red_done[b] = 0;
+    mbar_init(xbar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // the activations first (one row per token, raw bf16 into the staging area), then the ring
+    if (lane == 0) mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * a.K * 2);
+    __syncwarp();
+    if (lane < a.M)
+      bulk_g2s(xs + lane * a.tok_stride, a.x + static_cast<int64_t>(lane) * a.K, static_cast<uint32_t>(a.K) * 2, xbar);
+    if (lane == 0)
+      for (int st = 0; st < min(nst, a.NS); ++st) issue(st);
+  }
+
+  // ---- stage the activations in place (all threads): item = (token, group, lane t).
+  // A group's raw bf16 and its staged fp16 occupy the same 2G bytes; the four
+  // lanes of a group read all their raw values before any of them writes.
+  {
+    mbar_wait(xbar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait);
+    const int items = a.M * a.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
+    for (int i0 = 0; i0 < items; i0 += blockDim.x) {
+      const int i = i0 + tid;
+      const bool act = i < items;
+      const int ii = act ? i : 0;
+      const int t = ii & 3, mg = ii >> 2;
+      const int m = mg / a.Gn, gg = mg - m * a.Gn;
+      const uint8_t *src = xs + m * a.tok_stride + (gg * G + Span::start(t)) * 2;
+      uint32_t raw[SL / 2];
+#pragma unroll
+      for (int v = 0; v < SL / 8; ++v) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(src + 16 * v);
+        raw[4 * v] = q.x;
+        raw[4 * v + 1] = q.y;
+        raw[4 * v + 2] = q.z;
+        raw[4 * v + 3] = q.w;
+      }
+      float v8[U][8];
+      float amax = 0.0f, sx = 0.0f;
+      static_for<0, U>([&](auto C) {
+        static_for<0, 8>([&](auto S) {
+          constexpr int c = C.value, m2 = S.value >> 2, lohi = (S.value >> 1) & 1, hf = S.value & 1;
+          constexpr int e0 = Span::index(c, m2, lohi, hf, 0), e1 = Span::index(c, m2, lohi, hf, 1);
+          const uint32_t r0v = raw[e0 >> 1] >> ((e0 & 1) * 16), r1v = raw[e1 >> 1] >> ((e1 & 1) * 16);
+          const uint32_t bits16 = (e0 == e1 || !(t & 1)) ? r0v : r1v;
+          const float v = bf16_bits_to_float(bits16 & 0xFFFFu);
+          v8[c][S.value] = v;
+          amax = fmaxf(amax, fabsf(v));
+          sx += v;
+        });
+      });
+      __syncwarp();  // every lane of the warp has read its raw values
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+      sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+      // power of two 2^e with max|x| * 2^e in [2^14, 2^15) (e clamped to normal fp32 powers)
+      int e = 0;
+      if (amax > 0.0f) {
+        const int be = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+        e = min(max(14 - (be == 0 ? -127 : be - 127), -126), 126);
+      }
+      // 2^-e as 2^-e_lo * 2^-e_hi: the fold applies one half to D - 1024 sum B and
+      // the other to the scale, so neither product leaves the fp32 range
+      const int e_hi = e >> 1, e_lo = e - e_hi;
+      const float inv_lo = __uint_as_float(static_cast<uint32_t>(127 - e_lo) << 23);
+      const float inv_hi = __uint_as_float(static_cast<uint32_t>(127 - e_hi) << 23);
+      float offp = 0.0f;
+      uint8_t *dst = xs + m * a.tok_stride + (gg * U) * 64 + t * 16;
+      static_for<0, U>([&](auto C) {
+        constexpr int c = C.value;
+        uint32_t hw[4];
+        static_for<0, 4>([&](auto R) {
+          constexpr int m2 = R.value >> 1, lohi = R.value & 1;
+          const float f = __uint_as_float(static_cast<uint32_t>(e - Span::shift(m2, lohi) + 127) << 23);
+          const __half lo = __float2half_rn(v8[c][2 * R.value] * f);
+          const __half hi = __float2half_rn(v8[c][2 * R.value + 1] * f);
+          offp += __half2float(lo) + __half2float(hi);
+          hw[R.value] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+        });
+        if (act) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      });
+      offp += __shfl_xor_sync(0xffffffffu, offp, 1);
+      offp += __shfl_xor_sync(0xffffffffu, offp, 2);
+      if (act && t == 0) tab[m * a.Gn + gg] = make_float4(1024.0f * offp, sx, inv_lo, inv_hi);
+    }
+    // zero blocks, and the table rows of padding tokens
+    const int zbytes = a.zero_stride + U * 64;
+    for (int i = tid; i < zbytes / 16; i += blockDim.x)
+      reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = a.M * a.Gn + tid; i < MP * a.Gn; i += blockDim.x) tab[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    bool ok = true;
+    int st = a.NS;
+    for (; st < nst; ++st) {
+      const int s = st % a.NS;
+      int got = 1;
+      if (lane == 0) got = mbar_wait(&empty[s], ((st / a.NS) - 1) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait);
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) issue(st);
+    }
+    if (!ok && lane == 0) {  // let the copies already issued land before the CTA exits (bounded)
+      mbar_drain(xbar, 0);
+      for (int j = max(0, st - a.NS); j < st; ++j) mbar_drain(&full[j % a.NS], (j / a.NS) & 1);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int cw = warp - 1;
+  const int g = lane >> 2, t = lane & 3;
+  const int my_m = g / GS, my_j = g % GS;          // this lane's B column: token, group slot
+  const bool my_real = my_m < a.M;
+  const uint8_t *xs_lane = xs + (my_real ? my_m : 0) * a.tok_stride + t * 16;
+  const uint8_t *zero_lane = zero + (GS == 1 ? 0 : (my_m & 1)) * a.zero_stride + t * 16;
+  const int lw0 = LaneWords<BITS, G>::first(t) * 4;
+  const int nper = a.Kc / (GS * G);
+
+  for (int st = cw; st < nst; st += a.W) {
+    const int s = st % a.NS;
+    if (!mbar_wait(&full[s], (st / a.NS) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait)) break;
+    const int T = st / a.nch, ch = st - T * a.nch;
+    const int64_t rb = tile_base(T);
+    const int v0 = static_cast<int>(r0 + static_cast<int64_t>(T) * kRows - rb);  // rows [v0, 16) are new
+    auto row_ok = [&](int r) { return r >= v0 && rb + r < r1; };
+    const uint8_t *stg = ring + static_cast<size_t>(s) * a.stage_bytes;
+    const uint8_t *wr0 = stg + g * a.pitch_w + lw0;
+    const uint8_t *wr1 = wr0 + 8 * a.pitch_w;
+    const uint8_t *sr0 = stg + a.s_off + g * a.pitch_s, *sr1 = sr0 + 8 * a.pitch_s;
+    const uint8_t *br0 = stg + a.b_off + g * a.pitch_s, *br1 = br0 + 8 * a.pitch_s;
+    const int gch0 = ch * gpc;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+
+    for (int p = 0; p < nper; ++p) {
+      float d[NACC][4];
+#pragma unroll
+      for (int i = 0; i < NACC; ++i) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.0f;
+      static_for<0, GS>([&](auto J) {
+        constexpr int j = J.value;
+        const int gi = p * GS + j;
+        uint32_t w0[NWD], w1[NWD];
+        lds_words<NWD>(wr0 + gi * GBYTES, w0);
+        lds_words<NWD>(wr1 + gi * GBYTES, w1);
+        const uint8_t *bp = (my_real && my_j == j) ? xs_lane + (gch0 + gi) * (U * 64) : zero_lane;
+        static_for<0, U>([&](auto C) {
+          constexpr int c = C.value;
+          const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);
+          uint32_t p0[2][2], p1[2][2];
+          unit_pairs<BITS, G, c>(w0, t, p0);
+          unit_pairs<BITS, G, c>(w1, t, p1);
+          constexpr int i0 = (2 * (j * U + c)) % NACC, i1 = (2 * (j * U + c) + 1) % NACC;
+          mma16816(d[i0], p0[0][0], p1[0][0], p0[0][1], p1[0][1], bv.x, bv.y);
+          mma16816(d[i1], p0[1][0], p1[1][0], p0[1][1], p1[1][1], bv.z, bv.w);
+        });
+      });
+      float D[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        D[i] = d[0][i];
+#pragma unroll
+        for (int c = 1; c < NACC; ++c) D[i] += d[c][i];
+      }
+      // fold: D[0] = (row g, col 2t), D[1] = (row g, col 2t+1), D[2], D[3] = rows g+8
+      if constexpr (GS >= 2) {
+        const int gl = p * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
+        const int mt = (2 * t) / GS;
+        const float2 s0 = __half22float2(*reinterpret_cast<const __half2 *>(sr0 + gl * 2));
+        const float2 s1 = __half22float2(*reinterpret_cast<const __half2 *>(sr1 + gl * 2));
+        const float2 b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
+        const float2 b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
+        const float4 T0 = tab[mt * a.Gn + gch0 + gl], T1 = tab[mt * a.Gn + gch0 + gl + 1];
+        acc[0] = fmaf(s0.x * T0.w, (D[0] - T0.x) * T0.z, fmaf(b0.x, T0.y, acc[0]));
+        acc[1] = fmaf(s0.y * T1.w, (D[1] - T1.x) * T1.z, fmaf(b0.y, T1.y, acc[1]));
+        acc[2] = fmaf(s1.x * T0.w, (D[2] - T0.x) * T0.z, fmaf(b1.x, T0.y, acc[2]));
+        acc[3] = fmaf(s1.y * T1.w, (D[3] - T1.x) * T1.z, fmaf(b1.y, T1.y, acc[3]));
+      } else {
+        const int gl = p;
+        const float s0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
+        const float s1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
+        const float b0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
+        const float b1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
+        const float4 T0 = tab[(2 * t) * a.Gn + gch0 + gl], T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
+        acc[0] = fmaf(s0 * T0.w, (D[0] - T0.x) * T0.z, fmaf(b0, T0.y, acc[0]));
+        acc[1] = fmaf(s0 * T1.w, (D[1] - T1.x) * T1.z, fmaf(b0, T1.y, acc[1]));
+        acc[2] = fmaf(s1 * T0.w, (D[2] - T0.x) * T0.z, fmaf(b1, T0.y, acc[2]));
+        acc[3] = fmaf(s1 * T1.w, (D[3] - T1.x) * T1.z, fmaf(b1, T1.y, acc[3]));
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+
+    // Per (row, token) partials of this chunk: GS >= 2 sums the lane's two
+    // columns (same token) and then the lanes sharing the token.
+    float v[4];
+    if constexpr (GS >= 2) {
+      v[0] = acc[0] + acc[1];
+      v[1] = acc[2] + acc[3];
+      if constexpr (GS >= 4) {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+        v[1] += __shfl_xor_sync(0xffffffffu, v[1], 1);
+      }
+      if constexpr (GS >= 8) {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+        v[1] += __shfl_xor_sync(0xffffffffu, v[1], 2);
+      }
+    } else {
+      v[0] = acc[0];
+      v[1] = acc[1];
+      v[2] = acc[2];
+      v[3] = acc[3];
+    }
+    // holder lanes: GS >= 2 -> lanes with t % (GS/2) == 0 hold (rows g, g+8; token 2t/GS)
+    //               GS == 1 -> every lane holds (rows g, g+8; tokens 2t, 2t+1)
+    const bool holder = (GS == 1) || (t % (GS / 2 > 0 ? GS / 2 : 1) == 0);
+    auto put = [&](float *dstv, bool direct) {
+      if (!holder) return;
+      if constexpr (GS >= 2) {
+        const int tok = (2 * t) / GS;
+        if (direct) {
+          if (tok < a.M) {
+            if (row_ok(g)) a.y[static_cast<int64_t>(tok) * a.N + rb + g] = __float2bfloat16_rn(v[0]);
+            if (row_ok(g + 8)) a.y[static_cast<int64_t>(tok) * a.N + rb + g + 8] = __float2bfloat16_rn(v[1]);
+          }
+        } else {
+          dstv[g * MP + tok] = v[0];
+          dstv[(g + 8) * MP + tok] = v[1];
+        }
+      } else {
+        if (direct) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int tok = 2 * t + (q & 1), row = g + 8 * (q >> 1);
+            if (tok < a.M && row_ok(row)) a.y[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(v[q]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dstv[(g + 8 * (q >> 1)) * MP + 2 * t + (q & 1)] = v[q];
+        }
+      }
+    };
+    if (a.nch == 1) {
+      put(nullptr, true);
+      continue;
+    }
+    const int b = T % kRedBufs;
+    const int u = T / kRedBufs;
+    // buffer b is free once the u earlier tiles that used it have been summed
+    if (!spin_until_at_least(&red_done[b], u, abort_flag)) break;
+    float *rbuf = red + static_cast<size_t>(b) * a.nch * kRows * MP;
+    put(rbuf + static_cast<size_t>(ch) * kRows * MP, false);
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      atomicAdd(&red_ready[b], 1);
+    }
+    if (ch == a.nch - 1) {
+      if (!spin_until_at_least(&red_ready[b], (u + 1) * a.nch, abort_flag)) break;
+      __threadfence_block();
+      for (int idx = lane; idx < kRows * MP; idx += 32) {
+        const int row = idx / MP, tok = idx - row * MP;
+        float sum = 0.0f;
+        for (int c2 = 0; c2 < a.nch; ++c2) sum += rbuf[(static_cast<size_t>(c2) * kRows + row) * MP + tok];
+        if (tok < a.M && row_ok(row)) a.y[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(sum);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        atomicAdd(&red_done[b], 1);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host plan
+// ---------------------------------------------------------------------------
+struct Plan {
+  Args a;
+  int threads, grid;
+  size_t smem;
+};
+
+static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+// Smallest multiple of 16 bytes >= v with pitch % mod == rem.
+static int64_t pitch_at(int64_t v, int mod, int rem) {
+  int64_t p = round_up(v, 16);
+  while (p % mod != rem) p += 16;
+  return p;
+}
+
+// Row pitch of a stage's codes: rows one warp-wide shared-memory read touches
+// (8, 4 or 2 of them, by the read width) land on distinct banks.
+static int64_t code_pitch(int64_t row_bytes, int bits, int G) {
+  const int nwd = bits == 4 ? G / 32 : bits == 8 ? G / 16 : (G >= 64 ? G / 64 : 1);
+  if ((bits == 2 && G == 32) || nwd == 1 || nwd == 8) return pitch_at(row_bytes, 32, 16);
+  if (nwd == 2) return pitch_at(row_bytes, 64, 32);
+  return pitch_at(row_bytes, 128, 64);
+}
+
+static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl) {
+  if (!(bits == 2 || bits == 4 || bits == 8) || !(G == 32 || G == 64 || G == 128)) return false;
+  if (M < 1 || M > 8 || N < 1 || K < 1 || K % (8 * G) != 0) return false;
+  if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 30)) return false;
+  if (N < kRows) return false;  // every CTA owns at least one whole 16-row tile
+  const int MP = pow2_tokens(static_cast<int>(M));
+  const int64_t Gn = K / G, units = K / (8 * G);
+  const int U = G / 32;
+  // K chunk: the largest multiple u of 8 groups dividing K whose 16-row stage
+  // of codes stays within the target
+  int64_t u = 1;
+  for (int64_t c = 1; c <= units; ++c)
+    if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= kStageTarget) u = c;
+  const int64_t Kc = 8 * G * u, nch = K / Kc, gpc = Kc / G;
+  Args &a = pl.a;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.Gn = static_cast<int>(Gn);
+  a.Kc = static_cast<int>(Kc);
+  a.nch = static_cast<int>(nch);
+  a.pitch_w = static_cast<int>(code_pitch(Kc * bits / 8, bits, G));
+  a.pitch_s = static_cast<int>(pitch_at(gpc * 2, 32, 16));
+  if (a.pitch_w / 8 > 256 || a.pitch_s / 8 > 256) return false;  // TMA box width (64-bit elements)
+  a.w_box_x = static_cast<int>(Kc * bits / 64);
+  a.sb_box_x = static_cast<int>(gpc / 4);
+  a.s_off = kRows * a.pitch_w;
+  a.b_off = a.s_off + kRows * a.pitch_s;
+  a.stage_bytes = static_cast<int>(round_up(a.b_off + kRows * a.pitch_s, 128));
+  a.tok_stride = static_cast<int>(2 * K + 64);
+  a.zero_stride = static_cast<int>(round_up(U * 64, 128) + 64);
+  const int64_t budget = 227 * 1024;
+  struct Layout {
+    int64_t xs_off, zero_off, tab_off, red_off, bar_off, total;
+  };
+  auto layout = [&](int ns) {
+    Layout L;
+    int64_t off = static_cast<int64_t>(ns) * a.stage_bytes;
+    L.xs_off = off;
+    off += M * a.tok_stride;
+    L.zero_off = round_up(off, 128) + 64;
+    off = L.zero_off + a.zero_stride + U * 64;
+    L.tab_off = round_up(off, 16);
+    off = L.tab_off + static_cast<int64_t>(MP) * Gn * 16;
+    L.red_off = off;
+    off += static_cast<int64_t>(kRedBufs) * nch * kRows * MP * 4;
+    L.bar_off = round_up(off, 8);
+    L.total = L.bar_off + (2 * ns + 1) * 8 + (2 * kRedBufs + 1) * 4;
+    return L;
+  };
+  // consumer warps: a divisor of the ring depth, so every ring slot has one
+  // consumer warp and each of its full barriers is awaited phase after phase.
+  // Take the depth that fits and allows the most consumers (then the deepest).
+  auto consumers = [](int ns) {
+    for (int w = kMaxConsumers; w >= 1; --w)
+      if (ns % w == 0) return w;
+    return 1;
+  };
+  int best_ns = 0;
+  for (int ns = 2; ns <= kMaxStages; ++ns) {
+    if (layout(ns).total > budget) break;
+    if (best_ns == 0 || consumers(ns) >= consumers(best_ns)) best_ns = ns;
+  }
+  if (best_ns == 0) return false;
+  const Layout L = layout(best_ns);
+  a.NS = best_ns;
+  a.W = consumers(best_ns);
+  a.xs_off = static_cast<int>(L.xs_off);
+  a.zero_off = static_cast<int>(L.zero_off);
+  a.tab_off = static_cast<int>(L.tab_off);
+  a.red_off = static_cast<int>(L.red_off);
+  a.bar_off = static_cast<int>(L.bar_off);
+  pl.smem = static_cast<size_t>(L.total);
+  pl.threads = 32 * (a.W + 1);
+  pl.grid = static_cast<int>(std::min<int64_t>(sms, N / kRows));
+  return true;
+}
+
+struct Maps {
+  CUtensorMap w, s, b;
+};
+
+template <int BITS, int G, int MP>
+static cudaError_t launch(const Plan &pl, const Maps &mp, cudaStream_t stream) {
+  auto kern = qmv_tc_kernel<BITS, G, MP>;
+  static thread_local int cached_dev = -1;
+  static thread_local size_t cached_smem = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev || pl.smem > cached_smem) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pl.smem))) !=
+        cudaSuccess)
+      return e;
+    cached_dev = dev;
+    cached_smem = pl.smem;
+  }
+  kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.a, mp.w, mp.s, mp.b);
+  return cudaGetLastError();
+}
+
+template <int BITS, int G>
+static cudaError_t launch_mp(const Plan &pl, const Maps &mp, cudaStream_t stream) {
+  switch (pow2_tokens(pl.a.M)) {
+    case 1: return launch<BITS, G, 1>(pl, mp, stream);
+    case 2: return launch<BITS, G, 2>(pl, mp, stream);
+    case 4: return launch<BITS, G, 4>(pl, mp, stream);
+    default: return launch<BITS, G, 8>(pl, mp, stream);
+  }
+}
+
+template <int BITS>
+static cudaError_t launch_g(const Plan &pl, const Maps &mp, int G, cudaStream_t stream) {
+  switch (G) {
+    case 32: return launch_mp<BITS, 32>(pl, mp, stream);
+    case 64: return launch_mp<BITS, 64>(pl, mp, stream);
+    default: return launch_mp<BITS, 128>(pl, mp, stream);
+  }
+}
+
+// A [rows x row_bytes] row-major array as 64-bit elements, boxes of 16 rows x
+// box_bytes (the stage pitch; columns past the end of a row read as zeros).
+static bool encode_rows(CUtensorMap *map, const void *base, int64_t rows, int64_t row_bytes, int box_bytes) {
+  auto fn = qmm::encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes / 8), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes / 8), static_cast<cuuint32_t>(kRows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits) {
+  tc::Plan pl;
+  return tc::make_plan(M, N, K, G, bits, 148, pl);
+}
+
+cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                          const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s) {
+  static thread_local int cached_dev = -1, sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  tc::Plan pl;
+  if (!tc::make_plan(M, N, K, G, bits, sms, pl)) return cudaErrorInvalidValue;
+  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.packed = packed;
+  pl.a.scales = reinterpret_cast<const __half *>(scales);
+  pl.a.biases = reinterpret_cast<const __half *>(biases);
+  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  tc::Maps mp;
+  const int64_t row_bytes = K * bits / 8, sb_bytes = K / G * 2;
+  if (!tc::encode_rows(&mp.w, packed, N, row_bytes, pl.a.pitch_w) ||
+      !tc::encode_rows(&mp.s, scales, N, sb_bytes, pl.a.pitch_s) ||
+      !tc::encode_rows(&mp.b, biases, N, sb_bytes, pl.a.pitch_s))
+    return cudaErrorInvalidValue;
+  switch (bits) {
+    case 2: return tc::launch_g<2>(pl, mp, G, s);
+    case 4: return tc::launch_g<4>(pl, mp, G, s);
+    default: return tc::launch_g<8>(pl, mp, G, s);
+  }
+}
+
+cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_qmv_tc_fault, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  return cudaMemcpyToSymbol(g_qmv_tc_fault, &zero, sizeof(uint32_t));
+}
+
+}  // namespace aq
