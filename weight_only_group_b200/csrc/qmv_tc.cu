@@ -11,29 +11,29 @@
 // extraction plus one FMA per weight and activation reads from shared memory
 // took longer than streaming the weights at B200's HBM rate (measured: the
 // arithmetic of a 14336x4096 4-bit call alone ran 1.4x longer than its copies
-// alone).  Here the arithmetic per weight is half a logic op: codes become
-// exact fp16 values 1024 + c two at a time (one LOP3 or PRMT), straight into
-// the A registers of mma.sync m16n8k16 (fp32 accumulate); the tensor core does
-// the multiply-adds.  mma.sync rather than tcgen05: its B operand sits in
-// registers, so the per-lane zero masking below costs one select per group,
-// while a shared-memory B operand would need eight zero-padded copies of x.
+// alone).  Here the integer tensor cores (mma.sync m16n8k32, u8 x u8 / u8 x s8,
+// int32 accumulate) do the multiply-adds and the CUDA cores only unpack codes
+// into bytes: three logic ops per 8 codes at 4 bits, none at 8 bits.  mma.sync
+// rather than tcgen05: its B operand sits in registers, so the per-lane zero
+// masking below costs one select per group, while a shared-memory B operand
+// would need eight zero-padded copies of x.
 //
 // Layout of the arithmetic:
-//  * MMA rows = 16 rows of W (a tile); MMA K = 16 codes of one group (codes
-//    are permuted inside the group so each lane's A registers come from its
-//    own packed words; the activations are staged in the same permutation).
-//    A field sitting 4*j bits (4-bit) or 2*j bits (2-bit) up in its 16-bit
-//    half reads as 1024 + 2^(bits*j) q, so its activation is staged times
-//    2^(-bits*j).
+//  * MMA rows = 16 rows of W (a tile); MMA K = 32 codes of one group, as
+//    bytes (codes are permuted inside the group so each lane's A registers
+//    come from its own packed words; the activations are staged in the same
+//    permutation).
+//  * Activations: per group, x_int = rint(x * 2^e) with 2^e the power of two
+//    that puts the group's largest |x| in [2^13, 2^14), so |x_int| <= 2^14
+//    and the rounding error is at most 2^-14 of the group's largest |x|.
+//    x_int = 256 * hi + lo with lo in [0, 255] (u8) and hi in [-64, 64] (s8);
+//    two MMAs per A tile give sum q*lo and sum q*hi exactly in int32.
 //  * MMA columns: with MP = M rounded up to a power of two, column n is token
 //    n / (8/MP) and group slot n % (8/MP).  A lane reads the real activations
 //    only while the current group's slot is its column's slot, and zeros
 //    otherwise, so one accumulator holds 8/MP groups side by side and is
 //    folded once per 8/MP groups:
-//        y += s * 2^-e * (D - 1024 * sum B) + b * sum x
-//    where B = x * 2^e (* 2^(-bits*j)) in fp16 and 2^e is a power of two
-//    that puts the group's largest |x| in [2^14, 2^15): bf16 values scaled so
-//    are exact in fp16, and every product is exact in fp32.
+//        y += s * 2^-e * (256 * D_hi + D_lo) + b * sum x
 //  * Streaming: a producer warp copies (16-row tile, K chunk) stages into a
 //    shared-memory ring: three 2-D TMA boxes (codes, scales, biases; 64-bit
 //    elements, box rows padded so that the lanes of one shared-memory read hit
@@ -68,8 +68,8 @@ constexpr int kMaxConsumers = 12;   // consumer warps per CTA at most
 constexpr int kRedBufs = 2;         // tiles whose chunk partials can be in flight
 constexpr int kMaxStages = 16;
 constexpr int kStageTarget = 16 * 1024;  // packed bytes of one stage we aim for (<= 1 KB per row)
-constexpr int kAcc = 4;                  // independent accumulator chains per warp
-constexpr uint32_t kMagic2 = 0x64006400u;  // fp16 pair (1024, 1024)
+constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
 
 __host__ __device__ constexpr int pow2_tokens(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
@@ -81,22 +81,19 @@ struct LaneWords {
 };
 
 // Activations one lane stages per group: a run of consecutive elements
-// starting at span_start(t); element span_index(...) of that run pairs with
-// half hf of A pair (m2, lohi) of the lane's 16-byte unit c.
+// starting at start(t); element index(c, s, i, hh) of that run meets byte i of
+// A register set s (s = 0: MMA k 4t..4t+3, s = 1: k 16+4t..16+4t+3) of the
+// lane's K tile c (32 codes).  hh: the half of a shared word that a lane of a
+// 2-bit, G = 32 pair owns (t & 1).
 template <int BITS, int G>
 struct LaneSpan {
   static constexpr int length = (BITS == 2 && G == 32) ? 16 : G / 4;
   AQ_DEVICE static int start(int t) { return (BITS == 2 && G == 32) ? 16 * (t >> 1) : t * (G / 4); }
-  // hh: which half of the shared word a lane of a 2-bit, G = 32 pair owns (t & 1)
-  __host__ __device__ static constexpr int index(int c, int m2, int lohi, int hf, int hh) {
-    return BITS == 4   ? 8 * c + 2 * m2 + lohi + 4 * hf
-           : BITS == 8 ? 4 * (2 * c + m2) + lohi + 2 * hf
-           : G >= 64   ? 16 * (c >> 1) + 4 * (c & 1) + 2 * m2 + lohi + 8 * hf
-                       : 4 * hh + 2 * m2 + lohi + 8 * hf;
-  }
-  // the field of that element sits 2^shift above the bottom of its fp16 mantissa
-  __host__ __device__ static constexpr int shift(int m2, int lohi) {
-    return BITS == 4 ? 4 * lohi : BITS == 2 ? 2 * (2 * m2 + lohi) : 0;
+  __host__ __device__ static constexpr int index(int c, int s, int i, int hh) {
+    return BITS == 4   ? 8 * c + 2 * i + s
+           : BITS == 8 ? 4 * (2 * c + s) + i
+           : G >= 64   ? 16 * (c >> 1) + 2 * (c & 1) + s + 4 * i
+                       : 2 * hh + s + 4 * i;
   }
 };
 
@@ -120,41 +117,36 @@ AQ_DEVICE void lds_words(const uint8_t *p, uint32_t (&w)[N]) {
   }
 }
 
-// fp16 pairs (1024 + c_lo, 1024 + c_hi) of unit C from one row's lane words:
-// p[m2][lohi] feeds MMA 2C + m2, A register "k 2t..2t+1" (lohi 0) or
-// "k 2t+8..2t+9" (lohi 1).
+// The codes of K tile C of one row as bytes: a[0] = the 4 codes of register
+// set 0, a[1] = set 1 (positions as in LaneSpan::index).
 template <int BITS, int G, int C>
-AQ_DEVICE void unit_pairs(const uint32_t (&w)[LaneWords<BITS, G>::count], int t, uint32_t (&p)[2][2]) {
+AQ_DEVICE void tile_codes(const uint32_t (&w)[LaneWords<BITS, G>::count], int t, uint32_t (&a)[2]) {
   if constexpr (BITS == 4) {
-    const uint32_t v0 = w[C], v1 = w[C] >> 8;
-    p[0][0] = lop3_and_or<0x000F000Fu>(v0, kMagic2);
-    p[0][1] = lop3_and_or<0x00F000F0u>(v0, kMagic2);
-    p[1][0] = lop3_and_or<0x000F000Fu>(v1, kMagic2);
-    p[1][1] = lop3_and_or<0x00F000F0u>(v1, kMagic2);
-  } else if constexpr (BITS == 2) {
-    uint32_t v;
-    if constexpr (G == 32) {
-      v = w[0] >> ((t & 1) * 8);
-    } else {
-      v = (C & 1) ? (w[C >> 1] >> 8) : w[C >> 1];
-    }
-    p[0][0] = lop3_and_or<0x00030003u>(v, kMagic2);
-    p[0][1] = lop3_and_or<0x000C000Cu>(v, kMagic2);
-    p[1][0] = lop3_and_or<0x00300030u>(v, kMagic2);
-    p[1][1] = lop3_and_or<0x00C000C0u>(v, kMagic2);
+    a[0] = w[C] & 0x0F0F0F0Fu;
+    a[1] = (w[C] >> 4) & 0x0F0F0F0Fu;
+  } else if constexpr (BITS == 8) {
+    a[0] = w[2 * C];
+    a[1] = w[2 * C + 1];
+  } else if constexpr (G == 32) {
+    const uint32_t v = w[0] >> ((t & 1) * 4);
+    a[0] = v & 0x03030303u;
+    a[1] = (v >> 2) & 0x03030303u;
   } else {
-    p[0][0] = __byte_perm(w[2 * C], 0x64646464u, 0x4240);
-    p[0][1] = __byte_perm(w[2 * C], 0x64646464u, 0x4341);
-    p[1][0] = __byte_perm(w[2 * C + 1], 0x64646464u, 0x4240);
-    p[1][1] = __byte_perm(w[2 * C + 1], 0x64646464u, 0x4341);
+    const uint32_t v = (C & 1) ? (w[C >> 1] >> 4) : w[C >> 1];
+    a[0] = v & 0x03030303u;
+    a[1] = (v >> 2) & 0x03030303u;
   }
 }
 
-AQ_DEVICE void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                        uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+// d += A(16x32 u8) * B(32x8), B unsigned (u8) or signed (s8) bytes; int32 accumulate.
+AQ_DEVICE void mma_u8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+AQ_DEVICE void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
@@ -197,7 +189,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
                                                                   const __grid_constant__ CUtensorMap smap,
                                                                   const __grid_constant__ CUtensorMap bmap) {
   constexpr int GS = 8 / MP;                     // groups side by side in one accumulator
-  constexpr int U = G / 32;                      // 16-byte activation units (two MMAs) per lane per group
+  constexpr int U = G / 32;                      // K tiles (16 bytes of activation digits per lane) per group
   constexpr int NWD = LaneWords<BITS, G>::count;
   constexpr int GBYTES = G * BITS / 8;           // packed bytes of one group row
   constexpr int SL = LaneSpan<BITS, G>::length;
@@ -217,7 +209,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   volatile int *abort_flag = red_done + kRedBufs;
   uint8_t *xs = smem + a.xs_off;
   uint8_t *zero = smem + a.zero_off;
-  float4 *tab = reinterpret_cast<float4 *>(smem + a.tab_off);  // [MP][Gn]: (1024 sum B, sum x, 2^-e_lo, 2^-e_hi)
+  float4 *tab = reinterpret_cast<float4 *>(smem + a.tab_off);  // [MP][Gn]: (sum x, 2^-e_lo, 2^-e_hi, 0)
   float *red = reinterpret_cast<float *>(smem + a.red_off);    // [kRedBufs][nch][16][MP]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -265,87 +257,10 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       for (int st = 0; st < min(nst, a.NS); ++st) issue(st);
   }
 
-  // ---- stage the activations in place (all threads): item = (token, group, lane t).
-  // A group's raw bf16 and its staged fp16 occupy the same 2G bytes; the four
-  // lanes of a group read all their raw values before any of them writes.
-  {
-    mbar_wait(xbar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait);
-    const int items = a.M * a.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
-    for (int i0 = 0; i0 < items; i0 += blockDim.x) {
-      const int i = i0 + tid;
-      const bool act = i < items;
-      const int ii = act ? i : 0;
-      const int t = ii & 3, mg = ii >> 2;
-      const int m = mg / a.Gn, gg = mg - m * a.Gn;
-      const uint8_t *src = xs + m * a.tok_stride + (gg * G + Span::start(t)) * 2;
-      uint32_t raw[SL / 2];
-#pragma unroll
-      for (int v = 0; v < SL / 8; ++v) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(src + 16 * v);
-        raw[4 * v] = q.x;
-        raw[4 * v + 1] = q.y;
-        raw[4 * v + 2] = q.z;
-        raw[4 * v + 3] = q.w;
-      }
-      float v8[U][8];
-      float amax = 0.0f, sx = 0.0f;
-      static_for<0, U>([&](auto C) {
-        static_for<0, 8>([&](auto S) {
-          constexpr int c = C.value, m2 = S.value >> 2, lohi = (S.value >> 1) & 1, hf = S.value & 1;
-          constexpr int e0 = Span::index(c, m2, lohi, hf, 0), e1 = Span::index(c, m2, lohi, hf, 1);
-          const uint32_t r0v = raw[e0 >> 1] >> ((e0 & 1) * 16), r1v = raw[e1 >> 1] >> ((e1 & 1) * 16);
-          const uint32_t bits16 = (e0 == e1 || !(t & 1)) ? r0v : r1v;
-          const float v = bf16_bits_to_float(bits16 & 0xFFFFu);
-          v8[c][S.value] = v;
-          amax = fmaxf(amax, fabsf(v));
-          sx += v;
-        });
-      });
-      __syncwarp();  // every lane of the warp has read its raw values
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      sx += __shfl_xor_sync(0xffffffffu, sx, 1);
-      sx += __shfl_xor_sync(0xffffffffu, sx, 2);
-      // power of two 2^e with max|x| * 2^e in [2^14, 2^15) (e clamped to normal fp32 powers)
-      int e = 0;
-      if (amax > 0.0f) {
-        const int be = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
-        e = min(max(14 - (be == 0 ? -127 : be - 127), -126), 126);
-      }
-      // 2^-e as 2^-e_lo * 2^-e_hi: the fold applies one half to D - 1024 sum B and
-      // the other to the scale, so neither product leaves the fp32 range
-      const int e_hi = e >> 1, e_lo = e - e_hi;
-      const float inv_lo = __uint_as_float(static_cast<uint32_t>(127 - e_lo) << 23);
-      const float inv_hi = __uint_as_float(static_cast<uint32_t>(127 - e_hi) << 23);
-      float offp = 0.0f;
-      uint8_t *dst = xs + m * a.tok_stride + (gg * U) * 64 + t * 16;
-      static_for<0, U>([&](auto C) {
-        constexpr int c = C.value;
-        uint32_t hw[4];
-        static_for<0, 4>([&](auto R) {
-          constexpr int m2 = R.value >> 1, lohi = R.value & 1;
-          const float f = __uint_as_float(static_cast<uint32_t>(e - Span::shift(m2, lohi) + 127) << 23);
-          const __half lo = __float2half_rn(v8[c][2 * R.value] * f);
-          const __half hi = __float2half_rn(v8[c][2 * R.value + 1] * f);
-          offp += __half2float(lo) + __half2float(hi);
-          hw[R.value] = static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
-        });
-        if (act) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      });
-      offp += __shfl_xor_sync(0xffffffffu, offp, 1);
-      offp += __shfl_xor_sync(0xffffffffu, offp, 2);
-      if (act && t == 0) tab[m * a.Gn + gg] = make_float4(1024.0f * offp, sx, inv_lo, inv_hi);
-    }
-    // zero blocks, and the table rows of padding tokens
-    const int zbytes = a.zero_stride + U * 64;
-    for (int i = tid; i < zbytes / 16; i += blockDim.x)
-      reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
-    for (int i = a.M * a.Gn + tid; i < MP * a.Gn; i += blockDim.x) tab[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  }
-  __syncthreads();
-
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // (it stages nothing: its lane 0 may stall issuing copies, and the
+    // consumers must not wait for that before converting the activations)
     bool ok = true;
     int st = a.NS;
     for (; st < nst; ++st) {
@@ -364,6 +279,86 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     }
     return;
   }
+
+  // ---- consumers stage the activations in place: item = (token, group, lane t).
+  // A group's raw bf16 and its staged digits occupy the same 2G bytes; the four
+  // lanes of a group read all their raw values before any of them writes.
+  const int ctid = tid - 32, cthreads = a.W * 32;
+  {
+    mbar_wait(xbar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait);
+    const int items = a.M * a.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
+    for (int i0 = 0; i0 < items; i0 += cthreads) {
+      const int i = i0 + ctid;
+      const bool act = i < items;
+      const int ii = act ? i : 0;
+      const int t = ii & 3, mg = ii >> 2;
+      const int m = mg / a.Gn, gg = mg - m * a.Gn;
+      const uint8_t *src = xs + m * a.tok_stride + (gg * G + Span::start(t)) * 2;
+      uint32_t raw[SL / 2];
+#pragma unroll
+      for (int v = 0; v < SL / 8; ++v) {
+        const uint4 q = *reinterpret_cast<const uint4 *>(src + 16 * v);
+        raw[4 * v] = q.x;
+        raw[4 * v + 1] = q.y;
+        raw[4 * v + 2] = q.z;
+        raw[4 * v + 3] = q.w;
+      }
+      float v8[U][8];  // [tile][4 * set + byte]
+      float amax = 0.0f, sx = 0.0f;
+      static_for<0, U>([&](auto C) {
+        static_for<0, 8>([&](auto S) {
+          constexpr int c = C.value, st = S.value >> 2, i = S.value & 3;
+          constexpr int e0 = Span::index(c, st, i, 0), e1 = Span::index(c, st, i, 1);
+          const uint32_t r0v = raw[e0 >> 1] >> ((e0 & 1) * 16), r1v = raw[e1 >> 1] >> ((e1 & 1) * 16);
+          const uint32_t bits16 = (e0 == e1 || !(t & 1)) ? r0v : r1v;
+          const float v = bf16_bits_to_float(bits16 & 0xFFFFu);
+          v8[c][S.value] = v;
+          amax = fmaxf(amax, fabsf(v));
+          sx += v;
+        });
+      });
+      __syncwarp();  // every lane of the warp has read its raw values
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+      sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+      // power of two 2^e with max|x| * 2^e in [2^13, 2^14) (e clamped to normal fp32 powers)
+      int e = 0;
+      if (amax > 0.0f) {
+        const int be = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+        e = min(max(13 - (be == 0 ? -127 : be - 127), -126), 126);
+      }
+      // 2^-e as 2^-e_lo * 2^-e_hi: the fold applies one half to the integer dot
+      // product and the other to the scale, so neither product leaves fp32 range
+      const int e_hi = e >> 1, e_lo = e - e_hi;
+      const float inv_lo = __uint_as_float(static_cast<uint32_t>(127 - e_lo) << 23);
+      const float inv_hi = __uint_as_float(static_cast<uint32_t>(127 - e_hi) << 23);
+      const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+      uint8_t *dst = xs + m * a.tok_stride + (gg * U) * 64 + t * 16;
+      static_for<0, U>([&](auto C) {
+        constexpr int c = C.value;
+        uint32_t lo[2], hi[2];
+        static_for<0, 2>([&](auto S) {
+          // rint(v * 2^e) lands in the low 22 bits of v * 2^e + 1.5 * 2^23; its
+          // bytes 0 and 1 are the two's-complement digits lo and hi
+          uint32_t f[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) f[i] = __float_as_uint(fmaf(v8[c][4 * S.value + i], sc, kRoundMagic));
+          const uint32_t t01 = __byte_perm(f[0], f[1], 0x5140), t23 = __byte_perm(f[2], f[3], 0x5140);
+          lo[S.value] = __byte_perm(t01, t23, 0x5410);
+          hi[S.value] = __byte_perm(t01, t23, 0x7632);
+        });
+        if (act) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(lo[0], lo[1], hi[0], hi[1]);
+      });
+      if (act && t == 0) tab[m * a.Gn + gg] = make_float4(sx, inv_lo, inv_hi, 0.0f);
+    }
+    // zero blocks, and the table rows of padding tokens
+    const int zbytes = a.zero_stride + U * 64;
+    for (int i = ctid; i < zbytes / 16; i += cthreads) reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = a.M * a.Gn + ctid; i < MP * a.Gn; i += cthreads) tab[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+  // all consumer warps (not the producer) meet here: the staged activations are complete
+  asm volatile("bar.sync 1, %0;" ::"r"(cthreads) : "memory");
 
   // -------------------------------------------------------------- consumers
   const int cw = warp - 1;
@@ -391,9 +386,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 
     for (int p = 0; p < nper; ++p) {
-      float d[NACC][4];
+      int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
 #pragma unroll
-      for (int i = 0; i < NACC; ++i) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.0f;
+      for (int i = 0; i < NACC; ++i) dl[i][0] = dl[i][1] = dl[i][2] = dl[i][3] = dh[i][0] = dh[i][1] = dh[i][2] = dh[i][3] = 0;
       static_for<0, GS>([&](auto J) {
         constexpr int j = J.value;
         const int gi = p * GS + j;
@@ -403,21 +398,25 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const uint8_t *bp = (my_real && my_j == j) ? xs_lane + (gch0 + gi) * (U * 64) : zero_lane;
         static_for<0, U>([&](auto C) {
           constexpr int c = C.value;
-          const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);
-          uint32_t p0[2][2], p1[2][2];
-          unit_pairs<BITS, G, c>(w0, t, p0);
-          unit_pairs<BITS, G, c>(w1, t, p1);
-          constexpr int i0 = (2 * (j * U + c)) % NACC, i1 = (2 * (j * U + c) + 1) % NACC;
-          mma16816(d[i0], p0[0][0], p1[0][0], p0[0][1], p1[0][1], bv.x, bv.y);
-          mma16816(d[i1], p0[1][0], p1[1][0], p0[1][1], p1[1][1], bv.z, bv.w);
+          const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);  // lo set 0, lo set 1, hi set 0, hi set 1
+          uint32_t q0[2], q1[2];
+          tile_codes<BITS, G, c>(w0, t, q0);
+          tile_codes<BITS, G, c>(w1, t, q1);
+          constexpr int k = (j * U + c) % NACC;
+          mma_u8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
+          mma_u8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
         });
       });
-      float D[4];
+      float D[4];  // sum_k q_k x_int_k of the lane's 4 (row, column) cells, exact in int32
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        D[i] = d[0][i];
+        int lo = dl[0][i], hi = dh[0][i];
 #pragma unroll
-        for (int c = 1; c < NACC; ++c) D[i] += d[c][i];
+        for (int c = 1; c < NACC; ++c) {
+          lo += dl[c][i];
+          hi += dh[c][i];
+        }
+        D[i] = static_cast<float>(hi * 256 + lo);
       }
       // fold: D[0] = (row g, col 2t), D[1] = (row g, col 2t+1), D[2], D[3] = rows g+8
       if constexpr (GS >= 2) {
@@ -428,10 +427,10 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const float2 b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
         const float2 b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
         const float4 T0 = tab[mt * a.Gn + gch0 + gl], T1 = tab[mt * a.Gn + gch0 + gl + 1];
-        acc[0] = fmaf(s0.x * T0.w, (D[0] - T0.x) * T0.z, fmaf(b0.x, T0.y, acc[0]));
-        acc[1] = fmaf(s0.y * T1.w, (D[1] - T1.x) * T1.z, fmaf(b0.y, T1.y, acc[1]));
-        acc[2] = fmaf(s1.x * T0.w, (D[2] - T0.x) * T0.z, fmaf(b1.x, T0.y, acc[2]));
-        acc[3] = fmaf(s1.y * T1.w, (D[3] - T1.x) * T1.z, fmaf(b1.y, T1.y, acc[3]));
+        acc[0] = fmaf(s0.x * T0.z, D[0] * T0.y, fmaf(b0.x, T0.x, acc[0]));
+        acc[1] = fmaf(s0.y * T1.z, D[1] * T1.y, fmaf(b0.y, T1.x, acc[1]));
+        acc[2] = fmaf(s1.x * T0.z, D[2] * T0.y, fmaf(b1.x, T0.x, acc[2]));
+        acc[3] = fmaf(s1.y * T1.z, D[3] * T1.y, fmaf(b1.y, T1.x, acc[3]));
       } else {
         const int gl = p;
         const float s0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
@@ -439,10 +438,10 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const float b0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
         const float b1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
         const float4 T0 = tab[(2 * t) * a.Gn + gch0 + gl], T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
-        acc[0] = fmaf(s0 * T0.w, (D[0] - T0.x) * T0.z, fmaf(b0, T0.y, acc[0]));
-        acc[1] = fmaf(s0 * T1.w, (D[1] - T1.x) * T1.z, fmaf(b0, T1.y, acc[1]));
-        acc[2] = fmaf(s1 * T0.w, (D[2] - T0.x) * T0.z, fmaf(b1, T0.y, acc[2]));
-        acc[3] = fmaf(s1 * T1.w, (D[3] - T1.x) * T1.z, fmaf(b1, T1.y, acc[3]));
+        acc[0] = fmaf(s0 * T0.z, D[0] * T0.y, fmaf(b0, T0.x, acc[0]));
+        acc[1] = fmaf(s0 * T1.z, D[1] * T1.y, fmaf(b0, T1.x, acc[1]));
+        acc[2] = fmaf(s1 * T0.z, D[2] * T0.y, fmaf(b1, T0.x, acc[2]));
+        acc[3] = fmaf(s1 * T1.z, D[3] * T1.y, fmaf(b1, T1.x, acc[3]));
       }
     }
     __syncwarp();
