@@ -62,7 +62,7 @@ typedef enum {
 /* Kernel choice for aq_matmul_with (aq_matmul always uses AQ_KERNEL_AUTO). */
 typedef enum {
   AQ_KERNEL_AUTO = 0, /* host-side per-shape dispatch (see aq_dispatch) */
-  AQ_KERNEL_QMV = 1,  /* CUDA-core streaming kernel, M <= 8 */
+  AQ_KERNEL_QMV = 1,  /* decode kernel, M <= 8 (integer tensor cores; CUDA cores for 3-bit codes) */
   AQ_KERNEL_QMM = 2   /* tcgen05 / TMEM tensor-core kernel, any M */
 } aq_kernel;
 
@@ -92,16 +92,23 @@ aq_status aq_dequantize(const uint32_t *packed, const uint16_t *scales, const ui
 aq_status aq_dequantize_f32(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                             int64_t N, int64_t K, int G, int bits, float *w_out, aq_stream_t stream);
 
-/* Quantized matmul y[M,N] = x[M,K] @ dequant(W)^T, fp32 accumulation, bf16 (RNE)
- * output, without materialising dequant(W) in global memory.
+/* Quantized matmul y[M,N] = x[M,K] @ dequant(W)^T, bf16 (RNE) output, without
+ * materialising dequant(W) in global memory.
  * Source: anllm "Tutorial 10: Quantization", section 5, approach 2
  * (mx.quantized_matmul(..., transpose=True)); metalworking "MLX Quantization",
  * section "Mechanics" (QMV for decode, QMM for prefill, host-side per-shape
  * dispatch).  Accuracy: |y - y_ref| <= 8e-3 * (|y_ref| + rms(y_ref)) against the
- * exact product.  Kernels: QMV (CUDA cores, fp32 arithmetic on the exact codes)
- * for M <= 8; QMM (tensor cores) otherwise, on fp16 operands: weights
- * fp16_rn(fp32_rn(code*scale + bias)), activations scaled per row by an exact
- * power of two into fp16, fp32 accumulation. */
+ * exact product.  Kernels:
+ *  - QMV for M <= 8.  2/4/8-bit codes with K a multiple of 8*G: integer tensor
+ *    cores on the exact codes; each group's activations enter as 16-bit fixed
+ *    point, rint(x * 2^e) with 2^e the power of two that puts the group's
+ *    largest |x| in [2^13, 2^14) (error <= 2^-14 of that largest |x| per
+ *    element); group dot products exact in int32, then
+ *    y += scale * 2^-e * dot + bias * sum(x) in fp32.  Other shapes and 3-bit
+ *    codes: CUDA cores, fp32 arithmetic on the exact codes.
+ *  - QMM otherwise: tcgen05 tensor cores on fp16 operands, weights
+ *    fp16_rn(fp32_rn(code*scale + bias)), activations scaled per row by an
+ *    exact power of two into fp16, fp32 accumulation. */
 aq_status aq_matmul(const uint16_t *x_bf16, int64_t M, int64_t K,
                     const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                     int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
