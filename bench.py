@@ -214,9 +214,12 @@ def run_ours(args, rank, world, local_rank):
         sets.append(layer)
     torch.cuda.synchronize()
 
+    # Each launch may start while the previous one finishes (programmatic dependent
+    # launch): it reads its activations only after the previous kernel has
+    # completed, and the weights, which nothing writes during the step, before.
     def step(layer):
         for (p, s, b, x, y) in layer:
-            aq.aq_matmul(x, p, s, b, G, BITS, out=y)
+            aq.aq_matmul(x, p, s, b, G, BITS, out=y, overlap_previous=True)
 
     with torch.cuda.stream(stream):
         for _ in range(3):
@@ -271,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
     def e2e_step(layer):
         for (p, s, b, x, y), xh, yh in zip(layer, hx, hy):
             x.copy_(xh, non_blocking=True)
-            aq.aq_matmul(x, p, s, b, G, BITS, out=y)
+            aq.aq_matmul(x, p, s, b, G, BITS, out=y, overlap_previous=True)
             yh.copy_(y, non_blocking=True)
         torch.cuda.current_stream().synchronize()
         return float(hy[-1][0, 0])

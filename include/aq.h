@@ -113,6 +113,23 @@ aq_status aq_matmul(const uint16_t *x_bf16, int64_t M, int64_t K,
                     const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                     int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
 
+/* Flags of aq_matmul_ex. */
+enum {
+  /* Launch the decode kernel as a programmatic dependent of the kernel before it
+   * in `stream`, so its start overlaps that kernel's tail: it reads x only after
+   * the previous kernel has completed (its writes visible), but it reads the
+   * packed codes, scales and biases before.  The caller guarantees that no kernel
+   * still running in the stream writes those three arrays.  Honoured by the
+   * tensor-core QMV; other kernels launch as usual. */
+  AQ_MATMUL_OVERLAP_PREVIOUS = 1u
+};
+
+/* aq_matmul with flags (a bitwise OR of the AQ_MATMUL_* values; unknown bits ->
+ * AQ_ERR_INVALID_ARG).  Same results as aq_matmul, bit for bit. */
+aq_status aq_matmul_ex(const uint16_t *x_bf16, int64_t M, int64_t K,
+                       const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
+                       int64_t N, int G, int bits, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
+
 /* Bytes of workspace aq_matmul_ws needs for this shape (0 when the dispatched
  * kernel needs none, or when the arguments would be rejected).  Host only. */
 size_t aq_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K, int G, int bits);

@@ -135,6 +135,14 @@ def test_matmul_validation():
     assert L.aq_dequantize_f32(A, A, A, 4, 64, 64, 9, A, None) == aq.AQ_ERR_UNSUPPORTED
 
 
+def test_matmul_ex_flags():
+    L = aq.lib()
+    call = lambda flags: L.aq_matmul_ex(A, 1, 64, A, A, A, 8, 64, 4, A, flags, None)
+    assert call(2) == aq.AQ_ERR_INVALID_ARG          # unknown flag bit
+    assert call(1 << 31) == aq.AQ_ERR_INVALID_ARG
+    assert L.aq_matmul_ex(A, 0, 64, A, A, A, 8, 64, 4, A, aq.AQ_MATMUL_OVERLAP_PREVIOUS, None) == aq.AQ_ERR_INVALID_ARG
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

@@ -189,6 +189,57 @@ def test_qmv_extreme_activation_rows():
         assert ok, (m, worst)
 
 
+def _chain(ws, x, G, bits, overlap, graph=False):
+    """y_{i+1} = y_i @ dequant(W_i)^T through a list of square layers, on one stream."""
+    stream = torch.cuda.Stream()
+    outs = [torch.empty_like(x) for _ in ws]
+
+    def run():
+        cur = x
+        for (p, s, b), o in zip(ws, outs):
+            aq.aq_matmul(cur, p, s, b, G, bits, out=o, overlap_previous=overlap)
+            cur = o
+
+    with torch.cuda.stream(stream):
+        if graph:
+            run()  # warm-up outside the capture
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                run()
+            for o in outs:
+                o.zero_()
+            g.replay()
+        else:
+            run()
+    torch.cuda.synchronize()
+    return [o.clone() for o in outs]
+
+
+@pytest.mark.parametrize("graph", (False, True))
+def test_qmv_overlap_previous_chain(graph):
+    """Calls launched as programmatic dependents of the previous kernel, each
+    reading the previous call's output: identical, bit for bit, to plain launches
+    and within tolerance of the oracle chain."""
+    K = N = 4096
+    G, bits = 64, 4
+    ws = []
+    for i in range(4):
+        p, s, b = quantized(N, K, 7100 + i, True, G, bits)
+        ws.append(_to_gpu(p, s, b))
+    x = _x_gpu(activations_bits(1, K, 7199))
+    plain = _chain(ws, x, G, bits, False, graph)
+    over = _chain(ws, x, G, bits, True, graph)
+    for a_, b_ in zip(plain, over):
+        assert torch.equal(a_, b_)
+    # first two links against the oracle (the second on the GPU's first output)
+    p, s, b = quantized(N, K, 7100, True, G, bits)
+    y_ref = oracle.matmul(activations_bits(1, K, 7199), p, s, b, G, bits)
+    _assert_close(over[0], y_ref, "chain link 0")
+    x1 = synth.bf16_bits(over[0].cpu())
+    p, s, b = quantized(N, K, 7101, True, G, bits)
+    _assert_close(over[1], oracle.matmul(x1, p, s, b, G, bits), "chain link 1")
+
+
 def test_qmv_all_zero_codes_closed_form():
     """All codes 0: y[m, n] = sum_g bias[n, g] * sum_{k in g} x[m, k]."""
     M, N, K, G = 3, 77, 512, 64

@@ -33,6 +33,7 @@ AQ_ERR_DEVICE_FAULT = 5
 AQ_KERNEL_AUTO = 0
 AQ_KERNEL_QMV = 1
 AQ_KERNEL_QMM = 2
+AQ_MATMUL_OVERLAP_PREVIOUS = 1
 KERNELS = {"auto": AQ_KERNEL_AUTO, "qmv": AQ_KERNEL_QMV, "qmm": AQ_KERNEL_QMM}
 
 _lock = threading.Lock()
@@ -64,6 +65,7 @@ def lib() -> ctypes.CDLL:
             L.aq_dequantize_f32.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
             L.aq_matmul_with.argtypes = [i32, vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
+            L.aq_matmul_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, ctypes.c_uint32, vp]
             L.aq_matmul_ws.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, u64, vp]
             L.aq_matmul_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
             L.aq_matmul_workspace_bytes.restype = u64
@@ -197,9 +199,32 @@ def aq_matmul_with(kernel, x, packed, scales, biases, G: int, bits: int, out: to
     return out
 
 
-def aq_matmul(x, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None):
-    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T, kernel chosen per shape by the library."""
-    return aq_matmul_with(AQ_KERNEL_AUTO, x, packed, scales, biases, G, bits, out)
+def aq_matmul(x, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None,
+              overlap_previous: bool = False):
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T, kernel chosen per shape by the library.
+
+    overlap_previous: launch as a programmatic dependent of the kernel before it in
+    the stream (AQ_MATMUL_OVERLAP_PREVIOUS): x is read only after that kernel has
+    completed, the packed weights, scales and biases before, so no kernel still
+    running may write them."""
+    if not overlap_previous:
+        return aq_matmul_with(AQ_KERNEL_AUTO, x, packed, scales, biases, G, bits, out)
+    return aq_matmul_ex(x, packed, scales, biases, G, bits, AQ_MATMUL_OVERLAP_PREVIOUS, out)
+
+
+def aq_matmul_ex(x, packed, scales, biases, G: int, bits: int, flags: int, out: torch.Tensor | None = None):
+    """aq_matmul with AQ_MATMUL_* flags (see include/aq.h)."""
+    _need(x, "x", (torch.bfloat16,))
+    N = _qw(packed, scales, biases)
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16,))
+    with torch.cuda.device(x.device):
+        rc = lib().aq_matmul_ex(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, G,
+                                bits, out.data_ptr(), int(flags), _stream(x))
+    _check(rc, "aq_matmul_ex")
+    return out
 
 
 def aq_matmul_ws(x, packed, scales, biases, G: int, bits: int, workspace: torch.Tensor | None,

@@ -10,7 +10,7 @@ cudaError_t launch_quantize(const float *w, int64_t N, int64_t K, int G, int bit
 cudaError_t launch_dequantize(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                               int64_t N, int64_t K, int G, int bits, void *out, bool bf16_out, cudaStream_t s);
 cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, uint32_t flags, cudaStream_t s);
 size_t qmv_required_smem(int64_t M, int64_t K);
 bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t read_and_clear_qmv_fault(uint32_t *word);
@@ -166,10 +166,11 @@ static size_t workspace_for(aq_kernel kernel, int64_t M, int64_t K) {
 
 static aq_status matmul_run(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                             const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
-                            void *ws, aq_stream_t stream) {
+                            void *ws, aq_stream_t stream, uint32_t flags = 0) {
   aq_status st = check_device();
   if (st != AQ_OK) return st;
-  if (kernel == AQ_KERNEL_QMV) return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, stream));
+  if (kernel == AQ_KERNEL_QMV)
+    return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, flags, stream));
   return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, ws, stream));
 }
 
@@ -214,6 +215,18 @@ aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t
 aq_status aq_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                     const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, aq_stream_t stream) {
   return aq_matmul_with(AQ_KERNEL_AUTO, x, M, K, packed, scales, biases, N, G, bits, y, stream);
+}
+
+aq_status aq_matmul_ex(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, uint32_t flags,
+                       aq_stream_t stream) {
+  if (flags & ~static_cast<uint32_t>(AQ_MATMUL_OVERLAP_PREVIOUS)) return AQ_ERR_INVALID_ARG;
+  aq_kernel kernel = AQ_KERNEL_AUTO;
+  aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
+  if (st != AQ_OK) return st;
+  const size_t need = workspace_for(kernel, M, K);
+  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream, flags);
+  return aq_matmul_with(kernel, x, M, K, packed, scales, biases, N, G, bits, y, stream);
 }
 
 aq_status aq_device_fault(uint32_t *fault_word) {

@@ -640,7 +640,8 @@ static cudaError_t qmv_launch_bits(const uint16_t *x, int64_t M, int64_t K, cons
 
 bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                          const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
+                          const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, uint32_t flags,
+                          cudaStream_t s);
 
 size_t qmv_required_smem(int64_t M, int64_t K) { return qmv_smem_bytes(static_cast<int>(M), static_cast<int>(K)); }
 
@@ -660,8 +661,9 @@ cudaError_t read_and_clear_qmv_fault(uint32_t *word) {
 }
 
 cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s) {
-  if (qmv_tc_supported(M, N, K, G, bits)) return launch_qmv_tc(x, M, K, packed, scales, biases, N, G, bits, y, s);
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, uint32_t flags, cudaStream_t s) {
+  if (qmv_tc_supported(M, N, K, G, bits))
+    return launch_qmv_tc(x, M, K, packed, scales, biases, N, G, bits, y, flags, s);
   switch (bits) {
     case 2: return qmv_launch_bits<2>(x, M, K, packed, scales, biases, N, G, y, s);
     case 3: return qmv_launch_bits<3>(x, M, K, packed, scales, biases, N, G, y, s);

@@ -69,6 +69,7 @@ constexpr int kRedBufs = 2;         // tiles whose chunk partials can be in flig
 constexpr int kMaxStages = 16;
 constexpr int kStageTarget = 16 * 1024;  // packed bytes of one stage we aim for (<= 1 KB per row)
 constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
+constexpr int kEarlyStages = 2;          // weight stages issued before the previous kernel completes (overlap mode)
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
 
 __host__ __device__ constexpr int pow2_tokens(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
@@ -182,6 +183,7 @@ struct Args {
   int zero_off, zero_stride; // two zero blocks
   int tab_off, red_off, bar_off;
   int w_box_x, sb_box_x;     // TMA x coordinate step of one chunk (64-bit elements)
+  int early_w;               // weight stages issued before the previous kernel has completed
 };
 
 template <int BITS, int G, int MP>
@@ -247,14 +249,23 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     fence_barrier_init();
   }
   __syncthreads();
+  // A kernel launched after this one as a programmatic dependent may start its
+  // prologue now; it waits for this grid before reading anything it writes.
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp == 0) {
-    // the activations first (one row per token, raw bf16 into the staging area), then the ring
+    // Weights first when the caller allows it (they are not written by the
+    // kernel this one may overlap), then, once the kernel before has completed,
+    // the activations (one row per token, raw bf16 into the staging area).
+    const int early = min(min(nst, a.NS), a.early_w);  // never more than the ring holds
+    if (lane == 0)
+      for (int st = 0; st < early; ++st) issue(st);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (lane == 0) mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * a.K * 2);
     __syncwarp();
     if (lane < a.M)
       bulk_g2s(xs + lane * a.tok_stride, a.x + static_cast<int64_t>(lane) * a.K, static_cast<uint32_t>(a.K) * 2, xbar);
     if (lane == 0)
-      for (int st = 0; st < min(nst, a.NS); ++st) issue(st);
+      for (int st = early; st < min(nst, a.NS); ++st) issue(st);
   }
 
   if (warp == 0) {
@@ -639,7 +650,7 @@ struct Maps {
 };
 
 template <int BITS, int G, int MP>
-static cudaError_t launch(const Plan &pl, const Maps &mp, cudaStream_t stream) {
+static cudaError_t launch(const Plan &pl, const Maps &mp, bool overlap, cudaStream_t stream) {
   auto kern = qmv_tc_kernel<BITS, G, MP>;
   static thread_local int cached_dev = -1;
   static thread_local size_t cached_smem = 0;
@@ -653,26 +664,39 @@ static cudaError_t launch(const Plan &pl, const Maps &mp, cudaStream_t stream) {
     cached_dev = dev;
     cached_smem = pl.smem;
   }
-  kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.a, mp.w, mp.s, mp.b);
-  return cudaGetLastError();
+  if (!overlap) {
+    kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.a, mp.w, mp.s, mp.b);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(pl.threads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, pl.a, mp.w, mp.s, mp.b);
 }
 
 template <int BITS, int G>
-static cudaError_t launch_mp(const Plan &pl, const Maps &mp, cudaStream_t stream) {
+static cudaError_t launch_mp(const Plan &pl, const Maps &mp, bool overlap, cudaStream_t stream) {
   switch (pow2_tokens(pl.a.M)) {
-    case 1: return launch<BITS, G, 1>(pl, mp, stream);
-    case 2: return launch<BITS, G, 2>(pl, mp, stream);
-    case 4: return launch<BITS, G, 4>(pl, mp, stream);
-    default: return launch<BITS, G, 8>(pl, mp, stream);
+    case 1: return launch<BITS, G, 1>(pl, mp, overlap, stream);
+    case 2: return launch<BITS, G, 2>(pl, mp, overlap, stream);
+    case 4: return launch<BITS, G, 4>(pl, mp, overlap, stream);
+    default: return launch<BITS, G, 8>(pl, mp, overlap, stream);
   }
 }
 
 template <int BITS>
-static cudaError_t launch_g(const Plan &pl, const Maps &mp, int G, cudaStream_t stream) {
+static cudaError_t launch_g(const Plan &pl, const Maps &mp, int G, bool overlap, cudaStream_t stream) {
   switch (G) {
-    case 32: return launch_mp<BITS, 32>(pl, mp, stream);
-    case 64: return launch_mp<BITS, 64>(pl, mp, stream);
-    default: return launch_mp<BITS, 128>(pl, mp, stream);
+    case 32: return launch_mp<BITS, 32>(pl, mp, overlap, stream);
+    case 64: return launch_mp<BITS, 64>(pl, mp, overlap, stream);
+    default: return launch_mp<BITS, 128>(pl, mp, overlap, stream);
   }
 }
 
@@ -698,7 +722,8 @@ bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits) {
 }
 
 cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                          const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s) {
+                          const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, uint32_t flags,
+                          cudaStream_t s) {
   static thread_local int cached_dev = -1, sms = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -714,6 +739,8 @@ cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_
   pl.a.scales = reinterpret_cast<const __half *>(scales);
   pl.a.biases = reinterpret_cast<const __half *>(biases);
   pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
+  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
   tc::Maps mp;
   const int64_t row_bytes = K * bits / 8, sb_bytes = K / G * 2;
   if (!tc::encode_rows(&mp.w, packed, N, row_bytes, pl.a.pitch_w) ||
@@ -721,9 +748,9 @@ cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_
       !tc::encode_rows(&mp.b, biases, N, sb_bytes, pl.a.pitch_s))
     return cudaErrorInvalidValue;
   switch (bits) {
-    case 2: return tc::launch_g<2>(pl, mp, G, s);
-    case 4: return tc::launch_g<4>(pl, mp, G, s);
-    default: return tc::launch_g<8>(pl, mp, G, s);
+    case 2: return tc::launch_g<2>(pl, mp, G, overlap, s);
+    case 4: return tc::launch_g<4>(pl, mp, G, overlap, s);
+    default: return tc::launch_g<8>(pl, mp, G, overlap, s);
   }
 }
 
