@@ -69,7 +69,8 @@ constexpr int kRedBufs = 2;         // tiles whose chunk partials can be in flig
 constexpr int kMaxStages = 16;
 constexpr int kStageTarget = 16 * 1024;  // packed bytes of one stage we aim for (<= 1 KB per row)
 constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
-constexpr int kEarlyStages = 2;          // weight stages issued before the previous kernel completes (overlap mode)
+constexpr int kEarlyStages = 2;
+constexpr int kStageItems = 2;           // activation staging items per thread per round          // weight stages issued before the previous kernel completes (overlap mode)
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
 
 __host__ __device__ constexpr int pow2_tokens(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
@@ -298,70 +299,94 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   {
     mbar_wait(xbar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait);
     const int items = a.M * a.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
-    for (int i0 = 0; i0 < items; i0 += cthreads) {
-      const int i = i0 + ctid;
-      const bool act = i < items;
-      const int ii = act ? i : 0;
-      const int t = ii & 3, mg = ii >> 2;
-      const int m = mg / a.Gn, gg = mg - m * a.Gn;
-      const uint8_t *src = xs + m * a.tok_stride + (gg * G + Span::start(t)) * 2;
-      uint32_t raw[SL / 2];
+    // Each thread takes kStageItems items per round, processed side by side:
+    // the rounds are latency-bound chains (load, reduce across the quad, store).
+    constexpr int NI = kStageItems;
+    for (int i0 = 0; i0 < items; i0 += NI * cthreads) {
+      int tq[NI], mq[NI], gq[NI];
+      bool act[NI];
+      uint32_t raw[NI][SL / 2];
+      static_for<0, NI>([&](auto J) {
+        constexpr int j = J.value;
+        const int i = i0 + j * cthreads + ctid;
+        act[j] = i < items;
+        const int ii = act[j] ? i : 0;
+        tq[j] = ii & 3;
+        const int mg = ii >> 2;
+        mq[j] = mg / a.Gn;
+        gq[j] = mg - mq[j] * a.Gn;
+        const uint8_t *src = xs + mq[j] * a.tok_stride + (gq[j] * G + Span::start(tq[j])) * 2;
 #pragma unroll
-      for (int v = 0; v < SL / 8; ++v) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(src + 16 * v);
-        raw[4 * v] = q.x;
-        raw[4 * v + 1] = q.y;
-        raw[4 * v + 2] = q.z;
-        raw[4 * v + 3] = q.w;
-      }
-      float v8[U][8];  // [tile][4 * set + byte]
-      float amax = 0.0f, sx = 0.0f;
-      static_for<0, U>([&](auto C) {
-        static_for<0, 8>([&](auto S) {
-          constexpr int c = C.value, st = S.value >> 2, i = S.value & 3;
-          constexpr int e0 = Span::index(c, st, i, 0), e1 = Span::index(c, st, i, 1);
-          const uint32_t r0v = raw[e0 >> 1] >> ((e0 & 1) * 16), r1v = raw[e1 >> 1] >> ((e1 & 1) * 16);
-          const uint32_t bits16 = (e0 == e1 || !(t & 1)) ? r0v : r1v;
-          const float v = bf16_bits_to_float(bits16 & 0xFFFFu);
-          v8[c][S.value] = v;
-          amax = fmaxf(amax, fabsf(v));
-          sx += v;
+        for (int v = 0; v < SL / 8; ++v) {
+          const uint4 q = *reinterpret_cast<const uint4 *>(src + 16 * v);
+          raw[j][4 * v] = q.x;
+          raw[j][4 * v + 1] = q.y;
+          raw[j][4 * v + 2] = q.z;
+          raw[j][4 * v + 3] = q.w;
+        }
+      });
+      float v8[NI][U][8];  // [item][tile][4 * set + byte]
+      float amax[NI], sx[NI];
+      static_for<0, NI>([&](auto J) {
+        constexpr int j = J.value;
+        amax[j] = 0.0f;
+        sx[j] = 0.0f;
+        static_for<0, U>([&](auto C) {
+          static_for<0, 8>([&](auto S) {
+            constexpr int c = C.value, st = S.value >> 2, i = S.value & 3;
+            constexpr int e0 = Span::index(c, st, i, 0), e1 = Span::index(c, st, i, 1);
+            const uint32_t r0v = raw[j][e0 >> 1] >> ((e0 & 1) * 16), r1v = raw[j][e1 >> 1] >> ((e1 & 1) * 16);
+            const uint32_t bits16 = (e0 == e1 || !(tq[j] & 1)) ? r0v : r1v;
+            const float v = bf16_bits_to_float(bits16 & 0xFFFFu);
+            v8[j][c][S.value] = v;
+            amax[j] = fmaxf(amax[j], fabsf(v));
+            sx[j] += v;
+          });
         });
       });
       __syncwarp();  // every lane of the warp has read its raw values
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      sx += __shfl_xor_sync(0xffffffffu, sx, 1);
-      sx += __shfl_xor_sync(0xffffffffu, sx, 2);
-      // power of two 2^e with max|x| * 2^e in [2^13, 2^14) (e clamped to normal fp32 powers)
-      int e = 0;
-      if (amax > 0.0f) {
-        const int be = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
-        e = min(max(13 - (be == 0 ? -127 : be - 127), -126), 126);
-      }
-      // 2^-e as 2^-e_lo * 2^-e_hi: the fold applies one half to the integer dot
-      // product and the other to the scale, so neither product leaves fp32 range
-      const int e_hi = e >> 1, e_lo = e - e_hi;
-      const float inv_lo = __uint_as_float(static_cast<uint32_t>(127 - e_lo) << 23);
-      const float inv_hi = __uint_as_float(static_cast<uint32_t>(127 - e_hi) << 23);
-      const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-      uint8_t *dst = xs + m * a.tok_stride + (gg * U) * 64 + t * 16;
-      static_for<0, U>([&](auto C) {
-        constexpr int c = C.value;
-        uint32_t lo[2], hi[2];
-        static_for<0, 2>([&](auto S) {
-          // rint(v * 2^e) lands in the low 22 bits of v * 2^e + 1.5 * 2^23; its
-          // bytes 0 and 1 are the two's-complement digits lo and hi
-          uint32_t f[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) f[i] = __float_as_uint(fmaf(v8[c][4 * S.value + i], sc, kRoundMagic));
-          const uint32_t t01 = __byte_perm(f[0], f[1], 0x5140), t23 = __byte_perm(f[2], f[3], 0x5140);
-          lo[S.value] = __byte_perm(t01, t23, 0x5410);
-          hi[S.value] = __byte_perm(t01, t23, 0x7632);
-        });
-        if (act) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(lo[0], lo[1], hi[0], hi[1]);
+      static_for<0, NI>([&](auto J) {
+        constexpr int j = J.value;
+        amax[j] = fmaxf(amax[j], __shfl_xor_sync(0xffffffffu, amax[j], 1));
+        sx[j] += __shfl_xor_sync(0xffffffffu, sx[j], 1);
       });
-      if (act && t == 0) tab[m * a.Gn + gg] = make_float4(sx, inv_lo, inv_hi, 0.0f);
+      static_for<0, NI>([&](auto J) {
+        constexpr int j = J.value;
+        amax[j] = fmaxf(amax[j], __shfl_xor_sync(0xffffffffu, amax[j], 2));
+        sx[j] += __shfl_xor_sync(0xffffffffu, sx[j], 2);
+      });
+      static_for<0, NI>([&](auto J) {
+        constexpr int j = J.value;
+        // power of two 2^e with max|x| * 2^e in [2^13, 2^14) (e clamped to normal fp32 powers)
+        int e = 0;
+        if (amax[j] > 0.0f) {
+          const int be = static_cast<int>((__float_as_uint(amax[j]) >> 23) & 0xFFu);
+          e = min(max(13 - (be == 0 ? -127 : be - 127), -126), 126);
+        }
+        // 2^-e as 2^-e_lo * 2^-e_hi: the fold applies one half to the integer dot
+        // product and the other to the scale, so neither product leaves fp32 range
+        const int e_hi = e >> 1, e_lo = e - e_hi;
+        const float inv_lo = __uint_as_float(static_cast<uint32_t>(127 - e_lo) << 23);
+        const float inv_hi = __uint_as_float(static_cast<uint32_t>(127 - e_hi) << 23);
+        const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+        uint8_t *dst = xs + mq[j] * a.tok_stride + (gq[j] * U) * 64 + tq[j] * 16;
+        static_for<0, U>([&](auto C) {
+          constexpr int c = C.value;
+          uint32_t lo[2], hi[2];
+          static_for<0, 2>([&](auto S) {
+            // rint(v * 2^e) lands in the low 22 bits of v * 2^e + 1.5 * 2^23; its
+            // bytes 0 and 1 are the two's-complement digits lo and hi
+            uint32_t f[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) f[i] = __float_as_uint(fmaf(v8[j][c][4 * S.value + i], sc, kRoundMagic));
+            const uint32_t t01 = __byte_perm(f[0], f[1], 0x5140), t23 = __byte_perm(f[2], f[3], 0x5140);
+            lo[S.value] = __byte_perm(t01, t23, 0x5410);
+            hi[S.value] = __byte_perm(t01, t23, 0x7632);
+          });
+          if (act[j]) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(lo[0], lo[1], hi[0], hi[1]);
+        });
+        if (act[j] && tq[j] == 0) tab[mq[j] * a.Gn + gq[j]] = make_float4(sx[j], inv_lo, inv_hi, 0.0f);
+      });
     }
     // zero blocks, and the table rows of padding tokens
     const int zbytes = a.zero_stride + U * 64;
