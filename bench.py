@@ -58,27 +58,28 @@ def read_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash():
-    """Hash of every CUDA source of the library (a recorded ncu figure is only
-    reported while the kernels it was taken on are unchanged)."""
+def kernel_source_hash(files=None):
+    """Hash of CUDA sources of the library (all of them, or the named files of
+    csrc/): a recorded ncu figure is only reported while the kernel it was taken
+    on is unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_only_group_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(f.encode())
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    names = sorted(files) if files else sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    for f in names:
+        h.update(f.encode())
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(name):
-    """DRAM bytes per unit for a kernel from a committed ncu summary, if the kernel
-    sources have not changed since it was taken (else None)."""
+    """DRAM bytes per unit for a kernel from a committed ncu summary, if the sources
+    that kernel is built from have not changed since it was taken (else None)."""
     p = os.path.join(ROOT, "profiles", "counters.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(name)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("sources")):
         return None
     return e.get("dram_bytes_per_unit")
 
