@@ -341,14 +341,33 @@ def timed_graph(torch, stream, fn, reps_inner, reps_outer):
 
 def measure_sections(args, aq, torch, dev, stream, peaks):
     out = {}
-    want = set(args.sections.split(",")) if args.sections != "all" else {"qmm", "curve", "sweep", "quant"}
+    want = set(args.sections.split(",")) if args.sections != "all" else {"qmm", "curve", "sweep", "quant", "embed"}
     if "qmm" in want:
         out.update(section_qmm(args, aq, torch, dev, stream, peaks))
     if "curve" in want:
         out.update(section_curve(args, aq, torch, dev, stream, peaks))
     if "sweep" in want or "quant" in want:
         out.update(section_sweep_quant(args, aq, torch, dev, stream, peaks, want))
+    if "embed" in want:
+        out.update(section_embedding(args, aq, torch, dev, stream, peaks))
     return out
+
+
+def section_embedding(args, aq, torch, dev, stream, peaks):
+    """Quantized embedding lookup: 4096 random ids into a Llama-3-size table
+    (V = 128256, D = 4096), 4-bit G = 32; bytes = rows read + bf16 rows written."""
+    V, D, g, bits, T = 128256, 4096, 32, 4, 4096
+    w = torch.randn((V, D), device=dev, dtype=torch.float32, generator=torch.Generator(device=dev).manual_seed(5)) * 0.02
+    p, s, b = aq.aq_quantize(w, g, bits)
+    del w
+    torch.cuda.empty_cache()
+    ids = torch.randint(0, V, (T,), device=dev, dtype=torch.int32, generator=torch.Generator(device=dev).manual_seed(6))
+    o = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    ms = timed_graph(torch, stream, lambda i: aq.aq_embedding(ids, p, s, b, D, g, bits, out=o), 1, 20)
+    nbytes = T * (D * bits // 8 + 4 * D // g) + T * D * 2
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"embedding": {"V": V, "D": D, "T": T, "bits": bits, "G": g, "us": round(ms * 1e3, 2),
+                          "GBps": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}}
 
 
 def section_qmm(args, aq, torch, dev, stream, peaks):
@@ -503,7 +522,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--qmm-reps", type=int, default=20)
     ap.add_argument("--sections", default="all",
-                    help="all | none | comma list of qmm,curve,sweep,quant (secondary measurements)")
+                    help="all | none | comma list of qmm,curve,sweep,quant,embed (secondary measurements)")
     ap.add_argument("--no-sections", dest="sections", action="store_const", const="none")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-steps", type=int, default=30)

@@ -187,9 +187,30 @@ const char *aq_status_string(aq_status status);
 /* The last CUDA error code seen by this library on the calling thread (0 if none). */
 int aq_last_cuda_error(void);
 
+/* Quantized embedding lookup: out[t, :] = bf16_rn(fp32_rn(code*scale + bias))
+ * of row ids[t] of the packed table [V, D] (the row aq_dequantize would give).
+ * ids: device int32 [T] (4-byte aligned); packed/scales/biases as produced by
+ * aq_quantize on a [V, D] table and out, device bf16 [T, D], 16-byte aligned.
+ * D % G == 0.  T, V, D <= 0 or a null pointer -> AQ_ERR_INVALID_ARG.  An id
+ * outside [0, V) gives a zero row and sets bit 5 (AQ_FAULT_BAD_INDEX) of the
+ * device fault word.
+ * Source: anllm "Tutorial 10: Quantization", section 6 "Quantized
+ * Embeddings"; ExecuTorch "MLX backend — Quantization" (quantized embedding
+ * layers, G = 32 or 128). */
+aq_status aq_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, const uint16_t *scales,
+                       const uint16_t *biases, int64_t V, int64_t D, int G, int bits, uint16_t *out_bf16,
+                       aq_stream_t stream);
+
+/* Bits of the device fault word. */
+enum {
+  AQ_FAULT_WAIT_MASK = 0x1Fu, /* bits 0-4: a kernel gave up a bounded wait and returned early */
+  AQ_FAULT_BAD_INDEX = 0x20u  /* an embedding id was outside [0, V) */
+};
+
 /* Reads and clears the device-side fault word of the current device: non-zero
  * when a kernel gave up a bounded wait (an mbarrier that never completed) and
- * returned early; its output is then invalid.  Synchronizes the device. */
+ * returned early, its output then invalid (bits 0-4), or when an embedding id
+ * was out of range (bit 5).  Synchronizes the device. */
 aq_status aq_device_fault(uint32_t *fault_word);
 
 #ifdef __cplusplus

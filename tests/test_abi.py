@@ -143,6 +143,19 @@ def test_matmul_ex_flags():
     assert L.aq_matmul_ex(A, 0, 64, A, A, A, 8, 64, 4, A, aq.AQ_MATMUL_OVERLAP_PREVIOUS, None) == aq.AQ_ERR_INVALID_ARG
 
 
+def test_embedding_validation():
+    L = aq.lib()
+    call = lambda ids=A, T=4, V=100, D=64, G=64, bits=4, out=A: L.aq_embedding(ids, T, A, A, A, V, D, G, bits, out, None)
+    assert call(T=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(V=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(D=96) == aq.AQ_ERR_INVALID_ARG          # D % G != 0
+    assert call(G=16) == aq.AQ_ERR_UNSUPPORTED
+    assert call(bits=6) == aq.AQ_ERR_UNSUPPORTED
+    assert call(ids=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(ids=A + 2) == aq.AQ_ERR_ALIGNMENT         # ids need 4-byte alignment
+    assert call(out=U) == aq.AQ_ERR_ALIGNMENT
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

@@ -254,6 +254,52 @@ def test_qmv_all_zero_codes_closed_form():
     _assert_close(y, y_cf, "zero codes")
 
 
+# ----------------------------------------------------------------------------- quantized embedding lookup
+
+@pytest.mark.parametrize("bits", (2, 3, 4, 8))
+@pytest.mark.parametrize("G", (32, 64, 128))
+def test_embedding_rows_bitexact(bits, G):
+    """Each output row equals, bit for bit, the oracle's dequantized table row
+    for its id (ids with repeats, the first and the last row)."""
+    V, D = 1000, 512
+    p_ref, s_ref, b_ref = quantized(V, D, 8100 + G, True, G, bits)
+    rng = np.random.default_rng(8200 + bits + G)
+    ids = np.concatenate([[0, V - 1, 7, 7], rng.integers(0, V, 60)]).astype(np.int32)
+    out = aq.aq_embedding(torch.from_numpy(ids).cuda(), *_to_gpu(p_ref, s_ref, b_ref), D, G, bits)
+    torch.cuda.synchronize()
+    ref = oracle.dequantize_bf16(p_ref, s_ref, b_ref, D, G, bits)[ids]
+    assert np.array_equal(_u16(out), ref)
+
+
+def test_embedding_full_vocabulary_shape():
+    """A Llama-3-size table slice (V = 32768, D = 4096, int4 G = 32 as on the
+    ExecuTorch page): 4096 random ids, bit-exact against the oracle rows."""
+    V, D, G, bits = 32768, 4096, 32, 4
+    w = synth.weights(V, D, 8300)
+    p, s, b = aq.aq_quantize(torch.from_numpy(w).cuda(), G, bits)
+    ids = np.random.default_rng(8301).integers(0, V, 4096).astype(np.int32)
+    out = aq.aq_embedding(torch.from_numpy(ids).cuda(), p, s, b, D, G, bits)
+    torch.cuda.synchronize()
+    p_ref, s_ref, b_ref = oracle.quantize(w[np.unique(ids)], G, bits)  # rows quantize independently
+    ref = oracle.dequantize_bf16(p_ref, s_ref, b_ref, D, G, bits)
+    pos = {r: i for i, r in enumerate(np.unique(ids))}
+    assert np.array_equal(_u16(out), ref[[pos[r] for r in ids]])
+
+
+def test_embedding_bad_id_zero_row_and_fault_bit():
+    V, D, G, bits = 64, 256, 64, 4
+    p_ref, s_ref, b_ref = quantized(V, D, 8400, False, G, bits)
+    ids = np.array([3, -1, V, 5], dtype=np.int32)
+    assert aq.aq_device_fault() == 0
+    out = aq.aq_embedding(torch.from_numpy(ids).cuda(), *_to_gpu(p_ref, s_ref, b_ref), D, G, bits)
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() == aq.AQ_FAULT_BAD_INDEX
+    o = _u16(out)
+    ref = oracle.dequantize_bf16(p_ref, s_ref, b_ref, D, G, bits)
+    assert np.array_equal(o[0], ref[3]) and np.array_equal(o[3], ref[5])
+    assert not o[1].any() and not o[2].any()
+
+
 # ----------------------------------------------------------------------------- QMM (prefill, tcgen05)
 
 @pytest.mark.parametrize("c", synth.WORKLOADS[4].cases, ids=lambda c: c.name)

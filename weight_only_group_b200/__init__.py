@@ -34,6 +34,7 @@ AQ_KERNEL_AUTO = 0
 AQ_KERNEL_QMV = 1
 AQ_KERNEL_QMM = 2
 AQ_MATMUL_OVERLAP_PREVIOUS = 1
+AQ_FAULT_BAD_INDEX = 0x20
 KERNELS = {"auto": AQ_KERNEL_AUTO, "qmv": AQ_KERNEL_QMV, "qmm": AQ_KERNEL_QMM}
 
 _lock = threading.Lock()
@@ -66,6 +67,7 @@ def lib() -> ctypes.CDLL:
             L.aq_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
             L.aq_matmul_with.argtypes = [i32, vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
             L.aq_matmul_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, ctypes.c_uint32, vp]
+            L.aq_embedding.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_matmul_ws.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, u64, vp]
             L.aq_matmul_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
             L.aq_matmul_workspace_bytes.restype = u64
@@ -180,6 +182,23 @@ def aq_dequantize_f32(packed, scales, biases, K: int, G: int, bits: int, out: to
         rc = lib().aq_dequantize_f32(packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, K, G, bits,
                                      out.data_ptr(), _stream(packed))
     _check(rc, "aq_dequantize_f32")
+    return out
+
+
+def aq_embedding(ids, packed, scales, biases, D: int, G: int, bits: int, out: torch.Tensor | None = None):
+    """-> bf16 [T, D]: the dequantized rows ids[t] of the packed table [V, D] (ids: int32 [T] on the device)."""
+    if not (isinstance(ids, torch.Tensor) and ids.is_cuda and ids.dtype == torch.int32 and ids.dim() == 1
+            and ids.is_contiguous()):
+        raise ValueError("ids must be a contiguous 1-D int32 CUDA tensor")
+    V = _qw(packed, scales, biases)
+    T = ids.shape[0]
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.bfloat16, device=packed.device)
+    _need(out, "out", (torch.bfloat16,))
+    with torch.cuda.device(packed.device):
+        rc = lib().aq_embedding(ids.data_ptr(), T, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), V, D, G,
+                                bits, out.data_ptr(), _stream(packed))
+    _check(rc, "aq_embedding")
     return out
 
 

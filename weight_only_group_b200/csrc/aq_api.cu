@@ -15,6 +15,10 @@ size_t qmv_required_smem(int64_t M, int64_t K);
 bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t read_and_clear_qmv_fault(uint32_t *word);
 cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word);
+cudaError_t read_and_clear_embed_fault(uint32_t *word);
+cudaError_t launch_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, const uint16_t *scales,
+                             const uint16_t *biases, int64_t V, int64_t D, int G, int bits, uint16_t *out,
+                             cudaStream_t s);
 cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s);
 size_t qmm_workspace_bytes(int64_t M, int64_t K);
@@ -229,6 +233,20 @@ aq_status aq_matmul_ex(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
   return aq_matmul_with(kernel, x, M, K, packed, scales, biases, N, G, bits, y, stream);
 }
 
+aq_status aq_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, const uint16_t *scales,
+                       const uint16_t *biases, int64_t V, int64_t D, int G, int bits, uint16_t *out,
+                       aq_stream_t stream) {
+  if (T <= 0 || V <= 0 || T >= (int64_t(1) << 31)) return AQ_ERR_INVALID_ARG;
+  aq_status st = check_shape(V, D, G, bits);
+  if (st != AQ_OK) return st;
+  if (!ids || !packed || !scales || !biases || !out) return AQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ids) & 3u) != 0 || !aligned16(packed) || !aligned16(scales) ||
+      !aligned16(biases) || !aligned16(out))
+    return AQ_ERR_ALIGNMENT;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_embedding(ids, T, packed, scales, biases, V, D, G, bits, out, stream));
+}
+
 aq_status aq_device_fault(uint32_t *fault_word) {
   if (!fault_word) return AQ_ERR_INVALID_ARG;
   uint32_t a = 0, b = 0, c = 0;
@@ -237,7 +255,10 @@ aq_status aq_device_fault(uint32_t *fault_word) {
   st = from_cuda(aq::read_and_clear_qmv_fault(&b));
   if (st != AQ_OK) return st;
   st = from_cuda(aq::read_and_clear_qmv_tc_fault(&c));
-  *fault_word = a | b | c;
+  if (st != AQ_OK) return st;
+  uint32_t d = 0;
+  st = from_cuda(aq::read_and_clear_embed_fault(&d));
+  *fault_word = a | b | c | d;
   return st;
 }
 

@@ -22,6 +22,7 @@ enum : uint32_t {
   kFaultDequantWait = 1u << 2,  // dequant warps gave up waiting for packed data / a free A stage
   kFaultEpilogueWait = 1u << 3, // epilogue gave up waiting for the accumulator
   kFaultQmvWait = 1u << 4,      // QMV gave up waiting for a weight stage
+  kFaultBadIndex = 1u << 5,     // an embedding id outside [0, V): that output row was zeroed
 };
 
 // Upper bound of any spin on an mbarrier, in SM clock cycles (~1 s at 2 GHz).

@@ -196,7 +196,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   constexpr int NWD = LaneWords<BITS, G>::count;
   constexpr int GBYTES = G * BITS / 8;           // packed bytes of one group row
   constexpr int SL = LaneSpan<BITS, G>::length;
-  constexpr int NACC = kAcc;
+  // accumulator chains per digit plane: a group folded on its own has only
+  // G/32 MMAs per plane, and summing chains would cost more than it hides
+  constexpr int NACC = GS == 1 ? 1 : kAcc;
   using Span = LaneSpan<BITS, G>;
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -419,7 +421,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     const uint8_t *sr0 = stg + a.s_off + g * a.pitch_s, *sr1 = sr0 + 8 * a.pitch_s;
     const uint8_t *br0 = stg + a.b_off + g * a.pitch_s, *br1 = br0 + 8 * a.pitch_s;
     const int gch0 = ch * gpc;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float2 accA = make_float2(0.0f, 0.0f), accB = make_float2(0.0f, 0.0f);  // rows g, g+8 x columns 2t, 2t+1
 
     for (int p = 0; p < nper; ++p) {
       int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
@@ -454,32 +456,38 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         }
         D[i] = static_cast<float>(hi * 256 + lo);
       }
-      // fold: D[0] = (row g, col 2t), D[1] = (row g, col 2t+1), D[2], D[3] = rows g+8
+      // fold: D[0] = (row g, col 2t), D[1] = (row g, col 2t+1), D[2], D[3] = rows g+8.
+      // The two columns of a row go through packed fp32x2 operations.
+      float2 s0, s1, b0, b1;  // scale and bias of (row g | g+8) for columns 2t, 2t+1
+      float4 T0, T1;          // (sum x, 2^-e_lo, 2^-e_hi, 0) of columns 2t, 2t+1
       if constexpr (GS >= 2) {
         const int gl = p * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
         const int mt = (2 * t) / GS;
-        const float2 s0 = __half22float2(*reinterpret_cast<const __half2 *>(sr0 + gl * 2));
-        const float2 s1 = __half22float2(*reinterpret_cast<const __half2 *>(sr1 + gl * 2));
-        const float2 b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
-        const float2 b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
-        const float4 T0 = tab[mt * a.Gn + gch0 + gl], T1 = tab[mt * a.Gn + gch0 + gl + 1];
-        acc[0] = fmaf(s0.x * T0.z, D[0] * T0.y, fmaf(b0.x, T0.x, acc[0]));
-        acc[1] = fmaf(s0.y * T1.z, D[1] * T1.y, fmaf(b0.y, T1.x, acc[1]));
-        acc[2] = fmaf(s1.x * T0.z, D[2] * T0.y, fmaf(b1.x, T0.x, acc[2]));
-        acc[3] = fmaf(s1.y * T1.z, D[3] * T1.y, fmaf(b1.y, T1.x, acc[3]));
+        s0 = __half22float2(*reinterpret_cast<const __half2 *>(sr0 + gl * 2));
+        s1 = __half22float2(*reinterpret_cast<const __half2 *>(sr1 + gl * 2));
+        b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
+        b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
+        T0 = tab[mt * a.Gn + gch0 + gl];
+        T1 = tab[mt * a.Gn + gch0 + gl + 1];
       } else {
-        const int gl = p;
-        const float s0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
-        const float s1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
-        const float b0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
-        const float b1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
-        const float4 T0 = tab[(2 * t) * a.Gn + gch0 + gl], T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
-        acc[0] = fmaf(s0 * T0.z, D[0] * T0.y, fmaf(b0, T0.x, acc[0]));
-        acc[1] = fmaf(s0 * T1.z, D[1] * T1.y, fmaf(b0, T1.x, acc[1]));
-        acc[2] = fmaf(s1 * T0.z, D[2] * T0.y, fmaf(b1, T0.x, acc[2]));
-        acc[3] = fmaf(s1 * T1.z, D[3] * T1.y, fmaf(b1, T1.x, acc[3]));
+        const int gl = p;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
+        const float sv0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
+        const float sv1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
+        const float bv0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
+        const float bv1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
+        s0 = make_float2(sv0, sv0);
+        s1 = make_float2(sv1, sv1);
+        b0 = make_float2(bv0, bv0);
+        b1 = make_float2(bv1, bv1);
+        T0 = tab[(2 * t) * a.Gn + gch0 + gl];
+        T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
       }
+      const float2 tx = make_float2(T0.x, T1.x), ty = make_float2(T0.y, T1.y), tz = make_float2(T0.z, T1.z);
+      // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x
+      accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), ffma2(b0, tx, accA));
+      accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), ffma2(b1, tx, accB));
     }
+    const float acc[4] = {accA.x, accA.y, accB.x, accB.y};
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
 
