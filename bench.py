@@ -341,7 +341,8 @@ def timed_graph(torch, stream, fn, reps_inner, reps_outer):
 
 def measure_sections(args, aq, torch, dev, stream, peaks):
     out = {}
-    want = set(args.sections.split(",")) if args.sections != "all" else {"qmm", "curve", "sweep", "quant", "embed"}
+    want = set(args.sections.split(",")) if args.sections != "all" else {"qmm", "curve", "sweep", "quant", "embed",
+                                                                         "gather"}
     if "qmm" in want:
         out.update(section_qmm(args, aq, torch, dev, stream, peaks))
     if "curve" in want:
@@ -350,7 +351,34 @@ def measure_sections(args, aq, torch, dev, stream, peaks):
         out.update(section_sweep_quant(args, aq, torch, dev, stream, peaks, want))
     if "embed" in want:
         out.update(section_embedding(args, aq, torch, dev, stream, peaks))
+    if "gather" in want:
+        out.update(section_gather(args, aq, torch, dev, stream, peaks))
     return out
+
+
+def section_gather(args, aq, torch, dev, stream, peaks):
+    """MoE gather matmul: eight experts of a 14336 x 4096 projection (4-bit G64, a
+    Mixtral-8x7B-size w1), tokens routed top-2; weight GB/s of the expert rows
+    read.  Consecutive calls route to different experts (the stack, 264 MB, is
+    larger than L2), as consecutive tokens of a decode would."""
+    E, N, K = 8, 14336, 4096
+    w = torch.randn((E * N, K), device=dev, dtype=torch.float32, generator=torch.Generator(device=dev).manual_seed(7)) * 0.02
+    p, s, b = aq.aq_quantize(w, G, BITS)
+    del w
+    torch.cuda.empty_cache()
+    gp, gs, gb = p.view(E, N, -1), s.view(E, N, -1), b.view(E, N, -1)
+    res = {}
+    for tokens in (1, 4):
+        T = 2 * tokens
+        routes = [torch.tensor([(2 * r + j) % E for j in range(T)], dtype=torch.int32, device=dev) for r in range(4)]
+        x = synth.activations(T, K, 17).to(dev)
+        y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_gather_matmul(x, routes[i % 4], gp, gs, gb, G, BITS, out=y), 16, 20)
+        wb = T * weight_bytes(K, N)
+        gbs = wb / (ms * 1e-3) / 1e9
+        res[f"tokens{tokens}_top2"] = {"rows": T, "us": round(ms * 1e3, 2), "weight_GBps": round(gbs, 1),
+                                       "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    return {"gather_qmv": {"E": E, "N": N, "K": K, "bits": BITS, "G": G, "points": res}}
 
 
 def section_embedding(args, aq, torch, dev, stream, peaks):
@@ -522,7 +550,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--qmm-reps", type=int, default=20)
     ap.add_argument("--sections", default="all",
-                    help="all | none | comma list of qmm,curve,sweep,quant,embed (secondary measurements)")
+                    help="all | none | comma list of qmm,curve,sweep,quant,embed,gather (secondary measurements)")
     ap.add_argument("--no-sections", dest="sections", action="store_const", const="none")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-steps", type=int, default=30)

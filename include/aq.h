@@ -201,16 +201,31 @@ aq_status aq_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, co
                        const uint16_t *biases, int64_t V, int64_t D, int G, int bits, uint16_t *out_bf16,
                        aq_stream_t stream);
 
+/* Gather matmul for mixture-of-experts layers: for each token t,
+ * y[t, :] = x[t, :] @ dequant(W[experts[t]])^T, where W holds E experts of
+ * shape [N, K] stacked along the rows (packed [E, N, K*bits/32], scales and
+ * biases [E, N, K/G], each expert as aq_quantize produces it).  experts is a
+ * device int32 [T] (4-byte aligned); x bf16 [T, K] and y bf16 [T, N] on the
+ * device.  Each token streams its expert's weights (tokens sharing an expert
+ * read it again).  Shapes: bits in {2, 4, 8}, K a multiple of 8*G, N >= 16
+ * (others -> AQ_ERR_UNSUPPORTED); E*N < 2^31.  An expert id outside [0, E)
+ * gives a zero output row and sets AQ_FAULT_BAD_INDEX in the device fault word.
+ * Accuracy as aq_matmul.  Source: metalworking "MLX Quantization", the kernel
+ * family list ("gather variants for MoE experts"). */
+aq_status aq_gather_matmul(const uint16_t *x_bf16, int64_t T, int64_t K, const uint32_t *packed,
+                           const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
+                           const int32_t *experts, uint16_t *y_bf16, aq_stream_t stream);
+
 /* Bits of the device fault word. */
 enum {
   AQ_FAULT_WAIT_MASK = 0x1Fu, /* bits 0-4: a kernel gave up a bounded wait and returned early */
-  AQ_FAULT_BAD_INDEX = 0x20u  /* an embedding id was outside [0, V) */
+  AQ_FAULT_BAD_INDEX = 0x20u  /* an embedding id or an expert id was out of range */
 };
 
 /* Reads and clears the device-side fault word of the current device: non-zero
  * when a kernel gave up a bounded wait (an mbarrier that never completed) and
  * returned early, its output then invalid (bits 0-4), or when an embedding id
- * was out of range (bit 5).  Synchronizes the device. */
+ * or an expert id was out of range (bit 5).  Synchronizes the device. */
 aq_status aq_device_fault(uint32_t *fault_word);
 
 #ifdef __cplusplus

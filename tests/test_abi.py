@@ -156,6 +156,22 @@ def test_embedding_validation():
     assert call(out=U) == aq.AQ_ERR_ALIGNMENT
 
 
+def test_gather_matmul_validation():
+    L = aq.lib()
+    def call(x=A, T=2, K=4096, E=8, N=1024, G=64, bits=4, experts=A, y=A):
+        return L.aq_gather_matmul(x, T, K, A, A, A, E, N, G, bits, experts, y, None)
+    assert call(T=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(E=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(K=4000) == aq.AQ_ERR_INVALID_ARG         # K % G != 0
+    assert call(experts=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(experts=A + 2) == aq.AQ_ERR_ALIGNMENT
+    assert call(y=U) == aq.AQ_ERR_ALIGNMENT
+    assert call(bits=3) == aq.AQ_ERR_UNSUPPORTED          # the gather path is the tensor-core QMV (2/4/8-bit)
+    assert call(K=4096 + 64) == aq.AQ_ERR_UNSUPPORTED     # K not a multiple of 8*G
+    assert call(N=8) == aq.AQ_ERR_UNSUPPORTED             # fewer than 16 rows
+    assert call(E=1 << 20, N=4096) == aq.AQ_ERR_INVALID_ARG  # E*N >= 2^31
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

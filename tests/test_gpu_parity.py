@@ -254,6 +254,65 @@ def test_qmv_all_zero_codes_closed_form():
     _assert_close(y, y_cf, "zero codes")
 
 
+# ----------------------------------------------------------------------------- gather matmul (MoE experts)
+
+def _stacked_experts(E, N, K, seed, G, bits):
+    """E experts quantized by the oracle, stacked as [E, N, ...] on the GPU."""
+    parts = [quantized(N, K, seed + e, True, G, bits) for e in range(E)]
+    gp = torch.from_numpy(np.stack([p.view(np.int32) for p, _, _ in parts])).cuda()
+    gs = torch.from_numpy(np.stack([s.view(np.float16) for _, s, _ in parts])).cuda()
+    gb = torch.from_numpy(np.stack([b.view(np.float16) for _, _, b in parts])).cuda()
+    return parts, (gp, gs, gb)
+
+
+@pytest.mark.parametrize("bits,G", [(4, 64), (2, 32), (8, 128), (4, 32)])
+def test_gather_matmul_matches_oracle_per_token(bits, G):
+    """Token t against expert experts[t] (repeats included), each row within
+    tolerance of the oracle's product with that expert."""
+    E, N, K = 4, 512, 8 * G * 3
+    parts, (gp, gs, gb) = _stacked_experts(E, N, K, 9100 + bits * 10 + G, G, bits)
+    experts = np.array([0, 3, 3, 1, 0, 2, 1], dtype=np.int32)
+    xb = activations_bits(len(experts), K, 9199)
+    y = aq.aq_gather_matmul(_x_gpu(xb), torch.from_numpy(experts).cuda(), gp, gs, gb, G, bits)
+    torch.cuda.synchronize()
+    for t, e in enumerate(experts):
+        p, s, b = parts[e]
+        y_ref = oracle.matmul(xb[t:t + 1], p, s, b, G, bits)
+        _assert_close(y[t:t + 1], y_ref, f"gather token {t} expert {e}")
+
+
+def test_gather_matmul_mixtral_like_top2():
+    """Eight experts of a 2048 x 4096 projection, two tokens routed top-2 (four
+    token-expert rows); equal, bit for bit, to aq_matmul on each selected expert."""
+    E, N, K, G, bits = 8, 2048, 4096, 64, 4
+    w = torch.from_numpy(synth.weights(E * N, K, 9300)).cuda()
+    p, s, b = aq.aq_quantize(w, G, bits)
+    del w
+    gp, gs, gb = p.view(E, N, -1), s.view(E, N, -1), b.view(E, N, -1)
+    experts = torch.tensor([5, 1, 7, 5], dtype=torch.int32, device="cuda")
+    x = _x_gpu(activations_bits(4, K, 9301))
+    y = aq.aq_gather_matmul(x, experts, gp, gs, gb, G, bits)
+    for t, e in enumerate(experts.tolist()):
+        ref = aq.aq_matmul(x[t:t + 1], gp[e], gs[e], gb[e], G, bits)
+        assert torch.equal(y[t:t + 1], ref)
+
+
+def test_gather_matmul_bad_expert_zero_row_and_fault_bit():
+    E, N, K, G, bits = 2, 256, 512, 64, 4
+    parts, (gp, gs, gb) = _stacked_experts(E, N, K, 9400, G, bits)
+    experts = torch.tensor([1, 2, -1, 0], dtype=torch.int32, device="cuda")
+    xb = activations_bits(4, K, 9401)
+    assert aq.aq_device_fault() == 0
+    y = aq.aq_gather_matmul(_x_gpu(xb), experts, gp, gs, gb, G, bits)
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() == aq.AQ_FAULT_BAD_INDEX
+    yf = y.float().cpu().numpy()
+    assert not yf[1].any() and not yf[2].any()
+    for t, e in ((0, 1), (3, 0)):
+        p, s, b = parts[e]
+        _assert_close(y[t:t + 1], oracle.matmul(xb[t:t + 1], p, s, b, G, bits), f"token {t}")
+
+
 # ----------------------------------------------------------------------------- quantized embedding lookup
 
 @pytest.mark.parametrize("bits", (2, 3, 4, 8))

@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
             L.aq_matmul_with.argtypes = [i32, vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
             L.aq_matmul_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, ctypes.c_uint32, vp]
             L.aq_embedding.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp]
+            L.aq_gather_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, vp]
             L.aq_matmul_ws.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, u64, vp]
             L.aq_matmul_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
             L.aq_matmul_workspace_bytes.restype = u64
@@ -199,6 +200,33 @@ def aq_embedding(ids, packed, scales, biases, D: int, G: int, bits: int, out: to
         rc = lib().aq_embedding(ids.data_ptr(), T, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), V, D, G,
                                 bits, out.data_ptr(), _stream(packed))
     _check(rc, "aq_embedding")
+    return out
+
+
+def aq_gather_matmul(x, experts, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None):
+    """y [T, N] bf16: row t = x[t] @ dequant(W[experts[t]])^T for E stacked experts.
+
+    packed [E, N, K*bits/32] int32, scales/biases [E, N, K/G] fp16 (or the same arrays
+    flattened to [E*N, ...] with E given by experts' range: pass 3-D arrays); experts
+    int32 [T] on the device."""
+    _need(x, "x", (torch.bfloat16,))
+    if packed.dim() != 3 or scales.dim() != 3 or biases.dim() != 3:
+        raise ValueError("packed, scales and biases must be [E, N, ...]")
+    if not (isinstance(experts, torch.Tensor) and experts.is_cuda and experts.dtype == torch.int32
+            and experts.dim() == 1 and experts.is_contiguous()):
+        raise ValueError("experts must be a contiguous 1-D int32 CUDA tensor")
+    E, N = packed.shape[0], packed.shape[1]
+    _qw(packed.reshape(E * N, -1), scales.reshape(E * N, -1), biases.reshape(E * N, -1))
+    T, K = x.shape
+    if experts.shape[0] != T:
+        raise ValueError("experts must have one entry per token")
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16,))
+    with torch.cuda.device(x.device):
+        rc = lib().aq_gather_matmul(x.data_ptr(), T, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), E, N,
+                                    G, bits, experts.data_ptr(), out.data_ptr(), _stream(x))
+    _check(rc, "aq_gather_matmul")
     return out
 
 

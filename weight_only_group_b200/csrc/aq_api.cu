@@ -16,6 +16,10 @@ bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t read_and_clear_qmv_fault(uint32_t *word);
 cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word);
 cudaError_t read_and_clear_embed_fault(uint32_t *word);
+bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
+cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                             const uint16_t *biases, int64_t E, int64_t N, int G, int bits, const int32_t *experts,
+                             uint16_t *y, cudaStream_t s);
 cudaError_t launch_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, const uint16_t *scales,
                              const uint16_t *biases, int64_t V, int64_t D, int G, int bits, uint16_t *out,
                              cudaStream_t s);
@@ -245,6 +249,22 @@ aq_status aq_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, co
     return AQ_ERR_ALIGNMENT;
   if ((st = check_device()) != AQ_OK) return st;
   return from_cuda(aq::launch_embedding(ids, T, packed, scales, biases, V, D, G, bits, out, stream));
+}
+
+aq_status aq_gather_matmul(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                           const uint16_t *biases, int64_t E, int64_t N, int G, int bits, const int32_t *experts,
+                           uint16_t *y, aq_stream_t stream) {
+  if (T <= 0 || E <= 0 || T >= (int64_t(1) << 31)) return AQ_ERR_INVALID_ARG;
+  aq_status st = check_shape(N, K, G, bits);
+  if (st != AQ_OK) return st;
+  if (E * N >= (int64_t(1) << 31)) return AQ_ERR_INVALID_ARG;
+  if (!x || !packed || !scales || !biases || !experts || !y) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(biases) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(experts) & 3u) != 0)
+    return AQ_ERR_ALIGNMENT;
+  if (!aq::qmv_tc_supported(1, N, K, G, bits)) return AQ_ERR_UNSUPPORTED;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_gather_tc(x, T, K, packed, scales, biases, E, N, G, bits, experts, y, stream));
 }
 
 aq_status aq_device_fault(uint32_t *fault_word) {

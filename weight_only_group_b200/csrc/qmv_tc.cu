@@ -185,6 +185,11 @@ struct Args {
   int tab_off, red_off, bar_off;
   int w_box_x, sb_box_x;     // TMA x coordinate step of one chunk (64-bit elements)
   int early_w;               // weight stages issued before the previous kernel has completed
+  // gather mode (cta_per_tok > 0): token t = blockIdx.x / cta_per_tok multiplies
+  // its x row by expert experts[t] of E stacked [N, K] weights (rows e*N.. of
+  // the [E*N, K] maps); each of its cta_per_tok CTAs owns a slice of the N rows
+  const int32_t *experts;
+  int E, cta_per_tok;
 };
 
 template <int BITS, int G, int MP>
@@ -218,8 +223,26 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   float *red = reinterpret_cast<float *>(smem + a.red_off);    // [kRedBufs][nch][16][MP]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * a.N / gridDim.x;
-  const int64_t r1 = static_cast<int64_t>(blockIdx.x + 1) * a.N / gridDim.x;
+  int64_t r0, r1, wrow0 = 0;  // rows [r0, r1) of this CTA; first row of its weight matrix in the maps
+  const __nv_bfloat16 *xg = a.x;
+  __nv_bfloat16 *yg = a.y;
+  if (a.cta_per_tok > 0) {
+    const int tk = blockIdx.x / a.cta_per_tok, sub = blockIdx.x - tk * a.cta_per_tok;
+    r0 = static_cast<int64_t>(sub) * a.N / a.cta_per_tok;
+    r1 = static_cast<int64_t>(sub + 1) * a.N / a.cta_per_tok;
+    xg = a.x + static_cast<int64_t>(tk) * a.K;
+    yg = a.y + static_cast<int64_t>(tk) * a.N;
+    const int e = __ldg(a.experts + tk);
+    if (e < 0 || e >= a.E) {  // bad expert id: zero rows and a fault bit, before anything is issued
+      for (int64_t r = r0 + threadIdx.x; r < r1; r += blockDim.x) yg[r] = __float2bfloat16_rn(0.0f);
+      if (threadIdx.x == 0 && sub == 0) atomicOr(&g_qmv_tc_fault, kFaultBadIndex);
+      return;
+    }
+    wrow0 = static_cast<int64_t>(e) * a.N;
+  } else {
+    r0 = static_cast<int64_t>(blockIdx.x) * a.N / gridDim.x;
+    r1 = static_cast<int64_t>(blockIdx.x + 1) * a.N / gridDim.x;
+  }
   const int tiles = static_cast<int>((r1 - r0 + kRows - 1) / kRows);
   const int nst = tiles * a.nch;
   const int gpc = a.Kc / G;  // groups per chunk
@@ -233,7 +256,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   auto issue = [&](int st) {
     const int s = st % a.NS;
     const int T = st / a.nch, ch = st - T * a.nch;
-    const int rb = static_cast<int>(tile_base(T));
+    const int rb = static_cast<int>(wrow0 + tile_base(T));
     uint8_t *dst = ring + static_cast<size_t>(s) * a.stage_bytes;
     mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRows * (a.pitch_w + 2 * a.pitch_s)));
     tma_load_2d(dst, &wmap, &full[s], ch * a.w_box_x, rb);
@@ -266,7 +289,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     if (lane == 0) mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * a.K * 2);
     __syncwarp();
     if (lane < a.M)
-      bulk_g2s(xs + lane * a.tok_stride, a.x + static_cast<int64_t>(lane) * a.K, static_cast<uint32_t>(a.K) * 2, xbar);
+      bulk_g2s(xs + lane * a.tok_stride, xg + static_cast<int64_t>(lane) * a.K, static_cast<uint32_t>(a.K) * 2, xbar);
     if (lane == 0)
       for (int st = early; st < min(nst, a.NS); ++st) issue(st);
   }
@@ -520,8 +543,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const int tok = (2 * t) / GS;
         if (direct) {
           if (tok < a.M) {
-            if (row_ok(g)) a.y[static_cast<int64_t>(tok) * a.N + rb + g] = __float2bfloat16_rn(v[0]);
-            if (row_ok(g + 8)) a.y[static_cast<int64_t>(tok) * a.N + rb + g + 8] = __float2bfloat16_rn(v[1]);
+            if (row_ok(g)) yg[static_cast<int64_t>(tok) * a.N + rb + g] = __float2bfloat16_rn(v[0]);
+            if (row_ok(g + 8)) yg[static_cast<int64_t>(tok) * a.N + rb + g + 8] = __float2bfloat16_rn(v[1]);
           }
         } else {
           dstv[g * MP + tok] = v[0];
@@ -532,7 +555,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int tok = 2 * t + (q & 1), row = g + 8 * (q >> 1);
-            if (tok < a.M && row_ok(row)) a.y[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(v[q]);
+            if (tok < a.M && row_ok(row)) yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(v[q]);
           }
         } else {
 #pragma unroll
@@ -562,7 +585,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const int row = idx / MP, tok = idx - row * MP;
         float sum = 0.0f;
         for (int c2 = 0; c2 < a.nch; ++c2) sum += rbuf[(static_cast<size_t>(c2) * kRows + row) * MP + tok];
-        if (tok < a.M && row_ok(row)) a.y[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(sum);
+        if (tok < a.M && row_ok(row)) yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(sum);
       }
       __syncwarp();
       if (lane == 0) {
@@ -615,6 +638,10 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
     if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= kStageTarget) u = c;
   const int64_t Kc = 8 * G * u, nch = K / Kc, gpc = Kc / G;
   Args &a = pl.a;
+  a.early_w = 0;
+  a.experts = nullptr;
+  a.E = 1;
+  a.cta_per_tok = 0;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
@@ -784,6 +811,45 @@ cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_
     case 2: return tc::launch_g<2>(pl, mp, G, overlap, s);
     case 4: return tc::launch_g<4>(pl, mp, G, overlap, s);
     default: return tc::launch_g<8>(pl, mp, G, overlap, s);
+  }
+}
+
+cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                             const uint16_t *biases, int64_t E, int64_t N, int G, int bits, const int32_t *experts,
+                             uint16_t *y, cudaStream_t s) {
+  static thread_local int cached_dev = -1, sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  tc::Plan pl;
+  if (!tc::make_plan(1, N, K, G, bits, sms, pl)) return cudaErrorInvalidValue;
+  // CTAs per token: the SMs shared out between the tokens, each CTA >= 16 rows
+  const int64_t per_tok = std::max<int64_t>(1, std::min<int64_t>(sms / std::max<int64_t>(T, 1), N / tc::kRows));
+  if (T * per_tok >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  pl.grid = static_cast<int>(T * per_tok);
+  pl.a.cta_per_tok = static_cast<int>(per_tok);
+  pl.a.experts = experts;
+  pl.a.E = static_cast<int>(E);
+  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.packed = packed;
+  pl.a.scales = reinterpret_cast<const __half *>(scales);
+  pl.a.biases = reinterpret_cast<const __half *>(biases);
+  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  pl.a.early_w = 0;
+  tc::Maps mp;
+  const int64_t row_bytes = K * bits / 8, sb_bytes = K / G * 2;
+  if (!tc::encode_rows(&mp.w, packed, E * N, row_bytes, pl.a.pitch_w) ||
+      !tc::encode_rows(&mp.s, scales, E * N, sb_bytes, pl.a.pitch_s) ||
+      !tc::encode_rows(&mp.b, biases, E * N, sb_bytes, pl.a.pitch_s))
+    return cudaErrorInvalidValue;
+  switch (bits) {
+    case 2: return tc::launch_g<2>(pl, mp, G, false, s);
+    case 4: return tc::launch_g<4>(pl, mp, G, false, s);
+    default: return tc::launch_g<8>(pl, mp, G, false, s);
   }
 }
 
