@@ -44,6 +44,7 @@ class Oracle:
         lib = ctypes.CDLL(lib_path)
         i64, i32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
         lib.oracle_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp]
+        lib.oracle_quantize_mse.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp]
         lib.oracle_unpack_codes.argtypes = [vp, i64, i64, i32, vp]
         lib.oracle_dequantize_f32.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp]
         lib.oracle_dequantize_bf16.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp]
@@ -70,6 +71,18 @@ class Oracle:
         scales = np.zeros((N, K // G), dtype=np.uint16)
         biases = np.zeros((N, K // G), dtype=np.uint16)
         _check(self.lib.oracle_quantize(_p(w), N, K, G, bits, _p(packed), _p(scales), _p(biases)), "quantize")
+        return packed, scales, biases
+
+    def quantize_mse(self, w: np.ndarray, G: int, bits: int):
+        """Range-search quantize: same outputs and format as ``quantize``; each
+        group's grid is the shrunk [min, max] of least squared error."""
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        N, K = w.shape
+        packed = np.zeros((N, K * bits // 32), dtype=np.uint32)
+        scales = np.zeros((N, K // G), dtype=np.uint16)
+        biases = np.zeros((N, K // G), dtype=np.uint16)
+        _check(self.lib.oracle_quantize_mse(_p(w), N, K, G, bits, _p(packed), _p(scales), _p(biases)),
+               "quantize_mse")
         return packed, scales, biases
 
     def unpack_codes(self, packed: np.ndarray, K: int, bits: int) -> np.ndarray:
@@ -171,6 +184,10 @@ def num_threads() -> int:
 
 def quantize(w, G, bits):
     return default().quantize(w, G, bits)
+
+
+def quantize_mse(w, G, bits):
+    return default().quantize_mse(w, G, bits)
 
 
 def unpack_codes(packed, K, bits):

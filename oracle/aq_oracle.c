@@ -22,6 +22,9 @@
  *    groups run along in_features, i.e. along K within one output row).
  *  - Same tutorial, section 5 "Quantized Matrix Multiply": y = x @ W^T, and the
  *    fused product equals dequantize-then-multiply.
+ *  - "mlx-gptq" page, section "How it works": the range search (--mse) that
+ *    shrinks a group's min-max range when clipping its extremes costs less
+ *    error than the coarser step (oracle_quantize_mse; readings beside it).
  *
  * Readings where the pages are silent (each is also listed in the design notes):
  *  - scale = (max - min) / (2^bits - 1) and bias = min, both computed in fp32
@@ -191,6 +194,44 @@ static uint32_t get_code(const uint32_t *row, int64_t k, int bits)
     return q;
 }
 
+/* Group extremes, with a zero extreme taken as +0.0 (-0.0 and +0.0 are the
+ * same number, and the sign of a zero min or max is not a property of the set
+ * of values). */
+static void group_min_max(const float *v, int G, float *mn_out, float *mx_out)
+{
+    float mn = v[0], mx = v[0];
+    for (int i = 1; i < G; i++) {
+        if (v[i] < mn) mn = v[i];
+        if (v[i] > mx) mx = v[i];
+    }
+    if (mn == 0.0f) mn = 0.0f;
+    if (mx == 0.0f) mx = 0.0f;
+    *mn_out = mn;
+    *mx_out = mx;
+}
+
+/* Stored fp16 scale and bias of the affine grid spanning [lo, hi]:
+ * scale = fp32(fp32(hi - lo) / qmax), bias = lo, each rounded to fp16. */
+static void grid_params(float lo, float hi, uint32_t qmax, uint16_t *s16, uint16_t *b16)
+{
+    float d = hi - lo;                 /* fp32 subtraction */
+    float s32 = d / (float)qmax;       /* fp32 IEEE division */
+    *s16 = f16_bits_from_double((double)s32);
+    *b16 = f16_bits_from_double((double)lo);
+}
+
+/* Code of one value against the stored grid (sf, bf): the nearest grid point,
+ * ties to even, clamped to [0, qmax]; a zero scale gives code 0. */
+static uint32_t grid_code(float w, float sf, float bf, uint32_t qmax)
+{
+    if (sf == 0.0f) return 0u;
+    float t = (w - bf) / sf;   /* fp32 sub, fp32 div */
+    float r = rintf(t);        /* ties to even */
+    if (r < 0.0f) r = 0.0f;
+    if (r > (float)qmax) r = (float)qmax;
+    return (uint32_t)r;
+}
+
 int oracle_quantize(const float *w, int64_t N, int64_t K, int G, int bits,
                     uint32_t *packed, uint16_t *scales, uint16_t *biases)
 {
@@ -204,34 +245,102 @@ int oracle_quantize(const float *w, int64_t N, int64_t K, int G, int bits,
         for (int64_t j = 0; j < P; j++) pr[j] = 0u;
         for (int64_t g = 0; g < Gn; g++) {
             /* group = G contiguous elements of row n along K */
-            float mn = wr[g * G], mx = wr[g * G];
-            for (int64_t i = 1; i < G; i++) {
-                float v = wr[g * G + i];
-                if (v < mn) mn = v;
-                if (v > mx) mx = v;
-            }
-            /* -0.0 and +0.0 are the same number: a zero extreme is taken as +0.0 */
-            if (mn == 0.0f) mn = 0.0f;
-            if (mx == 0.0f) mx = 0.0f;
-            float d = mx - mn;                 /* fp32 subtraction */
-            float s32 = d / (float)qmax;       /* fp32 IEEE division */
-            uint16_t s16 = f16_bits_from_double((double)s32);
-            uint16_t b16 = f16_bits_from_double((double)mn);
+            float mn, mx;
+            group_min_max(wr + g * G, G, &mn, &mx);
+            uint16_t s16, b16;
+            grid_params(mn, mx, qmax, &s16, &b16);
             scales[n * Gn + g] = s16;
             biases[n * Gn + g] = b16;
             float sf = (float)f16_value(s16), bf = (float)f16_value(b16);
-            for (int64_t i = 0; i < G; i++) {
-                int64_t k = g * G + i;
-                uint32_t q = 0;
-                if (sf != 0.0f) {
-                    float t = (wr[k] - bf) / sf;   /* fp32 sub, fp32 div */
-                    float r = rintf(t);            /* ties to even */
-                    if (r < 0.0f) r = 0.0f;
-                    if (r > (float)qmax) r = (float)qmax;
-                    q = (uint32_t)r;
+            for (int64_t i = 0; i < G; i++)
+                put_code(pr, g * G + i, bits, grid_code(wr[g * G + i], sf, bf, qmax));
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Range-search quantize: per group, the shrunk [min, max] of least error     */
+/* ------------------------------------------------------------------------ */
+
+/* "mlx-gptq" page, "How it works": the range search shrinks a group's min-max
+ * range whenever clipping its extremes costs less error than the coarser step
+ * of the full range costs the rest of the group.  The page gives neither the
+ * grid of candidate ranges nor the error's arithmetic; the readings taken:
+ *  - candidates i = 0 .. 31 with shrink factor p_i = 1 - i/32 (exact in fp32),
+ *    i.e. every factor k/32 from 32/32 down to 1/32;
+ *    candidate i spans [lo, hi] = [fp32(p_i * min), fp32(p_i * max)] (both
+ *    bounds move toward zero; a zero bound is +0.0).  Candidate 0 is the plain
+ *    min-max grid, so the search never does worse than round-to-nearest;
+ *  - each candidate's fp16 scale/bias and codes are those of the plain
+ *    quantizer for [lo, hi]; values outside the range clamp to code 0 or qmax
+ *    (the clipping);
+ *  - its error is the sum of squared errors e = fp32(w - fp32(q*scale16 + bias16))
+ *    over the group, in fp32: e*e rounded, summed from zero in element order
+ *    within each run of 32 elements, and the runs' sums added pairwise ((r0 + r1) + (r2 + r3) for 128);
+ *  - the candidate of least error wins; equal errors keep the smaller i (the
+ *    wider range). */
+#define MSE_CANDIDATES 32
+#define MSE_STEP_DENOM 32
+
+static float run_error(const float *v, float sf, float bf, uint32_t qmax)
+{
+    float acc = 0.0f;
+    for (int j = 0; j < 32; j++) {
+        uint32_t q = grid_code(v[j], sf, bf, qmax);
+        float deq = (float)((double)q * (double)sf + (double)bf); /* exact, rounded once */
+        float e = v[j] - deq;
+        float e2 = e * e;
+        acc = acc + e2;
+    }
+    return acc;
+}
+
+static float group_error(const float *v, int G, float sf, float bf, uint32_t qmax)
+{
+    if (G == 32) return run_error(v, sf, bf, qmax);
+    if (G == 64) return run_error(v, sf, bf, qmax) + run_error(v + 32, sf, bf, qmax);
+    float a = run_error(v, sf, bf, qmax) + run_error(v + 32, sf, bf, qmax);
+    float b = run_error(v + 64, sf, bf, qmax) + run_error(v + 96, sf, bf, qmax);
+    return a + b;
+}
+
+int oracle_quantize_mse(const float *w, int64_t N, int64_t K, int G, int bits,
+                        uint32_t *packed, uint16_t *scales, uint16_t *biases)
+{
+    if (!w || !packed || !scales || !biases || bad_shape(N, K, G, bits)) return ORACLE_BAD_ARG;
+    const int64_t P = row_words(K, bits), Gn = K / G;
+    const uint32_t qmax = (1u << bits) - 1u;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        const float *wr = w + n * K;
+        uint32_t *pr = packed + n * P;
+        for (int64_t j = 0; j < P; j++) pr[j] = 0u;
+        for (int64_t g = 0; g < Gn; g++) {
+            const float *v = wr + g * G;
+            float mn, mx;
+            group_min_max(v, G, &mn, &mx);
+            uint16_t best_s = 0, best_b = 0;
+            float best_err = 0.0f;
+            for (int i = 0; i < MSE_CANDIDATES; i++) {
+                float p = 1.0f - (float)i / (float)MSE_STEP_DENOM;   /* exact */
+                float lo = p * mn, hi = p * mx;                        /* fp32 products */
+                if (lo == 0.0f) lo = 0.0f;
+                if (hi == 0.0f) hi = 0.0f;
+                uint16_t s16, b16;
+                grid_params(lo, hi, qmax, &s16, &b16);
+                float err = group_error(v, G, (float)f16_value(s16), (float)f16_value(b16), qmax);
+                if (i == 0 || err < best_err) {
+                    best_err = err;
+                    best_s = s16;
+                    best_b = b16;
                 }
-                put_code(pr, k, bits, q);
             }
+            scales[n * Gn + g] = best_s;
+            biases[n * Gn + g] = best_b;
+            float sf = (float)f16_value(best_s), bf = (float)f16_value(best_b);
+            for (int64_t i = 0; i < G; i++)
+                put_code(pr, g * G + i, bits, grid_code(v[i], sf, bf, qmax));
         }
     }
     return ORACLE_OK;

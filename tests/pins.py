@@ -83,3 +83,76 @@ def affine_values_f64(codes: np.ndarray, scales16: np.ndarray, biases16: np.ndar
     s = np.repeat(scales16.view(np.float16).astype(np.float64), G, axis=-1)
     b = np.repeat(biases16.view(np.float16).astype(np.float64), G, axis=-1)
     return codes.astype(np.float64) * s + b
+
+
+MSE_CANDIDATES = 32          # shrink factors p_i = 1 - i/32, i = 0..31
+
+
+def mse_candidate_bounds(mn: np.ndarray, mx: np.ndarray):
+    """All candidate ranges of the range search ("mlx-gptq" page, "How it
+    works": shrink the min-max range when clipping costs less): candidate i
+    spans [fp32(p_i*min), fp32(p_i*max)] with p_i = 1 - i/32, zero bounds +0.0.
+    Returns (lo, hi), each [..., 32] float32."""
+    p = (1.0 - np.arange(MSE_CANDIDATES, dtype=np.float64) / 32.0).astype(np.float32)
+    lo = (mn[..., None].astype(np.float32) * p).astype(np.float32)
+    hi = (mx[..., None].astype(np.float32) * p).astype(np.float32)
+    lo = np.where(lo == 0, np.float32(0.0), lo).astype(np.float32)
+    hi = np.where(hi == 0, np.float32(0.0), hi).astype(np.float32)
+    return lo, hi
+
+
+def numpy_quantize_mse(w: np.ndarray, G: int, bits: int):
+    """Vectorised NumPy statement of the range-search quantizer (same reading
+    as the oracle, independent code).  For every group and candidate range the
+    plain grid (fp16 scale/bias from [lo, hi], clamped codes), the fp32 squared
+    error summed in element order within each run of 32 and the run sums added
+    pairwise; the first candidate of least error wins."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    qmax = (1 << bits) - 1
+    wg = w.reshape(N, K // G, G)
+    mn = wg.min(axis=-1)
+    mx = wg.max(axis=-1)
+    mn = np.where(mn == 0, np.float32(0.0), mn).astype(np.float32)
+    mx = np.where(mx == 0, np.float32(0.0), mx).astype(np.float32)
+    lo, hi = mse_candidate_bounds(mn, mx)                                  # [N, Gn, C]
+    s16 = ((hi - lo).astype(np.float32) / np.float32(qmax)).astype(np.float32).astype(np.float16)
+    b16 = lo.astype(np.float16)
+    sf = s16.astype(np.float32)[..., None]                                 # [N, Gn, C, 1]
+    bf = b16.astype(np.float32)[..., None]
+    v = wg[:, :, None, :]                                                  # [N, Gn, 1, G]
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        t = ((v - bf).astype(np.float32) / sf).astype(np.float32)
+        q = np.clip(np.rint(t), 0, qmax)
+        q = np.where(sf == 0, 0, q)
+        deq = (q.astype(np.float64) * sf.astype(np.float64) + bf.astype(np.float64)).astype(np.float32)
+        e = (v - deq).astype(np.float32)
+        e2 = (e * e).astype(np.float32)
+        runs = []
+        for r in range(G // 32):
+            acc = np.zeros(e2.shape[:-1], dtype=np.float32)
+            for j in range(32):
+                acc = (acc + e2[..., 32 * r + j]).astype(np.float32)
+            runs.append(acc)
+        while len(runs) > 1:
+            runs = [(runs[i] + runs[i + 1]).astype(np.float32) for i in range(0, len(runs), 2)]
+    err = runs[0]                                                          # [N, Gn, C]
+    best = np.zeros(err.shape[:-1], dtype=np.int64)
+    best_err = err[..., 0].copy()
+    for i in range(1, MSE_CANDIDATES):
+        take = err[..., i] < best_err
+        best = np.where(take, i, best)
+        best_err = np.where(take, err[..., i], best_err)
+    pick = lambda a: np.take_along_axis(a, best[..., None], axis=-1)[..., 0]
+    s_best, b_best = pick(s16), pick(b16)
+    qb = np.take_along_axis(q, best[..., None, None], axis=2)[:, :, 0, :].astype(np.uint32).reshape(N, K)
+    packed = bitwise_pack(qb, bits)
+    return packed, s_best.view(np.uint16), b_best.view(np.uint16), qb.astype(np.uint8), best
+
+
+def group_sq_error_f64(w: np.ndarray, codes: np.ndarray, scales16: np.ndarray, biases16: np.ndarray, G: int):
+    """Exact-ish (fp64) squared reconstruction error of every group, [N, K/G]."""
+    w = np.asarray(w, dtype=np.float64)
+    d = w - affine_values_f64(codes, scales16, biases16, G)
+    N, K = w.shape
+    return (d * d).reshape(N, K // G, G).sum(axis=-1)

@@ -5,7 +5,10 @@ hand-derived groups (tests/golden/hand_groups.json), storage figures printed on
 the pages (tests/golden/storage_arithmetic.json), the shift/mask unpack printed
 in anllm 'Tutorial 10: Quantization' section 3, an independent NumPy quantizer,
 IEEE conversions from NumPy/PyTorch, brute-force fp64 matmul, closed forms and
-invariants.  ``test_planted_mistakes_are_caught`` rebuilds the oracle with
+invariants; for the range-search quantizer, hand-derived groups
+(tests/golden/range_search_groups.json), an independent NumPy statement and a
+brute-force fp64 check that the chosen range has the least error of all
+candidates.  ``test_planted_mistakes_are_caught`` rebuilds the oracle with
 plausible mistakes planted in it and checks that the pins reject each one.
 """
 import json
@@ -20,8 +23,8 @@ import torch
 
 import oracle
 import synth
-from pins import (affine_values_f64, bitwise_pack, bitwise_unpack, numpy_quantize, page_pack,
-                  page_unpack)
+from pins import (affine_values_f64, bitwise_pack, bitwise_unpack, group_sq_error_f64, mse_candidate_bounds,
+                  numpy_quantize, numpy_quantize_mse, page_pack, page_unpack)
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 BITS = (2, 3, 4, 8)
@@ -30,6 +33,11 @@ GROUPS = (32, 64, 128)
 
 def _hand_groups():
     with open(os.path.join(GOLDEN, "hand_groups.json")) as f:
+        return json.load(f)["groups"]
+
+
+def _range_search_groups():
+    with open(os.path.join(GOLDEN, "range_search_groups.json")) as f:
         return json.load(f)["groups"]
 
 
@@ -231,6 +239,116 @@ def test_degenerate_groups_reconstruct_the_bias():
 
 
 # --------------------------------------------------------------------------
+# Range-search quantizer ("mlx-gptq" page, "How it works": --mse)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("g", _range_search_groups(), ids=lambda g: g["name"])
+def test_range_search_hand_group(g):
+    w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+    bits, G = g["bits"], g["G"]
+    packed, scales, biases = oracle.quantize_mse(w, G, bits)
+    assert scales[0, 0] == int(g["scale_f16"], 16), hex(scales[0, 0])
+    assert biases[0, 0] == int(g["bias_f16"], 16), hex(biases[0, 0])
+    assert [int(x) for x in packed[0]] == [int(x, 16) for x in g["packed"]]
+    assert oracle.unpack_codes(packed, G, bits)[0].tolist() == g["codes"]
+    _, s0, b0 = oracle.quantize(w, G, bits)
+    assert s0[0, 0] == int(g["plain_scale_f16"], 16) and b0[0, 0] == int(g["plain_bias_f16"], 16)
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("G", GROUPS)
+def test_range_search_matches_numpy(bits, G):
+    w = synth.weights(24, 1024, seed=300 + bits * G)
+    got = oracle.quantize_mse(w, G, bits)
+    want = numpy_quantize_mse(w, G, bits)
+    for a, b in zip(got, want[:3]):
+        assert np.array_equal(a, b)
+
+
+def _candidate_sets(w, G, bits):
+    """Every candidate's (scale16, bias16) bits and its codes, [N, Gn, C] / [N, Gn, C, G]."""
+    N, K = w.shape
+    qmax = (1 << bits) - 1
+    wg = w.reshape(N, K // G, G)
+    mn = np.where(wg.min(-1) == 0, np.float32(0), wg.min(-1)).astype(np.float32)
+    mx = np.where(wg.max(-1) == 0, np.float32(0), wg.max(-1)).astype(np.float32)
+    lo, hi = mse_candidate_bounds(mn, mx)
+    s16 = ((hi - lo) / np.float32(qmax)).astype(np.float32).astype(np.float16)
+    b16 = lo.astype(np.float16)
+    return s16, b16
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("G", GROUPS)
+def test_range_search_choice_has_least_error_of_all_candidates(bits, G):
+    """Brute force in fp64: the chosen grid is one of the candidates, its codes
+    are the nearest clamped codes on that grid, and no candidate reconstructs
+    the group with a smaller squared error (beyond fp32 summation rounding)."""
+    N, K = 12, 512
+    w = synth.weights(N, K, seed=500 + bits + G)
+    w[0, :G] = np.linspace(-1, 3, G, dtype=np.float32)          # a skewed group
+    w[1, :G] = 0.0                                               # an all-zero group
+    p, s, b = oracle.quantize_mse(w, G, bits)
+    codes = bitwise_unpack(p, K, bits)
+    s16, b16 = _candidate_sets(w, G, bits)
+    Gn, qmax = K // G, (1 << bits) - 1
+    chosen_err = group_sq_error_f64(w, codes, s, b, G)
+    for n in range(N):
+        for g in range(Gn):
+            cand = list(zip(s16[n, g].view(np.uint16).tolist(), b16[n, g].view(np.uint16).tolist()))
+            assert (int(s[n, g]), int(b[n, g])) in cand
+            v = w[n, g * G:(g + 1) * G].astype(np.float32)
+            best = np.inf
+            for cs, cb in cand:
+                sf = np.array([cs], np.uint16).view(np.float16).astype(np.float32)[0]
+                bf = np.array([cb], np.uint16).view(np.float16).astype(np.float32)[0]
+                if sf == 0:
+                    q = np.zeros(G)
+                else:
+                    q = np.clip(np.rint(((v - bf).astype(np.float32) / sf).astype(np.float32)), 0, qmax)
+                d = v.astype(np.float64) - (q * np.float64(sf) + np.float64(bf))
+                best = min(best, float((d * d).sum()))
+                if (cs, cb) == (int(s[n, g]), int(b[n, g])):
+                    assert np.array_equal(codes[n, g * G:(g + 1) * G], q.astype(np.uint8))
+            assert chosen_err[n, g] <= best * (1 + 2e-5) + 1e-30, (n, g, chosen_err[n, g], best)
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("G", GROUPS)
+def test_range_search_never_worse_than_round_to_nearest(bits, G):
+    w = synth.weights(32, 2048, seed=700 + bits * G)
+    pm, sm, bm = oracle.quantize_mse(w, G, bits)
+    p0, s0, b0 = oracle.quantize(w, G, bits)
+    em = group_sq_error_f64(w, bitwise_unpack(pm, 2048, bits), sm, bm, G)
+    e0 = group_sq_error_f64(w, bitwise_unpack(p0, 2048, bits), s0, b0, G)
+    assert (em <= e0 * (1 + 2e-5) + 1e-30).all()
+    if bits <= 3:
+        # with outliers in the weights, clipping pays off at 2 and 3 bits
+        assert em.sum() < 0.9 * e0.sum()
+
+
+def test_range_search_degenerate_groups_equal_plain_quantizer():
+    w = np.full((3, 128), 0.0123, dtype=np.float32)
+    w[1, :64] = -3.5
+    w[2] = 0.0
+    for bits in BITS:
+        a = oracle.quantize_mse(w, 64, bits)
+        b = oracle.quantize(w, 64, bits)
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
+
+def test_range_search_8bit_keeps_plain_grid_on_gaussian_weights():
+    """At 8 bits the step is so fine that clipping never pays on N(0, 0.02) weights."""
+    w = synth.weights(16, 1024, seed=71, outliers=False)
+    for G in GROUPS:
+        a = oracle.quantize_mse(w, G, 8)
+        b = oracle.quantize(w, G, 8)
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
+
+# --------------------------------------------------------------------------
 # Dequantize
 # --------------------------------------------------------------------------
 
@@ -333,13 +451,24 @@ MUTATIONS = {
     "bias_sign": ("return (double)q * f16_value(srow[k / G]) + f16_value(brow[k / G]);",
                   "return (double)q * f16_value(srow[k / G]) - f16_value(brow[k / G]);"),
     "ties_away": ("float r = rintf(t);", "float r = roundf(t);"),
-    "fp32_scale_for_codes": ("float t = (wr[k] - bf) / sf;", "float t = (wr[k] - mn) / s32;"),
+    "fp32_scale_for_codes": ("grid_code(wr[g * G + i], sf, bf, qmax)",
+                             "grid_code(wr[g * G + i], (mx - mn) / (float)qmax, mn, qmax)"),
     "msb_first_packing": ("if ((q >> t) & 1u) row[bit / 32] |= (1u << (bit % 32));",
                           "if ((q >> t) & 1u) row[bit / 32] |= (1u << (31 - bit % 32));"),
     "group_index_off_by_one": ("uint32_t q = get_code(prow, k, bits);\n    return (double)q * f16_value(srow[k / G])",
                                "uint32_t q = get_code(prow, k, bits);\n    return (double)q * f16_value(srow[(k + 1) / G])"),
     "transposed_x_index": ("const uint16_t *xr = x_bf16 + m * K;", "const uint16_t *xr = x_bf16 + (M - 1 - m) * K;"),
     "scale_divides_by_2pow_bits": ("float s32 = d / (float)qmax;", "float s32 = d / (float)(qmax + 1u);"),
+    "mse_keeps_largest_error": ("if (i == 0 || err < best_err)", "if (i == 0 || err > best_err)"),
+    "mse_ties_take_narrowest": ("if (i == 0 || err < best_err)", "if (i == 0 || err <= best_err)"),
+    "mse_shrinks_top_only": ("float lo = p * mn, hi = p * mx;", "float lo = mn, hi = p * mx;"),
+    "mse_error_without_clipping": ("uint32_t q = grid_code(v[j], sf, bf, qmax);",
+                                   "uint32_t q = grid_code(v[j], sf, bf, 255u);"),
+    "mse_error_against_unrounded_bias": ("group_error(v, G, (float)f16_value(s16), (float)f16_value(b16), qmax)",
+                                         "group_error(v, G, (float)f16_value(s16), lo, qmax)"),
+    "mse_grid_step_sixteenth": ("#define MSE_STEP_DENOM 32", "#define MSE_STEP_DENOM 16"),
+    "mse_last_run_dropped": ("return run_error(v, sf, bf, qmax) + run_error(v + 32, sf, bf, qmax);",
+                             "return run_error(v, sf, bf, qmax);"),
 }
 
 
@@ -369,6 +498,20 @@ def _pins_pass(o: "oracle.Oracle") -> bool:
             y = o.matmul(synth.bf16_bits(x), p, s, b, G, bits)
             if not np.allclose(y, y_ref, rtol=1e-12, atol=1e-12):
                 return False
+        for g in _range_search_groups():
+            w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+            p, s, b = o.quantize_mse(w, g["G"], g["bits"])
+            if s[0, 0] != int(g["scale_f16"], 16) or b[0, 0] != int(g["bias_f16"], 16):
+                return False
+            if [int(x) for x in p[0]] != [int(x, 16) for x in g["packed"]]:
+                return False
+        for bits in BITS:
+            for G in (32, 64):
+                w = synth.weights(8, 256, seed=61 + bits)
+                got = o.quantize_mse(w, G, bits)
+                want = numpy_quantize_mse(w, G, bits)
+                if not all(np.array_equal(a, b) for a, b in zip(got, want[:3])):
+                    return False
         return True
     except ValueError:
         return False
