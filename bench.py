@@ -482,6 +482,11 @@ def section_sweep_quant(args, aq, torch, dev, stream, peaks, want):
     out["dequantize_bf16"] = {"K": K, "N": N, "bits": BITS, "G": G, "ms": round(ms_d, 4),
                               "GBps": round(dbytes / (ms_d * 1e-3) / 1e9, 1),
                               "frac_hbm": round(dbytes / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    # ---- range-search quantize (32 candidate grids per group; ALU-bound, one-off)
+    ms_m = timed_graph(torch, stream, lambda i: aq.aq_quantize_mse(w, G, BITS), 1, 3)
+    out["quantize_mse"] = {"K": K, "N": N, "bits": BITS, "G": G, "candidates": 32, "ms": round(ms_m, 3),
+                           "Gweights_per_s": round(N * K / (ms_m * 1e-3) / 1e9, 2),
+                           "x_plain_quantize_time": round(ms_m / ms_q, 2)}
     return out
 
 

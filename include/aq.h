@@ -81,6 +81,26 @@ size_t aq_packed_bytes(int64_t N, int64_t K, int G, int bits);
 aq_status aq_quantize(const float *w, int64_t N, int64_t K, int G, int bits,
                       uint32_t *packed, uint16_t *scales, uint16_t *biases, aq_stream_t stream);
 
+/* Range-search quantize: the same outputs, format and arguments as aq_quantize,
+ * with each group's grid chosen by a search over shrunk ranges.
+ * Source: "mlx-gptq" page, section "How it works" (--mse: a group's min-max
+ * range is shrunk when clipping its extremes costs less error than the coarser
+ * step costs the rest of the group; the pages give no grid, so these readings):
+ *  - candidates p = k/32, k = 32 down to 1; candidate p spans
+ *    [lo, hi] = [fp32(p*min), fp32(p*max)] (a zero bound is +0.0) and gets the
+ *    plain grid of that range: scale16 = fp16(fp32(hi - lo)/(2^bits - 1)),
+ *    bias16 = fp16(lo), codes clamp(rint_even((w - bias16)/scale16)), so values
+ *    outside [lo, hi] are clipped to the end codes; p = 1 is aq_quantize's grid;
+ *  - a candidate's error is the fp32 sum of e*e, e = fp32(w - fp32(q*scale16 +
+ *    bias16)), summed from zero in element order within each run of 32
+ *    elements, the runs' sums then added pairwise ((r0+r1)+(r2+r3) for G=128);
+ *  - the least error wins; equal errors keep the larger p.
+ * The result is bit-exact with that definition.  The squared error of the
+ * chosen grid is never above aq_quantize's (up to fp32 summation rounding).
+ * Cost: 32 candidate grids per group, ALU-bound (one-off, offline). */
+aq_status aq_quantize_mse(const float *w, int64_t N, int64_t K, int G, int bits,
+                          uint32_t *packed, uint16_t *scales, uint16_t *biases, aq_stream_t stream);
+
 /* Dequantize to bf16: w_out[n,k] = bf16_rn(fp32_rn(code*scale + bias)) (a single
  * fp32 rounding of the exact value, then RNE to bf16).
  * Source: anllm "Tutorial 10: Quantization", sections 3 and 7 (dequantize, then

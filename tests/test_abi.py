@@ -6,6 +6,7 @@ by argument validation before any CUDA call is made, so they run on a machine
 without a GPU.
 """
 import ctypes
+import functools
 import json
 import os
 import re
@@ -102,11 +103,13 @@ A = 0x10000  # 16-byte aligned
 U = 0x10004  # misaligned
 
 
-def _q(w=A, N=4, K=64, G=64, bits=4, p=A, s=A, b=A):
-    return aq.lib().aq_quantize(w, N, K, G, bits, p, s, b, None)
+def _q(w=A, N=4, K=64, G=64, bits=4, p=A, s=A, b=A, fn="aq_quantize"):
+    return getattr(aq.lib(), fn)(w, N, K, G, bits, p, s, b, None)
 
 
-def test_quantize_validation():
+@pytest.mark.parametrize("fn", ("aq_quantize", "aq_quantize_mse"))
+def test_quantize_validation(fn):
+    _q = functools.partial(globals()["_q"], fn=fn)
     assert _q(bits=5) == aq.AQ_ERR_UNSUPPORTED
     assert _q(G=16) == aq.AQ_ERR_UNSUPPORTED
     assert _q(K=96) == aq.AQ_ERR_INVALID_ARG

@@ -118,6 +118,85 @@ def test_quantize_special_values():
             assert np.array_equal(d.cpu().numpy(), oracle.dequantize_f32(p_ref, s_ref, b_ref, 256, G, bits))
 
 
+# ----------------------------------------------------------------------------- range-search quantize
+
+def _gpu_quantize_mse(w: np.ndarray, G: int, bits: int):
+    p, s, b = aq.aq_quantize_mse(torch.from_numpy(w).cuda(), G, bits)
+    torch.cuda.synchronize()
+    return p, s, b
+
+
+MSE_CASES = [(256, 512, 0, True), (64, 4096, 21, True), (37, 1024, 22, False)] + \
+    [(N, K, seed, outl) for (N, K, seed, outl, _, _) in EDGE_QUANT]
+
+
+@pytest.mark.parametrize("N,K,seed,outl", MSE_CASES)
+@pytest.mark.parametrize("bits", (2, 3, 4, 8))
+@pytest.mark.parametrize("G", (32, 64, 128))
+def test_quantize_mse_bitexact(N, K, seed, outl, G, bits):
+    if K % G:
+        pytest.skip("K not a multiple of G")
+    w = weights(N, K, seed, outl)
+    p_ref, s_ref, b_ref = oracle.quantize_mse(w, G, bits)
+    p, s, b = _gpu_quantize_mse(w, G, bits)
+    assert np.array_equal(_u16(s), s_ref)
+    assert np.array_equal(_u16(b), b_ref)
+    assert np.array_equal(_u32(p), p_ref)
+
+
+def test_quantize_mse_golden_and_special_values():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "range_search_groups.json")) as f:
+        groups = json.load(f)["groups"]
+    for g in groups:
+        w = np.array([float(v) for v in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+        p, s, b = _gpu_quantize_mse(w, g["G"], g["bits"])
+        assert int(_u16(s)[0, 0]) == int(g["scale_f16"], 16), g["name"]
+        assert int(_u16(b)[0, 0]) == int(g["bias_f16"], 16), g["name"]
+        assert [int(x) for x in _u32(p)[0]] == [int(x, 16) for x in g["packed"]], g["name"]
+    rng = np.random.default_rng(3)
+    w = rng.normal(0, 0.02, (8, 256)).astype(np.float32)
+    w[0, :64] = 0.25
+    w[1, :64] = 0.0
+    w[1, 3] = -0.0
+    w[2, :64] = np.arange(64, dtype=np.float32) * 2.0 ** -24 / 4
+    w[3, :64] = rng.normal(0, 1e3, 64).astype(np.float32)
+    w[4, :] = -np.abs(w[4, :])
+    w[5, 64:128] = np.float32(-0.0)
+    w[5, 70] = 1.0
+    w[6, :128] = rng.standard_t(1.5, 128).astype(np.float32) * 0.01   # heavy tails: deep shrinks
+    for G in (32, 64, 128):
+        for bits in (2, 3, 4, 8):
+            p_ref, s_ref, b_ref = oracle.quantize_mse(w, G, bits)
+            p, s, b = _gpu_quantize_mse(w, G, bits)
+            assert np.array_equal(_u16(s), s_ref), (G, bits)
+            assert np.array_equal(_u16(b), b_ref), (G, bits)
+            assert np.array_equal(_u32(p), p_ref), (G, bits)
+
+
+@pytest.mark.parametrize("G,bits", [(64, 4), (128, 2), (32, 3)])
+def test_quantize_mse_full_size_sampled_rows(G, bits):
+    """Llama-3-8B up-projection shape (W[14336, 4096]): bit-exact with the oracle on
+    sampled rows, and per group never a larger squared error than round-to-nearest."""
+    N, K = 14336, 4096
+    w = weights(N, K, 1202, True)
+    wd = torch.from_numpy(w).cuda()
+    p, s, b = aq.aq_quantize_mse(wd, G, bits)
+    p0, s0, b0 = aq.aq_quantize(wd, G, bits)
+    torch.cuda.synchronize()
+    rows = sample_rows(N, 192, seed=G + bits)
+    p_ref, s_ref, b_ref = oracle.quantize_mse(np.ascontiguousarray(w[rows]), G, bits)
+    assert np.array_equal(_u16(s)[rows], s_ref)
+    assert np.array_equal(_u16(b)[rows], b_ref)
+    assert np.array_equal(_u32(p)[rows], p_ref)
+    err = lambda q, sc, bi: ((wd.double() - aq.aq_dequantize_f32(q, sc, bi, K, G, bits).double()) ** 2
+                             ).view(N, K // G, G).sum(-1)
+    e_mse, e_rtn = err(p, s, b), err(p0, s0, b0)
+    assert bool((e_mse <= e_rtn * (1 + 2e-5) + 1e-30).all())
+    assert float(e_mse.sum()) < float(e_rtn.sum())
+
+
 # ----------------------------------------------------------------------------- QMV (decode)
 
 def _matmul_case(M, K, N, bits, G, seed, kernel, outl=True, full=True, n_rows=48):

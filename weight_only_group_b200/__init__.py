@@ -8,8 +8,9 @@ library's CUDA kernels; there is no CPU or PyTorch fallback, and importing the
 binding fails loudly when the library has not been built
 (``python -m weight_only_group_b200.build``).
 
-Names mirror the C entry points: ``aq_quantize``, ``aq_dequantize``,
-``aq_dequantize_f32``, ``aq_matmul``, ``aq_matmul_with``, ``aq_dispatch``,
+Names mirror the C entry points: ``aq_quantize``, ``aq_quantize_mse``,
+``aq_dequantize``, ``aq_dequantize_f32``, ``aq_matmul``, ``aq_matmul_with``,
+``aq_matmul_ex``, ``aq_embedding``, ``aq_gather_matmul``, ``aq_dispatch``,
 ``aq_matmul_ws``, ``aq_matmul_workspace_bytes``, ``aq_packed_words``,
 ``aq_packed_bytes``, ``aq_status_string``, ``aq_device_fault``.
 """
@@ -62,6 +63,7 @@ def lib() -> ctypes.CDLL:
             L.aq_packed_bytes.argtypes = [i64, i64, i32, i32]
             L.aq_packed_bytes.restype = u64
             L.aq_quantize.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
+            L.aq_quantize_mse.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
             L.aq_dequantize.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_dequantize_f32.argtypes = [vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
@@ -78,8 +80,8 @@ def lib() -> ctypes.CDLL:
             L.aq_status_string.restype = ctypes.c_char_p
             L.aq_last_cuda_error.restype = i32
             L.aq_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
-            for f in ("aq_quantize", "aq_dequantize", "aq_dequantize_f32", "aq_matmul", "aq_matmul_with",
-                      "aq_matmul_ws", "aq_device_fault"):
+            for f in ("aq_quantize", "aq_quantize_mse", "aq_dequantize", "aq_dequantize_f32", "aq_matmul",
+                      "aq_matmul_with", "aq_matmul_ws", "aq_device_fault"):
                 getattr(L, f).restype = i32
             _lib = L
     return _lib
@@ -137,18 +139,28 @@ _WORD = (torch.int32, torch.uint32)
 _HALF = (torch.float16, torch.int16, torch.uint16)
 
 
-def aq_quantize(w: torch.Tensor, G: int, bits: int):
-    """w fp32 [N, K] on the GPU -> (packed int32 [N, K*bits/32], scales fp16 [N, K/G], biases fp16 [N, K/G])."""
+def _quantize(fn: str, w: torch.Tensor, G: int, bits: int):
     _need(w, "w", (torch.float32,))
     N, K = w.shape
     packed = torch.empty((N, K * bits // 32), dtype=torch.int32, device=w.device)
     scales = torch.empty((N, max(K // G, 1)), dtype=torch.float16, device=w.device)
     biases = torch.empty_like(scales)
     with torch.cuda.device(w.device):
-        rc = lib().aq_quantize(w.data_ptr(), N, K, G, bits, packed.data_ptr(), scales.data_ptr(),
-                               biases.data_ptr(), _stream(w))
-    _check(rc, "aq_quantize")
+        rc = getattr(lib(), fn)(w.data_ptr(), N, K, G, bits, packed.data_ptr(), scales.data_ptr(),
+                                biases.data_ptr(), _stream(w))
+    _check(rc, fn)
     return packed, scales, biases
+
+
+def aq_quantize(w: torch.Tensor, G: int, bits: int):
+    """w fp32 [N, K] on the GPU -> (packed int32 [N, K*bits/32], scales fp16 [N, K/G], biases fp16 [N, K/G])."""
+    return _quantize("aq_quantize", w, G, bits)
+
+
+def aq_quantize_mse(w: torch.Tensor, G: int, bits: int):
+    """Range-search quantize (same outputs as ``aq_quantize``): each group's grid is
+    the shrunk [p*min, p*max], p = k/32, of least squared reconstruction error."""
+    return _quantize("aq_quantize_mse", w, G, bits)
 
 
 def _qw(packed, scales, biases):

@@ -7,6 +7,8 @@
 namespace aq {
 cudaError_t launch_quantize(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed,
                             uint16_t *scales, uint16_t *biases, cudaStream_t s);
+cudaError_t launch_quantize_mse(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed,
+                                uint16_t *scales, uint16_t *biases, cudaStream_t s);
 cudaError_t launch_dequantize(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                               int64_t N, int64_t K, int G, int bits, void *out, bool bf16_out, cudaStream_t s);
 cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
@@ -119,6 +121,16 @@ aq_status aq_quantize(const float *w, int64_t N, int64_t K, int G, int bits, uin
   if (!aligned16(w) || !aligned16(packed) || !aligned16(scales) || !aligned16(biases)) return AQ_ERR_ALIGNMENT;
   if ((st = check_device()) != AQ_OK) return st;
   return from_cuda(aq::launch_quantize(w, N, K, G, bits, packed, scales, biases, stream));
+}
+
+aq_status aq_quantize_mse(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed,
+                          uint16_t *scales, uint16_t *biases, aq_stream_t stream) {
+  aq_status st = check_shape(N, K, G, bits);
+  if (st != AQ_OK) return st;
+  if (!w || !packed || !scales || !biases) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(packed) || !aligned16(scales) || !aligned16(biases)) return AQ_ERR_ALIGNMENT;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_quantize_mse(w, N, K, G, bits, packed, scales, biases, stream));
 }
 
 static aq_status dequantize_common(const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,

@@ -50,8 +50,39 @@ AQ_DEVICE void load_chunk(const uint32_t *src, uint32_t (&w)[BITS]) {
   }
 }
 
+// Squared reconstruction error of one thread's 32 values on the grid (sf, bf),
+// in fp32: e = v - fp32(q*sf + bf) (q*sf is exact, so the fma rounds once),
+// e*e rounded, summed from zero in element order.  Every step is an explicit
+// round-to-nearest intrinsic so that no contraction changes the sum.
+template <int BITS>
+AQ_DEVICE float run_sq_error(const float (&v)[32], float sf, float bf) {
+  constexpr float qmax = float((1 << BITS) - 1);
+  const bool zero_scale = (sf == 0.0f);
+  float acc = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float t = __fdiv_rn(__fsub_rn(v[j], bf), sf);
+    t = fminf(fmaxf(rintf(t), 0.0f), qmax);
+    const float q = zero_scale ? 0.0f : t;
+    const float e = __fsub_rn(v[j], __fmaf_rn(q, sf, bf));
+    acc = __fadd_rn(acc, __fmul_rn(e, e));
+  }
+  return acc;
+}
+
 // One thread per 32-code chunk.  CPG = chunks per group (G/32).
-template <int BITS, int CPG>
+//
+// MSE = true is the range search of the "mlx-gptq" page, section "How it
+// works" (--mse): a group's min-max range is shrunk when clipping its extremes
+// costs less error than the coarser step costs the rest of the group.  The
+// candidates are [p*min, p*max] for p = k/32, k = 32 down to 1 (both bounds
+// move toward zero; a zero bound is +0.0), each quantized like the plain grid;
+// a candidate's error is the fp32 sum of its runs' squared errors, the CPG
+// runs of a group added pairwise by the xor shuffles ((r0 + r1) + (r2 + r3):
+// fp32 addition is commutative, so every lane of the group holds the same
+// sum).  The least error wins; equal errors keep the wider range.  Every lane
+// of a group takes the same decision from the same numbers.
+template <int BITS, int CPG, bool MSE>
 __global__ void __launch_bounds__(256) quantize_kernel(const float *__restrict__ w, int64_t n_chunks,
                                                        uint32_t *__restrict__ packed,
                                                        __half *__restrict__ scales,
@@ -82,14 +113,34 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float *__restrict__
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
-  if (!active) return;
   // -0.0 and +0.0 are the same number: a zero extreme is taken as +0.0.
   if (mn == 0.0f) mn = 0.0f;
   if (mx == 0.0f) mx = 0.0f;
   constexpr float qmax = float((1 << BITS) - 1);
-  const float s32 = __fdiv_rn(__fsub_rn(mx, mn), qmax);
-  const __half s16 = __float2half_rn(s32);
-  const __half b16 = __float2half_rn(mn);
+  __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), qmax));
+  __half b16 = __float2half_rn(mn);
+  if constexpr (MSE) {
+    // Inactive lanes (a whole group past the end, since n_chunks is a multiple
+    // of CPG) run the search on zeros so that the shuffles stay full-warp.
+    float best = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+      const float p = __fsub_rn(1.0f, __int2float_rn(i) * 0.03125f);  // exact
+      float lo = __fmul_rn(p, mn), hi = __fmul_rn(p, mx);
+      if (lo == 0.0f) lo = 0.0f;
+      if (hi == 0.0f) hi = 0.0f;
+      const __half cs = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), qmax));
+      const __half cb = __float2half_rn(lo);
+      float err = run_sq_error<BITS>(v, __half2float(cs), __half2float(cb));
+#pragma unroll
+      for (int o = 1; o < CPG; o <<= 1) err = __fadd_rn(err, __shfl_xor_sync(0xffffffffu, err, o));
+      if (i == 0 || err < best) {
+        best = err;
+        s16 = cs;
+        b16 = cb;
+      }
+    }
+  }
+  if (!active) return;
   const float sf = __half2float(s16), bf = __half2float(b16);
   const bool zero_scale = (sf == 0.0f);
   uint32_t out[BITS];
@@ -147,7 +198,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint32_t *__restr
   }
 }
 
-template <int BITS>
+template <int BITS, bool MSE>
 static cudaError_t launch_quantize_bits(const float *w, int64_t N, int64_t K, int G, uint32_t *packed,
                                         uint16_t *scales, uint16_t *biases, cudaStream_t s) {
   const int64_t n_chunks = N * K / 32;
@@ -155,21 +206,32 @@ static cudaError_t launch_quantize_bits(const float *w, int64_t N, int64_t K, in
   __half *sc = reinterpret_cast<__half *>(scales);
   __half *bi = reinterpret_cast<__half *>(biases);
   switch (G) {
-    case 32: quantize_kernel<BITS, 1><<<grid, 256, 0, s>>>(w, n_chunks, packed, sc, bi); break;
-    case 64: quantize_kernel<BITS, 2><<<grid, 256, 0, s>>>(w, n_chunks, packed, sc, bi); break;
-    default: quantize_kernel<BITS, 4><<<grid, 256, 0, s>>>(w, n_chunks, packed, sc, bi); break;
+    case 32: quantize_kernel<BITS, 1, MSE><<<grid, 256, 0, s>>>(w, n_chunks, packed, sc, bi); break;
+    case 64: quantize_kernel<BITS, 2, MSE><<<grid, 256, 0, s>>>(w, n_chunks, packed, sc, bi); break;
+    default: quantize_kernel<BITS, 4, MSE><<<grid, 256, 0, s>>>(w, n_chunks, packed, sc, bi); break;
   }
   return cudaGetLastError();
 }
 
+template <bool MSE>
+static cudaError_t launch_quantize_mode(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed,
+                                        uint16_t *scales, uint16_t *biases, cudaStream_t s) {
+  switch (bits) {
+    case 2: return launch_quantize_bits<2, MSE>(w, N, K, G, packed, scales, biases, s);
+    case 3: return launch_quantize_bits<3, MSE>(w, N, K, G, packed, scales, biases, s);
+    case 4: return launch_quantize_bits<4, MSE>(w, N, K, G, packed, scales, biases, s);
+    default: return launch_quantize_bits<8, MSE>(w, N, K, G, packed, scales, biases, s);
+  }
+}
+
 cudaError_t launch_quantize(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed,
                             uint16_t *scales, uint16_t *biases, cudaStream_t s) {
-  switch (bits) {
-    case 2: return launch_quantize_bits<2>(w, N, K, G, packed, scales, biases, s);
-    case 3: return launch_quantize_bits<3>(w, N, K, G, packed, scales, biases, s);
-    case 4: return launch_quantize_bits<4>(w, N, K, G, packed, scales, biases, s);
-    default: return launch_quantize_bits<8>(w, N, K, G, packed, scales, biases, s);
-  }
+  return launch_quantize_mode<false>(w, N, K, G, bits, packed, scales, biases, s);
+}
+
+cudaError_t launch_quantize_mse(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed,
+                                uint16_t *scales, uint16_t *biases, cudaStream_t s) {
+  return launch_quantize_mode<true>(w, N, K, G, bits, packed, scales, biases, s);
 }
 
 template <int BITS, bool BF16>
