@@ -260,7 +260,8 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "traffic_unit": "DRAM bytes read + written per decode step (3 launches), from ncu",
                 "peak_source": peaks["source"], "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
-                "kernel": "qmv_tc_kernel<bits=4,G=64,MP=1> (mma.sync m16n8k16 on exact fp16 codes; 3 launches per step)",
+                "kernel": ("qmv_tc_kernel<bits=4,G=64,MP=1> (mma.sync m16n8k32: u8 codes x 16-bit fixed-point "
+                           "activation digits, int32 accumulate; 3 launches per step)"),
                 "algorithmic_bytes_per_step": STEP_BYTES}
     del graph
 
