@@ -51,6 +51,10 @@ class Oracle:
         lib.oracle_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp]
         lib.oracle_matmul_sampled.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32,
                                               vp, i64, vp, i64, vp]
+        lib.oracle_mxfp4_quantize.argtypes = [vp, i64, i64, vp, vp]
+        lib.oracle_mxfp4_dequantize_f32.argtypes = [vp, vp, i64, i64, vp]
+        lib.oracle_mxfp4_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp]
+        lib.oracle_mxfp4_matmul_sampled.argtypes = [vp, i64, i64, vp, vp, i64, vp, i64, vp, i64, vp]
         lib.oracle_f16_round.argtypes = [vp, i64, vp]
         lib.oracle_bf16_round.argtypes = [vp, i64, vp]
         lib.oracle_f16_to_double.argtypes = [vp, i64, vp]
@@ -133,6 +137,47 @@ class Oracle:
                                               _p(mi), len(mi), _p(ni), len(ni), _p(y)), "matmul_sampled")
         return y
 
+    # ---- mxfp4 (E2M1 codes, E8M0 exponent per 32 along K)
+    def mxfp4_quantize(self, w: np.ndarray):
+        """w fp32 [N, K] -> (packed uint32 [N, K/8], scales uint8 [N, K/32])."""
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        N, K = w.shape
+        packed = np.zeros((N, K // 8), dtype=np.uint32)
+        scales = np.zeros((N, K // 32), dtype=np.uint8)
+        _check(self.lib.oracle_mxfp4_quantize(_p(w), N, K, _p(packed), _p(scales)), "mxfp4_quantize")
+        return packed, scales
+
+    def mxfp4_dequantize_f32(self, packed, scales, K: int) -> np.ndarray:
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        N = packed.shape[0]
+        out = np.zeros((N, K), dtype=np.float32)
+        _check(self.lib.oracle_mxfp4_dequantize_f32(_p(packed), _p(scales), N, K, _p(out)), "mxfp4_dequantize_f32")
+        return out
+
+    def mxfp4_matmul(self, x_bf16_bits, packed, scales) -> np.ndarray:
+        x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        M, K = x.shape
+        N = packed.shape[0]
+        y = np.zeros((M, N), dtype=np.float64)
+        _check(self.lib.oracle_mxfp4_matmul(_p(x), M, K, _p(packed), _p(scales), N, _p(y)), "mxfp4_matmul")
+        return y
+
+    def mxfp4_matmul_sampled(self, x_bf16_bits, packed, scales, m_idx, n_idx) -> np.ndarray:
+        x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        mi = np.ascontiguousarray(m_idx, dtype=np.int64)
+        ni = np.ascontiguousarray(n_idx, dtype=np.int64)
+        M, K = x.shape
+        N = packed.shape[0]
+        y = np.zeros((len(mi), len(ni)), dtype=np.float64)
+        _check(self.lib.oracle_mxfp4_matmul_sampled(_p(x), M, K, _p(packed), _p(scales), N, _p(mi), len(mi),
+                                                    _p(ni), len(ni), _p(y)), "mxfp4_matmul_sampled")
+        return y
+
     def f16_round(self, a: np.ndarray) -> np.ndarray:
         a = np.ascontiguousarray(a, dtype=np.float32)
         out = np.zeros(a.shape, dtype=np.uint16)
@@ -208,6 +253,22 @@ def matmul(x_bf16_bits, packed, scales, biases, G, bits):
 
 def matmul_sampled(x_bf16_bits, packed, scales, biases, G, bits, m_idx, n_idx):
     return default().matmul_sampled(x_bf16_bits, packed, scales, biases, G, bits, m_idx, n_idx)
+
+
+def mxfp4_quantize(w):
+    return default().mxfp4_quantize(w)
+
+
+def mxfp4_dequantize_f32(packed, scales, K):
+    return default().mxfp4_dequantize_f32(packed, scales, K)
+
+
+def mxfp4_matmul(x_bf16_bits, packed, scales):
+    return default().mxfp4_matmul(x_bf16_bits, packed, scales)
+
+
+def mxfp4_matmul_sampled(x_bf16_bits, packed, scales, m_idx, n_idx):
+    return default().mxfp4_matmul_sampled(x_bf16_bits, packed, scales, m_idx, n_idx)
 
 
 def f16_round(a):

@@ -22,6 +22,9 @@
  *    groups run along in_features, i.e. along K within one output row).
  *  - Same tutorial, section 5 "Quantized Matrix Multiply": y = x @ W^T, and the
  *    fused product equals dequantize-then-multiply.
+ *  - "metalworking — MLX Quantization" (newer modes) and "Quantizing a Model
+ *    for MLX", section "Modes, bits and mixed recipes": the mxfp4 block-scaled
+ *    mode (oracle_mxfp4_*; encodings and readings beside them).
  *  - "mlx-gptq" page, section "How it works": the range search (--mse) that
  *    shrinks a group's min-max range when clipping its extremes costs less
  *    error than the coarser step (oracle_quantize_mse; readings beside it).
@@ -452,6 +455,136 @@ int oracle_matmul(const uint16_t *x_bf16, int64_t M, int64_t K,
 }
 
 /* Number of threads the parallel loops above use. */
+/* ------------------------------------------------------------------------ */
+/* mxfp4: block-scaled fp4 (E2M1 elements, one E8M0 exponent per 32)         */
+/* ------------------------------------------------------------------------ */
+
+/* "metalworking — MLX Quantization" (the paragraph on the newer modes) and
+ * "Quantizing a Model for MLX", section "Modes, bits and mixed recipes": mxfp4
+ * is a block-scaled float mode with groups of 32 and 4-bit elements, storing an
+ * exponent per group instead of a scale and a bias.  The pages do not spell out
+ * the encodings; the readings follow the OCP Microscaling (MX) v1.0 formats that
+ * the name refers to, restated here:
+ *  - element code c (4 bits): sign = bit 3, exponent e = bits 2..1, mantissa
+ *    m = bit 0; magnitude m/2 for e = 0, else 2^(e-1) * (1 + m/2), i.e. the
+ *    magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 for codes 0..7;
+ *  - scale byte s: X = 2^(s - 127) (s = 255 is NaN and never produced);
+ *  - quantize a group of 32 along K: amax = max |w|; shared exponent
+ *    floor(log2 amax) - 2 (2 = the largest E2M1 exponent), clamped to
+ *    [-127, 127]; s = shared + 127; an all-zero group gets s = 0;
+ *  - each element: the E2M1 magnitude nearest to |w| / X, ties to the even code
+ *    (mantissa bit 0), values above 6 saturating to 6; the sign bit is set only
+ *    for negative values whose magnitude code is not 0 (zero is +0);
+ *  - codes pack 8 to a uint32, LSB first (code k at bits 4k..4k+3 of the row);
+ *  - dequantized value X * e2m1(c), exact in fp32 and bf16. */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+static double e2m1_value(uint32_t c)
+{
+    double v = E2M1_MAG[c & 7u];
+    return (c & 8u) ? -v : v;
+}
+
+static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 127); }
+
+static int bad_mx_shape(int64_t N, int64_t K) { return N <= 0 || K <= 0 || K % 32 != 0; }
+
+int oracle_mxfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales)
+{
+    if (!w || !packed || !scales || bad_mx_shape(N, K)) return ORACLE_BAD_ARG;
+    const int64_t P = K / 8, Gn = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        const float *wr = w + n * K;
+        uint32_t *pr = packed + n * P;
+        for (int64_t j = 0; j < P; j++) pr[j] = 0u;
+        for (int64_t g = 0; g < Gn; g++) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; i++) {
+                double a = fabs((double)wr[g * 32 + i]);
+                if (a > amax) amax = a;
+            }
+            int shared = -127;
+            if (amax > 0.0) {
+                int ex;
+                frexp(amax, &ex);           /* amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1 */
+                shared = (ex - 1) - 2;
+                if (shared < -127) shared = -127;
+                if (shared > 127) shared = 127;
+            }
+            scales[n * Gn + g] = (uint8_t)(shared + 127);
+            for (int i = 0; i < 32; i++) {
+                const double v = (double)wr[g * 32 + i];
+                const double t = fabs(v) * ldexp(1.0, -shared);   /* exact */
+                uint32_t best = 0;
+                double best_d = fabs(t - E2M1_MAG[0]);
+                for (uint32_t c = 1; c < 8; c++) {
+                    const double d = fabs(t - E2M1_MAG[c]);
+                    /* nearer wins; on a tie the even code (mantissa bit 0) wins */
+                    if (d < best_d || (d == best_d && (c & 1u) == 0u && (best & 1u) == 1u)) {
+                        best = c;
+                        best_d = d;
+                    }
+                }
+                if (v < 0.0 && best != 0u) best |= 8u;
+                put_code(pr, g * 32 + i, 4, best);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+static double mx_value(const uint32_t *prow, const uint8_t *srow, int64_t k)
+{
+    return e8m0_value(srow[k / 32]) * e2m1_value(get_code(prow, k, 4));
+}
+
+int oracle_mxfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K, float *out)
+{
+    if (!packed || !scales || !out || bad_mx_shape(N, K)) return ORACLE_BAD_ARG;
+    const int64_t P = K / 8, Gn = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++)
+            out[n * K + k] = (float)mx_value(packed + n * P, scales + n * Gn, k);
+    return ORACLE_OK;
+}
+
+int oracle_mxfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
+                        const uint8_t *scales, int64_t N, double *y)
+{
+    if (!x_bf16 || !packed || !scales || !y || M <= 0 || bad_mx_shape(N, K)) return ORACLE_BAD_ARG;
+    const int64_t P = K / 8, Gn = K / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t m = 0; m < M; m++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += bf16_value(x_bf16[m * K + k]) * mx_value(packed + n * P, scales + n * Gn, k);
+            y[m * N + n] = acc;
+        }
+    return ORACLE_OK;
+}
+
+int oracle_mxfp4_matmul_sampled(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
+                                const uint8_t *scales, int64_t N, const int64_t *m_idx, int64_t nm,
+                                const int64_t *n_idx, int64_t nn, double *y)
+{
+    if (!x_bf16 || !packed || !scales || !m_idx || !n_idx || !y || M <= 0 || bad_mx_shape(N, K)) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < nm; i++) if (m_idx[i] < 0 || m_idx[i] >= M) return ORACLE_BAD_ARG;
+    for (int64_t j = 0; j < nn; j++) if (n_idx[j] < 0 || n_idx[j] >= N) return ORACLE_BAD_ARG;
+    const int64_t P = K / 8, Gn = K / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t j = 0; j < nn; j++)
+        for (int64_t i = 0; i < nm; i++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += bf16_value(x_bf16[m_idx[i] * K + k]) * mx_value(packed + n_idx[j] * P, scales + n_idx[j] * Gn, k);
+            y[i * nn + j] = acc;
+        }
+    return ORACLE_OK;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -156,3 +156,43 @@ def group_sq_error_f64(w: np.ndarray, codes: np.ndarray, scales16: np.ndarray, b
     d = w - affine_values_f64(codes, scales16, biases16, G)
     N, K = w.shape
     return (d * d).reshape(N, K // G, G).sum(axis=-1)
+
+
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0])
+
+
+def numpy_mxfp4_quantize(w: np.ndarray):
+    """Independent NumPy statement of the mxfp4 quantizer (E2M1 codes, one E8M0
+    exponent per 32 along K; OCP MX v1.0 encodings).  The shared exponent comes
+    from NumPy's frexp; each element is the nearest of the 16 signed E2M1 values
+    to w / X (a search over all codes, ties to the even code), with the sign bit
+    dropped on a zero magnitude."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    wg = w.reshape(N, K // 32, 32).astype(np.float64)
+    amax = np.abs(wg).max(axis=-1)
+    _, ex = np.frexp(amax)
+    shared = np.where(amax > 0, np.clip(ex - 1 - 2, -127, 127), -127)
+    scales = (shared + 127).astype(np.uint8)
+    t = wg * np.ldexp(1.0, -shared)[..., None]
+    d = np.abs(t[..., None] - E2M1_VALUES)                         # [N, Gn, 32, 16]
+    # nearest; among equal distances an even code replaces an odd one
+    codes = np.zeros(d.shape[:-1], dtype=np.int64)
+    best = d[..., 0].copy()
+    for c in range(1, 16):
+        dc = d[..., c]
+        better = (dc < best) | ((dc == best) & ((c & 1) == 0) & ((codes & 1) == 1))
+        codes = np.where(better, c, codes)
+        best = np.where(better, dc, best)
+    codes = np.where((codes & 7) == 0, 0, codes)                    # zero magnitude: +0
+    # a negative value's nearest signed value is the negative one; fix sign explicitly
+    mag = codes & 7
+    codes = np.where((t < 0) & (mag != 0), mag | 8, mag)
+    codes = codes.reshape(N, K).astype(np.uint32)
+    return bitwise_pack(codes, 4), scales, codes.astype(np.uint8)
+
+
+def mxfp4_values_f64(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """X * e2m1(code) in fp64, X = 2^(s - 127) repeated over each group of 32."""
+    X = np.repeat(np.ldexp(1.0, scales.astype(np.int64) - 127), 32, axis=-1)
+    return E2M1_VALUES[codes.astype(np.int64)] * X

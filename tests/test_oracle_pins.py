@@ -8,7 +8,9 @@ IEEE conversions from NumPy/PyTorch, brute-force fp64 matmul, closed forms and
 invariants; for the range-search quantizer, hand-derived groups
 (tests/golden/range_search_groups.json), an independent NumPy statement and a
 brute-force fp64 check that the chosen range has the least error of all
-candidates.  ``test_planted_mistakes_are_caught`` rebuilds the oracle with
+candidates; for mxfp4, hand-derived groups (tests/golden/mxfp4_groups.json), an
+independent NumPy quantizer, a brute-force nearest-code check and the
+shared-exponent invariant.  ``test_planted_mistakes_are_caught`` rebuilds the oracle with
 plausible mistakes planted in it and checks that the pins reject each one.
 """
 import json
@@ -23,8 +25,9 @@ import torch
 
 import oracle
 import synth
-from pins import (affine_values_f64, bitwise_pack, bitwise_unpack, group_sq_error_f64, mse_candidate_bounds,
-                  numpy_quantize, numpy_quantize_mse, page_pack, page_unpack)
+from pins import (E2M1_VALUES, affine_values_f64, bitwise_pack, bitwise_unpack, group_sq_error_f64,
+                  mse_candidate_bounds, mxfp4_values_f64, numpy_mxfp4_quantize, numpy_quantize, numpy_quantize_mse,
+                  page_pack, page_unpack)
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 BITS = (2, 3, 4, 8)
@@ -38,6 +41,11 @@ def _hand_groups():
 
 def _range_search_groups():
     with open(os.path.join(GOLDEN, "range_search_groups.json")) as f:
+        return json.load(f)["groups"]
+
+
+def _mxfp4_groups():
+    with open(os.path.join(GOLDEN, "mxfp4_groups.json")) as f:
         return json.load(f)["groups"]
 
 
@@ -349,6 +357,74 @@ def test_range_search_8bit_keeps_plain_grid_on_gaussian_weights():
 
 
 # --------------------------------------------------------------------------
+# mxfp4 (block-scaled fp4: E2M1 codes, one E8M0 exponent per 32 along K)
+# --------------------------------------------------------------------------
+
+def _mx_weights(N, K, seed):
+    w = synth.weights(N, K, seed=seed)
+    w[0, :32] = 0.0                                   # all-zero group
+    w[1, :32] = np.float32(3e-39)                     # subnormal fp32 magnitudes: exponent clamps at -127
+    w[2, 32:64] *= np.float32(1e30)                   # large magnitudes
+    w[3, :] = -np.abs(w[3, :])                        # an all-negative row
+    w[4, :32] = np.float32(7.0) * np.sign(w[4, :32])  # saturating values
+    return w
+
+
+@pytest.mark.parametrize("g", _mxfp4_groups(), ids=lambda g: g["name"])
+def test_mxfp4_hand_group(g):
+    w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+    p, s = oracle.mxfp4_quantize(w)
+    assert int(s[0, 0]) == g["scale_e8m0"]
+    assert [int(x) for x in p[0]] == [int(x, 16) for x in g["packed"]]
+    assert oracle.unpack_codes(p, 32, 4)[0].tolist() == g["codes"]
+    d = oracle.mxfp4_dequantize_f32(p, s, 32)
+    assert np.array_equal(d, mxfp4_values_f64(np.array([g["codes"]]), s).astype(np.float32))
+
+
+def test_mxfp4_matches_numpy():
+    for seed in (5, 6):
+        w = _mx_weights(32, 2048, seed)
+        p, s = oracle.mxfp4_quantize(w)
+        p2, s2, _ = numpy_mxfp4_quantize(w)
+        assert np.array_equal(p, p2) and np.array_equal(s, s2)
+
+
+def test_mxfp4_every_code_is_nearest_and_scale_invariant():
+    """Brute force over all 16 codes in fp64: no code reconstructs an element more
+    closely than the chosen one (saturation included), and the shared exponent
+    puts max|w| / X in [4, 8) wherever it is not clamped."""
+    w = _mx_weights(16, 512, 9)
+    p, s = oracle.mxfp4_quantize(w)
+    codes = oracle.unpack_codes(p, 512, 4)
+    X = np.repeat(np.ldexp(1.0, s.astype(np.int64) - 127), 32, axis=-1)
+    chosen = np.abs(w.astype(np.float64) - E2M1_VALUES[codes.astype(np.int64)] * X)
+    every = np.abs(w.astype(np.float64)[..., None] - E2M1_VALUES * X[..., None])
+    assert (chosen <= every.min(axis=-1)).all()
+    amax = np.abs(w.astype(np.float64)).reshape(16, 16, 32).max(axis=-1)
+    Xg = np.ldexp(1.0, s.astype(np.int64) - 127)
+    free = (amax > 0) & (s > 0)
+    r = amax[free] / Xg[free]
+    assert ((r >= 4.0) & (r < 8.0)).all()
+    assert (s[amax == 0] == 0).all()
+    # zero magnitudes never carry the sign bit
+    assert not ((codes == 8).any())
+
+
+def test_mxfp4_dequantize_and_matmul():
+    w = _mx_weights(8, 256, 11)
+    w[2, 32:64] /= np.float32(1e30)
+    p, s = oracle.mxfp4_quantize(w)
+    codes = bitwise_unpack(p, 256, 4)
+    exact = mxfp4_values_f64(codes, s)
+    assert np.array_equal(oracle.mxfp4_dequantize_f32(p, s, 256), exact.astype(np.float32))
+    x = synth.activations(3, 256, seed=12)
+    y = oracle.mxfp4_matmul(synth.bf16_bits(x), p, s)
+    assert np.allclose(y, x.to(torch.float64).numpy() @ exact.T, rtol=1e-12, atol=1e-12)
+    ys = oracle.mxfp4_matmul_sampled(synth.bf16_bits(x), p, s, [2, 0], [7, 1, 4])
+    assert np.array_equal(ys, y[[2, 0]][:, [7, 1, 4]])
+
+
+# --------------------------------------------------------------------------
 # Dequantize
 # --------------------------------------------------------------------------
 
@@ -469,6 +545,12 @@ MUTATIONS = {
     "mse_grid_step_sixteenth": ("#define MSE_STEP_DENOM 32", "#define MSE_STEP_DENOM 16"),
     "mse_last_run_dropped": ("return run_error(v, sf, bf, qmax) + run_error(v + 32, sf, bf, qmax);",
                              "return run_error(v, sf, bf, qmax);"),
+    "mx_ties_to_odd": ("(d == best_d && (c & 1u) == 0u && (best & 1u) == 1u)", "(d == best_d)"),
+    "mx_shared_exponent_off_by_one": ("shared = (ex - 1) - 2;", "shared = (ex - 1) - 3;"),
+    "mx_signed_zero_code": ("if (v < 0.0 && best != 0u) best |= 8u;", "if (v < 0.0) best |= 8u;"),
+    "mx_scale_bias_128": ("static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 127); }",
+                          "static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 128); }"),
+    "mx_magnitude_table_swapped": ("{0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0}", "{0.0, 0.5, 1.0, 1.5, 2.0, 4.0, 3.0, 6.0}"),
 }
 
 
@@ -512,6 +594,19 @@ def _pins_pass(o: "oracle.Oracle") -> bool:
                 want = numpy_quantize_mse(w, G, bits)
                 if not all(np.array_equal(a, b) for a, b in zip(got, want[:3])):
                     return False
+        for g in _mxfp4_groups():
+            w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+            p, s = o.mxfp4_quantize(w)
+            if int(s[0, 0]) != g["scale_e8m0"] or [int(x) for x in p[0]] != [int(x, 16) for x in g["packed"]]:
+                return False
+            if not np.array_equal(o.mxfp4_dequantize_f32(p, s, 32),
+                                  mxfp4_values_f64(np.array([g["codes"]]), s).astype(np.float32)):
+                return False
+        w = _mx_weights(8, 256, 13)
+        p, s = o.mxfp4_quantize(w)
+        p2, s2, _ = numpy_mxfp4_quantize(w)
+        if not (np.array_equal(p, p2) and np.array_equal(s, s2)):
+            return False
         return True
     except ValueError:
         return False
