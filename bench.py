@@ -343,7 +343,7 @@ def timed_graph(torch, stream, fn, reps_inner, reps_outer):
 def measure_sections(args, aq, torch, dev, stream, peaks):
     out = {}
     want = set(args.sections.split(",")) if args.sections != "all" else {"qmm", "curve", "sweep", "quant", "embed",
-                                                                         "gather"}
+                                                                         "gather", "mxfp4"}
     if "qmm" in want:
         out.update(section_qmm(args, aq, torch, dev, stream, peaks))
     if "curve" in want:
@@ -354,6 +354,8 @@ def measure_sections(args, aq, torch, dev, stream, peaks):
         out.update(section_embedding(args, aq, torch, dev, stream, peaks))
     if "gather" in want:
         out.update(section_gather(args, aq, torch, dev, stream, peaks))
+    if "mxfp4" in want:
+        out.update(section_mxfp4(args, aq, torch, dev, stream, peaks))
     return out
 
 
@@ -380,6 +382,35 @@ def section_gather(args, aq, torch, dev, stream, peaks):
         res[f"tokens{tokens}_top2"] = {"rows": T, "us": round(ms * 1e3, 2), "weight_GBps": round(gbs, 1),
                                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
     return {"gather_qmv": {"E": E, "N": N, "K": K, "bits": BITS, "G": G, "points": res}}
+
+
+def section_mxfp4(args, aq, torch, dev, stream, peaks):
+    """mxfp4 decode (M = 1) on the integer tensor cores: weight GB/s (codes + E8M0
+    scales, N*K/2 + N*K/32 bytes) over rotating resident copies, and the quantizer."""
+    out = {}
+    x_cache = {}
+    for (K, N) in ((4096, 14336), (14336, 4096), (8192, 28672)):
+        w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 6 + K % 7)).to(dev)
+        base = aq.aq_mxfp4_quantize(w)
+        if (K, N) == (8192, 28672):
+            ms_q = timed_graph(torch, stream, lambda i: aq.aq_mxfp4_quantize(w), 1, 10)
+            out["mxfp4_quantize"] = {"K": K, "N": N, "ms": round(ms_q, 4),
+                                     "GBps": round((N * K * 4 + N * K // 2 + N * K // 32) / (ms_q * 1e-3) / 1e9, 1)}
+        del w
+        wb = N * K // 2 + N * K // 32
+        copies = max(2, -(-2 * L2_BYTES // wb) + 1)
+        qs = [base] + [tuple(t.clone() for t in base) for _ in range(copies - 1)]
+        x = x_cache.setdefault(K, synth.activations(1, K, 17).to(dev))
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_mxfp4_matmul(x, *qs[i % copies], out=y, overlap_previous=True),
+                         copies * 4, 20)
+        gbs = wb / (ms * 1e-3) / 1e9
+        out[f"mxfp4_qmv_K{K}_N{N}"] = {"us": round(ms * 1e3, 3), "weight_GBps": round(gbs, 1),
+                                       "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                       "kernel": "qmv_tc_kernel<4,32,1,mxfp4> (mma.sync m16n8k32 s8 codes)"}
+        del qs, base
+        torch.cuda.empty_cache()
+    return out
 
 
 def section_embedding(args, aq, torch, dev, stream, peaks):

@@ -236,6 +236,53 @@ aq_status aq_gather_matmul(const uint16_t *x_bf16, int64_t T, int64_t K, const u
                            const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
                            const int32_t *experts, uint16_t *y_bf16, aq_stream_t stream);
 
+/* ---- mxfp4: block-scaled fp4 ------------------------------------------------
+ * Source: metalworking "MLX Quantization" (the newer block-scaled float modes:
+ * mxfp4 with groups of 32) and "Quantizing a Model for MLX", section "Modes,
+ * bits and mixed recipes" (mxfp4: 4 bits, groups of 32, an exponent per group
+ * rather than a scale and a bias).  The pages leave the encodings open; these
+ * follow the OCP Microscaling v1.0 formats:
+ *  - packed: uint32 [N, K/8], E2M1 code k of a row at bits 4k..4k+3 (LSB
+ *    first); code bit 3 = sign, bits 2..1 = exponent, bit 0 = mantissa, so codes
+ *    0..7 are the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6;
+ *  - scales: uint8 [N, K/32], E8M0: byte s means X = 2^(s - 127) (255 = NaN);
+ *  - w ~= X * e2m1(code), no bias.
+ * Quantize, per 32 consecutive weights of a row: shared exponent
+ * floor(log2 max|w|) - 2, clamped to [-127, 127], s = shared + 127 (an all-zero
+ * group: s = 0); each code is the E2M1 magnitude nearest to |w| / X, ties to the
+ * even code, saturating at 6, with the sign bit only on a non-zero magnitude.
+ * Results are bit-exact with that definition.  Dequantized values are exact in
+ * fp32 and bf16.  K must be a multiple of 32 (else AQ_ERR_INVALID_ARG); every
+ * pointer 16-byte aligned (AQ_ERR_ALIGNMENT).  Inputs must be finite. */
+
+/* Bytes of codes + scales: N*K/2 + N*K/32 (4.25 bits per weight); 0 if invalid. */
+size_t aq_mxfp4_packed_bytes(int64_t N, int64_t K);
+
+/* Quantize fp32 W[N, K] (device) into packed codes and E8M0 scales (device,
+ * caller-allocated). */
+aq_status aq_mxfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
+                            aq_stream_t stream);
+
+/* Dequantize to bf16 [N, K] (exact). */
+aq_status aq_mxfp4_dequantize(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K,
+                              uint16_t *w_out_bf16, aq_stream_t stream);
+
+/* Dequantize to fp32 [N, K] (exact). */
+aq_status aq_mxfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K,
+                                  float *w_out, aq_stream_t stream);
+
+/* y[M, N] = x[M, K] @ dequant(W)^T (bf16 in and out, device) for decode,
+ * M <= 8, on the integer tensor cores: each code becomes the signed byte
+ * 2 * e2m1(code), the activations enter as 16-bit fixed point per group (as in
+ * aq_matmul's decode kernel) and the fold applies X / 2.  Supported shapes:
+ * M <= 8, N >= 16, K a multiple of 512 (others -> AQ_ERR_UNSUPPORTED).  flags:
+ * 0 or AQ_MATMUL_OVERLAP_PREVIOUS, as for aq_matmul_ex.  Accuracy as aq_matmul,
+ * provided X / 2 times the activations' per-group power of two stays within
+ * the fp32 range (true unless both the weights' scale and the activations are
+ * within a few octaves of the fp32 limits). */
+aq_status aq_mxfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
+                          const uint8_t *scales, int64_t N, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
+
 /* Bits of the device fault word. */
 enum {
   AQ_FAULT_WAIT_MASK = 0x1Fu, /* bits 0-4: a kernel gave up a bounded wait and returned early */

@@ -194,3 +194,22 @@ def test_workspace_validation():
     assert L.aq_matmul_ws(A, 512, 4096, A, A, A, 64, 64, 4, A, None, 0, None) == aq.AQ_ERR_INVALID_ARG
     assert L.aq_matmul_ws(A, 512, 4096, A, A, A, 64, 64, 4, A, A, 16, None) == aq.AQ_ERR_INVALID_ARG
     assert L.aq_matmul_ws(A, 512, 4096, A, A, A, 64, 64, 4, A, U, 1 << 30, None) == aq.AQ_ERR_ALIGNMENT
+
+
+def test_mxfp4_validation():
+    L = aq.lib()
+    assert aq.aq_mxfp4_packed_bytes(4096, 4096) == 4096 * 4096 // 2 + 4096 * 4096 // 32
+    assert aq.aq_mxfp4_packed_bytes(4, 48) == 0
+    assert L.aq_mxfp4_quantize(A, 4, 48, A, A, None) == aq.AQ_ERR_INVALID_ARG      # K % 32
+    assert L.aq_mxfp4_quantize(A, 0, 64, A, A, None) == aq.AQ_ERR_INVALID_ARG
+    assert L.aq_mxfp4_quantize(0, 4, 64, A, A, None) == aq.AQ_ERR_INVALID_ARG
+    assert L.aq_mxfp4_quantize(U, 4, 64, A, A, None) == aq.AQ_ERR_ALIGNMENT
+    assert L.aq_mxfp4_dequantize(A, U, 4, 64, A, None) == aq.AQ_ERR_ALIGNMENT
+    assert L.aq_mxfp4_dequantize_f32(A, A, 4, 40, A, None) == aq.AQ_ERR_INVALID_ARG
+    mm = lambda M=1, K=512, N=16, flags=0, x=A: L.aq_mxfp4_matmul(x, M, K, A, A, N, A, flags, None)
+    assert mm(K=256) == aq.AQ_ERR_UNSUPPORTED          # the decode kernel needs K % 512 == 0
+    assert mm(M=9) == aq.AQ_ERR_UNSUPPORTED            # decode only
+    assert mm(N=8) == aq.AQ_ERR_UNSUPPORTED            # at least one 16-row tile
+    assert mm(flags=2) == aq.AQ_ERR_INVALID_ARG
+    assert mm(x=U) == aq.AQ_ERR_ALIGNMENT
+    assert mm(M=0) == aq.AQ_ERR_INVALID_ARG

@@ -197,6 +197,76 @@ def test_quantize_mse_full_size_sampled_rows(G, bits):
     assert float(e_mse.sum()) < float(e_rtn.sum())
 
 
+# ----------------------------------------------------------------------------- mxfp4 (block-scaled fp4)
+
+def _mx_special(N, K, seed):
+    w = weights(N, K, seed, True).copy()
+    w[0, :32] = 0.0
+    w[1 % N, 32:64] = np.float32(3e-39)
+    w[2 % N, :32] = np.float32(7.0)
+    w[3 % N, :] = -np.abs(w[3 % N, :])
+    w[4 % N, 64:96] = np.float32(1e30) * np.sign(w[4 % N, 64:96])
+    w[5 % N, :32] = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25] * 4, dtype=np.float32)
+    return w
+
+
+@pytest.mark.parametrize("N,K,seed", [(8, 128, 31), (37, 1024, 32), (256, 4096, 33), (1, 32, 34)])
+def test_mxfp4_quantize_dequantize_bitexact(N, K, seed):
+    w = _mx_special(N, K, seed) if N >= 6 else weights(N, K, seed, False)
+    p_ref, s_ref = oracle.mxfp4_quantize(w)
+    p, s = aq.aq_mxfp4_quantize(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_u32(p), p_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    f_ref = oracle.mxfp4_dequantize_f32(p_ref, s_ref, K)
+    f = aq.aq_mxfp4_dequantize(p, s, K, fp32=True)
+    assert np.array_equal(f.cpu().numpy().view(np.uint32), f_ref.view(np.uint32))
+    b = aq.aq_mxfp4_dequantize(p, s, K)
+    assert np.array_equal(_u16(b), oracle.bf16_round(f_ref))
+
+
+def _mx_gpu(w):
+    p_ref, s_ref = oracle.mxfp4_quantize(w)
+    return p_ref, s_ref, torch.from_numpy(p_ref.view(np.int32)).cuda(), torch.from_numpy(s_ref).cuda()
+
+
+@pytest.mark.parametrize("M", (1, 2, 3, 4, 5, 8))
+@pytest.mark.parametrize("K,N", [(512, 16), (1024, 100), (4096, 600), (2560, 2600)])
+def test_mxfp4_matmul_matches_oracle(M, K, N):
+    w = weights(N, K, 40 + K + N, True)
+    p_ref, s_ref, p, s = _mx_gpu(w)
+    xb = activations_bits(M, K, 41 + M)
+    y = aq.aq_mxfp4_matmul(_x_gpu(xb), p, s)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.mxfp4_matmul(xb, p_ref, s_ref), f"mxfp4 M={M} K={K} N={N}")
+
+
+def test_mxfp4_matmul_special_weights_and_overlap():
+    w = _mx_special(64, 1024, 45)
+    w[4, 64:96] /= np.float32(1e28)      # large but within the decode kernel's fp32 fold range
+    p_ref, s_ref, p, s = _mx_gpu(w)
+    xb = activations_bits(3, 1024, 46)
+    y_ref = oracle.mxfp4_matmul(xb, p_ref, s_ref)
+    y0 = aq.aq_mxfp4_matmul(_x_gpu(xb), p, s)
+    y1 = aq.aq_mxfp4_matmul(_x_gpu(xb), p, s, overlap_previous=True)
+    torch.cuda.synchronize()
+    _assert_close(y0, y_ref, "mxfp4 special weights")
+    assert torch.equal(y0, y1)
+
+
+@pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
+def test_mxfp4_matmul_llama_shapes_sampled(K, N):
+    w = weights(N, K, 1202 if N == 14336 else 1203, True)
+    p_ref, s_ref, p, s = _mx_gpu(w)
+    xb = activations_bits(1, K, 47)
+    y = aq.aq_mxfp4_matmul(_x_gpu(xb), p, s)
+    torch.cuda.synchronize()
+    cols = sample_rows(N, 400, seed=K)
+    y_ref = oracle.mxfp4_matmul_sampled(xb, p_ref, s_ref, [0], cols)
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    _assert_close(y[:, torch.from_numpy(cols).cuda()], y_ref, f"mxfp4 {K}x{N} sampled", rms=rms)
+
+
 # ----------------------------------------------------------------------------- QMV (decode)
 
 def _matmul_case(M, K, N, bits, G, seed, kernel, outl=True, full=True, n_rows=48):

@@ -10,7 +10,9 @@ binding fails loudly when the library has not been built
 
 Names mirror the C entry points: ``aq_quantize``, ``aq_quantize_mse``,
 ``aq_dequantize``, ``aq_dequantize_f32``, ``aq_matmul``, ``aq_matmul_with``,
-``aq_matmul_ex``, ``aq_embedding``, ``aq_gather_matmul``, ``aq_dispatch``,
+``aq_matmul_ex``, ``aq_embedding``, ``aq_gather_matmul``, ``aq_mxfp4_quantize``,
+``aq_mxfp4_dequantize``, ``aq_mxfp4_dequantize_f32``, ``aq_mxfp4_matmul``,
+``aq_mxfp4_packed_bytes``, ``aq_dispatch``,
 ``aq_matmul_ws``, ``aq_matmul_workspace_bytes``, ``aq_packed_words``,
 ``aq_packed_bytes``, ``aq_status_string``, ``aq_device_fault``.
 """
@@ -72,6 +74,12 @@ def lib() -> ctypes.CDLL:
             L.aq_embedding.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_gather_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, vp]
             L.aq_matmul_ws.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, u64, vp]
+            L.aq_mxfp4_packed_bytes.argtypes = [i64, i64]
+            L.aq_mxfp4_packed_bytes.restype = u64
+            L.aq_mxfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+            L.aq_mxfp4_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
+            L.aq_mxfp4_dequantize_f32.argtypes = [vp, vp, i64, i64, vp, vp]
+            L.aq_mxfp4_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, ctypes.c_uint32, vp]
             L.aq_matmul_workspace_bytes.argtypes = [i64, i64, i64, i32, i32]
             L.aq_matmul_workspace_bytes.restype = u64
             L.aq_dispatch.argtypes = [i64, i64, i64, i32, i32]
@@ -313,3 +321,62 @@ def aq_device_fault() -> int:
     w = ctypes.c_uint32(0)
     _check(lib().aq_device_fault(ctypes.byref(w)), "aq_device_fault")
     return int(w.value)
+
+
+# ----------------------------------------------------------------------------- mxfp4 (block-scaled fp4)
+
+_BYTE = (torch.uint8,)
+
+
+def aq_mxfp4_packed_bytes(N: int, K: int) -> int:
+    return int(lib().aq_mxfp4_packed_bytes(N, K))
+
+
+def _mx(packed, scales):
+    _need(packed, "packed", _WORD)
+    _need(scales, "scales", _BYTE)
+    if packed.shape[0] != scales.shape[0]:
+        raise ValueError("packed and scales disagree on N")
+    return packed.shape[0]
+
+
+def aq_mxfp4_quantize(w: torch.Tensor):
+    """w fp32 [N, K] on the GPU -> (packed int32 [N, K/8] of E2M1 codes, scales uint8 [N, K/32] E8M0)."""
+    _need(w, "w", (torch.float32,))
+    N, K = w.shape
+    packed = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+    scales = torch.empty((N, max(K // 32, 1)), dtype=torch.uint8, device=w.device)
+    with torch.cuda.device(w.device):
+        rc = lib().aq_mxfp4_quantize(w.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), _stream(w))
+    _check(rc, "aq_mxfp4_quantize")
+    return packed, scales
+
+
+def aq_mxfp4_dequantize(packed, scales, K: int, out: torch.Tensor | None = None, fp32: bool = False):
+    """-> bf16 (or fp32) [N, K] = X * e2m1(code), exact."""
+    N = _mx(packed, scales)
+    dt = torch.float32 if fp32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((N, K), dtype=dt, device=packed.device)
+    _need(out, "out", (dt,))
+    fn = "aq_mxfp4_dequantize_f32" if fp32 else "aq_mxfp4_dequantize"
+    with torch.cuda.device(packed.device):
+        rc = getattr(lib(), fn)(packed.data_ptr(), scales.data_ptr(), N, K, out.data_ptr(), _stream(packed))
+    _check(rc, fn)
+    return out
+
+
+def aq_mxfp4_matmul(x, packed, scales, out: torch.Tensor | None = None, overlap_previous: bool = False):
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for mxfp4 weights (decode, M <= 8)."""
+    _need(x, "x", (torch.bfloat16,))
+    N = _mx(packed, scales)
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16,))
+    flags = AQ_MATMUL_OVERLAP_PREVIOUS if overlap_previous else 0
+    with torch.cuda.device(x.device):
+        rc = lib().aq_mxfp4_matmul(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), N, out.data_ptr(), flags,
+                                   _stream(x))
+    _check(rc, "aq_mxfp4_matmul")
+    return out

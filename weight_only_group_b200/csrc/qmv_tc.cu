@@ -87,12 +87,14 @@ struct LaneWords {
 // A register set s (s = 0: MMA k 4t..4t+3, s = 1: k 16+4t..16+4t+3) of the
 // lane's K tile c (32 codes).  hh: the half of a shared word that a lane of a
 // 2-bit, G = 32 pair owns (t & 1).
-template <int BITS, int G>
+// FMT 1 (mxfp4, 4-bit, G = 32): register set s holds codes 4s..4s+3 of the lane's word.
+template <int BITS, int G, int FMT = 0>
 struct LaneSpan {
   static constexpr int length = (BITS == 2 && G == 32) ? 16 : G / 4;
   AQ_DEVICE static int start(int t) { return (BITS == 2 && G == 32) ? 16 * (t >> 1) : t * (G / 4); }
   __host__ __device__ static constexpr int index(int c, int s, int i, int hh) {
-    return BITS == 4   ? 8 * c + 2 * i + s
+    return FMT == 1    ? 8 * c + 4 * s + i
+           : BITS == 4 ? 8 * c + 2 * i + s
            : BITS == 8 ? 4 * (2 * c + s) + i
            : G >= 64   ? 16 * (c >> 1) + 2 * (c & 1) + s + 4 * i
                        : 2 * hh + s + 4 * i;
@@ -151,6 +153,43 @@ AQ_DEVICE void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// The same with signed A bytes (mxfp4 values).
+AQ_DEVICE void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+AQ_DEVICE void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// prmt.b32 in its default mode: result byte n is byte (c >> 4n) & 7 of {b, a},
+// or, when bit 4n+3 of c is set, that byte's sign bit replicated.
+AQ_DEVICE uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Four E2M1 codes (the nibbles of c[15:0]: sign bit 3, magnitude bits 2..0) as
+// their values doubled, in signed bytes: 2 * {0, 0.5, 1, 1.5, 2, 3, 4, 6} = 0..12.
+// One lookup keeps the positive codes (a set sign bit replicates the table
+// byte's clear sign bit: 0), one with the sign bits flipped keeps the negative
+// ones; byte-wise pos - neg is formed without borrows between bytes.
+AQ_DEVICE uint32_t e2m1x2_bytes(uint32_t c) {
+  constexpr uint32_t kLo = 0x03020100u, kHi = 0x0C080604u;
+  const uint32_t pos = prmt(kLo, kHi, c);
+  const uint32_t neg = prmt(kLo, kHi, c ^ 0x8888u);
+  return ((pos | 0x80808080u) - neg) ^ 0x80808080u;
+}
+
+// X / 2 of an E8M0 scale byte (X = 2^(s - 127); the MMA sees values doubled).
+AQ_DEVICE float e8m0_half(uint32_t sb) {
+  return sb >= 2u ? (sb == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float((sb - 1u) << 23))
+                  : __uint_as_float(0x00200000u << sb);
+}
 
 // Bounded spin until *ctr >= target (shared-memory counter written by other
 // warps of the CTA); false on timeout (fault bit set, abort raised) or abort.
@@ -192,7 +231,7 @@ struct Args {
   int E, cta_per_tok;
 };
 
-template <int BITS, int G, int MP>
+template <int BITS, int G, int MP, int FMT>
 __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(const __grid_constant__ Args a, const __grid_constant__ CUtensorMap wmap,
                                                                   const __grid_constant__ CUtensorMap smap,
                                                                   const __grid_constant__ CUtensorMap bmap) {
@@ -200,11 +239,12 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   constexpr int U = G / 32;                      // K tiles (16 bytes of activation digits per lane) per group
   constexpr int NWD = LaneWords<BITS, G>::count;
   constexpr int GBYTES = G * BITS / 8;           // packed bytes of one group row
-  constexpr int SL = LaneSpan<BITS, G>::length;
+  constexpr int SL = LaneSpan<BITS, G, FMT>::length;
+  static_assert(FMT == 0 || (BITS == 4 && G == 32), "mxfp4: 4-bit codes, groups of 32");
   // accumulator chains per digit plane: a group folded on its own has only
   // G/32 MMAs per plane, and summing chains would cost more than it hides
   constexpr int NACC = GS == 1 ? 1 : kAcc;
-  using Span = LaneSpan<BITS, G>;
+  using Span = LaneSpan<BITS, G, FMT>;
 
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t *ring = smem;
@@ -258,10 +298,10 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     const int T = st / a.nch, ch = st - T * a.nch;
     const int rb = static_cast<int>(wrow0 + tile_base(T));
     uint8_t *dst = ring + static_cast<size_t>(s) * a.stage_bytes;
-    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRows * (a.pitch_w + 2 * a.pitch_s)));
+    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRows * (a.pitch_w + (FMT == 0 ? 2 : 1) * a.pitch_s)));
     tma_load_2d(dst, &wmap, &full[s], ch * a.w_box_x, rb);
     tma_load_2d(dst + a.s_off, &smap, &full[s], ch * a.sb_box_x, rb);
-    tma_load_2d(dst + a.b_off, &bmap, &full[s], ch * a.sb_box_x, rb);
+    if constexpr (FMT == 0) tma_load_2d(dst + a.b_off, &bmap, &full[s], ch * a.sb_box_x, rb);
   };
 
   if (tid == 0) {
@@ -461,11 +501,20 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           constexpr int c = C.value;
           const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);  // lo set 0, lo set 1, hi set 0, hi set 1
           uint32_t q0[2], q1[2];
-          tile_codes<BITS, G, c>(w0, t, q0);
-          tile_codes<BITS, G, c>(w1, t, q1);
           constexpr int k = (j * U + c) % NACC;
-          mma_u8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
-          mma_u8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
+          if constexpr (FMT == 1) {
+            q0[0] = e2m1x2_bytes(w0[0]);
+            q0[1] = e2m1x2_bytes(w0[0] >> 16);
+            q1[0] = e2m1x2_bytes(w1[0]);
+            q1[1] = e2m1x2_bytes(w1[0] >> 16);
+            mma_s8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
+            mma_s8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
+          } else {
+            tile_codes<BITS, G, c>(w0, t, q0);
+            tile_codes<BITS, G, c>(w1, t, q1);
+            mma_u8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
+            mma_u8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
+          }
         });
       });
       float D[4];  // sum_k q_k x_int_k of the lane's 4 (row, column) cells, exact in int32
@@ -486,18 +535,32 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       if constexpr (GS >= 2) {
         const int gl = p * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
         const int mt = (2 * t) / GS;
-        s0 = __half22float2(*reinterpret_cast<const __half2 *>(sr0 + gl * 2));
-        s1 = __half22float2(*reinterpret_cast<const __half2 *>(sr1 + gl * 2));
-        b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
-        b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
+        if constexpr (FMT == 1) {  // two E8M0 bytes per row (groups gl, gl + 1); no bias
+          const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
+          const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
+          s0 = make_float2(e8m0_half(e0 & 0xFFu), e8m0_half(e0 >> 8));
+          s1 = make_float2(e8m0_half(e1 & 0xFFu), e8m0_half(e1 >> 8));
+          b0 = b1 = make_float2(0.0f, 0.0f);
+        } else {
+          s0 = __half22float2(*reinterpret_cast<const __half2 *>(sr0 + gl * 2));
+          s1 = __half22float2(*reinterpret_cast<const __half2 *>(sr1 + gl * 2));
+          b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
+          b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
+        }
         T0 = tab[mt * a.Gn + gch0 + gl];
         T1 = tab[mt * a.Gn + gch0 + gl + 1];
       } else {
         const int gl = p;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
-        const float sv0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
-        const float sv1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
-        const float bv0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
-        const float bv1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
+        float sv0, sv1, bv0 = 0.0f, bv1 = 0.0f;
+        if constexpr (FMT == 1) {
+          sv0 = e8m0_half(sr0[gl]);
+          sv1 = e8m0_half(sr1[gl]);
+        } else {
+          sv0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
+          sv1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
+          bv0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
+          bv1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
+        }
         s0 = make_float2(sv0, sv0);
         s1 = make_float2(sv1, sv1);
         b0 = make_float2(bv0, bv0);
@@ -506,9 +569,14 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
       }
       const float2 tx = make_float2(T0.x, T1.x), ty = make_float2(T0.y, T1.y), tz = make_float2(T0.z, T1.z);
-      // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x
-      accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), ffma2(b0, tx, accA));
-      accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), ffma2(b1, tx, accB));
+      // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x   (mxfp4: s = X / 2, no bias)
+      if constexpr (FMT == 1) {
+        accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), accA);
+        accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), accB);
+      } else {
+        accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), ffma2(b0, tx, accA));
+        accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), ffma2(b1, tx, accB));
+      }
     }
     const float acc[4] = {accA.x, accA.y, accB.x, accB.y};
     __syncwarp();
@@ -623,9 +691,13 @@ static int64_t code_pitch(int64_t row_bytes, int bits, int G) {
   return pitch_at(row_bytes, 128, 64);
 }
 
-static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl) {
+// fmt 0: affine codes with fp16 scales and biases; fmt 1: mxfp4 (E2M1 codes,
+// one E8M0 byte per 32, no biases).
+static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt = 0) {
   if (!(bits == 2 || bits == 4 || bits == 8) || !(G == 32 || G == 64 || G == 128)) return false;
   if (M < 1 || M > 8 || N < 1 || K < 1 || K % (8 * G) != 0) return false;
+  // mxfp4 scale rows are K/32 bytes: a TMA row stride must be a multiple of 16 bytes
+  if (fmt == 1 && (bits != 4 || G != 32 || K % 512 != 0)) return false;
   if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 30)) return false;
   if (N < kRows) return false;  // every CTA owns at least one whole 16-row tile
   const int MP = pow2_tokens(static_cast<int>(M));
@@ -634,8 +706,11 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   // K chunk: the largest multiple u of 8 groups dividing K whose 16-row stage
   // of codes stays within the target
   int64_t u = 1;
+  // (mxfp4: an even number of units, so that every chunk's scale box starts on
+  // a 16-byte boundary: a chunk holds 8u scale bytes)
+  if (fmt == 1) u = 2;
   for (int64_t c = 1; c <= units; ++c)
-    if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= kStageTarget) u = c;
+    if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= kStageTarget && (fmt == 0 || c % 2 == 0)) u = c;
   const int64_t Kc = 8 * G * u, nch = K / Kc, gpc = Kc / G;
   Args &a = pl.a;
   a.early_w = 0;
@@ -649,13 +724,16 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.Kc = static_cast<int>(Kc);
   a.nch = static_cast<int>(nch);
   a.pitch_w = static_cast<int>(code_pitch(Kc * bits / 8, bits, G));
-  a.pitch_s = static_cast<int>(pitch_at(gpc * 2, 32, 16));
+  const int sbytes = fmt == 1 ? 1 : 2;  // bytes of one group's scale
+  a.pitch_s = static_cast<int>(pitch_at(gpc * sbytes, 32, 16));
   if (a.pitch_w / 8 > 256 || a.pitch_s / 8 > 256) return false;  // TMA box width (64-bit elements)
   a.w_box_x = static_cast<int>(Kc * bits / 64);
-  a.sb_box_x = static_cast<int>(gpc / 4);
+  a.sb_box_x = static_cast<int>(gpc * sbytes / 8);
+  // every tiled TMA copy starts on a 16-byte boundary: x * 8 bytes % 16 == 0 for every chunk
+  if (nch > 1 && (a.w_box_x % 2 != 0 || a.sb_box_x % 2 != 0)) return false;
   a.s_off = kRows * a.pitch_w;
   a.b_off = a.s_off + kRows * a.pitch_s;
-  a.stage_bytes = static_cast<int>(round_up(a.b_off + kRows * a.pitch_s, 128));
+  a.stage_bytes = static_cast<int>(round_up((fmt == 1 ? a.s_off : a.b_off) + kRows * a.pitch_s, 128));
   a.tok_stride = static_cast<int>(2 * K + 64);
   a.zero_stride = static_cast<int>(round_up(U * 64, 128) + 64);
   const int64_t budget = 227 * 1024;
@@ -709,9 +787,9 @@ struct Maps {
   CUtensorMap w, s, b;
 };
 
-template <int BITS, int G, int MP>
+template <int BITS, int G, int MP, int FMT>
 static cudaError_t launch(const Plan &pl, const Maps &mp, bool overlap, cudaStream_t stream) {
-  auto kern = qmv_tc_kernel<BITS, G, MP>;
+  auto kern = qmv_tc_kernel<BITS, G, MP, FMT>;
   static thread_local int cached_dev = -1;
   static thread_local size_t cached_smem = 0;
   int dev = 0;
@@ -741,13 +819,13 @@ static cudaError_t launch(const Plan &pl, const Maps &mp, bool overlap, cudaStre
   return cudaLaunchKernelEx(&cfg, kern, pl.a, mp.w, mp.s, mp.b);
 }
 
-template <int BITS, int G>
+template <int BITS, int G, int FMT = 0>
 static cudaError_t launch_mp(const Plan &pl, const Maps &mp, bool overlap, cudaStream_t stream) {
   switch (pow2_tokens(pl.a.M)) {
-    case 1: return launch<BITS, G, 1>(pl, mp, overlap, stream);
-    case 2: return launch<BITS, G, 2>(pl, mp, overlap, stream);
-    case 4: return launch<BITS, G, 4>(pl, mp, overlap, stream);
-    default: return launch<BITS, G, 8>(pl, mp, overlap, stream);
+    case 1: return launch<BITS, G, 1, FMT>(pl, mp, overlap, stream);
+    case 2: return launch<BITS, G, 2, FMT>(pl, mp, overlap, stream);
+    case 4: return launch<BITS, G, 4, FMT>(pl, mp, overlap, stream);
+    default: return launch<BITS, G, 8, FMT>(pl, mp, overlap, stream);
   }
 }
 
@@ -851,6 +929,38 @@ cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint
     case 4: return tc::launch_g<4>(pl, mp, G, false, s);
     default: return tc::launch_g<8>(pl, mp, G, false, s);
   }
+}
+
+bool mxfp4_tc_supported(int64_t M, int64_t N, int64_t K) {
+  tc::Plan pl;
+  return tc::make_plan(M, N, K, 32, 4, 148, pl, 1);
+}
+
+// mxfp4 (E2M1 codes packed 8 per word, one E8M0 scale byte per 32 along K).
+cudaError_t launch_mxfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
+                            int64_t N, uint16_t *y, uint32_t flags, cudaStream_t s) {
+  static thread_local int cached_dev = -1, sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  tc::Plan pl;
+  if (!tc::make_plan(M, N, K, 32, 4, sms, pl, 1)) return cudaErrorInvalidValue;
+  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.packed = packed;
+  pl.a.scales = reinterpret_cast<const __half *>(scales);  // read as bytes by the mxfp4 kernel
+  pl.a.biases = nullptr;
+  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
+  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
+  tc::Maps mp;
+  if (!tc::encode_rows(&mp.w, packed, N, K / 2, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 32, pl.a.pitch_s))
+    return cudaErrorInvalidValue;
+  mp.b = mp.s;  // no bias map: the kernel never reads this one
+  return tc::launch_mp<4, 32, 1>(pl, mp, overlap, s);
 }
 
 cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word) {
