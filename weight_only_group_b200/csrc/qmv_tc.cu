@@ -153,17 +153,6 @@ AQ_DEVICE void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// The same with signed A bytes (mxfp4 values).
-AQ_DEVICE void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-AQ_DEVICE void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // prmt.b32 in its default mode: result byte n is byte (c >> 4n) & 7 of {b, a},
 // or, when bit 4n+3 of c is set, that byte's sign bit replicated.
@@ -173,16 +162,19 @@ AQ_DEVICE uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
   return d;
 }
 
-// Four E2M1 codes (the nibbles of c[15:0]: sign bit 3, magnitude bits 2..0) as
-// their values doubled, in signed bytes: 2 * {0, 0.5, 1, 1.5, 2, 3, 4, 6} = 0..12.
-// One lookup keeps the positive codes (a set sign bit replicates the table
-// byte's clear sign bit: 0), one with the sign bits flipped keeps the negative
-// ones; byte-wise pos - neg is formed without borrows between bytes.
-AQ_DEVICE uint32_t e2m1x2_bytes(uint32_t c) {
+// Eight E2M1 codes of a word (nibbles: sign bit 3, magnitude bits 2..0) as their
+// doubled magnitudes 2 * {0, 0.5, 1, 1.5, 2, 3, 4, 6} = 0..12 in unsigned bytes,
+// split by sign: pos holds the positive codes (0 for the negative ones), neg the
+// negative ones.  Register set s takes codes 4s..4s+3.  One prmt looks up four
+// codes; a set sign bit replicates the table byte's clear sign bit, giving 0, so
+// the lookup with the sign bits flipped keeps exactly the negative codes.
+AQ_DEVICE void e2m1x2_split(uint32_t w, uint32_t (&pos)[2], uint32_t (&neg)[2]) {
   constexpr uint32_t kLo = 0x03020100u, kHi = 0x0C080604u;
-  const uint32_t pos = prmt(kLo, kHi, c);
-  const uint32_t neg = prmt(kLo, kHi, c ^ 0x8888u);
-  return ((pos | 0x80808080u) - neg) ^ 0x80808080u;
+  const uint32_t wn = w ^ 0x88888888u;
+  pos[0] = prmt(kLo, kHi, w);
+  neg[0] = prmt(kLo, kHi, wn);
+  pos[1] = prmt(kLo, kHi, w >> 16);
+  neg[1] = prmt(kLo, kHi, wn >> 16);
 }
 
 // X / 2 of an E8M0 scale byte (X = 2^(s - 127); the MMA sees values doubled).
@@ -488,8 +480,14 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
 
     for (int p = 0; p < nper; ++p) {
       int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
+      // mxfp4: the same sums over the negative codes' magnitudes, subtracted below
+      int nl[FMT == 1 ? NACC : 1][4], nh[FMT == 1 ? NACC : 1][4];
 #pragma unroll
       for (int i = 0; i < NACC; ++i) dl[i][0] = dl[i][1] = dl[i][2] = dl[i][3] = dh[i][0] = dh[i][1] = dh[i][2] = dh[i][3] = 0;
+      if constexpr (FMT == 1) {
+#pragma unroll
+        for (int i = 0; i < NACC; ++i) nl[i][0] = nl[i][1] = nl[i][2] = nl[i][3] = nh[i][0] = nh[i][1] = nh[i][2] = nh[i][3] = 0;
+      }
       static_for<0, GS>([&](auto J) {
         constexpr int j = J.value;
         const int gi = p * GS + j;
@@ -503,12 +501,13 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           uint32_t q0[2], q1[2];
           constexpr int k = (j * U + c) % NACC;
           if constexpr (FMT == 1) {
-            q0[0] = e2m1x2_bytes(w0[0]);
-            q0[1] = e2m1x2_bytes(w0[0] >> 16);
-            q1[0] = e2m1x2_bytes(w1[0]);
-            q1[1] = e2m1x2_bytes(w1[0] >> 16);
-            mma_s8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
-            mma_s8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
+            uint32_t n0[2], n1[2];
+            e2m1x2_split(w0[0], q0, n0);
+            e2m1x2_split(w1[0], q1, n1);
+            mma_u8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
+            mma_u8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
+            mma_u8u8(nl[k], n0[0], n1[0], n0[1], n1[1], bv.x, bv.y);
+            mma_u8s8(nh[k], n0[0], n1[0], n0[1], n1[1], bv.z, bv.w);
           } else {
             tile_codes<BITS, G, c>(w0, t, q0);
             tile_codes<BITS, G, c>(w1, t, q1);
@@ -525,6 +524,13 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         for (int c = 1; c < NACC; ++c) {
           lo += dl[c][i];
           hi += dh[c][i];
+        }
+        if constexpr (FMT == 1) {
+#pragma unroll
+          for (int c = 0; c < NACC; ++c) {
+            lo -= nl[c][i];
+            hi -= nh[c][i];
+          }
         }
         D[i] = static_cast<float>(hi * 256 + lo);
       }
