@@ -381,6 +381,27 @@ def section_gather(args, aq, torch, dev, stream, peaks):
         gbs = wb / (ms * 1e-3) / 1e9
         res[f"tokens{tokens}_top2"] = {"rows": T, "us": round(ms * 1e3, 2), "weight_GBps": round(gbs, 1),
                                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    # prefill form: 4096 routed rows (2048 tokens, top-2) grouped by expert, one matmul per expert.
+    # The call reads the per-expert counts on the host, so it is timed per call, not from a graph.
+    T = 4096
+    ex = torch.randint(0, E, (T,), dtype=torch.int32, device=dev, generator=torch.Generator(device=dev).manual_seed(8))
+    x = synth.activations(T, K, 18).to(dev)
+    y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            aq.aq_gather_matmul(x, ex, gp, gs, gb, G, BITS, out=y, grouped=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            aq.aq_gather_matmul(x, ex, gp, gs, gb, G, BITS, out=y, grouped=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 5
+    tf = 2.0 * T * N * K / (ms * 1e-3) / 1e12
+    res["prefill_grouped_4096_rows"] = {"rows": T, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                        "frac_bf16_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                                        "note": "includes routing, the host read of per-expert counts, gather/scatter"}
     return {"gather_qmv": {"E": E, "N": N, "K": K, "bits": BITS, "G": G, "points": res}}
 
 

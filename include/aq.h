@@ -236,6 +236,24 @@ aq_status aq_gather_matmul(const uint16_t *x_bf16, int64_t T, int64_t K, const u
                            const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
                            const int32_t *experts, uint16_t *y_bf16, aq_stream_t stream);
 
+/* Prefill form of aq_gather_matmul: the same result (y[t, :] = x[t, :] @
+ * dequant(W[experts[t]])^T, a zero row and AQ_FAULT_BAD_INDEX for an id outside
+ * [0, E)), computed by grouping the tokens by expert so that each expert's
+ * weights are multiplied once against all of its tokens: a routing kernel
+ * orders the tokens by expert, x rows are gathered into that order, each
+ * expert's rows go through aq_matmul's per-shape kernels (QMM at prefill
+ * sizes), and the rows are scattered back.  The host reads the E per-expert
+ * counts once, so the call synchronizes its stream (it cannot be captured in a
+ * CUDA graph).  Workspace (offsets, positions, x and y in expert order, the QMM
+ * workspace) comes from the stream-ordered allocator.  Shapes: as aq_matmul for
+ * every segment size, N a multiple of 8, each expert's packed/scale/bias block a
+ * multiple of 16 bytes, E <= 16384 (others -> AQ_ERR_UNSUPPORTED or
+ * AQ_ERR_INVALID_ARG).  Accuracy as aq_matmul.  Source: metalworking "MLX
+ * Quantization", the kernel family list ("gather variants for MoE experts"). */
+aq_status aq_gather_matmul_grouped(const uint16_t *x_bf16, int64_t T, int64_t K, const uint32_t *packed,
+                                   const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G,
+                                   int bits, const int32_t *experts, uint16_t *y_bf16, aq_stream_t stream);
+
 /* ---- mxfp4: block-scaled fp4 ------------------------------------------------
  * Source: metalworking "MLX Quantization" (the newer block-scaled float modes:
  * mxfp4 with groups of 32) and "Quantizing a Model for MLX", section "Modes,

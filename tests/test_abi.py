@@ -175,6 +175,20 @@ def test_gather_matmul_validation():
     assert call(E=1 << 20, N=4096) == aq.AQ_ERR_INVALID_ARG  # E*N >= 2^31
 
 
+def test_gather_matmul_grouped_validation():
+    L = aq.lib()
+    def call(x=A, T=64, K=4096, E=8, N=1024, G=64, bits=4, experts=A, y=A):
+        return L.aq_gather_matmul_grouped(x, T, K, A, A, A, E, N, G, bits, experts, y, None)
+    assert call(T=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(E=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(E=20000, N=64) == aq.AQ_ERR_INVALID_ARG    # more experts than the routing CTA takes
+    assert call(K=4000) == aq.AQ_ERR_INVALID_ARG           # K % G != 0
+    assert call(experts=A + 2) == aq.AQ_ERR_ALIGNMENT
+    assert call(x=U) == aq.AQ_ERR_ALIGNMENT
+    assert call(N=1028) == aq.AQ_ERR_UNSUPPORTED           # segments of y must stay 16-byte aligned
+    assert call(bits=5) == aq.AQ_ERR_UNSUPPORTED
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

@@ -197,6 +197,56 @@ def test_quantize_mse_full_size_sampled_rows(G, bits):
     assert float(e_mse.sum()) < float(e_rtn.sum())
 
 
+# ----------------------------------------------------------------------------- gather matmul, prefill form
+
+@pytest.mark.parametrize("T,E,N,K,G,bits", [(40, 4, 256, 512, 64, 4), (100, 3, 128, 1024, 32, 3),
+                                            (17, 5, 64, 256, 128, 8), (9, 2, 48, 512, 64, 2)])
+def test_gather_grouped_matches_oracle_per_token(T, E, N, K, G, bits):
+    ws = [weights(N, K, 600 + e, True) for e in range(E)]
+    qs = [oracle.quantize(w, G, bits) for w in ws]
+    packed = torch.from_numpy(np.stack([q[0] for q in qs]).view(np.int32)).cuda()
+    scales = torch.from_numpy(np.stack([q[1] for q in qs]).view(np.float16)).cuda()
+    biases = torch.from_numpy(np.stack([q[2] for q in qs]).view(np.float16)).cuda()
+    rng = np.random.default_rng(T + E)
+    ex = rng.integers(0, E, T).astype(np.int32)
+    ex[1] = E + 3                     # a bad id: zero row and a fault bit
+    ex[2:5] = 0                       # (expert E - 1 may end up empty on short inputs: that is allowed)
+    xb = activations_bits(T, K, 601)
+    y = aq.aq_gather_matmul(_x_gpu(xb), torch.from_numpy(ex).cuda(), packed, scales, biases, G, bits, grouped=True)
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() & aq.AQ_FAULT_BAD_INDEX
+    yc = y.float().cpu().numpy()
+    assert (yc[1] == 0).all()
+    for e in range(E):
+        rows = np.nonzero(ex == e)[0]
+        if len(rows):
+            y_ref = oracle.matmul(xb[rows], *qs[e], G, bits)
+            _assert_close(y[torch.from_numpy(rows).cuda()], y_ref, f"grouped gather expert {e}")
+
+
+def test_gather_grouped_mixtral_prefill_bitequal_per_expert():
+    """E = 8 experts of W[14336, 4096] (4-bit G64), 256 tokens routed top-2 (512 rows):
+    every row equals aq_matmul of that expert over the same rows, bit for bit."""
+    E, N, K, T = 8, 14336, 4096, 512
+    packed, scales, biases = [], [], []
+    for e in range(E):
+        w = torch.from_numpy(synth.weights(N, K, 700 + e, True)).cuda()
+        p, s, b = aq.aq_quantize(w, 64, 4)
+        packed.append(p); scales.append(s); biases.append(b)
+        del w
+    P, S, B = torch.stack(packed), torch.stack(scales), torch.stack(biases)
+    rng = np.random.default_rng(9)
+    ex = rng.integers(0, E, T).astype(np.int32)
+    x = _x_gpu(activations_bits(T, K, 701))
+    y = aq.aq_gather_matmul(x, torch.from_numpy(ex).cuda(), P, S, B, 64, 4, grouped=True)
+    for e in range(E):
+        rows = torch.from_numpy(np.nonzero(ex == e)[0]).cuda()
+        if len(rows):
+            ref = aq.aq_matmul(x[rows].contiguous(), P[e], S[e], B[e], 64, 4)
+            assert torch.equal(y[rows], ref), e
+    torch.cuda.synchronize()
+
+
 # ----------------------------------------------------------------------------- mxfp4 (block-scaled fp4)
 
 def _mx_special(N, K, seed):

@@ -10,7 +10,7 @@ binding fails loudly when the library has not been built
 
 Names mirror the C entry points: ``aq_quantize``, ``aq_quantize_mse``,
 ``aq_dequantize``, ``aq_dequantize_f32``, ``aq_matmul``, ``aq_matmul_with``,
-``aq_matmul_ex``, ``aq_embedding``, ``aq_gather_matmul``, ``aq_mxfp4_quantize``,
+``aq_matmul_ex``, ``aq_embedding``, ``aq_gather_matmul``, ``aq_gather_matmul_grouped``, ``aq_mxfp4_quantize``,
 ``aq_mxfp4_dequantize``, ``aq_mxfp4_dequantize_f32``, ``aq_mxfp4_matmul``,
 ``aq_mxfp4_packed_bytes``, ``aq_dispatch``,
 ``aq_matmul_ws``, ``aq_matmul_workspace_bytes``, ``aq_packed_words``,
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             L.aq_matmul_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, ctypes.c_uint32, vp]
             L.aq_embedding.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_gather_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, vp]
+            L.aq_gather_matmul_grouped.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, vp]
             L.aq_matmul_ws.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp, u64, vp]
             L.aq_mxfp4_packed_bytes.argtypes = [i64, i64]
             L.aq_mxfp4_packed_bytes.restype = u64
@@ -223,12 +224,14 @@ def aq_embedding(ids, packed, scales, biases, D: int, G: int, bits: int, out: to
     return out
 
 
-def aq_gather_matmul(x, experts, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None):
+def aq_gather_matmul(x, experts, packed, scales, biases, G: int, bits: int, out: torch.Tensor | None = None,
+                     grouped: bool = False):
     """y [T, N] bf16: row t = x[t] @ dequant(W[experts[t]])^T for E stacked experts.
 
-    packed [E, N, K*bits/32] int32, scales/biases [E, N, K/G] fp16 (or the same arrays
-    flattened to [E*N, ...] with E given by experts' range: pass 3-D arrays); experts
-    int32 [T] on the device."""
+    packed [E, N, K*bits/32] int32, scales/biases [E, N, K/G] fp16 (3-D arrays);
+    experts int32 [T] on the device.  grouped=True takes the prefill form
+    (aq_gather_matmul_grouped: tokens grouped by expert, one matmul per expert;
+    synchronizes the stream)."""
     _need(x, "x", (torch.bfloat16,))
     if packed.dim() != 3 or scales.dim() != 3 or biases.dim() != 3:
         raise ValueError("packed, scales and biases must be [E, N, ...]")
@@ -244,9 +247,10 @@ def aq_gather_matmul(x, experts, packed, scales, biases, G: int, bits: int, out:
         out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", (torch.bfloat16,))
     with torch.cuda.device(x.device):
-        rc = lib().aq_gather_matmul(x.data_ptr(), T, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), E, N,
-                                    G, bits, experts.data_ptr(), out.data_ptr(), _stream(x))
-    _check(rc, "aq_gather_matmul")
+        fn = "aq_gather_matmul_grouped" if grouped else "aq_gather_matmul"
+        rc = getattr(lib(), fn)(x.data_ptr(), T, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), E, N, G,
+                                bits, experts.data_ptr(), out.data_ptr(), _stream(x))
+    _check(rc, fn)
     return out
 
 

@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libaq.so")
 
-SOURCES = ["aq_api.cu", "quantize.cu", "qmv.cu", "qmv_tc.cu", "qmm.cu", "noalloc.cu", "embedding.cu", "mxfp4.cu"]
+SOURCES = ["aq_api.cu", "quantize.cu", "qmv.cu", "qmv_tc.cu", "qmm.cu", "noalloc.cu", "embedding.cu", "mxfp4.cu", "gather.cu"]
 HEADERS = ["common.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

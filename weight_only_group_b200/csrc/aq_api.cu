@@ -1,6 +1,8 @@
 // C ABI entry points: argument validation, per-shape dispatch, launches.
 // Method and layouts: see include/aq.h.
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -35,6 +37,14 @@ cudaError_t launch_mxfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t
 cudaError_t launch_mxfp4_dequantize(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K, void *out,
                                     bool bf16_out, cudaStream_t s);
 bool mxfp4_tc_supported(int64_t M, int64_t N, int64_t K);
+int gather_route_max_experts();
+cudaError_t launch_gather_route(const int32_t *experts, int64_t T, int64_t E, int32_t *offsets, int32_t *pos,
+                                cudaStream_t s);
+cudaError_t launch_gather_rows(const uint16_t *x, int64_t T, int64_t K, const int32_t *pos, uint16_t *x_sorted,
+                               cudaStream_t s);
+cudaError_t launch_scatter_rows(const uint16_t *y_sorted, int64_t T, int64_t N, const int32_t *pos,
+                                const int32_t *experts, int64_t E, uint16_t *y, cudaStream_t s);
+cudaError_t read_and_clear_gather_fault(uint32_t *word);
 cudaError_t launch_mxfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
                             int64_t N, uint16_t *y, uint32_t flags, cudaStream_t s);
 }  // namespace aq
@@ -293,6 +303,60 @@ aq_status aq_gather_matmul(const uint16_t *x, int64_t T, int64_t K, const uint32
   return from_cuda(aq::launch_gather_tc(x, T, K, packed, scales, biases, E, N, G, bits, experts, y, stream));
 }
 
+static size_t round16(size_t v) { return (v + 15) / 16 * 16; }
+
+aq_status aq_gather_matmul_grouped(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed,
+                                   const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
+                                   const int32_t *experts, uint16_t *y, aq_stream_t stream) {
+  if (T <= 0 || E <= 0 || T >= (int64_t(1) << 31)) return AQ_ERR_INVALID_ARG;
+  aq_status st = check_shape(N, K, G, bits);
+  if (st != AQ_OK) return st;
+  if (E * N >= (int64_t(1) << 31) || E > aq::gather_route_max_experts()) return AQ_ERR_INVALID_ARG;
+  if (!x || !packed || !scales || !biases || !experts || !y) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(biases) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(experts) & 3u) != 0)
+    return AQ_ERR_ALIGNMENT;
+  // every expert's arrays and every segment of the sorted rows start on 16 bytes
+  if (N % 8 != 0 || (N * K * bits / 8) % 16 != 0 || (N * (K / G) * 2) % 16 != 0) return AQ_ERR_UNSUPPORTED;
+  // every segment size from 1 to T must have a kernel
+  for (int64_t m = 1; m <= std::min<int64_t>(T, 9); ++m)
+    if (aq_dispatch(m, N, K, G, bits) < 0) return AQ_ERR_UNSUPPORTED;
+  if (T > 9 && aq_dispatch(T, N, K, G, bits) < 0) return AQ_ERR_UNSUPPORTED;
+  if ((st = check_device()) != AQ_OK) return st;
+
+  // one stream-ordered allocation: offsets [E+2], positions [T], x and y in
+  // segment order, and the QMM workspace for the largest possible segment
+  const size_t b_off = round16(static_cast<size_t>(E + 2) * 4), b_pos = round16(static_cast<size_t>(T) * 4);
+  const size_t b_x = round16(static_cast<size_t>(T) * K * 2), b_y = round16(static_cast<size_t>(T) * N * 2);
+  const size_t b_ws = round16(aq::qmm_workspace_bytes(T, K));
+  uint8_t *ws = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&ws), b_off + b_pos + b_x + b_y + b_ws, stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  int32_t *offsets = reinterpret_cast<int32_t *>(ws);
+  int32_t *pos = reinterpret_cast<int32_t *>(ws + b_off);
+  uint16_t *xs = reinterpret_cast<uint16_t *>(ws + b_off + b_pos);
+  uint16_t *ys = reinterpret_cast<uint16_t *>(ws + b_off + b_pos + b_x);
+  void *qws = ws + b_off + b_pos + b_x + b_y;
+  std::vector<int32_t> off(static_cast<size_t>(E + 2));
+  st = from_cuda(aq::launch_gather_route(experts, T, E, offsets, pos, stream));
+  if (st == AQ_OK)
+    st = from_cuda(cudaMemcpyAsync(off.data(), offsets, off.size() * 4, cudaMemcpyDeviceToHost, stream));
+  if (st == AQ_OK) st = from_cuda(cudaStreamSynchronize(stream));
+  if (st == AQ_OK) st = from_cuda(aq::launch_gather_rows(x, T, K, pos, xs, stream));
+  const int64_t P = K * bits / 32, Gn = K / G;
+  for (int64_t ex = 0; st == AQ_OK && ex < E; ++ex) {
+    const int64_t o = off[ex], cnt = off[ex + 1] - off[ex];
+    if (cnt <= 0) continue;
+    const aq_kernel k = static_cast<aq_kernel>(aq_dispatch(cnt, N, K, G, bits));
+    st = matmul_run(k, xs + o * K, cnt, K, packed + ex * N * P, scales + ex * N * Gn, biases + ex * N * Gn, N, G, bits,
+                    ys + o * N, qws, stream);
+  }
+  if (st == AQ_OK) st = from_cuda(aq::launch_scatter_rows(ys, T, N, pos, experts, E, y, stream));
+  e = cudaFreeAsync(ws, stream);
+  if (st == AQ_OK && e != cudaSuccess) st = from_cuda(e);
+  return st;
+}
+
 size_t aq_mxfp4_packed_bytes(int64_t N, int64_t K) {
   if (check_mx_shape(N, K) != AQ_OK) return 0;
   const size_t nk = static_cast<size_t>(N) * static_cast<size_t>(K);
@@ -351,9 +415,11 @@ aq_status aq_device_fault(uint32_t *fault_word) {
   if (st != AQ_OK) return st;
   st = from_cuda(aq::read_and_clear_qmv_tc_fault(&c));
   if (st != AQ_OK) return st;
-  uint32_t d = 0;
+  uint32_t d = 0, g = 0;
   st = from_cuda(aq::read_and_clear_embed_fault(&d));
-  *fault_word = a | b | c | d;
+  if (st != AQ_OK) return st;
+  st = from_cuda(aq::read_and_clear_gather_fault(&g));
+  *fault_word = a | b | c | d | g;
   return st;
 }
 
