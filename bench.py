@@ -428,7 +428,7 @@ def section_mxfp4(args, aq, torch, dev, stream, peaks):
         gbs = wb / (ms * 1e-3) / 1e9
         out[f"mxfp4_qmv_K{K}_N{N}"] = {"us": round(ms * 1e3, 3), "weight_GBps": round(gbs, 1),
                                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                                       "kernel": "qmv_tc_kernel<4,32,1,mxfp4> (mma.sync m16n8k32 s8 codes)"}
+                                       "kernel": "qmv_tc_kernel<4,32,1,mxfp4> (mma.sync m16n8k32, codes split by sign)"}
         del qs, base
         torch.cuda.empty_cache()
     return out

@@ -55,6 +55,11 @@ class Oracle:
         lib.oracle_mxfp4_dequantize_f32.argtypes = [vp, vp, i64, i64, vp]
         lib.oracle_mxfp4_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp]
         lib.oracle_mxfp4_matmul_sampled.argtypes = [vp, i64, i64, vp, vp, i64, vp, i64, vp, i64, vp]
+        lib.oracle_nvfp4_tensor_scale.argtypes = [vp, i64]
+        lib.oracle_nvfp4_tensor_scale.restype = ctypes.c_float
+        lib.oracle_nvfp4_quantize.argtypes = [vp, i64, i64, ctypes.c_float, vp, vp]
+        lib.oracle_nvfp4_dequantize_f32.argtypes = [vp, vp, ctypes.c_float, i64, i64, vp]
+        lib.oracle_nvfp4_matmul.argtypes = [vp, i64, i64, vp, vp, ctypes.c_float, i64, vp]
         lib.oracle_f16_round.argtypes = [vp, i64, vp]
         lib.oracle_bf16_round.argtypes = [vp, i64, vp]
         lib.oracle_f16_to_double.argtypes = [vp, i64, vp]
@@ -178,6 +183,35 @@ class Oracle:
                                                     _p(ni), len(ni), _p(y)), "mxfp4_matmul_sampled")
         return y
 
+    # ---- nvfp4 (E2M1 codes, E4M3 scale per 16 along K, fp32 scale per tensor)
+    def nvfp4_quantize(self, w: np.ndarray):
+        """w fp32 [N, K] -> (packed uint32 [N, K/8], scales uint8 [N, K/16] E4M3, g float)."""
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        N, K = w.shape
+        g = float(self.lib.oracle_nvfp4_tensor_scale(_p(w), w.size))
+        packed = np.zeros((N, K // 8), dtype=np.uint32)
+        scales = np.zeros((N, K // 16), dtype=np.uint8)
+        _check(self.lib.oracle_nvfp4_quantize(_p(w), N, K, g, _p(packed), _p(scales)), "nvfp4_quantize")
+        return packed, scales, g
+
+    def nvfp4_dequantize_f32(self, packed, scales, g: float, K: int) -> np.ndarray:
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        N = packed.shape[0]
+        out = np.zeros((N, K), dtype=np.float32)
+        _check(self.lib.oracle_nvfp4_dequantize_f32(_p(packed), _p(scales), g, N, K, _p(out)), "nvfp4_dequantize_f32")
+        return out
+
+    def nvfp4_matmul(self, x_bf16_bits, packed, scales, g: float) -> np.ndarray:
+        x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        M, K = x.shape
+        N = packed.shape[0]
+        y = np.zeros((M, N), dtype=np.float64)
+        _check(self.lib.oracle_nvfp4_matmul(_p(x), M, K, _p(packed), _p(scales), g, N, _p(y)), "nvfp4_matmul")
+        return y
+
     def f16_round(self, a: np.ndarray) -> np.ndarray:
         a = np.ascontiguousarray(a, dtype=np.float32)
         out = np.zeros(a.shape, dtype=np.uint16)
@@ -269,6 +303,18 @@ def mxfp4_matmul(x_bf16_bits, packed, scales):
 
 def mxfp4_matmul_sampled(x_bf16_bits, packed, scales, m_idx, n_idx):
     return default().mxfp4_matmul_sampled(x_bf16_bits, packed, scales, m_idx, n_idx)
+
+
+def nvfp4_quantize(w):
+    return default().nvfp4_quantize(w)
+
+
+def nvfp4_dequantize_f32(packed, scales, g, K):
+    return default().nvfp4_dequantize_f32(packed, scales, g, K)
+
+
+def nvfp4_matmul(x_bf16_bits, packed, scales, g):
+    return default().nvfp4_matmul(x_bf16_bits, packed, scales, g)
 
 
 def f16_round(a):

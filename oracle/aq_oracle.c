@@ -25,6 +25,9 @@
  *  - "metalworking — MLX Quantization" (newer modes) and "Quantizing a Model
  *    for MLX", section "Modes, bits and mixed recipes": the mxfp4 block-scaled
  *    mode (oracle_mxfp4_*; encodings and readings beside them).
+ *  - "ExecuTorch MLX backend — Quantization" (NVFP4 config) and "Quantizing a
+ *    Model for MLX", section "Modes, bits and mixed recipes": the nvfp4 mode
+ *    (oracle_nvfp4_*; encodings and readings beside them).
  *  - "mlx-gptq" page, section "How it works": the range search (--mse) that
  *    shrinks a group's min-max range when clipping its extremes costs less
  *    error than the coarser step (oracle_quantize_mse; readings beside it).
@@ -487,6 +490,22 @@ static double e2m1_value(uint32_t c)
 
 static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 127); }
 
+/* Nearest E2M1 magnitude code to t >= 0 (nearer wins; on a tie the even code,
+ * mantissa bit 0, wins). */
+static uint32_t e2m1_nearest(double t)
+{
+    uint32_t best = 0;
+    double best_d = fabs(t - E2M1_MAG[0]);
+    for (uint32_t c = 1; c < 8; c++) {
+        const double d = fabs(t - E2M1_MAG[c]);
+        if (d < best_d || (d == best_d && (c & 1u) == 0u && (best & 1u) == 1u)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return best;
+}
+
 static int bad_mx_shape(int64_t N, int64_t K) { return N <= 0 || K <= 0 || K % 32 != 0; }
 
 int oracle_mxfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales)
@@ -516,16 +535,7 @@ int oracle_mxfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed
             for (int i = 0; i < 32; i++) {
                 const double v = (double)wr[g * 32 + i];
                 const double t = fabs(v) * ldexp(1.0, -shared);   /* exact */
-                uint32_t best = 0;
-                double best_d = fabs(t - E2M1_MAG[0]);
-                for (uint32_t c = 1; c < 8; c++) {
-                    const double d = fabs(t - E2M1_MAG[c]);
-                    /* nearer wins; on a tie the even code (mantissa bit 0) wins */
-                    if (d < best_d || (d == best_d && (c & 1u) == 0u && (best & 1u) == 1u)) {
-                        best = c;
-                        best_d = d;
-                    }
-                }
+                uint32_t best = e2m1_nearest(t);
                 if (v < 0.0 && best != 0u) best |= 8u;
                 put_code(pr, g * 32 + i, 4, best);
             }
@@ -581,6 +591,127 @@ int oracle_mxfp4_matmul_sampled(const uint16_t *x_bf16, int64_t M, int64_t K, co
             for (int64_t k = 0; k < K; k++)
                 acc += bf16_value(x_bf16[m_idx[i] * K + k]) * mx_value(packed + n_idx[j] * P, scales + n_idx[j] * Gn, k);
             y[i * nn + j] = acc;
+        }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* nvfp4: E2M1 elements, one E4M3 scale per 16, one fp32 scale per tensor     */
+/* ------------------------------------------------------------------------ */
+
+/* "ExecuTorch MLX backend — Quantization" (NVFP4 weight-only config, group
+ * size 16) and "Quantizing a Model for MLX", section "Modes, bits and mixed
+ * recipes" (nvfp4: groups of 16, 4 bits).  The pages give no encodings; the
+ * readings follow NVIDIA's NVFP4 format, restated here:
+ *  - elements: E2M1 codes as in mxfp4 (packed 8 per uint32, LSB first);
+ *  - block scale: one E4M3 byte per 16 weights along K (sign 0, exponent bits
+ *    6..3 with bias 7, mantissa bits 2..0; subnormals m * 2^-9; largest 448);
+ *  - tensor scale: one fp32 value g = fp32(amax / 2688) (2688 = 6 * 448, the
+ *    largest E2M1 value times the largest E4M3 value); g = 1 for an all-zero
+ *    tensor;
+ *  - block scale byte: E4M3 nearest to fp32(amax_block / fp32(6 * g)), ties to
+ *    even, saturating at 448 (with this g no block goes past 448 beyond
+ *    rounding: the clamp is defensive);
+ *  - element: E2M1 nearest to fp32(|w| / fp32(scale * g)), ties to the even
+ *    code, saturating at 6, sign only on a non-zero magnitude; a zero block
+ *    scale gives code 0;
+ *  - value: fp32(fp32(e2m1 * scale) * g) (the first product is exact). */
+
+static uint8_t e4m3_bits_from_double(double v)   /* v >= 0, finite */
+{
+    double r = round_to_format(v, 3, -6);
+    if (r > 448.0) r = 448.0;                     /* saturate */
+    if (r == 0.0) return 0;
+    int ex;
+    frexp(r, &ex);
+    int e = ex - 1;
+    if (e < -6) return (uint8_t)ldexp(r, 9);      /* subnormal: m * 2^-9 */
+    uint8_t mant = (uint8_t)(ldexp(r, 3 - e) - 8.0);
+    return (uint8_t)(((e + 7) << 3) | mant);
+}
+
+static double e4m3_value(uint8_t b)
+{
+    int e = (b >> 3) & 15, m = b & 7;
+    if (e == 0) return ldexp((double)m, -9);
+    return ldexp(8.0 + m, e - 10);
+}
+
+float oracle_nvfp4_tensor_scale(const float *w, int64_t n)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; i++) {
+        float a = fabsf(w[i]);
+        if (a > amax) amax = a;
+    }
+    return amax > 0.0f ? amax / 2688.0f : 1.0f;   /* fp32 division */
+}
+
+int oracle_nvfp4_quantize(const float *w, int64_t N, int64_t K, float g, uint32_t *packed, uint8_t *scales)
+{
+    if (!w || !packed || !scales || N <= 0 || K <= 0 || K % 16 != 0 || !(g > 0.0f)) return ORACLE_BAD_ARG;
+    const int64_t P = K / 8, Gn = K / 16;
+    const float six_g = 6.0f * g;                 /* fp32 product */
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        const float *wr = w + n * K;
+        uint32_t *pr = packed + n * P;
+        for (int64_t j = 0; j < P; j++) pr[j] = 0u;
+        for (int64_t b = 0; b < Gn; b++) {
+            float amax = 0.0f;
+            for (int i = 0; i < 16; i++) {
+                float a = fabsf(wr[b * 16 + i]);
+                if (a > amax) amax = a;
+            }
+            const float s32 = amax / six_g;       /* fp32 division */
+            const uint8_t sb = e4m3_bits_from_double((double)s32);
+            scales[n * Gn + b] = sb;
+            const float denom = (float)e4m3_value(sb) * g;   /* fp32 product */
+            for (int i = 0; i < 16; i++) {
+                const float v = wr[b * 16 + i];
+                uint32_t c = 0;
+                if (sb != 0) {
+                    const float t = fabsf(v) / denom;        /* fp32 division */
+                    c = e2m1_nearest((double)t);
+                    if (v < 0.0f && c != 0u) c |= 8u;
+                }
+                put_code(pr, b * 16 + i, 4, c);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+static double nv_value(const uint32_t *prow, const uint8_t *srow, float g, int64_t k)
+{
+    const float vs = (float)(e2m1_value(get_code(prow, k, 4)) * e4m3_value(srow[k / 16]));   /* exact */
+    return (double)(vs * g);                                                                /* fp32 product */
+}
+
+int oracle_nvfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales, float g, int64_t N, int64_t K, float *out)
+{
+    if (!packed || !scales || !out || N <= 0 || K <= 0 || K % 16 != 0) return ORACLE_BAD_ARG;
+    const int64_t P = K / 8, Gn = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) out[n * K + k] = (float)nv_value(packed + n * P, scales + n * Gn, g, k);
+    return ORACLE_OK;
+}
+
+/* y = x @ W^T with W's values e2m1 * scale * g taken exactly (fp64), summed in fp64. */
+int oracle_nvfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
+                        float g, int64_t N, double *y)
+{
+    if (!x_bf16 || !packed || !scales || !y || M <= 0 || N <= 0 || K <= 0 || K % 16 != 0) return ORACLE_BAD_ARG;
+    const int64_t P = K / 8, Gn = K / 16;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t m = 0; m < M; m++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += bf16_value(x_bf16[m * K + k]) * e2m1_value(get_code(packed + n * P, k, 4)) *
+                       e4m3_value(scales[n * Gn + k / 16]);
+            y[m * N + n] = acc * (double)g;
         }
     return ORACLE_OK;
 }

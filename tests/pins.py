@@ -196,3 +196,47 @@ def mxfp4_values_f64(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """X * e2m1(code) in fp64, X = 2^(s - 127) repeated over each group of 32."""
     X = np.repeat(np.ldexp(1.0, scales.astype(np.int64) - 127), 32, axis=-1)
     return E2M1_VALUES[codes.astype(np.int64)] * X
+
+
+def e4m3_all_values() -> np.ndarray:
+    """Every finite non-negative E4M3 value by byte 0..126 (sign 0, exponent
+    bits 6..3 bias 7, mantissa bits 2..0; 0x7F is NaN)."""
+    b = np.arange(127)
+    e, m = b >> 3, b & 7
+    return np.where(e == 0, m * 2.0 ** -9, (8.0 + m) * np.ldexp(1.0, e - 10))
+
+
+def numpy_nvfp4_quantize(w: np.ndarray):
+    """Independent NumPy statement of the nvfp4 quantizer: tensor scale
+    g = fp32(amax / 2688); block byte = the E4M3 value nearest to
+    fp32(amax_b / fp32(6 g)) found by searching all 127 values (ties to the even
+    byte, saturating at 448); elements nearest of the 16 signed E2M1 values to
+    fp32(|w| / fp32(scale * g)), ties to the even code."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    amax = np.float32(np.abs(w).max())
+    g = np.float32(amax / np.float32(2688.0)) if amax > 0 else np.float32(1.0)
+    wb = w.reshape(N, K // 16, 16)
+    s32 = (np.abs(wb).max(axis=-1) / np.float32(np.float32(6.0) * g)).astype(np.float32).astype(np.float64)
+    vals = e4m3_all_values()
+    d = np.abs(s32[..., None] - vals)
+    sb = np.zeros(s32.shape, dtype=np.int64)
+    best = d[..., 0].copy()
+    for c in range(1, 127):
+        better = (d[..., c] < best) | ((d[..., c] == best) & ((c & 1) == 0) & ((sb & 1) == 1))
+        sb = np.where(better, c, sb)
+        best = np.where(better, d[..., c], best)
+    sv = vals[sb].astype(np.float32)
+    denom = (sv * g).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (np.abs(wb) / denom[..., None]).astype(np.float32).astype(np.float64)
+    dd = np.abs(t[..., None] - E2M1_VALUES[:8])
+    codes = np.zeros(t.shape, dtype=np.int64)
+    bestc = dd[..., 0].copy()
+    for c in range(1, 8):
+        better = (dd[..., c] < bestc) | ((dd[..., c] == bestc) & ((c & 1) == 0) & ((codes & 1) == 1))
+        codes = np.where(better, c, codes)
+        bestc = np.where(better, dd[..., c], bestc)
+    codes = np.where((sb == 0)[..., None], 0, codes)
+    codes = np.where((wb < 0) & (codes != 0), codes | 8, codes).reshape(N, K).astype(np.uint32)
+    return bitwise_pack(codes, 4), sb.astype(np.uint8), float(g), codes.astype(np.uint8)

@@ -26,8 +26,8 @@ import torch
 import oracle
 import synth
 from pins import (E2M1_VALUES, affine_values_f64, bitwise_pack, bitwise_unpack, group_sq_error_f64,
-                  mse_candidate_bounds, mxfp4_values_f64, numpy_mxfp4_quantize, numpy_quantize, numpy_quantize_mse,
-                  page_pack, page_unpack)
+                  e4m3_all_values, mse_candidate_bounds, mxfp4_values_f64, numpy_mxfp4_quantize, numpy_nvfp4_quantize,
+                  numpy_quantize, numpy_quantize_mse, page_pack, page_unpack)
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 BITS = (2, 3, 4, 8)
@@ -47,6 +47,11 @@ def _range_search_groups():
 def _mxfp4_groups():
     with open(os.path.join(GOLDEN, "mxfp4_groups.json")) as f:
         return json.load(f)["groups"]
+
+
+def _nvfp4_tensors():
+    with open(os.path.join(GOLDEN, "nvfp4_groups.json")) as f:
+        return json.load(f)["tensors"]
 
 
 def _storage():
@@ -425,6 +430,65 @@ def test_mxfp4_dequantize_and_matmul():
 
 
 # --------------------------------------------------------------------------
+# nvfp4 (E2M1 codes, E4M3 scale per 16 along K, fp32 scale per tensor)
+# --------------------------------------------------------------------------
+
+def _nv_weights(N, K, seed):
+    w = synth.weights(N, K, seed=seed)
+    w[0, :16] = 0.0                                  # zero block
+    w[1, 16:32] *= np.float32(1e-5)                  # subnormal E4M3 block scales
+    w[2, :] = -np.abs(w[2, :])
+    return w
+
+
+def _nv_values_f64(codes, scales, g):
+    sv = np.repeat(e4m3_all_values()[scales.astype(np.int64)], 16, axis=-1)
+    return E2M1_VALUES[codes.astype(np.int64)] * sv * g
+
+
+@pytest.mark.parametrize("tz", _nvfp4_tensors(), ids=lambda tz: tz["name"])
+def test_nvfp4_hand_tensor(tz):
+    w = np.array([float(s) for s in tz["w"]], dtype=np.float64).astype(np.float32)[None, :]
+    p, s, g = oracle.nvfp4_quantize(w)
+    assert g == float(tz["tensor_scale"])
+    assert [int(x) for x in s[0]] == [int(x, 16) for x in tz["scales_e4m3"]]
+    assert [int(x) for x in p[0]] == [int(x, 16) for x in tz["packed"]]
+    assert oracle.unpack_codes(p, tz["K"], 4)[0].tolist() == tz["codes"]
+
+
+def test_nvfp4_matches_numpy():
+    for seed in (21, 22):
+        w = _nv_weights(24, 1024, seed)
+        p, s, g = oracle.nvfp4_quantize(w)
+        p2, s2, g2, _ = numpy_nvfp4_quantize(w)
+        assert np.array_equal(p, p2) and np.array_equal(s, s2) and g == g2
+
+
+def test_nvfp4_e4m3_decoding_and_dequantize():
+    """E4M3 values are those of the format definition (a few checked by hand:
+    byte 0x7E = 448, 0x38 = 1, 0x08 = 2^-6, 0x01 = 2^-9), and dequantized weights
+    are fp32(fp32(e2m1 * scale) * g) exactly."""
+    v = e4m3_all_values()
+    assert v[0x7E] == 448.0 and v[0x38] == 1.0 and v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9
+    assert (np.diff(v) > 0).all()                      # bytes 0..126 increase strictly
+    w = _nv_weights(8, 256, 23)
+    p, s, g = oracle.nvfp4_quantize(w)
+    codes = bitwise_unpack(p, 256, 4)
+    sv = np.repeat(v[s.astype(np.int64)], 16, axis=-1)
+    expect = ((E2M1_VALUES[codes.astype(np.int64)] * sv).astype(np.float32) * np.float32(g)).astype(np.float32)
+    assert np.array_equal(oracle.nvfp4_dequantize_f32(p, s, g, 256), expect)
+
+
+def test_nvfp4_matmul_equals_dequantize_then_matmul():
+    w = _nv_weights(8, 256, 24)
+    p, s, g = oracle.nvfp4_quantize(w)
+    x = synth.activations(3, 256, seed=25)
+    y = oracle.nvfp4_matmul(synth.bf16_bits(x), p, s, g)
+    ref = x.to(torch.float64).numpy() @ _nv_values_f64(bitwise_unpack(p, 256, 4), s, g).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
 # Dequantize
 # --------------------------------------------------------------------------
 
@@ -551,6 +615,9 @@ MUTATIONS = {
     "mx_scale_bias_128": ("static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 127); }",
                           "static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 128); }"),
     "mx_magnitude_table_swapped": ("{0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0}", "{0.0, 0.5, 1.0, 1.5, 2.0, 4.0, 3.0, 6.0}"),
+    "nv_tensor_scale_448": ("return amax > 0.0f ? amax / 2688.0f : 1.0f;", "return amax > 0.0f ? amax / 448.0f : 1.0f;"),
+    "nv_elements_from_unrounded_scale": ("const float denom = (float)e4m3_value(sb) * g;", "const float denom = s32 * g;"),
+    "nv_e4m3_exponent_bias_8": ("return ldexp(8.0 + m, e - 10);", "return ldexp(8.0 + m, e - 11);"),
 }
 
 
@@ -606,6 +673,26 @@ def _pins_pass(o: "oracle.Oracle") -> bool:
         p, s = o.mxfp4_quantize(w)
         p2, s2, _ = numpy_mxfp4_quantize(w)
         if not (np.array_equal(p, p2) and np.array_equal(s, s2)):
+            return False
+        for tz in _nvfp4_tensors():
+            w = np.array([float(s) for s in tz["w"]], dtype=np.float64).astype(np.float32)[None, :]
+            p, s, g = o.nvfp4_quantize(w)
+            if [int(x) for x in s[0]] != [int(x, 16) for x in tz["scales_e4m3"]]:
+                return False
+            if [int(x) for x in p[0]] != [int(x, 16) for x in tz["packed"]]:
+                return False
+        w = _nv_weights(8, 256, 14)
+        w[3, :16] = np.float32(5.0)                  # a block whose scale saturates at 448 (amax / 6g > 448)
+        w[3, 0] = np.float32(-40000.0)
+        p, s, g = o.nvfp4_quantize(w)
+        p2, s2, g2, _ = numpy_nvfp4_quantize(w)
+        if not (np.array_equal(p, p2) and np.array_equal(s, s2) and g == g2):
+            return False
+        x = synth.activations(2, 256, seed=15)
+        y = o.nvfp4_matmul(synth.bf16_bits(x), p, s, g)
+        sv = np.repeat(e4m3_all_values()[s.astype(np.int64)], 16, axis=-1)
+        ref = x.to(torch.float64).numpy() @ (E2M1_VALUES[bitwise_unpack(p, 256, 4).astype(np.int64)] * sv * g).T
+        if not np.allclose(y, ref, rtol=1e-12, atol=1e-12):
             return False
         return True
     except ValueError:
