@@ -431,6 +431,24 @@ def section_mxfp4(args, aq, torch, dev, stream, peaks):
                                        "kernel": "qmv_tc_kernel<4,32,1,mxfp4> (mma.sync m16n8k32, codes split by sign)"}
         del qs, base
         torch.cuda.empty_cache()
+    # nvfp4: E4M3 scale per 16 + tensor scale (bytes N*K/2 + N*K/16)
+    for (K, N) in ((4096, 14336), (8192, 28672)):
+        w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 6 + 3 + K % 7)).to(dev)
+        base = aq.aq_nvfp4_quantize(w)
+        del w
+        wb = N * K // 2 + N * K // 16
+        copies = max(2, -(-2 * L2_BYTES // wb) + 1)
+        qs = [base] + [tuple(t.clone() for t in base) for _ in range(copies - 1)]
+        x = x_cache.setdefault(K, synth.activations(1, K, 17).to(dev))
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_nvfp4_matmul(x, *qs[i % copies], out=y, overlap_previous=True),
+                         copies * 4, 20)
+        gbs = wb / (ms * 1e-3) / 1e9
+        out[f"nvfp4_qmv_K{K}_N{N}"] = {"us": round(ms * 1e3, 3), "weight_GBps": round(gbs, 1),
+                                       "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                       "kernel": "qmv_tc_kernel<4,32,1,nvfp4> (two 16-groups per MMA K step)"}
+        del qs, base
+        torch.cuda.empty_cache()
     return out
 
 

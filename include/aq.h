@@ -301,6 +301,47 @@ aq_status aq_mxfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales,
 aq_status aq_mxfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
                           const uint8_t *scales, int64_t N, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
 
+/* ---- nvfp4: fp4 with E4M3 block scales and a tensor scale ------------------
+ * Source: ExecuTorch "MLX backend — Quantization" (the NVFP4 weight-only
+ * config, group size 16) and "Quantizing a Model for MLX", section "Modes, bits
+ * and mixed recipes" (nvfp4: groups of 16, 4 bits).  The pages leave the
+ * encodings open; these follow NVIDIA's NVFP4 format:
+ *  - packed: uint32 [N, K/8], E2M1 codes as for mxfp4;
+ *  - scales: uint8 [N, K/16], E4M3 (sign 0, exponent bits 6..3 with bias 7,
+ *    mantissa bits 2..0, subnormals m * 2^-9, largest 448);
+ *  - tensor_scale: one device fp32 g;
+ *  - w ~= e2m1(code) * scale * g.
+ * Quantize: g = fp32(max|w| / 2688) over the whole tensor (1 if it is all
+ * zero); block byte = E4M3 nearest to fp32(amax_block / fp32(6 * g)), ties to
+ * even, saturating at 448; element = E2M1 nearest to fp32(|w| / fp32(scale *
+ * g)), ties to the even code, sign only on a non-zero magnitude; a zero block
+ * scale gives code 0.  Bit-exact with that definition.  Dequantized value:
+ * fp32(fp32(e2m1 * scale) * g).  K must be a multiple of 32; packed, scales and
+ * outputs 16-byte aligned, tensor_scale 4-byte aligned.  Inputs must be finite. */
+
+/* Bytes of codes + scales + tensor scale: N*K/2 + N*K/16 + 4; 0 if invalid. */
+size_t aq_nvfp4_packed_bytes(int64_t N, int64_t K);
+
+/* Quantize fp32 W[N, K] (device); writes packed, scales and *tensor_scale (device). */
+aq_status aq_nvfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
+                            float *tensor_scale, aq_stream_t stream);
+
+/* Dequantize to bf16 (RNE of the fp32 value) or fp32 [N, K]. */
+aq_status aq_nvfp4_dequantize(const uint32_t *packed, const uint8_t *scales, const float *tensor_scale, int64_t N,
+                              int64_t K, uint16_t *w_out_bf16, aq_stream_t stream);
+aq_status aq_nvfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales, const float *tensor_scale,
+                                  int64_t N, int64_t K, float *w_out, aq_stream_t stream);
+
+/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device) for decode, M <= 4, on the
+ * integer tensor cores: one MMA K step spans two 16-weight groups, whose halves
+ * feed two accumulator columns; each column is folded with its E4M3 scale and
+ * the output multiplied by g.  Supported: M <= 4, N >= 16, K a multiple of 256
+ * (others -> AQ_ERR_UNSUPPORTED).  flags: 0 or AQ_MATMUL_OVERLAP_PREVIOUS.
+ * Accuracy as aq_matmul. */
+aq_status aq_nvfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
+                          const uint8_t *scales, const float *tensor_scale, int64_t N, uint16_t *y_bf16,
+                          uint32_t flags, aq_stream_t stream);
+
 /* Bits of the device fault word. */
 enum {
   AQ_FAULT_WAIT_MASK = 0x1Fu, /* bits 0-4: a kernel gave up a bounded wait and returned early */

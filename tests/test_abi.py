@@ -227,3 +227,18 @@ def test_mxfp4_validation():
     assert mm(flags=2) == aq.AQ_ERR_INVALID_ARG
     assert mm(x=U) == aq.AQ_ERR_ALIGNMENT
     assert mm(M=0) == aq.AQ_ERR_INVALID_ARG
+
+
+def test_nvfp4_validation():
+    L = aq.lib()
+    assert aq.aq_nvfp4_packed_bytes(4096, 4096) == 4096 * 4096 // 2 + 4096 * 4096 // 16 + 4
+    assert L.aq_nvfp4_quantize(A, 4, 48, A, A, A, None) == aq.AQ_ERR_INVALID_ARG     # K % 32
+    assert L.aq_nvfp4_quantize(A, 4, 64, A, A, 0, None) == aq.AQ_ERR_INVALID_ARG     # no tensor scale
+    assert L.aq_nvfp4_quantize(A, 4, 64, A, A, A + 2, None) == aq.AQ_ERR_ALIGNMENT
+    assert L.aq_nvfp4_dequantize(A, U, A, 4, 64, A, None) == aq.AQ_ERR_ALIGNMENT
+    mm = lambda M=1, K=512, N=16, flags=0: L.aq_nvfp4_matmul(A, M, K, A, A, A, N, A, flags, None)
+    assert mm(M=5) == aq.AQ_ERR_UNSUPPORTED        # two group slots per token: M <= 4
+    assert mm(K=208) == aq.AQ_ERR_INVALID_ARG      # K % 32 != 0
+    assert mm(K=288) == aq.AQ_ERR_UNSUPPORTED      # the decode kernel needs K % 256 == 0
+    assert mm(N=8) == aq.AQ_ERR_UNSUPPORTED
+    assert mm(flags=4) == aq.AQ_ERR_INVALID_ARG

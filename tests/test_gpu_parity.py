@@ -317,6 +317,73 @@ def test_mxfp4_matmul_llama_shapes_sampled(K, N):
     _assert_close(y[:, torch.from_numpy(cols).cuda()], y_ref, f"mxfp4 {K}x{N} sampled", rms=rms)
 
 
+# ----------------------------------------------------------------------------- nvfp4
+
+def _nv_special(N, K, seed):
+    w = weights(N, K, seed, True).copy()
+    w[0, :16] = 0.0
+    w[1 % N, 16:32] *= np.float32(1e-5)             # subnormal E4M3 block scales
+    w[2 % N, :] = -np.abs(w[2 % N, :])
+    return w
+
+
+@pytest.mark.parametrize("N,K,seed", [(8, 128, 51), (37, 1024, 52), (256, 4096, 53)])
+def test_nvfp4_quantize_dequantize_bitexact(N, K, seed):
+    w = _nv_special(N, K, seed)
+    p_ref, s_ref, g_ref = oracle.nvfp4_quantize(w)
+    p, s, g = aq.aq_nvfp4_quantize(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert float(g.cpu()[0]) == g_ref
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(_u32(p), p_ref)
+    f_ref = oracle.nvfp4_dequantize_f32(p_ref, s_ref, g_ref, K)
+    f = aq.aq_nvfp4_dequantize(p, s, g, K, fp32=True)
+    assert np.array_equal(f.cpu().numpy().view(np.uint32), f_ref.view(np.uint32))
+    b = aq.aq_nvfp4_dequantize(p, s, g, K)
+    assert np.array_equal(_u16(b), oracle.bf16_round(f_ref))
+
+
+def _nv_gpu(w):
+    p_ref, s_ref, g_ref = oracle.nvfp4_quantize(w)
+    return (p_ref, s_ref, g_ref, torch.from_numpy(p_ref.view(np.int32)).cuda(), torch.from_numpy(s_ref).cuda(),
+            torch.tensor([g_ref], dtype=torch.float32).cuda())
+
+
+@pytest.mark.parametrize("M", (1, 2, 3, 4))
+@pytest.mark.parametrize("K,N", [(256, 16), (1024, 100), (4096, 600), (2560, 2600)])
+def test_nvfp4_matmul_matches_oracle(M, K, N):
+    w = weights(N, K, 60 + K + N, True)
+    p_ref, s_ref, g_ref, p, s, g = _nv_gpu(w)
+    xb = activations_bits(M, K, 61 + M)
+    y = aq.aq_nvfp4_matmul(_x_gpu(xb), p, s, g)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.nvfp4_matmul(xb, p_ref, s_ref, g_ref), f"nvfp4 M={M} K={K} N={N}")
+
+
+def test_nvfp4_matmul_special_weights_and_overlap():
+    w = _nv_special(64, 1024, 65)
+    p_ref, s_ref, g_ref, p, s, g = _nv_gpu(w)
+    xb = activations_bits(4, 1024, 66)
+    y0 = aq.aq_nvfp4_matmul(_x_gpu(xb), p, s, g)
+    y1 = aq.aq_nvfp4_matmul(_x_gpu(xb), p, s, g, overlap_previous=True)
+    torch.cuda.synchronize()
+    _assert_close(y0, oracle.nvfp4_matmul(xb, p_ref, s_ref, g_ref), "nvfp4 special weights")
+    assert torch.equal(y0, y1)
+
+
+def test_nvfp4_matmul_llama_shape_sampled():
+    K, N = 4096, 14336
+    w = weights(N, K, 1202, True)
+    p_ref, s_ref, g_ref, p, s, g = _nv_gpu(w)
+    xb = activations_bits(1, K, 67)
+    y = aq.aq_nvfp4_matmul(_x_gpu(xb), p, s, g)
+    torch.cuda.synchronize()
+    cols = sample_rows(N, 300, seed=68)
+    y_ref = oracle.nvfp4_matmul(xb, p_ref[cols], s_ref[cols], g_ref)
+    _assert_close(y[:, torch.from_numpy(cols).cuda()], y_ref, "nvfp4 4096x14336 sampled",
+                  rms=float(np.sqrt(np.mean(y_ref ** 2))))
+
+
 # ----------------------------------------------------------------------------- QMV (decode)
 
 def _matmul_case(M, K, N, bits, G, seed, kernel, outl=True, full=True, n_rows=48):

@@ -1,5 +1,7 @@
-// mxfp4 quantize and dequantize: block-scaled fp4, one E8M0 exponent per 32
-// weights along K, 4-bit E2M1 codes packed 8 per uint32 (LSB first).
+// mxfp4 and nvfp4 quantize and dequantize (block-scaled fp4).
+//
+// mxfp4: one E8M0 exponent per 32 weights along K, 4-bit E2M1 codes packed 8
+// per uint32 (LSB first).
 //
 // Mode: "metalworking — MLX Quantization" (the newer block-scaled modes, mxfp4
 // with groups of 32) and "Quantizing a Model for MLX", section "Modes, bits and
@@ -13,6 +15,10 @@
 // nearest to |w| / X, ties to the even code, saturating at 6; the sign bit is
 // set only on a non-zero magnitude.  One thread per group (32 weights), as in
 // the affine quantizer.
+#include <cuda_fp8.h>
+
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace aq {
@@ -104,7 +110,137 @@ __global__ void __launch_bounds__(256) mxfp4_dequantize_kernel(const uint32_t *_
   }
 }
 
+// ---- nvfp4 ("ExecuTorch MLX backend — Quantization": NVFP4 weight-only config,
+// groups of 16; "Quantizing a Model for MLX", "Modes, bits and mixed recipes").
+// Encodings as read from NVIDIA's NVFP4: E2M1 codes as above; one E4M3 byte per
+// 16 weights; one fp32 tensor scale g = amax / 2688 (6 * 448), 1 for an
+// all-zero tensor.  Block byte: E4M3 nearest to fp32(amax_block / fp32(6 g)),
+// ties to even, saturating at 448.  Element: E2M1 nearest to
+// fp32(|w| / fp32(scale * g)), ties to the even code; a zero block scale gives
+// code 0.  Value: fp32(fp32(e2m1 * scale) * g).
+
+// Value of an E4M3 byte (sign 0 here), exact in fp32.
+AQ_DEVICE float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  return e == 0u ? __uint_as_float(0x3B000000u) * static_cast<float>(m)   // m * 2^-9
+                 : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// max |w| over the tensor into *amax_bits (the bits of a non-negative float,
+// zeroed before the launch: integer order equals float order there).
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const float4 *__restrict__ w, int64_t n4,
+                                                         uint32_t *__restrict__ amax_bits) {
+  float m = 0.0f;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += int64_t(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(w + i);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+// The tensor scale from the amax held in the same word.
+__global__ void nvfp4_tensor_scale_kernel(float *gscale) {
+  const float amax = *gscale;
+  *gscale = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// One thread per block of 16 weights.
+__global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const float *__restrict__ w, int64_t blocks,
+                                                             const float *__restrict__ gscale,
+                                                             uint32_t *__restrict__ packed, uint8_t *__restrict__ scales) {
+  const int64_t bi = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (bi >= blocks) return;
+  const float g = __ldg(gscale);
+  float v[16];
+  const float4 *src = reinterpret_cast<const float4 *>(w + bi * 16);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 t = __ldg(src + i);
+    v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float s32 = __fdiv_rn(amax, __fmul_rn(6.0f, g));
+  const uint32_t sb = static_cast<uint32_t>(__nv_cvt_float_to_fp8(s32, __NV_SATFINITE, __NV_E4M3));
+  const float denom = __fmul_rn(e4m3_value(sb), g);
+  uint32_t out[2] = {0u, 0u};
+  if (sb != 0u) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t mag = e2m1_magnitude_code(__fdiv_rn(fabsf(v[j]), denom));
+      const uint32_t code = mag | ((v[j] < 0.0f && mag != 0u) ? 8u : 0u);
+      out[j / 8] |= code << (4 * (j % 8));
+    }
+  }
+  reinterpret_cast<uint2 *>(packed)[bi] = make_uint2(out[0], out[1]);
+  scales[bi] = static_cast<uint8_t>(sb);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) nvfp4_dequantize_kernel(const uint32_t *__restrict__ packed,
+                                                               const uint8_t *__restrict__ scales,
+                                                               const float *__restrict__ gscale, int64_t blocks,
+                                                               void *__restrict__ out) {
+  const int64_t bi = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (bi >= blocks) return;
+  const uint2 wv = ldg_nc8(packed + bi * 2);
+  const uint32_t words[2] = {wv.x, wv.y};
+  const float sv = e4m3_value(__ldg(scales + bi)), g = __ldg(gscale);
+  constexpr float kMag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  float v[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t c = (words[j / 8] >> (4 * (j % 8))) & 0xFu;
+    const float m = __fmul_rn(__fmul_rn(kMag[c & 7u], sv), g);
+    v[j] = (c & 8u) ? -m : m;
+  }
+  if constexpr (BF16) {
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + bi * 16);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      uint32_t u[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
+        u[k] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+      dst[i] = make_uint4(u[0], u[1], u[2], u[3]);
+    }
+  } else {
+    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + bi * 16);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_nvfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
+                                  float *gscale, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(gscale, 0, sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  const int64_t n4 = N * K / 4;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 148 * 8));
+  nvfp4_amax_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4 *>(w), n4, reinterpret_cast<uint32_t *>(gscale));
+  nvfp4_tensor_scale_kernel<<<1, 1, 0, s>>>(gscale);
+  const int64_t blocks = N * K / 16;
+  nvfp4_quantize_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0, s>>>(w, blocks, gscale, packed, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_dequantize(const uint32_t *packed, const uint8_t *scales, const float *gscale, int64_t N,
+                                    int64_t K, void *out, bool bf16_out, cudaStream_t s) {
+  const int64_t blocks = N * K / 16;
+  const unsigned grid = static_cast<unsigned>((blocks + 255) / 256);
+  if (bf16_out)
+    nvfp4_dequantize_kernel<true><<<grid, 256, 0, s>>>(packed, scales, gscale, blocks, out);
+  else
+    nvfp4_dequantize_kernel<false><<<grid, 256, 0, s>>>(packed, scales, gscale, blocks, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_mxfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
                                   cudaStream_t s) {

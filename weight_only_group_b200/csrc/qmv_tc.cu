@@ -87,13 +87,14 @@ struct LaneWords {
 // A register set s (s = 0: MMA k 4t..4t+3, s = 1: k 16+4t..16+4t+3) of the
 // lane's K tile c (32 codes).  hh: the half of a shared word that a lane of a
 // 2-bit, G = 32 pair owns (t & 1).
-// FMT 1 (mxfp4, 4-bit, G = 32): register set s holds codes 4s..4s+3 of the lane's word.
+// FMT 1, 2 (mxfp4, nvfp4; 4-bit codes, 32-code spans): register set s holds
+// codes 4s..4s+3 of the lane's word.
 template <int BITS, int G, int FMT = 0>
 struct LaneSpan {
   static constexpr int length = (BITS == 2 && G == 32) ? 16 : G / 4;
   AQ_DEVICE static int start(int t) { return (BITS == 2 && G == 32) ? 16 * (t >> 1) : t * (G / 4); }
   __host__ __device__ static constexpr int index(int c, int s, int i, int hh) {
-    return FMT == 1    ? 8 * c + 4 * s + i
+    return FMT >= 1    ? 8 * c + 4 * s + i
            : BITS == 4 ? 8 * c + 2 * i + s
            : BITS == 8 ? 4 * (2 * c + s) + i
            : G >= 64   ? 16 * (c >> 1) + 2 * (c & 1) + s + 4 * i
@@ -177,6 +178,15 @@ AQ_DEVICE void e2m1x2_split(uint32_t w, uint32_t (&pos)[2], uint32_t (&neg)[2]) 
   neg[1] = prmt(kLo, kHi, wn >> 16);
 }
 
+// Half of an E4M3 scale byte's value (sign 0, exponent bits 6..3 with bias 7,
+// mantissa bits 2..0; subnormals m * 2^-9; 0x7F is NaN).
+AQ_DEVICE float e4m3_half(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  if (b == 0x7Fu) return __uint_as_float(0x7FC00000u);
+  return e == 0u ? __uint_as_float(0x3A800000u) * static_cast<float>(m)   // m * 2^-10
+                 : __uint_as_float(((e + 119u) << 23) | (m << 20));
+}
+
 // X / 2 of an E8M0 scale byte (X = 2^(s - 127); the MMA sees values doubled).
 AQ_DEVICE float e8m0_half(uint32_t sb) {
   return sb >= 2u ? (sb == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float((sb - 1u) << 23))
@@ -221,6 +231,7 @@ struct Args {
   // the [E*N, K] maps); each of its cta_per_tok CTAs owns a slice of the N rows
   const int32_t *experts;
   int E, cta_per_tok;
+  const float *gscale;  // nvfp4: the tensor scale (device), applied to every output
 };
 
 template <int BITS, int G, int MP, int FMT>
@@ -232,7 +243,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   constexpr int NWD = LaneWords<BITS, G>::count;
   constexpr int GBYTES = G * BITS / 8;           // packed bytes of one group row
   constexpr int SL = LaneSpan<BITS, G, FMT>::length;
-  static_assert(FMT == 0 || (BITS == 4 && G == 32), "mxfp4: 4-bit codes, groups of 32");
+  static_assert(FMT == 0 || (BITS == 4 && G == 32), "mxfp4 / nvfp4: 4-bit codes in 32-code spans");
+  // nvfp4: a 32-code span holds two 16-weight groups, fed to two columns of one MMA
+  static_assert(FMT != 2 || MP <= 4, "nvfp4 needs two group slots per token");
   // accumulator chains per digit plane: a group folded on its own has only
   // G/32 MMAs per plane, and summing chains would cost more than it hides
   constexpr int NACC = GS == 1 ? 1 : kAcc;
@@ -461,7 +474,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   const uint8_t *xs_lane = xs + (my_real ? my_m : 0) * a.tok_stride + t * 16;
   const uint8_t *zero_lane = zero + (GS == 1 ? 0 : (my_m & 1)) * a.zero_stride + t * 16;
   const int lw0 = LaneWords<BITS, G>::first(t) * 4;
-  const int nper = a.Kc / (GS * G);
+  constexpr int SPANS = FMT == 2 ? GS / 2 : GS;  // 32-code spans (MMA K steps) per fold
+  const int nper = a.Kc / (SPANS * G);
+  const float gs = FMT == 2 ? __ldg(a.gscale) : 1.0f;
 
   for (int st = cw; st < nst; st += a.W) {
     const int s = st % a.NS;
@@ -481,26 +496,29 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     for (int p = 0; p < nper; ++p) {
       int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
       // mxfp4: the same sums over the negative codes' magnitudes, subtracted below
-      int nl[FMT == 1 ? NACC : 1][4], nh[FMT == 1 ? NACC : 1][4];
+      int nl[FMT >= 1 ? NACC : 1][4], nh[FMT >= 1 ? NACC : 1][4];
 #pragma unroll
       for (int i = 0; i < NACC; ++i) dl[i][0] = dl[i][1] = dl[i][2] = dl[i][3] = dh[i][0] = dh[i][1] = dh[i][2] = dh[i][3] = 0;
-      if constexpr (FMT == 1) {
+      if constexpr (FMT >= 1) {
 #pragma unroll
         for (int i = 0; i < NACC; ++i) nl[i][0] = nl[i][1] = nl[i][2] = nl[i][3] = nh[i][0] = nh[i][1] = nh[i][2] = nh[i][3] = 0;
       }
-      static_for<0, GS>([&](auto J) {
+      static_for<0, SPANS>([&](auto J) {
         constexpr int j = J.value;
-        const int gi = p * GS + j;
+        const int gi = p * SPANS + j;
         uint32_t w0[NWD], w1[NWD];
         lds_words<NWD>(wr0 + gi * GBYTES, w0);
         lds_words<NWD>(wr1 + gi * GBYTES, w1);
-        const uint8_t *bp = (my_real && my_j == j) ? xs_lane + (gch0 + gi) * (U * 64) : zero_lane;
+        // nvfp4: the span's first 16 codes (lanes t = 0, 1) go to slot 2j, the
+        // other 16 (t = 2, 3) to slot 2j + 1
+        const bool live = my_real && (FMT == 2 ? my_j == 2 * j + (t >> 1) : my_j == j);
+        const uint8_t *bp = live ? xs_lane + (gch0 + gi) * (U * 64) : zero_lane;
         static_for<0, U>([&](auto C) {
           constexpr int c = C.value;
           const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);  // lo set 0, lo set 1, hi set 0, hi set 1
           uint32_t q0[2], q1[2];
           constexpr int k = (j * U + c) % NACC;
-          if constexpr (FMT == 1) {
+          if constexpr (FMT >= 1) {
             uint32_t n0[2], n1[2];
             e2m1x2_split(w0[0], q0, n0);
             e2m1x2_split(w1[0], q1, n1);
@@ -525,7 +543,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           lo += dl[c][i];
           hi += dh[c][i];
         }
-        if constexpr (FMT == 1) {
+        if constexpr (FMT >= 1) {
 #pragma unroll
           for (int c = 0; c < NACC; ++c) {
             lo -= nl[c][i];
@@ -541,7 +559,13 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       if constexpr (GS >= 2) {
         const int gl = p * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
         const int mt = (2 * t) / GS;
-        if constexpr (FMT == 1) {  // two E8M0 bytes per row (groups gl, gl + 1); no bias
+        if constexpr (FMT == 2) {  // two E4M3 bytes per row (16-groups gl, gl + 1, one span); no bias
+          const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
+          const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
+          s0 = make_float2(e4m3_half(e0 & 0xFFu), e4m3_half(e0 >> 8));
+          s1 = make_float2(e4m3_half(e1 & 0xFFu), e4m3_half(e1 >> 8));
+          b0 = b1 = make_float2(0.0f, 0.0f);
+        } else if constexpr (FMT == 1) {  // two E8M0 bytes per row (groups gl, gl + 1); no bias
           const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
           const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
           s0 = make_float2(e8m0_half(e0 & 0xFFu), e8m0_half(e0 >> 8));
@@ -553,8 +577,12 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
           b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
         }
-        T0 = tab[mt * a.Gn + gch0 + gl];
-        T1 = tab[mt * a.Gn + gch0 + gl + 1];
+        if constexpr (FMT == 2) {  // both columns lie in span gl / 2 of the chunk
+          T0 = T1 = tab[mt * a.Gn + gch0 + gl / 2];
+        } else {
+          T0 = tab[mt * a.Gn + gch0 + gl];
+          T1 = tab[mt * a.Gn + gch0 + gl + 1];
+        }
       } else {
         const int gl = p;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
         float sv0, sv1, bv0 = 0.0f, bv1 = 0.0f;
@@ -617,8 +645,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const int tok = (2 * t) / GS;
         if (direct) {
           if (tok < a.M) {
-            if (row_ok(g)) yg[static_cast<int64_t>(tok) * a.N + rb + g] = __float2bfloat16_rn(v[0]);
-            if (row_ok(g + 8)) yg[static_cast<int64_t>(tok) * a.N + rb + g + 8] = __float2bfloat16_rn(v[1]);
+            if (row_ok(g)) yg[static_cast<int64_t>(tok) * a.N + rb + g] = __float2bfloat16_rn(FMT == 2 ? v[0] * gs : v[0]);
+            if (row_ok(g + 8))
+              yg[static_cast<int64_t>(tok) * a.N + rb + g + 8] = __float2bfloat16_rn(FMT == 2 ? v[1] * gs : v[1]);
           }
         } else {
           dstv[g * MP + tok] = v[0];
@@ -659,7 +688,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const int row = idx / MP, tok = idx - row * MP;
         float sum = 0.0f;
         for (int c2 = 0; c2 < a.nch; ++c2) sum += rbuf[(static_cast<size_t>(c2) * kRows + row) * MP + tok];
-        if (tok < a.M && row_ok(row)) yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(sum);
+        if (tok < a.M && row_ok(row))
+          yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(FMT == 2 ? sum * gs : sum);
       }
       __syncwarp();
       if (lane == 0) {
@@ -698,12 +728,15 @@ static int64_t code_pitch(int64_t row_bytes, int bits, int G) {
 }
 
 // fmt 0: affine codes with fp16 scales and biases; fmt 1: mxfp4 (E2M1 codes,
-// one E8M0 byte per 32, no biases).
+// one E8M0 byte per 32, no biases); fmt 2: nvfp4 (E2M1 codes, one E4M3 byte per
+// 16, i.e. two per 32-code span, a tensor scale, no biases; M <= 4).
 static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt = 0) {
   if (!(bits == 2 || bits == 4 || bits == 8) || !(G == 32 || G == 64 || G == 128)) return false;
   if (M < 1 || M > 8 || N < 1 || K < 1 || K % (8 * G) != 0) return false;
   // mxfp4 scale rows are K/32 bytes: a TMA row stride must be a multiple of 16 bytes
   if (fmt == 1 && (bits != 4 || G != 32 || K % 512 != 0)) return false;
+  // nvfp4 scale rows are K/16 bytes
+  if (fmt == 2 && (bits != 4 || G != 32 || K % 256 != 0 || M > 4)) return false;
   if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 30)) return false;
   if (N < kRows) return false;  // every CTA owns at least one whole 16-row tile
   const int MP = pow2_tokens(static_cast<int>(M));
@@ -723,6 +756,7 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.experts = nullptr;
   a.E = 1;
   a.cta_per_tok = 0;
+  a.gscale = nullptr;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.K = static_cast<int>(K);
@@ -730,7 +764,7 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.Kc = static_cast<int>(Kc);
   a.nch = static_cast<int>(nch);
   a.pitch_w = static_cast<int>(code_pitch(Kc * bits / 8, bits, G));
-  const int sbytes = fmt == 1 ? 1 : 2;  // bytes of one group's scale
+  const int sbytes = fmt == 1 ? 1 : 2;  // scale bytes per 32-code span (nvfp4: two E4M3 bytes)
   a.pitch_s = static_cast<int>(pitch_at(gpc * sbytes, 32, 16));
   if (a.pitch_w / 8 > 256 || a.pitch_s / 8 > 256) return false;  // TMA box width (64-bit elements)
   a.w_box_x = static_cast<int>(Kc * bits / 64);
@@ -739,7 +773,7 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   if (nch > 1 && (a.w_box_x % 2 != 0 || a.sb_box_x % 2 != 0)) return false;
   a.s_off = kRows * a.pitch_w;
   a.b_off = a.s_off + kRows * a.pitch_s;
-  a.stage_bytes = static_cast<int>(round_up((fmt == 1 ? a.s_off : a.b_off) + kRows * a.pitch_s, 128));
+  a.stage_bytes = static_cast<int>(round_up((fmt >= 1 ? a.s_off : a.b_off) + kRows * a.pitch_s, 128));
   a.tok_stride = static_cast<int>(2 * K + 64);
   a.zero_stride = static_cast<int>(round_up(U * 64, 128) + 64);
   const int64_t budget = 227 * 1024;
@@ -967,6 +1001,44 @@ cudaError_t launch_mxfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
     return cudaErrorInvalidValue;
   mp.b = mp.s;  // no bias map: the kernel never reads this one
   return tc::launch_mp<4, 32, 1>(pl, mp, overlap, s);
+}
+
+bool nvfp4_tc_supported(int64_t M, int64_t N, int64_t K) {
+  tc::Plan pl;
+  return tc::make_plan(M, N, K, 32, 4, 148, pl, 2);
+}
+
+// nvfp4 (E2M1 codes packed 8 per word, one E4M3 byte per 16 along K, the fp32
+// tensor scale at gscale on the device).
+cudaError_t launch_nvfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
+                            const float *gscale, int64_t N, uint16_t *y, uint32_t flags, cudaStream_t s) {
+  static thread_local int cached_dev = -1, sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  tc::Plan pl;
+  if (!tc::make_plan(M, N, K, 32, 4, sms, pl, 2)) return cudaErrorInvalidValue;
+  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.packed = packed;
+  pl.a.scales = reinterpret_cast<const __half *>(scales);  // read as bytes by the nvfp4 kernel
+  pl.a.biases = nullptr;
+  pl.a.gscale = gscale;
+  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
+  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
+  tc::Maps mp;
+  if (!tc::encode_rows(&mp.w, packed, N, K / 2, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 16, pl.a.pitch_s))
+    return cudaErrorInvalidValue;
+  mp.b = mp.s;  // no bias map: the kernel never reads this one
+  switch (tc::pow2_tokens(pl.a.M)) {
+    case 1: return tc::launch<4, 32, 1, 2>(pl, mp, overlap, s);
+    case 2: return tc::launch<4, 32, 2, 2>(pl, mp, overlap, s);
+    default: return tc::launch<4, 32, 4, 2>(pl, mp, overlap, s);
+  }
 }
 
 cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word) {
