@@ -55,6 +55,9 @@ class Oracle:
         lib.oracle_mxfp4_dequantize_f32.argtypes = [vp, vp, i64, i64, vp]
         lib.oracle_mxfp4_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp]
         lib.oracle_mxfp4_matmul_sampled.argtypes = [vp, i64, i64, vp, vp, i64, vp, i64, vp, i64, vp]
+        lib.oracle_mxfp8_quantize.argtypes = [vp, i64, i64, vp, vp]
+        lib.oracle_mxfp8_dequantize_f32.argtypes = [vp, vp, i64, i64, vp]
+        lib.oracle_mxfp8_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp]
         lib.oracle_nvfp4_tensor_scale.argtypes = [vp, i64]
         lib.oracle_nvfp4_tensor_scale.restype = ctypes.c_float
         lib.oracle_nvfp4_quantize.argtypes = [vp, i64, i64, ctypes.c_float, vp, vp]
@@ -183,6 +186,34 @@ class Oracle:
                                                     _p(ni), len(ni), _p(y)), "mxfp4_matmul_sampled")
         return y
 
+    # ---- mxfp8 (E4M3 codes, E8M0 exponent per 32 along K)
+    def mxfp8_quantize(self, w: np.ndarray):
+        """w fp32 [N, K] -> (packed uint32 [N, K/4], scales uint8 [N, K/32])."""
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        N, K = w.shape
+        packed = np.zeros((N, K // 4), dtype=np.uint32)
+        scales = np.zeros((N, K // 32), dtype=np.uint8)
+        _check(self.lib.oracle_mxfp8_quantize(_p(w), N, K, _p(packed), _p(scales)), "mxfp8_quantize")
+        return packed, scales
+
+    def mxfp8_dequantize_f32(self, packed, scales, K: int) -> np.ndarray:
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        N = packed.shape[0]
+        out = np.zeros((N, K), dtype=np.float32)
+        _check(self.lib.oracle_mxfp8_dequantize_f32(_p(packed), _p(scales), N, K, _p(out)), "mxfp8_dequantize_f32")
+        return out
+
+    def mxfp8_matmul(self, x_bf16_bits, packed, scales) -> np.ndarray:
+        x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint8)
+        M, K = x.shape
+        N = packed.shape[0]
+        y = np.zeros((M, N), dtype=np.float64)
+        _check(self.lib.oracle_mxfp8_matmul(_p(x), M, K, _p(packed), _p(scales), N, _p(y)), "mxfp8_matmul")
+        return y
+
     # ---- nvfp4 (E2M1 codes, E4M3 scale per 16 along K, fp32 scale per tensor)
     def nvfp4_quantize(self, w: np.ndarray):
         """w fp32 [N, K] -> (packed uint32 [N, K/8], scales uint8 [N, K/16] E4M3, g float)."""
@@ -303,6 +334,18 @@ def mxfp4_matmul(x_bf16_bits, packed, scales):
 
 def mxfp4_matmul_sampled(x_bf16_bits, packed, scales, m_idx, n_idx):
     return default().mxfp4_matmul_sampled(x_bf16_bits, packed, scales, m_idx, n_idx)
+
+
+def mxfp8_quantize(w):
+    return default().mxfp8_quantize(w)
+
+
+def mxfp8_dequantize_f32(packed, scales, K):
+    return default().mxfp8_dequantize_f32(packed, scales, K)
+
+
+def mxfp8_matmul(x_bf16_bits, packed, scales):
+    return default().mxfp8_matmul(x_bf16_bits, packed, scales)
 
 
 def nvfp4_quantize(w):

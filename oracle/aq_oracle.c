@@ -25,6 +25,7 @@
  *  - "metalworking — MLX Quantization" (newer modes) and "Quantizing a Model
  *    for MLX", section "Modes, bits and mixed recipes": the mxfp4 block-scaled
  *    mode (oracle_mxfp4_*; encodings and readings beside them).
+ *  - the same two pages on mxfp8 (oracle_mxfp8_*; encodings beside them).
  *  - "ExecuTorch MLX backend — Quantization" (NVFP4 config) and "Quantizing a
  *    Model for MLX", section "Modes, bits and mixed recipes": the nvfp4 mode
  *    (oracle_nvfp4_*; encodings and readings beside them).
@@ -712,6 +713,95 @@ int oracle_nvfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint
                 acc += bf16_value(x_bf16[m * K + k]) * e2m1_value(get_code(packed + n * P, k, 4)) *
                        e4m3_value(scales[n * Gn + k / 16]);
             y[m * N + n] = acc * (double)g;
+        }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* mxfp8: E4M3 elements, one E8M0 exponent per 32                             */
+/* ------------------------------------------------------------------------ */
+
+/* "metalworking — MLX Quantization" (the newer modes: mxfp8 with groups of 32)
+ * and "Quantizing a Model for MLX", section "Modes, bits and mixed recipes"
+ * (mxfp8: groups of 32, 8 bits, an exponent per group).  Encodings as read from
+ * the OCP Microscaling v1.0 MXFP8 (E4M3) format:
+ *  - code byte: sign bit 7, then the E4M3 magnitude (exponent bits 6..3 with
+ *    bias 7, mantissa bits 2..0, subnormals m * 2^-9, largest 448); packed 4
+ *    per uint32, LSB first (as 8-bit affine codes);
+ *  - scale byte s: X = 2^(s - 127), as for mxfp4;
+ *  - quantize a group of 32: shared exponent floor(log2 amax) - 8 (8 = the
+ *    largest E4M3 exponent), clamped to [-127, 127]; an all-zero group gets
+ *    s = 0; each element the E4M3 magnitude nearest to |w| / X (exact in fp64),
+ *    ties to even, saturating at 448; sign only on a non-zero magnitude;
+ *  - value X * e4m3(code), exact in fp64 (rounded once to fp32 / bf16). */
+static double e4m3_signed_value(uint32_t c)
+{
+    double v = e4m3_value((uint8_t)(c & 0x7Fu));
+    return (c & 0x80u) ? -v : v;
+}
+
+int oracle_mxfp8_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales)
+{
+    if (!w || !packed || !scales || bad_mx_shape(N, K)) return ORACLE_BAD_ARG;
+    const int64_t P = K / 4, Gn = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        const float *wr = w + n * K;
+        uint32_t *pr = packed + n * P;
+        for (int64_t j = 0; j < P; j++) pr[j] = 0u;
+        for (int64_t g = 0; g < Gn; g++) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; i++) {
+                double a = fabs((double)wr[g * 32 + i]);
+                if (a > amax) amax = a;
+            }
+            int shared = -127;
+            if (amax > 0.0) {
+                int ex;
+                frexp(amax, &ex);           /* floor(log2 amax) = ex - 1 */
+                shared = (ex - 1) - 8;
+                if (shared < -127) shared = -127;
+                if (shared > 127) shared = 127;
+            }
+            scales[n * Gn + g] = (uint8_t)(shared + 127);
+            for (int i = 0; i < 32; i++) {
+                const double v = (double)wr[g * 32 + i];
+                uint32_t c = e4m3_bits_from_double(fabs(v) * ldexp(1.0, -shared));   /* exact product */
+                if (v < 0.0 && c != 0u) c |= 0x80u;
+                put_code(pr, g * 32 + i, 8, c);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+static double mx8_value(const uint32_t *prow, const uint8_t *srow, int64_t k)
+{
+    return e8m0_value(srow[k / 32]) * e4m3_signed_value(get_code(prow, k, 8));
+}
+
+int oracle_mxfp8_dequantize_f32(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K, float *out)
+{
+    if (!packed || !scales || !out || bad_mx_shape(N, K)) return ORACLE_BAD_ARG;
+    const int64_t P = K / 4, Gn = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t k = 0; k < K; k++) out[n * K + k] = (float)mx8_value(packed + n * P, scales + n * Gn, k);
+    return ORACLE_OK;
+}
+
+int oracle_mxfp8_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
+                        const uint8_t *scales, int64_t N, double *y)
+{
+    if (!x_bf16 || !packed || !scales || !y || M <= 0 || bad_mx_shape(N, K)) return ORACLE_BAD_ARG;
+    const int64_t P = K / 4, Gn = K / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t m = 0; m < M; m++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += bf16_value(x_bf16[m * K + k]) * mx8_value(packed + n * P, scales + n * Gn, k);
+            y[m * N + n] = acc;
         }
     return ORACLE_OK;
 }

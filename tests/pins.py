@@ -240,3 +240,27 @@ def numpy_nvfp4_quantize(w: np.ndarray):
     codes = np.where((sb == 0)[..., None], 0, codes)
     codes = np.where((wb < 0) & (codes != 0), codes | 8, codes).reshape(N, K).astype(np.uint32)
     return bitwise_pack(codes, 4), sb.astype(np.uint8), float(g), codes.astype(np.uint8)
+
+
+def numpy_mxfp8_quantize(w: np.ndarray):
+    """Independent NumPy statement of the mxfp8 quantizer: shared exponent from
+    frexp, each element the E4M3 magnitude nearest to |w| / X found by searching
+    all 127 values (ties to the even byte, saturating at 448 since 448 is the
+    largest), sign only on a non-zero magnitude."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    wg = w.reshape(N, K // 32, 32).astype(np.float64)
+    amax = np.abs(wg).max(axis=-1)
+    _, ex = np.frexp(amax)
+    shared = np.where(amax > 0, np.clip(ex - 1 - 8, -127, 127), -127)
+    t = np.abs(wg) * np.ldexp(1.0, -shared)[..., None]
+    vals = e4m3_all_values()
+    d = np.abs(t[..., None] - vals)
+    c = np.zeros(t.shape, dtype=np.int64)
+    best = d[..., 0].copy()
+    for b in range(1, 127):
+        better = (d[..., b] < best) | ((d[..., b] == best) & ((b & 1) == 0) & ((c & 1) == 1))
+        c = np.where(better, b, c)
+        best = np.where(better, d[..., b], best)
+    c = np.where((wg < 0) & (c != 0), c | 0x80, c).reshape(N, K).astype(np.uint32)
+    return bitwise_pack(c, 8), (shared + 127).astype(np.uint8), c.astype(np.uint8)

@@ -26,7 +26,8 @@ import torch
 import oracle
 import synth
 from pins import (E2M1_VALUES, affine_values_f64, bitwise_pack, bitwise_unpack, group_sq_error_f64,
-                  e4m3_all_values, mse_candidate_bounds, mxfp4_values_f64, numpy_mxfp4_quantize, numpy_nvfp4_quantize,
+                  e4m3_all_values, mse_candidate_bounds, mxfp4_values_f64, numpy_mxfp4_quantize, numpy_mxfp8_quantize,
+                  numpy_nvfp4_quantize,
                   numpy_quantize, numpy_quantize_mse, page_pack, page_unpack)
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
@@ -46,6 +47,11 @@ def _range_search_groups():
 
 def _mxfp4_groups():
     with open(os.path.join(GOLDEN, "mxfp4_groups.json")) as f:
+        return json.load(f)["groups"]
+
+
+def _mxfp8_groups():
+    with open(os.path.join(GOLDEN, "mxfp8_groups.json")) as f:
         return json.load(f)["groups"]
 
 
@@ -430,6 +436,50 @@ def test_mxfp4_dequantize_and_matmul():
 
 
 # --------------------------------------------------------------------------
+# mxfp8 (E4M3 codes, one E8M0 exponent per 32 along K)
+# --------------------------------------------------------------------------
+
+def _mx8_values_f64(codes, scales):
+    mag = e4m3_all_values()[(codes & 0x7F).astype(np.int64)]
+    X = np.repeat(np.ldexp(1.0, scales.astype(np.int64) - 127), 32, axis=-1)
+    return np.where(codes & 0x80, -mag, mag) * X
+
+
+@pytest.mark.parametrize("g", _mxfp8_groups(), ids=lambda g: g["name"])
+def test_mxfp8_hand_group(g):
+    w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+    p, s = oracle.mxfp8_quantize(w)
+    assert int(s[0, 0]) == g["scale_e8m0"]
+    assert [int(x) for x in p[0]] == [int(x, 16) for x in g["packed"]]
+    assert oracle.unpack_codes(p, 32, 8)[0].tolist() == g["codes"]
+
+
+def test_mxfp8_matches_numpy_and_invariants():
+    for seed in (31, 32):
+        w = _mx_weights(16, 1024, seed)
+        p, s = oracle.mxfp8_quantize(w)
+        p2, s2, codes = numpy_mxfp8_quantize(w)
+        assert np.array_equal(p, p2) and np.array_equal(s, s2)
+        # shared exponent: max|w| / X in [256, 512) where not clamped
+        amax = np.abs(w.astype(np.float64)).reshape(16, 32, 32).max(axis=-1)
+        r = amax[(amax > 0) & (s > 0)] / np.ldexp(1.0, s[(amax > 0) & (s > 0)].astype(np.int64) - 127)
+        assert ((r >= 256) & (r < 512)).all()
+        assert not (codes == 0x80).any()
+        d = oracle.mxfp8_dequantize_f32(p, s, 1024)
+        assert np.array_equal(d, _mx8_values_f64(codes, s).astype(np.float32))
+
+
+def test_mxfp8_matmul_equals_dequantize_then_matmul():
+    w = _mx_weights(8, 256, 33)
+    w[2, 32:64] /= np.float32(1e30)
+    p, s = oracle.mxfp8_quantize(w)
+    x = synth.activations(3, 256, seed=34)
+    y = oracle.mxfp8_matmul(synth.bf16_bits(x), p, s)
+    ref = x.to(torch.float64).numpy() @ _mx8_values_f64(oracle.unpack_codes(p, 256, 8), s).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
 # nvfp4 (E2M1 codes, E4M3 scale per 16 along K, fp32 scale per tensor)
 # --------------------------------------------------------------------------
 
@@ -615,6 +665,9 @@ MUTATIONS = {
     "mx_scale_bias_128": ("static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 127); }",
                           "static double e8m0_value(uint8_t s) { return ldexp(1.0, (int)s - 128); }"),
     "mx_magnitude_table_swapped": ("{0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0}", "{0.0, 0.5, 1.0, 1.5, 2.0, 4.0, 3.0, 6.0}"),
+    "e4m3_no_saturation": ("    if (r > 448.0) r = 448.0;                     /* saturate */\n", ""),
+    "mx8_shared_exponent_off_by_one": ("shared = (ex - 1) - 8;", "shared = (ex - 1) - 7;"),
+    "mx8_signed_zero_code": ("if (v < 0.0 && c != 0u) c |= 0x80u;", "if (v < 0.0) c |= 0x80u;"),
     "nv_tensor_scale_448": ("return amax > 0.0f ? amax / 2688.0f : 1.0f;", "return amax > 0.0f ? amax / 448.0f : 1.0f;"),
     "nv_elements_from_unrounded_scale": ("const float denom = (float)e4m3_value(sb) * g;", "const float denom = s32 * g;"),
     "nv_e4m3_exponent_bias_8": ("return ldexp(8.0 + m, e - 10);", "return ldexp(8.0 + m, e - 11);"),
@@ -681,6 +734,16 @@ def _pins_pass(o: "oracle.Oracle") -> bool:
                 return False
             if [int(x) for x in p[0]] != [int(x, 16) for x in tz["packed"]]:
                 return False
+        for g in _mxfp8_groups():
+            w = np.array([float(s) for s in g["w"]], dtype=np.float64).astype(np.float32)[None, :]
+            p, s = o.mxfp8_quantize(w)
+            if int(s[0, 0]) != g["scale_e8m0"] or [int(x) for x in p[0]] != [int(x, 16) for x in g["packed"]]:
+                return False
+        w = _mx_weights(8, 256, 16)
+        p, s = o.mxfp8_quantize(w)
+        p2, s2, _ = numpy_mxfp8_quantize(w)
+        if not (np.array_equal(p, p2) and np.array_equal(s, s2)):
+            return False
         w = _nv_weights(8, 256, 14)
         w[3, :16] = np.float32(5.0)                  # a block whose scale saturates at 448 (amax / 6g > 448)
         w[3, 0] = np.float32(-40000.0)
