@@ -431,6 +431,24 @@ def section_mxfp4(args, aq, torch, dev, stream, peaks):
                                        "kernel": "qmv_tc_kernel<4,32,1,mxfp4> (mma.sync m16n8k32, codes split by sign)"}
         del qs, base
         torch.cuda.empty_cache()
+    # mxfp8: E4M3 codes + E8M0 per 32 (bytes N*K + N*K/32), f16 MMAs
+    for (K, N) in ((4096, 14336), (8192, 28672)):
+        w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 6 + 5 + K % 7)).to(dev)
+        base = aq.aq_mxfp8_quantize(w)
+        del w
+        wb = N * K + N * K // 32
+        copies = max(2, -(-2 * L2_BYTES // wb) + 1)
+        qs = [base] + [tuple(t.clone() for t in base) for _ in range(copies - 1)]
+        x = x_cache.setdefault(K, synth.activations(1, K, 17).to(dev))
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_mxfp8_matmul(x, *qs[i % copies], out=y, overlap_previous=True),
+                         copies * 4, 20)
+        gbs = wb / (ms * 1e-3) / 1e9
+        out[f"mxfp8_qmv_K{K}_N{N}"] = {"us": round(ms * 1e3, 3), "weight_GBps": round(gbs, 1),
+                                       "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                       "kernel": "qmv_tc_kernel<8,32,1,mxfp8> (mma.sync m16n8k16 f16, E4M3 widened)"}
+        del qs, base
+        torch.cuda.empty_cache()
     # nvfp4: E4M3 scale per 16 + tensor scale (bytes N*K/2 + N*K/16)
     for (K, N) in ((4096, 14336), (8192, 28672)):
         w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 6 + 3 + K % 7)).to(dev)

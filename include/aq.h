@@ -301,6 +301,41 @@ aq_status aq_mxfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales,
 aq_status aq_mxfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
                           const uint8_t *scales, int64_t N, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
 
+/* ---- mxfp8: block-scaled fp8 ------------------------------------------------
+ * Source: metalworking "MLX Quantization" (the newer modes: mxfp8 with groups of
+ * 32) and "Quantizing a Model for MLX", section "Modes, bits and mixed recipes"
+ * (mxfp8: 8 bits, groups of 32, an exponent per group).  Encodings as read from
+ * the OCP Microscaling v1.0 MXFP8 (E4M3) format:
+ *  - packed: uint32 [N, K/4], code k of a row in byte k (LSB first); code = sign
+ *    bit 7 + E4M3 magnitude (exponent bits 6..3 with bias 7, mantissa bits
+ *    2..0, subnormals m * 2^-9, largest 448);
+ *  - scales: uint8 [N, K/32], E8M0 as for mxfp4 (X = 2^(s - 127)).
+ * Quantize: shared exponent floor(log2 max|w|) - 8, clamped to [-127, 127] (an
+ * all-zero group: s = 0); element = E4M3 magnitude nearest to |w| / X, ties to
+ * even, saturating at 448; sign only on a non-zero magnitude.  Bit-exact with
+ * that definition.  Dequantized value: X * e4m3(code) rounded once to fp32 (then
+ * bf16 RNE).  K a multiple of 32; pointers 16-byte aligned. */
+
+/* Bytes of codes + scales: N*K + N*K/32; 0 if invalid. */
+size_t aq_mxfp8_packed_bytes(int64_t N, int64_t K);
+
+aq_status aq_mxfp8_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
+                            aq_stream_t stream);
+aq_status aq_mxfp8_dequantize(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K,
+                              uint16_t *w_out_bf16, aq_stream_t stream);
+aq_status aq_mxfp8_dequantize_f32(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K,
+                                  float *w_out, aq_stream_t stream);
+
+/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device) for decode, M <= 8.  E4M3
+ * codes do not fit the integer MMA: each pair is widened to fp16x2 (exact) and
+ * multiplied on the tensor cores (mma.sync m16n8k16, fp32 accumulate) against
+ * the activations staged as fp16 x * 2^e per group (exact for |x| above 2^-14
+ * of the group's largest); the fold applies X * 2^-e.  Supported: M <= 8,
+ * N >= 16, K a multiple of 512 (others -> AQ_ERR_UNSUPPORTED).  flags: 0 or
+ * AQ_MATMUL_OVERLAP_PREVIOUS.  Accuracy as aq_matmul. */
+aq_status aq_mxfp8_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
+                          const uint8_t *scales, int64_t N, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
+
 /* ---- nvfp4: fp4 with E4M3 block scales and a tensor scale ------------------
  * Source: ExecuTorch "MLX backend — Quantization" (the NVFP4 weight-only
  * config, group size 16) and "Quantizing a Model for MLX", section "Modes, bits

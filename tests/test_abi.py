@@ -242,3 +242,16 @@ def test_nvfp4_validation():
     assert mm(K=288) == aq.AQ_ERR_UNSUPPORTED      # the decode kernel needs K % 256 == 0
     assert mm(N=8) == aq.AQ_ERR_UNSUPPORTED
     assert mm(flags=4) == aq.AQ_ERR_INVALID_ARG
+
+
+def test_mxfp8_validation():
+    L = aq.lib()
+    assert aq.aq_mxfp8_packed_bytes(4096, 4096) == 4096 * 4096 + 4096 * 4096 // 32
+    assert L.aq_mxfp8_quantize(A, 4, 48, A, A, None) == aq.AQ_ERR_INVALID_ARG
+    assert L.aq_mxfp8_quantize(U, 4, 64, A, A, None) == aq.AQ_ERR_ALIGNMENT
+    assert L.aq_mxfp8_dequantize_f32(A, A, 4, 40, A, None) == aq.AQ_ERR_INVALID_ARG
+    mm = lambda M=1, K=512, N=16, flags=0: L.aq_mxfp8_matmul(A, M, K, A, A, N, A, flags, None)
+    assert mm(K=256) == aq.AQ_ERR_UNSUPPORTED
+    assert mm(M=9) == aq.AQ_ERR_UNSUPPORTED
+    assert mm(N=8) == aq.AQ_ERR_UNSUPPORTED
+    assert mm(flags=8) == aq.AQ_ERR_INVALID_ARG

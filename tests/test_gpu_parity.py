@@ -317,6 +317,55 @@ def test_mxfp4_matmul_llama_shapes_sampled(K, N):
     _assert_close(y[:, torch.from_numpy(cols).cuda()], y_ref, f"mxfp4 {K}x{N} sampled", rms=rms)
 
 
+# ----------------------------------------------------------------------------- mxfp8
+
+@pytest.mark.parametrize("N,K,seed", [(8, 128, 71), (37, 1024, 72), (256, 4096, 73)])
+def test_mxfp8_quantize_dequantize_bitexact(N, K, seed):
+    w = _mx_special(N, K, seed)
+    w[6 % N, :32] = np.array([448, 460, 480, 232, 1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10] * 4, dtype=np.float32)
+    p_ref, s_ref = oracle.mxfp8_quantize(w)
+    p, s = aq.aq_mxfp8_quantize(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_u32(p), p_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    f_ref = oracle.mxfp8_dequantize_f32(p_ref, s_ref, K)
+    f = aq.aq_mxfp8_dequantize(p, s, K, fp32=True)
+    assert np.array_equal(f.cpu().numpy().view(np.uint32), f_ref.view(np.uint32))
+    b = aq.aq_mxfp8_dequantize(p, s, K)
+    assert np.array_equal(_u16(b), oracle.bf16_round(f_ref))
+
+
+def _mx8_gpu(w):
+    p_ref, s_ref = oracle.mxfp8_quantize(w)
+    return p_ref, s_ref, torch.from_numpy(p_ref.view(np.int32)).cuda(), torch.from_numpy(s_ref).cuda()
+
+
+@pytest.mark.parametrize("M", (1, 2, 3, 4, 5, 8))
+@pytest.mark.parametrize("K,N", [(512, 16), (1024, 100), (4096, 600), (2560, 2600)])
+def test_mxfp8_matmul_matches_oracle(M, K, N):
+    w = weights(N, K, 80 + K + N, True)
+    p_ref, s_ref, p, s = _mx8_gpu(w)
+    xb = activations_bits(M, K, 81 + M)
+    y = aq.aq_mxfp8_matmul(_x_gpu(xb), p, s)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.mxfp8_matmul(xb, p_ref, s_ref), f"mxfp8 M={M} K={K} N={N}")
+
+
+def test_mxfp8_matmul_overlap_and_llama_shape():
+    K, N = 4096, 14336
+    w = weights(N, K, 1202, True)
+    p_ref, s_ref, p, s = _mx8_gpu(w)
+    xb = activations_bits(1, K, 82)
+    y0 = aq.aq_mxfp8_matmul(_x_gpu(xb), p, s)
+    y1 = aq.aq_mxfp8_matmul(_x_gpu(xb), p, s, overlap_previous=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    cols = sample_rows(N, 300, seed=83)
+    y_ref = oracle.mxfp8_matmul(xb, p_ref[cols], s_ref[cols])
+    _assert_close(y0[:, torch.from_numpy(cols).cuda()], y_ref, "mxfp8 4096x14336 sampled",
+                  rms=float(np.sqrt(np.mean(y_ref ** 2))))
+
+
 # ----------------------------------------------------------------------------- nvfp4
 
 def _nv_special(N, K, seed):

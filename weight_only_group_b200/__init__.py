@@ -13,7 +13,8 @@ Names mirror the C entry points: ``aq_quantize``, ``aq_quantize_mse``,
 ``aq_matmul_ex``, ``aq_embedding``, ``aq_gather_matmul``, ``aq_gather_matmul_grouped``, ``aq_mxfp4_quantize``,
 ``aq_mxfp4_dequantize``, ``aq_mxfp4_dequantize_f32``, ``aq_mxfp4_matmul``,
 ``aq_mxfp4_packed_bytes``, ``aq_nvfp4_quantize``, ``aq_nvfp4_dequantize``,
-``aq_nvfp4_dequantize_f32``, ``aq_nvfp4_matmul``, ``aq_nvfp4_packed_bytes``, ``aq_dispatch``,
+``aq_nvfp4_dequantize_f32``, ``aq_nvfp4_matmul``, ``aq_nvfp4_packed_bytes``, ``aq_mxfp8_quantize``,
+``aq_mxfp8_dequantize``, ``aq_mxfp8_dequantize_f32``, ``aq_mxfp8_matmul``, ``aq_mxfp8_packed_bytes``, ``aq_dispatch``,
 ``aq_matmul_ws``, ``aq_matmul_workspace_bytes``, ``aq_packed_words``,
 ``aq_packed_bytes``, ``aq_status_string``, ``aq_device_fault``.
 """
@@ -82,6 +83,12 @@ def lib() -> ctypes.CDLL:
             L.aq_mxfp4_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
             L.aq_mxfp4_dequantize_f32.argtypes = [vp, vp, i64, i64, vp, vp]
             L.aq_mxfp4_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, ctypes.c_uint32, vp]
+            L.aq_mxfp8_packed_bytes.argtypes = [i64, i64]
+            L.aq_mxfp8_packed_bytes.restype = u64
+            L.aq_mxfp8_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+            L.aq_mxfp8_dequantize.argtypes = [vp, vp, i64, i64, vp, vp]
+            L.aq_mxfp8_dequantize_f32.argtypes = [vp, vp, i64, i64, vp, vp]
+            L.aq_mxfp8_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, ctypes.c_uint32, vp]
             L.aq_nvfp4_packed_bytes.argtypes = [i64, i64]
             L.aq_nvfp4_packed_bytes.restype = u64
             L.aq_nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp]
@@ -448,4 +455,52 @@ def aq_nvfp4_matmul(x, packed, scales, g, out: torch.Tensor | None = None, overl
         rc = lib().aq_nvfp4_matmul(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), g.data_ptr(), N,
                                    out.data_ptr(), flags, _stream(x))
     _check(rc, "aq_nvfp4_matmul")
+    return out
+
+
+# ----------------------------------------------------------------------------- mxfp8 (E4M3 codes, E8M0 per 32)
+
+def aq_mxfp8_packed_bytes(N: int, K: int) -> int:
+    return int(lib().aq_mxfp8_packed_bytes(N, K))
+
+
+def aq_mxfp8_quantize(w: torch.Tensor):
+    """w fp32 [N, K] on the GPU -> (packed int32 [N, K/4] of E4M3 codes, scales uint8 [N, K/32] E8M0)."""
+    _need(w, "w", (torch.float32,))
+    N, K = w.shape
+    packed = torch.empty((N, K // 4), dtype=torch.int32, device=w.device)
+    scales = torch.empty((N, max(K // 32, 1)), dtype=torch.uint8, device=w.device)
+    with torch.cuda.device(w.device):
+        rc = lib().aq_mxfp8_quantize(w.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), _stream(w))
+    _check(rc, "aq_mxfp8_quantize")
+    return packed, scales
+
+
+def aq_mxfp8_dequantize(packed, scales, K: int, out: torch.Tensor | None = None, fp32: bool = False):
+    """-> bf16 (or fp32) [N, K] = X * e4m3(code)."""
+    N = _mx(packed, scales)
+    dt = torch.float32 if fp32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((N, K), dtype=dt, device=packed.device)
+    _need(out, "out", (dt,))
+    fn = "aq_mxfp8_dequantize_f32" if fp32 else "aq_mxfp8_dequantize"
+    with torch.cuda.device(packed.device):
+        rc = getattr(lib(), fn)(packed.data_ptr(), scales.data_ptr(), N, K, out.data_ptr(), _stream(packed))
+    _check(rc, fn)
+    return out
+
+
+def aq_mxfp8_matmul(x, packed, scales, out: torch.Tensor | None = None, overlap_previous: bool = False):
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for mxfp8 weights (decode, M <= 8)."""
+    _need(x, "x", (torch.bfloat16,))
+    N = _mx(packed, scales)
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16,))
+    flags = AQ_MATMUL_OVERLAP_PREVIOUS if overlap_previous else 0
+    with torch.cuda.device(x.device):
+        rc = lib().aq_mxfp8_matmul(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), N, out.data_ptr(), flags,
+                                   _stream(x))
+    _check(rc, "aq_mxfp8_matmul")
     return out

@@ -43,6 +43,13 @@ cudaError_t launch_nvfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t
 cudaError_t launch_nvfp4_dequantize(const uint32_t *packed, const uint8_t *scales, const float *gscale, int64_t N,
                                     int64_t K, void *out, bool bf16_out, cudaStream_t s);
 bool nvfp4_tc_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_mxfp8_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
+                                  cudaStream_t s);
+cudaError_t launch_mxfp8_dequantize(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K, void *out,
+                                    bool bf16_out, cudaStream_t s);
+bool mxfp8_tc_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_mxfp8_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
+                            int64_t N, uint16_t *y, uint32_t flags, cudaStream_t s);
 cudaError_t launch_nvfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
                             const float *gscale, int64_t N, uint16_t *y, uint32_t flags, cudaStream_t s);
 cudaError_t launch_gather_route(const int32_t *experts, int64_t T, int64_t E, int32_t *offsets, int32_t *pos,
@@ -466,6 +473,55 @@ aq_status aq_nvfp4_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_
   if (!aq::nvfp4_tc_supported(M, N, K)) return AQ_ERR_UNSUPPORTED;
   if ((st = check_device()) != AQ_OK) return st;
   return from_cuda(aq::launch_nvfp4_tc(x, M, K, packed, scales, tensor_scale, N, y, flags, stream));
+}
+
+size_t aq_mxfp8_packed_bytes(int64_t N, int64_t K) {
+  if (check_mx_shape(N, K) != AQ_OK) return 0;
+  const size_t nk = static_cast<size_t>(N) * static_cast<size_t>(K);
+  return nk + nk / 32;
+}
+
+aq_status aq_mxfp8_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
+                            aq_stream_t stream) {
+  aq_status st = check_mx_shape(N, K);
+  if (st != AQ_OK) return st;
+  if (!w || !packed || !scales) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(packed) || !aligned16(scales)) return AQ_ERR_ALIGNMENT;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_mxfp8_quantize(w, N, K, packed, scales, stream));
+}
+
+static aq_status mxfp8_dequantize_common(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K, void *out,
+                                         bool bf16, aq_stream_t stream) {
+  aq_status st = check_mx_shape(N, K);
+  if (st != AQ_OK) return st;
+  if (!packed || !scales || !out) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(scales) || !aligned16(out)) return AQ_ERR_ALIGNMENT;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_mxfp8_dequantize(packed, scales, N, K, out, bf16, stream));
+}
+
+aq_status aq_mxfp8_dequantize(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K,
+                              uint16_t *w_out_bf16, aq_stream_t stream) {
+  return mxfp8_dequantize_common(packed, scales, N, K, w_out_bf16, true, stream);
+}
+
+aq_status aq_mxfp8_dequantize_f32(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K, float *w_out,
+                                  aq_stream_t stream) {
+  return mxfp8_dequantize_common(packed, scales, N, K, w_out, false, stream);
+}
+
+aq_status aq_mxfp8_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
+                          int64_t N, uint16_t *y, uint32_t flags, aq_stream_t stream) {
+  aq_status st = check_mx_shape(N, K);
+  if (st != AQ_OK) return st;
+  if (M <= 0 || M > kMaxDim) return AQ_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<uint32_t>(AQ_MATMUL_OVERLAP_PREVIOUS)) != 0) return AQ_ERR_INVALID_ARG;
+  if (!x || !packed || !scales || !y) return AQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return AQ_ERR_ALIGNMENT;
+  if (!aq::mxfp8_tc_supported(M, N, K)) return AQ_ERR_UNSUPPORTED;
+  if ((st = check_device()) != AQ_OK) return st;
+  return from_cuda(aq::launch_mxfp8_tc(x, M, K, packed, scales, N, y, flags, stream));
 }
 
 aq_status aq_device_fault(uint32_t *fault_word) {

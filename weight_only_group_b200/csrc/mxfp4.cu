@@ -1,4 +1,4 @@
-// mxfp4 and nvfp4 quantize and dequantize (block-scaled fp4).
+// Block-scaled float modes: mxfp4, nvfp4 and mxfp8 quantize and dequantize.
 //
 // mxfp4: one E8M0 exponent per 32 weights along K, 4-bit E2M1 codes packed 8
 // per uint32 (LSB first).
@@ -216,7 +216,97 @@ __global__ void __launch_bounds__(256) nvfp4_dequantize_kernel(const uint32_t *_
   }
 }
 
+// ---- mxfp8 (the same pages: mxfp8, groups of 32, 8 bits).  OCP MX v1.0 MXFP8
+// (E4M3) as read: code = sign bit 7 + E4M3 magnitude; shared exponent
+// floor(log2 max|w|) - 8 (8 = the largest E4M3 exponent), clamped to
+// [-127, 127]; element = E4M3 nearest to |w| / X, ties to even, saturating at
+// 448; sign only on a non-zero magnitude.  One thread per group of 32.
+__global__ void __launch_bounds__(256) mxfp8_quantize_kernel(const float *__restrict__ w, int64_t groups,
+                                                             uint32_t *__restrict__ packed, uint8_t *__restrict__ scales) {
+  const int64_t gi = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gi >= groups) return;
+  float v[32];
+  const float4 *src = reinterpret_cast<const float4 *>(w + gi * 32);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 t = __ldg(src + i);
+    v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  int shared = -127;
+  const int be = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+  if (amax > 0.0f && be > 0) shared = max(be - 127 - 8, -127);
+  // 1/X = 2^-shared, shared in [-127, 119]: a normal fp32 power of two, and |w| / X < 512
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - shared) << 23);
+  uint32_t out[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t mag = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fmul_rn(fabsf(v[j]), inv), __NV_SATFINITE, __NV_E4M3));
+    const uint32_t code = mag | ((v[j] < 0.0f && mag != 0u) ? 0x80u : 0u);
+    out[j / 4] |= code << (8 * (j % 4));
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(packed + gi * 8);
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  scales[gi] = static_cast<uint8_t>(shared + 127);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) mxfp8_dequantize_kernel(const uint32_t *__restrict__ packed,
+                                                               const uint8_t *__restrict__ scales, int64_t groups,
+                                                               void *__restrict__ out) {
+  const int64_t gi = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (gi >= groups) return;
+  const uint4 w0 = ldg_nc16(packed + gi * 8), w1 = ldg_nc16(packed + gi * 8 + 4);
+  const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  const float X = e8m0_value(__ldg(scales + gi));
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t c = (words[j / 4] >> (8 * (j % 4))) & 0xFFu;
+    const float m = __fmul_rn(X, e4m3_value(c & 0x7Fu));   // X * e4m3: one rounding (exact unless subnormal)
+    v[j] = (c & 0x80u) ? -m : m;
+  }
+  if constexpr (BF16) {
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + gi * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t u[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
+        u[k] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+      dst[i] = make_uint4(u[0], u[1], u[2], u[3]);
+    }
+  } else {
+    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(out) + gi * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_mxfp8_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
+                                  cudaStream_t s) {
+  const int64_t groups = N * K / 32;
+  mxfp8_quantize_kernel<<<static_cast<unsigned>((groups + 255) / 256), 256, 0, s>>>(w, groups, packed, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp8_dequantize(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K, void *out,
+                                    bool bf16_out, cudaStream_t s) {
+  const int64_t groups = N * K / 32;
+  const unsigned grid = static_cast<unsigned>((groups + 255) / 256);
+  if (bf16_out)
+    mxfp8_dequantize_kernel<true><<<grid, 256, 0, s>>>(packed, scales, groups, out);
+  else
+    mxfp8_dequantize_kernel<false><<<grid, 256, 0, s>>>(packed, scales, groups, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_nvfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
                                   float *gscale, cudaStream_t s) {

@@ -48,6 +48,7 @@
 //  * Every wait is bounded; a timeout sets a bit of g_qmv_tc_fault.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp8.h>
 
 #include <algorithm>
 
@@ -88,7 +89,8 @@ struct LaneWords {
 // lane's K tile c (32 codes).  hh: the half of a shared word that a lane of a
 // 2-bit, G = 32 pair owns (t & 1).
 // FMT 1, 2 (mxfp4, nvfp4; 4-bit codes, 32-code spans): register set s holds
-// codes 4s..4s+3 of the lane's word.
+// codes 4s..4s+3 of the lane's word.  FMT 3 (mxfp8): staged slot s holds
+// elements 4s..4s+3 of the lane's run as two fp16 pairs.
 template <int BITS, int G, int FMT = 0>
 struct LaneSpan {
   static constexpr int length = (BITS == 2 && G == 32) ? 16 : G / 4;
@@ -178,6 +180,25 @@ AQ_DEVICE void e2m1x2_split(uint32_t w, uint32_t (&pos)[2], uint32_t (&neg)[2]) 
   neg[1] = prmt(kLo, kHi, wn >> 16);
 }
 
+// d += A(16x16 f16) * B(16x8 f16), fp32 accumulate (mxfp8: E4M3 codes widened to fp16).
+AQ_DEVICE void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 codes (the low 16 bits of w: first code in the low byte) as fp16x2,
+// first code in the low half (exact: E4M3 values are fp16 values).
+AQ_DEVICE uint32_t e4m3x2_to_f16x2(uint32_t w) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// X of an E8M0 scale byte (s = 0: 2^-127, a subnormal; 255: NaN).
+AQ_DEVICE float e8m0_full(uint32_t sb) {
+  return sb == 0u ? __uint_as_float(0x00400000u) : (sb == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float(sb << 23));
+}
+
 // Half of an E4M3 scale byte's value (sign 0, exponent bits 6..3 with bias 7,
 // mantissa bits 2..0; subnormals m * 2^-9; 0x7F is NaN).
 AQ_DEVICE float e4m3_half(uint32_t b) {
@@ -243,7 +264,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   constexpr int NWD = LaneWords<BITS, G>::count;
   constexpr int GBYTES = G * BITS / 8;           // packed bytes of one group row
   constexpr int SL = LaneSpan<BITS, G, FMT>::length;
-  static_assert(FMT == 0 || (BITS == 4 && G == 32), "mxfp4 / nvfp4: 4-bit codes in 32-code spans");
+  static_assert(FMT == 0 || FMT == 3 || (BITS == 4 && G == 32), "mxfp4 / nvfp4: 4-bit codes in 32-code spans");
+  static_assert(FMT != 3 || (BITS == 8 && G == 32), "mxfp8: 8-bit codes, groups of 32");
   // nvfp4: a 32-code span holds two 16-weight groups, fed to two columns of one MMA
   static_assert(FMT != 2 || MP <= 4, "nvfp4 needs two group slots per token");
   // accumulator chains per digit plane: a group folded on its own has only
@@ -442,6 +464,16 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         uint8_t *dst = xs + mq[j] * a.tok_stride + (gq[j] * U) * 64 + tq[j] * 16;
         static_for<0, U>([&](auto C) {
           constexpr int c = C.value;
+          if constexpr (FMT == 3) {  // fp16 pairs (elements 2i, 2i+1) of x * 2^e: exact in fp16's normal range
+            uint32_t h[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const __half2 p = __floats2half2_rn(v8[j][c][2 * i] * sc, v8[j][c][2 * i + 1] * sc);
+              h[i] = *reinterpret_cast<const uint32_t *>(&p);
+            }
+            if (act[j]) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(h[0], h[1], h[2], h[3]);
+            return;
+          }
           uint32_t lo[2], hi[2];
           static_for<0, 2>([&](auto S) {
             // rint(v * 2^e) lands in the low 22 bits of v * 2^e + 1.5 * 2^23; its
@@ -497,11 +529,16 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
       // mxfp4: the same sums over the negative codes' magnitudes, subtracted below
       int nl[FMT >= 1 ? NACC : 1][4], nh[FMT >= 1 ? NACC : 1][4];
+      float fa[FMT == 3 ? NACC : 1][4];  // mxfp8: fp32 accumulators of the f16 MMAs
 #pragma unroll
       for (int i = 0; i < NACC; ++i) dl[i][0] = dl[i][1] = dl[i][2] = dl[i][3] = dh[i][0] = dh[i][1] = dh[i][2] = dh[i][3] = 0;
-      if constexpr (FMT >= 1) {
+      if constexpr (FMT == 1 || FMT == 2) {
 #pragma unroll
         for (int i = 0; i < NACC; ++i) nl[i][0] = nl[i][1] = nl[i][2] = nl[i][3] = nh[i][0] = nh[i][1] = nh[i][2] = nh[i][3] = 0;
+      }
+      if constexpr (FMT == 3) {
+#pragma unroll
+        for (int i = 0; i < NACC; ++i) fa[i][0] = fa[i][1] = fa[i][2] = fa[i][3] = 0.0f;
       }
       static_for<0, SPANS>([&](auto J) {
         constexpr int j = J.value;
@@ -518,7 +555,13 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);  // lo set 0, lo set 1, hi set 0, hi set 1
           uint32_t q0[2], q1[2];
           constexpr int k = (j * U + c) % NACC;
-          if constexpr (FMT >= 1) {
+          if constexpr (FMT == 3) {
+            // two k16 MMAs: codes 0..3 of the lane's run (words w[0]), then 4..7 (w[1])
+            mma_f16(fa[k], e4m3x2_to_f16x2(w0[0]), e4m3x2_to_f16x2(w1[0]), e4m3x2_to_f16x2(w0[0] >> 16),
+                    e4m3x2_to_f16x2(w1[0] >> 16), bv.x, bv.y);
+            mma_f16(fa[(k + 1) % NACC], e4m3x2_to_f16x2(w0[1]), e4m3x2_to_f16x2(w1[1]), e4m3x2_to_f16x2(w0[1] >> 16),
+                    e4m3x2_to_f16x2(w1[1] >> 16), bv.z, bv.w);
+          } else if constexpr (FMT >= 1) {
             uint32_t n0[2], n1[2];
             e2m1x2_split(w0[0], q0, n0);
             e2m1x2_split(w1[0], q1, n1);
@@ -543,14 +586,21 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           lo += dl[c][i];
           hi += dh[c][i];
         }
-        if constexpr (FMT >= 1) {
+        if constexpr (FMT == 1 || FMT == 2) {
 #pragma unroll
           for (int c = 0; c < NACC; ++c) {
             lo -= nl[c][i];
             hi -= nh[c][i];
           }
         }
-        D[i] = static_cast<float>(hi * 256 + lo);
+        if constexpr (FMT == 3) {  // fp32 sums of the f16 products
+          float f = fa[0][i];
+#pragma unroll
+          for (int c = 1; c < NACC; ++c) f += fa[c][i];
+          D[i] = f;
+        } else {
+          D[i] = static_cast<float>(hi * 256 + lo);
+        }
       }
       // fold: D[0] = (row g, col 2t), D[1] = (row g, col 2t+1), D[2], D[3] = rows g+8.
       // The two columns of a row go through packed fp32x2 operations.
@@ -564,6 +614,12 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
           s0 = make_float2(e4m3_half(e0 & 0xFFu), e4m3_half(e0 >> 8));
           s1 = make_float2(e4m3_half(e1 & 0xFFu), e4m3_half(e1 >> 8));
+          b0 = b1 = make_float2(0.0f, 0.0f);
+        } else if constexpr (FMT == 3) {  // two E8M0 bytes per row (groups gl, gl + 1): X; no bias
+          const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
+          const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
+          s0 = make_float2(e8m0_full(e0 & 0xFFu), e8m0_full(e0 >> 8));
+          s1 = make_float2(e8m0_full(e1 & 0xFFu), e8m0_full(e1 >> 8));
           b0 = b1 = make_float2(0.0f, 0.0f);
         } else if constexpr (FMT == 1) {  // two E8M0 bytes per row (groups gl, gl + 1); no bias
           const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
@@ -589,6 +645,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         if constexpr (FMT == 1) {
           sv0 = e8m0_half(sr0[gl]);
           sv1 = e8m0_half(sr1[gl]);
+        } else if constexpr (FMT == 3) {
+          sv0 = e8m0_full(sr0[gl]);
+          sv1 = e8m0_full(sr1[gl]);
         } else {
           sv0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
           sv1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
@@ -603,8 +662,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
       }
       const float2 tx = make_float2(T0.x, T1.x), ty = make_float2(T0.y, T1.y), tz = make_float2(T0.z, T1.z);
-      // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x   (mxfp4: s = X / 2, no bias)
-      if constexpr (FMT == 1) {
+      // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x   (block-scaled modes: no bias)
+      if constexpr (FMT >= 1) {
         accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), accA);
         accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), accB);
       } else {
@@ -737,6 +796,8 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   if (fmt == 1 && (bits != 4 || G != 32 || K % 512 != 0)) return false;
   // nvfp4 scale rows are K/16 bytes
   if (fmt == 2 && (bits != 4 || G != 32 || K % 256 != 0 || M > 4)) return false;
+  // mxfp8: 8-bit codes, scale rows of K/32 bytes as for mxfp4
+  if (fmt == 3 && (bits != 8 || G != 32 || K % 512 != 0)) return false;
   if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 30)) return false;
   if (N < kRows) return false;  // every CTA owns at least one whole 16-row tile
   const int MP = pow2_tokens(static_cast<int>(M));
@@ -747,9 +808,10 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   int64_t u = 1;
   // (mxfp4: an even number of units, so that every chunk's scale box starts on
   // a 16-byte boundary: a chunk holds 8u scale bytes)
-  if (fmt == 1) u = 2;
+  const bool even_units = fmt == 1 || fmt == 3;
+  if (even_units) u = 2;
   for (int64_t c = 1; c <= units; ++c)
-    if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= kStageTarget && (fmt == 0 || c % 2 == 0)) u = c;
+    if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= kStageTarget && (!even_units || c % 2 == 0)) u = c;
   const int64_t Kc = 8 * G * u, nch = K / Kc, gpc = Kc / G;
   Args &a = pl.a;
   a.early_w = 0;
@@ -764,7 +826,7 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.Kc = static_cast<int>(Kc);
   a.nch = static_cast<int>(nch);
   a.pitch_w = static_cast<int>(code_pitch(Kc * bits / 8, bits, G));
-  const int sbytes = fmt == 1 ? 1 : 2;  // scale bytes per 32-code span (nvfp4: two E4M3 bytes)
+  const int sbytes = (fmt == 1 || fmt == 3) ? 1 : 2;  // scale bytes per 32-code span (nvfp4: two E4M3 bytes)
   a.pitch_s = static_cast<int>(pitch_at(gpc * sbytes, 32, 16));
   if (a.pitch_w / 8 > 256 || a.pitch_s / 8 > 256) return false;  // TMA box width (64-bit elements)
   a.w_box_x = static_cast<int>(Kc * bits / 64);
@@ -1001,6 +1063,38 @@ cudaError_t launch_mxfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
     return cudaErrorInvalidValue;
   mp.b = mp.s;  // no bias map: the kernel never reads this one
   return tc::launch_mp<4, 32, 1>(pl, mp, overlap, s);
+}
+
+bool mxfp8_tc_supported(int64_t M, int64_t N, int64_t K) {
+  tc::Plan pl;
+  return tc::make_plan(M, N, K, 32, 8, 148, pl, 3);
+}
+
+// mxfp8 (E4M3 codes packed 4 per word, one E8M0 byte per 32 along K).
+cudaError_t launch_mxfp8_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *scales,
+                            int64_t N, uint16_t *y, uint32_t flags, cudaStream_t s) {
+  static thread_local int cached_dev = -1, sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  tc::Plan pl;
+  if (!tc::make_plan(M, N, K, 32, 8, sms, pl, 3)) return cudaErrorInvalidValue;
+  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.packed = packed;
+  pl.a.scales = reinterpret_cast<const __half *>(scales);  // read as bytes by the mxfp8 kernel
+  pl.a.biases = nullptr;
+  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
+  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
+  tc::Maps mp;
+  if (!tc::encode_rows(&mp.w, packed, N, K, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 32, pl.a.pitch_s))
+    return cudaErrorInvalidValue;
+  mp.b = mp.s;  // no bias map: the kernel never reads this one
+  return tc::launch_mp<8, 32, 3>(pl, mp, overlap, s);
 }
 
 bool nvfp4_tc_supported(int64_t M, int64_t N, int64_t K) {
