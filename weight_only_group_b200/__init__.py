@@ -20,6 +20,7 @@ Names mirror the C entry points: ``aq_quantize``, ``aq_quantize_mse``,
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -142,6 +143,13 @@ def _stream(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
+def _on(dev: torch.device):
+    """The device context for a call: entered only when dev is not already current."""
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
+
+
 def _need(t: torch.Tensor, name: str, dtypes, ndim: int = 2) -> None:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -168,7 +176,7 @@ def _quantize(fn: str, w: torch.Tensor, G: int, bits: int):
     packed = torch.empty((N, K * bits // 32), dtype=torch.int32, device=w.device)
     scales = torch.empty((N, max(K // G, 1)), dtype=torch.float16, device=w.device)
     biases = torch.empty_like(scales)
-    with torch.cuda.device(w.device):
+    with _on(w.device):
         rc = getattr(lib(), fn)(w.data_ptr(), N, K, G, bits, packed.data_ptr(), scales.data_ptr(),
                                 biases.data_ptr(), _stream(w))
     _check(rc, fn)
@@ -201,7 +209,7 @@ def aq_dequantize(packed, scales, biases, K: int, G: int, bits: int, out: torch.
     if out is None:
         out = torch.empty((N, K), dtype=torch.bfloat16, device=packed.device)
     _need(out, "out", (torch.bfloat16,))
-    with torch.cuda.device(packed.device):
+    with _on(packed.device):
         rc = lib().aq_dequantize(packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, K, G, bits,
                                  out.data_ptr(), _stream(packed))
     _check(rc, "aq_dequantize")
@@ -214,7 +222,7 @@ def aq_dequantize_f32(packed, scales, biases, K: int, G: int, bits: int, out: to
     if out is None:
         out = torch.empty((N, K), dtype=torch.float32, device=packed.device)
     _need(out, "out", (torch.float32,))
-    with torch.cuda.device(packed.device):
+    with _on(packed.device):
         rc = lib().aq_dequantize_f32(packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, K, G, bits,
                                      out.data_ptr(), _stream(packed))
     _check(rc, "aq_dequantize_f32")
@@ -231,7 +239,7 @@ def aq_embedding(ids, packed, scales, biases, D: int, G: int, bits: int, out: to
     if out is None:
         out = torch.empty((T, D), dtype=torch.bfloat16, device=packed.device)
     _need(out, "out", (torch.bfloat16,))
-    with torch.cuda.device(packed.device):
+    with _on(packed.device):
         rc = lib().aq_embedding(ids.data_ptr(), T, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), V, D, G,
                                 bits, out.data_ptr(), _stream(packed))
     _check(rc, "aq_embedding")
@@ -260,7 +268,7 @@ def aq_gather_matmul(x, experts, packed, scales, biases, G: int, bits: int, out:
     if out is None:
         out = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", (torch.bfloat16,))
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         fn = "aq_gather_matmul_grouped" if grouped else "aq_gather_matmul"
         rc = getattr(lib(), fn)(x.data_ptr(), T, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), E, N, G,
                                 bits, experts.data_ptr(), out.data_ptr(), _stream(x))
@@ -277,7 +285,7 @@ def aq_matmul_with(kernel, x, packed, scales, biases, G: int, bits: int, out: to
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", (torch.bfloat16,))
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         rc = lib().aq_matmul_with(k, x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(),
                                   biases.data_ptr(), N, G, bits, out.data_ptr(), _stream(x))
     _check(rc, "aq_matmul")
@@ -305,7 +313,7 @@ def aq_matmul_ex(x, packed, scales, biases, G: int, bits: int, flags: int, out: 
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", (torch.bfloat16,))
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         rc = lib().aq_matmul_ex(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, G,
                                 bits, out.data_ptr(), int(flags), _stream(x))
     _check(rc, "aq_matmul_ex")
@@ -327,7 +335,7 @@ def aq_matmul_ws(x, packed, scales, biases, G: int, bits: int, workspace: torch.
         if workspace.device.type != "cuda" or not workspace.is_contiguous():
             raise ValueError("workspace must be a contiguous CUDA tensor")
         wp, wb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         rc = lib().aq_matmul_ws(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), N, G,
                                 bits, out.data_ptr(), wp, wb, _stream(x))
     _check(rc, "aq_matmul_ws")
@@ -364,7 +372,7 @@ def aq_mxfp4_quantize(w: torch.Tensor):
     N, K = w.shape
     packed = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
     scales = torch.empty((N, max(K // 32, 1)), dtype=torch.uint8, device=w.device)
-    with torch.cuda.device(w.device):
+    with _on(w.device):
         rc = lib().aq_mxfp4_quantize(w.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), _stream(w))
     _check(rc, "aq_mxfp4_quantize")
     return packed, scales
@@ -378,7 +386,7 @@ def aq_mxfp4_dequantize(packed, scales, K: int, out: torch.Tensor | None = None,
         out = torch.empty((N, K), dtype=dt, device=packed.device)
     _need(out, "out", (dt,))
     fn = "aq_mxfp4_dequantize_f32" if fp32 else "aq_mxfp4_dequantize"
-    with torch.cuda.device(packed.device):
+    with _on(packed.device):
         rc = getattr(lib(), fn)(packed.data_ptr(), scales.data_ptr(), N, K, out.data_ptr(), _stream(packed))
     _check(rc, fn)
     return out
@@ -393,7 +401,7 @@ def aq_mxfp4_matmul(x, packed, scales, out: torch.Tensor | None = None, overlap_
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", (torch.bfloat16,))
     flags = AQ_MATMUL_OVERLAP_PREVIOUS if overlap_previous else 0
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         rc = lib().aq_mxfp4_matmul(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), N, out.data_ptr(), flags,
                                    _stream(x))
     _check(rc, "aq_mxfp4_matmul")
@@ -414,7 +422,7 @@ def aq_nvfp4_quantize(w: torch.Tensor):
     packed = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
     scales = torch.empty((N, max(K // 16, 1)), dtype=torch.uint8, device=w.device)
     g = torch.empty((1,), dtype=torch.float32, device=w.device)
-    with torch.cuda.device(w.device):
+    with _on(w.device):
         rc = lib().aq_nvfp4_quantize(w.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), g.data_ptr(), _stream(w))
     _check(rc, "aq_nvfp4_quantize")
     return packed, scales, g
@@ -435,7 +443,7 @@ def aq_nvfp4_dequantize(packed, scales, g, K: int, out: torch.Tensor | None = No
         out = torch.empty((N, K), dtype=dt, device=packed.device)
     _need(out, "out", (dt,))
     fn = "aq_nvfp4_dequantize_f32" if fp32 else "aq_nvfp4_dequantize"
-    with torch.cuda.device(packed.device):
+    with _on(packed.device):
         rc = getattr(lib(), fn)(packed.data_ptr(), scales.data_ptr(), g.data_ptr(), N, K, out.data_ptr(),
                                 _stream(packed))
     _check(rc, fn)
@@ -451,7 +459,7 @@ def aq_nvfp4_matmul(x, packed, scales, g, out: torch.Tensor | None = None, overl
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", (torch.bfloat16,))
     flags = AQ_MATMUL_OVERLAP_PREVIOUS if overlap_previous else 0
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         rc = lib().aq_nvfp4_matmul(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), g.data_ptr(), N,
                                    out.data_ptr(), flags, _stream(x))
     _check(rc, "aq_nvfp4_matmul")
@@ -470,7 +478,7 @@ def aq_mxfp8_quantize(w: torch.Tensor):
     N, K = w.shape
     packed = torch.empty((N, K // 4), dtype=torch.int32, device=w.device)
     scales = torch.empty((N, max(K // 32, 1)), dtype=torch.uint8, device=w.device)
-    with torch.cuda.device(w.device):
+    with _on(w.device):
         rc = lib().aq_mxfp8_quantize(w.data_ptr(), N, K, packed.data_ptr(), scales.data_ptr(), _stream(w))
     _check(rc, "aq_mxfp8_quantize")
     return packed, scales
@@ -484,7 +492,7 @@ def aq_mxfp8_dequantize(packed, scales, K: int, out: torch.Tensor | None = None,
         out = torch.empty((N, K), dtype=dt, device=packed.device)
     _need(out, "out", (dt,))
     fn = "aq_mxfp8_dequantize_f32" if fp32 else "aq_mxfp8_dequantize"
-    with torch.cuda.device(packed.device):
+    with _on(packed.device):
         rc = getattr(lib(), fn)(packed.data_ptr(), scales.data_ptr(), N, K, out.data_ptr(), _stream(packed))
     _check(rc, fn)
     return out
@@ -499,7 +507,7 @@ def aq_mxfp8_matmul(x, packed, scales, out: torch.Tensor | None = None, overlap_
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", (torch.bfloat16,))
     flags = AQ_MATMUL_OVERLAP_PREVIOUS if overlap_previous else 0
-    with torch.cuda.device(x.device):
+    with _on(x.device):
         rc = lib().aq_mxfp8_matmul(x.data_ptr(), M, K, packed.data_ptr(), scales.data_ptr(), N, out.data_ptr(), flags,
                                    _stream(x))
     _check(rc, "aq_mxfp8_matmul")
