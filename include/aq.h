@@ -367,11 +367,13 @@ aq_status aq_nvfp4_dequantize(const uint32_t *packed, const uint8_t *scales, con
 aq_status aq_nvfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales, const float *tensor_scale,
                                   int64_t N, int64_t K, float *w_out, aq_stream_t stream);
 
-/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device) for decode, M <= 4, on the
+/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device) for decode, M <= 8, on the
  * integer tensor cores: one MMA K step spans two 16-weight groups, whose halves
  * feed two accumulator columns; each column is folded with its E4M3 scale and
- * the output multiplied by g.  Supported: M <= 4, N >= 16, K a multiple of 256
- * (others -> AQ_ERR_UNSUPPORTED).  flags: 0 or AQ_MATMUL_OVERLAP_PREVIOUS.
+ * the output multiplied by g.  One launch holds up to 4 tokens; M = 5..8 runs as
+ * two launches (rows 0..3, then the rest), reading the weights twice.
+ * Supported: M <= 8, N >= 16, K a multiple of 256 (others ->
+ * AQ_ERR_UNSUPPORTED).  flags: 0 or AQ_MATMUL_OVERLAP_PREVIOUS (both launches).
  * Accuracy as aq_matmul. */
 aq_status aq_nvfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
                           const uint8_t *scales, const float *tensor_scale, int64_t N, uint16_t *y_bf16,

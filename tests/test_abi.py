@@ -237,7 +237,7 @@ def test_nvfp4_validation():
     assert L.aq_nvfp4_quantize(A, 4, 64, A, A, A + 2, None) == aq.AQ_ERR_ALIGNMENT
     assert L.aq_nvfp4_dequantize(A, U, A, 4, 64, A, None) == aq.AQ_ERR_ALIGNMENT
     mm = lambda M=1, K=512, N=16, flags=0: L.aq_nvfp4_matmul(A, M, K, A, A, A, N, A, flags, None)
-    assert mm(M=5) == aq.AQ_ERR_UNSUPPORTED        # two group slots per token: M <= 4
+    assert mm(M=9) == aq.AQ_ERR_UNSUPPORTED        # decode only (M = 5..8 runs as two launches)
     assert mm(K=208) == aq.AQ_ERR_INVALID_ARG      # K % 32 != 0
     assert mm(K=288) == aq.AQ_ERR_UNSUPPORTED      # the decode kernel needs K % 256 == 0
     assert mm(N=8) == aq.AQ_ERR_UNSUPPORTED

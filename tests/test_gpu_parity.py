@@ -398,7 +398,7 @@ def _nv_gpu(w):
             torch.tensor([g_ref], dtype=torch.float32).cuda())
 
 
-@pytest.mark.parametrize("M", (1, 2, 3, 4))
+@pytest.mark.parametrize("M", (1, 2, 3, 4, 5, 8))
 @pytest.mark.parametrize("K,N", [(256, 16), (1024, 100), (4096, 600), (2560, 2600)])
 def test_nvfp4_matmul_matches_oracle(M, K, N):
     w = weights(N, K, 60 + K + N, True)

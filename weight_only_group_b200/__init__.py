@@ -451,7 +451,7 @@ def aq_nvfp4_dequantize(packed, scales, g, K: int, out: torch.Tensor | None = No
 
 
 def aq_nvfp4_matmul(x, packed, scales, g, out: torch.Tensor | None = None, overlap_previous: bool = False):
-    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for nvfp4 weights (decode, M <= 4)."""
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for nvfp4 weights (decode, M <= 8)."""
     _need(x, "x", (torch.bfloat16,))
     N = _nv(packed, scales, g)
     M, K = x.shape

@@ -470,9 +470,15 @@ aq_status aq_nvfp4_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) ||
       (reinterpret_cast<uintptr_t>(tensor_scale) & 3u) != 0)
     return AQ_ERR_ALIGNMENT;
-  if (!aq::nvfp4_tc_supported(M, N, K)) return AQ_ERR_UNSUPPORTED;
+  // the decode kernel holds up to 4 tokens (two group slots per token); M = 5..8
+  // runs as two launches, rows 0..3 and 4..M-1 (the weights are read twice)
+  if (M > 8 || !aq::nvfp4_tc_supported(std::min<int64_t>(M, 4), N, K)) return AQ_ERR_UNSUPPORTED;
   if ((st = check_device()) != AQ_OK) return st;
-  return from_cuda(aq::launch_nvfp4_tc(x, M, K, packed, scales, tensor_scale, N, y, flags, stream));
+  const int64_t m0 = std::min<int64_t>(M, 4);
+  st = from_cuda(aq::launch_nvfp4_tc(x, m0, K, packed, scales, tensor_scale, N, y, flags, stream));
+  if (st == AQ_OK && M > m0)
+    st = from_cuda(aq::launch_nvfp4_tc(x + m0 * K, M - m0, K, packed, scales, tensor_scale, N, y + m0 * N, flags, stream));
+  return st;
 }
 
 size_t aq_mxfp8_packed_bytes(int64_t N, int64_t K) {
