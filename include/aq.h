@@ -31,7 +31,16 @@
  * aq_matmul_with take it from CUDA's stream-ordered allocator (cudaMallocAsync /
  * cudaFreeAsync on `stream`), aq_matmul_ws takes it from the caller.
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- * stream); outputs are valid once the stream reaches the call.
+ * stream); outputs are valid once the stream reaches the call.  The one
+ * exception is aq_gather_matmul_grouped, which reads per-expert counts on the
+ * host and so synchronizes its stream.
+ *
+ * Entry points beyond quantize / dequantize / matmul, each documented below:
+ *   aq_quantize_mse           range-search quantizer (same format)
+ *   aq_embedding              dequantized rows of a packed table by id
+ *   aq_gather_matmul(_grouped) MoE: each token times its routed expert
+ *   aq_mxfp4_* / aq_nvfp4_* / aq_mxfp8_*  the block-scaled float modes
+ *                              (their own packed layouts, no biases)
  * Errors: arguments are validated synchronously, before anything is launched;
  * a rejected call launches nothing and returns a non-zero status.  Nothing is
  * thrown across the ABI and no kernel traps.
