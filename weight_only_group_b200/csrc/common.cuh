@@ -133,7 +133,7 @@ AQ_DEVICE void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *ba
                : "memory");
 }
 
-// 2-D tiled TMA load global -> shared (no multicast), completing on an
+// 2-D tiled TMA load global -> this CTA's shared memory, completing on an
 // mbarrier; c0 is the innermost coordinate, c0 * element size % 16 == 0.
 AQ_DEVICE void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
   asm volatile(
