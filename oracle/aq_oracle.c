@@ -645,7 +645,12 @@ float oracle_nvfp4_tensor_scale(const float *w, int64_t n)
         float a = fabsf(w[i]);
         if (a > amax) amax = a;
     }
-    return amax > 0.0f ? amax / 2688.0f : 1.0f;   /* fp32 division */
+    if (!(amax > 0.0f)) return 1.0f;
+    /* fp32 division; a tensor so small that amax / 2688 falls below the smallest
+     * normal fp32 (2^-126) takes g = 2^-126, so g is never zero or subnormal and
+     * every finite input quantizes (the pages are silent here: reading) */
+    const float g = amax / 2688.0f;
+    return g < 0x1p-126f ? 0x1p-126f : g;
 }
 
 int oracle_nvfp4_quantize(const float *w, int64_t N, int64_t K, float g, uint32_t *packed, uint8_t *scales)

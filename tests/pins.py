@@ -208,7 +208,7 @@ def e4m3_all_values() -> np.ndarray:
 
 def numpy_nvfp4_quantize(w: np.ndarray):
     """Independent NumPy statement of the nvfp4 quantizer: tensor scale
-    g = fp32(amax / 2688); block byte = the E4M3 value nearest to
+    g = fp32(amax / 2688), at least 2^-126; block byte = the E4M3 value nearest to
     fp32(amax_b / fp32(6 g)) found by searching all 127 values (ties to the even
     byte, saturating at 448); elements nearest of the 16 signed E2M1 values to
     fp32(|w| / fp32(scale * g)), ties to the even code."""
@@ -216,6 +216,7 @@ def numpy_nvfp4_quantize(w: np.ndarray):
     N, K = w.shape
     amax = np.float32(np.abs(w).max())
     g = np.float32(amax / np.float32(2688.0)) if amax > 0 else np.float32(1.0)
+    g = max(g, np.float32(2.0 ** -126))  # never below the smallest normal fp32
     wb = w.reshape(N, K // 16, 16)
     s32 = (np.abs(wb).max(axis=-1) / np.float32(np.float32(6.0) * g)).astype(np.float32).astype(np.float64)
     vals = e4m3_all_values()

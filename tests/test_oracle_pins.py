@@ -506,6 +506,25 @@ def test_nvfp4_hand_tensor(tz):
     assert oracle.unpack_codes(p, tz["K"], 4)[0].tolist() == tz["codes"]
 
 
+def test_nvfp4_tiny_tensor_keeps_a_normal_tensor_scale():
+    """A tensor whose amax / 2688 underflows (here a lone 1.4e-45 among zeros)
+    still quantizes: g is held at 2^-126, the smallest normal fp32, never 0 or a
+    subnormal, and the numpy statement agrees bit for bit."""
+    for amax in (1.4e-45, 2.0 ** -130, 3.0e-36):
+        w = np.zeros((2, 64), dtype=np.float32)
+        w[0, 17] = np.float32(amax)
+        w[1, 40] = -np.float32(amax) / np.float32(2)
+        p, s, g = oracle.nvfp4_quantize(w)
+        assert g == 2.0 ** -126
+        p2, s2, g2, _ = numpy_nvfp4_quantize(w)
+        assert np.array_equal(p, p2) and np.array_equal(s, s2) and g == g2
+    # just above the floor, g is the plain quotient
+    w = np.zeros((1, 16), dtype=np.float32)
+    w[0, 0] = np.float32(2.0 ** -100)
+    _, _, g = oracle.nvfp4_quantize(w)
+    assert g == float(np.float32(np.float32(2.0 ** -100) / np.float32(2688.0)))
+
+
 def test_nvfp4_matches_numpy():
     for seed in (21, 22):
         w = _nv_weights(24, 1024, seed)
@@ -668,7 +687,7 @@ MUTATIONS = {
     "e4m3_no_saturation": ("    if (r > 448.0) r = 448.0;                     /* saturate */\n", ""),
     "mx8_shared_exponent_off_by_one": ("shared = (ex - 1) - 8;", "shared = (ex - 1) - 7;"),
     "mx8_signed_zero_code": ("if (v < 0.0 && c != 0u) c |= 0x80u;", "if (v < 0.0) c |= 0x80u;"),
-    "nv_tensor_scale_448": ("return amax > 0.0f ? amax / 2688.0f : 1.0f;", "return amax > 0.0f ? amax / 448.0f : 1.0f;"),
+    "nv_tensor_scale_448": ("const float g = amax / 2688.0f;", "const float g = amax / 448.0f;"),
     "nv_elements_from_unrounded_scale": ("const float denom = (float)e4m3_value(sb) * g;", "const float denom = s32 * g;"),
     "nv_e4m3_exponent_bias_8": ("return ldexp(8.0 + m, e - 10);", "return ldexp(8.0 + m, e - 11);"),
 }
