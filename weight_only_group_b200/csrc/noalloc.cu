@@ -13,6 +13,8 @@
 //    does not expose it to the plugin.
 // For them this entry point uses g_static_workspace below instead of calling
 // cudaMalloc/cudaMallocAsync or any allocating library routine.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -22,6 +24,8 @@ cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s);
 size_t qmm_workspace_bytes(int64_t M, int64_t K);
 bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits);
+aq_status api_from_cuda(cudaError_t e);
+aq_status api_check_device();
 }  // namespace aq
 
 namespace {
@@ -29,17 +33,35 @@ namespace {
 // The fixed workspace: every GPU that loads this library holds these bytes
 // until the process exits.  Host code must not pass the symbol itself to a
 // kernel (on the host it names a host-side stand-in); the device address comes
-// from cudaGetSymbolAddress, once per device, in static_workspace_address().
+// from cudaGetSymbolAddress in static_workspace_address().
 static __device__ __align__(256) uint8_t g_static_workspace[AQ_QMM_STATIC_WORKSPACE_BYTES];
 
 constexpr int kMaxDevices = 64;
 
-// Device address of g_static_workspace on the current device, looked up on the
-// first call made with that device current (the lookup may load the module, so
-// that first call should happen before any stream capture).  nullptr on error.
+// cuCtxGetCurrent, resolved through the runtime (no link-time libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CtxGetCurrentFn ctx_get_current() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_static_workspace in the current context.  It is looked up
+// with cudaGetSymbolAddress (which may load the module) on the first call made
+// with a device current, and again whenever that device's context has changed
+// since (after cudaDeviceReset the array may sit elsewhere); such a call should
+// not be inside a stream capture.  nullptr on error (*err set).
 void *static_workspace_address(cudaError_t *err) {
   static std::mutex mu;
   static void *addr[kMaxDevices] = {nullptr};
+  static CUcontext owner[kMaxDevices] = {nullptr};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -50,27 +72,31 @@ void *static_workspace_address(cudaError_t *err) {
     *err = cudaErrorInvalidDevice;
     return nullptr;
   }
+  // the current context (none yet before the runtime's first real call on the
+  // device: the lookup below then creates it)
+  const CtxGetCurrentFn get = ctx_get_current();
+  CUcontext ctx = nullptr;
+  if (get == nullptr || get(&ctx) != CUDA_SUCCESS) {
+    *err = cudaErrorNotSupported;
+    return nullptr;
+  }
   std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || ctx == nullptr || owner[dev] != ctx) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess || p == nullptr) {
       *err = (e != cudaSuccess) ? e : cudaErrorInvalidSymbol;
       return nullptr;
     }
+    if (get(&ctx) != CUDA_SUCCESS) {
+      *err = cudaErrorNotSupported;
+      return nullptr;
+    }
     addr[dev] = p;
+    owner[dev] = ctx;
   }
   *err = cudaSuccess;
   return addr[dev];
-}
-
-bool is_sm100(cudaError_t *err) {
-  int dev = 0, major = 0, minor = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  *err = e;
-  return e == cudaSuccess && major == 10 && minor == 0;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -92,12 +118,12 @@ extern "C" aq_status aq_matmul_qmm_static(const uint16_t *x_bf16, int64_t M, int
   // The fp16 activations and row scales must fit the fixed array.
   if (M > (int64_t(1) << 40) / K || aq::qmm_workspace_bytes(M, K) > AQ_QMM_STATIC_WORKSPACE_BYTES)
     return AQ_ERR_UNSUPPORTED;
+  aq_status st = aq::api_check_device();
+  if (st != AQ_OK) return st;
   cudaError_t e = cudaSuccess;
-  if (!is_sm100(&e)) return e != cudaSuccess ? AQ_ERR_CUDA : AQ_ERR_UNSUPPORTED;
   void *ws = static_workspace_address(&e);
-  if (ws == nullptr) return AQ_ERR_CUDA;
+  if (ws == nullptr) return aq::api_from_cuda(e);
   // The pre-pass writes every byte of the workspace that the matmul then reads,
   // so nothing left over from an earlier call needs clearing.
-  e = aq::launch_qmm(x_bf16, M, K, packed, scales, biases, N, G, bits, y_bf16, ws, stream);
-  return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+  return aq::api_from_cuda(aq::launch_qmm(x_bf16, M, K, packed, scales, biases, N, G, bits, y_bf16, ws, stream));
 }
