@@ -392,6 +392,37 @@ def test_nvfp4_quantize_dequantize_bitexact(N, K, seed):
     assert np.array_equal(_u16(b), oracle.bf16_round(f_ref))
 
 
+def _nv_tiny_tensors():
+    """Tensors whose amax / 2688 lies below the smallest normal fp32 (the tensor
+    scale is then held at 2^-126): the hand-derived golden tensor, a lone fp32
+    subnormal among zeros, and seeded weights scaled down to ~1e-36."""
+    import json
+    import os
+    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "nvfp4_groups.json")))["tensors"]
+    tz = next(t for t in gold if t["name"] == "subnormal_amax_tensor_scale_floor")
+    w_gold = np.array([float(v) for v in tz["w"]], dtype=np.float64).astype(np.float32)[None, :]
+    lone = np.zeros((1, 64), dtype=np.float32)
+    lone[0, 17] = np.float32(1.4e-45)
+    scaled = (weights(16, 256, 58, True) * np.float32(1e-36)).astype(np.float32)
+    return [w_gold, lone, scaled]
+
+
+@pytest.mark.parametrize("which", [0, 1, 2])
+def test_nvfp4_tiny_tensor_scale_floor_bitexact(which):
+    w = _nv_tiny_tensors()[which]
+    K = w.shape[1]
+    p_ref, s_ref, g_ref = oracle.nvfp4_quantize(w)
+    assert g_ref == 2.0 ** -126
+    p, s, g = aq.aq_nvfp4_quantize(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert float(g.cpu()[0]) == g_ref
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(_u32(p), p_ref)
+    f_ref = oracle.nvfp4_dequantize_f32(p_ref, s_ref, g_ref, K)
+    f = aq.aq_nvfp4_dequantize(p, s, g, K, fp32=True)
+    assert np.array_equal(f.cpu().numpy().view(np.uint32), f_ref.view(np.uint32))
+
+
 def _nv_gpu(w):
     p_ref, s_ref, g_ref = oracle.nvfp4_quantize(w)
     return (p_ref, s_ref, g_ref, torch.from_numpy(p_ref.view(np.int32)).cuda(), torch.from_numpy(s_ref).cuda(),
@@ -612,6 +643,34 @@ def test_gather_matmul_mixtral_like_top2():
         assert torch.equal(y[t:t + 1], ref)
 
 
+def test_qmv_wait_limit_runs_out_cleanly_then_next_call_is_correct():
+    """A decode launch whose bounded waits may last only 64 SM cycles cannot see
+    its activations land in time (a copy from memory takes thousands of
+    cycles): the wait runs out, the kernel sets its bit in the fault word, waits
+    for its own copies in flight and returns.  The context stays usable: with
+    the default limit restored the same call is correct and leaves no fault."""
+    M, K, N, G, bits = 1, 1024, 512, 64, 4
+    p, s, b = quantized(N, K, 9101, True, G, bits)
+    xb = activations_bits(M, K, 9102)
+    pg, sg, bg = _to_gpu(p, s, b)
+    x = _x_gpu(xb)
+    assert aq.aq_dispatch(M, N, K, G, bits) == aq.AQ_KERNEL_QMV
+    assert aq.aq_device_fault() == 0
+    aq.aq_set_wait_limit(64)
+    try:
+        aq.aq_matmul_with("qmv", x, pg, sg, bg, G, bits)
+        torch.cuda.synchronize()
+    finally:
+        aq.aq_set_wait_limit(0)
+    fault = aq.aq_device_fault()
+    assert fault & 0x1F, f"fault word {fault:#x}: no wait ran out"
+    assert not fault & aq.AQ_FAULT_BAD_INDEX
+    y = aq.aq_matmul_with("qmv", x, pg, sg, bg, G, bits)
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() == 0
+    _assert_close(y, oracle.matmul(xb, p, s, b, G, bits), "after the timeout")
+
+
 def test_gather_matmul_bad_expert_zero_row_and_fault_bit():
     E, N, K, G, bits = 2, 256, 512, 64, 4
     parts, (gp, gs, gb) = _stacked_experts(E, N, K, 9400, G, bits)
@@ -689,7 +748,8 @@ def test_qmm_bits_groups(bits, G):
 
 
 @pytest.mark.parametrize("M,K,N", [(1, 128, 128), (9, 256, 130), (64, 512, 256), (65, 384, 200),
-                                   (129, 640, 129), (256, 1024, 1000), (257, 128, 384), (700, 2048, 300)])
+                                   (129, 640, 129), (256, 1024, 1000), (257, 128, 384), (700, 2048, 300),
+                                   (200, 256, 276), (3, 512, 257), (130, 96, 513), (1, 64, 1), (131, 192, 20)])
 def test_qmm_ragged(M, K, N):
     _matmul_case(M, K, N, 4, 64 if K % 64 == 0 else 32, 9000 + M + N, "qmm")
 
@@ -722,7 +782,10 @@ def test_qmm_workspace_entry_point_matches():
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     y1 = aq.aq_matmul_ws(x, pg, sg, bg, G, bits, ws)
     y2 = aq.aq_matmul(x, pg, sg, bg, G, bits)
-    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    # two kernels (workspace and workspace-free), both within the tolerance of the oracle
+    y_ref = oracle.matmul(activations_bits(M, K, 432), p_ref, s_ref, b_ref, G, bits)
+    _assert_close(y1, y_ref, "aq_matmul_ws")
+    _assert_close(y2, y_ref, "aq_matmul")
     with pytest.raises(aq.AqError):
         aq.aq_matmul_ws(x, pg, sg, bg, G, bits, ws[: need // 2])
     # a decode shape needs none
@@ -749,6 +812,51 @@ def test_qmm_extreme_activation_rows():
     for m in range(M):
         ok, worst = oracle.tolerance_ok(y[m], y_ref[m], RTOL)
         assert ok, (m, worst)
+
+
+def test_qmm_prefill_allocates_nothing_and_replays_from_a_graph():
+    """aq_matmul at a prefill shape (the tensor-core kernel) takes no device
+    memory: the stream-ordered allocator's pool does not grow across the call,
+    and the call can be recorded into a CUDA graph and replayed on new
+    activations with the eager result."""
+    M, K, N, G, bits = 640, 1024, 768, 64, 4
+    p_ref, s_ref, b_ref = quantized(N, K, 441, True, G, bits)
+    pg, sg, bg = _to_gpu(p_ref, s_ref, b_ref)
+    xb1, xb2 = activations_bits(M, K, 442), activations_bits(M, K, 443)
+    x = _x_gpu(xb1)
+    assert aq.aq_dispatch(M, N, K, G, bits) == aq.AQ_KERNEL_QMM
+    y_eager = aq.aq_matmul(x, pg, sg, bg, G, bits)
+    torch.cuda.synchronize()
+    try:
+        from cuda.bindings import runtime as rt
+        err, pool = rt.cudaDeviceGetDefaultMemPool(torch.cuda.current_device())
+        assert err == rt.cudaError_t.cudaSuccess
+        attr = rt.cudaMemPoolAttr
+        err, = rt.cudaMemPoolSetAttribute(pool, attr.cudaMemPoolAttrUsedMemHigh, rt.cuuint64_t(0))
+        assert err == rt.cudaError_t.cudaSuccess
+        err, before = rt.cudaMemPoolGetAttribute(pool, attr.cudaMemPoolAttrUsedMemCurrent)
+        have_pool = True
+    except ImportError:
+        have_pool = False
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    aq.aq_matmul(x, pg, sg, bg, G, bits, out=y)
+    torch.cuda.synchronize()
+    if have_pool:
+        err, high = rt.cudaMemPoolGetAttribute(pool, attr.cudaMemPoolAttrUsedMemHigh)
+        assert int(high) <= int(before), "the call allocated from the stream-ordered pool"
+    assert torch.equal(y.view(torch.int16), y_eager.view(torch.int16))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        aq.aq_matmul(x, pg, sg, bg, G, bits, out=y)
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_eager.view(torch.int16))
+    x.copy_(_x_gpu(xb2))
+    g.replay()
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.matmul(xb2, p_ref, s_ref, b_ref, G, bits), "graph replay on new activations")
+    del g
 
 
 def test_kernels_agree_on_small_m():

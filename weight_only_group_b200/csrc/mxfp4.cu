@@ -113,8 +113,8 @@ __global__ void __launch_bounds__(256) mxfp4_dequantize_kernel(const uint32_t *_
 // ---- nvfp4 ("ExecuTorch MLX backend — Quantization": NVFP4 weight-only config,
 // groups of 16; "Quantizing a Model for MLX", "Modes, bits and mixed recipes").
 // Encodings as read from NVIDIA's NVFP4: E2M1 codes as above; one E4M3 byte per
-// 16 weights; one fp32 tensor scale g = amax / 2688 (6 * 448), 1 for an
-// all-zero tensor.  Block byte: E4M3 nearest to fp32(amax_block / fp32(6 g)),
+// 16 weights; one fp32 tensor scale g = amax / 2688 (6 * 448), at least 2^-126,
+// 1 for an all-zero tensor.  Block byte: E4M3 nearest to fp32(amax_block / fp32(6 g)),
 // ties to even, saturating at 448.  Element: E2M1 nearest to
 // fp32(|w| / fp32(scale * g)), ties to the even code; a zero block scale gives
 // code 0.  Value: fp32(fp32(e2m1 * scale) * g).
@@ -143,7 +143,9 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const float4 *__restric
 // The tensor scale from the amax held in the same word.
 __global__ void nvfp4_tensor_scale_kernel(float *gscale) {
   const float amax = *gscale;
-  *gscale = amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+  // below the smallest normal fp32 the tensor scale is held at 2^-126, so it is
+  // never zero or subnormal
+  *gscale = amax > 0.0f ? fmaxf(__fdiv_rn(amax, 2688.0f), __uint_as_float(0x00800000u)) : 1.0f;
 }
 
 // One thread per block of 16 weights.
