@@ -180,10 +180,63 @@ def aggregate_gbs(bytes_per_step, steps_per_rank, world, ms_max):
 
 # ----------------------------------------------------------------------------- our implementation
 
+def run_sharded(args, rank, world, local_rank):
+    """The decode step with W split along N over the ranks (weight_only_group_b200.shard):
+    each rank streams its rows of the three linears and one NCCL all-gather per step
+    assembles the three y.  The job processes STEP_BYTES per step whatever the
+    number of ranks (strong scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    import weight_only_group_b200 as aq
+    from weight_only_group_b200 import shard
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = read_peaks()
+    layer = []
+    for si, (K, N) in enumerate(DECODE_SHAPES):
+        seed = 1000 + 100 * 2 + si
+        w = torch.from_numpy(synth.weights(N, K, seed)).to(dev)
+        p, s, b = aq.aq_quantize(w, G, BITS)
+        del w
+        pl, sl, bl, n0, n1 = shard.shard_rows(p, s, b, world, rank)
+        layer.append((pl.contiguous(), sl.contiguous(), bl.contiguous(), synth.activations(1, K, seed + 1).to(dev), N))
+
+    def step():
+        ys = [aq.aq_matmul(x, p, s, b, G, BITS, overlap_previous=True) for (p, s, b, x, N) in layer]
+        return [shard.all_gather_columns(y, N) for y, (_, _, _, _, N) in zip(ys, layer)]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rank_barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    rank_barrier(dev)
+    ms_max = reduce_max(e0.elapsed_time(e1), dev)
+    value = STEP_BYTES * args.steps / (ms_max * 1e-3) / 1e9
+    return {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 6), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic (seeded; shapes of Llama-3-8B linears; no checkpoints)",
+            "config": {"workload": WORKLOAD, "M": 1, "bits": BITS, "G": G, "shapes_KN": DECODE_SHAPES,
+                       "parallelism": f"W split along N over {world} ranks; one NCCL all-gather of y per linear",
+                       "l2": "each rank's slice is read once per step (no rotation)"},
+            "gpu_launches": args.steps * len(DECODE_SHAPES),
+            "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(value / world / peaks["hbm_gbs"], 4), "traffic": None}}, {}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import weight_only_group_b200 as aq
 
+    if args.shard and world > 1:
+        return run_sharded(args, rank, world, local_rank)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
 
@@ -260,8 +313,8 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "traffic_unit": "DRAM bytes read + written per decode step (3 launches), from ncu",
                 "peak_source": peaks["source"], "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
-                "kernel": ("qmv_tc_kernel<bits=4,G=64,MP=1> (mma.sync m16n8k32: u8 codes x 16-bit fixed-point "
-                           "activation digits, int32 accumulate; 3 launches per step)"),
+                "kernel": ("qmv_tc_kernel<bits=4,G=64,MP=1> (mma.sync m16n8k32: u8 codes x 8-bit digits of "
+                           "16-bit fixed-point activations, int32 accumulate, fp32 fold; 3 launches per step)"),
                 "algorithmic_bytes_per_step": STEP_BYTES}
     del graph
 
@@ -312,7 +365,7 @@ def run_ours(args, rank, world, local_rank):
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": steps,
             "warmup": reps_w * copies, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8",
             "data": "synthetic (seeded; shapes of Llama-3-8B linears; no checkpoints)",
             "config": {"workload": WORKLOAD, "M": 1, "bits": BITS, "G": G, "shapes_KN": DECODE_SHAPES,
                        "parallelism": f"replicas x{world} (no data-path collective)",
@@ -320,8 +373,26 @@ def run_ours(args, rank, world, local_rank):
                              f"126 MiB L2); step replayed from a CUDA graph"},
             "pct_of_hbm_peak": round(value / world / peaks["hbm_gbs"] * 100, 2),
             "roofline": roofline, "e2e": e2e, "gpu_launches": steps * len(DECODE_SHAPES),
-            "clocks": clocks, "sections": sections}
-    return line
+            "clocks": clocks}
+    line.update(compact_sections(sections))
+    return line, sections
+
+
+def compact_sections(sec):
+    """The headline figures of every workload, small enough for the final line:
+    per-shape decode GB/s, the M = 1..8 curve, the bits x G sweep (GB/s) and the
+    prefill QMM points (TFLOP/s and fraction of the burst bf16 peak)."""
+    out = {}
+    if "decode_shapes" in sec:
+        out["decode_shapes_GBps"] = {k: v["weight_GBps"] for k, v in sec["decode_shapes"].items()}
+    if "qmv_small_m" in sec:
+        out["small_m_GBps"] = {k: v["weight_GBps"] for k, v in sec["qmv_small_m"]["curve"].items()}
+    if "qmv_bits_group_sweep" in sec:
+        out["sweep_GBps"] = {k: v["weight_GBps"] for k, v in sec["qmv_bits_group_sweep"]["points"].items()}
+    if "qmm_prefill" in sec:
+        out["qmm_prefill"] = {k: [v["TFLOP/s"], v["frac_of_burst"]] for k, v in sec["qmm_prefill"]["points"].items()}
+        out["qmm_prefill_unit"] = "[TFLOP/s, fraction of the measured burst bf16 peak]"
+    return out
 
 
 def timed_graph(torch, stream, fn, reps_inner, reps_outer):
@@ -349,8 +420,10 @@ def timed_graph(torch, stream, fn, reps_inner, reps_outer):
 
 def measure_sections(args, aq, torch, dev, stream, peaks):
     out = {}
-    want = set(args.sections.split(",")) if args.sections != "all" else {"qmm", "curve", "sweep", "quant", "embed",
-                                                                         "gather", "mxfp4"}
+    want = set(args.sections.split(",")) if args.sections != "all" else {"shapes", "qmm", "curve", "sweep", "quant",
+                                                                         "embed", "gather", "mxfp4"}
+    if "shapes" in want:
+        out.update(section_decode_shapes(args, aq, torch, dev, stream, peaks))
     if "qmm" in want:
         out.update(section_qmm(args, aq, torch, dev, stream, peaks))
     if "curve" in want:
@@ -494,28 +567,61 @@ def section_embedding(args, aq, torch, dev, stream, peaks):
                           "GBps": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}}
 
 
+QMM_POINTS = [(M, K, N) for (K, N) in ((4096, 14336), (14336, 4096)) for M in (512, 2048, 8192)]
+
+
 def section_qmm(args, aq, torch, dev, stream, peaks):
+    """Prefill QMM (the tensor-core kernel) at every M x (K, N) point of the
+    prefill workload: TFLOP/s (2*M*N*K per call) against the measured bf16
+    dense peak (burst: the kernel is timed on its own, back to back)."""
     out = {}
-    # ---- QMM prefill: M = 8192, K = 4096, N = 14336 (the tensor-core kernel)
-    M, K, N = 8192, 4096, 14336
-    w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 5 + 4)).to(dev)
-    p, s, b = aq.aq_quantize(w, G, BITS)
-    del w
-    x = synth.activations(M, K, 7).to(dev)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, p, s, b, G, BITS, out=y), 2, max(2, args.qmm_reps))
-    flops = 2.0 * M * N * K
-    tf = flops / (ms * 1e-3) / 1e12
-    out["qmm_prefill"] = {"value": round(tf, 1), "unit": "TFLOP/s", "M": M, "K": K, "N": N, "bits": BITS, "G": G,
-                          "ms": round(ms, 4), "kernel": "qmm_kernel<4,256> (tcgen05, A=dequantized W in TMEM)",
-                          "roofline": {"bound": "tensor", "achieved": round(tf, 1),
-                                       "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                                       "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
-                                       "frac_of_burst": round(tf / peaks["bf16_tflops"], 4),
-                                       "traffic": recorded_traffic("qmm_prefill")}}
-    del p, s, b, x, y
+    wcache = {}
+    for (M, K, N) in QMM_POINTS:
+        if (K, N) not in wcache:
+            wcache.clear()
+            torch.cuda.empty_cache()
+            w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 5 + (0 if K == 4096 else 1))).to(dev)
+            wcache[(K, N)] = aq.aq_quantize(w, G, BITS)
+            del w
+        p, s, b = wcache[(K, N)]
+        x = synth.activations(M, K, 7).to(dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        reps = max(2, args.qmm_reps * 8192 // (4 * M))
+        ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, p, s, b, G, BITS, out=y), 2, reps)
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[f"M{M}_K{K}_N{N}"] = {"TFLOP/s": round(tf, 1), "us": round(ms * 1e3, 2),
+                                  "frac_of_burst": round(tf / peaks["bf16_tflops"], 4),
+                                  "frac_of_sustained": round(tf / peaks["bf16_tflops_sustained"], 4)}
+        del x, y
+    wcache.clear()
     torch.cuda.empty_cache()
-    return out
+    return {"qmm_prefill": {"bits": BITS, "G": G, "peak_burst": peaks["bf16_tflops"],
+                            "peak_sustained": peaks["bf16_tflops_sustained"], "points": out,
+                            "traffic": recorded_traffic("qmm_prefill")}}
+
+
+def section_decode_shapes(args, aq, torch, dev, stream, peaks):
+    """Each decode linear on its own (M = 1, 4-bit G64): back-to-back launches of
+    that shape over rotating resident weight copies (larger than L2), each
+    launched as a programmatic dependent of the one before, as in the step."""
+    out = {}
+    for si, (K, N) in enumerate(DECODE_SHAPES):
+        w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 2 + si)).to(dev)
+        base = aq.aq_quantize(w, G, BITS)
+        del w
+        wb = weight_bytes(K, N)
+        copies = max(2, -(-2 * L2_BYTES // wb) + 1)
+        ws = [base] + [tuple(t.clone() for t in base) for _ in range(copies - 1)]
+        x = synth.activations(1, K, 1000 + 100 * 2 + si + 1).to(dev)
+        y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, *ws[i % copies], G, BITS, out=y,
+                                                               overlap_previous=True), copies * 8, 20)
+        gbs = wb / (ms * 1e-3) / 1e9
+        out[f"K{K}_N{N}"] = {"us": round(ms * 1e3, 3), "weight_GBps": round(gbs, 1),
+                             "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        del ws, base
+        torch.cuda.empty_cache()
+    return {"decode_shapes": out}
 
 
 def section_curve(args, aq, torch, dev, stream, peaks):
@@ -532,8 +638,10 @@ def section_curve(args, aq, torch, dev, stream, peaks):
     for M in (1, 2, 3, 4, 5, 6, 8):
         x = synth.activations(M, K, 11).to(dev)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, *ws[i % copies], G, BITS, out=y), copies * 8, 50)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, *ws[i % copies], G, BITS, out=y,
+                                                               overlap_previous=True), copies * 8, 50)
         curve[str(M)] = {"us": round(ms * 1e3, 3), "weight_GBps": round(wb / (ms * 1e-3) / 1e9, 1),
+                         "frac_hbm": round(wb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                          "kernel": ["qmv", "qmm"][aq.aq_dispatch(M, N, K, G, BITS) - 1]}
     out["qmv_small_m"] = {"K": K, "N": N, "bits": BITS, "G": G, "curve": curve}
     del ws, base
@@ -550,14 +658,15 @@ def section_sweep_quant(args, aq, torch, dev, stream, peaks, want):
     x = synth.activations(1, K, 13).to(dev)
     y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
     for bits in ((2, 3, 4, 8) if "sweep" in want else ()):
-        for g in ((32, 64, 128) if bits == 4 else (64,)):
+        for g in (32, 64, 128):
             q = aq.aq_quantize(w, g, bits)
             wb = weight_bytes(K, N, g, bits)
             copies = max(2, -(-2 * L2_BYTES // wb) + 1)
             qs = [q] + [tuple(t.clone() for t in q) for _ in range(copies - 1)]
             ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, *qs[i % copies], g, bits, out=y), copies * 4,
                              20)
-            sweep[f"b{bits}_G{g}"] = {"us": round(ms * 1e3, 2), "weight_GBps": round(wb / (ms * 1e-3) / 1e9, 1)}
+            sweep[f"b{bits}_G{g}"] = {"us": round(ms * 1e3, 2), "weight_GBps": round(wb / (ms * 1e-3) / 1e9, 1),
+                                      "frac_hbm": round(wb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
             del qs, q
             torch.cuda.empty_cache()
     if sweep:
@@ -678,8 +787,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--qmm-reps", type=int, default=20)
     ap.add_argument("--sections", default="all",
-                    help="all | none | comma list of qmm,curve,sweep,quant,embed,gather (secondary measurements)")
+                    help="all | none | comma list of shapes,qmm,curve,sweep,quant,embed,gather,mxfp4 (secondary measurements)")
     ap.add_argument("--no-sections", dest="sections", action="store_const", const="none")
+    ap.add_argument("--shard", action="store_true",
+                    help="with N > 1 ranks: split W along N (one all-gather of y per step) instead of replicas")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle work the reference arm's warm-up and timed steps aim at")
@@ -708,9 +819,11 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
         pg = True
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line, sections = run_ours(args, rank, world, local_rank)
         if rank == 0:
             line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+            if sections:  # the detail, on a line of its own before the result line
+                print(json.dumps({"sections": sections}), flush=True)
             print(json.dumps(line), flush=True)
     finally:
         if pg:

@@ -71,8 +71,11 @@ typedef enum {
 /* Kernel choice for aq_matmul_with (aq_matmul always uses AQ_KERNEL_AUTO). */
 typedef enum {
   AQ_KERNEL_AUTO = 0, /* host-side per-shape dispatch (see aq_dispatch) */
-  AQ_KERNEL_QMV = 1,  /* decode kernel, M <= 8 (integer tensor cores; CUDA cores for 3-bit codes) */
-  AQ_KERNEL_QMM = 2   /* tcgen05 / TMEM tensor-core kernel, any M */
+  AQ_KERNEL_QMV = 1,  /* decode kernel, M <= 8: tcgen05 integer MMA for 2/4/8-bit codes where the shape
+                         allows (K a multiple of 256, 128 at G = 32), else AQ_KERNEL_QMV_SYNC's kernels */
+  AQ_KERNEL_QMM = 2,  /* tcgen05 / TMEM tensor-core kernel, any M */
+  AQ_KERNEL_QMV_SYNC = 3 /* decode kernel, M <= 8, on warp-level integer MMAs (mma.sync; CUDA cores for 3-bit
+                            codes and shapes the tensor-core plans reject); same results within the tolerance */
 } aq_kernel;
 
 /* Words of the packed code array: N*K*bits/32 (0 if the arguments are invalid). */
@@ -190,7 +193,8 @@ aq_status aq_matmul_ws(const uint16_t *x_bf16, int64_t M, int64_t K,
  * exceeds AQ_QMM_STATIC_WORKSPACE_BYTES -> AQ_ERR_UNSUPPORTED, checked before
  * anything is launched; otherwise as aq_matmul_with.
  * The first call on each device looks up the array's device address (which may
- * load the module): make that first call before any stream capture.
+ * load the module), and so does the first call after that device's context has
+ * been recreated (cudaDeviceReset): make such a call before any stream capture.
  * Every call shares the one array per device, so calls that can overlap on the
  * GPU (different streams, or graphs replayed concurrently) race on it; serialize
  * them.  The array keeps the last call's contents; nothing in it needs to start
@@ -199,9 +203,10 @@ aq_status aq_matmul_qmm_static(const uint16_t *x_bf16, int64_t M, int64_t K,
                                const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                                int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
 
-/* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV returns AQ_ERR_UNSUPPORTED
- * when M > 8 or its shared-memory staging of x does not fit; AQ_KERNEL_QMM
- * returns AQ_ERR_UNSUPPORTED when K*bits is not a multiple of 128. */
+/* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV and AQ_KERNEL_QMV_SYNC
+ * return AQ_ERR_UNSUPPORTED when M > 8 or the shared-memory staging of x does
+ * not fit; AQ_KERNEL_QMM returns AQ_ERR_UNSUPPORTED when K*bits is not a
+ * multiple of 128. */
 aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x_bf16, int64_t M, int64_t K,
                          const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                          int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
@@ -393,6 +398,25 @@ enum {
   AQ_FAULT_WAIT_MASK = 0x1Fu, /* bits 0-4: a kernel gave up a bounded wait and returned early */
   AQ_FAULT_BAD_INDEX = 0x20u  /* an embedding id or an expert id was out of range */
 };
+
+/* Limit, in SM clock cycles, of every bounded wait of the decode kernel (the
+ * tensor-core QMV behind aq_matmul for M <= 8, the gather matmul and the
+ * block-scaled decode matmuls) in launches made after this call, from any
+ * thread; cycles <= 0 restores the default of 2e9 cycles (about one second).
+ * No counterpart on the pages: it exists to test the timeout path.  A wait that
+ * runs out sets a bit of AQ_FAULT_WAIT_MASK in the device fault word, the
+ * kernel stops issuing work, waits for its own copies in flight and returns;
+ * that call's output is then invalid.  A limit far below the time a copy from
+ * HBM takes (a few thousand cycles) makes the waits run out on purpose. */
+void aq_set_wait_limit(int64_t cycles);
+
+/* on != 0: every decode-kernel launch made afterwards (from any thread) also
+ * waits, after staging its activations, on a barrier that nothing completes,
+ * so that this bounded wait runs out (after aq_set_wait_limit's limit): the
+ * launch sets its fault bit, issues no more work, waits for its own copies in
+ * flight and returns, its output invalid.  on = 0 restores normal launches.
+ * No counterpart on the pages: it exists to test the timeout path. */
+void aq_set_wait_stall(int on);
 
 /* Reads and clears the device-side fault word of the current device: non-zero
  * when a kernel gave up a bounded wait (an mbarrier that never completed) and

@@ -488,6 +488,17 @@ def test_qmv_decode_workloads(c):
     assert aq.aq_dispatch(c.M, c.N, c.K, c.G, c.bits) == aq.AQ_KERNEL_QMV
 
 
+@pytest.mark.parametrize("kernel", ["qmv", "qmv_sync"])
+@pytest.mark.parametrize("M,K,N,bits,G", [(1, 4096, 4096, 4, 64), (3, 1024, 200, 4, 64), (8, 2048, 129, 4, 32),
+                                          (5, 1536, 384, 8, 128), (2, 4096, 640, 2, 32), (7, 768, 1000, 2, 128),
+                                          (1, 14336, 256, 4, 64), (6, 256, 1, 8, 64), (4, 512, 16, 4, 128)])
+def test_decode_kernels_match_oracle(kernel, M, K, N, bits, G):
+    """Both decode kernels (tcgen05 and mma.sync) on the same shapes: ragged row
+    tiles, a single row, K split across a cluster (few row tiles), every code
+    width the tensor-core kernels take and every group size."""
+    _matmul_case(M, K, N, bits, G, 9500 + M * 31 + N + bits + G, kernel)
+
+
 @pytest.mark.parametrize("c", synth.WORKLOADS[2].cases, ids=lambda c: c.name)
 def test_qmv_small_m(c):
     _matmul_case(c.M, c.K, c.N, c.bits, c.G, c.w_seed, "qmv", c.outliers)
@@ -643,12 +654,12 @@ def test_gather_matmul_mixtral_like_top2():
         assert torch.equal(y[t:t + 1], ref)
 
 
-def test_qmv_wait_limit_runs_out_cleanly_then_next_call_is_correct():
-    """A decode launch whose bounded waits may last only 64 SM cycles cannot see
-    its activations land in time (a copy from memory takes thousands of
-    cycles): the wait runs out, the kernel sets its bit in the fault word, waits
-    for its own copies in flight and returns.  The context stays usable: with
-    the default limit restored the same call is correct and leaves no fault."""
+def test_qmv_wait_runs_out_cleanly_then_next_call_is_correct():
+    """A decode launch that also waits on a barrier nothing completes, with its
+    bounded waits limited to 20,000 SM cycles: that wait runs out, the kernel
+    sets its bit in the fault word, issues no more work, waits for its own
+    copies in flight and returns.  The context stays usable: with normal
+    launches restored the same call is correct and leaves no fault."""
     M, K, N, G, bits = 1, 1024, 512, 64, 4
     p, s, b = quantized(N, K, 9101, True, G, bits)
     xb = activations_bits(M, K, 9102)
@@ -656,14 +667,16 @@ def test_qmv_wait_limit_runs_out_cleanly_then_next_call_is_correct():
     x = _x_gpu(xb)
     assert aq.aq_dispatch(M, N, K, G, bits) == aq.AQ_KERNEL_QMV
     assert aq.aq_device_fault() == 0
-    aq.aq_set_wait_limit(64)
+    aq.aq_set_wait_limit(20000)
+    aq.aq_set_wait_stall(True)
     try:
         aq.aq_matmul_with("qmv", x, pg, sg, bg, G, bits)
         torch.cuda.synchronize()
     finally:
+        aq.aq_set_wait_stall(False)
         aq.aq_set_wait_limit(0)
     fault = aq.aq_device_fault()
-    assert fault & 0x1F, f"fault word {fault:#x}: no wait ran out"
+    assert fault & 0x10, f"fault word {fault:#x}: the decode kernel's wait did not run out"
     assert not fault & aq.AQ_FAULT_BAD_INDEX
     y = aq.aq_matmul_with("qmv", x, pg, sg, bg, G, bits)
     torch.cuda.synchronize()

@@ -16,7 +16,7 @@ Names mirror the C entry points: ``aq_quantize``, ``aq_quantize_mse``,
 ``aq_nvfp4_dequantize_f32``, ``aq_nvfp4_matmul``, ``aq_nvfp4_packed_bytes``, ``aq_mxfp8_quantize``,
 ``aq_mxfp8_dequantize``, ``aq_mxfp8_dequantize_f32``, ``aq_mxfp8_matmul``, ``aq_mxfp8_packed_bytes``, ``aq_dispatch``,
 ``aq_matmul_ws``, ``aq_matmul_workspace_bytes``, ``aq_packed_words``,
-``aq_packed_bytes``, ``aq_status_string``, ``aq_device_fault``.
+``aq_packed_bytes``, ``aq_status_string``, ``aq_device_fault``, ``aq_set_wait_limit``, ``aq_set_wait_stall``.
 """
 from __future__ import annotations
 
@@ -39,9 +39,10 @@ AQ_ERR_DEVICE_FAULT = 5
 AQ_KERNEL_AUTO = 0
 AQ_KERNEL_QMV = 1
 AQ_KERNEL_QMM = 2
+AQ_KERNEL_QMV_SYNC = 3
 AQ_MATMUL_OVERLAP_PREVIOUS = 1
 AQ_FAULT_BAD_INDEX = 0x20
-KERNELS = {"auto": AQ_KERNEL_AUTO, "qmv": AQ_KERNEL_QMV, "qmm": AQ_KERNEL_QMM}
+KERNELS = {"auto": AQ_KERNEL_AUTO, "qmv": AQ_KERNEL_QMV, "qmm": AQ_KERNEL_QMM, "qmv_sync": AQ_KERNEL_QMV_SYNC}
 
 _lock = threading.Lock()
 _lib = None
@@ -104,6 +105,10 @@ def lib() -> ctypes.CDLL:
             L.aq_status_string.restype = ctypes.c_char_p
             L.aq_last_cuda_error.restype = i32
             L.aq_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+            L.aq_set_wait_limit.argtypes = [i64]
+            L.aq_set_wait_limit.restype = None
+            L.aq_set_wait_stall.argtypes = [i32]
+            L.aq_set_wait_stall.restype = None
             for f in ("aq_quantize", "aq_quantize_mse", "aq_dequantize", "aq_dequantize_f32", "aq_matmul",
                       "aq_matmul_with", "aq_matmul_ws", "aq_device_fault"):
                 getattr(L, f).restype = i32
@@ -139,7 +144,13 @@ def aq_last_cuda_error() -> int:
 
 # ----------------------------------------------------------------------------- device calls
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(t: torch.Tensor) -> int:
+    """The current CUDA stream of t's device, as the raw handle the library takes."""
+    if _raw_stream is not None:
+        return _raw_stream(t.device.index if t.device.index is not None else torch.cuda.current_device())
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
@@ -347,6 +358,19 @@ def aq_device_fault() -> int:
     w = ctypes.c_uint32(0)
     _check(lib().aq_device_fault(ctypes.byref(w)), "aq_device_fault")
     return int(w.value)
+
+
+def aq_set_wait_limit(cycles: int) -> None:
+    """Limit (SM clock cycles) of the decode kernel's bounded waits in later
+    launches; cycles <= 0 restores the default (about one second).  For tests
+    of the timeout path (see include/aq.h)."""
+    lib().aq_set_wait_limit(int(cycles))
+
+
+def aq_set_wait_stall(on: bool) -> None:
+    """Make later decode-kernel launches wait on a barrier nothing completes, so
+    that their bounded wait runs out (a test of the timeout path; see include/aq.h)."""
+    lib().aq_set_wait_stall(1 if on else 0)
 
 
 # ----------------------------------------------------------------------------- mxfp4 (block-scaled fp4)

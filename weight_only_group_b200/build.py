@@ -21,8 +21,8 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libaq.so")
 
-SOURCES = ["aq_api.cu", "quantize.cu", "qmv.cu", "qmv_tc.cu", "qmm.cu", "noalloc.cu", "embedding.cu", "mxfp4.cu", "gather.cu"]
-HEADERS = ["common.cuh"]
+SOURCES = ["aq_api.cu", "quantize.cu", "qmv.cu", "qmv_tc.cu", "qmv_umma.cu", "qmm.cu", "qmm2.cu", "noalloc.cu", "embedding.cu", "mxfp4.cu", "gather.cu"]
+HEADERS = ["common.cuh", "tc05.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

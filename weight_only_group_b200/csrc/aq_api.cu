@@ -19,6 +19,8 @@ size_t qmv_required_smem(int64_t M, int64_t K);
 bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t read_and_clear_qmv_fault(uint32_t *word);
 cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word);
+void set_qmv_tc_wait_limit(long long cycles);
+void set_qmv_tc_wait_stall(bool on);
 cudaError_t read_and_clear_embed_fault(uint32_t *word);
 bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed, const uint16_t *scales,
@@ -31,6 +33,17 @@ cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s);
 size_t qmm_workspace_bytes(int64_t M, int64_t K);
 bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits);
+cudaError_t launch_qmm2(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
+bool qmm2_supports(int64_t M, int64_t N, int64_t K, int G, int bits);
+cudaError_t read_and_clear_qmm2_fault(uint32_t *word);
+bool qmv_umma_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
+cudaError_t launch_qmv_umma(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                            const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, uint32_t flags,
+                            cudaStream_t s);
+void set_qmv_umma_wait_limit(long long cycles);
+void set_qmv_umma_wait_stall(bool on);
+cudaError_t read_and_clear_qmv5_fault(uint32_t *word);
 cudaError_t read_and_clear_fault(uint32_t *word);
 cudaError_t launch_mxfp4_quantize(const float *w, int64_t N, int64_t K, uint32_t *packed, uint8_t *scales,
                                   cudaStream_t s);
@@ -123,6 +136,14 @@ aq_status check_mx_shape(int64_t N, int64_t K) {
 
 }  // namespace
 
+namespace aq {
+// Status helpers shared with the entry points defined in other files of this
+// library, so that every entry point records CUDA errors and rejects devices
+// the same way.
+aq_status api_from_cuda(cudaError_t e) { return from_cuda(e); }
+aq_status api_check_device() { return check_device(); }
+}  // namespace aq
+
 extern "C" {
 
 size_t aq_packed_words(int64_t N, int64_t K, int bits) {
@@ -150,6 +171,16 @@ const char *aq_status_string(aq_status status) {
 }
 
 int aq_last_cuda_error(void) { return t_last_cuda_error; }
+
+void aq_set_wait_limit(int64_t cycles) {
+  aq::set_qmv_tc_wait_limit(static_cast<long long>(cycles));
+  aq::set_qmv_umma_wait_limit(static_cast<long long>(cycles));
+}
+
+void aq_set_wait_stall(int on) {
+  aq::set_qmv_tc_wait_stall(on != 0);
+  aq::set_qmv_umma_wait_stall(on != 0);
+}
 
 aq_status aq_quantize(const float *w, int64_t N, int64_t K, int G, int bits, uint32_t *packed, uint16_t *scales,
                       uint16_t *biases, aq_stream_t stream) {
@@ -213,7 +244,8 @@ static aq_status matmul_prepare(aq_kernel &kernel, const uint16_t *x, int64_t M,
     if (k < 0) return AQ_ERR_UNSUPPORTED;
     kernel = static_cast<aq_kernel>(k);
   }
-  if (kernel == AQ_KERNEL_QMV) return qmv_fits(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
+  if (kernel == AQ_KERNEL_QMV || kernel == AQ_KERNEL_QMV_SYNC)
+    return qmv_fits(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
   if (kernel == AQ_KERNEL_QMM) return aq::qmm_supports(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
   return AQ_ERR_INVALID_ARG;
 }
@@ -222,13 +254,18 @@ static size_t workspace_for(aq_kernel kernel, int64_t M, int64_t K) {
   return kernel == AQ_KERNEL_QMM ? aq::qmm_workspace_bytes(M, K) : 0;
 }
 
+// ws == nullptr: the tensor-core matmul without workspace (qmm2.cu); else the
+// one that takes the fp16 activations from the caller's workspace (qmm.cu).
 static aq_status matmul_run(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                             const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
                             void *ws, aq_stream_t stream, uint32_t flags = 0) {
   aq_status st = check_device();
   if (st != AQ_OK) return st;
-  if (kernel == AQ_KERNEL_QMV)
+  if (kernel == AQ_KERNEL_QMV && aq::qmv_umma_supported(M, N, K, G, bits))
+    return from_cuda(aq::launch_qmv_umma(x, M, K, packed, scales, biases, N, G, bits, y, flags, stream));
+  if (kernel == AQ_KERNEL_QMV || kernel == AQ_KERNEL_QMV_SYNC)
     return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, flags, stream));
+  if (ws == nullptr) return from_cuda(aq::launch_qmm2(x, M, K, packed, scales, biases, N, G, bits, y, stream));
   return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, ws, stream));
 }
 
@@ -257,17 +294,9 @@ aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t
                          aq_stream_t stream) {
   aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
   if (st != AQ_OK) return st;
-  const size_t need = workspace_for(kernel, M, K);
-  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream);
-  if ((st = check_device()) != AQ_OK) return st;
-  // workspace from the stream-ordered allocator, released on the same stream
-  void *ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, need, stream);
-  if (e != cudaSuccess) return from_cuda(e);
-  st = matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, ws, stream);
-  e = cudaFreeAsync(ws, stream);
-  if (st == AQ_OK && e != cudaSuccess) st = from_cuda(e);
-  return st;
+  // no workspace and no allocation: the tensor-core path keeps its per-row
+  // activation scales inside y (qmm2.cu)
+  return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream);
 }
 
 aq_status aq_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
@@ -282,9 +311,7 @@ aq_status aq_matmul_ex(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
   aq_kernel kernel = AQ_KERNEL_AUTO;
   aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
   if (st != AQ_OK) return st;
-  const size_t need = workspace_for(kernel, M, K);
-  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream, flags);
-  return aq_matmul_with(kernel, x, M, K, packed, scales, biases, N, G, bits, y, stream);
+  return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream, flags);
 }
 
 aq_status aq_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, const uint16_t *scales,
@@ -539,11 +566,16 @@ aq_status aq_device_fault(uint32_t *fault_word) {
   if (st != AQ_OK) return st;
   st = from_cuda(aq::read_and_clear_qmv_tc_fault(&c));
   if (st != AQ_OK) return st;
-  uint32_t d = 0, g = 0;
+  uint32_t d = 0, g = 0, h = 0;
   st = from_cuda(aq::read_and_clear_embed_fault(&d));
   if (st != AQ_OK) return st;
   st = from_cuda(aq::read_and_clear_gather_fault(&g));
-  *fault_word = a | b | c | d | g;
+  if (st != AQ_OK) return st;
+  st = from_cuda(aq::read_and_clear_qmm2_fault(&h));
+  if (st != AQ_OK) return st;
+  uint32_t u = 0;
+  st = from_cuda(aq::read_and_clear_qmv5_fault(&u));
+  *fault_word = a | b | c | d | g | h | u;
   return st;
 }
 

@@ -97,14 +97,15 @@ AQ_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Bounded wait: true once the phase with the given parity has completed; false
 // on timeout (the fault bit is OR-ed into *fault and *abort_flag is raised) or
 // when another thread of the CTA has already raised *abort_flag.
+// `limit` is the number of SM clock cycles after which the wait gives up.
 AQ_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *fault,
-                         uint32_t fault_bit) {
+                         uint32_t fault_bit, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(fault, fault_bit);
       *abort_flag = 1;
       return false;
@@ -221,6 +222,56 @@ AQ_DEVICE uint32_t extract_code(const uint32_t (&w)[BITS]) {
   } else {
     return __funnelshift_r(w[word], w[word + 1], off) & mask;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Host: encoded 2-D TMA descriptors, cached per thread.  A descriptor is a pure
+// function of its arguments (base address, element type, sizes, strides, box,
+// swizzle), so a hit returns exactly what encoding again would; the cache only
+// saves the driver call on repeated calls with the same operands.
+// ---------------------------------------------------------------------------
+struct TmapKey {
+  const void *base;
+  uint64_t dim0, dim1, stride1;
+  uint32_t box0, box1, dtype, swizzle;
+  bool operator==(const TmapKey &o) const {
+    return base == o.base && dim0 == o.dim0 && dim1 == o.dim1 && stride1 == o.stride1 && box0 == o.box0 &&
+           box1 == o.box1 && dtype == o.dtype && swizzle == o.swizzle;
+  }
+};
+
+template <class EncodeFn>
+inline bool encode_2d_cached(EncodeFn fn, CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
+                             uint64_t dim0, uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                             CUtensorMapSwizzle swizzle) {
+  constexpr int kSlots = 64;
+  struct Slot {
+    TmapKey key;
+    CUtensorMap map;
+    bool used;
+  };
+  static thread_local Slot slots[kSlots] = {};
+  const TmapKey key{base, dim0, dim1, stride1_bytes, box0, box1, static_cast<uint32_t>(dtype),
+                    static_cast<uint32_t>(swizzle)};
+  uint64_t h = reinterpret_cast<uintptr_t>(base) ^ (dim0 * 0x9E3779B97F4A7C15ull) ^ (dim1 << 17) ^ (box0 << 7) ^
+               (uint64_t(box1) << 29) ^ (uint64_t(dtype) << 3) ^ (uint64_t(swizzle) << 11);
+  h ^= h >> 29;
+  Slot &sl = slots[h % kSlots];
+  if (sl.used && sl.key == key) {
+    *map = sl.map;
+    return true;
+  }
+  cuuint64_t dims[2] = {dim0, dim1};
+  cuuint64_t strides[1] = {stride1_bytes};
+  cuuint32_t box[2] = {box0, box1};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  sl.key = key;
+  sl.map = *map;
+  sl.used = true;
+  return true;
 }
 
 template <int N>

@@ -51,6 +51,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -66,7 +67,11 @@ namespace tc {
 
 constexpr int kRows = 16;           // rows of W per tile (the MMA's M)
 constexpr int kMaxConsumers = 12;   // consumer warps per CTA at most
-constexpr int kRedBufs = 2;         // tiles whose chunk partials can be in flight
+constexpr int kRedBufs = 4;         // tiles whose partial sums can be in flight
+constexpr int kDualSmem = 112 * 1024;   // shared memory of a CTA that shares its SM with the next launch's
+constexpr int kDualConsumers = 8;       // consumer warps of such a CTA
+constexpr int kDualMinStages = 4;
+constexpr int kUnitCodes = 1 << 20;     // codes of a row a work unit covers at least (where the stage allows)
 constexpr int kMaxStages = 16;
 constexpr int kStageTarget = 16 * 1024;  // packed bytes of one stage we aim for (<= 1 KB per row)
 constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
@@ -216,13 +221,13 @@ AQ_DEVICE float e8m0_half(uint32_t sb) {
 
 // Bounded spin until *ctr >= target (shared-memory counter written by other
 // warps of the CTA); false on timeout (fault bit set, abort raised) or abort.
-AQ_DEVICE bool spin_until_at_least(int *ctr, int target, volatile int *abort_flag) {
+AQ_DEVICE bool spin_until_at_least(int *ctr, int target, volatile int *abort_flag, long long limit) {
   volatile int *c = ctr;
   if (*c >= target) return true;
   const long long t0 = clock64();
   while (*c < target) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_qmv_tc_fault, kFaultQmvWait);
       *abort_flag = 1;
       return false;
@@ -240,6 +245,12 @@ struct Args {
   int M, N, K, Gn;
   int W, NS;                 // consumer warps, ring stages
   int Kc, nch;               // K chunk of a stage, chunks per row
+  int nper;                  // work units per stage
+  int fpu;                   // folds per work unit
+  int parts;                 // units per 16-row tile (nch * nper): partial sums reduced per tile
+  int red_bufs;              // tiles whose partials can be in flight at once
+  long long wait_cycles;     // limit of every bounded wait, in SM clock cycles
+  int stall;                 // nonzero: the consumers also wait on a barrier nothing completes (timeout test)
   int pitch_w, pitch_s;      // bytes per row of codes / of scales (biases) in a stage
   int s_off, b_off, stage_bytes;
   int xs_off, tok_stride;    // staged activations: token m at xs_off + m * tok_stride
@@ -278,16 +289,18 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.bar_off);
   uint64_t *empty = full + a.NS;
   uint64_t *xbar = empty + a.NS;
+  uint64_t *stall_bar = xbar + 1;  // no thread ever arrives on it (the timeout test waits on it)
   // chunk partials of a tile: red_ready[b] counts partials written into buffer
   // b, red_done[b] the tiles summed out of it (monotonic, so a waiter can never
   // mistake an older round for the one it needs)
-  int *red_ready = reinterpret_cast<int *>(xbar + 1);
-  int *red_done = red_ready + kRedBufs;
-  volatile int *abort_flag = red_done + kRedBufs;
+  int *red_ready = reinterpret_cast<int *>(xbar + 2);
+  int *red_done = red_ready + a.red_bufs;
+  volatile int *abort_flag = red_done + a.red_bufs;
+  int *issued_ctr = red_done + a.red_bufs + 1;  // stages the producer issued (read after an abort)
   uint8_t *xs = smem + a.xs_off;
   uint8_t *zero = smem + a.zero_off;
   float4 *tab = reinterpret_cast<float4 *>(smem + a.tab_off);  // [MP][Gn]: (sum x, 2^-e_lo, 2^-e_hi, 0)
-  float *red = reinterpret_cast<float *>(smem + a.red_off);    // [kRedBufs][nch][16][MP]
+  float *red = reinterpret_cast<float *>(smem + a.red_off);    // [red_bufs][parts][16][MP]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int64_t r0, r1, wrow0 = 0;  // rows [r0, r1) of this CTA; first row of its weight matrix in the maps
@@ -312,6 +325,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   }
   const int tiles = static_cast<int>((r1 - r0 + kRows - 1) / kRows);
   const int nst = tiles * a.nch;
+  const long long wlim = a.wait_cycles;
   const int gpc = a.Kc / G;  // groups per chunk
 
   // One stage: rows of codes, scales and biases of (tile, chunk); whole producer warp.
@@ -334,11 +348,13 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   if (tid == 0) {
     for (int s = 0; s < a.NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], a.nper);  // every unit (fold) of a stage releases it once
     }
-    for (int b = 0; b < kRedBufs; ++b) red_ready[b] = red_done[b] = 0;
+    for (int b = 0; b < a.red_bufs; ++b) red_ready[b] = red_done[b] = 0;
     mbar_init(xbar, 1);
+    mbar_init(stall_bar, 1);
     *abort_flag = 0;
+    *issued_ctr = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -365,31 +381,24 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     // ------------------------------------------------------------ producer
     // (it stages nothing: its lane 0 may stall issuing copies, and the
     // consumers must not wait for that before converting the activations)
-    bool ok = true;
-    int st = a.NS;
+    int st = min(nst, a.NS);
     for (; st < nst; ++st) {
       const int s = st % a.NS;
       int got = 1;
-      if (lane == 0) got = mbar_wait(&empty[s], ((st / a.NS) - 1) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait);
-      if (!__shfl_sync(0xffffffffu, got, 0)) {
-        ok = false;
-        break;
-      }
+      if (lane == 0)
+        got = mbar_wait(&empty[s], ((st / a.NS) - 1) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
       if (lane == 0) issue(st);
     }
-    if (!ok && lane == 0) {  // let the copies already issued land before the CTA exits (bounded)
-      mbar_drain(xbar, 0);
-      for (int j = max(0, st - a.NS); j < st; ++j) mbar_drain(&full[j % a.NS], (j / a.NS) & 1);
-    }
-    return;
-  }
+    if (lane == 0) *issued_ctr = st;
+  } else {
 
   // ---- consumers stage the activations in place: item = (token, group, lane t).
   // A group's raw bf16 and its staged digits occupy the same 2G bytes; the four
   // lanes of a group read all their raw values before any of them writes.
   const int ctid = tid - 32, cthreads = a.W * 32;
   {
-    mbar_wait(xbar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait);
+    mbar_wait(xbar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
     const int items = a.M * a.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
     // Each thread takes kStageItems items per round, processed side by side:
     // the rounds are latency-bound chains (load, reduce across the quad, store).
@@ -497,6 +506,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   }
   // all consumer warps (not the producer) meet here: the staged activations are complete
   asm volatile("bar.sync 1, %0;" ::"r"(cthreads) : "memory");
+  // timeout test: a wait on a barrier that nothing completes runs out, raises
+  // the abort flag and sets the fault bit; every other wait then gives up
+  if (a.stall) mbar_wait(stall_bar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
 
   // -------------------------------------------------------------- consumers
   const int cw = warp - 1;
@@ -507,12 +519,17 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   const uint8_t *zero_lane = zero + (GS == 1 ? 0 : (my_m & 1)) * a.zero_stride + t * 16;
   const int lw0 = LaneWords<BITS, G>::first(t) * 4;
   constexpr int SPANS = FMT == 2 ? GS / 2 : GS;  // 32-code spans (MMA K steps) per fold
-  const int nper = a.Kc / (SPANS * G);
   const float gs = FMT == 2 ? __ldg(a.gscale) : 1.0f;
 
-  for (int st = cw; st < nst; st += a.W) {
+  // Work units: unit u is fold p of stage st (u = st * nper + p), dealt to the
+  // consumer warps round-robin, so a stage is shared by several warps and the
+  // last stages of a launch spread over all of them.  W divides NS * nper, so
+  // the units a warp meets in one ring slot are consecutive phases of it.
+  const int nunits = nst * a.nper;
+  for (int u = cw; u < nunits; u += a.W) {
+    const int st = u / a.nper, p = u - st * a.nper;
     const int s = st % a.NS;
-    if (!mbar_wait(&full[s], (st / a.NS) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait)) break;
+    if (!mbar_wait(&full[s], (st / a.NS) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim)) break;
     const int T = st / a.nch, ch = st - T * a.nch;
     const int64_t rb = tile_base(T);
     const int v0 = static_cast<int>(r0 + static_cast<int64_t>(T) * kRows - rb);  // rows [v0, 16) are new
@@ -525,7 +542,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     const int gch0 = ch * gpc;
     float2 accA = make_float2(0.0f, 0.0f), accB = make_float2(0.0f, 0.0f);  // rows g, g+8 x columns 2t, 2t+1
 
-    for (int p = 0; p < nper; ++p) {
+    for (int pf = p * a.fpu; pf < (p + 1) * a.fpu; ++pf) {  // the unit's folds
       int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
       // mxfp4: the same sums over the negative codes' magnitudes, subtracted below
       int nl[FMT >= 1 ? NACC : 1][4], nh[FMT >= 1 ? NACC : 1][4];
@@ -542,7 +559,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       }
       static_for<0, SPANS>([&](auto J) {
         constexpr int j = J.value;
-        const int gi = p * SPANS + j;
+        const int gi = pf * SPANS + j;
         uint32_t w0[NWD], w1[NWD];
         lds_words<NWD>(wr0 + gi * GBYTES, w0);
         lds_words<NWD>(wr1 + gi * GBYTES, w1);
@@ -607,7 +624,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       float2 s0, s1, b0, b1;  // scale and bias of (row g | g+8) for columns 2t, 2t+1
       float4 T0, T1;          // (sum x, 2^-e_lo, 2^-e_hi, 0) of columns 2t, 2t+1
       if constexpr (GS >= 2) {
-        const int gl = p * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
+        const int gl = pf * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
         const int mt = (2 * t) / GS;
         if constexpr (FMT == 2) {  // two E4M3 bytes per row (16-groups gl, gl + 1, one span); no bias
           const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
@@ -640,7 +657,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           T1 = tab[mt * a.Gn + gch0 + gl + 1];
         }
       } else {
-        const int gl = p;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
+        const int gl = pf;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
         float sv0, sv1, bv0 = 0.0f, bv1 = 0.0f;
         if constexpr (FMT == 1) {
           sv0 = e8m0_half(sr0[gl]);
@@ -725,37 +742,49 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         }
       }
     };
-    if (a.nch == 1) {
+    if (a.parts == 1) {
       put(nullptr, true);
       continue;
     }
-    const int b = T % kRedBufs;
-    const int u = T / kRedBufs;
-    // buffer b is free once the u earlier tiles that used it have been summed
-    if (!spin_until_at_least(&red_done[b], u, abort_flag)) break;
-    float *rbuf = red + static_cast<size_t>(b) * a.nch * kRows * MP;
-    put(rbuf + static_cast<size_t>(ch) * kRows * MP, false);
+    const int b = T % a.red_bufs;
+    const int rnd = T / a.red_bufs;
+    // buffer b is free once the rnd earlier tiles that used it have been summed
+    if (!spin_until_at_least(&red_done[b], rnd, abort_flag, wlim)) break;
+    float *rbuf = red + static_cast<size_t>(b) * a.parts * kRows * MP;
+    put(rbuf + static_cast<size_t>(ch * a.nper + p) * kRows * MP, false);
+    __syncwarp();
+    // The warp whose partial completes the tile sums all of them, in part
+    // order (so the result does not depend on which warp finished last).
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      last = atomicAdd(&red_ready[b], 1) == (rnd + 1) * a.parts - 1;
+      __threadfence_block();
+    }
+    if (!__shfl_sync(0xffffffffu, last, 0)) continue;
+    for (int idx = lane; idx < kRows * MP; idx += 32) {
+      const int row = idx / MP, tok = idx - row * MP;
+      float sum = 0.0f;
+      for (int c2 = 0; c2 < a.parts; ++c2) sum += rbuf[(static_cast<size_t>(c2) * kRows + row) * MP + tok];
+      if (tok < a.M && row_ok(row))
+        yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(FMT == 2 ? sum * gs : sum);
+    }
     __syncwarp();
     if (lane == 0) {
       __threadfence_block();
-      atomicAdd(&red_ready[b], 1);
+      atomicAdd(&red_done[b], 1);
     }
-    if (ch == a.nch - 1) {
-      if (!spin_until_at_least(&red_ready[b], (u + 1) * a.nch, abort_flag)) break;
-      __threadfence_block();
-      for (int idx = lane; idx < kRows * MP; idx += 32) {
-        const int row = idx / MP, tok = idx - row * MP;
-        float sum = 0.0f;
-        for (int c2 = 0; c2 < a.nch; ++c2) sum += rbuf[(static_cast<size_t>(c2) * kRows + row) * MP + tok];
-        if (tok < a.M && row_ok(row))
-          yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(FMT == 2 ? sum * gs : sum);
-      }
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence_block();
-        atomicAdd(&red_done[b], 1);
-      }
-    }
+  }
+  }  // consumers
+
+  // After an abort, copies that were issued but never consumed may still be
+  // landing in this CTA's shared memory: wait for them (bounded) before the
+  // CTA exits.  In a normal run every issued stage was awaited by a consumer.
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    const int issued = *issued_ctr;
+    mbar_drain(xbar, 0);
+    for (int j = max(0, issued - a.NS); j < issued; ++j) mbar_drain(&full[j % a.NS], (j / a.NS) & 1);
   }
 }
 
@@ -789,7 +818,11 @@ static int64_t code_pitch(int64_t row_bytes, int bits, int G) {
 // fmt 0: affine codes with fp16 scales and biases; fmt 1: mxfp4 (E2M1 codes,
 // one E8M0 byte per 32, no biases); fmt 2: nvfp4 (E2M1 codes, one E4M3 byte per
 // 16, i.e. two per 32-code span, a tensor scale, no biases; M <= 4).
-static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt = 0) {
+// dual: the plan for two CTAs per SM (this kernel's and the next launch's, when
+// that one is a programmatic dependent): at most kDualSmem bytes of shared
+// memory and kDualConsumers consumer warps, at least kDualMinStages stages.
+static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt = 0,
+                      bool dual = false, int stage_target = kStageTarget) {
   if (!(bits == 2 || bits == 4 || bits == 8) || !(G == 32 || G == 64 || G == 128)) return false;
   if (M < 1 || M > 8 || N < 1 || K < 1 || K % (8 * G) != 0) return false;
   // mxfp4 scale rows are K/32 bytes: a TMA row stride must be a multiple of 16 bytes
@@ -811,7 +844,7 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   const bool even_units = fmt == 1 || fmt == 3;
   if (even_units) u = 2;
   for (int64_t c = 1; c <= units; ++c)
-    if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= kStageTarget && (!even_units || c % 2 == 0)) u = c;
+    if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= stage_target && (!even_units || c % 2 == 0)) u = c;
   const int64_t Kc = 8 * G * u, nch = K / Kc, gpc = Kc / G;
   Args &a = pl.a;
   a.early_w = 0;
@@ -838,7 +871,24 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.stage_bytes = static_cast<int>(round_up((fmt >= 1 ? a.s_off : a.b_off) + kRows * a.pitch_s, 128));
   a.tok_stride = static_cast<int>(2 * K + 64);
   a.zero_stride = static_cast<int>(round_up(U * 64, 128) + 64);
-  const int64_t budget = 227 * 1024;
+  // work units: fpu folds (a fold: 8/MP groups side by side; nvfp4: twice as
+  // many 16-weight groups) of one stage, at least kUnitCodes codes of a row
+  // where the stage allows.  The kernel is issue-bound, and every unit costs a
+  // partial-sum reduction, so a unit is a whole stage (measured: units of 512
+  // codes were 17% slower on the 33 MB decode launches)
+  const int GS = 8 / MP, SPANS = fmt == 2 ? GS / 2 : GS;
+  const int64_t fold = static_cast<int64_t>(SPANS) * G;  // codes of a row per fold
+  a.fpu = 1;
+  while (fold * a.fpu * 2 <= kUnitCodes && Kc % (fold * a.fpu * 2) == 0) a.fpu *= 2;
+  a.nper = static_cast<int>(Kc / (fold * a.fpu));
+  a.parts = static_cast<int>(nch) * a.nper;
+  // tiles in flight: the units in progress (one per warp, at most
+  // kMaxConsumers) span at most two tiles once a tile has that many units
+  a.red_bufs = a.parts == 1 ? 1 : a.parts >= 2 * kMaxConsumers ? 2 : a.parts >= kMaxConsumers ? 3 : kRedBufs;
+  a.wait_cycles = kWaitCycles;
+  a.stall = 0;
+  const int64_t budget = dual ? kDualSmem : 227 * 1024;
+  const int max_w = dual ? kDualConsumers : kMaxConsumers;
   struct Layout {
     int64_t xs_off, zero_off, tab_off, red_off, bar_off, total;
   };
@@ -852,17 +902,19 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
     L.tab_off = round_up(off, 16);
     off = L.tab_off + static_cast<int64_t>(MP) * Gn * 16;
     L.red_off = off;
-    off += static_cast<int64_t>(kRedBufs) * nch * kRows * MP * 4;
+    off += static_cast<int64_t>(a.red_bufs) * a.parts * kRows * MP * 4;
     L.bar_off = round_up(off, 8);
-    L.total = L.bar_off + (2 * ns + 1) * 8 + (2 * kRedBufs + 1) * 4;
+    L.total = L.bar_off + (2 * ns + 2) * 8 + (2 * a.red_bufs + 2) * 4;
     return L;
   };
-  // consumer warps: a divisor of the ring depth, so every ring slot has one
-  // consumer warp and each of its full barriers is awaited phase after phase.
-  // Take the depth that fits and allows the most consumers (then the deepest).
-  auto consumers = [](int ns) {
-    for (int w = kMaxConsumers; w >= 1; --w)
-      if (ns % w == 0) return w;
+  // consumer warps: a divisor of NS * nper, so the units one warp takes in a
+  // ring slot are consecutive phases of that slot's barriers (a warp never
+  // waits on a phase two ahead of the barrier's).  Take the depth that fits and
+  // allows the most consumers (then the deepest).
+  const int nper = a.nper;
+  auto consumers = [&](int ns) {
+    for (int w = max_w; w >= 1; --w)
+      if ((ns * nper) % w == 0) return w;
     return 1;
   };
   int best_ns = 0;
@@ -870,7 +922,7 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
     if (layout(ns).total > budget) break;
     if (best_ns == 0 || consumers(ns) >= consumers(best_ns)) best_ns = ns;
   }
-  if (best_ns == 0) return false;
+  if (best_ns == 0 || (dual && best_ns < kDualMinStages)) return false;
   const Layout L = layout(best_ns);
   a.NS = best_ns;
   a.W = consumers(best_ns);
@@ -889,9 +941,73 @@ struct Maps {
   CUtensorMap w, s, b;
 };
 
+// The operands of a call (everything in Args that is not layout).
+static void copy_operands(Args &dst, const Args &src) {
+  dst.x = src.x;
+  dst.packed = src.packed;
+  dst.scales = src.scales;
+  dst.biases = src.biases;
+  dst.y = src.y;
+  dst.experts = src.experts;
+  dst.E = src.E;
+  dst.cta_per_tok = src.cta_per_tok;
+  dst.gscale = src.gscale;
+}
+
+#ifndef AQ_QMV_DUAL_POLICY
+#define AQ_QMV_DUAL_POLICY 0  // 0: never two CTAs per SM; 1: with overlapping calls; 2: always
+#endif
+
+// The two-CTAs-per-SM plan for a call, if the policy wants one and it fits.
+static const Plan *dual_plan(const Plan &pl, bool overlap, int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
+                             int fmt, Plan &out) {
+  if (AQ_QMV_DUAL_POLICY == 0 || (AQ_QMV_DUAL_POLICY == 1 && !overlap)) return nullptr;
+  if (pl.a.cta_per_tok > 0) return nullptr;
+  // the ring must hold kDualMinStages stages beside the staged activations:
+  // at large K (or M) with stages of half the usual size
+  if (!make_plan(M, N, K, G, bits, sms, out, fmt, true) &&
+      !make_plan(M, N, K, G, bits, sms, out, fmt, true, kStageTarget / 2))
+    return nullptr;
+  copy_operands(out.a, pl.a);
+  return &out;
+}
+
+// Limit of the kernel's bounded waits, in SM clock cycles (aq_set_wait_limit).
+static std::atomic<long long> g_wait_limit{kWaitCycles};
+static std::atomic<bool> g_wait_stall{false};  // aq_set_wait_stall
+
+// Registers per thread of a kernel instantiation (cached per thread and device).
 template <int BITS, int G, int MP, int FMT>
-static cudaError_t launch(const Plan &pl, const Maps &mp, bool overlap, cudaStream_t stream) {
+static int kernel_regs() {
+  static thread_local int cached_dev = -1, regs = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1 << 20;
+  if (dev != cached_dev) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, qmv_tc_kernel<BITS, G, MP, FMT>) != cudaSuccess) return 1 << 20;
+    regs = fa.numRegs;
+    cached_dev = dev;
+  }
+  return regs;
+}
+
+// pl: the plan for one CTA per SM; dual (may be null): the plan for two per SM,
+// used when the kernel's registers allow two such CTAs on an SM.  With a dual
+// plan and overlap, every stage of the ring is issued before the kernel waits
+// for the one before it: its CTAs run beside that kernel's, so the weights
+// stream while the previous kernel finishes.
+template <int BITS, int G, int MP, int FMT>
+static cudaError_t launch(const Plan &pl_one, const Plan *dual, const Maps &mp, bool overlap, cudaStream_t stream) {
   auto kern = qmv_tc_kernel<BITS, G, MP, FMT>;
+  const Plan *use = &pl_one;
+  if (dual != nullptr) {
+    const int regs = (kernel_regs<BITS, G, MP, FMT>() + 7) / 8 * 8;
+    if (2 * regs * dual->threads <= 65536) use = dual;
+  }
+  Plan pl = *use;
+  pl.a.early_w = overlap ? (use == dual ? pl.a.NS : kEarlyStages) : 0;
+  pl.a.wait_cycles = g_wait_limit.load(std::memory_order_relaxed);
+  pl.a.stall = g_wait_stall.load(std::memory_order_relaxed) ? 1 : 0;
   static thread_local int cached_dev = -1;
   static thread_local size_t cached_smem = 0;
   int dev = 0;
@@ -922,21 +1038,22 @@ static cudaError_t launch(const Plan &pl, const Maps &mp, bool overlap, cudaStre
 }
 
 template <int BITS, int G, int FMT = 0>
-static cudaError_t launch_mp(const Plan &pl, const Maps &mp, bool overlap, cudaStream_t stream) {
+static cudaError_t launch_mp(const Plan &pl, const Plan *dual, const Maps &mp, bool overlap, cudaStream_t stream) {
   switch (pow2_tokens(pl.a.M)) {
-    case 1: return launch<BITS, G, 1, FMT>(pl, mp, overlap, stream);
-    case 2: return launch<BITS, G, 2, FMT>(pl, mp, overlap, stream);
-    case 4: return launch<BITS, G, 4, FMT>(pl, mp, overlap, stream);
-    default: return launch<BITS, G, 8, FMT>(pl, mp, overlap, stream);
+    case 1: return launch<BITS, G, 1, FMT>(pl, dual, mp, overlap, stream);
+    case 2: return launch<BITS, G, 2, FMT>(pl, dual, mp, overlap, stream);
+    case 4: return launch<BITS, G, 4, FMT>(pl, dual, mp, overlap, stream);
+    default: return launch<BITS, G, 8, FMT>(pl, dual, mp, overlap, stream);
   }
 }
 
 template <int BITS>
-static cudaError_t launch_g(const Plan &pl, const Maps &mp, int G, bool overlap, cudaStream_t stream) {
+static cudaError_t launch_g(const Plan &pl, const Plan *dual, const Maps &mp, int G, bool overlap,
+                            cudaStream_t stream) {
   switch (G) {
-    case 32: return launch_mp<BITS, 32>(pl, mp, overlap, stream);
-    case 64: return launch_mp<BITS, 64>(pl, mp, overlap, stream);
-    default: return launch_mp<BITS, 128>(pl, mp, overlap, stream);
+    case 32: return launch_mp<BITS, 32>(pl, dual, mp, overlap, stream);
+    case 64: return launch_mp<BITS, 64>(pl, dual, mp, overlap, stream);
+    default: return launch_mp<BITS, 128>(pl, dual, mp, overlap, stream);
   }
 }
 
@@ -945,13 +1062,10 @@ static cudaError_t launch_g(const Plan &pl, const Maps &mp, int G, bool overlap,
 static bool encode_rows(CUtensorMap *map, const void *base, int64_t rows, int64_t row_bytes, int box_bytes) {
   auto fn = qmm::encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes / 8), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes / 8), static_cast<cuuint32_t>(kRows)};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_2d_cached(fn, map, CU_TENSOR_MAP_DATA_TYPE_UINT64, base, static_cast<uint64_t>(row_bytes / 8),
+                          static_cast<uint64_t>(rows), static_cast<uint64_t>(row_bytes),
+                          static_cast<uint32_t>(box_bytes / 8), static_cast<uint32_t>(kRows),
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace tc
@@ -980,7 +1094,8 @@ cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_
   pl.a.biases = reinterpret_cast<const __half *>(biases);
   pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
-  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
+  tc::Plan dpl;
+  const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, G, bits, sms, 0, dpl);
   tc::Maps mp;
   const int64_t row_bytes = K * bits / 8, sb_bytes = K / G * 2;
   if (!tc::encode_rows(&mp.w, packed, N, row_bytes, pl.a.pitch_w) ||
@@ -988,9 +1103,9 @@ cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_
       !tc::encode_rows(&mp.b, biases, N, sb_bytes, pl.a.pitch_s))
     return cudaErrorInvalidValue;
   switch (bits) {
-    case 2: return tc::launch_g<2>(pl, mp, G, overlap, s);
-    case 4: return tc::launch_g<4>(pl, mp, G, overlap, s);
-    default: return tc::launch_g<8>(pl, mp, G, overlap, s);
+    case 2: return tc::launch_g<2>(pl, dual, mp, G, overlap, s);
+    case 4: return tc::launch_g<4>(pl, dual, mp, G, overlap, s);
+    default: return tc::launch_g<8>(pl, dual, mp, G, overlap, s);
   }
 }
 
@@ -1019,7 +1134,6 @@ cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint
   pl.a.scales = reinterpret_cast<const __half *>(scales);
   pl.a.biases = reinterpret_cast<const __half *>(biases);
   pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
-  pl.a.early_w = 0;
   tc::Maps mp;
   const int64_t row_bytes = K * bits / 8, sb_bytes = K / G * 2;
   if (!tc::encode_rows(&mp.w, packed, E * N, row_bytes, pl.a.pitch_w) ||
@@ -1027,9 +1141,9 @@ cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint
       !tc::encode_rows(&mp.b, biases, E * N, sb_bytes, pl.a.pitch_s))
     return cudaErrorInvalidValue;
   switch (bits) {
-    case 2: return tc::launch_g<2>(pl, mp, G, false, s);
-    case 4: return tc::launch_g<4>(pl, mp, G, false, s);
-    default: return tc::launch_g<8>(pl, mp, G, false, s);
+    case 2: return tc::launch_g<2>(pl, nullptr, mp, G, false, s);
+    case 4: return tc::launch_g<4>(pl, nullptr, mp, G, false, s);
+    default: return tc::launch_g<8>(pl, nullptr, mp, G, false, s);
   }
 }
 
@@ -1057,12 +1171,13 @@ cudaError_t launch_mxfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
   pl.a.biases = nullptr;
   pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
-  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
+  tc::Plan dpl;
+  const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, 32, 4, sms, 1, dpl);
   tc::Maps mp;
   if (!tc::encode_rows(&mp.w, packed, N, K / 2, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 32, pl.a.pitch_s))
     return cudaErrorInvalidValue;
   mp.b = mp.s;  // no bias map: the kernel never reads this one
-  return tc::launch_mp<4, 32, 1>(pl, mp, overlap, s);
+  return tc::launch_mp<4, 32, 1>(pl, dual, mp, overlap, s);
 }
 
 bool mxfp8_tc_supported(int64_t M, int64_t N, int64_t K) {
@@ -1089,12 +1204,13 @@ cudaError_t launch_mxfp8_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
   pl.a.biases = nullptr;
   pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
-  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
+  tc::Plan dpl;
+  const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, 32, 8, sms, 3, dpl);
   tc::Maps mp;
   if (!tc::encode_rows(&mp.w, packed, N, K, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 32, pl.a.pitch_s))
     return cudaErrorInvalidValue;
   mp.b = mp.s;  // no bias map: the kernel never reads this one
-  return tc::launch_mp<8, 32, 3>(pl, mp, overlap, s);
+  return tc::launch_mp<8, 32, 3>(pl, dual, mp, overlap, s);
 }
 
 bool nvfp4_tc_supported(int64_t M, int64_t N, int64_t K) {
@@ -1123,17 +1239,21 @@ cudaError_t launch_nvfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
   pl.a.gscale = gscale;
   pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
-  pl.a.early_w = overlap ? tc::kEarlyStages : 0;
+  tc::Plan dpl;
+  const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, 32, 4, sms, 2, dpl);
   tc::Maps mp;
   if (!tc::encode_rows(&mp.w, packed, N, K / 2, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 16, pl.a.pitch_s))
     return cudaErrorInvalidValue;
   mp.b = mp.s;  // no bias map: the kernel never reads this one
   switch (tc::pow2_tokens(pl.a.M)) {
-    case 1: return tc::launch<4, 32, 1, 2>(pl, mp, overlap, s);
-    case 2: return tc::launch<4, 32, 2, 2>(pl, mp, overlap, s);
-    default: return tc::launch<4, 32, 4, 2>(pl, mp, overlap, s);
+    case 1: return tc::launch<4, 32, 1, 2>(pl, dual, mp, overlap, s);
+    case 2: return tc::launch<4, 32, 2, 2>(pl, dual, mp, overlap, s);
+    default: return tc::launch<4, 32, 4, 2>(pl, dual, mp, overlap, s);
   }
 }
+
+void set_qmv_tc_wait_limit(long long cycles) { tc::g_wait_limit.store(cycles > 0 ? cycles : kWaitCycles); }
+void set_qmv_tc_wait_stall(bool on) { tc::g_wait_stall.store(on); }
 
 cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word) {
   cudaError_t e = cudaMemcpyFromSymbol(word, g_qmv_tc_fault, sizeof(uint32_t));
