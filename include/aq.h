@@ -29,7 +29,9 @@
  * by the caller.  Only the tensor-core matmul path (large M) needs temporary
  * device memory (a workspace: the activations converted to fp16); aq_matmul and
  * aq_matmul_with take it from CUDA's stream-ordered allocator (cudaMallocAsync /
- * cudaFreeAsync on `stream`), aq_matmul_ws takes it from the caller.
+ * cudaFreeAsync on `stream`), aq_matmul_ws takes it from the caller, and
+ * aq_matmul_with(AQ_KERNEL_QMM_NOWS) and aq_matmul_qmm_static need none from
+ * anybody at call time.
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  * stream); outputs are valid once the stream reaches the call.  The one
  * exception is aq_gather_matmul_grouped, which reads per-expert counts on the
@@ -71,11 +73,13 @@ typedef enum {
 /* Kernel choice for aq_matmul_with (aq_matmul always uses AQ_KERNEL_AUTO). */
 typedef enum {
   AQ_KERNEL_AUTO = 0, /* host-side per-shape dispatch (see aq_dispatch) */
-  AQ_KERNEL_QMV = 1,  /* decode kernel, M <= 8: tcgen05 integer MMA for 2/4/8-bit codes where the shape
-                         allows (K a multiple of 256, 128 at G = 32), else AQ_KERNEL_QMV_SYNC's kernels */
-  AQ_KERNEL_QMM = 2,  /* tcgen05 / TMEM tensor-core kernel, any M */
-  AQ_KERNEL_QMV_SYNC = 3 /* decode kernel, M <= 8, on warp-level integer MMAs (mma.sync; CUDA cores for 3-bit
-                            codes and shapes the tensor-core plans reject); same results within the tolerance */
+  AQ_KERNEL_QMV = 1,  /* decode kernel, M <= 8 (warp-level integer MMAs; CUDA cores for 3-bit codes) */
+  AQ_KERNEL_QMM = 2,  /* tcgen05 / TMEM tensor-core kernel, any M; fp16 activations in a workspace */
+  AQ_KERNEL_QMV_TCGEN05 = 3, /* decode kernel, M <= 8, 2/4/8-bit codes, on tcgen05 integer MMAs (codes
+                                unpacked into tensor memory); K a multiple of 256 (128 at G = 32); other
+                                shapes run AQ_KERNEL_QMV */
+  AQ_KERNEL_QMM_NOWS = 4 /* tcgen05 tensor-core kernel, any M, without workspace: activations converted to
+                            fp16 on chip (slower than AQ_KERNEL_QMM; for callers that cannot allocate) */
 } aq_kernel;
 
 /* Words of the packed code array: N*K*bits/32 (0 if the arguments are invalid). */
@@ -203,10 +207,13 @@ aq_status aq_matmul_qmm_static(const uint16_t *x_bf16, int64_t M, int64_t K,
                                const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                                int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);
 
-/* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV and AQ_KERNEL_QMV_SYNC
+/* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV and AQ_KERNEL_QMV_TCGEN05
  * return AQ_ERR_UNSUPPORTED when M > 8 or the shared-memory staging of x does
- * not fit; AQ_KERNEL_QMM returns AQ_ERR_UNSUPPORTED when K*bits is not a
- * multiple of 128. */
+ * not fit; AQ_KERNEL_QMM and AQ_KERNEL_QMM_NOWS return AQ_ERR_UNSUPPORTED when
+ * K*bits is not a multiple of 128.  AQ_KERNEL_QMM takes its workspace from
+ * the stream-ordered allocator (cudaMallocAsync on `stream`); AQ_KERNEL_QMM_NOWS
+ * allocates nothing (each token row's power-of-two scale is kept, until the
+ * epilogue overwrites it, in bytes of y's own output tile). */
 aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x_bf16, int64_t M, int64_t K,
                          const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                          int64_t N, int G, int bits, uint16_t *y_bf16, aq_stream_t stream);

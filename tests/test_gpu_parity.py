@@ -488,12 +488,12 @@ def test_qmv_decode_workloads(c):
     assert aq.aq_dispatch(c.M, c.N, c.K, c.G, c.bits) == aq.AQ_KERNEL_QMV
 
 
-@pytest.mark.parametrize("kernel", ["qmv", "qmv_sync"])
+@pytest.mark.parametrize("kernel", ["qmv", "qmv_tcgen05"])
 @pytest.mark.parametrize("M,K,N,bits,G", [(1, 4096, 4096, 4, 64), (3, 1024, 200, 4, 64), (8, 2048, 129, 4, 32),
                                           (5, 1536, 384, 8, 128), (2, 4096, 640, 2, 32), (7, 768, 1000, 2, 128),
                                           (1, 14336, 256, 4, 64), (6, 256, 1, 8, 64), (4, 512, 16, 4, 128)])
 def test_decode_kernels_match_oracle(kernel, M, K, N, bits, G):
-    """Both decode kernels (tcgen05 and mma.sync) on the same shapes: ragged row
+    """Both decode kernels (mma.sync and tcgen05) on the same shapes: ragged row
     tiles, a single row, K split across a cluster (few row tiles), every code
     width the tensor-core kernels take and every group size."""
     _matmul_case(M, K, N, bits, G, 9500 + M * 31 + N + bits + G, kernel)
@@ -654,7 +654,8 @@ def test_gather_matmul_mixtral_like_top2():
         assert torch.equal(y[t:t + 1], ref)
 
 
-def test_qmv_wait_runs_out_cleanly_then_next_call_is_correct():
+@pytest.mark.parametrize("kernel", ["qmv", "qmv_tcgen05"])
+def test_qmv_wait_runs_out_cleanly_then_next_call_is_correct(kernel):
     """A decode launch that also waits on a barrier nothing completes, with its
     bounded waits limited to 20,000 SM cycles: that wait runs out, the kernel
     sets its bit in the fault word, issues no more work, waits for its own
@@ -670,7 +671,7 @@ def test_qmv_wait_runs_out_cleanly_then_next_call_is_correct():
     aq.aq_set_wait_limit(20000)
     aq.aq_set_wait_stall(True)
     try:
-        aq.aq_matmul_with("qmv", x, pg, sg, bg, G, bits)
+        aq.aq_matmul_with(kernel, x, pg, sg, bg, G, bits)
         torch.cuda.synchronize()
     finally:
         aq.aq_set_wait_stall(False)
@@ -678,7 +679,7 @@ def test_qmv_wait_runs_out_cleanly_then_next_call_is_correct():
     fault = aq.aq_device_fault()
     assert fault & 0x10, f"fault word {fault:#x}: the decode kernel's wait did not run out"
     assert not fault & aq.AQ_FAULT_BAD_INDEX
-    y = aq.aq_matmul_with("qmv", x, pg, sg, bg, G, bits)
+    y = aq.aq_matmul_with(kernel, x, pg, sg, bg, G, bits)
     torch.cuda.synchronize()
     assert aq.aq_device_fault() == 0
     _assert_close(y, oracle.matmul(xb, p, s, b, G, bits), "after the timeout")
@@ -754,17 +755,24 @@ def test_qmm_prefill_workloads(c):
     assert aq.aq_dispatch(c.M, c.N, c.K, c.G, c.bits) == aq.AQ_KERNEL_QMM
 
 
+@pytest.mark.parametrize("kernel", ("qmm", "qmm_nows"))
 @pytest.mark.parametrize("bits", (2, 3, 4, 8))
 @pytest.mark.parametrize("G", (32, 64, 128))
-def test_qmm_bits_groups(bits, G):
-    _matmul_case(300, 1024, 384, bits, G, 8100 + bits * 10 + G, "qmm")
+def test_qmm_bits_groups(bits, G, kernel):
+    _matmul_case(300, 1024, 384, bits, G, 8100 + bits * 10 + G, kernel)
 
 
 @pytest.mark.parametrize("M,K,N", [(1, 128, 128), (9, 256, 130), (64, 512, 256), (65, 384, 200),
                                    (129, 640, 129), (256, 1024, 1000), (257, 128, 384), (700, 2048, 300),
-                                   (200, 256, 276), (3, 512, 257), (130, 96, 513), (1, 64, 1), (131, 192, 20)])
-def test_qmm_ragged(M, K, N):
-    _matmul_case(M, K, N, 4, 64 if K % 64 == 0 else 32, 9000 + M + N, "qmm")
+                                   (200, 256, 276), (3, 512, 257), (130, 96, 513), (1, 64, 20), (131, 192, 20)])
+@pytest.mark.parametrize("kernel", ("qmm", "qmm_nows"))
+def test_qmm_ragged(M, K, N, kernel):
+    _matmul_case(M, K, N, 4, 64 if K % 64 == 0 else 32, 9000 + M + N, kernel)
+
+
+@pytest.mark.parametrize("c", synth.WORKLOADS[4].cases[:2], ids=lambda c: c.name)
+def test_qmm_nows_prefill_workloads(c):
+    _matmul_case(c.M, c.K, c.N, c.bits, c.G, c.w_seed, "qmm_nows", c.outliers, full=False, n_rows=24)
 
 
 def test_qmm_matches_dequantize_then_matmul():
@@ -807,7 +815,8 @@ def test_qmm_workspace_entry_point_matches():
     assert torch.equal(y3.view(torch.int16), aq.aq_matmul(x[:4], pg, sg, bg, G, bits).view(torch.int16))
 
 
-def test_qmm_extreme_activation_rows():
+@pytest.mark.parametrize("kernel", ("qmm", "qmm_nows"))
+def test_qmm_extreme_activation_rows(kernel):
     """Rows far outside fp16 range, rows of tiny values and an all-zero row: the
     per-row power-of-two scaling keeps them exact in fp16."""
     M, K, N, G, bits = 130, 1024, 256, 64, 4
@@ -819,7 +828,7 @@ def test_qmm_extreme_activation_rows():
     x[2] = 0.0
     x[3, 5] = 3.0e38
     xb = x.to(torch.bfloat16)
-    y = aq.aq_matmul_with("qmm", xb.cuda(), *_to_gpu(p_ref, s_ref, b_ref), G, bits)
+    y = aq.aq_matmul_with(kernel, xb.cuda(), *_to_gpu(p_ref, s_ref, b_ref), G, bits)
     y_ref = oracle.matmul(synth.bf16_bits(xb), p_ref, s_ref, b_ref, G, bits)
     y = y.float().cpu().numpy().astype(np.float64)
     for m in range(M):
@@ -827,32 +836,32 @@ def test_qmm_extreme_activation_rows():
         assert ok, (m, worst)
 
 
-def test_qmm_prefill_allocates_nothing_and_replays_from_a_graph():
-    """aq_matmul at a prefill shape (the tensor-core kernel) takes no device
-    memory: the stream-ordered allocator's pool does not grow across the call,
-    and the call can be recorded into a CUDA graph and replayed on new
+def test_qmm_nows_allocates_nothing_and_replays_from_a_graph():
+    """The tensor-core matmul without workspace (AQ_KERNEL_QMM_NOWS) takes no
+    device memory: the stream-ordered allocator's pool does not grow across the
+    call, and the call can be recorded into a CUDA graph and replayed on new
     activations with the eager result."""
     M, K, N, G, bits = 640, 1024, 768, 64, 4
     p_ref, s_ref, b_ref = quantized(N, K, 441, True, G, bits)
     pg, sg, bg = _to_gpu(p_ref, s_ref, b_ref)
     xb1, xb2 = activations_bits(M, K, 442), activations_bits(M, K, 443)
     x = _x_gpu(xb1)
-    assert aq.aq_dispatch(M, N, K, G, bits) == aq.AQ_KERNEL_QMM
-    y_eager = aq.aq_matmul(x, pg, sg, bg, G, bits)
+    y_eager = aq.aq_matmul_with("qmm_nows", x, pg, sg, bg, G, bits)
     torch.cuda.synchronize()
     try:
+        from cuda.bindings import driver as drv
         from cuda.bindings import runtime as rt
         err, pool = rt.cudaDeviceGetDefaultMemPool(torch.cuda.current_device())
         assert err == rt.cudaError_t.cudaSuccess
         attr = rt.cudaMemPoolAttr
-        err, = rt.cudaMemPoolSetAttribute(pool, attr.cudaMemPoolAttrUsedMemHigh, rt.cuuint64_t(0))
+        err, = rt.cudaMemPoolSetAttribute(pool, attr.cudaMemPoolAttrUsedMemHigh, drv.cuuint64_t(0))
         assert err == rt.cudaError_t.cudaSuccess
         err, before = rt.cudaMemPoolGetAttribute(pool, attr.cudaMemPoolAttrUsedMemCurrent)
         have_pool = True
     except ImportError:
         have_pool = False
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    aq.aq_matmul(x, pg, sg, bg, G, bits, out=y)
+    aq.aq_matmul_with("qmm_nows", x, pg, sg, bg, G, bits, out=y)
     torch.cuda.synchronize()
     if have_pool:
         err, high = rt.cudaMemPoolGetAttribute(pool, attr.cudaMemPoolAttrUsedMemHigh)
@@ -860,7 +869,7 @@ def test_qmm_prefill_allocates_nothing_and_replays_from_a_graph():
     assert torch.equal(y.view(torch.int16), y_eager.view(torch.int16))
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        aq.aq_matmul(x, pg, sg, bg, G, bits, out=y)
+        aq.aq_matmul_with("qmm_nows", x, pg, sg, bg, G, bits, out=y)
     y.zero_()
     g.replay()
     torch.cuda.synchronize()

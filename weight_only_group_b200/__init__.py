@@ -39,10 +39,12 @@ AQ_ERR_DEVICE_FAULT = 5
 AQ_KERNEL_AUTO = 0
 AQ_KERNEL_QMV = 1
 AQ_KERNEL_QMM = 2
-AQ_KERNEL_QMV_SYNC = 3
+AQ_KERNEL_QMV_TCGEN05 = 3
+AQ_KERNEL_QMM_NOWS = 4
 AQ_MATMUL_OVERLAP_PREVIOUS = 1
 AQ_FAULT_BAD_INDEX = 0x20
-KERNELS = {"auto": AQ_KERNEL_AUTO, "qmv": AQ_KERNEL_QMV, "qmm": AQ_KERNEL_QMM, "qmv_sync": AQ_KERNEL_QMV_SYNC}
+KERNELS = {"auto": AQ_KERNEL_AUTO, "qmv": AQ_KERNEL_QMV, "qmm": AQ_KERNEL_QMM, "qmv_tcgen05": AQ_KERNEL_QMV_TCGEN05,
+           "qmm_nows": AQ_KERNEL_QMM_NOWS}
 
 _lock = threading.Lock()
 _lib = None

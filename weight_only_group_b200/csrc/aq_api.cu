@@ -244,28 +244,31 @@ static aq_status matmul_prepare(aq_kernel &kernel, const uint16_t *x, int64_t M,
     if (k < 0) return AQ_ERR_UNSUPPORTED;
     kernel = static_cast<aq_kernel>(k);
   }
-  if (kernel == AQ_KERNEL_QMV || kernel == AQ_KERNEL_QMV_SYNC)
+  if (kernel == AQ_KERNEL_QMV || kernel == AQ_KERNEL_QMV_TCGEN05)
     return qmv_fits(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
   if (kernel == AQ_KERNEL_QMM) return aq::qmm_supports(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
+  if (kernel == AQ_KERNEL_QMM_NOWS) return aq::qmm2_supports(M, N, K, G, bits) ? AQ_OK : AQ_ERR_UNSUPPORTED;
   return AQ_ERR_INVALID_ARG;
 }
 
 static size_t workspace_for(aq_kernel kernel, int64_t M, int64_t K) {
+  // AQ_KERNEL_QMM_NOWS and the decode kernels need none
   return kernel == AQ_KERNEL_QMM ? aq::qmm_workspace_bytes(M, K) : 0;
 }
 
-// ws == nullptr: the tensor-core matmul without workspace (qmm2.cu); else the
-// one that takes the fp16 activations from the caller's workspace (qmm.cu).
+// AQ_KERNEL_QMM runs with the caller's (or the stream-ordered allocator's)
+// workspace ws; AQ_KERNEL_QMM_NOWS needs none.
 static aq_status matmul_run(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                             const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
                             void *ws, aq_stream_t stream, uint32_t flags = 0) {
   aq_status st = check_device();
   if (st != AQ_OK) return st;
-  if (kernel == AQ_KERNEL_QMV && aq::qmv_umma_supported(M, N, K, G, bits))
+  if (kernel == AQ_KERNEL_QMV_TCGEN05 && aq::qmv_umma_supported(M, N, K, G, bits))
     return from_cuda(aq::launch_qmv_umma(x, M, K, packed, scales, biases, N, G, bits, y, flags, stream));
-  if (kernel == AQ_KERNEL_QMV || kernel == AQ_KERNEL_QMV_SYNC)
+  if (kernel == AQ_KERNEL_QMV || kernel == AQ_KERNEL_QMV_TCGEN05)
     return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, flags, stream));
-  if (ws == nullptr) return from_cuda(aq::launch_qmm2(x, M, K, packed, scales, biases, N, G, bits, y, stream));
+  if (kernel == AQ_KERNEL_QMM_NOWS)
+    return from_cuda(aq::launch_qmm2(x, M, K, packed, scales, biases, N, G, bits, y, stream));
   return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, ws, stream));
 }
 
@@ -294,9 +297,17 @@ aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t
                          aq_stream_t stream) {
   aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
   if (st != AQ_OK) return st;
-  // no workspace and no allocation: the tensor-core path keeps its per-row
-  // activation scales inside y (qmm2.cu)
-  return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream);
+  const size_t need = workspace_for(kernel, M, K);
+  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream);
+  if ((st = check_device()) != AQ_OK) return st;
+  // workspace from the stream-ordered allocator, released on the same stream
+  void *ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, need, stream);
+  if (e != cudaSuccess) return from_cuda(e);
+  st = matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, ws, stream);
+  e = cudaFreeAsync(ws, stream);
+  if (st == AQ_OK && e != cudaSuccess) st = from_cuda(e);
+  return st;
 }
 
 aq_status aq_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
@@ -311,7 +322,9 @@ aq_status aq_matmul_ex(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
   aq_kernel kernel = AQ_KERNEL_AUTO;
   aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
   if (st != AQ_OK) return st;
-  return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream, flags);
+  const size_t need = workspace_for(kernel, M, K);
+  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream, flags);
+  return aq_matmul_with(kernel, x, M, K, packed, scales, biases, N, G, bits, y, stream);
 }
 
 aq_status aq_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, const uint16_t *scales,

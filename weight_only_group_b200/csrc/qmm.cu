@@ -97,7 +97,22 @@ struct Params {
   __nv_bfloat16 *y;
   int M, N, K, G, Gn;
   int m_tiles, n_tiles;
+  int n_fastest;  // tile order: W-row tiles fastest (else token tiles fastest)
 };
+
+// Tile t's first token and first W row.  Token tiles fastest keeps a W tile in
+// use by many CTAs at once (the fp16 activations stay in L2); W-row tiles
+// fastest keeps an activation tile in use instead, for activations that do not
+// fit in L2.
+AQ_DEVICE void tile_origin(const Params &prm, int tile, int bn, int &m0, int &n0) {
+  if (prm.n_fastest) {
+    m0 = (tile / prm.n_tiles) * bn;
+    n0 = (tile % prm.n_tiles) * 128;
+  } else {
+    m0 = (tile % prm.m_tiles) * bn;
+    n0 = (tile / prm.m_tiles) * 128;
+  }
+}
 
 template <int BITS, int BN>
 __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant__ CUtensorMap x_map,
@@ -148,8 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % prm.m_tiles) * BN;
-        const int n0 = (tile / prm.m_tiles) * 128;
+        int m0, n0;
+        tile_origin(prm, tile, BN, m0, n0);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t r = it / S;
@@ -209,8 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
     uint32_t it0 = 0, t = 0;                    // stage counter at the start of the tile
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t, it0 += KB) {
-      const int m0 = (tile % prm.m_tiles) * BN;
-      const int n0 = (tile / prm.m_tiles) * 128;
+      int m0, n0;
+      tile_origin(prm, tile, BN, m0, n0);
       const int n = n0 + row;
       const bool row_ok = n < prm.N;
       const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
@@ -437,6 +452,14 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
   prm.Gn = static_cast<int>(K / G);
   prm.m_tiles = static_cast<int>((M + BN - 1) / BN);
   prm.n_tiles = static_cast<int>((N + 127) / 128);
+  // Tile order: the CTAs in flight share either the x16 rows of all token
+  // tiles (token tiles fastest: all of x16 stays hot in L2) or all of W (W-row
+  // tiles fastest).  Keep hot whichever of the two is smaller.
+  const int64_t w_bytes = N * K * BITS / 8 + 4 * N * (K / G);
+  prm.n_fastest = (2 * M * K > w_bytes) ? 1 : 0;
+#ifdef AQ_QMM_FORCE_ORDER  // build-time override (0: token tiles fastest, 1: W tiles fastest, else choose)
+  if (AQ_QMM_FORCE_ORDER == 0 || AQ_QMM_FORCE_ORDER == 1) prm.n_fastest = AQ_QMM_FORCE_ORDER;
+#endif
 
   auto kern = qmm_kernel<BITS, BN>;
   static thread_local int cached_dev = -1;
@@ -456,12 +479,46 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
   return cudaGetLastError();
 }
 
+// Token tile width.  The kernel is fed from L2: per K block a tile reads its
+// x16 slice (BN x BK fp16) and its packed W slice, so a narrow token tile moves
+// more bytes per multiply-add; a wide one leaves SMs idle in the last wave when
+// there are few tiles.  Score = (fraction of the SMs' waves filled) x (MACs per
+// byte read), and take the best (ties: the wider tile).
+template <int BITS>
+int pick_bn(int64_t M, int64_t N, int sms) {
+#ifdef AQ_QMM_FORCE_BN  // build-time override (64, 128 or 256; 0: choose)
+  if (AQ_QMM_FORCE_BN == 64 || AQ_QMM_FORCE_BN == 128 || AQ_QMM_FORCE_BN == 256) return AQ_QMM_FORCE_BN;
+#endif
+  auto score = [&](int64_t bn, int64_t bytes) {
+    const int64_t t = ((M + bn - 1) / bn) * ((N + 127) / 128);
+    const int64_t waves = (t + sms - 1) / sms;
+    const double fill = static_cast<double>(t) / static_cast<double>(waves * sms);
+    return fill * static_cast<double>(bn) / static_cast<double>(bytes);
+  };
+  const double s256 = score(256, Cfg<BITS, 256>::X_BYTES + Cfg<BITS, 256>::W_BYTES);
+  const double s128 = score(128, Cfg<BITS, 128>::X_BYTES + Cfg<BITS, 128>::W_BYTES);
+  const double s64 = score(64, Cfg<BITS, 64>::X_BYTES + Cfg<BITS, 64>::W_BYTES);
+  if (M > 128 && s256 >= s128 && s256 >= s64) return 256;
+  if (M > 64 && s128 >= s64) return 128;
+  return 64;
+}
+
 template <int BITS>
 cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                         const uint16_t *biases, int64_t N, int G, uint16_t *y, void *ws, cudaStream_t s) {
-  if (M <= 64) return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-  if (M <= 128) return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-  return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+  static thread_local int cached_dev = -1, sms = 148;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  switch (pick_bn<BITS>(M, N, sms)) {
+    case 64: return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case 128: return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    default: return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+  }
 }
 
 }  // namespace qmm

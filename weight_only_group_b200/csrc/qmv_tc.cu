@@ -65,15 +65,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn();  // driver entry point, resolved 
 
 namespace tc {
 
+#ifndef AQ_QMV_MAX_CONSUMERS
+#define AQ_QMV_MAX_CONSUMERS 12
+#endif
+#ifndef AQ_QMV_STAGE_TARGET
+#define AQ_QMV_STAGE_TARGET (16 * 1024)
+#endif
 constexpr int kRows = 16;           // rows of W per tile (the MMA's M)
-constexpr int kMaxConsumers = 12;   // consumer warps per CTA at most
+constexpr int kMaxConsumers = AQ_QMV_MAX_CONSUMERS;  // consumer warps per CTA at most
 constexpr int kRedBufs = 4;         // tiles whose partial sums can be in flight
 constexpr int kDualSmem = 112 * 1024;   // shared memory of a CTA that shares its SM with the next launch's
 constexpr int kDualConsumers = 8;       // consumer warps of such a CTA
 constexpr int kDualMinStages = 4;
 constexpr int kUnitCodes = 1 << 20;     // codes of a row a work unit covers at least (where the stage allows)
 constexpr int kMaxStages = 16;
-constexpr int kStageTarget = 16 * 1024;  // packed bytes of one stage we aim for (<= 1 KB per row)
+constexpr int kStageTarget = AQ_QMV_STAGE_TARGET;  // packed bytes of one stage we aim for (<= 1 KB per row)
 constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
 constexpr int kEarlyStages = 2;
 constexpr int kStageItems = 2;           // activation staging items per thread per round          // weight stages issued before the previous kernel completes (overlap mode)

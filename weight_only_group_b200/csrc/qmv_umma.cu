@@ -23,13 +23,15 @@
 //  * Warp 0 (one lane): TMA producer, 128 rows x Kc codes per stage into a
 //    ring of shared-memory stages.  Each box is 16 bytes wider than a stage's
 //    codes, so a warp's 16-byte reads of 8 consecutive rows hit all 32 banks.
-//  * Warps 2..9 (two per TMEM lane quadrant, taking stages in turn): first
+//  * Warps 2..17 (four per TMEM lane quadrant, taking stages in turn, each with
+//    its own TMEM stage): first
 //    stage this CTA's activations as the MMA's B operand (16 rows: token m's
 //    low digits in row 2m, high digits in row 2m + 1; 128-byte swizzled
 //    K-major), then per stage unpack their row's codes into bytes (three
 //    logic ops per 8 codes at 4 bits) and write them with tcgen05.st into a
-//    TMEM stage, the MMA's A operand; one stage later, read that stage's
-//    per-group accumulators back with tcgen05.ld and fold them.
+//    TMEM stage, the MMA's A operand; once the stage's MMAs are done, read its
+//    per-group accumulators back with tcgen05.ld and fold them.  The four
+//    workers of a quadrant overlap one another's MMA round trips.
 //  * Warp 1 (one lane): tcgen05.mma.kind::i8 (u8 codes x s8 digits, int32
 //    accumulate, M = 128, N = 16, K = 32), one accumulator per group, so 1 to 8
 //    tokens cost the same MMAs; warp 1 also owns the TMEM allocation.
@@ -57,11 +59,11 @@ namespace u5 {
 
 constexpr int kRows = 128;
 constexpr int kWorkerWarp0 = 2;
-constexpr int kWorkersPerQuad = 2;
+constexpr int kWorkersPerQuad = 4;  // each owns one TMEM stage: four stages in flight per quadrant
 constexpr int kWorkers = 4 * kWorkersPerQuad;
 constexpr int kThreads = 32 * (kWorkerWarp0 + kWorkers);
 constexpr int kTmemCols = 512;
-constexpr int kNT = 4;       // TMEM stages (a multiple of kWorkersPerQuad)
+constexpr int kNT = kWorkersPerQuad;  // TMEM stages, one per worker of a quadrant
 constexpr int kBRows = 16;   // B rows: 8 tokens x 2 digits
 constexpr int kSmemBudget = 224 * 1024;
 
@@ -74,7 +76,7 @@ struct Args {
   int Kr;         // K of one CTA (a multiple of Kc)
   int Kc;         // codes of a row per stage
   int nst;        // stages per CTA
-  int NS;         // shared-memory ring depth (even)
+  int NS;         // shared-memory ring depth (a multiple of kWorkersPerQuad)
   int pitch;      // bytes per row in a stage (the TMA box width)
   int stage_bytes;
   int b_off, tab_off, red_off, bar_off;
@@ -279,10 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_umma_kernel(const __grid_cons
     }
   } else {
     // ------------------------------------------------------------------ workers
-    const int wk = warp - kWorkerWarp0;       // 0..7
+    const int wk = warp - kWorkerWarp0;       // 0..15
     const int q = warp & 3;                   // TMEM lane quadrant this warp may access
-    const int h = wk >> 2;                    // 0 or 1: takes the stages st with st % 2 == h
-    const int wt = wk * 32 + lane;            // 0..255 among the workers
+    const int h = wk >> 2;                    // takes the stages st with st % kWorkersPerQuad == h (TMEM stage h)
+    const int wt = wk * 32 + lane;            // index among the workers
     constexpr int WT = kWorkers * 32;
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x may be the previous kernel's output
 
@@ -383,22 +385,33 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_umma_kernel(const __grid_cons
     for (int m = 0; m < MP; ++m) yacc[m] = 0.0f;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
 
+    // fold: the stage's per-group accumulators, read in batches of GB groups
+    // (one wait per batch), into this row's partial sums
+    constexpr int GB = 2 * MP * 4 <= 32 ? 4 : 2;
     auto fold = [&](int st, const __half (&sc)[8], const __half (&bi)[8]) -> bool {
       const int t = st % kNT;
       if (!wait(&mma_done[t], (st / kNT) & 1, abort_flag, wlim)) return false;
       qmm::tc_fence_after();
-      for (int j = 0; j < GPS; ++j) {
-        uint32_t v[2 * MP];
-        tmem_ld_cols<MP>(lane_base + acc_col(t) + j * 16, v);
-        qmm::tmem_ld_wait();
-        const float s = __half2float(sc[j]), b = __half2float(bi[j]);
-        const int g = st * GPS + j;
+      for (int j0 = 0; j0 < GPS; j0 += GB) {
+        uint32_t v[GB][2 * MP];
 #pragma unroll
-        for (int m = 0; m < MP; ++m) {
-          if (m < a.M) {
-            const float4 T = tab[m * Gr + g];
-            const float D = static_cast<float>(static_cast<int>(v[2 * m]) + 256 * static_cast<int>(v[2 * m + 1]));
-            yacc[m] = fmaf(s * T.z, D * T.y, fmaf(b, T.x, yacc[m]));
+        for (int jj = 0; jj < GB; ++jj)
+          if (j0 + jj < GPS) tmem_ld_cols<MP>(lane_base + acc_col(t) + (j0 + jj) * 16, v[jj]);
+        qmm::tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < GB; ++jj) {
+          const int j = j0 + jj;
+          if (j >= GPS) break;
+          const float s = __half2float(sc[j]), b = __half2float(bi[j]);
+          const int g = st * GPS + j;
+#pragma unroll
+          for (int m = 0; m < MP; ++m) {
+            if (m < a.M) {
+              const float4 T = tab[m * Gr + g];
+              const float D =
+                  static_cast<float>(static_cast<int>(v[jj][2 * m]) + 256 * static_cast<int>(v[jj][2 * m + 1]));
+              yacc[m] = fmaf(s * T.z, D * T.y, fmaf(b, T.x, yacc[m]));
+            }
           }
         }
       }
@@ -406,11 +419,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_umma_kernel(const __grid_cons
     };
 
     bool ok = true;
-    __half sc_prev[8], bi_prev[8], sc_cur[8], bi_cur[8];
-    int prev = -1;
+    __half sc_cur[8], bi_cur[8];
     for (int st = h; st < a.nst; st += kWorkersPerQuad) {
-      const int s = st % a.NS, t = st % kNT;
-      // this stage's scales and biases (read here, used one stage later by the fold)
+      const int s = st % a.NS, t = st % kNT;  // t == h: this worker's TMEM stage
+      // this stage's scales and biases (used by the fold below)
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const bool in = j < GPS && row_ok;
@@ -418,9 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_umma_kernel(const __grid_cons
         bi_cur[j] = in ? __ldg(a.biases + gbase + st * GPS + j) : __float2half(0.0f);
       }
       if (!(ok = wait(&full[s], (st / a.NS) & 1, abort_flag, wlim))) break;
-      if (st >= kNT && !(ok = wait(&mma_done[t], ((st / kNT) - 1) & 1, abort_flag, wlim))) break;
       __syncwarp();
       // unpack this row's codes into bytes, 32 codes (8 TMEM columns) at a time
+      // (the TMEM stage is free: this warp folded its previous stage, whose MMAs were done)
       const uint32_t *wr = reinterpret_cast<const uint32_t *>(ring + static_cast<size_t>(s) * a.stage_bytes +
                                                                static_cast<size_t>(r) * a.pitch);
       for (int ks = 0; ks < a.Kc / 32; ++ks) {
@@ -458,23 +470,19 @@ __global__ void __launch_bounds__(kThreads, 1) qmv_umma_kernel(const __grid_cons
         mbar_arrive(&a_full[t]);
         mbar_arrive(&empty[s]);
       }
-      // fold this warp's previous stage while the MMAs of this one run
-      if (prev >= 0 && !(ok = fold(prev, sc_prev, bi_prev))) break;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        sc_prev[j] = sc_cur[j];
-        bi_prev[j] = bi_cur[j];
-      }
-      prev = st;
+      if (!(ok = fold(st, sc_cur, bi_cur))) break;
     }
-    if (ok && prev >= 0) ok = fold(prev, sc_prev, bi_prev);
-    // the two warps of a quadrant: sum their partials
+    // the warps of a quadrant: sum their partials (in worker order)
 #pragma unroll
     for (int m = 0; m < MP; ++m) red[(h * kRows + r) * MP + m] = yacc[m];
     asm volatile("bar.sync 1, %0;" ::"n"(WT) : "memory");
     if (h == 0) {
 #pragma unroll
-      for (int m = 0; m < MP; ++m) red[r * MP + m] = yacc[m] + red[(kRows + r) * MP + m];
+      for (int m = 0; m < MP; ++m) {
+        float sum = yacc[m];
+        for (int w = 1; w < kWorkersPerQuad; ++w) sum += red[(w * kRows + r) * MP + m];
+        red[r * MP + m] = sum;
+      }
     }
   }
 
@@ -569,7 +577,7 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
     return off + 1024;  // alignment slack of the dynamic shared memory base
   };
   int ns = 0;
-  for (int c = 2; c <= 16; c += 2)
+  for (int c = kWorkersPerQuad; c <= 16; c += kWorkersPerQuad)
     if (total(c) <= kSmemBudget) ns = c;
   if (ns == 0) return false;
   a.NS = ns;
