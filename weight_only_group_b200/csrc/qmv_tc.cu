@@ -11,8 +11,8 @@
 // extraction plus one FMA per weight and activation reads from shared memory
 // took longer than streaming the weights at B200's HBM rate (measured: the
 // arithmetic of a 14336x4096 4-bit call alone ran 1.4x longer than its copies
-// alone).  Here the integer tensor cores (mma.sync m16n8k32, u8 x u8 / u8 x s8,
-// int32 accumulate) do the multiply-adds and the CUDA cores only unpack codes
+// alone).  Here the integer tensor cores (mma.sync m16n8k32, u8 x s8, int32
+// accumulate) do the multiply-adds and the CUDA cores only unpack codes
 // into bytes: three logic ops per 8 codes at 4 bits, none at 8 bits.  mma.sync
 // rather than tcgen05: its B operand sits in registers, so the per-lane zero
 // masking below costs one select per group, while a shared-memory B operand
@@ -26,14 +26,20 @@
 //  * Activations: per group, x_int = rint(x * 2^e) with 2^e the power of two
 //    that puts the group's largest |x| in [2^13, 2^14), so |x_int| <= 2^14
 //    and the rounding error is at most 2^-14 of the group's largest |x|.
-//    x_int = 256 * hi + lo with lo in [0, 255] (u8) and hi in [-64, 64] (s8);
-//    two MMAs per A tile give sum q*lo and sum q*hi exactly in int32.
-//  * MMA columns: with MP = M rounded up to a power of two, column n is token
-//    n / (8/MP) and group slot n % (8/MP).  A lane reads the real activations
-//    only while the current group's slot is its column's slot, and zeros
-//    otherwise, so one accumulator holds 8/MP groups side by side and is
-//    folded once per 8/MP groups:
+//    x_int = 256 * hi + lo with signed digits, lo in [-128, 127] and hi in
+//    [-64, 64]; u8 codes x s8 digits give sum q*lo and sum q*hi exactly in
+//    int32.
+//  * MMA columns (affine codes): column n = 2p + d holds digit plane d of
+//    position p, so one MMA per A tile yields both digit sums.  With MP = M
+//    rounded up to a power of two, the four positions of an MMA are tokens
+//    p / (4/MP) and group slots p % (4/MP) (MP <= 4), or four tokens (MP = 8,
+//    two MMAs per A tile).  A lane reads the real activations only while the
+//    current group's slot is its column's slot, and zeros otherwise, so one
+//    accumulator holds 4/MP groups side by side and is folded once per 4/MP
+//    groups:
 //        y += s * 2^-e * (256 * D_hi + D_lo) + b * sum x
+//    (The block-scaled formats keep one digit plane per MMA, columns = token x
+//    group slot, 8/MP slots per fold.)
 //  * Streaming: a producer warp copies (16-row tile, K chunk) stages into a
 //    shared-memory ring: three 2-D TMA boxes (codes, scales, biases; 64-bit
 //    elements, box rows padded so that the lanes of one shared-memory read hit
@@ -288,6 +294,14 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   // accumulator chains per digit plane: a group folded on its own has only
   // G/32 MMAs per plane, and summing chains would cost more than it hides
   constexpr int NACC = GS == 1 ? 1 : kAcc;
+  // Affine codes (FMT 0): both digit planes go through one MMA, in adjacent
+  // columns (column 2p + d: position p, digit d, both digits signed bytes), so
+  // one MMA per K tile serves up to four tokens.  Position p is token p / GS1,
+  // group slot p % GS1 of the fold.
+  constexpr int TPM = MP >= 4 ? 4 : MP;   // tokens per MMA
+  constexpr int NMMA = MP > 4 ? 2 : 1;    // MMAs per K tile (token halves)
+  constexpr int GS1 = 4 / TPM;            // group slots per fold
+  constexpr int NACC1 = GS1 == 1 ? 1 : kAcc;
   using Span = LaneSpan<BITS, G, FMT>;
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -491,14 +505,20 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           }
           uint32_t lo[2], hi[2];
           static_for<0, 2>([&](auto S) {
-            // rint(v * 2^e) lands in the low 22 bits of v * 2^e + 1.5 * 2^23; its
-            // bytes 0 and 1 are the two's-complement digits lo and hi
-            uint32_t f[4];
+            // x_int = rint(v * 2^e) lands in the low 22 bits of v * 2^e + 1.5 * 2^23
+            // (two's complement).  Signed digits x_int = 256 * hi + lo with lo in
+            // [-128, 127] and hi in [-64, 64]: lo is byte 0 of x_int, hi is
+            // byte 1 of x_int + 128 (an integer add on the bit pattern).
+            uint32_t f[4], f2[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) f[i] = __float_as_uint(fmaf(v8[j][c][4 * S.value + i], sc, kRoundMagic));
-            const uint32_t t01 = __byte_perm(f[0], f[1], 0x5140), t23 = __byte_perm(f[2], f[3], 0x5140);
+            for (int i = 0; i < 4; ++i) {
+              f[i] = __float_as_uint(fmaf(v8[j][c][4 * S.value + i], sc, kRoundMagic));
+              f2[i] = f[i] + 128u;
+            }
+            const uint32_t t01 = __byte_perm(f[0], f[1], 0x40), t23 = __byte_perm(f[2], f[3], 0x40);
+            const uint32_t u01 = __byte_perm(f2[0], f2[1], 0x51), u23 = __byte_perm(f2[2], f2[3], 0x51);
             lo[S.value] = __byte_perm(t01, t23, 0x5410);
-            hi[S.value] = __byte_perm(t01, t23, 0x7632);
+            hi[S.value] = __byte_perm(u01, u23, 0x5410);
           });
           if (act[j]) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(lo[0], lo[1], hi[0], hi[1]);
         });
@@ -524,8 +544,20 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   const uint8_t *xs_lane = xs + (my_real ? my_m : 0) * a.tok_stride + t * 16;
   const uint8_t *zero_lane = zero + (GS == 1 ? 0 : (my_m & 1)) * a.zero_stride + t * 16;
   const int lw0 = LaneWords<BITS, G>::first(t) * 4;
-  constexpr int SPANS = FMT == 2 ? GS / 2 : GS;  // 32-code spans (MMA K steps) per fold
+  constexpr int SPANS = FMT == 0 ? GS1 : FMT == 2 ? GS / 2 : GS;  // 32-code spans (MMA K steps) per fold
   const float gs = FMT == 2 ? __ldg(a.gscale) : 1.0f;
+  // FMT 0: B column g = 2p + d of this lane (token, slot and digit plane it
+  // feeds) and the accumulator columns 2t, 2t+1 it receives (position t)
+  const int b_slot = (g >> 1) % GS1;
+  int b_tok[NMMA];
+  const uint8_t *b_lane[NMMA];
+#pragma unroll
+  for (int h = 0; h < NMMA; ++h) {
+    b_tok[h] = h * 4 + (g >> 1) / GS1;
+    b_lane[h] = xs + (b_tok[h] < a.M ? b_tok[h] : 0) * a.tok_stride + t * 16 + (g & 1) * 8;
+  }
+  const uint8_t *zb_lane = zero + t * 16 + (g & 1) * 8;
+  const int c_slot = t % GS1;
 
   // Work units: unit u is fold p of stage st (u = st * nper + p), dealt to the
   // consumer warps round-robin, so a stage is shared by several warps and the
@@ -546,205 +578,281 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     const uint8_t *sr0 = stg + a.s_off + g * a.pitch_s, *sr1 = sr0 + 8 * a.pitch_s;
     const uint8_t *br0 = stg + a.b_off + g * a.pitch_s, *br1 = br0 + 8 * a.pitch_s;
     const int gch0 = ch * gpc;
-    float2 accA = make_float2(0.0f, 0.0f), accB = make_float2(0.0f, 0.0f);  // rows g, g+8 x columns 2t, 2t+1
-
-    for (int pf = p * a.fpu; pf < (p + 1) * a.fpu; ++pf) {  // the unit's folds
-      int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
-      // mxfp4: the same sums over the negative codes' magnitudes, subtracted below
-      int nl[FMT >= 1 ? NACC : 1][4], nh[FMT >= 1 ? NACC : 1][4];
-      float fa[FMT == 3 ? NACC : 1][4];  // mxfp8: fp32 accumulators of the f16 MMAs
+    // Per (row, token) partials of this unit, held by some lanes: value q is
+    // (row vrow[q], token vtok[q]) of the tile.
+    float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    int vrow[4] = {0, 0, 0, 0}, vtok[4] = {0, 0, 0, 0};
+    int nv = 0;
+    bool holder = false;
+    if constexpr (FMT == 0) {
+      float2 acc1[NMMA];  // rows (g, g+8) of token h * 4 + t / GS1
 #pragma unroll
-      for (int i = 0; i < NACC; ++i) dl[i][0] = dl[i][1] = dl[i][2] = dl[i][3] = dh[i][0] = dh[i][1] = dh[i][2] = dh[i][3] = 0;
-      if constexpr (FMT == 1 || FMT == 2) {
+      for (int h = 0; h < NMMA; ++h) acc1[h] = make_float2(0.0f, 0.0f);
+      for (int pf = p * a.fpu; pf < (p + 1) * a.fpu; ++pf) {  // the unit's folds
+        int dd[NMMA][NACC1][4];  // (lo, hi) digit sums of rows g and g+8 at position t
 #pragma unroll
-        for (int i = 0; i < NACC; ++i) nl[i][0] = nl[i][1] = nl[i][2] = nl[i][3] = nh[i][0] = nh[i][1] = nh[i][2] = nh[i][3] = 0;
-      }
-      if constexpr (FMT == 3) {
+        for (int h = 0; h < NMMA; ++h)
 #pragma unroll
-        for (int i = 0; i < NACC; ++i) fa[i][0] = fa[i][1] = fa[i][2] = fa[i][3] = 0.0f;
-      }
-      static_for<0, SPANS>([&](auto J) {
-        constexpr int j = J.value;
-        const int gi = pf * SPANS + j;
-        uint32_t w0[NWD], w1[NWD];
-        lds_words<NWD>(wr0 + gi * GBYTES, w0);
-        lds_words<NWD>(wr1 + gi * GBYTES, w1);
-        // nvfp4: the span's first 16 codes (lanes t = 0, 1) go to slot 2j, the
-        // other 16 (t = 2, 3) to slot 2j + 1
-        const bool live = my_real && (FMT == 2 ? my_j == 2 * j + (t >> 1) : my_j == j);
-        const uint8_t *bp = live ? xs_lane + (gch0 + gi) * (U * 64) : zero_lane;
-        static_for<0, U>([&](auto C) {
-          constexpr int c = C.value;
-          const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);  // lo set 0, lo set 1, hi set 0, hi set 1
-          uint32_t q0[2], q1[2];
-          constexpr int k = (j * U + c) % NACC;
-          if constexpr (FMT == 3) {
-            // two k16 MMAs: codes 0..3 of the lane's run (words w[0]), then 4..7 (w[1])
-            mma_f16(fa[k], e4m3x2_to_f16x2(w0[0]), e4m3x2_to_f16x2(w1[0]), e4m3x2_to_f16x2(w0[0] >> 16),
-                    e4m3x2_to_f16x2(w1[0] >> 16), bv.x, bv.y);
-            mma_f16(fa[(k + 1) % NACC], e4m3x2_to_f16x2(w0[1]), e4m3x2_to_f16x2(w1[1]), e4m3x2_to_f16x2(w0[1] >> 16),
-                    e4m3x2_to_f16x2(w1[1] >> 16), bv.z, bv.w);
-          } else if constexpr (FMT >= 1) {
-            uint32_t n0[2], n1[2];
-            e2m1x2_split(w0[0], q0, n0);
-            e2m1x2_split(w1[0], q1, n1);
-            mma_u8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
-            mma_u8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
-            mma_u8u8(nl[k], n0[0], n1[0], n0[1], n1[1], bv.x, bv.y);
-            mma_u8s8(nh[k], n0[0], n1[0], n0[1], n1[1], bv.z, bv.w);
-          } else {
+          for (int i = 0; i < NACC1; ++i) dd[h][i][0] = dd[h][i][1] = dd[h][i][2] = dd[h][i][3] = 0;
+        static_for<0, SPANS>([&](auto J) {
+          constexpr int j = J.value;
+          const int gi = pf * SPANS + j;
+          uint32_t w0[NWD], w1[NWD];
+          lds_words<NWD>(wr0 + gi * GBYTES, w0);
+          lds_words<NWD>(wr1 + gi * GBYTES, w1);
+          static_for<0, U>([&](auto C) {
+            constexpr int c = C.value;
+            constexpr int k = (j * U + c) % NACC1;
+            uint32_t q0[2], q1[2];
             tile_codes<BITS, G, c>(w0, t, q0);
             tile_codes<BITS, G, c>(w1, t, q1);
-            mma_u8u8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
-            mma_u8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
-          }
+            static_for<0, NMMA>([&](auto H) {
+              constexpr int h = H.value;
+              const bool live = b_slot == j && b_tok[h] < a.M;
+              const uint8_t *bp = live ? b_lane[h] + (gch0 + gi) * (U * 64) + c * 64 : zb_lane + c * 64;
+              const uint2 bv = *reinterpret_cast<const uint2 *>(bp);
+              mma_u8s8(dd[h][k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
+            });
+          });
         });
-      });
-      float D[4];  // sum_k q_k x_int_k of the lane's 4 (row, column) cells, exact in int32
+        // fold: y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x, rows g and g+8 side by side
+        const int gl = pf * SPANS + c_slot;
+        const float2 sv = make_float2(__half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2)),
+                                      __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2)));
+        const float2 bv2 = make_float2(__half2float(*reinterpret_cast<const __half *>(br0 + gl * 2)),
+                                       __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2)));
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        int lo = dl[0][i], hi = dh[0][i];
+        for (int h = 0; h < NMMA; ++h) {
+          int lo0 = dd[h][0][0], hi0 = dd[h][0][1], lo1 = dd[h][0][2], hi1 = dd[h][0][3];
 #pragma unroll
-        for (int c = 1; c < NACC; ++c) {
-          lo += dl[c][i];
-          hi += dh[c][i];
+          for (int i = 1; i < NACC1; ++i) {
+            lo0 += dd[h][i][0];
+            hi0 += dd[h][i][1];
+            lo1 += dd[h][i][2];
+            hi1 += dd[h][i][3];
+          }
+          const float2 D = make_float2(static_cast<float>(lo0 + 256 * hi0), static_cast<float>(lo1 + 256 * hi1));
+          const float4 T4 = tab[(h * 4 + t / GS1) * a.Gn + gch0 + gl];
+          acc1[h] = ffma2(__fmul2_rn(sv, make_float2(T4.z, T4.z)), __fmul2_rn(D, make_float2(T4.y, T4.y)),
+                          ffma2(bv2, make_float2(T4.x, T4.x), acc1[h]));
         }
-        if constexpr (FMT == 1 || FMT == 2) {
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      // the lanes of one token (t / GS1 equal) sum their group slots
 #pragma unroll
-          for (int c = 0; c < NACC; ++c) {
-            lo -= nl[c][i];
-            hi -= nh[c][i];
+      for (int h = 0; h < NMMA; ++h) {
+        float e0 = acc1[h].x, e1 = acc1[h].y;
+        if constexpr (GS1 >= 2) {
+          e0 += __shfl_xor_sync(0xffffffffu, e0, 1);
+          e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
+        }
+        if constexpr (GS1 >= 4) {
+          e0 += __shfl_xor_sync(0xffffffffu, e0, 2);
+          e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
+        }
+        v[2 * h] = e0;
+        v[2 * h + 1] = e1;
+        vrow[2 * h] = g;
+        vrow[2 * h + 1] = g + 8;
+        vtok[2 * h] = vtok[2 * h + 1] = h * 4 + t / GS1;
+      }
+      nv = 2 * NMMA;
+      holder = c_slot == 0;
+    } else {
+      float2 accA = make_float2(0.0f, 0.0f), accB = make_float2(0.0f, 0.0f);  // rows g, g+8 x columns 2t, 2t+1
+
+      for (int pf = p * a.fpu; pf < (p + 1) * a.fpu; ++pf) {  // the unit's folds
+        int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
+        // mxfp4: the same sums over the negative codes' magnitudes, subtracted below
+        int nl[FMT >= 1 ? NACC : 1][4], nh[FMT >= 1 ? NACC : 1][4];
+        float fa[FMT == 3 ? NACC : 1][4];  // mxfp8: fp32 accumulators of the f16 MMAs
+  #pragma unroll
+        for (int i = 0; i < NACC; ++i) dl[i][0] = dl[i][1] = dl[i][2] = dl[i][3] = dh[i][0] = dh[i][1] = dh[i][2] = dh[i][3] = 0;
+        if constexpr (FMT == 1 || FMT == 2) {
+  #pragma unroll
+          for (int i = 0; i < NACC; ++i) nl[i][0] = nl[i][1] = nl[i][2] = nl[i][3] = nh[i][0] = nh[i][1] = nh[i][2] = nh[i][3] = 0;
+        }
+        if constexpr (FMT == 3) {
+  #pragma unroll
+          for (int i = 0; i < NACC; ++i) fa[i][0] = fa[i][1] = fa[i][2] = fa[i][3] = 0.0f;
+        }
+        static_for<0, SPANS>([&](auto J) {
+          constexpr int j = J.value;
+          const int gi = pf * SPANS + j;
+          uint32_t w0[NWD], w1[NWD];
+          lds_words<NWD>(wr0 + gi * GBYTES, w0);
+          lds_words<NWD>(wr1 + gi * GBYTES, w1);
+          // nvfp4: the span's first 16 codes (lanes t = 0, 1) go to slot 2j, the
+          // other 16 (t = 2, 3) to slot 2j + 1
+          const bool live = my_real && (FMT == 2 ? my_j == 2 * j + (t >> 1) : my_j == j);
+          const uint8_t *bp = live ? xs_lane + (gch0 + gi) * (U * 64) : zero_lane;
+          static_for<0, U>([&](auto C) {
+            constexpr int c = C.value;
+            const uint4 bv = *reinterpret_cast<const uint4 *>(bp + c * 64);  // lo set 0, lo set 1, hi set 0, hi set 1
+            uint32_t q0[2], q1[2];
+            constexpr int k = (j * U + c) % NACC;
+            if constexpr (FMT == 3) {
+              // two k16 MMAs: codes 0..3 of the lane's run (words w[0]), then 4..7 (w[1])
+              mma_f16(fa[k], e4m3x2_to_f16x2(w0[0]), e4m3x2_to_f16x2(w1[0]), e4m3x2_to_f16x2(w0[0] >> 16),
+                      e4m3x2_to_f16x2(w1[0] >> 16), bv.x, bv.y);
+              mma_f16(fa[(k + 1) % NACC], e4m3x2_to_f16x2(w0[1]), e4m3x2_to_f16x2(w1[1]), e4m3x2_to_f16x2(w0[1] >> 16),
+                      e4m3x2_to_f16x2(w1[1] >> 16), bv.z, bv.w);
+            } else if constexpr (FMT >= 1) {
+              uint32_t n0[2], n1[2];
+              e2m1x2_split(w0[0], q0, n0);
+              e2m1x2_split(w1[0], q1, n1);
+              mma_u8s8(dl[k], q0[0], q1[0], q0[1], q1[1], bv.x, bv.y);
+              mma_u8s8(dh[k], q0[0], q1[0], q0[1], q1[1], bv.z, bv.w);
+              mma_u8s8(nl[k], n0[0], n1[0], n0[1], n1[1], bv.x, bv.y);
+              mma_u8s8(nh[k], n0[0], n1[0], n0[1], n1[1], bv.z, bv.w);
+            }
+          });
+        });
+        float D[4];  // sum_k q_k x_int_k of the lane's 4 (row, column) cells, exact in int32
+  #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int lo = dl[0][i], hi = dh[0][i];
+  #pragma unroll
+          for (int c = 1; c < NACC; ++c) {
+            lo += dl[c][i];
+            hi += dh[c][i];
+          }
+          if constexpr (FMT == 1 || FMT == 2) {
+  #pragma unroll
+            for (int c = 0; c < NACC; ++c) {
+              lo -= nl[c][i];
+              hi -= nh[c][i];
+            }
+          }
+          if constexpr (FMT == 3) {  // fp32 sums of the f16 products
+            float f = fa[0][i];
+  #pragma unroll
+            for (int c = 1; c < NACC; ++c) f += fa[c][i];
+            D[i] = f;
+          } else {
+            D[i] = static_cast<float>(hi * 256 + lo);
           }
         }
-        if constexpr (FMT == 3) {  // fp32 sums of the f16 products
-          float f = fa[0][i];
-#pragma unroll
-          for (int c = 1; c < NACC; ++c) f += fa[c][i];
-          D[i] = f;
+        // fold: D[0] = (row g, col 2t), D[1] = (row g, col 2t+1), D[2], D[3] = rows g+8.
+        // The two columns of a row go through packed fp32x2 operations.
+        float2 s0, s1, b0, b1;  // scale and bias of (row g | g+8) for columns 2t, 2t+1
+        float4 T0, T1;          // (sum x, 2^-e_lo, 2^-e_hi, 0) of columns 2t, 2t+1
+        if constexpr (GS >= 2) {
+          const int gl = pf * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
+          const int mt = (2 * t) / GS;
+          if constexpr (FMT == 2) {  // two E4M3 bytes per row (16-groups gl, gl + 1, one span); no bias
+            const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
+            const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
+            s0 = make_float2(e4m3_half(e0 & 0xFFu), e4m3_half(e0 >> 8));
+            s1 = make_float2(e4m3_half(e1 & 0xFFu), e4m3_half(e1 >> 8));
+            b0 = b1 = make_float2(0.0f, 0.0f);
+          } else if constexpr (FMT == 3) {  // two E8M0 bytes per row (groups gl, gl + 1): X; no bias
+            const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
+            const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
+            s0 = make_float2(e8m0_full(e0 & 0xFFu), e8m0_full(e0 >> 8));
+            s1 = make_float2(e8m0_full(e1 & 0xFFu), e8m0_full(e1 >> 8));
+            b0 = b1 = make_float2(0.0f, 0.0f);
+          } else if constexpr (FMT == 1) {  // two E8M0 bytes per row (groups gl, gl + 1); no bias
+            const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
+            const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
+            s0 = make_float2(e8m0_half(e0 & 0xFFu), e8m0_half(e0 >> 8));
+            s1 = make_float2(e8m0_half(e1 & 0xFFu), e8m0_half(e1 >> 8));
+            b0 = b1 = make_float2(0.0f, 0.0f);
+          } else {
+            s0 = __half22float2(*reinterpret_cast<const __half2 *>(sr0 + gl * 2));
+            s1 = __half22float2(*reinterpret_cast<const __half2 *>(sr1 + gl * 2));
+            b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
+            b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
+          }
+          if constexpr (FMT == 2) {  // both columns lie in span gl / 2 of the chunk
+            T0 = T1 = tab[mt * a.Gn + gch0 + gl / 2];
+          } else {
+            T0 = tab[mt * a.Gn + gch0 + gl];
+            T1 = tab[mt * a.Gn + gch0 + gl + 1];
+          }
         } else {
-          D[i] = static_cast<float>(hi * 256 + lo);
+          const int gl = pf;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
+          float sv0, sv1, bv0 = 0.0f, bv1 = 0.0f;
+          if constexpr (FMT == 1) {
+            sv0 = e8m0_half(sr0[gl]);
+            sv1 = e8m0_half(sr1[gl]);
+          } else if constexpr (FMT == 3) {
+            sv0 = e8m0_full(sr0[gl]);
+            sv1 = e8m0_full(sr1[gl]);
+          } else {
+            sv0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
+            sv1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
+            bv0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
+            bv1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
+          }
+          s0 = make_float2(sv0, sv0);
+          s1 = make_float2(sv1, sv1);
+          b0 = make_float2(bv0, bv0);
+          b1 = make_float2(bv1, bv1);
+          T0 = tab[(2 * t) * a.Gn + gch0 + gl];
+          T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
+        }
+        const float2 tx = make_float2(T0.x, T1.x), ty = make_float2(T0.y, T1.y), tz = make_float2(T0.z, T1.z);
+        // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x   (block-scaled modes: no bias)
+        if constexpr (FMT >= 1) {
+          accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), accA);
+          accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), accB);
+        } else {
+          accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), ffma2(b0, tx, accA));
+          accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), ffma2(b1, tx, accB));
         }
       }
-      // fold: D[0] = (row g, col 2t), D[1] = (row g, col 2t+1), D[2], D[3] = rows g+8.
-      // The two columns of a row go through packed fp32x2 operations.
-      float2 s0, s1, b0, b1;  // scale and bias of (row g | g+8) for columns 2t, 2t+1
-      float4 T0, T1;          // (sum x, 2^-e_lo, 2^-e_hi, 0) of columns 2t, 2t+1
-      if constexpr (GS >= 2) {
-        const int gl = pf * GS + (2 * t) % GS;  // group (in the chunk) of column 2t; 2t+1 is the next one
-        const int mt = (2 * t) / GS;
-        if constexpr (FMT == 2) {  // two E4M3 bytes per row (16-groups gl, gl + 1, one span); no bias
-          const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
-          const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
-          s0 = make_float2(e4m3_half(e0 & 0xFFu), e4m3_half(e0 >> 8));
-          s1 = make_float2(e4m3_half(e1 & 0xFFu), e4m3_half(e1 >> 8));
-          b0 = b1 = make_float2(0.0f, 0.0f);
-        } else if constexpr (FMT == 3) {  // two E8M0 bytes per row (groups gl, gl + 1): X; no bias
-          const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
-          const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
-          s0 = make_float2(e8m0_full(e0 & 0xFFu), e8m0_full(e0 >> 8));
-          s1 = make_float2(e8m0_full(e1 & 0xFFu), e8m0_full(e1 >> 8));
-          b0 = b1 = make_float2(0.0f, 0.0f);
-        } else if constexpr (FMT == 1) {  // two E8M0 bytes per row (groups gl, gl + 1); no bias
-          const uint32_t e0 = *reinterpret_cast<const uint16_t *>(sr0 + gl);
-          const uint32_t e1 = *reinterpret_cast<const uint16_t *>(sr1 + gl);
-          s0 = make_float2(e8m0_half(e0 & 0xFFu), e8m0_half(e0 >> 8));
-          s1 = make_float2(e8m0_half(e1 & 0xFFu), e8m0_half(e1 >> 8));
-          b0 = b1 = make_float2(0.0f, 0.0f);
-        } else {
-          s0 = __half22float2(*reinterpret_cast<const __half2 *>(sr0 + gl * 2));
-          s1 = __half22float2(*reinterpret_cast<const __half2 *>(sr1 + gl * 2));
-          b0 = __half22float2(*reinterpret_cast<const __half2 *>(br0 + gl * 2));
-          b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
-        }
-        if constexpr (FMT == 2) {  // both columns lie in span gl / 2 of the chunk
-          T0 = T1 = tab[mt * a.Gn + gch0 + gl / 2];
-        } else {
-          T0 = tab[mt * a.Gn + gch0 + gl];
-          T1 = tab[mt * a.Gn + gch0 + gl + 1];
-        }
-      } else {
-        const int gl = pf;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
-        float sv0, sv1, bv0 = 0.0f, bv1 = 0.0f;
-        if constexpr (FMT == 1) {
-          sv0 = e8m0_half(sr0[gl]);
-          sv1 = e8m0_half(sr1[gl]);
-        } else if constexpr (FMT == 3) {
-          sv0 = e8m0_full(sr0[gl]);
-          sv1 = e8m0_full(sr1[gl]);
-        } else {
-          sv0 = __half2float(*reinterpret_cast<const __half *>(sr0 + gl * 2));
-          sv1 = __half2float(*reinterpret_cast<const __half *>(sr1 + gl * 2));
-          bv0 = __half2float(*reinterpret_cast<const __half *>(br0 + gl * 2));
-          bv1 = __half2float(*reinterpret_cast<const __half *>(br1 + gl * 2));
-        }
-        s0 = make_float2(sv0, sv0);
-        s1 = make_float2(sv1, sv1);
-        b0 = make_float2(bv0, bv0);
-        b1 = make_float2(bv1, bv1);
-        T0 = tab[(2 * t) * a.Gn + gch0 + gl];
-        T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
-      }
-      const float2 tx = make_float2(T0.x, T1.x), ty = make_float2(T0.y, T1.y), tz = make_float2(T0.z, T1.z);
-      // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x   (block-scaled modes: no bias)
-      if constexpr (FMT >= 1) {
-        accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), accA);
-        accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), accB);
-      } else {
-        accA = ffma2(__fmul2_rn(s0, tz), __fmul2_rn(make_float2(D[0], D[1]), ty), ffma2(b0, tx, accA));
-        accB = ffma2(__fmul2_rn(s1, tz), __fmul2_rn(make_float2(D[2], D[3]), ty), ffma2(b1, tx, accB));
-      }
-    }
-    const float acc[4] = {accA.x, accA.y, accB.x, accB.y};
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+      const float acc[4] = {accA.x, accA.y, accB.x, accB.y};
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
 
-    // Per (row, token) partials of this chunk: GS >= 2 sums the lane's two
-    // columns (same token) and then the lanes sharing the token.
-    float v[4];
-    if constexpr (GS >= 2) {
-      v[0] = acc[0] + acc[1];
-      v[1] = acc[2] + acc[3];
-      if constexpr (GS >= 4) {
-        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-        v[1] += __shfl_xor_sync(0xffffffffu, v[1], 1);
+      // Per (row, token) partials of this chunk: GS >= 2 sums the lane's two
+      // columns (same token) and then the lanes sharing the token.
+      if constexpr (GS >= 2) {
+        v[0] = acc[0] + acc[1];
+        v[1] = acc[2] + acc[3];
+        if constexpr (GS >= 4) {
+          v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+          v[1] += __shfl_xor_sync(0xffffffffu, v[1], 1);
+        }
+        if constexpr (GS >= 8) {
+          v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
+          v[1] += __shfl_xor_sync(0xffffffffu, v[1], 2);
+        }
+      } else {
+        v[0] = acc[0];
+        v[1] = acc[1];
+        v[2] = acc[2];
+        v[3] = acc[3];
       }
-      if constexpr (GS >= 8) {
-        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 2);
-        v[1] += __shfl_xor_sync(0xffffffffu, v[1], 2);
+      // holder lanes: GS >= 2 -> lanes with t % (GS/2) == 0 hold (rows g, g+8; token 2t/GS)
+      //               GS == 1 -> every lane holds (rows g, g+8; tokens 2t, 2t+1)
+      holder = (GS == 1) || (t % (GS / 2 > 0 ? GS / 2 : 1) == 0);
+      if constexpr (GS >= 2) {
+        nv = 2;
+        vrow[0] = g;
+        vrow[1] = g + 8;
+        vtok[0] = vtok[1] = (2 * t) / GS;
+      } else {
+        nv = 4;
+  #pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          vrow[q] = g + 8 * (q >> 1);
+          vtok[q] = 2 * t + (q & 1);
+        }
       }
-    } else {
-      v[0] = acc[0];
-      v[1] = acc[1];
-      v[2] = acc[2];
-      v[3] = acc[3];
     }
-    // holder lanes: GS >= 2 -> lanes with t % (GS/2) == 0 hold (rows g, g+8; token 2t/GS)
-    //               GS == 1 -> every lane holds (rows g, g+8; tokens 2t, 2t+1)
-    const bool holder = (GS == 1) || (t % (GS / 2 > 0 ? GS / 2 : 1) == 0);
     auto put = [&](float *dstv, bool direct) {
       if (!holder) return;
-      if constexpr (GS >= 2) {
-        const int tok = (2 * t) / GS;
-        if (direct) {
-          if (tok < a.M) {
-            if (row_ok(g)) yg[static_cast<int64_t>(tok) * a.N + rb + g] = __float2bfloat16_rn(FMT == 2 ? v[0] * gs : v[0]);
-            if (row_ok(g + 8))
-              yg[static_cast<int64_t>(tok) * a.N + rb + g + 8] = __float2bfloat16_rn(FMT == 2 ? v[1] * gs : v[1]);
-          }
-        } else {
-          dstv[g * MP + tok] = v[0];
-          dstv[(g + 8) * MP + tok] = v[1];
-        }
-      } else {
-        if (direct) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int tok = 2 * t + (q & 1), row = g + 8 * (q >> 1);
-            if (tok < a.M && row_ok(row)) yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(v[q]);
-          }
+      for (int q = 0; q < 4; ++q) {
+        if (q >= nv) break;
+        if (direct) {
+          if (vtok[q] < a.M && row_ok(vrow[q]))
+            yg[static_cast<int64_t>(vtok[q]) * a.N + rb + vrow[q]] = __float2bfloat16_rn(FMT == 2 ? v[q] * gs : v[q]);
         } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dstv[(g + 8 * (q >> 1)) * MP + 2 * t + (q & 1)] = v[q];
+          dstv[vrow[q] * MP + vtok[q]] = v[q];
         }
       }
     };
@@ -877,12 +985,14 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.stage_bytes = static_cast<int>(round_up((fmt >= 1 ? a.s_off : a.b_off) + kRows * a.pitch_s, 128));
   a.tok_stride = static_cast<int>(2 * K + 64);
   a.zero_stride = static_cast<int>(round_up(U * 64, 128) + 64);
-  // work units: fpu folds (a fold: 8/MP groups side by side; nvfp4: twice as
+  // work units: fpu folds (a fold: the groups side by side above; nvfp4: twice as
   // many 16-weight groups) of one stage, at least kUnitCodes codes of a row
   // where the stage allows.  The kernel is issue-bound, and every unit costs a
   // partial-sum reduction, so a unit is a whole stage (measured: units of 512
   // codes were 17% slower on the 33 MB decode launches)
-  const int GS = 8 / MP, SPANS = fmt == 2 ? GS / 2 : GS;
+  // (a fold: the affine format holds 4/MP groups side by side, or one for
+  // MP = 8; the block-scaled formats 8/MP)
+  const int GS = 8 / MP, SPANS = fmt == 0 ? (MP >= 4 ? 1 : 4 / MP) : fmt == 2 ? GS / 2 : GS;
   const int64_t fold = static_cast<int64_t>(SPANS) * G;  // codes of a row per fold
   a.fpu = 1;
   while (fold * a.fpu * 2 <= kUnitCodes && Kc % (fold * a.fpu * 2) == 0) a.fpu *= 2;
