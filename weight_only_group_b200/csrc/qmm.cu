@@ -104,13 +104,14 @@ struct Params {
 // use by many CTAs at once (the fp16 activations stay in L2); W-row tiles
 // fastest keeps an activation tile in use instead, for activations that do not
 // fit in L2.
-AQ_DEVICE void tile_origin(const Params &prm, int tile, int bn, int &m0, int &n0) {
+// A tile is bn tokens x wr rows of W.
+AQ_DEVICE void tile_origin(const Params &prm, int tile, int bn, int wr, int &m0, int &n0) {
   if (prm.n_fastest) {
     m0 = (tile / prm.n_tiles) * bn;
-    n0 = (tile % prm.n_tiles) * 128;
+    n0 = (tile % prm.n_tiles) * wr;
   } else {
     m0 = (tile % prm.m_tiles) * bn;
-    n0 = (tile / prm.m_tiles) * 128;
+    n0 = (tile / prm.m_tiles) * wr;
   }
 }
 
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         int m0, n0;
-        tile_origin(prm, tile, BN, m0, n0);
+        tile_origin(prm, tile, BN, 128, m0, n0);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t r = it / S;
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t, it0 += KB) {
       int m0, n0;
-      tile_origin(prm, tile, BN, m0, n0);
+      tile_origin(prm, tile, BN, 128, m0, n0);
       const int n = n0 + row;
       const bool row_ok = n < prm.N;
       const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
@@ -318,6 +319,313 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
   if (warp == 1) {
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair kernel (tcgen05 cta_group::2).  Two CTAs of a cluster share one
+// 256 x BN tile: CTA r owns W rows n0 + 128 r .. + 127 (its TMEM lanes, its A
+// operand, its half of the accumulator) and tokens m0 + r BN/2 .. of the x16
+// tile (its half of the B operand).  CTA 0 issues one M = 256 MMA per K = 16
+// step for both; the tensor cores exchange the B halves.  Per K block a CTA
+// thus stages BN/2 token rows instead of BN, which halves the shared-memory
+// writes and the B reads per multiply-add and the L2 traffic behind them (the
+// single-CTA kernel ran at about 800 cycles per 64-deep K block against 512
+// of tensor work, with the stage ring unable to cover the load latency).
+//   * both CTAs: TMA producer (warp 0) into their own stage ring, completing
+//     on their own `full` barrier; dequant warps wait on it, write their A
+//     stage into their own TMEM and arrive on CTA 0's `a_full` (eight
+//     arrivals: four quadrant warps per CTA);
+//   * CTA 0 warp 1: waits `a_full`, issues the pair MMAs, and commits with a
+//     multicast arrive on both CTAs' `empty` (stage reuse) and `acc_full`;
+//   * epilogue: each CTA reads its own accumulator rows, then arrives on CTA
+//     0's `acc_empty` (24 arrivals).
+// TMEM is allocated with cta_group::2 by warp 1 of both CTAs and freed after
+// a cluster barrier that follows every MMA and every accumulator read.
+// ---------------------------------------------------------------------------
+template <int BITS, int BN>
+struct PairCfg {
+  static constexpr int BK = (BITS == 3) ? 128 : 64;
+  static constexpr int BKW = BK * BITS / 32;
+  static constexpr int XH = BN / 2;                          // token rows of the x16 tile in this CTA
+  static constexpr int X_BYTES = XH * BK * 2;
+  static constexpr int W_BYTES = 128 * BKW * 4;
+  static constexpr int STAGE_BYTES = ((X_BYTES + W_BYTES + 1023) / 1024) * 1024;
+  static constexpr int SMEM_BUDGET = 225 * 1024;
+  static constexpr int A_COLS = BK / 2;
+  static constexpr int A_COL0 = BN;
+  static constexpr int STAGES = std::min(std::min(12, SMEM_BUDGET / STAGE_BYTES), (kTmemCols - A_COL0) / A_COLS);
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512 /*barriers*/;
+  static_assert(STAGES >= 2, "not enough shared memory for two stages");
+  static_assert((3 * STAGES + 2) * 8 + 8 <= 512, "barrier area");
+  static_assert(XH % 8 == 0 && BN <= 256 && BN % 32 == 0, "pair MMA N");
+};
+
+AQ_DEVICE uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+AQ_DEVICE void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive (release, cluster scope) on the barrier at the same offset in CTA `cta` of the cluster.
+AQ_DEVICE void mbar_arrive_at(uint64_t *bar, uint32_t cta) {
+  uint32_t addr;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(smem_u32(bar)), "r"(cta));
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+AQ_DEVICE bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (for barriers the other CTA arrives on).
+AQ_DEVICE bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t fault_bit) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(&g_fault_word, fault_bit);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+AQ_DEVICE void tc_mma_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs once the MMAs issued so far have completed.
+AQ_DEVICE void tc_commit_pair(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+// kind::f16 instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, M = 256, N = bn.
+__host__ __device__ constexpr uint32_t idesc_pair(int bn) {
+  return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+template <int BITS, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    qmm_pair_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map, Params prm) {
+  using C = PairCfg<BITS, BN>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES);
+  uint64_t *empty = full + S;
+  uint64_t *a_full = empty + S;
+  uint64_t *acc_full = a_full + S;
+  uint64_t *acc_empty = acc_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+  const int total_tiles = prm.m_tiles * prm.n_tiles;
+  const int KB = (prm.K + C::BK - 1) / C::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&a_full[s], 8);  // one warp per TMEM lane quadrant, in each CTA
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * 4 * kDequantPerQuadrant);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers and TMEM exist before either uses the other's
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (each CTA)
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&x_map)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&w_map)) : "memory");
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += npairs) {
+        int m0, n0;
+        tile_origin(prm, tile, BN, 256, m0, n0);
+        const int xrow = m0 + static_cast<int>(rank) * C::XH;
+        const int wrow = n0 + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t r = it / S;
+          if (r >= 1 && !(ok = mbar_wait_cluster(&empty[s], (r - 1) & 1, abort_flag, kFaultProducerWait))) break;
+          uint8_t *xs = smem + s * C::STAGE_BYTES;
+          uint8_t *ws = xs + C::X_BYTES;
+          mbar_arrive_expect_tx(&full[s], C::X_BYTES + C::W_BYTES);
+#pragma unroll
+          for (int a = 0; a < C::BK / 64; ++a)
+            tma_load_2d(xs + a * C::XH * 128, &x_map, &full[s], kb * C::BK + a * 64, xrow);
+          tma_load_2d(ws, &w_map, &full[s], kb * C::BKW, wrow);
+        }
+      }
+      const uint32_t issued = it;
+      for (uint32_t j = (issued > static_cast<uint32_t>(S) ? issued - S : 0); j < issued; ++j)
+        mbar_drain(&full[j % S], (j / S) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (CTA 0)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_pair(BN);
+      uint32_t it = 0, t = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++t) {
+        if (t >= 1 && !(ok = mbar_wait_cluster(acc_empty, (t - 1) & 1, abort_flag, kFaultMmaWait))) break;
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t r = it / S;
+          // a_full: both CTAs' A stages are written, and each dequant warp saw its CTA's stage land
+          if (!(ok = mbar_wait_cluster(&a_full[s], r & 1, abort_flag, kFaultMmaWait))) break;
+          tc_fence_after();
+          const uint32_t xs_addr = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t a_tmem = tmem_base + C::A_COL0 + s * C::A_COLS;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            const uint32_t b_addr = xs_addr + (kk / 4) * C::XH * 128 + (kk % 4) * 32;
+            tc_mma_pair(tmem_base + kAccCol, a_tmem + kk * 8, sw128_kmajor_desc(b_addr), idesc,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[s]);
+        }
+        if (ok) tc_commit_pair(acc_full);
+      }
+      if (it > 0) mbar_drain(&empty[(it - 1) % S], ((it - 1) / S) & 1);
+    }
+  } else if (warp >= kDequantWarp0) {
+    // ------------------------------------------------------------------ dequant + epilogue (each CTA)
+    const int q = warp & 3;
+    const int h = (warp - kDequantWarp0) >> 2;
+    constexpr int H = kDequantPerQuadrant;
+    const int row = q * 32 + lane;
+    constexpr int CH = C::BK / 32;
+    uint32_t it0 = 0, t = 0;
+    bool ok = true;
+    for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++t, it0 += KB) {
+      int m0, n0;
+      tile_origin(prm, tile, BN, 256, m0, n0);
+      const int n = n0 + static_cast<int>(rank) * 128 + row;
+      const bool row_ok = n < prm.N;
+      const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
+      auto load_sb = [&](int kb, uint16_t (&sc)[CH], uint16_t (&bi)[CH]) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int g = (kb * C::BK + c * 32) / prm.G;
+          const bool in = row_ok && kb < KB && g < prm.Gn;
+          sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
+          bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
+        }
+      };
+      uint16_t sc_pf[2][CH], bi_pf[2][CH];
+      load_sb(h, sc_pf[0], bi_pf[0]);
+      load_sb(h + H, sc_pf[1], bi_pf[1]);
+      int slot = 0;
+      for (int kb = h; kb < KB; kb += H, slot ^= 1) {
+        const uint32_t it = it0 + kb;
+        const int s = it % S;
+        const uint32_t r = it / S;
+        uint16_t sc[CH], bi[CH];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          sc[c] = sc_pf[slot][c];
+          bi[c] = bi_pf[slot][c];
+        }
+        load_sb(kb + 2 * H, sc_pf[slot], bi_pf[slot]);
+        if (!(ok = mbar_wait(&full[s], r & 1, abort_flag, kFaultDequantWait))) break;
+        if (r >= 1 && !(ok = mbar_wait_cluster(&empty[s], (r - 1) & 1, abort_flag, kFaultDequantWait))) break;
+        __syncwarp();
+        const uint32_t *wrow =
+            reinterpret_cast<const uint32_t *>(smem + s * C::STAGE_BYTES + C::X_BYTES) + row * C::BKW;
+        const uint32_t a_tmem = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::A_COL0 + s * C::A_COLS;
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          uint32_t w[BITS];
+          if constexpr (BITS == 4) {
+            const uint4 v4 = *reinterpret_cast<const uint4 *>(wrow + c * 4);
+            w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+          } else if constexpr (BITS == 8) {
+            const uint4 a4 = reinterpret_cast<const uint4 *>(wrow + c * 8)[0];
+            const uint4 b4 = reinterpret_cast<const uint4 *>(wrow + c * 8)[1];
+            w[0] = a4.x; w[1] = a4.y; w[2] = a4.z; w[3] = a4.w;
+            w[4] = b4.x; w[5] = b4.y; w[6] = b4.z; w[7] = b4.w;
+          } else {
+#pragma unroll
+            for (int i = 0; i < BITS; ++i) w[i] = wrow[c * BITS + i];
+          }
+          uint32_t packed_cols[16];
+          dequant_chunk_f16<BITS>(w, sc[c], bi[c], packed_cols);
+          tmem_st16(a_tmem + c * 16, packed_cols);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_at(&a_full[s], 0);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------------- epilogue
+      if (!(ok = mbar_wait_cluster(acc_full, t & 1, abort_flag, kFaultEpilogueWait))) break;
+      __syncwarp();
+      tc_fence_after();
+#pragma unroll 1
+      for (int col = h * 32; col < BN; col += H * 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + col, v);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int m = m0 + col + i;
+            if (m < prm.M)
+              prm.y[static_cast<int64_t>(m) * prm.N + n] =
+                  __float2bfloat16_rn(__uint_as_float(v[i]) * __ldg(prm.row_scale + m));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_at(acc_empty, 0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no MMA of the pair and no accumulator read is outstanding in either CTA
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                  : "memory");
   }
 }
@@ -479,28 +787,107 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
   return cudaGetLastError();
 }
 
-// Token tile width.  The kernel is fed from L2: per K block a tile reads its
-// x16 slice (BN x BK fp16) and its packed W slice, so a narrow token tile moves
-// more bytes per multiply-add; a wide one leaves SMs idle in the last wave when
-// there are few tiles.  Score = (fraction of the SMs' waves filled) x (MACs per
-// byte read), and take the best (ties: the wider tile).
-template <int BITS>
-int pick_bn(int64_t M, int64_t N, int sms) {
-#ifdef AQ_QMM_FORCE_BN  // build-time override (64, 128 or 256; 0: choose)
-  if (AQ_QMM_FORCE_BN == 64 || AQ_QMM_FORCE_BN == 128 || AQ_QMM_FORCE_BN == 256) return AQ_QMM_FORCE_BN;
+template <int BITS, int BN>
+cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                        const uint16_t *biases, int64_t N, int G, uint16_t *y, void *workspace, cudaStream_t stream) {
+  using C = PairCfg<BITS, BN>;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  __half *x16 = reinterpret_cast<__half *>(workspace);
+  float *row_scale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + ((M * K * 2 + 255) / 256) * 256);
+  x_to_f16_rows_kernel<BITS><<<static_cast<unsigned>(M), kPrepThreads, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
+  CUtensorMap x_map, w_map;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(C::XH)};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const int64_t P = K * BITS / 32;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(P) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(C::BKW), 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(packed), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  Params prm;
+  prm.scales = reinterpret_cast<const __half *>(scales);
+  prm.biases = reinterpret_cast<const __half *>(biases);
+  prm.row_scale = row_scale;
+  prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  prm.M = static_cast<int>(M);
+  prm.N = static_cast<int>(N);
+  prm.K = static_cast<int>(K);
+  prm.G = G;
+  prm.Gn = static_cast<int>(K / G);
+  prm.m_tiles = static_cast<int>((M + BN - 1) / BN);
+  prm.n_tiles = static_cast<int>((N + 255) / 256);
+  const int64_t w_bytes = N * K * BITS / 8 + 4 * N * (K / G);
+  prm.n_fastest = (2 * M * K > w_bytes) ? 1 : 0;
+#ifdef AQ_QMM_FORCE_ORDER
+  if (AQ_QMM_FORCE_ORDER == 0 || AQ_QMM_FORCE_ORDER == 1) prm.n_fastest = AQ_QMM_FORCE_ORDER;
 #endif
-  auto score = [&](int64_t bn, int64_t bytes) {
-    const int64_t t = ((M + bn - 1) / bn) * ((N + 127) / 128);
-    const int64_t waves = (t + sms - 1) / sms;
-    const double fill = static_cast<double>(t) / static_cast<double>(waves * sms);
-    return fill * static_cast<double>(bn) / static_cast<double>(bytes);
+
+  auto kern = qmm_pair_kernel<BITS, BN>;
+  static thread_local int cached_dev = -1;
+  static thread_local int sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
+      return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
+  const int pairs = static_cast<int>(std::min<int64_t>(tiles, std::max(1, sms / 2)));
+  kern<<<2 * pairs, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, prm);
+  return cudaGetLastError();
+}
+
+// Tile shape.  Both kernels are fed from L2 through a ring of stages, and the
+// measured load latency (about 4000 SM cycles) spread over the ring's depth
+// bounds the time per 64-deep K block from below, next to the tensor work of
+// the block (2 cycles per token column for 128 W rows).  Model the time of a
+// launch as waves x K blocks x max(tensor time, latency / stages) and take the
+// fastest shape: the CTA pair at 256 or 128 tokens, or one CTA at 256, 128 or
+// 64 tokens (pairs fill the SMs in units of two).  Ties go to the earlier one.
+enum Shape { kPair256 = 0, kPair128 = 1, kOne256 = 2, kOne128 = 3, kOne64 = 4 };
+
+template <int BITS>
+int pick_shape(int64_t M, int64_t N, int sms) {
+#ifdef AQ_QMM_FORCE_SHAPE  // build-time override (0..4 as in Shape; else choose)
+  if (AQ_QMM_FORCE_SHAPE >= 0 && AQ_QMM_FORCE_SHAPE <= 4) return AQ_QMM_FORCE_SHAPE;
+#endif
+  constexpr double kLatency = 4000.0;
+  auto cost = [&](int64_t bn, int64_t rows, int64_t slots, int stages) {
+    const int64_t t = ((M + bn - 1) / bn) * ((N + rows - 1) / rows);
+    const int64_t waves = (t + slots - 1) / slots;
+    return static_cast<double>(waves) * std::max(2.0 * static_cast<double>(bn), kLatency / stages);
   };
-  const double s256 = score(256, Cfg<BITS, 256>::X_BYTES + Cfg<BITS, 256>::W_BYTES);
-  const double s128 = score(128, Cfg<BITS, 128>::X_BYTES + Cfg<BITS, 128>::W_BYTES);
-  const double s64 = score(64, Cfg<BITS, 64>::X_BYTES + Cfg<BITS, 64>::W_BYTES);
-  if (M > 128 && s256 >= s128 && s256 >= s64) return 256;
-  if (M > 64 && s128 >= s64) return 128;
-  return 64;
+  const int64_t pairs = std::max(1, sms / 2);
+  double c[5];
+  c[kPair256] = cost(256, 256, pairs, PairCfg<BITS, 256>::STAGES);
+  c[kPair128] = cost(128, 256, pairs, PairCfg<BITS, 128>::STAGES);
+  c[kOne256] = cost(256, 128, sms, Cfg<BITS, 256>::STAGES);
+  c[kOne128] = cost(128, 128, sms, Cfg<BITS, 128>::STAGES);
+  c[kOne64] = cost(64, 128, sms, Cfg<BITS, 64>::STAGES);
+  int best = kPair256;
+  for (int i = 1; i < 5; ++i)
+    if (c[i] < c[best]) best = i;
+  return best;
 }
 
 template <int BITS>
@@ -514,10 +901,12 @@ cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     cached_dev = dev;
   }
-  switch (pick_bn<BITS>(M, N, sms)) {
-    case 64: return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-    case 128: return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-    default: return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+  switch (pick_shape<BITS>(M, N, sms)) {
+    case kPair256: return launch_pair<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case kPair128: return launch_pair<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case kOne256: return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case kOne128: return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    default: return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, ws, s);
   }
 }
 
