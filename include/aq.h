@@ -166,6 +166,41 @@ aq_status aq_matmul_ex(const uint16_t *x_bf16, int64_t M, int64_t K,
                        const uint32_t *packed, const uint16_t *scales, const uint16_t *biases,
                        int64_t N, int G, int bits, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
 
+/* One matmul of aq_matmul_sequence: y [M, N] = x [M, K] . dequant(W)^T with W
+ * given as packed [N, K*bits/32], scales and biases [N, K/G] (the layouts of
+ * aq_matmul).  Device pointers, 16-byte aligned. */
+typedef struct {
+  const uint16_t *x_bf16;
+  const uint32_t *packed;
+  const uint16_t *scales;
+  const uint16_t *biases;
+  uint16_t *y_bf16;
+  int64_t N;
+  int64_t K;
+} aq_matmul_desc;
+
+/* Decode matmuls of one step in a single launch ("MLX Quantization",
+ * "Mechanics": QMV streams each weight once per decode step; several linears
+ * run back to back).  Computes calls[j] for j = 0 .. n-1 (1 <= n <= 4) in
+ * order, all with the same M (1..8), G and bits (2, 4 or 8), each with its own
+ * N and K, with the arithmetic and accuracy of aq_matmul's tensor-core QMV.
+ * Ordering: matmul j reads its x only after every element of matmul j-1's y is
+ * written, so calls[j].x_bf16 may be calls[j-1].y_bf16 (a chain of linears);
+ * the weights of matmul j stream while matmul j-1 finishes.  No other
+ * overlap between one call's y and any call's inputs is allowed.
+ * The launch places one CTA on each SM and synchronises them between the
+ * matmuls; it needs every one of its CTAs resident at once, so it must not
+ * share the GPU with kernels that hold SMs for long (a barrier wait that runs
+ * out sets a bit of aq_device_fault and the results are undefined).
+ * flags: 0 or AQ_MATMUL_OVERLAP_PREVIOUS (the first matmul's weights may be
+ * read before the previous kernel in the stream completes).
+ * Errors: n outside 1..4, a null pointer, unknown flags -> AQ_ERR_INVALID_ARG;
+ * M > 8, bits not 2/4/8, G not 32/64/128, or a shape the decode kernel does not
+ * take (K a multiple of 8*G, N >= 16) -> AQ_ERR_UNSUPPORTED; unaligned
+ * pointers -> AQ_ERR_ALIGNMENT.  Asynchronous on `stream`; allocates nothing. */
+aq_status aq_matmul_sequence(const aq_matmul_desc *calls, int n, int64_t M, int G, int bits, uint32_t flags,
+                             aq_stream_t stream);
+
 /* Bytes of workspace aq_matmul_ws needs for this shape (0 when the dispatched
  * kernel needs none, or when the arguments would be rejected).  Host only. */
 size_t aq_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K, int G, int bits);

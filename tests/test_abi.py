@@ -146,6 +146,32 @@ def test_matmul_ex_flags():
     assert L.aq_matmul_ex(A, 0, 64, A, A, A, 8, 64, 4, A, aq.AQ_MATMUL_OVERLAP_PREVIOUS, None) == aq.AQ_ERR_INVALID_ARG
 
 
+def test_matmul_sequence_validation():
+    """Argument checks of aq_matmul_sequence, all before any device work."""
+    L = aq.lib()
+    D = aq._MatmulDesc
+
+    def call(n=2, M=1, G=64, bits=4, flags=0, **kw):
+        f = dict(x_bf16=A, packed=A, scales=A, biases=A, y_bf16=A, N=1024, K=2048)
+        f.update(kw)
+        arr = (D * 4)(*[D(**f) for _ in range(4)])
+        return L.aq_matmul_sequence(arr, n, M, G, bits, flags, None)
+
+    assert L.aq_matmul_sequence(None, 1, 1, 64, 4, 0, None) == aq.AQ_ERR_INVALID_ARG
+    assert call(n=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(n=5) == aq.AQ_ERR_INVALID_ARG
+    assert call(M=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(flags=2) == aq.AQ_ERR_INVALID_ARG
+    assert call(x_bf16=0) == aq.AQ_ERR_INVALID_ARG
+    assert call(M=9) == aq.AQ_ERR_UNSUPPORTED
+    assert call(bits=3) == aq.AQ_ERR_UNSUPPORTED
+    assert call(G=16) == aq.AQ_ERR_UNSUPPORTED
+    assert call(y_bf16=U) == aq.AQ_ERR_ALIGNMENT
+    assert call(K=96) == aq.AQ_ERR_INVALID_ARG      # K not a multiple of G
+    assert call(K=64 * 4) == aq.AQ_ERR_UNSUPPORTED  # K not a multiple of 8 G
+    assert call(N=8) == aq.AQ_ERR_UNSUPPORTED       # fewer than 16 rows
+
+
 def test_embedding_validation():
     L = aq.lib()
     call = lambda ids=A, T=4, V=100, D=64, G=64, bits=4, out=A: L.aq_embedding(ids, T, A, A, A, V, D, G, bits, out, None)

@@ -911,3 +911,87 @@ def test_rejects_misaligned_device_pointer():
                                 torch.empty(1, 8, dtype=torch.bfloat16, device="cuda").data_ptr(), None)
         aq._check(rc, "aq_matmul")
     assert e.value.status == aq.AQ_ERR_ALIGNMENT
+
+
+# ----------------------------------------------------------------------------- sequence launches
+
+SEQ_SHAPES = [(2048, 1024), (1024, 2048), (2048, 512)]  # (K, N) of three independent matmuls
+
+
+@pytest.mark.parametrize("M,G,bits", [(1, 64, 4), (2, 64, 4), (3, 128, 4), (5, 32, 8), (8, 64, 2)])
+def test_matmul_sequence_equals_single_calls(M, G, bits):
+    """Three matmuls in one launch give, bit for bit, what three aq_matmul
+    calls give (each row's arithmetic is the same), and each is within the
+    matmul tolerance of the oracle."""
+    calls, refs = [], []
+    for j, (K, N) in enumerate(SEQ_SHAPES):
+        p, s, b = quantized(N, K, 9500 + j, True, G, bits)
+        xb = activations_bits(M, K, 9510 + j)
+        pg, sg, bg = _to_gpu(p, s, b)
+        calls.append((_x_gpu(xb), pg, sg, bg, None))
+        refs.append((xb, p, s, b))
+    outs = aq.aq_matmul_sequence(calls, G, bits)
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() == 0
+    for j, ((x, pg, sg, bg, _), (xb, p, s, b), y) in enumerate(zip(calls, refs, outs)):
+        y1 = aq.aq_matmul(x, pg, sg, bg, G, bits)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), f"matmul {j} differs from its single call"
+        _assert_close(y, oracle.matmul(xb, p, s, b, G, bits), f"sequence matmul {j}")
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_matmul_sequence_chain_reads_the_previous_output(M):
+    """y0 = x0 W0^T, y1 = y0 W1^T, y2 = y1 W2^T in one launch: each matmul
+    reads the output the matmul before it wrote in the same launch (checked
+    against the oracle applied to the GPU's own y0 and y1, repeated so that a
+    read before the write would show)."""
+    G, bits = 64, 4
+    dims = [2048, 1024, 1536, 512]  # K0, N0 = K1, N1 = K2, N2
+    ws = []
+    for j in range(3):
+        K, N = dims[j], dims[j + 1]
+        p, s, b = quantized(N, K, 9600 + j, True, G, bits)
+        ws.append(((p, s, b), _to_gpu(p, s, b)))
+    xb = activations_bits(M, dims[0], 9610)
+    x0 = _x_gpu(xb)
+    for rep in range(3):
+        y0 = torch.full((M, dims[1]), float("nan"), dtype=torch.bfloat16, device="cuda")
+        y1 = torch.full((M, dims[2]), float("nan"), dtype=torch.bfloat16, device="cuda")
+        y2 = torch.empty((M, dims[3]), dtype=torch.bfloat16, device="cuda")
+        aq.aq_matmul_sequence([(x0, *ws[0][1], y0), (y0, *ws[1][1], y1), (y1, *ws[2][1], y2)], G, bits)
+        torch.cuda.synchronize()
+        assert aq.aq_device_fault() == 0
+        inp = [xb, _u16(y0), _u16(y1)]
+        for j, y in enumerate((y0, y1, y2)):
+            p, s, b = ws[j][0]
+            assert torch.isfinite(y.float()).all(), f"rep {rep}: matmul {j} read an unwritten input"
+            _assert_close(y, oracle.matmul(inp[j], p, s, b, G, bits), f"rep {rep} chain matmul {j}")
+
+
+def test_matmul_sequence_wait_runs_out_cleanly():
+    """A sequence launch whose waits run out (a barrier nothing completes)
+    sets the decode fault bit and returns; after the fault is read the next
+    sequence launch is correct."""
+    G, bits, M = 64, 4, 1
+    calls, refs = [], []
+    for j, (K, N) in enumerate(SEQ_SHAPES):
+        p, s, b = quantized(N, K, 9700 + j, False, G, bits)
+        xb = activations_bits(M, K, 9710 + j)
+        calls.append((_x_gpu(xb), *_to_gpu(p, s, b), None))
+        refs.append((xb, p, s, b))
+    assert aq.aq_device_fault() == 0
+    aq.aq_set_wait_limit(20000)
+    aq.aq_set_wait_stall(True)
+    try:
+        aq.aq_matmul_sequence(calls, G, bits)
+        torch.cuda.synchronize()
+    finally:
+        aq.aq_set_wait_stall(False)
+        aq.aq_set_wait_limit(0)
+    assert aq.aq_device_fault() & 0x10
+    outs = aq.aq_matmul_sequence(calls, G, bits)
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() == 0
+    for j, (y, (xb, p, s, b)) in enumerate(zip(outs, refs)):
+        _assert_close(y, oracle.matmul(xb, p, s, b, G, bits), f"after the timeout, matmul {j}")

@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
             L.aq_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
             L.aq_matmul_with.argtypes = [i32, vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, vp]
             L.aq_matmul_ex.argtypes = [vp, i64, i64, vp, vp, vp, i64, i32, i32, vp, ctypes.c_uint32, vp]
+            L.aq_matmul_sequence.argtypes = [ctypes.POINTER(_MatmulDesc), i32, i64, i32, i32, ctypes.c_uint32, vp]
             L.aq_embedding.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp]
             L.aq_gather_matmul.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, vp]
             L.aq_gather_matmul_grouped.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, i32, i32, vp, vp, vp]
@@ -331,6 +332,48 @@ def aq_matmul_ex(x, packed, scales, biases, G: int, bits: int, flags: int, out: 
                                 bits, out.data_ptr(), int(flags), _stream(x))
     _check(rc, "aq_matmul_ex")
     return out
+
+
+class _MatmulDesc(ctypes.Structure):
+    """aq_matmul_desc of include/aq.h."""
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("biases", ctypes.c_void_p), ("y_bf16", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+def aq_matmul_sequence(calls, G: int, bits: int, overlap_previous: bool = False):
+    """Several decode matmuls in one launch (aq_matmul_sequence of include/aq.h).
+
+    ``calls`` is a list of (x, packed, scales, biases, out) with x [M, K_j]
+    bf16 and out [M, N_j] bf16 (out may be None: allocated here).  Matmul j
+    reads its x only after matmul j-1's output is complete, so a call's x may
+    be the previous call's out.  Returns the list of outputs."""
+    if not 1 <= len(calls) <= 4:
+        raise ValueError("aq_matmul_sequence takes 1 to 4 matmuls")
+    descs = (_MatmulDesc * len(calls))()
+    outs = []
+    M = None
+    dev = None
+    for j, (x, packed, scales, biases, out) in enumerate(calls):
+        _need(x, "x", (torch.bfloat16,))
+        N = _qw(packed, scales, biases)
+        Mj, K = x.shape
+        if M is None:
+            M, dev = Mj, x.device
+        elif Mj != M or x.device != dev:
+            raise ValueError("every matmul of a sequence has the same M and device")
+        if out is None:
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+        _need(out, "out", (torch.bfloat16,))
+        if tuple(out.shape) != (M, N):
+            raise ValueError(f"out of matmul {j} must be [{M}, {N}]")
+        descs[j] = _MatmulDesc(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), out.data_ptr(),
+                               N, K)
+        outs.append(out)
+    flags = AQ_MATMUL_OVERLAP_PREVIOUS if overlap_previous else 0
+    with _on(dev):
+        rc = lib().aq_matmul_sequence(descs, len(calls), M, G, bits, flags, _stream(calls[0][0]))
+    _check(rc, "aq_matmul_sequence")
+    return outs
 
 
 def aq_matmul_ws(x, packed, scales, biases, G: int, bits: int, workspace: torch.Tensor | None,

@@ -23,6 +23,8 @@ void set_qmv_tc_wait_limit(long long cycles);
 void set_qmv_tc_wait_stall(bool on);
 cudaError_t read_and_clear_embed_fault(uint32_t *word);
 bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
+bool qmv_tc_seq_supported(int n, const int64_t *N, const int64_t *K, int64_t M, int G, int bits);
+cudaError_t launch_qmv_tc_seq(int n, const SeqCall *calls, int64_t M, int G, int bits, uint32_t flags, cudaStream_t s);
 cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed, const uint16_t *scales,
                              const uint16_t *biases, int64_t E, int64_t N, int G, int bits, const int32_t *experts,
                              uint16_t *y, cudaStream_t s);
@@ -325,6 +327,31 @@ aq_status aq_matmul_ex(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
   const size_t need = workspace_for(kernel, M, K);
   if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream, flags);
   return aq_matmul_with(kernel, x, M, K, packed, scales, biases, N, G, bits, y, stream);
+}
+
+aq_status aq_matmul_sequence(const aq_matmul_desc *calls, int n, int64_t M, int G, int bits, uint32_t flags,
+                             aq_stream_t stream) {
+  if (!calls || n < 1 || n > 4 || M < 1) return AQ_ERR_INVALID_ARG;
+  if (flags & ~static_cast<uint32_t>(AQ_MATMUL_OVERLAP_PREVIOUS)) return AQ_ERR_INVALID_ARG;
+  if (M > 8 || !(bits == 2 || bits == 4 || bits == 8)) return AQ_ERR_UNSUPPORTED;
+  aq::SeqCall sc[4];
+  int64_t N[4], K[4];
+  for (int j = 0; j < n; ++j) {
+    const aq_matmul_desc &c = calls[j];
+    aq_status st = check_shape(c.N, c.K, G, bits);
+    if (st != AQ_OK) return st;
+    if (!c.x_bf16 || !c.packed || !c.scales || !c.biases || !c.y_bf16) return AQ_ERR_INVALID_ARG;
+    if (!aligned16(c.x_bf16) || !aligned16(c.packed) || !aligned16(c.scales) || !aligned16(c.biases) ||
+        !aligned16(c.y_bf16))
+      return AQ_ERR_ALIGNMENT;
+    sc[j] = aq::SeqCall{c.x_bf16, c.packed, c.scales, c.biases, c.y_bf16, c.N, c.K};
+    N[j] = c.N;
+    K[j] = c.K;
+  }
+  if (!aq::qmv_tc_seq_supported(n, N, K, M, G, bits)) return AQ_ERR_UNSUPPORTED;
+  aq_status st = check_device();
+  if (st != AQ_OK) return st;
+  return from_cuda(aq::launch_qmv_tc_seq(n, sc, M, G, bits, flags, stream));
 }
 
 aq_status aq_embedding(const int32_t *ids, int64_t T, const uint32_t *packed, const uint16_t *scales,

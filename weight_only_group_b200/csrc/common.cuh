@@ -14,6 +14,16 @@
 
 namespace aq {
 
+// One matmul of a sequence launch (device pointers; bf16 x [M, K], y [M, N]).
+struct SeqCall {
+  const uint16_t *x;
+  const uint32_t *packed;
+  const uint16_t *scales, *biases;
+  uint16_t *y;
+  int64_t N, K;
+};
+
+
 // Bits of the device-side fault word (defined next to the only kernel with
 // waits): set, never trapped, when a bounded wait gives up.
 enum : uint32_t {

@@ -370,36 +370,21 @@ AQ_DEVICE uint32_t cluster_rank() {
 AQ_DEVICE void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive (release, cluster scope) on the barrier at the same offset in CTA `cta` of the cluster.
+// Arrive on the barrier at the same offset in CTA `cta` of the cluster.  The
+// default (CTA-scope) release: a cluster-scope release would first wait for
+// this thread's outstanding global loads (the scale prefetches), which put a
+// full memory round trip into every K block.  What the arrive publishes is
+// ordered by other means: tcgen05.st by wait::st and fence::before_thread_sync,
+// the stage's TMA data by the barrier this thread waited on before.
 AQ_DEVICE void mbar_arrive_at(uint64_t *bar, uint32_t cta) {
   uint32_t addr;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(smem_u32(bar)), "r"(cta));
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
-AQ_DEVICE bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait with cluster-scope acquire (for barriers the other CTA arrives on).
+// Bounded wait on a barrier that the other CTA of the pair (or its tensor
+// core commits) may complete.
 AQ_DEVICE bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t fault_bit) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      atomicOr(&g_fault_word, fault_bit);
-      *abort_flag = 1;
-      return false;
-    }
-  }
+  return mbar_wait(bar, parity, abort_flag, fault_bit);
 }
 AQ_DEVICE void tc_mma_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -857,37 +842,37 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   return cudaGetLastError();
 }
 
-// Tile shape.  Both kernels are fed from L2 through a ring of stages, and the
-// measured load latency (about 4000 SM cycles) spread over the ring's depth
-// bounds the time per 64-deep K block from below, next to the tensor work of
-// the block (2 cycles per token column for 128 W rows).  Model the time of a
-// launch as waves x K blocks x max(tensor time, latency / stages) and take the
-// fastest shape: the CTA pair at 256 or 128 tokens, or one CTA at 256, 128 or
-// 64 tokens (pairs fill the SMs in units of two).  Ties go to the earlier one.
-enum Shape { kPair256 = 0, kPair128 = 1, kOne256 = 2, kOne128 = 3, kOne64 = 4 };
+// Tile shape.  Measured on B200 (4-bit, G = 64): both kernels take about
+// 750-800 SM cycles per 64-deep K block at every token-tile width, more than
+// the tensor work of the block (2 cycles per token column), so what decides
+// is how many multiply-adds a block carries and how well the tiles fill the
+// SMs.  The CTA pair (256 x 256 tiles) carries the most per block and frees
+// half of each CTA's L2 traffic; it was as fast as the single CTA or faster
+// (up to 1.3x at K = 14336) wherever its tiles filled at least one wave of
+// pairs.  With fewer tiles than pairs, one CTA per tile: the width that best
+// trades wave fill against bytes moved per multiply-add (the x16 slice, BN x
+// BK fp16, plus the packed W slice).
+enum Shape { kPair256 = 0, kOne256 = 1, kOne128 = 2, kOne64 = 3 };
 
 template <int BITS>
 int pick_shape(int64_t M, int64_t N, int sms) {
-#ifdef AQ_QMM_FORCE_SHAPE  // build-time override (0..4 as in Shape; else choose)
-  if (AQ_QMM_FORCE_SHAPE >= 0 && AQ_QMM_FORCE_SHAPE <= 4) return AQ_QMM_FORCE_SHAPE;
+#ifdef AQ_QMM_FORCE_SHAPE  // build-time override (0..3 as in Shape; else choose)
+  if (AQ_QMM_FORCE_SHAPE >= 0 && AQ_QMM_FORCE_SHAPE <= 3) return AQ_QMM_FORCE_SHAPE;
 #endif
-  constexpr double kLatency = 4000.0;
-  auto cost = [&](int64_t bn, int64_t rows, int64_t slots, int stages) {
-    const int64_t t = ((M + bn - 1) / bn) * ((N + rows - 1) / rows);
-    const int64_t waves = (t + slots - 1) / slots;
-    return static_cast<double>(waves) * std::max(2.0 * static_cast<double>(bn), kLatency / stages);
+  const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  if (M > 128 && pair_tiles >= std::max(1, sms / 2)) return kPair256;
+  auto score = [&](int64_t bn, int64_t bytes) {
+    const int64_t t = ((M + bn - 1) / bn) * ((N + 127) / 128);
+    const int64_t waves = (t + sms - 1) / sms;
+    const double fill = static_cast<double>(t) / static_cast<double>(waves * sms);
+    return fill * static_cast<double>(bn) / static_cast<double>(bytes);
   };
-  const int64_t pairs = std::max(1, sms / 2);
-  double c[5];
-  c[kPair256] = cost(256, 256, pairs, PairCfg<BITS, 256>::STAGES);
-  c[kPair128] = cost(128, 256, pairs, PairCfg<BITS, 128>::STAGES);
-  c[kOne256] = cost(256, 128, sms, Cfg<BITS, 256>::STAGES);
-  c[kOne128] = cost(128, 128, sms, Cfg<BITS, 128>::STAGES);
-  c[kOne64] = cost(64, 128, sms, Cfg<BITS, 64>::STAGES);
-  int best = kPair256;
-  for (int i = 1; i < 5; ++i)
-    if (c[i] < c[best]) best = i;
-  return best;
+  const double s256 = score(256, Cfg<BITS, 256>::X_BYTES + Cfg<BITS, 256>::W_BYTES);
+  const double s128 = score(128, Cfg<BITS, 128>::X_BYTES + Cfg<BITS, 128>::W_BYTES);
+  const double s64 = score(64, Cfg<BITS, 64>::X_BYTES + Cfg<BITS, 64>::W_BYTES);
+  if (M > 128 && s256 >= s128 && s256 >= s64) return kOne256;
+  if (M > 64 && s128 >= s64) return kOne128;
+  return kOne64;
 }
 
 template <int BITS>
@@ -903,7 +888,6 @@ cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   }
   switch (pick_shape<BITS>(M, N, sms)) {
     case kPair256: return launch_pair<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-    case kPair128: return launch_pair<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
     case kOne256: return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
     case kOne128: return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
     default: return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, ws, s);

@@ -249,26 +249,43 @@ AQ_DEVICE bool spin_until_at_least(int *ctr, int target, volatile int *abort_fla
   return true;
 }
 
-struct Args {
+// One matmul of a launch.  A sequence launch runs several, in order: the
+// activations of matmul j are read only after every output of matmul j - 1 is
+// complete (so y of one may be x of the next), while the weights of matmul j
+// stream into the ring as soon as it has room.
+struct Job {
   const __nv_bfloat16 *x;
-  const uint32_t *packed;
-  const __half *scales, *biases;
   __nv_bfloat16 *y;
-  int M, N, K, Gn;
-  int W, NS;                 // consumer warps, ring stages
+  int N, K, Gn;
   int Kc, nch;               // K chunk of a stage, chunks per row
-  int nper;                  // work units per stage
   int fpu;                   // folds per work unit
   int parts;                 // units per 16-row tile (nch * nper): partial sums reduced per tile
+  int pitch_w, pitch_s;      // bytes per row of codes / of scales (biases) in a stage
+  int s_off, b_off;          // scales and biases inside a stage
+  int tok_stride;            // staged activations: token m at xs_off + m * tok_stride
+  int w_box_x, sb_box_x;     // TMA x coordinate step of one chunk (64-bit elements)
+};
+constexpr int kSeqMax = 4;   // matmuls of one sequence launch at most
+
+template <int NJ>
+struct JobMaps {
+  CUtensorMap w[NJ], s[NJ], b[NJ];  // codes, scales, biases of each matmul
+};
+
+struct Args {
+  Job job[kSeqMax];
+  int njobs;
+  unsigned *gbar;            // sequence launches: grid barrier (count, generation) between matmuls
+  int M;
+  int W, NS;                 // consumer warps, ring stages
+  int nper;                  // work units per stage
   int red_bufs;              // tiles whose partials can be in flight at once
   long long wait_cycles;     // limit of every bounded wait, in SM clock cycles
   int stall;                 // nonzero: the consumers also wait on a barrier nothing completes (timeout test)
-  int pitch_w, pitch_s;      // bytes per row of codes / of scales (biases) in a stage
-  int s_off, b_off, stage_bytes;
-  int xs_off, tok_stride;    // staged activations: token m at xs_off + m * tok_stride
+  int stage_bytes;
+  int xs_off;
   int zero_off, zero_stride; // two zero blocks
   int tab_off, red_off, bar_off;
-  int w_box_x, sb_box_x;     // TMA x coordinate step of one chunk (64-bit elements)
   int early_w;               // weight stages issued before the previous kernel has completed
   // gather mode (cta_per_tok > 0): token t = blockIdx.x / cta_per_tok multiplies
   // its x row by expert experts[t] of E stacked [N, K] weights (rows e*N.. of
@@ -278,10 +295,37 @@ struct Args {
   const float *gscale;  // nvfp4: the tensor scale (device), applied to every output
 };
 
-template <int BITS, int G, int MP, int FMT>
-__global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(const __grid_constant__ Args a, const __grid_constant__ CUtensorMap wmap,
-                                                                  const __grid_constant__ CUtensorMap smap,
-                                                                  const __grid_constant__ CUtensorMap bmap) {
+// Grid-wide barrier of a sequence launch (every CTA of the grid is resident:
+// one CTA per SM, at most one per SM fits).  gbar[0] counts arrivals, gbar[1]
+// is the generation; the last arrival resets the count and advances the
+// generation, so the pair is ready for the next barrier and the next launch.
+// Bounded: false after `limit` cycles (fault bit set, abort raised).
+AQ_DEVICE bool grid_barrier(unsigned *gbar, unsigned nblocks, volatile int *abort_flag, long long limit) {
+  volatile unsigned *gen = gbar + 1;
+  const unsigned g0 = *gen;
+  __threadfence();
+  if (atomicAdd(gbar, 1u) == nblocks - 1) {
+    atomicExch(gbar, 0u);
+    __threadfence();
+    atomicAdd(gbar + 1, 1u);
+    return true;
+  }
+  const long long t0 = clock64();
+  while (*gen == g0) {
+    if (*abort_flag || clock64() - t0 > limit) {
+      atomicOr(&g_qmv_tc_fault, kFaultQmvWait);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(128);
+  }
+  __threadfence();
+  return true;
+}
+
+template <int BITS, int G, int MP, int FMT, int NJ = 1>
+__global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(const __grid_constant__ Args a,
+                                                                  const __grid_constant__ JobMaps<NJ> mp) {
   constexpr int GS = 8 / MP;                     // groups side by side in one accumulator
   constexpr int U = G / 32;                      // K tiles (16 bytes of activation digits per lane) per group
   constexpr int NWD = LaneWords<BITS, G>::count;
@@ -301,10 +345,18 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   constexpr int TPM = MP >= 4 ? 4 : MP;   // tokens per MMA
   constexpr int NMMA = MP > 4 ? 2 : 1;    // MMAs per K tile (token halves)
   constexpr int GS1 = 4 / TPM;            // group slots per fold
-  constexpr int NACC1 = GS1 == 1 ? 1 : kAcc;
+  constexpr int NACC1 = GS1 == 1 ? 1 : GS1 == 4 ? 4 : kAcc;  // one token: four chains of two MMAs per fold
   using Span = LaneSpan<BITS, G, FMT>;
 
   extern __shared__ __align__(128) uint8_t smem[];
+  // The tensor maps live in the launch's parameters, which a decode launch
+  // finds cold in every cache: start fetching them before anything else (the
+  // first copy would otherwise wait for the parameter read, then for the map).
+  if (threadIdx.x == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.w[0])) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.s[0])) : "memory");
+    if constexpr (FMT == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.b[0])) : "memory");
+  }
   uint8_t *ring = smem;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.bar_off);
   uint64_t *empty = full + a.NS;
@@ -317,52 +369,67 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   int *red_done = red_ready + a.red_bufs;
   volatile int *abort_flag = red_done + a.red_bufs;
   int *issued_ctr = red_done + a.red_bufs + 1;  // stages the producer issued (read after an abort)
+  int *x_issued = issued_ctr + 1;                // activation copies issued (one per matmul)
   uint8_t *xs = smem + a.xs_off;
   uint8_t *zero = smem + a.zero_off;
   float4 *tab = reinterpret_cast<float4 *>(smem + a.tab_off);  // [MP][Gn]: (sum x, 2^-e_lo, 2^-e_hi, 0)
   float *red = reinterpret_cast<float *>(smem + a.red_off);    // [red_bufs][parts][16][MP]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int64_t r0, r1, wrow0 = 0;  // rows [r0, r1) of this CTA; first row of its weight matrix in the maps
-  const __nv_bfloat16 *xg = a.x;
-  __nv_bfloat16 *yg = a.y;
+  const Job &J0 = a.job[0];
+  int64_t gr0 = 0, gr1 = 0, wrow0 = 0;  // gather mode: rows [gr0, gr1) of this CTA; first row of its expert
+  const __nv_bfloat16 *xg = J0.x;       // gather mode: this CTA's token row
+  __nv_bfloat16 *yg0 = J0.y;
   if (a.cta_per_tok > 0) {
     const int tk = blockIdx.x / a.cta_per_tok, sub = blockIdx.x - tk * a.cta_per_tok;
-    r0 = static_cast<int64_t>(sub) * a.N / a.cta_per_tok;
-    r1 = static_cast<int64_t>(sub + 1) * a.N / a.cta_per_tok;
-    xg = a.x + static_cast<int64_t>(tk) * a.K;
-    yg = a.y + static_cast<int64_t>(tk) * a.N;
+    gr0 = static_cast<int64_t>(sub) * J0.N / a.cta_per_tok;
+    gr1 = static_cast<int64_t>(sub + 1) * J0.N / a.cta_per_tok;
+    xg = J0.x + static_cast<int64_t>(tk) * J0.K;
+    yg0 = J0.y + static_cast<int64_t>(tk) * J0.N;
     const int e = __ldg(a.experts + tk);
     if (e < 0 || e >= a.E) {  // bad expert id: zero rows and a fault bit, before anything is issued
-      for (int64_t r = r0 + threadIdx.x; r < r1; r += blockDim.x) yg[r] = __float2bfloat16_rn(0.0f);
+      for (int64_t r = gr0 + threadIdx.x; r < gr1; r += blockDim.x) yg0[r] = __float2bfloat16_rn(0.0f);
       if (threadIdx.x == 0 && sub == 0) atomicOr(&g_qmv_tc_fault, kFaultBadIndex);
       return;
     }
-    wrow0 = static_cast<int64_t>(e) * a.N;
-  } else {
-    r0 = static_cast<int64_t>(blockIdx.x) * a.N / gridDim.x;
-    r1 = static_cast<int64_t>(blockIdx.x + 1) * a.N / gridDim.x;
+    wrow0 = static_cast<int64_t>(e) * J0.N;
   }
-  const int tiles = static_cast<int>((r1 - r0 + kRows - 1) / kRows);
-  const int nst = tiles * a.nch;
+  // rows [r0, r1) of this CTA in matmul jx, and its stages (tiles x chunks)
+  auto cta_rows = [&](int jx, int64_t &r0, int64_t &r1) {
+    if (a.cta_per_tok > 0) {
+      r0 = gr0;
+      r1 = gr1;
+    } else {
+      r0 = static_cast<int64_t>(blockIdx.x) * a.job[jx].N / gridDim.x;
+      r1 = static_cast<int64_t>(blockIdx.x + 1) * a.job[jx].N / gridDim.x;
+    }
+  };
+  auto job_stages = [&](int jx) {
+    int64_t r0, r1;
+    cta_rows(jx, r0, r1);
+    return static_cast<int>((r1 - r0 + kRows - 1) / kRows) * a.job[jx].nch;
+  };
   const long long wlim = a.wait_cycles;
-  const int gpc = a.Kc / G;  // groups per chunk
 
   // One stage: rows of codes, scales and biases of (tile, chunk); whole producer warp.
   // First W row of tile T.  A CTA owns >= 16 rows, so its last tile is moved
   // up to end at r1: its first rows repeat rows of the tile before (read again
   // from L2, not stored twice) and every stage is three whole TMA boxes.
-  auto tile_base = [&](int T) { return min(r0 + static_cast<int64_t>(T) * kRows, r1 - kRows); };
-  // One stage: 16 rows of codes, scales and biases of (tile, chunk); one lane.
-  auto issue = [&](int st) {
-    const int s = st % a.NS;
-    const int T = st / a.nch, ch = st - T * a.nch;
-    const int rb = static_cast<int>(wrow0 + tile_base(T));
+  auto tile_base = [&](int64_t r0, int64_t r1, int T) { return min(r0 + static_cast<int64_t>(T) * kRows, r1 - kRows); };
+  // One stage: 16 rows of codes, scales and biases of (tile, chunk) of matmul
+  // jx, into ring slot gst % NS (gst counts the stages of all matmuls); one lane.
+  auto issue = [&](int jx, int st, int gst) {
+    const Job &Jb = a.job[jx];
+    int64_t r0, r1;
+    cta_rows(jx, r0, r1);
+    const int s = gst % a.NS;
+    const int T = st / Jb.nch, ch = st - T * Jb.nch;
+    const int rb = static_cast<int>(wrow0 + tile_base(r0, r1, T));
     uint8_t *dst = ring + static_cast<size_t>(s) * a.stage_bytes;
-    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRows * (a.pitch_w + (FMT == 0 ? 2 : 1) * a.pitch_s)));
-    tma_load_2d(dst, &wmap, &full[s], ch * a.w_box_x, rb);
-    tma_load_2d(dst + a.s_off, &smap, &full[s], ch * a.sb_box_x, rb);
-    if constexpr (FMT == 0) tma_load_2d(dst + a.b_off, &bmap, &full[s], ch * a.sb_box_x, rb);
+    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRows * (Jb.pitch_w + (FMT == 0 ? 2 : 1) * Jb.pitch_s)));
+    tma_load_2d(dst, &mp.w[jx], &full[s], ch * Jb.w_box_x, rb);
+    tma_load_2d(dst + Jb.s_off, &mp.s[jx], &full[s], ch * Jb.sb_box_x, rb);
+    if constexpr (FMT == 0) tma_load_2d(dst + Jb.b_off, &mp.b[jx], &full[s], ch * Jb.sb_box_x, rb);
   };
 
   if (tid == 0) {
@@ -375,6 +442,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     mbar_init(stall_bar, 1);
     *abort_flag = 0;
     *issued_ctr = 0;
+    *x_issued = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -382,44 +450,53 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   // prologue now; it waits for this grid before reading anything it writes.
   if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     // Weights first when the caller allows it (they are not written by the
     // kernel this one may overlap), then, once the kernel before has completed,
-    // the activations (one row per token, raw bf16 into the staging area).
-    const int early = min(min(nst, a.NS), a.early_w);  // never more than the ring holds
+    // the activations of the first matmul (one row per token, raw bf16 into
+    // the staging area), then every stage of every matmul in order, each as
+    // soon as its ring slot is free.  (The producer stages nothing: its lane 0
+    // may stall issuing copies, and the consumers must not wait for that before
+    // converting the activations.)
+    const int nst0 = job_stages(0);
+    const int early = min(min(nst0, a.NS), a.early_w);  // never more than the ring holds
     if (lane == 0)
-      for (int st = 0; st < early; ++st) issue(st);
+      for (int st = 0; st < early; ++st) issue(0, st, st);
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (lane == 0) mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * a.K * 2);
+    if (lane == 0) mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * J0.K * 2);
     __syncwarp();
     if (lane < a.M)
-      bulk_g2s(xs + lane * a.tok_stride, xg + static_cast<int64_t>(lane) * a.K, static_cast<uint32_t>(a.K) * 2, xbar);
-    if (lane == 0)
-      for (int st = early; st < min(nst, a.NS); ++st) issue(st);
-  }
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // (it stages nothing: its lane 0 may stall issuing copies, and the
-    // consumers must not wait for that before converting the activations)
-    int st = min(nst, a.NS);
-    for (; st < nst; ++st) {
-      const int s = st % a.NS;
-      int got = 1;
-      if (lane == 0)
-        got = mbar_wait(&empty[s], ((st / a.NS) - 1) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
-      if (!__shfl_sync(0xffffffffu, got, 0)) break;
-      if (lane == 0) issue(st);
+      bulk_g2s(xs + lane * J0.tok_stride, xg + static_cast<int64_t>(lane) * J0.K, static_cast<uint32_t>(J0.K) * 2,
+               xbar);
+    if (lane == 0) {
+      *x_issued = 1;
+      int gst = early;
+      bool ok = true;
+      for (int jx = 0; jx < a.njobs && ok; ++jx) {
+        const int nstj = jx == 0 ? nst0 : job_stages(jx);
+        for (int st = jx == 0 ? early : 0; st < nstj; ++st, ++gst) {
+          const int s = gst % a.NS;
+          if (gst >= a.NS &&
+              !mbar_wait(&empty[s], ((gst / a.NS) - 1) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim)) {
+            ok = false;
+            break;
+          }
+          issue(jx, st, gst);
+        }
+      }
+      *issued_ctr = gst;
     }
-    if (lane == 0) *issued_ctr = st;
+    __syncwarp();
   } else {
 
   // ---- consumers stage the activations in place: item = (token, group, lane t).
   // A group's raw bf16 and its staged digits occupy the same 2G bytes; the four
   // lanes of a group read all their raw values before any of them writes.
   const int ctid = tid - 32, cthreads = a.W * 32;
-  {
-    mbar_wait(xbar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
-    const int items = a.M * a.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
+  auto stage_acts = [&](int jx) {
+    const Job &Jb = a.job[jx];
+    mbar_wait(xbar, jx & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
+    const int items = a.M * Jb.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
     // Each thread takes kStageItems items per round, processed side by side:
     // the rounds are latency-bound chains (load, reduce across the quad, store).
     constexpr int NI = kStageItems;
@@ -434,9 +511,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const int ii = act[j] ? i : 0;
         tq[j] = ii & 3;
         const int mg = ii >> 2;
-        mq[j] = mg / a.Gn;
-        gq[j] = mg - mq[j] * a.Gn;
-        const uint8_t *src = xs + mq[j] * a.tok_stride + (gq[j] * G + Span::start(tq[j])) * 2;
+        mq[j] = mg / Jb.Gn;
+        gq[j] = mg - mq[j] * Jb.Gn;
+        const uint8_t *src = xs + mq[j] * Jb.tok_stride + (gq[j] * G + Span::start(tq[j])) * 2;
 #pragma unroll
         for (int v = 0; v < SL / 8; ++v) {
           const uint4 q = *reinterpret_cast<const uint4 *>(src + 16 * v);
@@ -490,7 +567,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const float inv_lo = __uint_as_float(static_cast<uint32_t>(127 - e_lo) << 23);
         const float inv_hi = __uint_as_float(static_cast<uint32_t>(127 - e_hi) << 23);
         const float sc = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
-        uint8_t *dst = xs + mq[j] * a.tok_stride + (gq[j] * U) * 64 + tq[j] * 16;
+        uint8_t *dst = xs + mq[j] * Jb.tok_stride + (gq[j] * U) * 64 + tq[j] * 16;
         static_for<0, U>([&](auto C) {
           constexpr int c = C.value;
           if constexpr (FMT == 3) {  // fp16 pairs (elements 2i, 2i+1) of x * 2^e: exact in fp16's normal range
@@ -522,16 +599,17 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           });
           if (act[j]) *reinterpret_cast<uint4 *>(dst + c * 64) = make_uint4(lo[0], lo[1], hi[0], hi[1]);
         });
-        if (act[j] && tq[j] == 0) tab[mq[j] * a.Gn + gq[j]] = make_float4(sx[j], inv_lo, inv_hi, 0.0f);
+        if (act[j] && tq[j] == 0) tab[mq[j] * Jb.Gn + gq[j]] = make_float4(sx[j], inv_lo, inv_hi, 0.0f);
       });
     }
     // zero blocks, and the table rows of padding tokens
     const int zbytes = a.zero_stride + U * 64;
     for (int i = ctid; i < zbytes / 16; i += cthreads) reinterpret_cast<uint4 *>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
-    for (int i = a.M * a.Gn + ctid; i < MP * a.Gn; i += cthreads) tab[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  }
-  // all consumer warps (not the producer) meet here: the staged activations are complete
-  asm volatile("bar.sync 1, %0;" ::"r"(cthreads) : "memory");
+    for (int i = a.M * Jb.Gn + ctid; i < MP * Jb.Gn; i += cthreads) tab[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    // all consumer warps (not the producer) meet here: the staged activations are complete
+    asm volatile("bar.sync 1, %0;" ::"r"(cthreads) : "memory");
+  };
+  stage_acts(0);
   // timeout test: a wait on a barrier that nothing completes runs out, raises
   // the abort flag and sets the fault bit; every other wait then gives up
   if (a.stall) mbar_wait(stall_bar, 0, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
@@ -541,7 +619,6 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   const int g = lane >> 2, t = lane & 3;
   const int my_m = g / GS, my_j = g % GS;          // this lane's B column: token, group slot
   const bool my_real = my_m < a.M;
-  const uint8_t *xs_lane = xs + (my_real ? my_m : 0) * a.tok_stride + t * 16;
   const uint8_t *zero_lane = zero + (GS == 1 ? 0 : (my_m & 1)) * a.zero_stride + t * 16;
   const int lw0 = LaneWords<BITS, G>::first(t) * 4;
   constexpr int SPANS = FMT == 0 ? GS1 : FMT == 2 ? GS / 2 : GS;  // 32-code spans (MMA K steps) per fold
@@ -550,12 +627,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   // feeds) and the accumulator columns 2t, 2t+1 it receives (position t)
   const int b_slot = (g >> 1) % GS1;
   int b_tok[NMMA];
-  const uint8_t *b_lane[NMMA];
 #pragma unroll
-  for (int h = 0; h < NMMA; ++h) {
-    b_tok[h] = h * 4 + (g >> 1) / GS1;
-    b_lane[h] = xs + (b_tok[h] < a.M ? b_tok[h] : 0) * a.tok_stride + t * 16 + (g & 1) * 8;
-  }
+  for (int h = 0; h < NMMA; ++h) b_tok[h] = h * 4 + (g >> 1) / GS1;
   const uint8_t *zb_lane = zero + t * 16 + (g & 1) * 8;
   const int c_slot = t % GS1;
 
@@ -563,20 +636,60 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   // consumer warps round-robin, so a stage is shared by several warps and the
   // last stages of a launch spread over all of them.  W divides NS * nper, so
   // the units a warp meets in one ring slot are consecutive phases of it.
+  // Units are numbered across the matmuls of a launch (their stages follow one
+  // another in the ring), so warp cw takes global units cw, cw + W, ...
+  int gbase = 0;  // stages of the matmuls before this one
+  bool run = true;
+  // Every consumer warp walks every matmul, also after a failed wait (then
+  // without taking units), so that all of them meet at the named barriers.
+  for (int jx = 0; jx < a.njobs; ++jx) {
+  const Job &Jb = a.job[jx];
+  if (jx > 0) {
+    // Every unit of matmul jx - 1 in this CTA is done (its outputs stored);
+    // once every CTA is that far, the activations of matmul jx may be read.
+    asm volatile("bar.sync 1, %0;" ::"r"(cthreads) : "memory");
+    if (ctid == 0) {
+      for (int b = 0; b < a.red_bufs; ++b) red_ready[b] = red_done[b] = 0;  // tile numbers restart
+      if (grid_barrier(a.gbar, gridDim.x, abort_flag, wlim)) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");  // the copy below reads other CTAs' stores
+        mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * Jb.K * 2);
+        for (int m = 0; m < a.M; ++m)
+          bulk_g2s(xs + m * Jb.tok_stride, Jb.x + static_cast<int64_t>(m) * Jb.K, static_cast<uint32_t>(Jb.K) * 2,
+                   xbar);
+        *x_issued = jx + 1;
+      }
+    }
+    stage_acts(jx);
+    if (*abort_flag) run = false;
+  }
+  int64_t r0, r1;
+  cta_rows(jx, r0, r1);
+  const int nst = static_cast<int>((r1 - r0 + kRows - 1) / kRows) * Jb.nch;
+  const int gpc = Jb.Kc / G;  // groups per chunk
+  __nv_bfloat16 *yg = a.cta_per_tok > 0 ? yg0 : Jb.y;
+  const uint8_t *xs_lane = xs + (my_real ? my_m : 0) * Jb.tok_stride + t * 16;
+  const uint8_t *b_lane[NMMA];
+#pragma unroll
+  for (int h = 0; h < NMMA; ++h) b_lane[h] = xs + (b_tok[h] < a.M ? b_tok[h] : 0) * Jb.tok_stride + t * 16 + (g & 1) * 8;
   const int nunits = nst * a.nper;
-  for (int u = cw; u < nunits; u += a.W) {
+  const int ubase = gbase * a.nper;
+  for (int u = ((cw - ubase) % a.W + a.W) % a.W; run && u < nunits; u += a.W) {
     const int st = u / a.nper, p = u - st * a.nper;
-    const int s = st % a.NS;
-    if (!mbar_wait(&full[s], (st / a.NS) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim)) break;
-    const int T = st / a.nch, ch = st - T * a.nch;
-    const int64_t rb = tile_base(T);
+    const int gst = gbase + st;
+    const int s = gst % a.NS;
+    if (!mbar_wait(&full[s], (gst / a.NS) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim)) {
+      run = false;
+      break;
+    }
+    const int T = st / Jb.nch, ch = st - T * Jb.nch;
+    const int64_t rb = tile_base(r0, r1, T);
     const int v0 = static_cast<int>(r0 + static_cast<int64_t>(T) * kRows - rb);  // rows [v0, 16) are new
     auto row_ok = [&](int r) { return r >= v0 && rb + r < r1; };
     const uint8_t *stg = ring + static_cast<size_t>(s) * a.stage_bytes;
-    const uint8_t *wr0 = stg + g * a.pitch_w + lw0;
-    const uint8_t *wr1 = wr0 + 8 * a.pitch_w;
-    const uint8_t *sr0 = stg + a.s_off + g * a.pitch_s, *sr1 = sr0 + 8 * a.pitch_s;
-    const uint8_t *br0 = stg + a.b_off + g * a.pitch_s, *br1 = br0 + 8 * a.pitch_s;
+    const uint8_t *wr0 = stg + g * Jb.pitch_w + lw0;
+    const uint8_t *wr1 = wr0 + 8 * Jb.pitch_w;
+    const uint8_t *sr0 = stg + Jb.s_off + g * Jb.pitch_s, *sr1 = sr0 + 8 * Jb.pitch_s;
+    const uint8_t *br0 = stg + Jb.b_off + g * Jb.pitch_s, *br1 = br0 + 8 * Jb.pitch_s;
     const int gch0 = ch * gpc;
     // Per (row, token) partials of this unit, held by some lanes: value q is
     // (row vrow[q], token vtok[q]) of the tile.
@@ -588,7 +701,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       float2 acc1[NMMA];  // rows (g, g+8) of token h * 4 + t / GS1
 #pragma unroll
       for (int h = 0; h < NMMA; ++h) acc1[h] = make_float2(0.0f, 0.0f);
-      for (int pf = p * a.fpu; pf < (p + 1) * a.fpu; ++pf) {  // the unit's folds
+      for (int pf = p * Jb.fpu; pf < (p + 1) * Jb.fpu; ++pf) {  // the unit's folds
         int dd[NMMA][NACC1][4];  // (lo, hi) digit sums of rows g and g+8 at position t
 #pragma unroll
         for (int h = 0; h < NMMA; ++h)
@@ -632,7 +745,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
             hi1 += dd[h][i][3];
           }
           const float2 D = make_float2(static_cast<float>(lo0 + 256 * hi0), static_cast<float>(lo1 + 256 * hi1));
-          const float4 T4 = tab[(h * 4 + t / GS1) * a.Gn + gch0 + gl];
+          const float4 T4 = tab[(h * 4 + t / GS1) * Jb.Gn + gch0 + gl];
           acc1[h] = ffma2(__fmul2_rn(sv, make_float2(T4.z, T4.z)), __fmul2_rn(D, make_float2(T4.y, T4.y)),
                           ffma2(bv2, make_float2(T4.x, T4.x), acc1[h]));
         }
@@ -662,7 +775,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     } else {
       float2 accA = make_float2(0.0f, 0.0f), accB = make_float2(0.0f, 0.0f);  // rows g, g+8 x columns 2t, 2t+1
 
-      for (int pf = p * a.fpu; pf < (p + 1) * a.fpu; ++pf) {  // the unit's folds
+      for (int pf = p * Jb.fpu; pf < (p + 1) * Jb.fpu; ++pf) {  // the unit's folds
         int dl[NACC][4], dh[NACC][4];  // sum q * lo, sum q * hi
         // mxfp4: the same sums over the negative codes' magnitudes, subtracted below
         int nl[FMT >= 1 ? NACC : 1][4], nh[FMT >= 1 ? NACC : 1][4];
@@ -766,10 +879,10 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
             b1 = __half22float2(*reinterpret_cast<const __half2 *>(br1 + gl * 2));
           }
           if constexpr (FMT == 2) {  // both columns lie in span gl / 2 of the chunk
-            T0 = T1 = tab[mt * a.Gn + gch0 + gl / 2];
+            T0 = T1 = tab[mt * Jb.Gn + gch0 + gl / 2];
           } else {
-            T0 = tab[mt * a.Gn + gch0 + gl];
-            T1 = tab[mt * a.Gn + gch0 + gl + 1];
+            T0 = tab[mt * Jb.Gn + gch0 + gl];
+            T1 = tab[mt * Jb.Gn + gch0 + gl + 1];
           }
         } else {
           const int gl = pf;  // one group; columns 2t, 2t+1 are tokens 2t, 2t+1
@@ -790,8 +903,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           s1 = make_float2(sv1, sv1);
           b0 = make_float2(bv0, bv0);
           b1 = make_float2(bv1, bv1);
-          T0 = tab[(2 * t) * a.Gn + gch0 + gl];
-          T1 = tab[(2 * t + 1) * a.Gn + gch0 + gl];
+          T0 = tab[(2 * t) * Jb.Gn + gch0 + gl];
+          T1 = tab[(2 * t + 1) * Jb.Gn + gch0 + gl];
         }
         const float2 tx = make_float2(T0.x, T1.x), ty = make_float2(T0.y, T1.y), tz = make_float2(T0.z, T1.z);
         // y += (s * 2^-e_hi) * (D * 2^-e_lo) + b * sum x   (block-scaled modes: no bias)
@@ -850,21 +963,24 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         if (q >= nv) break;
         if (direct) {
           if (vtok[q] < a.M && row_ok(vrow[q]))
-            yg[static_cast<int64_t>(vtok[q]) * a.N + rb + vrow[q]] = __float2bfloat16_rn(FMT == 2 ? v[q] * gs : v[q]);
+            yg[static_cast<int64_t>(vtok[q]) * Jb.N + rb + vrow[q]] = __float2bfloat16_rn(FMT == 2 ? v[q] * gs : v[q]);
         } else {
           dstv[vrow[q] * MP + vtok[q]] = v[q];
         }
       }
     };
-    if (a.parts == 1) {
+    if (Jb.parts == 1) {
       put(nullptr, true);
       continue;
     }
     const int b = T % a.red_bufs;
     const int rnd = T / a.red_bufs;
     // buffer b is free once the rnd earlier tiles that used it have been summed
-    if (!spin_until_at_least(&red_done[b], rnd, abort_flag, wlim)) break;
-    float *rbuf = red + static_cast<size_t>(b) * a.parts * kRows * MP;
+    if (!spin_until_at_least(&red_done[b], rnd, abort_flag, wlim)) {
+      run = false;
+      break;
+    }
+    float *rbuf = red + static_cast<size_t>(b) * Jb.parts * kRows * MP;
     put(rbuf + static_cast<size_t>(ch * a.nper + p) * kRows * MP, false);
     __syncwarp();
     // The warp whose partial completes the tile sums all of them, in part
@@ -872,16 +988,16 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     int last = 0;
     if (lane == 0) {
       __threadfence_block();
-      last = atomicAdd(&red_ready[b], 1) == (rnd + 1) * a.parts - 1;
+      last = atomicAdd(&red_ready[b], 1) == (rnd + 1) * Jb.parts - 1;
       __threadfence_block();
     }
     if (!__shfl_sync(0xffffffffu, last, 0)) continue;
     for (int idx = lane; idx < kRows * MP; idx += 32) {
       const int row = idx / MP, tok = idx - row * MP;
       float sum = 0.0f;
-      for (int c2 = 0; c2 < a.parts; ++c2) sum += rbuf[(static_cast<size_t>(c2) * kRows + row) * MP + tok];
+      for (int c2 = 0; c2 < Jb.parts; ++c2) sum += rbuf[(static_cast<size_t>(c2) * kRows + row) * MP + tok];
       if (tok < a.M && row_ok(row))
-        yg[static_cast<int64_t>(tok) * a.N + rb + row] = __float2bfloat16_rn(FMT == 2 ? sum * gs : sum);
+        yg[static_cast<int64_t>(tok) * Jb.N + rb + row] = __float2bfloat16_rn(FMT == 2 ? sum * gs : sum);
     }
     __syncwarp();
     if (lane == 0) {
@@ -889,6 +1005,8 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       atomicAdd(&red_done[b], 1);
     }
   }
+  gbase += nst;
+  }  // matmuls
   }  // consumers
 
   // After an abort, copies that were issued but never consumed may still be
@@ -897,7 +1015,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   __syncthreads();
   if (tid == 0 && *abort_flag) {
     const int issued = *issued_ctr;
-    mbar_drain(xbar, 0);
+    if (*x_issued > 0) mbar_drain(xbar, (*x_issued - 1) & 1);
     for (int j = max(0, issued - a.NS); j < issued; ++j) mbar_drain(&full[j % a.NS], (j / a.NS) & 1);
   }
 }
@@ -927,6 +1045,65 @@ static int64_t code_pitch(int64_t row_bytes, int bits, int G) {
   if ((bits == 2 && G == 32) || nwd == 1 || nwd == 8) return pitch_at(row_bytes, 32, 16);
   if (nwd == 2) return pitch_at(row_bytes, 64, 32);
   return pitch_at(row_bytes, 128, 64);
+}
+
+// Shared-memory layout of a launch (ring depth, consumer warps, offsets) for
+// staged activations of tok_stride bytes per token, tables of Gn groups and
+// `parts` partials per tile (the largest over the matmuls of a sequence);
+// the grid: one CTA per SM, each owning at least one 16-row tile of the
+// smallest matmul (min_rows rows).
+static bool place(Plan &pl, int64_t M, int U, int64_t tok_stride, int64_t Gn, int parts, bool dual, int sms,
+                  int64_t min_rows) {
+  Args &a = pl.a;
+  const int MP = pow2_tokens(static_cast<int>(M));
+  const int64_t budget = dual ? kDualSmem : 227 * 1024;
+  const int max_w = dual ? kDualConsumers : kMaxConsumers;
+  struct Layout {
+    int64_t xs_off, zero_off, tab_off, red_off, bar_off, total;
+  };
+  auto layout = [&](int ns) {
+    Layout L;
+    int64_t off = static_cast<int64_t>(ns) * a.stage_bytes;
+    L.xs_off = off;
+    off += M * tok_stride;
+    L.zero_off = round_up(off, 128) + 64;
+    off = L.zero_off + a.zero_stride + U * 64;
+    L.tab_off = round_up(off, 16);
+    off = L.tab_off + static_cast<int64_t>(MP) * Gn * 16;
+    L.red_off = off;
+    off += static_cast<int64_t>(a.red_bufs) * parts * kRows * MP * 4;
+    L.bar_off = round_up(off, 8);
+    L.total = L.bar_off + (2 * ns + 2) * 8 + (2 * a.red_bufs + 3) * 4;
+    return L;
+  };
+  // consumer warps: a divisor of NS * nper, so the units one warp takes in a
+  // ring slot are consecutive phases of that slot's barriers (a warp never
+  // waits on a phase two ahead of the barrier's).  Take the depth that fits and
+  // allows the most consumers (then the deepest).
+  const int nper = a.nper;
+  auto consumers = [&](int ns) {
+    for (int w = max_w; w >= 1; --w)
+      if ((ns * nper) % w == 0) return w;
+    return 1;
+  };
+  int best_ns = 0;
+  for (int ns = 2; ns <= kMaxStages; ++ns) {
+    if (layout(ns).total > budget) break;
+    if (best_ns == 0 || consumers(ns) >= consumers(best_ns)) best_ns = ns;
+  }
+  if (best_ns == 0 || (dual && best_ns < kDualMinStages)) return false;
+  const Layout L = layout(best_ns);
+  a.NS = best_ns;
+  a.W = consumers(best_ns);
+  a.xs_off = static_cast<int>(L.xs_off);
+  a.zero_off = static_cast<int>(L.zero_off);
+  a.tab_off = static_cast<int>(L.tab_off);
+  a.red_off = static_cast<int>(L.red_off);
+  a.bar_off = static_cast<int>(L.bar_off);
+  pl.smem = static_cast<size_t>(L.total);
+  pl.threads = 32 * (a.W + 1);
+  pl.grid = static_cast<int>(std::min<int64_t>(sms, min_rows / kRows));
+  return true;
 }
 
 // fmt 0: affine codes with fp16 scales and biases; fmt 1: mxfp4 (E2M1 codes,
@@ -962,28 +1139,30 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   const int64_t Kc = 8 * G * u, nch = K / Kc, gpc = Kc / G;
   Args &a = pl.a;
   a.early_w = 0;
+  a.njobs = 1;
+  a.gbar = nullptr;
   a.experts = nullptr;
   a.E = 1;
   a.cta_per_tok = 0;
   a.gscale = nullptr;
   a.M = static_cast<int>(M);
-  a.N = static_cast<int>(N);
-  a.K = static_cast<int>(K);
-  a.Gn = static_cast<int>(Gn);
-  a.Kc = static_cast<int>(Kc);
-  a.nch = static_cast<int>(nch);
-  a.pitch_w = static_cast<int>(code_pitch(Kc * bits / 8, bits, G));
+  a.job[0].N = static_cast<int>(N);
+  a.job[0].K = static_cast<int>(K);
+  a.job[0].Gn = static_cast<int>(Gn);
+  a.job[0].Kc = static_cast<int>(Kc);
+  a.job[0].nch = static_cast<int>(nch);
+  a.job[0].pitch_w = static_cast<int>(code_pitch(Kc * bits / 8, bits, G));
   const int sbytes = (fmt == 1 || fmt == 3) ? 1 : 2;  // scale bytes per 32-code span (nvfp4: two E4M3 bytes)
-  a.pitch_s = static_cast<int>(pitch_at(gpc * sbytes, 32, 16));
-  if (a.pitch_w / 8 > 256 || a.pitch_s / 8 > 256) return false;  // TMA box width (64-bit elements)
-  a.w_box_x = static_cast<int>(Kc * bits / 64);
-  a.sb_box_x = static_cast<int>(gpc * sbytes / 8);
+  a.job[0].pitch_s = static_cast<int>(pitch_at(gpc * sbytes, 32, 16));
+  if (a.job[0].pitch_w / 8 > 256 || a.job[0].pitch_s / 8 > 256) return false;  // TMA box width (64-bit elements)
+  a.job[0].w_box_x = static_cast<int>(Kc * bits / 64);
+  a.job[0].sb_box_x = static_cast<int>(gpc * sbytes / 8);
   // every tiled TMA copy starts on a 16-byte boundary: x * 8 bytes % 16 == 0 for every chunk
-  if (nch > 1 && (a.w_box_x % 2 != 0 || a.sb_box_x % 2 != 0)) return false;
-  a.s_off = kRows * a.pitch_w;
-  a.b_off = a.s_off + kRows * a.pitch_s;
-  a.stage_bytes = static_cast<int>(round_up((fmt >= 1 ? a.s_off : a.b_off) + kRows * a.pitch_s, 128));
-  a.tok_stride = static_cast<int>(2 * K + 64);
+  if (nch > 1 && (a.job[0].w_box_x % 2 != 0 || a.job[0].sb_box_x % 2 != 0)) return false;
+  a.job[0].s_off = kRows * a.job[0].pitch_w;
+  a.job[0].b_off = a.job[0].s_off + kRows * a.job[0].pitch_s;
+  a.stage_bytes = static_cast<int>(round_up((fmt >= 1 ? a.job[0].s_off : a.job[0].b_off) + kRows * a.job[0].pitch_s, 128));
+  a.job[0].tok_stride = static_cast<int>(2 * K + 64);
   a.zero_stride = static_cast<int>(round_up(U * 64, 128) + 64);
   // work units: fpu folds (a fold: the groups side by side above; nvfp4: twice as
   // many 16-weight groups) of one stage, at least kUnitCodes codes of a row
@@ -994,76 +1173,23 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   // MP = 8; the block-scaled formats 8/MP)
   const int GS = 8 / MP, SPANS = fmt == 0 ? (MP >= 4 ? 1 : 4 / MP) : fmt == 2 ? GS / 2 : GS;
   const int64_t fold = static_cast<int64_t>(SPANS) * G;  // codes of a row per fold
-  a.fpu = 1;
-  while (fold * a.fpu * 2 <= kUnitCodes && Kc % (fold * a.fpu * 2) == 0) a.fpu *= 2;
-  a.nper = static_cast<int>(Kc / (fold * a.fpu));
-  a.parts = static_cast<int>(nch) * a.nper;
+  a.job[0].fpu = 1;
+  while (fold * a.job[0].fpu * 2 <= kUnitCodes && Kc % (fold * a.job[0].fpu * 2) == 0) a.job[0].fpu *= 2;
+  a.nper = static_cast<int>(Kc / (fold * a.job[0].fpu));
+  a.job[0].parts = static_cast<int>(nch) * a.nper;
   // tiles in flight: the units in progress (one per warp, at most
   // kMaxConsumers) span at most two tiles once a tile has that many units
-  a.red_bufs = a.parts == 1 ? 1 : a.parts >= 2 * kMaxConsumers ? 2 : a.parts >= kMaxConsumers ? 3 : kRedBufs;
+  a.red_bufs = a.job[0].parts == 1 ? 1 : a.job[0].parts >= 2 * kMaxConsumers ? 2 : a.job[0].parts >= kMaxConsumers ? 3 : kRedBufs;
   a.wait_cycles = kWaitCycles;
   a.stall = 0;
-  const int64_t budget = dual ? kDualSmem : 227 * 1024;
-  const int max_w = dual ? kDualConsumers : kMaxConsumers;
-  struct Layout {
-    int64_t xs_off, zero_off, tab_off, red_off, bar_off, total;
-  };
-  auto layout = [&](int ns) {
-    Layout L;
-    int64_t off = static_cast<int64_t>(ns) * a.stage_bytes;
-    L.xs_off = off;
-    off += M * a.tok_stride;
-    L.zero_off = round_up(off, 128) + 64;
-    off = L.zero_off + a.zero_stride + U * 64;
-    L.tab_off = round_up(off, 16);
-    off = L.tab_off + static_cast<int64_t>(MP) * Gn * 16;
-    L.red_off = off;
-    off += static_cast<int64_t>(a.red_bufs) * a.parts * kRows * MP * 4;
-    L.bar_off = round_up(off, 8);
-    L.total = L.bar_off + (2 * ns + 2) * 8 + (2 * a.red_bufs + 2) * 4;
-    return L;
-  };
-  // consumer warps: a divisor of NS * nper, so the units one warp takes in a
-  // ring slot are consecutive phases of that slot's barriers (a warp never
-  // waits on a phase two ahead of the barrier's).  Take the depth that fits and
-  // allows the most consumers (then the deepest).
-  const int nper = a.nper;
-  auto consumers = [&](int ns) {
-    for (int w = max_w; w >= 1; --w)
-      if ((ns * nper) % w == 0) return w;
-    return 1;
-  };
-  int best_ns = 0;
-  for (int ns = 2; ns <= kMaxStages; ++ns) {
-    if (layout(ns).total > budget) break;
-    if (best_ns == 0 || consumers(ns) >= consumers(best_ns)) best_ns = ns;
-  }
-  if (best_ns == 0 || (dual && best_ns < kDualMinStages)) return false;
-  const Layout L = layout(best_ns);
-  a.NS = best_ns;
-  a.W = consumers(best_ns);
-  a.xs_off = static_cast<int>(L.xs_off);
-  a.zero_off = static_cast<int>(L.zero_off);
-  a.tab_off = static_cast<int>(L.tab_off);
-  a.red_off = static_cast<int>(L.red_off);
-  a.bar_off = static_cast<int>(L.bar_off);
-  pl.smem = static_cast<size_t>(L.total);
-  pl.threads = 32 * (a.W + 1);
-  pl.grid = static_cast<int>(std::min<int64_t>(sms, N / kRows));
-  return true;
+  return place(pl, M, U, a.job[0].tok_stride, Gn, a.job[0].parts, dual, sms, N);
 }
-
-struct Maps {
-  CUtensorMap w, s, b;
-};
+using Maps = JobMaps<1>;
 
 // The operands of a call (everything in Args that is not layout).
 static void copy_operands(Args &dst, const Args &src) {
-  dst.x = src.x;
-  dst.packed = src.packed;
-  dst.scales = src.scales;
-  dst.biases = src.biases;
-  dst.y = src.y;
+  dst.job[0].x = src.job[0].x;
+  dst.job[0].y = src.job[0].y;
   dst.experts = src.experts;
   dst.E = src.E;
   dst.cta_per_tok = src.cta_per_tok;
@@ -1137,7 +1263,7 @@ static cudaError_t launch(const Plan &pl_one, const Plan *dual, const Maps &mp, 
     cached_smem = pl.smem;
   }
   if (!overlap) {
-    kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.a, mp.w, mp.s, mp.b);
+    kern<<<pl.grid, pl.threads, pl.smem, stream>>>(pl.a, mp);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -1150,7 +1276,7 @@ static cudaError_t launch(const Plan &pl_one, const Plan *dual, const Maps &mp, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, pl.a, mp.w, mp.s, mp.b);
+  return cudaLaunchKernelEx(&cfg, kern, pl.a, mp);
 }
 
 template <int BITS, int G, int FMT = 0>
@@ -1184,6 +1310,91 @@ static bool encode_rows(CUtensorMap *map, const void *base, int64_t rows, int64_
                           CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// ---------------------------------------------------------------------------
+// Sequence launches: several matmuls (same M, G, bits) in one grid
+// ---------------------------------------------------------------------------
+// Grid barriers of sequence launches, one (count, generation) pair per slot.
+// Consecutive launches take consecutive slots, so launches in flight at the
+// same time on different streams share none unless kSeqBarSlots of them do.
+constexpr int kSeqBarSlots = 64;
+__device__ unsigned g_seq_bar[kSeqBarSlots][2];
+
+static bool make_seq_plan(int n, const int64_t *N, const int64_t *K, int64_t M, int G, int bits, int sms, Plan &pl) {
+  if (n < 1 || n > kSeqMax) return false;
+  Plan pj[kSeqMax];
+  for (int j = 0; j < n; ++j)
+    if (!make_plan(M, N[j], K[j], G, bits, sms, pj[j])) return false;
+  pl = pj[0];
+  Args &a = pl.a;
+  a.njobs = n;
+  int64_t tok = 0, gn = 0, rows = N[0];
+  int parts = 0, stage = 0, red = 0;
+  for (int j = 0; j < n; ++j) {
+    if (pj[j].a.nper != a.nper) return false;  // one unit size for the whole ring
+    a.job[j] = pj[j].a.job[0];
+    tok = std::max<int64_t>(tok, a.job[j].tok_stride);
+    gn = std::max<int64_t>(gn, a.job[j].Gn);
+    parts = std::max(parts, a.job[j].parts);
+    stage = std::max(stage, pj[j].a.stage_bytes);
+    red = std::max(red, pj[j].a.red_bufs);
+    rows = std::min(rows, N[j]);
+  }
+  a.stage_bytes = stage;
+  a.red_bufs = red;
+  return place(pl, M, G / 32, tok, gn, parts, false, sms, rows);
+}
+
+template <int BITS, int G, int MP>
+static cudaError_t launch_seq(const Plan &pl_in, const JobMaps<kSeqMax> &mp, bool overlap, cudaStream_t stream) {
+  auto kern = qmv_tc_kernel<BITS, G, MP, 0, kSeqMax>;
+  Plan pl = pl_in;
+  pl.a.early_w = overlap ? kEarlyStages : 0;
+  pl.a.wait_cycles = g_wait_limit.load(std::memory_order_relaxed);
+  pl.a.stall = g_wait_stall.load(std::memory_order_relaxed) ? 1 : 0;
+  static thread_local int cached_dev = -1;
+  static thread_local size_t cached_smem = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev || pl.smem > cached_smem) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pl.smem))) !=
+        cudaSuccess)
+      return e;
+    cached_dev = dev;
+    cached_smem = pl.smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(pl.threads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, pl.a, mp);
+}
+
+template <int BITS, int G>
+static cudaError_t launch_seq_mp(const Plan &pl, const JobMaps<kSeqMax> &mp, bool overlap, cudaStream_t stream) {
+  switch (pow2_tokens(pl.a.M)) {
+    case 1: return launch_seq<BITS, G, 1>(pl, mp, overlap, stream);
+    case 2: return launch_seq<BITS, G, 2>(pl, mp, overlap, stream);
+    case 4: return launch_seq<BITS, G, 4>(pl, mp, overlap, stream);
+    default: return launch_seq<BITS, G, 8>(pl, mp, overlap, stream);
+  }
+}
+
+template <int BITS>
+static cudaError_t launch_seq_g(const Plan &pl, const JobMaps<kSeqMax> &mp, int G, bool overlap, cudaStream_t stream) {
+  switch (G) {
+    case 32: return launch_seq_mp<BITS, 32>(pl, mp, overlap, stream);
+    case 64: return launch_seq_mp<BITS, 64>(pl, mp, overlap, stream);
+    default: return launch_seq_mp<BITS, 128>(pl, mp, overlap, stream);
+  }
+}
+
 }  // namespace tc
 
 bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits) {
@@ -1204,24 +1415,72 @@ cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_
   }
   tc::Plan pl;
   if (!tc::make_plan(M, N, K, G, bits, sms, pl)) return cudaErrorInvalidValue;
-  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-  pl.a.packed = packed;
-  pl.a.scales = reinterpret_cast<const __half *>(scales);
-  pl.a.biases = reinterpret_cast<const __half *>(biases);
-  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  pl.a.job[0].x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.job[0].y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
   tc::Plan dpl;
   const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, G, bits, sms, 0, dpl);
   tc::Maps mp;
   const int64_t row_bytes = K * bits / 8, sb_bytes = K / G * 2;
-  if (!tc::encode_rows(&mp.w, packed, N, row_bytes, pl.a.pitch_w) ||
-      !tc::encode_rows(&mp.s, scales, N, sb_bytes, pl.a.pitch_s) ||
-      !tc::encode_rows(&mp.b, biases, N, sb_bytes, pl.a.pitch_s))
+  if (!tc::encode_rows(&mp.w[0], packed, N, row_bytes, pl.a.job[0].pitch_w) ||
+      !tc::encode_rows(&mp.s[0], scales, N, sb_bytes, pl.a.job[0].pitch_s) ||
+      !tc::encode_rows(&mp.b[0], biases, N, sb_bytes, pl.a.job[0].pitch_s))
     return cudaErrorInvalidValue;
   switch (bits) {
     case 2: return tc::launch_g<2>(pl, dual, mp, G, overlap, s);
     case 4: return tc::launch_g<4>(pl, dual, mp, G, overlap, s);
     default: return tc::launch_g<8>(pl, dual, mp, G, overlap, s);
+  }
+}
+
+bool qmv_tc_seq_supported(int n, const int64_t *N, const int64_t *K, int64_t M, int G, int bits) {
+  tc::Plan pl;
+  return tc::make_seq_plan(n, N, K, M, G, bits, 148, pl);
+}
+
+cudaError_t launch_qmv_tc_seq(int n, const SeqCall *calls, int64_t M, int G, int bits, uint32_t flags, cudaStream_t s) {
+  static thread_local int cached_dev = -1, sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  if (n < 1 || n > tc::kSeqMax) return cudaErrorInvalidValue;
+  int64_t N[tc::kSeqMax], K[tc::kSeqMax];
+  for (int j = 0; j < n; ++j) {
+    N[j] = calls[j].N;
+    K[j] = calls[j].K;
+  }
+  tc::Plan pl;
+  if (!tc::make_seq_plan(n, N, K, M, G, bits, sms, pl)) return cudaErrorInvalidValue;
+  tc::JobMaps<tc::kSeqMax> mp;
+  for (int j = 0; j < n; ++j) {
+    pl.a.job[j].x = reinterpret_cast<const __nv_bfloat16 *>(calls[j].x);
+    pl.a.job[j].y = reinterpret_cast<__nv_bfloat16 *>(calls[j].y);
+    const int64_t row_bytes = K[j] * bits / 8, sb_bytes = K[j] / G * 2;
+    if (!tc::encode_rows(&mp.w[j], calls[j].packed, N[j], row_bytes, pl.a.job[j].pitch_w) ||
+        !tc::encode_rows(&mp.s[j], calls[j].scales, N[j], sb_bytes, pl.a.job[j].pitch_s) ||
+        !tc::encode_rows(&mp.b[j], calls[j].biases, N[j], sb_bytes, pl.a.job[j].pitch_s))
+      return cudaErrorInvalidValue;
+  }
+  for (int j = n; j < tc::kSeqMax; ++j) {  // unused entries: copies of the first (never read)
+    mp.w[j] = mp.w[0];
+    mp.s[j] = mp.s[0];
+    mp.b[j] = mp.b[0];
+  }
+  // a grid barrier slot for this launch
+  static std::atomic<unsigned> next_slot{0};
+  void *bar = nullptr;
+  if ((e = cudaGetSymbolAddress(&bar, tc::g_seq_bar)) != cudaSuccess) return e;
+  const unsigned slot = next_slot.fetch_add(1, std::memory_order_relaxed) % tc::kSeqBarSlots;
+  pl.a.gbar = reinterpret_cast<unsigned *>(bar) + 2 * slot;
+  const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
+  switch (bits) {
+    case 2: return tc::launch_seq_g<2>(pl, mp, G, overlap, s);
+    case 4: return tc::launch_seq_g<4>(pl, mp, G, overlap, s);
+    default: return tc::launch_seq_g<8>(pl, mp, G, overlap, s);
   }
 }
 
@@ -1245,16 +1504,13 @@ cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint
   pl.a.cta_per_tok = static_cast<int>(per_tok);
   pl.a.experts = experts;
   pl.a.E = static_cast<int>(E);
-  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-  pl.a.packed = packed;
-  pl.a.scales = reinterpret_cast<const __half *>(scales);
-  pl.a.biases = reinterpret_cast<const __half *>(biases);
-  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  pl.a.job[0].x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.job[0].y = reinterpret_cast<__nv_bfloat16 *>(y);
   tc::Maps mp;
   const int64_t row_bytes = K * bits / 8, sb_bytes = K / G * 2;
-  if (!tc::encode_rows(&mp.w, packed, E * N, row_bytes, pl.a.pitch_w) ||
-      !tc::encode_rows(&mp.s, scales, E * N, sb_bytes, pl.a.pitch_s) ||
-      !tc::encode_rows(&mp.b, biases, E * N, sb_bytes, pl.a.pitch_s))
+  if (!tc::encode_rows(&mp.w[0], packed, E * N, row_bytes, pl.a.job[0].pitch_w) ||
+      !tc::encode_rows(&mp.s[0], scales, E * N, sb_bytes, pl.a.job[0].pitch_s) ||
+      !tc::encode_rows(&mp.b[0], biases, E * N, sb_bytes, pl.a.job[0].pitch_s))
     return cudaErrorInvalidValue;
   switch (bits) {
     case 2: return tc::launch_g<2>(pl, nullptr, mp, G, false, s);
@@ -1281,18 +1537,15 @@ cudaError_t launch_mxfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
   }
   tc::Plan pl;
   if (!tc::make_plan(M, N, K, 32, 4, sms, pl, 1)) return cudaErrorInvalidValue;
-  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-  pl.a.packed = packed;
-  pl.a.scales = reinterpret_cast<const __half *>(scales);  // read as bytes by the mxfp4 kernel
-  pl.a.biases = nullptr;
-  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  pl.a.job[0].x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.job[0].y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
   tc::Plan dpl;
   const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, 32, 4, sms, 1, dpl);
   tc::Maps mp;
-  if (!tc::encode_rows(&mp.w, packed, N, K / 2, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 32, pl.a.pitch_s))
+  if (!tc::encode_rows(&mp.w[0], packed, N, K / 2, pl.a.job[0].pitch_w) || !tc::encode_rows(&mp.s[0], scales, N, K / 32, pl.a.job[0].pitch_s))
     return cudaErrorInvalidValue;
-  mp.b = mp.s;  // no bias map: the kernel never reads this one
+  mp.b[0] = mp.s[0];  // no bias map: the kernel never reads this one
   return tc::launch_mp<4, 32, 1>(pl, dual, mp, overlap, s);
 }
 
@@ -1314,18 +1567,15 @@ cudaError_t launch_mxfp8_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
   }
   tc::Plan pl;
   if (!tc::make_plan(M, N, K, 32, 8, sms, pl, 3)) return cudaErrorInvalidValue;
-  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-  pl.a.packed = packed;
-  pl.a.scales = reinterpret_cast<const __half *>(scales);  // read as bytes by the mxfp8 kernel
-  pl.a.biases = nullptr;
-  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  pl.a.job[0].x = reinterpret_cast<const __nv_bfloat16 *>(x);
+  pl.a.job[0].y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
   tc::Plan dpl;
   const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, 32, 8, sms, 3, dpl);
   tc::Maps mp;
-  if (!tc::encode_rows(&mp.w, packed, N, K, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 32, pl.a.pitch_s))
+  if (!tc::encode_rows(&mp.w[0], packed, N, K, pl.a.job[0].pitch_w) || !tc::encode_rows(&mp.s[0], scales, N, K / 32, pl.a.job[0].pitch_s))
     return cudaErrorInvalidValue;
-  mp.b = mp.s;  // no bias map: the kernel never reads this one
+  mp.b[0] = mp.s[0];  // no bias map: the kernel never reads this one
   return tc::launch_mp<8, 32, 3>(pl, dual, mp, overlap, s);
 }
 
@@ -1348,19 +1598,16 @@ cudaError_t launch_nvfp4_tc(const uint16_t *x, int64_t M, int64_t K, const uint3
   }
   tc::Plan pl;
   if (!tc::make_plan(M, N, K, 32, 4, sms, pl, 2)) return cudaErrorInvalidValue;
-  pl.a.x = reinterpret_cast<const __nv_bfloat16 *>(x);
-  pl.a.packed = packed;
-  pl.a.scales = reinterpret_cast<const __half *>(scales);  // read as bytes by the nvfp4 kernel
-  pl.a.biases = nullptr;
+  pl.a.job[0].x = reinterpret_cast<const __nv_bfloat16 *>(x);
   pl.a.gscale = gscale;
-  pl.a.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  pl.a.job[0].y = reinterpret_cast<__nv_bfloat16 *>(y);
   const bool overlap = (flags & AQ_MATMUL_OVERLAP_PREVIOUS) != 0;
   tc::Plan dpl;
   const tc::Plan *dual = tc::dual_plan(pl, overlap, M, N, K, 32, 4, sms, 2, dpl);
   tc::Maps mp;
-  if (!tc::encode_rows(&mp.w, packed, N, K / 2, pl.a.pitch_w) || !tc::encode_rows(&mp.s, scales, N, K / 16, pl.a.pitch_s))
+  if (!tc::encode_rows(&mp.w[0], packed, N, K / 2, pl.a.job[0].pitch_w) || !tc::encode_rows(&mp.s[0], scales, N, K / 16, pl.a.job[0].pitch_s))
     return cudaErrorInvalidValue;
-  mp.b = mp.s;  // no bias map: the kernel never reads this one
+  mp.b[0] = mp.s[0];  // no bias map: the kernel never reads this one
   switch (tc::pow2_tokens(pl.a.M)) {
     case 1: return tc::launch<4, 32, 1, 2>(pl, dual, mp, overlap, s);
     case 2: return tc::launch<4, 32, 2, 2>(pl, dual, mp, overlap, s);
@@ -1375,6 +1622,11 @@ cudaError_t read_and_clear_qmv_tc_fault(uint32_t *word) {
   cudaError_t e = cudaMemcpyFromSymbol(word, g_qmv_tc_fault, sizeof(uint32_t));
   if (e != cudaSuccess) return e;
   const uint32_t zero = 0;
+  if (*word != 0) {
+    // a sequence launch that gave up may have left a grid barrier half passed
+    static const unsigned zeros[tc::kSeqBarSlots][2] = {};
+    if ((e = cudaMemcpyToSymbol(tc::g_seq_bar, zeros, sizeof(zeros))) != cudaSuccess) return e;
+  }
   return cudaMemcpyToSymbol(g_qmv_tc_fault, &zero, sizeof(uint32_t));
 }
 
