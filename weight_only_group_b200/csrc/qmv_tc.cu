@@ -1173,8 +1173,11 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   // MP = 8; the block-scaled formats 8/MP)
   const int GS = 8 / MP, SPANS = fmt == 0 ? (MP >= 4 ? 1 : 4 / MP) : fmt == 2 ? GS / 2 : GS;
   const int64_t fold = static_cast<int64_t>(SPANS) * G;  // codes of a row per fold
+  // folds per unit: the largest divisor of the stage's folds within kUnitCodes
+  const int64_t stage_folds = Kc / fold;
   a.job[0].fpu = 1;
-  while (fold * a.job[0].fpu * 2 <= kUnitCodes && Kc % (fold * a.job[0].fpu * 2) == 0) a.job[0].fpu *= 2;
+  for (int64_t d = 1; d <= stage_folds; ++d)
+    if (stage_folds % d == 0 && fold * d <= kUnitCodes) a.job[0].fpu = static_cast<int>(d);
   a.nper = static_cast<int>(Kc / (fold * a.job[0].fpu));
   a.job[0].parts = static_cast<int>(nch) * a.nper;
   // tiles in flight: the units in progress (one per warp, at most
