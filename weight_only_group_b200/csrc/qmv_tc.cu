@@ -45,12 +45,16 @@
 //    elements, box rows padded so that the lanes of one shared-memory read hit
 //    distinct banks).  A CTA owns >= 16 rows; its last tile is moved up to end
 //    on its last row, so it repeats a few rows just read (L2 hits, masked out
-//    of the output) and never reads another CTA's rows.  The activations
-//    arrive by one bulk copy per token and are converted in place.
-//    Consumer warps (a divisor of the ring depth: one warp per slot) take
-//    whole stages round-robin.  The chunks of one tile are
-//    summed in chunk order through shared memory by the warp that handled the
-//    last chunk (deterministic), then stored as bf16 (RNE).
+//    of the output) and never reads another CTA's rows.  The consumer warps
+//    read the activations with plain loads (a copy through the copy engine
+//    would queue behind the weight stages) and stage their digits in shared
+//    memory.  Consumer warps (a divisor of the ring depth: one warp per slot)
+//    take whole stages round-robin.  The chunks of one tile are summed in
+//    chunk order through shared memory by the warp that handled the last chunk
+//    (deterministic), then stored as bf16 (RNE).
+//  * Sequence launches run up to four matmuls in one grid: the ring carries
+//    their stages back to back, and a grid-wide barrier separates the end of
+//    one matmul from the activation loads of the next.
 //  * Every wait is bounded; a timeout sets a bit of g_qmv_tc_fault.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -87,7 +91,6 @@ constexpr int kUnitCodes = 1 << 20;     // codes of a row a work unit covers at 
 constexpr int kMaxStages = 16;
 constexpr int kStageTarget = AQ_QMV_STAGE_TARGET;  // packed bytes of one stage we aim for (<= 1 KB per row)
 constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
-constexpr int kEarlyStages = 2;
 constexpr int kStageItems = 2;           // activation staging items per thread per round          // weight stages issued before the previous kernel completes (overlap mode)
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds |v| < 2^22 to an integer
 
@@ -286,7 +289,6 @@ struct Args {
   int xs_off;
   int zero_off, zero_stride; // two zero blocks
   int tab_off, red_off, bar_off;
-  int early_w;               // weight stages issued before the previous kernel has completed
   // gather mode (cta_per_tok > 0): token t = blockIdx.x / cta_per_tok multiplies
   // its x row by expert experts[t] of E stacked [N, K] weights (rows e*N.. of
   // the [E*N, K] maps); each of its cta_per_tok CTAs owns a slice of the N rows
@@ -360,16 +362,14 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   uint8_t *ring = smem;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.bar_off);
   uint64_t *empty = full + a.NS;
-  uint64_t *xbar = empty + a.NS;
-  uint64_t *stall_bar = xbar + 1;  // no thread ever arrives on it (the timeout test waits on it)
+  uint64_t *stall_bar = empty + a.NS;  // no thread ever arrives on it (the timeout test waits on it)
   // chunk partials of a tile: red_ready[b] counts partials written into buffer
   // b, red_done[b] the tiles summed out of it (monotonic, so a waiter can never
   // mistake an older round for the one it needs)
-  int *red_ready = reinterpret_cast<int *>(xbar + 2);
+  int *red_ready = reinterpret_cast<int *>(stall_bar + 2);  // (one barrier slot spare)
   int *red_done = red_ready + a.red_bufs;
   volatile int *abort_flag = red_done + a.red_bufs;
   int *issued_ctr = red_done + a.red_bufs + 1;  // stages the producer issued (read after an abort)
-  int *x_issued = issued_ctr + 1;                // activation copies issued (one per matmul)
   uint8_t *xs = smem + a.xs_off;
   uint8_t *zero = smem + a.zero_off;
   float4 *tab = reinterpret_cast<float4 *>(smem + a.tab_off);  // [MP][Gn]: (sum x, 2^-e_lo, 2^-e_hi, 0)
@@ -377,6 +377,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const Job &J0 = a.job[0];
+  // matmul jx's fields, by value: read from the parameters once per matmul (a
+  // single-matmul launch indexes them at compile-time offsets)
+  auto job_of = [&](int jx) -> Job { return a.job[NJ == 1 ? 0 : jx]; };
   int64_t gr0 = 0, gr1 = 0, wrow0 = 0;  // gather mode: rows [gr0, gr1) of this CTA; first row of its expert
   const __nv_bfloat16 *xg = J0.x;       // gather mode: this CTA's token row
   __nv_bfloat16 *yg0 = J0.y;
@@ -400,14 +403,15 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       r0 = gr0;
       r1 = gr1;
     } else {
-      r0 = static_cast<int64_t>(blockIdx.x) * a.job[jx].N / gridDim.x;
-      r1 = static_cast<int64_t>(blockIdx.x + 1) * a.job[jx].N / gridDim.x;
+      const int64_t n = job_of(jx).N;
+      r0 = static_cast<int64_t>(blockIdx.x) * n / gridDim.x;
+      r1 = static_cast<int64_t>(blockIdx.x + 1) * n / gridDim.x;
     }
   };
   auto job_stages = [&](int jx) {
     int64_t r0, r1;
     cta_rows(jx, r0, r1);
-    return static_cast<int>((r1 - r0 + kRows - 1) / kRows) * a.job[jx].nch;
+    return static_cast<int>((r1 - r0 + kRows - 1) / kRows) * job_of(jx).nch;
   };
   const long long wlim = a.wait_cycles;
 
@@ -418,18 +422,15 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   auto tile_base = [&](int64_t r0, int64_t r1, int T) { return min(r0 + static_cast<int64_t>(T) * kRows, r1 - kRows); };
   // One stage: 16 rows of codes, scales and biases of (tile, chunk) of matmul
   // jx, into ring slot gst % NS (gst counts the stages of all matmuls); one lane.
-  auto issue = [&](int jx, int st, int gst) {
-    const Job &Jb = a.job[jx];
-    int64_t r0, r1;
-    cta_rows(jx, r0, r1);
+  auto issue = [&](int jx, const Job &Jb, int64_t r0, int64_t r1, int st, int gst) {
     const int s = gst % a.NS;
     const int T = st / Jb.nch, ch = st - T * Jb.nch;
     const int rb = static_cast<int>(wrow0 + tile_base(r0, r1, T));
     uint8_t *dst = ring + static_cast<size_t>(s) * a.stage_bytes;
     mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kRows * (Jb.pitch_w + (FMT == 0 ? 2 : 1) * Jb.pitch_s)));
-    tma_load_2d(dst, &mp.w[jx], &full[s], ch * Jb.w_box_x, rb);
-    tma_load_2d(dst + Jb.s_off, &mp.s[jx], &full[s], ch * Jb.sb_box_x, rb);
-    if constexpr (FMT == 0) tma_load_2d(dst + Jb.b_off, &mp.b[jx], &full[s], ch * Jb.sb_box_x, rb);
+    tma_load_2d(dst, &mp.w[NJ == 1 ? 0 : jx], &full[s], ch * Jb.w_box_x, rb);
+    tma_load_2d(dst + Jb.s_off, &mp.s[NJ == 1 ? 0 : jx], &full[s], ch * Jb.sb_box_x, rb);
+    if constexpr (FMT == 0) tma_load_2d(dst + Jb.b_off, &mp.b[NJ == 1 ? 0 : jx], &full[s], ch * Jb.sb_box_x, rb);
   };
 
   if (tid == 0) {
@@ -438,11 +439,9 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       mbar_init(&empty[s], a.nper);  // every unit (fold) of a stage releases it once
     }
     for (int b = 0; b < a.red_bufs; ++b) red_ready[b] = red_done[b] = 0;
-    mbar_init(xbar, 1);
     mbar_init(stall_bar, 1);
     *abort_flag = 0;
     *issued_ctr = 0;
-    *x_issued = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -451,37 +450,27 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // Weights first when the caller allows it (they are not written by the
-    // kernel this one may overlap), then, once the kernel before has completed,
-    // the activations of the first matmul (one row per token, raw bf16 into
-    // the staging area), then every stage of every matmul in order, each as
-    // soon as its ring slot is free.  (The producer stages nothing: its lane 0
-    // may stall issuing copies, and the consumers must not wait for that before
-    // converting the activations.)
-    const int nst0 = job_stages(0);
-    const int early = min(min(nst0, a.NS), a.early_w);  // never more than the ring holds
-    if (lane == 0)
-      for (int st = 0; st < early; ++st) issue(0, st, st);
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (lane == 0) mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * J0.K * 2);
-    __syncwarp();
-    if (lane < a.M)
-      bulk_g2s(xs + lane * J0.tok_stride, xg + static_cast<int64_t>(lane) * J0.K, static_cast<uint32_t>(J0.K) * 2,
-               xbar);
+    // Every stage of every matmul in order, each as soon as its ring slot is
+    // free.  The weights are not written by a kernel this one may overlap (the
+    // caller's promise for programmatic dependent launches), so the producer
+    // does not wait for the kernel before; the activations are loaded by the
+    // consumers, outside the copy engine, so they never queue behind weights.
     if (lane == 0) {
-      *x_issued = 1;
-      int gst = early;
+      int gst = 0;
       bool ok = true;
       for (int jx = 0; jx < a.njobs && ok; ++jx) {
-        const int nstj = jx == 0 ? nst0 : job_stages(jx);
-        for (int st = jx == 0 ? early : 0; st < nstj; ++st, ++gst) {
+        const Job jb = job_of(jx);
+        int64_t q0, q1;
+        cta_rows(jx, q0, q1);
+        const int nstj = job_stages(jx);
+        for (int st = 0; st < nstj; ++st, ++gst) {
           const int s = gst % a.NS;
           if (gst >= a.NS &&
               !mbar_wait(&empty[s], ((gst / a.NS) - 1) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim)) {
             ok = false;
             break;
           }
-          issue(jx, st, gst);
+          issue(jx, jb, q0, q1, st, gst);
         }
       }
       *issued_ctr = gst;
@@ -489,13 +478,16 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     __syncwarp();
   } else {
 
-  // ---- consumers stage the activations in place: item = (token, group, lane t).
-  // A group's raw bf16 and its staged digits occupy the same 2G bytes; the four
-  // lanes of a group read all their raw values before any of them writes.
+  // ---- consumers stage the activations: item = (token, group, lane t).  The
+  // raw bf16 values come straight from global memory (plain loads: the
+  // activations of a later matmul were written by other CTAs of this launch,
+  // made visible by the grid barrier), the digits go to shared memory.
   const int ctid = tid - 32, cthreads = a.W * 32;
   auto stage_acts = [&](int jx) {
-    const Job &Jb = a.job[jx];
-    mbar_wait(xbar, jx & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim);
+    const Job Jb = job_of(jx);
+    // x of the first matmul may be the output of the kernel this one overlaps
+    if (jx == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+    const __nv_bfloat16 *xsrc = (a.cta_per_tok > 0) ? xg : Jb.x;
     const int items = a.M * Jb.Gn * 4;  // a multiple of 4, so the 4 items of a group share one quad of lanes
     // Each thread takes kStageItems items per round, processed side by side:
     // the rounds are latency-bound chains (load, reduce across the quad, store).
@@ -513,10 +505,11 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
         const int mg = ii >> 2;
         mq[j] = mg / Jb.Gn;
         gq[j] = mg - mq[j] * Jb.Gn;
-        const uint8_t *src = xs + mq[j] * Jb.tok_stride + (gq[j] * G + Span::start(tq[j])) * 2;
+        const uint4 *src = reinterpret_cast<const uint4 *>(xsrc + static_cast<int64_t>(mq[j]) * Jb.K + gq[j] * G +
+                                                           Span::start(tq[j]));
 #pragma unroll
         for (int v = 0; v < SL / 8; ++v) {
-          const uint4 q = *reinterpret_cast<const uint4 *>(src + 16 * v);
+          const uint4 q = act[j] ? src[v] : make_uint4(0u, 0u, 0u, 0u);
           raw[j][4 * v] = q.x;
           raw[j][4 * v + 1] = q.y;
           raw[j][4 * v + 2] = q.z;
@@ -643,22 +636,17 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   // Every consumer warp walks every matmul, also after a failed wait (then
   // without taking units), so that all of them meet at the named barriers.
   for (int jx = 0; jx < a.njobs; ++jx) {
-  const Job &Jb = a.job[jx];
+  const Job Jb = job_of(jx);
   if (jx > 0) {
     // Every unit of matmul jx - 1 in this CTA is done (its outputs stored);
     // once every CTA is that far, the activations of matmul jx may be read.
     asm volatile("bar.sync 1, %0;" ::"r"(cthreads) : "memory");
     if (ctid == 0) {
       for (int b = 0; b < a.red_bufs; ++b) red_ready[b] = red_done[b] = 0;  // tile numbers restart
-      if (grid_barrier(a.gbar, gridDim.x, abort_flag, wlim)) {
-        asm volatile("fence.proxy.async.global;" ::: "memory");  // the copy below reads other CTAs' stores
-        mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(a.M) * Jb.K * 2);
-        for (int m = 0; m < a.M; ++m)
-          bulk_g2s(xs + m * Jb.tok_stride, Jb.x + static_cast<int64_t>(m) * Jb.K, static_cast<uint32_t>(Jb.K) * 2,
-                   xbar);
-        *x_issued = jx + 1;
-      }
+      grid_barrier(a.gbar, gridDim.x, abort_flag, wlim);
     }
+    asm volatile("bar.sync 1, %0;" ::"r"(cthreads) : "memory");  // ... and this CTA knows it
+    __threadfence();
     stage_acts(jx);
     if (*abort_flag) run = false;
   }
@@ -1015,7 +1003,6 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   __syncthreads();
   if (tid == 0 && *abort_flag) {
     const int issued = *issued_ctr;
-    if (*x_issued > 0) mbar_drain(xbar, (*x_issued - 1) & 1);
     for (int j = max(0, issued - a.NS); j < issued; ++j) mbar_drain(&full[j % a.NS], (j / a.NS) & 1);
   }
 }
@@ -1138,7 +1125,6 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
     if (units % c == 0 && kRows * 8 * G * c * bits / 8 <= stage_target && (!even_units || c % 2 == 0)) u = c;
   const int64_t Kc = 8 * G * u, nch = K / Kc, gpc = Kc / G;
   Args &a = pl.a;
-  a.early_w = 0;
   a.njobs = 1;
   a.gbar = nullptr;
   a.experts = nullptr;
@@ -1250,7 +1236,6 @@ static cudaError_t launch(const Plan &pl_one, const Plan *dual, const Maps &mp, 
     if (2 * regs * dual->threads <= 65536) use = dual;
   }
   Plan pl = *use;
-  pl.a.early_w = overlap ? (use == dual ? pl.a.NS : kEarlyStages) : 0;
   pl.a.wait_cycles = g_wait_limit.load(std::memory_order_relaxed);
   pl.a.stall = g_wait_stall.load(std::memory_order_relaxed) ? 1 : 0;
   static thread_local int cached_dev = -1;
@@ -1351,7 +1336,6 @@ template <int BITS, int G, int MP>
 static cudaError_t launch_seq(const Plan &pl_in, const JobMaps<kSeqMax> &mp, bool overlap, cudaStream_t stream) {
   auto kern = qmv_tc_kernel<BITS, G, MP, 0, kSeqMax>;
   Plan pl = pl_in;
-  pl.a.early_w = overlap ? kEarlyStages : 0;
   pl.a.wait_cycles = g_wait_limit.load(std::memory_order_relaxed);
   pl.a.stall = g_wait_stall.load(std::memory_order_relaxed) ? 1 : 0;
   static thread_local int cached_dev = -1;
