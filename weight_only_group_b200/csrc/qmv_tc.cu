@@ -78,6 +78,9 @@ namespace tc {
 #ifndef AQ_QMV_MAX_CONSUMERS
 #define AQ_QMV_MAX_CONSUMERS 12
 #endif
+#ifndef AQ_QMV_INFLIGHT
+#define AQ_QMV_INFLIGHT 6
+#endif
 #ifndef AQ_QMV_STAGE_TARGET
 #define AQ_QMV_STAGE_TARGET (16 * 1024)
 #endif
@@ -89,6 +92,11 @@ constexpr int kDualConsumers = 8;       // consumer warps of such a CTA
 constexpr int kDualMinStages = 4;
 constexpr int kUnitCodes = 1 << 20;     // codes of a row a work unit covers at least (where the stage allows)
 constexpr int kMaxStages = 16;
+// Weight stages the producer keeps in flight (issued, not yet landed).  Enough
+// to cover HBM latency at an SM's share of the bandwidth; more only lengthens
+// the queue that every other load of the SM (activations, barrier traffic)
+// waits behind.
+constexpr int kInflight = AQ_QMV_INFLIGHT;
 constexpr int kStageTarget = AQ_QMV_STAGE_TARGET;  // packed bytes of one stage we aim for (<= 1 KB per row)
 constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
 constexpr int kStageItems = 2;           // activation staging items per thread per round          // weight stages issued before the previous kernel completes (overlap mode)
@@ -302,26 +310,33 @@ struct Args {
 // is the generation; the last arrival resets the count and advances the
 // generation, so the pair is ready for the next barrier and the next launch.
 // Bounded: false after `limit` cycles (fault bit set, abort raised).
+AQ_DEVICE unsigned ld_acquire_gpu(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+AQ_DEVICE unsigned atom_add_acq_rel_gpu(unsigned *p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 AQ_DEVICE bool grid_barrier(unsigned *gbar, unsigned nblocks, volatile int *abort_flag, long long limit) {
-  volatile unsigned *gen = gbar + 1;
-  const unsigned g0 = *gen;
-  __threadfence();
-  if (atomicAdd(gbar, 1u) == nblocks - 1) {
+  const unsigned g0 = ld_acquire_gpu(gbar + 1);
+  // release: this CTA's outputs (ordered before by the CTA barrier) go with the arrival
+  if (atom_add_acq_rel_gpu(gbar, 1u) == nblocks - 1) {
     atomicExch(gbar, 0u);
-    __threadfence();
-    atomicAdd(gbar + 1, 1u);
+    atom_add_acq_rel_gpu(gbar + 1, 1u);
     return true;
   }
   const long long t0 = clock64();
-  while (*gen == g0) {
+  while (ld_acquire_gpu(gbar + 1) == g0) {
     if (*abort_flag || clock64() - t0 > limit) {
       atomicOr(&g_qmv_tc_fault, kFaultQmvWait);
       *abort_flag = 1;
       return false;
     }
-    __nanosleep(128);
+    __nanosleep(64);
   }
-  __threadfence();
   return true;
 }
 
@@ -467,6 +482,14 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
           const int s = gst % a.NS;
           if (gst >= a.NS &&
               !mbar_wait(&empty[s], ((gst / a.NS) - 1) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim)) {
+            ok = false;
+            break;
+          }
+          // the stage kInflight back has landed (its slot is issued again only
+          // NS > kInflight stages later, so the phase waited for is current)
+          const int back = gst - kInflight;
+          if (back >= 0 && kInflight < a.NS &&
+              !mbar_wait(&full[back % a.NS], (back / a.NS) & 1, abort_flag, &g_qmv_tc_fault, kFaultQmvWait, wlim)) {
             ok = false;
             break;
           }
