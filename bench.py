@@ -389,6 +389,8 @@ def compact_sections(sec):
         out["small_m_GBps"] = {k: v["weight_GBps"] for k, v in sec["qmv_small_m"]["curve"].items()}
     if "qmv_bits_group_sweep" in sec:
         out["sweep_GBps"] = {k: v["weight_GBps"] for k, v in sec["qmv_bits_group_sweep"]["points"].items()}
+    if "decode_sequence" in sec:
+        out["decode_sequence_GBps"] = {k: v["weight_GBps"] for k, v in sec["decode_sequence"].items()}
     if "qmm_prefill" in sec:
         out["qmm_prefill"] = {k: [v["TFLOP/s"], v["frac_of_burst"]] for k, v in sec["qmm_prefill"]["points"].items()}
         out["qmm_prefill_unit"] = "[TFLOP/s, fraction of the measured burst bf16 peak]"
@@ -420,10 +422,12 @@ def timed_graph(torch, stream, fn, reps_inner, reps_outer):
 
 def measure_sections(args, aq, torch, dev, stream, peaks):
     out = {}
-    want = set(args.sections.split(",")) if args.sections != "all" else {"shapes", "qmm", "curve", "sweep", "quant",
-                                                                         "embed", "gather", "mxfp4"}
+    want = set(args.sections.split(",")) if args.sections != "all" else {"shapes", "seq", "qmm", "curve", "sweep",
+                                                                         "quant", "embed", "gather", "mxfp4"}
     if "shapes" in want:
         out.update(section_decode_shapes(args, aq, torch, dev, stream, peaks))
+    if "seq" in want:
+        out.update(section_decode_sequence(args, aq, torch, dev, stream, peaks))
     if "qmm" in want:
         out.update(section_qmm(args, aq, torch, dev, stream, peaks))
     if "curve" in want:
@@ -624,6 +628,40 @@ def section_decode_shapes(args, aq, torch, dev, stream, peaks):
     return {"decode_shapes": out}
 
 
+def section_decode_sequence(args, aq, torch, dev, stream, peaks):
+    """The decode step's three linears as one aq_matmul_sequence launch (the
+    weights of each linear stream while the one before finishes; a grid barrier
+    before each linear's activations), against three launches, over rotating
+    resident weight sets larger than L2."""
+    base = []
+    for si, (K, N) in enumerate(DECODE_SHAPES):
+        w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 2 + si)).to(dev)
+        base.append(aq.aq_quantize(w, G, BITS))
+        del w
+    copies = max(2, -(-2 * L2_BYTES // STEP_BYTES) + 1)
+    out = {}
+    for M in (1, 2, 4):
+        sets = []
+        for c in range(copies):
+            sets.append([(tuple(t.clone() for t in base[si]) if c else base[si]) +
+                         (synth.activations(M, K, 7 + si).to(dev), torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+                         for si, (K, N) in enumerate(DECODE_SHAPES)])
+
+        def three(i):
+            for (p, s, b, x, y) in sets[i % copies]:
+                aq.aq_matmul(x, p, s, b, G, BITS, out=y, overlap_previous=True)
+
+        def seq(i):
+            aq.aq_matmul_sequence([(x, p, s, b, y) for (p, s, b, x, y) in sets[i % copies]], G, BITS,
+                                  overlap_previous=True)
+        for name, fn in (("three_launches", three), ("sequence", seq)):
+            ms = timed_graph(torch, stream, fn, copies * 4, 10)
+            out[f"M{M}_{name}"] = {"us": round(ms * 1e3, 2), "weight_GBps": round(STEP_BYTES / (ms * 1e-3) / 1e9, 1)}
+        del sets
+        torch.cuda.empty_cache()
+    return {"decode_sequence": out}
+
+
 def section_curve(args, aq, torch, dev, stream, peaks):
     out = {}
     # ---- QMV small-M curve on K=4096, N=14336 (rotating weight copies)
@@ -787,7 +825,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--qmm-reps", type=int, default=20)
     ap.add_argument("--sections", default="all",
-                    help="all | none | comma list of shapes,qmm,curve,sweep,quant,embed,gather,mxfp4 (secondary measurements)")
+                    help="all | none | comma list of shapes,seq,qmm,curve,sweep,quant,embed,gather,mxfp4 (secondary measurements)")
     ap.add_argument("--no-sections", dest="sections", action="store_const", const="none")
     ap.add_argument("--shard", action="store_true",
                     help="with N > 1 ranks: split W along N (one all-gather of y per step) instead of replicas")

@@ -28,8 +28,9 @@
  * Ownership: every pointer argument is DEVICE memory, allocated, owned and freed
  * by the caller.  Only the tensor-core matmul path (large M) needs temporary
  * device memory (a workspace: the activations converted to fp16); aq_matmul and
- * aq_matmul_with take it from CUDA's stream-ordered allocator (cudaMallocAsync /
- * cudaFreeAsync on `stream`), aq_matmul_ws takes it from the caller, and
+ * aq_matmul_with take it, stream-ordered on `stream`, from a memory pool the
+ * library creates per device and keeps (it holds the largest workspace in use
+ * at once until the process exits), aq_matmul_ws takes it from the caller, and
  * aq_matmul_with(AQ_KERNEL_QMM_NOWS) and aq_matmul_qmm_static need none from
  * anybody at call time.
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
@@ -246,7 +247,7 @@ aq_status aq_matmul_qmm_static(const uint16_t *x_bf16, int64_t M, int64_t K,
  * return AQ_ERR_UNSUPPORTED when M > 8 or the shared-memory staging of x does
  * not fit; AQ_KERNEL_QMM and AQ_KERNEL_QMM_NOWS return AQ_ERR_UNSUPPORTED when
  * K*bits is not a multiple of 128.  AQ_KERNEL_QMM takes its workspace from
- * the stream-ordered allocator (cudaMallocAsync on `stream`); AQ_KERNEL_QMM_NOWS
+ * the library's stream-ordered pool (see Ownership above); AQ_KERNEL_QMM_NOWS
  * allocates nothing (each token row's power-of-two scale is kept, until the
  * epilogue overwrites it, in bytes of y's own output tile). */
 aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x_bf16, int64_t M, int64_t K,
@@ -301,7 +302,7 @@ aq_status aq_gather_matmul(const uint16_t *x_bf16, int64_t T, int64_t K, const u
  * sizes), and the rows are scattered back.  The host reads the E per-expert
  * counts once, so the call synchronizes its stream (it cannot be captured in a
  * CUDA graph).  Workspace (offsets, positions, x and y in expert order, the QMM
- * workspace) comes from the stream-ordered allocator.  Shapes: as aq_matmul for
+ * workspace) comes from the library's stream-ordered pool.  Shapes: as aq_matmul for
  * every segment size, N a multiple of 8, each expert's packed/scale/bias block a
  * multiple of 16 bytes, E <= 16384 (others -> AQ_ERR_UNSUPPORTED or
  * AQ_ERR_INVALID_ARG).  Accuracy as aq_matmul.  Source: metalworking "MLX

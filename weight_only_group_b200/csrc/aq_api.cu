@@ -1,5 +1,7 @@
 // C ABI entry points: argument validation, per-shape dispatch, launches.
 // Method and layouts: see include/aq.h.
+#include <cuda.h>
+
 #include <algorithm>
 #include <mutex>
 #include <vector>
@@ -145,6 +147,66 @@ namespace aq {
 aq_status api_from_cuda(cudaError_t e) { return from_cuda(e); }
 aq_status api_check_device() { return check_device(); }
 }  // namespace aq
+
+// Workspace of the calls that need one comes from a stream-ordered memory pool
+// of the library's own, one per device (and context), which keeps its memory
+// between calls.  The device's default pool hands memory back to the system at
+// every synchronisation (release threshold 0): measured on B200, a prefill call
+// after a synchronisation then spent up to tens of milliseconds mapping its
+// workspace again.  The pool holds the largest workspace in use at once until
+// the process exits.
+namespace {
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CtxGetCurrentFn ws_ctx_get_current() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+cudaError_t ws_pool(cudaMemPool_t *out) {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDev] = {};
+  static CUcontext owners[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if ((e = cudaFree(nullptr)) != cudaSuccess) return e;  // the device's context exists
+  const CtxGetCurrentFn get = ws_ctx_get_current();
+  CUcontext ctx = nullptr;
+  if (get == nullptr || get(&ctx) != CUDA_SUCCESS) return cudaErrorNotSupported;
+  std::lock_guard<std::mutex> lock(mu);
+  if (pools[dev] == nullptr || owners[dev] != ctx) {  // first use, or the context was recreated
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess) return e;
+    uint64_t keep = ~uint64_t(0);
+    if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) return e;
+    pools[dev] = pool;
+    owners[dev] = ctx;
+  }
+  *out = pools[dev];
+  return cudaSuccess;
+}
+
+cudaError_t ws_alloc(void **p, size_t bytes, cudaStream_t s) {
+  cudaMemPool_t pool = nullptr;
+  cudaError_t e = ws_pool(&pool);
+  if (e != cudaSuccess) return e;
+  return cudaMallocFromPoolAsync(p, bytes, pool, s);
+}
+}  // namespace
 
 extern "C" {
 
@@ -302,9 +364,9 @@ aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t
   const size_t need = workspace_for(kernel, M, K);
   if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream);
   if ((st = check_device()) != AQ_OK) return st;
-  // workspace from the stream-ordered allocator, released on the same stream
+  // workspace from the library's stream-ordered pool, released on the same stream
   void *ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, need, stream);
+  cudaError_t e = ws_alloc(&ws, need, stream);
   if (e != cudaSuccess) return from_cuda(e);
   st = matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, ws, stream);
   e = cudaFreeAsync(ws, stream);
@@ -411,7 +473,7 @@ aq_status aq_gather_matmul_grouped(const uint16_t *x, int64_t T, int64_t K, cons
   const size_t b_x = round16(static_cast<size_t>(T) * K * 2), b_y = round16(static_cast<size_t>(T) * N * 2);
   const size_t b_ws = round16(aq::qmm_workspace_bytes(T, K));
   uint8_t *ws = nullptr;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&ws), b_off + b_pos + b_x + b_y + b_ws, stream);
+  cudaError_t e = ws_alloc(reinterpret_cast<void **>(&ws), b_off + b_pos + b_x + b_y + b_ws, stream);
   if (e != cudaSuccess) return from_cuda(e);
   int32_t *offsets = reinterpret_cast<int32_t *>(ws);
   int32_t *pos = reinterpret_cast<int32_t *>(ws + b_off);
