@@ -35,8 +35,9 @@
  * anybody at call time.
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  * stream); outputs are valid once the stream reaches the call.  The one
- * exception is aq_gather_matmul_grouped, which reads per-expert counts on the
- * host and so synchronizes its stream.
+ * exception is aq_gather_matmul_grouped with more than 256 experts (or K*bits
+ * not a multiple of 128), which reads per-expert counts on the host and so
+ * synchronizes its stream.
  *
  * Entry points beyond quantize / dequantize / matmul, each documented below:
  *   aq_quantize_mse           range-search quantizer (same format)
@@ -297,11 +298,14 @@ aq_status aq_gather_matmul(const uint16_t *x_bf16, int64_t T, int64_t K, const u
  * dequant(W[experts[t]])^T, a zero row and AQ_FAULT_BAD_INDEX for an id outside
  * [0, E)), computed by grouping the tokens by expert so that each expert's
  * weights are multiplied once against all of its tokens: a routing kernel
- * orders the tokens by expert, x rows are gathered into that order, each
- * expert's rows go through aq_matmul's per-shape kernels (QMM at prefill
- * sizes), and the rows are scattered back.  The host reads the E per-expert
- * counts once, so the call synchronizes its stream (it cannot be captured in a
- * CUDA graph).  Workspace (offsets, positions, x and y in expert order, the QMM
+ * orders the tokens by expert, x rows are gathered into that order, and the
+ * rows are scattered back after the matmul.  With E <= 256 and K*bits a
+ * multiple of 128 the matmul is ONE tensor-core launch over every expert's
+ * segment, whose tile count the kernel reads from the device-side segment
+ * offsets: the call is asynchronous and can be captured in a CUDA graph.
+ * Otherwise each expert's rows go through aq_matmul's per-shape kernels; the
+ * host then reads the E per-expert counts once, so the call synchronizes its
+ * stream (and cannot be captured).  Workspace (offsets, positions, x and y in expert order, the QMM
  * workspace) comes from the library's stream-ordered pool.  Shapes: as aq_matmul for
  * every segment size, N a multiple of 8, each expert's packed/scale/bias block a
  * multiple of 16 bytes, E <= 16384 (others -> AQ_ERR_UNSUPPORTED or

@@ -25,6 +25,10 @@ void set_qmv_tc_wait_limit(long long cycles);
 void set_qmv_tc_wait_stall(bool on);
 cudaError_t read_and_clear_embed_fault(uint32_t *word);
 bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
+constexpr int64_t kQmmGroupMaxE = 256;  // experts of one grouped prefill launch at most
+cudaError_t launch_qmm_grouped(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed,
+                               const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
+                               const int32_t *offsets, uint16_t *y, void *ws, cudaStream_t s);
 bool qmv_tc_seq_supported(int n, const int64_t *N, const int64_t *K, int64_t M, int G, int bits);
 cudaError_t launch_qmv_tc_seq(int n, const SeqCall *calls, int64_t M, int G, int bits, uint32_t flags, cudaStream_t s);
 cudaError_t launch_gather_tc(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed, const uint16_t *scales,
@@ -179,10 +183,13 @@ cudaError_t ws_pool(cudaMemPool_t *out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  if ((e = cudaFree(nullptr)) != cudaSuccess) return e;  // the device's context exists
   const CtxGetCurrentFn get = ws_ctx_get_current();
   CUcontext ctx = nullptr;
   if (get == nullptr || get(&ctx) != CUDA_SUCCESS) return cudaErrorNotSupported;
+  if (ctx == nullptr) {  // the runtime has not made the device's context current yet
+    if ((e = cudaFree(nullptr)) != cudaSuccess) return e;
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorNotSupported;
+  }
   std::lock_guard<std::mutex> lock(mu);
   if (pools[dev] == nullptr || owners[dev] != ctx) {  // first use, or the context was recreated
     cudaMemPoolProps props = {};
@@ -201,8 +208,14 @@ cudaError_t ws_pool(cudaMemPool_t *out) {
 }
 
 cudaError_t ws_alloc(void **p, size_t bytes, cudaStream_t s) {
+  // in a stream capture the allocation becomes a graph memory node: leave it to
+  // the graph's own allocator (and create no pool while capturing)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return e;
+  if (cap != cudaStreamCaptureStatusNone) return cudaMallocAsync(p, bytes, s);
   cudaMemPool_t pool = nullptr;
-  cudaError_t e = ws_pool(&pool);
+  e = ws_pool(&pool);
   if (e != cudaSuccess) return e;
   return cudaMallocFromPoolAsync(p, bytes, pool, s);
 }
@@ -480,8 +493,19 @@ aq_status aq_gather_matmul_grouped(const uint16_t *x, int64_t T, int64_t K, cons
   uint16_t *xs = reinterpret_cast<uint16_t *>(ws + b_off + b_pos);
   uint16_t *ys = reinterpret_cast<uint16_t *>(ws + b_off + b_pos + b_x);
   void *qws = ws + b_off + b_pos + b_x + b_y;
-  std::vector<int32_t> off(static_cast<size_t>(E + 2));
   st = from_cuda(aq::launch_gather_route(experts, T, E, offsets, pos, stream));
+  if (E <= aq::kQmmGroupMaxE && aq::qmm_supports(T, N, K, G, bits)) {
+    // one matmul launch over every expert's segment, read from the device
+    // offsets: nothing goes back to the host
+    if (st == AQ_OK) st = from_cuda(aq::launch_gather_rows(x, T, K, pos, xs, stream));
+    if (st == AQ_OK)
+      st = from_cuda(aq::launch_qmm_grouped(xs, T, K, packed, scales, biases, E, N, G, bits, offsets, ys, qws, stream));
+    if (st == AQ_OK) st = from_cuda(aq::launch_scatter_rows(ys, T, N, pos, experts, E, y, stream));
+    e = cudaFreeAsync(ws, stream);
+    if (st == AQ_OK && e != cudaSuccess) st = from_cuda(e);
+    return st;
+  }
+  std::vector<int32_t> off(static_cast<size_t>(E + 2));
   if (st == AQ_OK)
     st = from_cuda(cudaMemcpyAsync(off.data(), offsets, off.size() * 4, cudaMemcpyDeviceToHost, stream));
   if (st == AQ_OK) st = from_cuda(cudaStreamSynchronize(stream));

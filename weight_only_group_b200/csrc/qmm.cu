@@ -71,6 +71,9 @@ AQ_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_fla
 // ---------------------------------------------------------------------------
 // Tile configuration
 // ---------------------------------------------------------------------------
+constexpr int kGroupMaxE = 256;  // experts of a grouped launch at most (their tables live in shared memory)
+constexpr int kGroupTabBytes = (2 * kGroupMaxE + 4) * 4;
+
 template <int BITS, int BN>
 struct Cfg {
   static constexpr int BK = (BITS == 3) ? 128 : 64;         // K per stage (elements)
@@ -82,7 +85,7 @@ struct Cfg {
   static constexpr int A_COLS = BK / 2;                     // TMEM columns per A stage (2 bf16 per column)
   static constexpr int A_COL0 = BN;                         // first TMEM column of the A stages
   static constexpr int STAGES = std::min(std::min(6, SMEM_BUDGET / STAGE_BYTES), (kTmemCols - A_COL0) / A_COLS);
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + kGroupTabBytes;
   static_assert(STAGES >= 2, "not enough shared memory for two stages");
   static_assert(A_COL0 + STAGES * A_COLS <= kTmemCols, "TMEM budget");
   static_assert(BN <= 256 && BN % 16 == 0, "MMA N");
@@ -98,6 +101,17 @@ struct Params {
   int M, N, K, G, Gn;
   int m_tiles, n_tiles;
   int n_fastest;  // tile order: W-row tiles fastest (else token tiles fastest)
+  // grouped mode (E experts > 0): the M token rows are E consecutive segments,
+  // segment e = rows [offsets[e], offsets[e+1]) multiplied by expert e (rows
+  // e*N .. e*N+N-1 of the stacked W); offsets live in device memory
+  const int32_t *offsets;
+  int E;
+};
+
+// One tile of a launch: its first token row and first W row in the maps, the
+// W row within the weight matrix (or expert), and the end of its token rows.
+struct TileRef {
+  int m0, n0, wrow, mend;
 };
 
 // Tile t's first token and first W row.  Token tiles fastest keeps a W tile in
@@ -115,6 +129,30 @@ AQ_DEVICE void tile_origin(const Params &prm, int tile, int bn, int wr, int &m0,
   }
 }
 
+// Tile t of a launch.  Grouped mode: tiles run over (segment tile, W tile)
+// pairs, W tiles fastest; seg[] holds the E + 1 segment offsets and mtp[] the
+// prefix sums of each segment's token tiles.
+AQ_DEVICE TileRef tile_at(const Params &prm, const int *seg, const int *mtp, int tile, int bn) {
+  TileRef r;
+  if (prm.E == 0) {
+    tile_origin(prm, tile, bn, 128, r.m0, r.n0);
+    r.wrow = r.n0;
+    r.mend = prm.M;
+    return r;
+  }
+  const int nt = tile % prm.n_tiles, mg = tile / prm.n_tiles;
+  int lo = 0, hi = prm.E - 1;  // the segment e with mtp[e] <= mg < mtp[e + 1]
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (mtp[mid] <= mg) lo = mid; else hi = mid - 1;
+  }
+  r.m0 = seg[lo] + (mg - mtp[lo]) * bn;
+  r.n0 = nt * 128;
+  r.wrow = lo * prm.N + r.n0;
+  r.mend = seg[lo + 1];
+  return r;
+}
+
 template <int BITS, int BN>
 __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant__ CUtensorMap x_map,
                                                           const __grid_constant__ CUtensorMap w_map, Params prm) {
@@ -129,10 +167,19 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
   uint64_t *acc_empty = acc_full + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *seg = reinterpret_cast<int *>(smem + S * C::STAGE_BYTES + 256);  // grouped: [E + 1] offsets
+  int *mtp = seg + kGroupMaxE + 2;                                     // grouped: [E + 1] tile prefix sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total_tiles = prm.m_tiles * prm.n_tiles;
   const int KB = (prm.K + C::BK - 1) / C::BK;
+  if (prm.E > 0 && threadIdx.x == 64) {  // warp 2 (otherwise idle) reads the segments
+    int run = 0;
+    for (int e = 0; e <= prm.E; ++e) {
+      seg[e] = __ldg(prm.offsets + e);
+      mtp[e] = run;
+      if (e < prm.E) run += (__ldg(prm.offsets + e + 1) - seg[e] + BN - 1) / BN;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -155,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = prm.E > 0 ? prm.n_tiles * mtp[prm.E] : prm.m_tiles * prm.n_tiles;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -164,8 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        int m0, n0;
-        tile_origin(prm, tile, BN, 128, m0, n0);
+        const TileRef tr = tile_at(prm, seg, mtp, tile, BN);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           const uint32_t r = it / S;
@@ -174,8 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
           uint8_t *ws = xs + C::X_BYTES;
           mbar_arrive_expect_tx(&full[s], C::X_BYTES + C::W_BYTES);
 #pragma unroll
-          for (int a = 0; a < C::BK / 64; ++a) tma_load_2d(xs + a * BN * 128, &x_map, &full[s], kb * C::BK + a * 64, m0);
-          tma_load_2d(ws, &w_map, &full[s], kb * C::BKW, n0);
+          for (int a = 0; a < C::BK / 64; ++a)
+            tma_load_2d(xs + a * BN * 128, &x_map, &full[s], kb * C::BK + a * 64, tr.m0);
+          tma_load_2d(ws, &w_map, &full[s], kb * C::BKW, tr.wrow);
         }
       }
       // drain: wait (bounded) until every issued load has landed
@@ -225,11 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
     uint32_t it0 = 0, t = 0;                    // stage counter at the start of the tile
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++t, it0 += KB) {
-      int m0, n0;
-      tile_origin(prm, tile, BN, 128, m0, n0);
-      const int n = n0 + row;
+      const TileRef tr = tile_at(prm, seg, mtp, tile, BN);
+      const int m0 = tr.m0;
+      const int n = tr.n0 + row;
       const bool row_ok = n < prm.N;
-      const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
+      const int64_t g_row = static_cast<int64_t>(row_ok ? tr.wrow + row : 0) * prm.Gn;
       // scales/biases (fp16 bits) of this thread's chunks, prefetched for this
       // warp's next two K blocks (its turns come every H blocks)
       auto load_sb = [&](int kb, uint16_t (&sc)[CH], uint16_t (&bi)[CH]) {
@@ -301,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int m = m0 + col + i;
-            if (m < prm.M)
+            if (m < tr.mend)
               prm.y[static_cast<int64_t>(m) * prm.N + n] =
                   __float2bfloat16_rn(__uint_as_float(v[i]) * __ldg(prm.row_scale + m));
           }
@@ -734,6 +782,8 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
       return cudaErrorInvalidValue;
   }
   Params prm;
+  prm.offsets = nullptr;
+  prm.E = 0;
   prm.scales = reinterpret_cast<const __half *>(scales);
   prm.biases = reinterpret_cast<const __half *>(biases);
   prm.row_scale = row_scale;
@@ -768,6 +818,78 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
   }
   const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
   const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, prm);
+  return cudaGetLastError();
+}
+
+// Grouped launch: x [T, K] holds E segments of token rows (device offsets
+// [E + 1]); segment e is multiplied by expert e of the stacked W [E*N, K], all
+// in one persistent launch whose tile count each CTA reads from the offsets.
+template <int BITS, int BN>
+cudaError_t launch_grouped_t(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed, const uint16_t *scales,
+                             const uint16_t *biases, int64_t E, int64_t N, int G, const int32_t *offsets, uint16_t *y,
+                             void *workspace, cudaStream_t stream) {
+  using C = Cfg<BITS, BN>;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  __half *x16 = reinterpret_cast<__half *>(workspace);
+  float *row_scale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + ((T * K * 2 + 255) / 256) * 256);
+  x_to_f16_rows_kernel<BITS><<<static_cast<unsigned>(T), kPrepThreads, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
+  CUtensorMap x_map, w_map;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(BN)};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const int64_t P = K * BITS / 32;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(E * N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(P) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(C::BKW), 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(packed), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  Params prm;
+  prm.offsets = offsets;
+  prm.E = static_cast<int>(E);
+  prm.scales = reinterpret_cast<const __half *>(scales);
+  prm.biases = reinterpret_cast<const __half *>(biases);
+  prm.row_scale = row_scale;
+  prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  prm.M = static_cast<int>(T);
+  prm.N = static_cast<int>(N);
+  prm.K = static_cast<int>(K);
+  prm.G = G;
+  prm.Gn = static_cast<int>(K / G);
+  prm.m_tiles = 0;  // from the offsets, on the device
+  prm.n_tiles = static_cast<int>((N + 127) / 128);
+  prm.n_fastest = 1;
+  auto kern = qmm_kernel<BITS, BN>;
+  static thread_local int cached_dev = -1;
+  static thread_local int sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
+      return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  // at most ceil(T / BN) + E token tiles (each segment adds at most one partial tile)
+  const int64_t bound = static_cast<int64_t>(prm.n_tiles) * ((T + BN - 1) / BN + E);
+  const int grid = static_cast<int>(std::min<int64_t>(bound, sms));
   kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, prm);
   return cudaGetLastError();
 }
@@ -807,6 +929,8 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
       return cudaErrorInvalidValue;
   }
   Params prm;
+  prm.offsets = nullptr;
+  prm.E = 0;
   prm.scales = reinterpret_cast<const __half *>(scales);
   prm.biases = reinterpret_cast<const __half *>(biases);
   prm.row_scale = row_scale;
@@ -842,16 +966,13 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   return cudaGetLastError();
 }
 
-// Tile shape.  Measured on B200 (4-bit, G = 64): both kernels take about
-// 750-800 SM cycles per 64-deep K block at every token-tile width, more than
-// the tensor work of the block (2 cycles per token column), so what decides
-// is how many multiply-adds a block carries and how well the tiles fill the
-// SMs.  The CTA pair (256 x 256 tiles) carries the most per block and frees
-// half of each CTA's L2 traffic; it was as fast as the single CTA or faster
-// (up to 1.3x at K = 14336) wherever its tiles filled at least one wave of
-// pairs.  With fewer tiles than pairs, one CTA per tile: the width that best
-// trades wave fill against bytes moved per multiply-add (the x16 slice, BN x
-// BK fp16, plus the packed W slice).
+// Tile shape.  Measured on B200 (4-bit, G = 64, TFLOP/s, pair / one CTA at
+// 256 / one CTA at 128 tokens): M = 512, 2048, 8192 at K = 4096, N = 14336:
+// 532/540/344, 742/744/461, 901/895/510; at K = 14336, N = 4096: 501/383/485,
+// 1016/763/571, 1197/946/611.  The CTA pair carries the most multiply-adds per
+// staged byte and is never slower, so every M > 128 takes it.  Smaller M: one
+// CTA per tile, the width that best trades wave fill against bytes moved per
+// multiply-add (the x16 slice, BN x BK fp16, plus the packed W slice).
 enum Shape { kPair256 = 0, kOne256 = 1, kOne128 = 2, kOne64 = 3 };
 
 template <int BITS>
@@ -859,8 +980,7 @@ int pick_shape(int64_t M, int64_t N, int sms) {
 #ifdef AQ_QMM_FORCE_SHAPE  // build-time override (0..3 as in Shape; else choose)
   if (AQ_QMM_FORCE_SHAPE >= 0 && AQ_QMM_FORCE_SHAPE <= 3) return AQ_QMM_FORCE_SHAPE;
 #endif
-  const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-  if (M > 128 && pair_tiles >= std::max(1, sms / 2)) return kPair256;
+  if (M > 128) return kPair256;
   auto score = [&](int64_t bn, int64_t bytes) {
     const int64_t t = ((M + bn - 1) / bn) * ((N + 127) / 128);
     const int64_t waves = (t + sms - 1) / sms;
@@ -895,6 +1015,31 @@ cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
 }
 
 }  // namespace qmm
+
+// Grouped prefill (see launch_grouped_t): BN by the mean segment length.
+cudaError_t launch_qmm_grouped(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed,
+                               const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
+                               const int32_t *offsets, uint16_t *y, void *ws, cudaStream_t s) {
+  if (E < 1 || E > qmm::kGroupMaxE) return cudaErrorInvalidValue;
+  const int64_t mean = (T + E - 1) / E;
+  const int bn = mean <= 96 ? 64 : mean <= 384 ? 128 : 256;
+#define AQ_GROUPED(B, N_)                                                                                          \
+  case N_: return qmm::launch_grouped_t<B, N_>(x, T, K, packed, scales, biases, E, N, G, offsets, y, ws, s);
+#define AQ_GROUPED_BITS(B)                                                                                         \
+  switch (bn) {                                                                                                    \
+    AQ_GROUPED(B, 64)                                                                                              \
+    AQ_GROUPED(B, 128)                                                                                             \
+    default: return qmm::launch_grouped_t<B, 256>(x, T, K, packed, scales, biases, E, N, G, offsets, y, ws, s);    \
+  }
+  switch (bits) {
+    case 2: AQ_GROUPED_BITS(2)
+    case 3: AQ_GROUPED_BITS(3)
+    case 4: AQ_GROUPED_BITS(4)
+    default: AQ_GROUPED_BITS(8)
+  }
+#undef AQ_GROUPED_BITS
+#undef AQ_GROUPED
+}
 
 bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits) {
   (void)G;
