@@ -313,8 +313,8 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "traffic_unit": "DRAM bytes read + written per decode step (3 launches), from ncu",
                 "peak_source": peaks["source"], "frac_of_8TBs_nominal": round(achieved / 8000.0, 4),
-                "kernel": ("qmv_tc_kernel<bits=4,G=64,MP=1> (mma.sync m16n8k32: u8 codes x 8-bit digits of "
-                           "16-bit fixed-point activations, int32 accumulate, fp32 fold; 3 launches per step)"),
+                "kernel": ("qmv_tc_kernel<bits=4,G=64,MP=1> (mma.sync m16n8k32: u8 codes x both signed-byte digit planes of "
+                           "16-bit fixed-point activations in one MMA, int32 accumulate, fp32 fold; 3 launches per step)"),
                 "algorithmic_bytes_per_step": STEP_BYTES}
     del graph
 
@@ -580,7 +580,11 @@ def section_qmm(args, aq, torch, dev, stream, peaks):
     dense peak (burst: the kernel is timed on its own, back to back)."""
     out = {}
     wcache = {}
-    for (M, K, N) in QMM_POINTS:
+    points = QMM_POINTS
+    if args.qmm_points:
+        want = {tuple(int(v) for v in t.split("x")) for t in args.qmm_points.split(",")}
+        points = [pt for pt in QMM_POINTS if pt in want]
+    for (M, K, N) in points:
         if (K, N) not in wcache:
             wcache.clear()
             torch.cuda.empty_cache()
@@ -824,6 +828,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--qmm-reps", type=int, default=20)
+    ap.add_argument("--qmm-points", default="",
+                    help="comma list of MxKxN prefill points to run (default: every point of the prefill workload)")
     ap.add_argument("--sections", default="all",
                     help="all | none | comma list of shapes,seq,qmm,curve,sweep,quant,embed,gather,mxfp4 (secondary measurements)")
     ap.add_argument("--no-sections", dest="sections", action="store_const", const="none")
