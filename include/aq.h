@@ -350,7 +350,7 @@ aq_status aq_mxfp4_dequantize(const uint32_t *packed, const uint8_t *scales, int
 aq_status aq_mxfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K,
                                   float *w_out, aq_stream_t stream);
 
-/* y[M, N] = x[M, K] @ dequant(W)^T (bf16 in and out, device) for decode,
+/* y[M, N] = x[M, K] @ dequant(W)^T (bf16 in and out, device).  Decode,
  * M <= 8, on the integer tensor cores: each code becomes the signed byte
  * 2 * e2m1(code), the activations enter as 16-bit fixed point per group (as in
  * aq_matmul's decode kernel) and the fold applies X / 2.  Supported shapes:
@@ -358,7 +358,14 @@ aq_status aq_mxfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales,
  * 0 or AQ_MATMUL_OVERLAP_PREVIOUS, as for aq_matmul_ex.  Accuracy as aq_matmul,
  * provided X / 2 times the activations' per-group power of two stays within
  * the fp32 range (true unless both the weights' scale and the activations are
- * within a few octaves of the fp32 limits). */
+ * within a few octaves of the fp32 limits).
+ * Prefill, M > 8: the tensor-core matmul of aq_matmul (tcgen05, fp16
+ * operands, fp32 accumulation): the codes are dequantized to fp16 on chip,
+ * each W row scaled by a power of two 2^-B chosen from its largest block scale
+ * so that every value of a group within 2^22 of that scale is exact (the
+ * epilogue multiplies by 2^B); smaller groups round as fp16 subnormals, below
+ * the matmul tolerance.  The activations' fp16 workspace comes from the
+ * library's pool; flags are then ignored. */
 aq_status aq_mxfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
                           const uint8_t *scales, int64_t N, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
 
@@ -387,13 +394,20 @@ aq_status aq_mxfp8_dequantize(const uint32_t *packed, const uint8_t *scales, int
 aq_status aq_mxfp8_dequantize_f32(const uint32_t *packed, const uint8_t *scales, int64_t N, int64_t K,
                                   float *w_out, aq_stream_t stream);
 
-/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device) for decode, M <= 8.  E4M3
+/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device).  Decode, M <= 8: E4M3
  * codes do not fit the integer MMA: each pair is widened to fp16x2 (exact) and
  * multiplied on the tensor cores (mma.sync m16n8k16, fp32 accumulate) against
  * the activations staged as fp16 x * 2^e per group (exact for |x| above 2^-14
  * of the group's largest); the fold applies X * 2^-e.  Supported: M <= 8,
  * N >= 16, K a multiple of 512 (others -> AQ_ERR_UNSUPPORTED).  flags: 0 or
- * AQ_MATMUL_OVERLAP_PREVIOUS.  Accuracy as aq_matmul. */
+ * AQ_MATMUL_OVERLAP_PREVIOUS.  Accuracy as aq_matmul.
+ * Prefill, M > 8: the tensor-core matmul of aq_matmul (tcgen05, fp16
+ * operands, fp32 accumulation): the codes are dequantized to fp16 on chip,
+ * each W row scaled by a power of two 2^-B chosen from its largest block scale
+ * so that every value of a group within 2^22 of that scale is exact (the
+ * epilogue multiplies by 2^B); smaller groups round as fp16 subnormals, below
+ * the matmul tolerance.  The activations' fp16 workspace comes from the
+ * library's pool; flags are then ignored. */
 aq_status aq_mxfp8_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
                           const uint8_t *scales, int64_t N, uint16_t *y_bf16, uint32_t flags, aq_stream_t stream);
 
@@ -428,14 +442,21 @@ aq_status aq_nvfp4_dequantize(const uint32_t *packed, const uint8_t *scales, con
 aq_status aq_nvfp4_dequantize_f32(const uint32_t *packed, const uint8_t *scales, const float *tensor_scale,
                                   int64_t N, int64_t K, float *w_out, aq_stream_t stream);
 
-/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device) for decode, M <= 8, on the
+/* y[M, N] = x[M, K] @ dequant(W)^T (bf16, device).  Decode, M <= 8, on the
  * integer tensor cores: one MMA K step spans two 16-weight groups, whose halves
  * feed two accumulator columns; each column is folded with its E4M3 scale and
  * the output multiplied by g.  One launch holds up to 4 tokens; M = 5..8 runs as
  * two launches (rows 0..3, then the rest), reading the weights twice.
  * Supported: M <= 8, N >= 16, K a multiple of 256 (others ->
  * AQ_ERR_UNSUPPORTED).  flags: 0 or AQ_MATMUL_OVERLAP_PREVIOUS (both launches).
- * Accuracy as aq_matmul. */
+ * Accuracy as aq_matmul.
+ * Prefill, M > 8: the tensor-core matmul of aq_matmul (tcgen05, fp16
+ * operands, fp32 accumulation): the codes are dequantized to fp16 on chip,
+ * each W row scaled by a power of two 2^-B chosen from its largest block scale
+ * so that every value of a group within 2^22 of that scale is exact (the
+ * epilogue multiplies by 2^B); smaller groups round as fp16 subnormals, below
+ * the matmul tolerance.  The activations' fp16 workspace comes from the
+ * library's pool; flags are then ignored.  The tensor scale g multiplies every output. */
 aq_status aq_nvfp4_matmul(const uint16_t *x_bf16, int64_t M, int64_t K, const uint32_t *packed,
                           const uint8_t *scales, const float *tensor_scale, int64_t N, uint16_t *y_bf16,
                           uint32_t flags, aq_stream_t stream);

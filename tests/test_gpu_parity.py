@@ -995,3 +995,54 @@ def test_matmul_sequence_wait_runs_out_cleanly():
     assert aq.aq_device_fault() == 0
     for j, (y, (xb, p, s, b)) in enumerate(zip(outs, refs)):
         _assert_close(y, oracle.matmul(xb, p, s, b, G, bits), f"after the timeout, matmul {j}")
+
+
+# ----------------------------------------------------------------------------- block-scaled prefill (M > 8)
+
+BS_PREFILL = [(9, 512, 16), (100, 1024, 100), (300, 4096, 600), (130, 2560, 2600)]
+
+
+@pytest.mark.parametrize("M,K,N", BS_PREFILL)
+def test_block_scaled_prefill_matches_oracle(M, K, N):
+    """mxfp4, nvfp4 and mxfp8 with more than 8 activation rows: the tensor-core
+    matmul (codes dequantized to fp16 on chip, each row scaled by a power of
+    two) against the oracle's exact product."""
+    w = weights(N, K, 80 + K + N, True)
+    xb = activations_bits(M, K, 81 + M)
+    x = _x_gpu(xb)
+    p_ref, s_ref, p, s = _mx_gpu(w)
+    y = aq.aq_mxfp4_matmul(x, p, s)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.mxfp4_matmul(xb, p_ref, s_ref), f"mxfp4 prefill M={M} K={K} N={N}")
+    p_ref, s_ref, p, s = _mx8_gpu(w)
+    y = aq.aq_mxfp8_matmul(x, p, s)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.mxfp8_matmul(xb, p_ref, s_ref), f"mxfp8 prefill M={M} K={K} N={N}")
+    p_ref, s_ref, g_ref, p, s, g = _nv_gpu(w)
+    y = aq.aq_nvfp4_matmul(x, p, s, g)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.nvfp4_matmul(xb, p_ref, s_ref, g_ref), f"nvfp4 prefill M={M} K={K} N={N}")
+    assert aq.aq_device_fault() == 0
+
+
+def test_block_scaled_prefill_special_weights():
+    """Zero groups, subnormal and huge block scales and one-signed rows: every
+    row's power of two keeps its largest groups exact in fp16."""
+    M = 40
+    xb = activations_bits(M, 1024, 85)
+    x = _x_gpu(xb)
+    w = _mx_special(64, 1024, 86)
+    p_ref, s_ref, p, s = _mx_gpu(w)
+    y = aq.aq_mxfp4_matmul(x, p, s)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.mxfp4_matmul(xb, p_ref, s_ref), "mxfp4 prefill special")
+    p_ref, s_ref, p, s = _mx8_gpu(w)
+    y = aq.aq_mxfp8_matmul(x, p, s)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.mxfp8_matmul(xb, p_ref, s_ref), "mxfp8 prefill special")
+    w = _nv_special(64, 1024, 87)
+    p_ref, s_ref, g_ref, p, s, g = _nv_gpu(w)
+    y = aq.aq_nvfp4_matmul(x, p, s, g)
+    torch.cuda.synchronize()
+    _assert_close(y, oracle.nvfp4_matmul(xb, p_ref, s_ref, g_ref), "nvfp4 prefill special")
+    assert aq.aq_device_fault() == 0

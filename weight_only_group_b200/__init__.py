@@ -462,7 +462,7 @@ def aq_mxfp4_dequantize(packed, scales, K: int, out: torch.Tensor | None = None,
 
 
 def aq_mxfp4_matmul(x, packed, scales, out: torch.Tensor | None = None, overlap_previous: bool = False):
-    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for mxfp4 weights (decode, M <= 8)."""
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for mxfp4 weights (decode up to M = 8, tensor-core prefill above)."""
     _need(x, "x", (torch.bfloat16,))
     N = _mx(packed, scales)
     M, K = x.shape
@@ -520,7 +520,7 @@ def aq_nvfp4_dequantize(packed, scales, g, K: int, out: torch.Tensor | None = No
 
 
 def aq_nvfp4_matmul(x, packed, scales, g, out: torch.Tensor | None = None, overlap_previous: bool = False):
-    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for nvfp4 weights (decode, M <= 8)."""
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for nvfp4 weights (decode up to M = 8, tensor-core prefill above)."""
     _need(x, "x", (torch.bfloat16,))
     N = _nv(packed, scales, g)
     M, K = x.shape
@@ -568,7 +568,7 @@ def aq_mxfp8_dequantize(packed, scales, K: int, out: torch.Tensor | None = None,
 
 
 def aq_mxfp8_matmul(x, packed, scales, out: torch.Tensor | None = None, overlap_previous: bool = False):
-    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for mxfp8 weights (decode, M <= 8)."""
+    """y [M, N] bf16 = x [M, K] bf16 @ dequant(W)^T for mxfp8 weights (decode up to M = 8, tensor-core prefill above)."""
     _need(x, "x", (torch.bfloat16,))
     N = _mx(packed, scales)
     M, K = x.shape

@@ -26,6 +26,9 @@ void set_qmv_tc_wait_stall(bool on);
 cudaError_t read_and_clear_embed_fault(uint32_t *word);
 bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 constexpr int64_t kQmmGroupMaxE = 256;  // experts of one grouped prefill launch at most
+cudaError_t launch_qmm_block_scaled(int fmt, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                                    const uint8_t *scales, const float *gscale, int64_t N, uint16_t *y, void *ws,
+                                    cudaStream_t s);
 cudaError_t launch_qmm_grouped(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed,
                                const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
                                const int32_t *offsets, uint16_t *y, void *ws, cudaStream_t s);
@@ -205,6 +208,20 @@ cudaError_t ws_pool(cudaMemPool_t *out) {
   }
   *out = pools[dev];
   return cudaSuccess;
+}
+
+cudaError_t ws_alloc(void **p, size_t bytes, cudaStream_t s);
+
+// Prefill (M > 8) of a block-scaled format on the tensor-core matmul, with its
+// fp16 activation workspace from the library's pool.
+cudaError_t block_scaled_prefill(int fmt, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                                 const uint8_t *scales, const float *gscale, int64_t N, uint16_t *y, cudaStream_t s) {
+  void *ws = nullptr;
+  cudaError_t e = ws_alloc(&ws, aq::qmm_workspace_bytes(M, K), s);
+  if (e != cudaSuccess) return e;
+  const cudaError_t le = aq::launch_qmm_block_scaled(fmt, x, M, K, packed, scales, gscale, N, y, ws, s);
+  e = cudaFreeAsync(ws, s);
+  return le != cudaSuccess ? le : e;
 }
 
 cudaError_t ws_alloc(void **p, size_t bytes, cudaStream_t s) {
@@ -568,6 +585,10 @@ aq_status aq_mxfp4_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_
   if ((flags & ~static_cast<uint32_t>(AQ_MATMUL_OVERLAP_PREVIOUS)) != 0) return AQ_ERR_INVALID_ARG;
   if (!x || !packed || !scales || !y) return AQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return AQ_ERR_ALIGNMENT;
+  if (M > 8) {  // prefill: the tensor-core matmul
+    if ((st = check_device()) != AQ_OK) return st;
+    return from_cuda(block_scaled_prefill(1, x, M, K, packed, scales, nullptr, N, y, stream));
+  }
   if (!aq::mxfp4_tc_supported(M, N, K)) return AQ_ERR_UNSUPPORTED;
   if ((st = check_device()) != AQ_OK) return st;
   return from_cuda(aq::launch_mxfp4_tc(x, M, K, packed, scales, N, y, flags, stream));
@@ -623,9 +644,13 @@ aq_status aq_nvfp4_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y) ||
       (reinterpret_cast<uintptr_t>(tensor_scale) & 3u) != 0)
     return AQ_ERR_ALIGNMENT;
+  if (M > 8) {  // prefill: the tensor-core matmul
+    if ((st = check_device()) != AQ_OK) return st;
+    return from_cuda(block_scaled_prefill(2, x, M, K, packed, scales, tensor_scale, N, y, stream));
+  }
   // the decode kernel holds up to 4 tokens (two group slots per token); M = 5..8
   // runs as two launches, rows 0..3 and 4..M-1 (the weights are read twice)
-  if (M > 8 || !aq::nvfp4_tc_supported(std::min<int64_t>(M, 4), N, K)) return AQ_ERR_UNSUPPORTED;
+  if (!aq::nvfp4_tc_supported(std::min<int64_t>(M, 4), N, K)) return AQ_ERR_UNSUPPORTED;
   if ((st = check_device()) != AQ_OK) return st;
   const int64_t m0 = std::min<int64_t>(M, 4);
   st = from_cuda(aq::launch_nvfp4_tc(x, m0, K, packed, scales, tensor_scale, N, y, flags, stream));
@@ -678,6 +703,10 @@ aq_status aq_mxfp8_matmul(const uint16_t *x, int64_t M, int64_t K, const uint32_
   if ((flags & ~static_cast<uint32_t>(AQ_MATMUL_OVERLAP_PREVIOUS)) != 0) return AQ_ERR_INVALID_ARG;
   if (!x || !packed || !scales || !y) return AQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return AQ_ERR_ALIGNMENT;
+  if (M > 8) {  // prefill: the tensor-core matmul
+    if ((st = check_device()) != AQ_OK) return st;
+    return from_cuda(block_scaled_prefill(3, x, M, K, packed, scales, nullptr, N, y, stream));
+  }
   if (!aq::mxfp8_tc_supported(M, N, K)) return AQ_ERR_UNSUPPORTED;
   if ((st = check_device()) != AQ_OK) return st;
   return from_cuda(aq::launch_mxfp8_tc(x, M, K, packed, scales, N, y, flags, stream));

@@ -106,6 +106,11 @@ struct Params {
   // e*N .. e*N+N-1 of the stacked W); offsets live in device memory
   const int32_t *offsets;
   int E;
+  // block-scaled formats: one scale byte per 32 codes (mxfp4 / mxfp8, E8M0) or
+  // per 16 (nvfp4, E4M3) in rows of sb_row bytes, and nvfp4's tensor scale
+  const uint8_t *bscales;
+  int sb_row;
+  const float *gscale;
 };
 
 // One tile of a launch: its first token row and first W row in the maps, the
@@ -153,7 +158,8 @@ AQ_DEVICE TileRef tile_at(const Params &prm, const int *seg, const int *mtp, int
   return r;
 }
 
-template <int BITS, int BN>
+// FMT: 0 affine (fp16 scale and bias per G codes); 1 mxfp4, 2 nvfp4, 3 mxfp8.
+template <int BITS, int BN, int FMT = 0>
 __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant__ CUtensorMap x_map,
                                                           const __grid_constant__ CUtensorMap w_map, Params prm) {
   using C = Cfg<BITS, BN>;
@@ -278,15 +284,47 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
       const int n = tr.n0 + row;
       const bool row_ok = n < prm.N;
       const int64_t g_row = static_cast<int64_t>(row_ok ? tr.wrow + row : 0) * prm.Gn;
-      // scales/biases (fp16 bits) of this thread's chunks, prefetched for this
-      // warp's next two K blocks (its turns come every H blocks)
+      // Block-scaled formats: this row's power of two 2^-B (from its largest
+      // scale byte; positive E4M3 and E8M0 order like their bits) keeps every
+      // dequantized value within fp16; the epilogue multiplies by 2^B.
+      const uint8_t *sbrow = nullptr;
+      int bexp = 0;
+      float rowfac = 1.0f;
+      if constexpr (FMT != 0) {
+        sbrow = prm.bscales + static_cast<int64_t>(row_ok ? tr.wrow + row : 0) * prm.sb_row;
+        uint32_t mx = 0;
+        if (row_ok)
+          for (int i = 0; i < prm.sb_row / 16; ++i) {
+            const uint4 v = ldg_nc16(sbrow + 16 * i);
+            mx = __vmaxu4(mx, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
+          }
+        mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
+        if constexpr (FMT == 2) {
+          const float vmax = e4m3_value(mx);
+          bexp = vmax > 0.0f ? static_cast<int>((__float_as_uint(vmax) >> 23) & 0xFFu) - 127 + 1 - 13 : 0;
+          rowfac = pow2f_exact(bexp) * __ldg(prm.gscale);
+        } else {
+          bexp = static_cast<int>(mx) - 127 - (FMT == 1 ? 13 : 7);
+          rowfac = pow2f_exact(bexp);
+        }
+      }
+      // scales/biases (fp16 bits; block-scaled: the chunk's scale bytes) of this
+      // thread's chunks, prefetched for this warp's next two K blocks (its turns
+      // come every H blocks)
       auto load_sb = [&](int kb, uint16_t (&sc)[CH], uint16_t (&bi)[CH]) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          const int g = (kb * C::BK + c * 32) / prm.G;
-          const bool in = row_ok && kb < KB && g < prm.Gn;
-          sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
-          bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
+          if constexpr (FMT == 0) {
+            const int g = (kb * C::BK + c * 32) / prm.G;
+            const bool in = row_ok && kb < KB && g < prm.Gn;
+            sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
+            bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
+          } else {
+            const int g32 = (kb * C::BK + c * 32) / 32;  // the chunk's 32-code span
+            const bool in = row_ok && kb < KB && g32 < prm.K / 32;
+            sc[c] = !in ? uint16_t(0) : FMT == 2 ? ldg_nc2(sbrow + 2 * g32) : static_cast<uint16_t>(sbrow[g32]);
+            bi[c] = 0;
+          }
         }
       };
       uint16_t sc_pf[2][CH], bi_pf[2][CH];
@@ -326,7 +364,20 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
             for (int i = 0; i < BITS; ++i) w[i] = wrow[c * BITS + i];
           }
           uint32_t packed_cols[16];
-          dequant_chunk_f16<BITS>(w, sc[c], bi[c], packed_cols);
+          if constexpr (FMT == 0) {
+            dequant_chunk_f16<BITS>(w, sc[c], bi[c], packed_cols);
+          } else if constexpr (FMT == 1) {
+            const __half2 f = __float2half2_rn(pow2f_exact(static_cast<int>(sc[c]) - 127 - bexp));
+            dequant_chunk_e2m1(reinterpret_cast<const uint32_t(&)[4]>(w), f, f, packed_cols);
+          } else if constexpr (FMT == 2) {
+            const float p2 = pow2f_exact(-bexp);
+            const __half2 f0 = __float2half2_rn(e4m3_value(sc[c] & 0xFFu) * p2);
+            const __half2 f1 = __float2half2_rn(e4m3_value(sc[c] >> 8) * p2);
+            dequant_chunk_e2m1(reinterpret_cast<const uint32_t(&)[4]>(w), f0, f1, packed_cols);
+          } else {
+            const __half2 f = __float2half2_rn(pow2f_exact(static_cast<int>(sc[c]) - 127 - bexp + 8));
+            dequant_chunk_e4m3(reinterpret_cast<const uint32_t(&)[8]>(w), f, packed_cols);
+          }
           tmem_st16(a_tmem + c * 16, packed_cols);
         }
         tmem_st_wait();
@@ -351,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
             const int m = m0 + col + i;
             if (m < tr.mend)
               prm.y[static_cast<int64_t>(m) * prm.N + n] =
-                  __float2bfloat16_rn(__uint_as_float(v[i]) * __ldg(prm.row_scale + m));
+                  __float2bfloat16_rn(__uint_as_float(v[i]) * __ldg(prm.row_scale + m) * rowfac);
           }
         }
       }
@@ -784,6 +835,9 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
   Params prm;
   prm.offsets = nullptr;
   prm.E = 0;
+  prm.bscales = nullptr;
+  prm.sb_row = 0;
+  prm.gscale = nullptr;
   prm.scales = reinterpret_cast<const __half *>(scales);
   prm.biases = reinterpret_cast<const __half *>(biases);
   prm.row_scale = row_scale;
@@ -805,6 +859,81 @@ cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *pa
 #endif
 
   auto kern = qmm_kernel<BITS, BN>;
+  static thread_local int cached_dev = -1;
+  static thread_local int sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
+      return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+  kern<<<grid, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, prm);
+  return cudaGetLastError();
+}
+
+// Block-scaled prefill (FMT 1 mxfp4, 2 nvfp4, 3 mxfp8) on the single-CTA
+// kernel: codes as the affine 4-bit / 8-bit layouts, one scale byte per 32
+// (or 16) codes, and the dequantization of tc05.cuh.
+template <int FMT, int BN>
+cudaError_t launch_fmt_t(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint8_t *bscales,
+                         const float *gscale, int64_t N, uint16_t *y, void *workspace, cudaStream_t stream) {
+  constexpr int BITS = FMT == 3 ? 8 : 4;
+  using C = Cfg<BITS, BN>;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  __half *x16 = reinterpret_cast<__half *>(workspace);
+  float *row_scale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + ((M * K * 2 + 255) / 256) * 256);
+  x_to_f16_rows_kernel<BITS><<<static_cast<unsigned>(M), kPrepThreads, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
+  CUtensorMap x_map, w_map;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(BN)};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const int64_t P = K * BITS / 32;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(P) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(C::BKW), 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(packed), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  Params prm;
+  prm.offsets = nullptr;
+  prm.E = 0;
+  prm.bscales = bscales;
+  prm.sb_row = static_cast<int>(FMT == 2 ? K / 16 : K / 32);
+  prm.gscale = gscale;
+  prm.scales = nullptr;
+  prm.biases = nullptr;
+  prm.row_scale = row_scale;
+  prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  prm.M = static_cast<int>(M);
+  prm.N = static_cast<int>(N);
+  prm.K = static_cast<int>(K);
+  prm.G = 32;
+  prm.Gn = static_cast<int>(K / 32);
+  prm.m_tiles = static_cast<int>((M + BN - 1) / BN);
+  prm.n_tiles = static_cast<int>((N + 127) / 128);
+  const int64_t w_bytes = N * K * BITS / 8 + prm.sb_row * N;
+  prm.n_fastest = (2 * M * K > w_bytes) ? 1 : 0;
+  auto kern = qmm_kernel<BITS, BN, FMT>;
   static thread_local int cached_dev = -1;
   static thread_local int sms = 0;
   int dev = 0;
@@ -863,6 +992,9 @@ cudaError_t launch_grouped_t(const uint16_t *x, int64_t T, int64_t K, const uint
   Params prm;
   prm.offsets = offsets;
   prm.E = static_cast<int>(E);
+  prm.bscales = nullptr;
+  prm.sb_row = 0;
+  prm.gscale = nullptr;
   prm.scales = reinterpret_cast<const __half *>(scales);
   prm.biases = reinterpret_cast<const __half *>(biases);
   prm.row_scale = row_scale;
@@ -931,6 +1063,9 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   Params prm;
   prm.offsets = nullptr;
   prm.E = 0;
+  prm.bscales = nullptr;
+  prm.sb_row = 0;
+  prm.gscale = nullptr;
   prm.scales = reinterpret_cast<const __half *>(scales);
   prm.biases = reinterpret_cast<const __half *>(biases);
   prm.row_scale = row_scale;
@@ -1015,6 +1150,27 @@ cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
 }
 
 }  // namespace qmm
+
+// Block-scaled prefill: fmt 1 mxfp4, 2 nvfp4 (gscale: its tensor scale on the
+// device), 3 mxfp8; token tile 64 / 128 / 256 by M as the affine single CTA.
+cudaError_t launch_qmm_block_scaled(int fmt, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
+                                    const uint8_t *scales, const float *gscale, int64_t N, uint16_t *y, void *ws,
+                                    cudaStream_t s) {
+  const int bn = M <= 64 ? 64 : M <= 128 ? 128 : 256;
+#define AQ_FMT_BN(F)                                                                                               \
+  switch (bn) {                                                                                                    \
+    case 64: return qmm::launch_fmt_t<F, 64>(x, M, K, packed, scales, gscale, N, y, ws, s);                       \
+    case 128: return qmm::launch_fmt_t<F, 128>(x, M, K, packed, scales, gscale, N, y, ws, s);                     \
+    default: return qmm::launch_fmt_t<F, 256>(x, M, K, packed, scales, gscale, N, y, ws, s);                      \
+  }
+  switch (fmt) {
+    case 1: AQ_FMT_BN(1)
+    case 2: AQ_FMT_BN(2)
+    case 3: AQ_FMT_BN(3)
+    default: return cudaErrorInvalidValue;
+  }
+#undef AQ_FMT_BN
+}
 
 // Grouped prefill (see launch_grouped_t): BN by the mean segment length.
 cudaError_t launch_qmm_grouped(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed,

@@ -151,6 +151,66 @@ AQ_DEVICE void dequant_chunk_f16(const uint32_t (&w)[BITS], uint16_t sc_bits, ui
   }
 }
 
+// ---------------------------------------------------------------------------
+// Block-scaled formats (prefill): one 32-code chunk into 16 TMEM columns of
+// fp16 pairs, each value scaled by a power of two 2^-B of its W row (B from
+// the row's largest scale, so every value is an exact fp16 for groups within
+// 2^22 of the row's largest; the epilogue multiplies by 2^B).
+//
+// E2M1 code m (sign in bit 3) as fp16 bits ((m & 7) << 9 | (m & 8) << 12) is
+// the code's value times 2^-14 (exponent field and mantissa bit line up; the
+// one subnormal code, 0.5, becomes fp16's subnormal 2^-15); E4M3 byte b as
+// ((b & 0x7F) << 7 | (b & 0x80) << 8) is its value times 2^-8.  The chunk is
+// then one packed fp16 multiply by the group's factor (exact: a power of two,
+// or an E4M3 value for nvfp4), in the pair order of the affine 4-bit and
+// 8-bit paths (so the same x16 interleave serves).
+// ---------------------------------------------------------------------------
+// E2M1 chunk (mxfp4, nvfp4): f_lo scales words 0-1 (codes 0..15), f_hi words
+// 2-3 (codes 16..31): the same factor for mxfp4, the two 16-code groups' for
+// nvfp4.  Each factor is a value of at most 4 significant bits.
+AQ_DEVICE void dequant_chunk_e2m1(const uint32_t (&w)[4], __half2 f_lo, __half2 f_hi, uint32_t (&cols)[16]) {
+  const __half2 two14 = __half2half2(__ushort_as_half(0x7400));  // 2^14: the bits above read as value * 2^-14
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 f = i < 2 ? f_lo : f_hi;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t v = (w[i] >> (4 * j)) & 0x000F000Fu;  // codes j and j + 4 of the word
+      const uint32_t h = ((v & 0x00070007u) << 9) | ((v & 0x00080008u) << 12);
+      __half2 x = __hmul2(*reinterpret_cast<const __half2 *>(&h), two14);  // the E2M1 values, exact
+      x = __hmul2(x, f);
+      cols[4 * i + j] = *reinterpret_cast<uint32_t *>(&x);
+    }
+  }
+}
+// E4M3 chunk (mxfp8; four codes per word, natural order): f = the group's
+// factor times 2^8 (the bits above read as value * 2^-8).
+AQ_DEVICE void dequant_chunk_e4m3(const uint32_t (&w)[8], __half2 f, uint32_t (&cols)[16]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t v = w[i] >> (16 * j);
+      const uint32_t b0 = v & 0xFFu, b1 = (v >> 8) & 0xFFu;
+      const uint32_t h = (((b0 & 0x7Fu) << 7) | ((b0 & 0x80u) << 8)) |
+                         ((((b1 & 0x7Fu) << 7) | ((b1 & 0x80u) << 8)) << 16);
+      __half2 x = __hmul2(*reinterpret_cast<const __half2 *>(&h), f);
+      cols[2 * i + j] = *reinterpret_cast<uint32_t *>(&x);
+    }
+  }
+}
+// 2^e as an fp32 (exact for e in [-149, 127]; 0 below)
+AQ_DEVICE float pow2f_exact(int e) {
+  if (e >= -126) return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+  if (e >= -149) return __uint_as_float(1u << (e + 149));
+  return 0.0f;
+}
+// value of an E4M3 byte (exact in fp32)
+AQ_DEVICE float e4m3_value(uint32_t b) {
+  const uint16_t h = static_cast<uint16_t>(((b & 0x7Fu) << 7) | ((b & 0x80u) << 8));  // value * 2^-8
+  return __half2float(__ushort_as_half(h)) * 256.0f;
+}
+
 // K order of x16 inside each block of 8 (4-bit) or 16 (2-bit) elements: slot t
 // holds element kx_perm(t) of the block, matching the pairs of dequant_chunk_f16.
 __host__ __device__ constexpr int kx_block(int bits) { return bits == 4 ? 8 : bits == 2 ? 16 : 1; }
