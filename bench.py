@@ -551,6 +551,23 @@ def section_mxfp4(args, aq, torch, dev, stream, peaks):
                                        "kernel": "qmv_tc_kernel<4,32,1,nvfp4> (two 16-groups per MMA K step)"}
         del qs, base
         torch.cuda.empty_cache()
+    # prefill (M = 2048, K = 4096, N = 14336) of the three formats on the tcgen05 matmul
+    M, K, N = 2048, 4096, 14336
+    w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 6 + 9)).to(dev)
+    x = synth.activations(M, K, 19).to(dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    for name, quant, call in (("mxfp4", aq.aq_mxfp4_quantize, aq.aq_mxfp4_matmul),
+                              ("nvfp4", aq.aq_nvfp4_quantize, aq.aq_nvfp4_matmul),
+                              ("mxfp8", aq.aq_mxfp8_quantize, aq.aq_mxfp8_matmul)):
+        q = quant(w)
+        ms = timed_graph(torch, stream, lambda i: call(x, *q, out=y), 2, 10)
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[f"{name}_qmm_M{M}_K{K}_N{N}"] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1),
+                                             "frac_of_burst": round(tf / peaks["bf16_tflops"], 4),
+                                             "kernel": "qmm_kernel (tcgen05 kind::f16, codes dequantized to fp16)"}
+        del q
+    del w, x, y
+    torch.cuda.empty_cache()
     return out
 
 
