@@ -490,7 +490,7 @@ def section_gather(args, aq, torch, dev, stream, peaks):
     tf = 2.0 * T * N * K / (ms * 1e-3) / 1e12
     res["prefill_grouped_4096_rows"] = {"rows": T, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
                                         "frac_bf16_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
-                                        "note": "includes routing, the host read of per-expert counts, gather/scatter"}
+                                        "note": "includes routing and the gather/scatter copies; one matmul launch over all experts, no host read"}
     return {"gather_qmv": {"E": E, "N": N, "K": K, "bits": BITS, "G": G, "points": res}}
 
 

@@ -53,7 +53,11 @@ __device__ uint32_t g_fault_word = 0;
 
 namespace qmm {
 
-constexpr int kDequantPerQuadrant = 3;  // dequant warps per TMEM lane quadrant; they take turns on K blocks
+constexpr int kDequantPerQuadrant = 3;
+// Turns of scale / bias loads a dequant warp keeps in flight: a global load
+// issued from an SM with a full ring of tile copies outstanding waits behind
+// them (microseconds), so they are requested this many turns ahead.
+constexpr int kSbAhead = 4;  // dequant warps per TMEM lane quadrant; they take turns on K blocks
 constexpr int kDequantWarp0 = 4;        // warps 4.. dequantize + epilogue
 constexpr int kThreads = 32 * (kDequantWarp0 + 4 * kDequantPerQuadrant);
 constexpr int kTmemCols = 512;
@@ -327,21 +331,29 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
           }
         }
       };
-      uint16_t sc_pf[2][CH], bi_pf[2][CH];
-      load_sb(h, sc_pf[0], bi_pf[0]);
-      load_sb(h + H, sc_pf[1], bi_pf[1]);
-      int slot = 0;
-      for (int kb = h; kb < KB; kb += H, slot ^= 1) {
+      // a queue of the next kSbAhead turns' scales, shifted by one each turn
+      // (static indices keep it in registers)
+      uint16_t sc_pf[kSbAhead][CH], bi_pf[kSbAhead][CH];
+#pragma unroll
+      for (int i = 0; i < kSbAhead; ++i) load_sb(h + i * H, sc_pf[i], bi_pf[i]);
+      for (int kb = h; kb < KB; kb += H) {
         const uint32_t it = it0 + kb;
         const int s = it % S;
         const uint32_t r = it / S;
         uint16_t sc[CH], bi[CH];
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          sc[c] = sc_pf[slot][c];
-          bi[c] = bi_pf[slot][c];
+          sc[c] = sc_pf[0][c];
+          bi[c] = bi_pf[0][c];
         }
-        load_sb(kb + 2 * H, sc_pf[slot], bi_pf[slot]);
+#pragma unroll
+        for (int i = 0; i + 1 < kSbAhead; ++i)
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            sc_pf[i][c] = sc_pf[i + 1][c];
+            bi_pf[i][c] = bi_pf[i + 1][c];
+          }
+        load_sb(kb + kSbAhead * H, sc_pf[kSbAhead - 1], bi_pf[kSbAhead - 1]);
         if (!(ok = mbar_wait(&full[s], r & 1, abort_flag, kFaultDequantWait))) break;
         if (r >= 1 && !(ok = mbar_wait(&empty[s], (r - 1) & 1, abort_flag, kFaultDequantWait))) break;
         __syncwarp();  // lanes leave the spin at different times; tcgen05.st needs the whole warp
@@ -632,21 +644,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
         }
       };
-      uint16_t sc_pf[2][CH], bi_pf[2][CH];
-      load_sb(h, sc_pf[0], bi_pf[0]);
-      load_sb(h + H, sc_pf[1], bi_pf[1]);
-      int slot = 0;
-      for (int kb = h; kb < KB; kb += H, slot ^= 1) {
+      // a queue of the next kSbAhead turns' scales, shifted by one each turn
+      // (static indices keep it in registers)
+      uint16_t sc_pf[kSbAhead][CH], bi_pf[kSbAhead][CH];
+#pragma unroll
+      for (int i = 0; i < kSbAhead; ++i) load_sb(h + i * H, sc_pf[i], bi_pf[i]);
+      for (int kb = h; kb < KB; kb += H) {
         const uint32_t it = it0 + kb;
         const int s = it % S;
         const uint32_t r = it / S;
         uint16_t sc[CH], bi[CH];
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          sc[c] = sc_pf[slot][c];
-          bi[c] = bi_pf[slot][c];
+          sc[c] = sc_pf[0][c];
+          bi[c] = bi_pf[0][c];
         }
-        load_sb(kb + 2 * H, sc_pf[slot], bi_pf[slot]);
+#pragma unroll
+        for (int i = 0; i + 1 < kSbAhead; ++i)
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            sc_pf[i][c] = sc_pf[i + 1][c];
+            bi_pf[i][c] = bi_pf[i + 1][c];
+          }
+        load_sb(kb + kSbAhead * H, sc_pf[kSbAhead - 1], bi_pf[kSbAhead - 1]);
         if (!(ok = mbar_wait(&full[s], r & 1, abort_flag, kFaultDequantWait))) break;
         if (r >= 1 && !(ok = mbar_wait_cluster(&empty[s], (r - 1) & 1, abort_flag, kFaultDequantWait))) break;
         __syncwarp();
