@@ -463,11 +463,13 @@ struct PairCfg {
   static constexpr int X_BYTES = XH * BK * 2;
   static constexpr int W_BYTES = 128 * BKW * 4;
   static constexpr int STAGE_BYTES = ((X_BYTES + W_BYTES + 1023) / 1024) * 1024;
-  static constexpr int SMEM_BUDGET = 225 * 1024;
+  // epilogue staging: per dequant warp two 32 x 32 bf16 output boxes for TMA stores
+  static constexpr int EPI_BYTES = 4 * kDequantPerQuadrant * 2 * 2048;
+  static constexpr int SMEM_BUDGET = 225 * 1024 - EPI_BYTES;
   static constexpr int A_COLS = BK / 2;
   static constexpr int A_COL0 = BN;
   static constexpr int STAGES = std::min(std::min(12, SMEM_BUDGET / STAGE_BYTES), (kTmemCols - A_COL0) / A_COLS);
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512 /*barriers*/;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512 /*barriers*/ + EPI_BYTES;
   static_assert(STAGES >= 2, "not enough shared memory for two stages");
   static_assert((3 * STAGES + 2) * 8 + 8 <= 512, "barrier area");
   static_assert(XH % 8 == 0 && BN <= 256 && BN % 32 == 0, "pair MMA N");
@@ -513,6 +515,18 @@ AQ_DEVICE void tc_commit_pair(uint64_t *bar) {
       "h"(static_cast<uint16_t>(3))
       : "memory");
 }
+// TMA store of a 2-D box from shared memory, in this thread's bulk group.
+AQ_DEVICE void tma_store_2d(const CUtensorMap *map, const void *src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+AQ_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+AQ_DEVICE void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+AQ_DEVICE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // kind::f16 instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, M = 256, N = bn.
 __host__ __device__ constexpr uint32_t idesc_pair(int bn) {
   return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
@@ -520,7 +534,8 @@ __host__ __device__ constexpr uint32_t idesc_pair(int bn) {
 
 template <int BITS, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    qmm_pair_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map, Params prm) {
+    qmm_pair_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map,
+                    const __grid_constant__ CUtensorMap y_map, Params prm) {
   using C = PairCfg<BITS, BN>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -627,6 +642,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     constexpr int H = kDequantPerQuadrant;
     const int row = q * 32 + lane;
     constexpr int CH = C::BK / 32;
+    uint8_t *ebox = smem + S * C::STAGE_BYTES + 512 + (warp - kDequantWarp0) * 2 * 2048;  // two output boxes
+    int eb = 0;
     uint32_t it0 = 0, t = 0;
     bool ok = true;
     for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++t, it0 += KB) {
@@ -702,25 +719,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait_cluster(acc_full, t & 1, abort_flag, kFaultEpilogueWait))) break;
       __syncwarp();
       tc_fence_after();
+      // Each 32-column block: this warp's 32 rows x 32 tokens, scaled and
+      // rounded into a shared-memory box (token-major, the layout of y) and
+      // written by one TMA store, which clips rows past N and tokens past M.
 #pragma unroll 1
       for (int col = h * 32; col < BN; col += H * 32) {
         uint32_t v[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + col, v);
+        const int mlane = m0 + col + lane;
+        const float rs = mlane < prm.M ? __ldg(prm.row_scale + mlane) : 0.0f;  // token col + lane's scale
         tmem_ld_wait();
-        if (row_ok) {
+        uint8_t *box = ebox + eb * 2048;
+        if (lane == 0) bulk_wait_read<1>();  // the store that last read this box is done with it
+        __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int m = m0 + col + i;
-            if (m < prm.M)
-              prm.y[static_cast<int64_t>(m) * prm.N + n] =
-                  __float2bfloat16_rn(__uint_as_float(v[i]) * __ldg(prm.row_scale + m));
-          }
+        for (int i = 0; i < 32; ++i) {
+          const float r = __shfl_sync(0xffffffffu, rs, i);
+          *reinterpret_cast<__nv_bfloat16 *>(box + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]) * r);
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the copy engine reads the box
+        __syncwarp();
+        const int bn0 = n0 + static_cast<int>(rank) * 128 + q * 32;
+        if (lane == 0 && bn0 < prm.N && m0 + col < prm.M) {  // (a box wholly past the edges is not stored)
+          tma_store_2d(&y_map, box, bn0, m0 + col);
+          bulk_commit();
+        }
+        eb ^= 1;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_at(acc_empty, 0);
     }
+    if (lane == 0) bulk_wait_all();  // this warp's output stores have completed
   }
 
   tc_fence_before();
@@ -1080,6 +1110,16 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  CUtensorMap y_map;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&y_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   Params prm;
   prm.offsets = nullptr;
   prm.E = 0;
@@ -1117,7 +1157,7 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   }
   const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
   const int pairs = static_cast<int>(std::min<int64_t>(tiles, std::max(1, sms / 2)));
-  kern<<<2 * pairs, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, prm);
+  kern<<<2 * pairs, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, y_map, prm);
   return cudaGetLastError();
 }
 
@@ -1135,7 +1175,7 @@ int pick_shape(int64_t M, int64_t N, int sms) {
 #ifdef AQ_QMM_FORCE_SHAPE  // build-time override (0..3 as in Shape; else choose)
   if (AQ_QMM_FORCE_SHAPE >= 0 && AQ_QMM_FORCE_SHAPE <= 3) return AQ_QMM_FORCE_SHAPE;
 #endif
-  if (M > 128) return kPair256;
+  if (M > 128 && N % 8 == 0) return kPair256;  // (the pair's output stores need 16-byte rows of y)
   auto score = [&](int64_t bn, int64_t bytes) {
     const int64_t t = ((M + bn - 1) / bn) * ((N + 127) / 128);
     const int64_t waves = (t + sms - 1) / sms;
