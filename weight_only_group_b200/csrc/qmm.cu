@@ -54,10 +54,12 @@ __device__ uint32_t g_fault_word = 0;
 namespace qmm {
 
 constexpr int kDequantPerQuadrant = 3;
-// Turns of scale / bias loads a dequant warp keeps in flight: a global load
-// issued from an SM with a full ring of tile copies outstanding waits behind
-// them (microseconds), so they are requested this many turns ahead.
-constexpr int kSbAhead = 4;  // dequant warps per TMEM lane quadrant; they take turns on K blocks
+// Turns of scale / bias loads a dequant warp keeps in flight (a register queue
+// with static indices; 4 was slower than 2, measured).  These loads hit L1:
+// shared memory left unused by a kernel is L1 on this part, and every 24 KB
+// more shared memory per CTA cost ~5-25% at K = 14336 (measured), so the
+// kernels keep their shared memory tight.
+constexpr int kSbAhead = 2;  // dequant warps per TMEM lane quadrant; they take turns on K blocks
 constexpr int kDequantWarp0 = 4;        // warps 4.. dequantize + epilogue
 constexpr int kThreads = 32 * (kDequantWarp0 + 4 * kDequantPerQuadrant);
 constexpr int kTmemCols = 512;
@@ -463,8 +465,8 @@ struct PairCfg {
   static constexpr int X_BYTES = XH * BK * 2;
   static constexpr int W_BYTES = 128 * BKW * 4;
   static constexpr int STAGE_BYTES = ((X_BYTES + W_BYTES + 1023) / 1024) * 1024;
-  // epilogue staging: per dequant warp two 32 x 32 bf16 output boxes for TMA stores
-  static constexpr int EPI_BYTES = 4 * kDequantPerQuadrant * 2 * 2048;
+  // epilogue staging: per dequant warp one 32 x 32 bf16 output box for TMA stores
+  static constexpr int EPI_BYTES = 4 * kDequantPerQuadrant * 2048;
   static constexpr int SMEM_BUDGET = 225 * 1024 - EPI_BYTES;
   static constexpr int A_COLS = BK / 2;
   static constexpr int A_COL0 = BN;
@@ -642,8 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     constexpr int H = kDequantPerQuadrant;
     const int row = q * 32 + lane;
     constexpr int CH = C::BK / 32;
-    uint8_t *ebox = smem + S * C::STAGE_BYTES + 512 + (warp - kDequantWarp0) * 2 * 2048;  // two output boxes
-    int eb = 0;
+    uint8_t *ebox = smem + S * C::STAGE_BYTES + 512 + (warp - kDequantWarp0) * 2048;  // this warp's output box
     uint32_t it0 = 0, t = 0;
     bool ok = true;
     for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++t, it0 += KB) {
@@ -729,8 +730,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int mlane = m0 + col + lane;
         const float rs = mlane < prm.M ? __ldg(prm.row_scale + mlane) : 0.0f;  // token col + lane's scale
         tmem_ld_wait();
-        uint8_t *box = ebox + eb * 2048;
-        if (lane == 0) bulk_wait_read<1>();  // the store that last read this box is done with it
+        uint8_t *box = ebox;
+        if (lane == 0) bulk_wait_read<0>();  // the store that last read this box is done with it
         __syncwarp();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -744,7 +745,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tma_store_2d(&y_map, box, bn0, m0 + col);
           bulk_commit();
         }
-        eb ^= 1;
       }
       tc_fence_before();
       __syncwarp();
