@@ -418,15 +418,20 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
       r0 = gr0;
       r1 = gr1;
     } else {
-      const int64_t n = job_of(jx).N;
-      r0 = static_cast<int64_t>(blockIdx.x) * n / gridDim.x;
-      r1 = static_cast<int64_t>(blockIdx.x + 1) * n / gridDim.x;
+      const uint32_t n = static_cast<uint32_t>(job_of(jx).N);
+      if (n <= 0xFFFFFFFFu / gridDim.x) {  // 32-bit division (the 64-bit one is a long software routine)
+        r0 = (blockIdx.x * n) / gridDim.x;
+        r1 = ((blockIdx.x + 1) * n) / gridDim.x;
+      } else {
+        r0 = static_cast<int64_t>(blockIdx.x) * n / gridDim.x;
+        r1 = static_cast<int64_t>(blockIdx.x + 1) * n / gridDim.x;
+      }
     }
   };
   auto job_stages = [&](int jx) {
     int64_t r0, r1;
     cta_rows(jx, r0, r1);
-    return static_cast<int>((r1 - r0 + kRows - 1) / kRows) * job_of(jx).nch;
+    return static_cast<int>(static_cast<uint32_t>(r1 - r0 + kRows - 1) / kRows) * job_of(jx).nch;
   };
   const long long wlim = a.wait_cycles;
 
@@ -675,7 +680,7 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
   }
   int64_t r0, r1;
   cta_rows(jx, r0, r1);
-  const int nst = static_cast<int>((r1 - r0 + kRows - 1) / kRows) * Jb.nch;
+  const int nst = static_cast<int>(static_cast<uint32_t>(r1 - r0 + kRows - 1) / kRows) * Jb.nch;
   const int gpc = Jb.Kc / G;  // groups per chunk
   __nv_bfloat16 *yg = a.cta_per_tok > 0 ? yg0 : Jb.y;
   const uint8_t *xs_lane = xs + (my_real ? my_m : 0) * Jb.tok_stride + t * 16;
