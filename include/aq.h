@@ -27,7 +27,9 @@
  *   y        bf16 bits [M, N]       y = x @ dequant(W)^T
  * Ownership: every pointer argument is DEVICE memory, allocated, owned and freed
  * by the caller.  Only the tensor-core matmul path (large M) needs temporary
- * device memory (a workspace: the activations converted to fp16); aq_matmul and
+ * device memory (a workspace: the activations converted to fp16 and, for a
+ * product of few 256 x 256 tiles, the fp32 partial sums of its K split);
+ * aq_matmul and
  * aq_matmul_with take it, stream-ordered on `stream`, from a memory pool the
  * library creates per device and keeps (it holds the largest workspace in use
  * at once until the process exits), aq_matmul_ws takes it from the caller, and
@@ -204,7 +206,14 @@ aq_status aq_matmul_sequence(const aq_matmul_desc *calls, int n, int64_t M, int 
                              aq_stream_t stream);
 
 /* Bytes of workspace aq_matmul_ws needs for this shape (0 when the dispatched
- * kernel needs none, or when the arguments would be rejected).  Host only. */
+ * kernel needs none, or when the arguments would be rejected).  Host only.
+ * For AQ_KERNEL_QMM: the fp16 activations (2*M*K bytes) and their row scales
+ * (4*M), each rounded up to 256.  When M > 128 and N % 8 == 0 the product runs
+ * in T = ceil(M/256)*ceil(N/256) tiles on up to 74 CTA pairs; when T <= 37,
+ * each tile's K range is cut into ks = min(74 / T, 4, KB / 32) parts (KB: K
+ * blocks of 64, or 128 for 3-bit codes; split when ks >= 2), which adds T*24
+ * uint32 arrival counters (rounded up to 256) and ks*T*2*128*256 fp32 partial
+ * sums.  The parts are added in a fixed order, so results repeat bit for bit. */
 size_t aq_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K, int G, int bits);
 
 /* aq_matmul with caller-provided workspace: `workspace` is device memory of at
@@ -219,7 +228,9 @@ aq_status aq_matmul_ws(const uint16_t *x_bf16, int64_t M, int64_t K,
 /* Size of the fixed device workspace behind aq_matmul_qmm_static: 80 MiB.  A
  * call needs 2*M*K + 4*M bytes (each term rounded up to 256; the fp16
  * activations and their row scales), so for example M = 8192 with K = 4096, or
- * M = 2048 with K = 14336, fit. */
+ * M = 2048 with K = 14336, fit.  A shape with a K split (aq_matmul_workspace_bytes)
+ * runs it when the whole of that workspace fits, and unsplit otherwise (same
+ * results within the tolerance). */
 #define AQ_QMM_STATIC_WORKSPACE_BYTES (80u * 1024u * 1024u)
 
 /* The tensor-core matmul (AQ_KERNEL_QMM) without any allocation: its workspace
@@ -230,7 +241,7 @@ aq_status aq_matmul_ws(const uint16_t *x_bf16, int64_t M, int64_t K,
  * captured into graphs whose launch path rejects memory-allocation nodes, or
  * runtimes that reserve the whole device up front and forbid later cudaMalloc.
  * Same arguments, layouts and result as aq_matmul_with(AQ_KERNEL_QMM, ...).
- * Errors: shapes whose workspace (aq_matmul_workspace_bytes for a QMM shape)
+ * Errors: shapes whose activations' workspace (2*M*K + 4*M bytes, as above)
  * exceeds AQ_QMM_STATIC_WORKSPACE_BYTES -> AQ_ERR_UNSUPPORTED, checked before
  * anything is launched; otherwise as aq_matmul_with.
  * The first call on each device looks up the array's device address (which may

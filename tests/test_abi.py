@@ -228,6 +228,29 @@ def test_workspace_size_rule():
     assert aq.aq_matmul_workspace_bytes(512, 4096, 4000, 64, 4) == 0       # rejected shape
 
 
+def test_workspace_size_k_split():
+    """A CTA-pair shape (M > 128, N % 8 == 0) whose T tiles of 256 x 256 fill at
+    most half of 74 pairs cuts each tile's K range into ks = min(74 // T, 4,
+    K blocks // 32) parts (K blocks of 64, 128 for 3-bit codes; split when
+    ks >= 2).  Its workspace then adds one uint32 arrival counter per (tile, CTA,
+    dequant warp), 256-byte padded, and ks*T*2*128*256 fp32 partial sums to the
+    activations' part; other shapes need the activations' part alone."""
+    def base(M, K):
+        r = lambda b: (b + 255) // 256 * 256
+        return r(M * K * 2) + r(M * 4)
+    tile2 = 2 * 128 * 256 * 4
+    ws = aq.aq_matmul_workspace_bytes
+    assert ws(512, 4096, 14336, 64, 4) == base(512, 14336) + 3072 + 2 * 32 * tile2   # 32 tiles, 2 parts
+    assert ws(257, 776, 8192, 128, 2) == base(257, 8192) + 768 + 4 * 8 * tile2      # 8 tiles, 4 parts (2-bit)
+    assert ws(129, 256, 6144, 32, 8) == base(129, 6144) + 256 + 3 * 1 * tile2       # 1 tile, 96 blocks: 3 parts
+    assert ws(256, 9472, 4096, 64, 4) == base(256, 4096) + 3584 + 2 * 37 * tile2     # 37 tiles: 74 items
+    assert ws(160, 264, 6144, 32, 3) == base(160, 6144)          # 3-bit: 48 blocks of 128, too few for two parts
+    assert ws(256, 9728, 4096, 64, 4) == base(256, 4096)         # 38 tiles: more than half the pairs
+    assert ws(2048, 4096, 14336, 64, 4) == base(2048, 14336)     # 128 tiles
+    assert ws(700, 300, 2048, 64, 4) == base(700, 2048)          # 32 K blocks
+    assert ws(128, 4096, 14336, 64, 4) == base(128, 14336)       # single-CTA kernel
+
+
 def test_workspace_validation():
     L = aq.lib()
     # a QMM shape with no workspace -> invalid argument, before any CUDA call

@@ -793,6 +793,38 @@ def test_qmm_matches_dequantize_then_matmul():
     assert float(err.max()) < 2 ** -8  # bf16 output rounding (<= 2^-9 |y|) plus fp32 summation order
 
 
+@pytest.mark.parametrize("M,K,N,bits,G", [(300, 4096, 1000, 4, 64), (160, 8192, 264, 3, 32),
+                                         (257, 8192, 776, 2, 128), (129, 6144, 256, 8, 32),
+                                         (200, 4096, 520, 4, 32), (256, 4096, 9472, 4, 64)])
+def test_qmm_pair_k_split(M, K, N, bits, G):
+    """CTA-pair launches whose tiles fill at most half of the pairs cut each
+    tile's K range into parts: 8 tiles x 2, 2 x 2, 8 x 4, 1 x 3 and 3 x 2 here
+    (ragged M and N), and 37 x 2 = 74 items, one per pair.  The parts' fp32 sums
+    meet in the workspace and the last part adds them in part order, so the
+    product matches the oracle and repeats bit for bit whichever part finishes
+    last."""
+    p_ref, s_ref, b_ref = quantized(N, K, 9400 + bits, True, G, bits)
+    pg, sg, bg = _to_gpu(p_ref, s_ref, b_ref)
+    xb = activations_bits(M, K, 9401 + bits)
+    x = _x_gpu(xb)
+    assert aq.aq_dispatch(M, N, K, G, bits) == aq.AQ_KERNEL_QMM
+    y = aq.aq_matmul(x, pg, sg, bg, G, bits)
+    if M * N * K <= 2e9:
+        y_ref = oracle.matmul(xb, p_ref, s_ref, b_ref, G, bits)
+        _assert_close(y, y_ref, f"k-split M={M} K={K} N={N} b={bits}")
+    else:  # sampled rows, every column (every tile)
+        rows = sample_rows(M, 24, 9402)
+        y_ref = oracle.matmul_sampled(xb, p_ref, s_ref, b_ref, G, bits, rows, np.arange(N))
+        rms = float(np.sqrt(np.mean(y_ref ** 2)))
+        _assert_close(y[torch.from_numpy(rows).cuda()], y_ref, f"k-split M={M} K={K} N={N} (sampled)", rms)
+    for _ in range(3):
+        assert torch.equal(aq.aq_matmul(x, pg, sg, bg, G, bits).view(torch.int16), y.view(torch.int16))
+    need = aq.aq_matmul_workspace_bytes(M, N, K, G, bits)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    assert torch.equal(aq.aq_matmul_ws(x, pg, sg, bg, G, bits, ws).view(torch.int16), y.view(torch.int16))
+    assert aq.aq_device_fault() == 0
+
+
 def test_qmm_workspace_entry_point_matches():
     M, K, N, G, bits = 700, 2048, 640, 64, 4
     p_ref, s_ref, b_ref = quantized(N, K, 431, True, G, bits)

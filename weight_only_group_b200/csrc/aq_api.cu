@@ -41,8 +41,10 @@ cudaError_t launch_embedding(const int32_t *ids, int64_t T, const uint32_t *pack
                              const uint16_t *biases, int64_t V, int64_t D, int G, int bits, uint16_t *out,
                              cudaStream_t s);
 cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s);
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, size_t ws_bytes,
+                       cudaStream_t s);
 size_t qmm_workspace_bytes(int64_t M, int64_t K);
+size_t qmm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits);
 bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits);
 cudaError_t launch_qmm2(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                         const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, cudaStream_t s);
@@ -345,16 +347,16 @@ static aq_status matmul_prepare(aq_kernel &kernel, const uint16_t *x, int64_t M,
   return AQ_ERR_INVALID_ARG;
 }
 
-static size_t workspace_for(aq_kernel kernel, int64_t M, int64_t K) {
+static size_t workspace_for(aq_kernel kernel, int64_t M, int64_t N, int64_t K, int bits) {
   // AQ_KERNEL_QMM_NOWS and the decode kernels need none
-  return kernel == AQ_KERNEL_QMM ? aq::qmm_workspace_bytes(M, K) : 0;
+  return kernel == AQ_KERNEL_QMM ? aq::qmm_workspace_bytes(M, N, K, bits) : 0;
 }
 
 // AQ_KERNEL_QMM runs with the caller's (or the stream-ordered allocator's)
 // workspace ws; AQ_KERNEL_QMM_NOWS needs none.
 static aq_status matmul_run(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                             const uint16_t *scales, const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y,
-                            void *ws, aq_stream_t stream, uint32_t flags = 0) {
+                            void *ws, size_t ws_bytes, aq_stream_t stream, uint32_t flags = 0) {
   aq_status st = check_device();
   if (st != AQ_OK) return st;
   if (kernel == AQ_KERNEL_QMV_TCGEN05 && aq::qmv_umma_supported(M, N, K, G, bits))
@@ -363,13 +365,13 @@ static aq_status matmul_run(aq_kernel kernel, const uint16_t *x, int64_t M, int6
     return from_cuda(aq::launch_qmv(x, M, K, packed, scales, biases, N, G, bits, y, flags, stream));
   if (kernel == AQ_KERNEL_QMM_NOWS)
     return from_cuda(aq::launch_qmm2(x, M, K, packed, scales, biases, N, G, bits, y, stream));
-  return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, ws, stream));
+  return from_cuda(aq::launch_qmm(x, M, K, packed, scales, biases, N, G, bits, y, ws, ws_bytes, stream));
 }
 
 size_t aq_matmul_workspace_bytes(int64_t M, int64_t N, int64_t K, int G, int bits) {
   const int k = aq_dispatch(M, N, K, G, bits);
   if (k < 0) return 0;
-  return workspace_for(static_cast<aq_kernel>(k), M, K);
+  return workspace_for(static_cast<aq_kernel>(k), M, N, K, bits);
 }
 
 aq_status aq_matmul_ws(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
@@ -378,12 +380,12 @@ aq_status aq_matmul_ws(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
   aq_kernel kernel = AQ_KERNEL_AUTO;
   aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
   if (st != AQ_OK) return st;
-  const size_t need = workspace_for(kernel, M, K);
+  const size_t need = workspace_for(kernel, M, N, K, bits);
   if (need > 0) {
     if (!workspace || workspace_bytes < need) return AQ_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return AQ_ERR_ALIGNMENT;
   }
-  return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, workspace, stream);
+  return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, workspace, workspace_bytes, stream);
 }
 
 aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
@@ -391,14 +393,14 @@ aq_status aq_matmul_with(aq_kernel kernel, const uint16_t *x, int64_t M, int64_t
                          aq_stream_t stream) {
   aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
   if (st != AQ_OK) return st;
-  const size_t need = workspace_for(kernel, M, K);
-  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream);
+  const size_t need = workspace_for(kernel, M, N, K, bits);
+  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, 0, stream);
   if ((st = check_device()) != AQ_OK) return st;
   // workspace from the library's stream-ordered pool, released on the same stream
   void *ws = nullptr;
   cudaError_t e = ws_alloc(&ws, need, stream);
   if (e != cudaSuccess) return from_cuda(e);
-  st = matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, ws, stream);
+  st = matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, ws, need, stream);
   e = cudaFreeAsync(ws, stream);
   if (st == AQ_OK && e != cudaSuccess) st = from_cuda(e);
   return st;
@@ -416,8 +418,8 @@ aq_status aq_matmul_ex(const uint16_t *x, int64_t M, int64_t K, const uint32_t *
   aq_kernel kernel = AQ_KERNEL_AUTO;
   aq_status st = matmul_prepare(kernel, x, M, K, packed, scales, biases, N, G, bits, y);
   if (st != AQ_OK) return st;
-  const size_t need = workspace_for(kernel, M, K);
-  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, stream, flags);
+  const size_t need = workspace_for(kernel, M, N, K, bits);
+  if (need == 0) return matmul_run(kernel, x, M, K, packed, scales, biases, N, G, bits, y, nullptr, 0, stream, flags);
   return aq_matmul_with(kernel, x, M, K, packed, scales, biases, N, G, bits, y, stream);
 }
 
@@ -533,7 +535,7 @@ aq_status aq_gather_matmul_grouped(const uint16_t *x, int64_t T, int64_t K, cons
     if (cnt <= 0) continue;
     const aq_kernel k = static_cast<aq_kernel>(aq_dispatch(cnt, N, K, G, bits));
     st = matmul_run(k, xs + o * K, cnt, K, packed + ex * N * P, scales + ex * N * Gn, biases + ex * N * Gn, N, G, bits,
-                    ys + o * N, qws, stream);
+                    ys + o * N, qws, b_ws, stream);
   }
   if (st == AQ_OK) st = from_cuda(aq::launch_scatter_rows(ys, T, N, pos, experts, E, y, stream));
   e = cudaFreeAsync(ws, stream);

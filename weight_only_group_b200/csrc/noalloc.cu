@@ -21,7 +21,8 @@
 
 namespace aq {
 cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s);
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, size_t ws_bytes,
+                       cudaStream_t s);
 size_t qmm_workspace_bytes(int64_t M, int64_t K);
 bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits);
 aq_status api_from_cuda(cudaError_t e);
@@ -123,7 +124,10 @@ extern "C" aq_status aq_matmul_qmm_static(const uint16_t *x_bf16, int64_t M, int
   cudaError_t e = cudaSuccess;
   void *ws = static_workspace_address(&e);
   if (ws == nullptr) return aq::api_from_cuda(e);
-  // The pre-pass writes every byte of the workspace that the matmul then reads,
-  // so nothing left over from an earlier call needs clearing.
-  return aq::api_from_cuda(aq::launch_qmm(x_bf16, M, K, packed, scales, biases, N, G, bits, y_bf16, ws, stream));
+  // The pre-pass writes (or clears) every byte of the workspace that the matmul
+  // reads before writing it, so nothing left over from an earlier call matters.
+  // A K-split launch also needs room for its partial sums after the
+  // activations; without it the launch runs unsplit.
+  return aq::api_from_cuda(aq::launch_qmm(x_bf16, M, K, packed, scales, biases, N, G, bits, y_bf16, ws,
+                                          AQ_QMM_STATIC_WORKSPACE_BYTES, stream));
 }

@@ -117,6 +117,14 @@ struct Params {
   const uint8_t *bscales;
   int sb_row;
   const float *gscale;
+  // K split of the CTA-pair kernel: each tile's K blocks are cut into ksplit
+  // contiguous parts, one work item each (tile w % tiles, part w / tiles for
+  // item w).  Every part writes its fp32 sums to `partial`; the part that
+  // arrives last on the tile's counters (`arrivals`, zeroed by the pre-pass)
+  // adds the parts in part order and writes y.
+  int ksplit = 1;
+  float *partial = nullptr;
+  uint32_t *arrivals = nullptr;
 };
 
 // One tile of a launch: its first token row and first W row in the maps, the
@@ -529,12 +537,45 @@ template <int N>
 AQ_DEVICE void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
 AQ_DEVICE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// The work items of one CTA pair: items pair, pair + npairs, ... of the
+// launch, item w being K part w / tiles of tile w % tiles.
+struct PairItem {
+  int tile, kb0, kb1;  // tile index (tile_origin) and its K blocks [kb0, kb1)
+  int part;            // K part of the tile (0 .. ksplit - 1)
+};
+template <bool SPLIT>
+struct PairCursor {
+  uint32_t w, P, T, KB, ks;
+  AQ_DEVICE PairCursor(const Params &prm, int pair, int npairs, int KB_)
+      : w(pair), P(npairs), T(prm.m_tiles * prm.n_tiles), KB(KB_), ks(SPLIT ? prm.ksplit : 1) {}
+  AQ_DEVICE bool next(PairItem &it) {
+    if constexpr (!SPLIT) {
+      if (w >= T) return false;
+      it.tile = static_cast<int>(w);
+      it.part = 0;
+      it.kb0 = 0;
+      it.kb1 = static_cast<int>(KB);
+      w += P;
+      return true;
+    }
+    if (w >= T * ks) return false;
+    const uint32_t part = w / T;
+    it.tile = static_cast<int>(w - part * T);
+    it.part = static_cast<int>(part);
+    it.kb0 = static_cast<int>(part * KB / ks);  // (KB * ks < 2^32: the host caps ks at 4)
+    it.kb1 = static_cast<int>((part + 1) * KB / ks);
+    w += P;
+    return true;
+  }
+};
+
 // kind::f16 instruction descriptor: fp32 accumulator, fp16 A and B, both K-major, M = 256, N = bn.
 __host__ __device__ constexpr uint32_t idesc_pair(int bn) {
   return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-template <int BITS, int BN>
+// SPLIT: the launch cuts tiles into K parts (Params::ksplit > 1).
+template <int BITS, int BN, bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     qmm_pair_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map,
                     const __grid_constant__ CUtensorMap y_map, Params prm) {
@@ -553,7 +594,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
-  const int total_tiles = prm.m_tiles * prm.n_tiles;
   const int KB = (prm.K + C::BK - 1) / C::BK;
 
   if (threadIdx.x == 0) {
@@ -586,12 +626,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&w_map)) : "memory");
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = pair; tile < total_tiles && ok; tile += npairs) {
+      PairCursor<SPLIT> cur(prm, pair, npairs, KB);
+      PairItem item;
+      while (ok && cur.next(item)) {
         int m0, n0;
-        tile_origin(prm, tile, BN, 256, m0, n0);
+        tile_origin(prm, item.tile, BN, 256, m0, n0);
         const int xrow = m0 + static_cast<int>(rank) * C::XH;
         const int wrow = n0 + static_cast<int>(rank) * 128;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kb = item.kb0; kb < item.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t r = it / S;
           if (r >= 1 && !(ok = mbar_wait_cluster(&empty[s], (r - 1) & 1, abort_flag, kFaultProducerWait))) break;
@@ -614,10 +656,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_pair(BN);
       uint32_t it = 0, t = 0;
       bool ok = true;
-      for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++t) {
+      PairCursor<SPLIT> cur(prm, pair, npairs, KB);
+      PairItem item;
+      for (; ok && cur.next(item); ++t) {
+        const int kb0 = item.kb0;
         if (t >= 1 && !(ok = mbar_wait_cluster(acc_empty, (t - 1) & 1, abort_flag, kFaultMmaWait))) break;
         tc_fence_after();
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kb = kb0; kb < item.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t r = it / S;
           // a_full: both CTAs' A stages are written, and each dequant warp saw its CTA's stage land
@@ -629,7 +674,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < C::BK / 16; ++kk) {
             const uint32_t b_addr = xs_addr + (kk / 4) * C::XH * 128 + (kk % 4) * 32;
             tc_mma_pair(tmem_base + kAccCol, a_tmem + kk * 8, sw128_kmajor_desc(b_addr), idesc,
-                        (kb > 0 || kk > 0) ? 1u : 0u);
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[s]);
         }
@@ -644,12 +689,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     constexpr int H = kDequantPerQuadrant;
     const int row = q * 32 + lane;
     constexpr int CH = C::BK / 32;
-    uint8_t *ebox = smem + S * C::STAGE_BYTES + 512 + (warp - kDequantWarp0) * 2048;  // this warp's output box
+    const int widx = warp - kDequantWarp0;
+    uint8_t *ebox = smem + S * C::STAGE_BYTES + 512 + widx * 2048;  // this warp's output box
     uint32_t it0 = 0, t = 0;
     bool ok = true;
-    for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++t, it0 += KB) {
+    PairCursor<SPLIT> cur(prm, pair, npairs, KB);
+    PairItem item;
+    for (; ok && cur.next(item); ++t) {
+      const int tile = item.tile, kb0 = item.kb0, kb1 = item.kb1;
       int m0, n0;
       tile_origin(prm, tile, BN, 256, m0, n0);
+      const uint32_t itb = it0;  // ring position of this item's first K block
+      it0 += static_cast<uint32_t>(kb1 - kb0);
       const int n = n0 + static_cast<int>(rank) * 128 + row;
       const bool row_ok = n < prm.N;
       const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
@@ -657,7 +708,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
           const int g = (kb * C::BK + c * 32) / prm.G;
-          const bool in = row_ok && kb < KB && g < prm.Gn;
+          const bool in = row_ok && kb < kb1 && g < prm.Gn;
           sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
           bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
         }
@@ -666,9 +717,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // (static indices keep it in registers)
       uint16_t sc_pf[kSbAhead][CH], bi_pf[kSbAhead][CH];
 #pragma unroll
-      for (int i = 0; i < kSbAhead; ++i) load_sb(h + i * H, sc_pf[i], bi_pf[i]);
-      for (int kb = h; kb < KB; kb += H) {
-        const uint32_t it = it0 + kb;
+      for (int i = 0; i < kSbAhead; ++i) load_sb(kb0 + h + i * H, sc_pf[i], bi_pf[i]);
+      for (int kb = kb0 + h; kb < kb1; kb += H) {
+        const uint32_t it = itb + static_cast<uint32_t>(kb - kb0);
         const int s = it % S;
         const uint32_t r = it / S;
         uint16_t sc[CH], bi[CH];
@@ -693,21 +744,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t a_tmem = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::A_COL0 + s * C::A_COLS;
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          uint32_t w[BITS];
+          uint32_t wv[BITS];
           if constexpr (BITS == 4) {
             const uint4 v4 = *reinterpret_cast<const uint4 *>(wrow + c * 4);
-            w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
+            wv[0] = v4.x; wv[1] = v4.y; wv[2] = v4.z; wv[3] = v4.w;
           } else if constexpr (BITS == 8) {
             const uint4 a4 = reinterpret_cast<const uint4 *>(wrow + c * 8)[0];
             const uint4 b4 = reinterpret_cast<const uint4 *>(wrow + c * 8)[1];
-            w[0] = a4.x; w[1] = a4.y; w[2] = a4.z; w[3] = a4.w;
-            w[4] = b4.x; w[5] = b4.y; w[6] = b4.z; w[7] = b4.w;
+            wv[0] = a4.x; wv[1] = a4.y; wv[2] = a4.z; wv[3] = a4.w;
+            wv[4] = b4.x; wv[5] = b4.y; wv[6] = b4.z; wv[7] = b4.w;
           } else {
 #pragma unroll
-            for (int i = 0; i < BITS; ++i) w[i] = wrow[c * BITS + i];
+            for (int i = 0; i < BITS; ++i) wv[i] = wrow[c * BITS + i];
           }
           uint32_t packed_cols[16];
-          dequant_chunk_f16<BITS>(w, sc[c], bi[c], packed_cols);
+          dequant_chunk_f16<BITS>(wv, sc[c], bi[c], packed_cols);
           tmem_st16(a_tmem + c * 16, packed_cols);
         }
         tmem_st_wait();
@@ -720,35 +771,106 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait_cluster(acc_full, t & 1, abort_flag, kFaultEpilogueWait))) break;
       __syncwarp();
       tc_fence_after();
-      // Each 32-column block: this warp's 32 rows x 32 tokens, scaled and
-      // rounded into a shared-memory box (token-major, the layout of y) and
-      // written by one TMA store, which clips rows past N and tokens past M.
-#pragma unroll 1
-      for (int col = h * 32; col < BN; col += H * 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + col, v);
+      const int bn0 = n0 + static_cast<int>(rank) * 128 + q * 32;
+      // Row scale of token m0 + col + lane (the lane's token in a 32-column block).
+      auto load_rs = [&](int col) {
         const int mlane = m0 + col + lane;
-        const float rs = mlane < prm.M ? __ldg(prm.row_scale + mlane) : 0.0f;  // token col + lane's scale
-        tmem_ld_wait();
-        uint8_t *box = ebox;
+        return mlane < prm.M ? __ldg(prm.row_scale + mlane) : 0.0f;
+      };
+      // One 32-column block: this warp's 32 rows x 32 tokens (v, fp32 sums of
+      // lane `lane`'s row), scaled and rounded into a shared-memory box
+      // (token-major, the layout of y) and written by one TMA store, which
+      // clips rows past N and tokens past M.
+      auto emit_box = [&](int col, const float (&v)[32], float rs) {
         if (lane == 0) bulk_wait_read<0>();  // the store that last read this box is done with it
         __syncwarp();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float r = __shfl_sync(0xffffffffu, rs, i);
-          *reinterpret_cast<__nv_bfloat16 *>(box + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]) * r);
+          const float rsi = __shfl_sync(0xffffffffu, rs, i);
+          *reinterpret_cast<__nv_bfloat16 *>(ebox + i * 64 + lane * 2) = __float2bfloat16_rn(v[i] * rsi);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the copy engine reads the box
         __syncwarp();
-        const int bn0 = n0 + static_cast<int>(rank) * 128 + q * 32;
         if (lane == 0 && bn0 < prm.N && m0 + col < prm.M) {  // (a box wholly past the edges is not stored)
-          tma_store_2d(&y_map, box, bn0, m0 + col);
+          tma_store_2d(&y_map, ebox, bn0, m0 + col);
           bulk_commit();
         }
+      };
+      if constexpr (!SPLIT) {
+#pragma unroll 1
+        for (int col = h * 32; col < BN; col += H * 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + col, v);
+          const float rs = load_rs(col);  // (in flight with the accumulator read)
+          tmem_ld_wait();
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+          emit_box(col, f, rs);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_at(acc_empty, 0);
+      } else {
+        // This part's sums of the warp's blocks go to `partial`, which frees
+        // the accumulator; the warp that arrives last on this (tile, CTA,
+        // warp) counter adds every part's sums in part order, so the result
+        // does not depend on which part finished last.  Layout: [part][tile]
+        // [CTA][quadrant][32-token block] chunks of 32 rows x 32 tokens, each
+        // as [token / 4][row][token % 4], so that one float4 store or load of
+        // the warp covers 512 contiguous bytes.
+        const int T = prm.m_tiles * prm.n_tiles;
+        auto chunk = [&](int part, int col) {
+          return reinterpret_cast<float4 *>(prm.partial) +
+                 ((((static_cast<int64_t>(part) * T + tile) * 2 + rank) * 4 + q) * (BN / 32) + col / 32) * 256 + lane;
+        };
+#pragma unroll 1
+        for (int col = h * 32; col < BN; col += H * 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + col, v);
+          tmem_ld_wait();
+          float4 *dst = chunk(item.part, col);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            __stcg(dst + i * 32, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])));
+        }
+        tc_fence_before();
+        __syncwarp();  // (also: every lane's partial sums are written)
+        uint32_t before = 0;
+        if (lane == 0) {
+          mbar_arrive_at(acc_empty, 0);
+          __threadfence();  // the warp's partial sums are visible before its count (a cumulative fence)
+          before = atomicAdd(prm.arrivals + (tile * 2 + static_cast<int>(rank)) * (4 * H) + widx, 1u);
+          // the last part: the other parts' counts seen here order their sums before the reads below
+          if (before == static_cast<uint32_t>(prm.ksplit - 1)) __threadfence();
+        }
+        before = __shfl_sync(0xffffffffu, before, 0);
+        __syncwarp();
+        if (before == static_cast<uint32_t>(prm.ksplit - 1)) {
+#pragma unroll 1
+          for (int col = h * 32; col < BN; col += H * 32) {
+            const float rs = load_rs(col);
+            float v[32];
+#pragma unroll 1
+            for (int k = 0; k < prm.ksplit; ++k) {  // in part order
+              const float4 *src = chunk(k, col);
+              float4 f[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] = __ldcg(src + i * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                if (k == 0) {
+                  v[4 * i] = f[i].x; v[4 * i + 1] = f[i].y; v[4 * i + 2] = f[i].z; v[4 * i + 3] = f[i].w;
+                } else {
+                  v[4 * i] += f[i].x; v[4 * i + 1] += f[i].y; v[4 * i + 2] += f[i].z; v[4 * i + 3] += f[i].w;
+                }
+              }
+            }
+            emit_box(col, v, rs);
+          }
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_at(acc_empty, 0);
     }
     if (lane == 0) bulk_wait_all();  // this warp's output stores have completed
   }
@@ -776,9 +898,13 @@ constexpr int kPrepThreads = 256;
 template <int BITS>
 __global__ void __launch_bounds__(kPrepThreads) x_to_f16_rows_kernel(const __nv_bfloat16 *__restrict__ x, int K,
                                                                      __half *__restrict__ x16,
-                                                                     float *__restrict__ row_scale) {
+                                                                     float *__restrict__ row_scale,
+                                                                     uint32_t *__restrict__ zero = nullptr,
+                                                                     int nzero = 0) {
   __shared__ float red[kPrepThreads / 32];
   const int64_t m = blockIdx.x;
+  if (m == 0)  // counters of the matmul that follows
+    for (int i = threadIdx.x; i < nzero; i += kPrepThreads) zero[i] = 0;
   const uint4 *src = reinterpret_cast<const uint4 *>(x + m * K);
   const int n16 = K / 16;  // 16-element steps (K is a multiple of 32)
   float amax = 0.0f;
@@ -835,6 +961,44 @@ __global__ void __launch_bounds__(kPrepThreads) x_to_f16_rows_kernel(const __nv_
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+inline int64_t round256(int64_t b) { return (b + 255) / 256 * 256; }
+
+// The activations' workspace: x16 (fp16 [M, K]) + row_scale (fp32 [M]), each 256-byte padded.
+inline size_t x16_bytes(int64_t M, int64_t K) { return static_cast<size_t>(round256(M * K * 2) + round256(M * 4)); }
+
+// CTA-pair tiles (256 W rows x 256 tokens) of an M x N product.
+inline int64_t pair_tiles(int64_t M, int64_t N) { return ((M + 255) / 256) * ((N + 255) / 256); }
+
+// The pair kernel serves every M > 128 whose y rows are whole 16-byte units.
+inline bool pick_shape_is_pair(int64_t M, int64_t N) { return M > 128 && N % 8 == 0; }
+
+// K parts per tile of a pair launch.  When the tiles fill at most half of the
+// 74 CTA pairs of a 148-SM part, each tile's K range is cut into up to four
+// parts (one work item each, at least 32 K blocks per part), so that more
+// pairs work; the parts' fp32 sums meet in the workspace.  (Sharing out only
+// the last wave's tiles among all pairs, "stream-K", measured slower here: a
+// shared tile costs its pairs ~4 us to publish their sums and the last one
+// 6-8 us to add them, more than the idle pairs of a last wave cost.)  The
+// choice depends on the shape alone, so the workspace size is known before
+// the launch.
+inline int pair_ksplit(int64_t M, int64_t N, int64_t K, int bits) {
+  constexpr int64_t kPairs = 74;
+  const int64_t T = pair_tiles(M, N);
+  const int64_t KB = (K + (bits == 3 ? 127 : 63)) / (bits == 3 ? 128 : 64);
+  const int64_t ks = std::min<int64_t>(std::min<int64_t>(kPairs / T, 4), KB / 32);
+  return ks >= 2 ? static_cast<int>(ks) : 1;
+}
+
+// Workspace bytes of the split beyond the activations' part: one arrival
+// counter per (tile, CTA, dequant warp), 256-byte padded, then [ksplit][tile]
+// [CTA][128 rows][256 tokens] fp32 partial sums.
+inline size_t pair_split_bytes(int64_t M, int64_t N, int64_t K, int bits) {
+  const int ks = pair_ksplit(M, N, K, bits);
+  if (ks == 1) return 0;
+  const int64_t T = pair_tiles(M, N);
+  return static_cast<size_t>(round256(T * 2 * 4 * kDequantPerQuadrant * 4) + ks * T * 2 * 128 * 256 * 4);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1078,14 +1242,24 @@ cudaError_t launch_grouped_t(const uint16_t *x, int64_t T, int64_t K, const uint
 
 template <int BITS, int BN>
 cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                        const uint16_t *biases, int64_t N, int G, uint16_t *y, void *workspace, cudaStream_t stream) {
+                        const uint16_t *biases, int64_t N, int G, uint16_t *y, void *workspace, size_t ws_bytes,
+                        cudaStream_t stream) {
   using C = PairCfg<BITS, BN>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  __half *x16 = reinterpret_cast<__half *>(workspace);
-  float *row_scale = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) + ((M * K * 2 + 255) / 256) * 256);
+  uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+  __half *x16 = reinterpret_cast<__half *>(ws);
+  float *row_scale = reinterpret_cast<float *>(ws + round256(M * K * 2));
+  // the K split, when the caller's workspace holds its counters and partial sums
+  static_assert(BN == 256, "the split's workspace is sized for 256-token tiles");
+  int ksplit = pair_ksplit(M, N, K, BITS);
+  const size_t base = x16_bytes(M, K);
+  if (ksplit > 1 && ws_bytes < base + pair_split_bytes(M, N, K, BITS)) ksplit = 1;
+  uint32_t *arrivals = ksplit > 1 ? reinterpret_cast<uint32_t *>(ws + base) : nullptr;
+  const int n_arrivals = ksplit > 1 ? static_cast<int>(pair_tiles(M, N) * 2 * 4 * kDequantPerQuadrant) : 0;
+  float *partial = ksplit > 1 ? reinterpret_cast<float *>(ws + base + round256(int64_t(n_arrivals) * 4)) : nullptr;
   x_to_f16_rows_kernel<BITS><<<static_cast<unsigned>(M), kPrepThreads, 0, stream>>>(
-      reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale);
+      reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale, arrivals, n_arrivals);
   cudaError_t pe = cudaGetLastError();
   if (pe != cudaSuccess) return pe;
   CUtensorMap x_map, w_map;
@@ -1142,21 +1316,25 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
 #ifdef AQ_QMM_FORCE_ORDER
   if (AQ_QMM_FORCE_ORDER == 0 || AQ_QMM_FORCE_ORDER == 1) prm.n_fastest = AQ_QMM_FORCE_ORDER;
 #endif
+  prm.ksplit = ksplit;
+  prm.partial = partial;
+  prm.arrivals = arrivals;
 
-  auto kern = qmm_pair_kernel<BITS, BN>;
+  auto kern = ksplit > 1 ? qmm_pair_kernel<BITS, BN, true> : qmm_pair_kernel<BITS, BN, false>;
   static thread_local int cached_dev = -1;
   static thread_local int sms = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev != cached_dev) {
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
-      return e;
+    for (auto k : {qmm_pair_kernel<BITS, BN, true>, qmm_pair_kernel<BITS, BN, false>})
+      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
+        return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     cached_dev = dev;
   }
-  const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
-  const int pairs = static_cast<int>(std::min<int64_t>(tiles, std::max(1, sms / 2)));
+  const int64_t items = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles * ksplit;
+  const int pairs = static_cast<int>(std::min<int64_t>(items, std::max(1, sms / 2)));
   kern<<<2 * pairs, kThreads, C::SMEM_BYTES, stream>>>(x_map, w_map, y_map, prm);
   return cudaGetLastError();
 }
@@ -1175,7 +1353,7 @@ int pick_shape(int64_t M, int64_t N, int sms) {
 #ifdef AQ_QMM_FORCE_SHAPE  // build-time override (0..3 as in Shape; else choose)
   if (AQ_QMM_FORCE_SHAPE >= 0 && AQ_QMM_FORCE_SHAPE <= 3) return AQ_QMM_FORCE_SHAPE;
 #endif
-  if (M > 128 && N % 8 == 0) return kPair256;  // (the pair's output stores need 16-byte rows of y)
+  if (pick_shape_is_pair(M, N)) return kPair256;  // (the pair's output stores need 16-byte rows of y)
   auto score = [&](int64_t bn, int64_t bytes) {
     const int64_t t = ((M + bn - 1) / bn) * ((N + 127) / 128);
     const int64_t waves = (t + sms - 1) / sms;
@@ -1192,7 +1370,8 @@ int pick_shape(int64_t M, int64_t N, int sms) {
 
 template <int BITS>
 cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                        const uint16_t *biases, int64_t N, int G, uint16_t *y, void *ws, cudaStream_t s) {
+                        const uint16_t *biases, int64_t N, int G, uint16_t *y, void *ws, size_t ws_bytes,
+                        cudaStream_t s) {
   static thread_local int cached_dev = -1, sms = 148;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1202,7 +1381,7 @@ cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
     cached_dev = dev;
   }
   switch (pick_shape<BITS>(M, N, sms)) {
-    case kPair256: return launch_pair<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case kPair256: return launch_pair<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, ws_bytes, s);
     case kOne256: return launch_t<BITS, 256>(x, M, K, packed, scales, biases, N, G, y, ws, s);
     case kOne128: return launch_t<BITS, 128>(x, M, K, packed, scales, biases, N, G, y, ws, s);
     default: return launch_t<BITS, 64>(x, M, K, packed, scales, biases, N, G, y, ws, s);
@@ -1265,18 +1444,24 @@ bool qmm_supports(int64_t M, int64_t N, int64_t K, int G, int bits) {
   return true;
 }
 
-// Workspace of the QMM path: x16 (fp16 [M, K], 256-byte padded) + row_scale (fp32 [M]).
-size_t qmm_workspace_bytes(int64_t M, int64_t K) {
-  return static_cast<size_t>((M * K * 2 + 255) / 256 * 256) + static_cast<size_t>((M * 4 + 255) / 256 * 256);
+// Workspace of the QMM paths' activations: x16 (fp16 [M, K]) + row_scale (fp32 [M]).
+size_t qmm_workspace_bytes(int64_t M, int64_t K) { return qmm::x16_bytes(M, K); }
+
+// Workspace of the affine QMM path: the activations' part plus, for a
+// K-split CTA-pair launch, its counters and fp32 partial sums.
+size_t qmm_workspace_bytes(int64_t M, int64_t N, int64_t K, int bits) {
+  return qmm_workspace_bytes(M, K) + (qmm::pick_shape_is_pair(M, N) ? qmm::pair_split_bytes(M, N, K, bits) : 0);
 }
 
+// ws_bytes: the workspace's size; the K split runs only when it holds that part too.
 cudaError_t launch_qmm(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
-                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, cudaStream_t s) {
+                       const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, void *ws, size_t ws_bytes,
+                       cudaStream_t s) {
   switch (bits) {
-    case 2: return qmm::launch_bits<2>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-    case 3: return qmm::launch_bits<3>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-    case 4: return qmm::launch_bits<4>(x, M, K, packed, scales, biases, N, G, y, ws, s);
-    default: return qmm::launch_bits<8>(x, M, K, packed, scales, biases, N, G, y, ws, s);
+    case 2: return qmm::launch_bits<2>(x, M, K, packed, scales, biases, N, G, y, ws, ws_bytes, s);
+    case 3: return qmm::launch_bits<3>(x, M, K, packed, scales, biases, N, G, y, ws, ws_bytes, s);
+    case 4: return qmm::launch_bits<4>(x, M, K, packed, scales, biases, N, G, y, ws, ws_bytes, s);
+    default: return qmm::launch_bits<8>(x, M, K, packed, scales, biases, N, G, y, ws, ws_bytes, s);
   }
 }
 
