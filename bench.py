@@ -387,6 +387,8 @@ def compact_sections(sec):
         out["decode_shapes_GBps"] = {k: v["weight_GBps"] for k, v in sec["decode_shapes"].items()}
     if "qmv_small_m" in sec:
         out["small_m_GBps"] = {k: v["weight_GBps"] for k, v in sec["qmv_small_m"]["curve"].items()}
+    if "qmv_small_m_long_k" in sec:
+        out["small_m_long_k_GBps"] = {k: v["weight_GBps"] for k, v in sec["qmv_small_m_long_k"]["curve"].items()}
     if "qmv_bits_group_sweep" in sec:
         out["sweep_GBps"] = {k: v["weight_GBps"] for k, v in sec["qmv_bits_group_sweep"]["points"].items()}
     if "decode_sequence" in sec:
@@ -703,6 +705,25 @@ def section_curve(args, aq, torch, dev, stream, peaks):
                          "frac_hbm": round(wb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                          "kernel": ["qmv", "qmm"][aq.aq_dispatch(M, N, K, G, BITS) - 1]}
     out["qmv_small_m"] = {"K": K, "N": N, "bits": BITS, "G": G, "curve": curve}
+    del ws, base
+    torch.cuda.empty_cache()
+    # ---- the same curve at a long K (K=14336, N=4096: M > 4 runs as token chunks of one launch each)
+    K, N = 14336, 4096
+    w = torch.from_numpy(synth.weights(N, K, 1000 + 100 * 3 + 1)).to(dev)
+    base = aq.aq_quantize(w, G, BITS)
+    del w
+    wb = weight_bytes(K, N)
+    copies = max(2, -(-2 * L2_BYTES // wb) + 1)
+    ws = [base] + [tuple(t.clone() for t in base) for _ in range(copies - 1)]
+    curve = {}
+    for M in (1, 2, 3, 4, 5, 6, 8):
+        x = synth.activations(M, K, 12).to(dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, *ws[i % copies], G, BITS, out=y,
+                                                               overlap_previous=True), copies * 8, 20)
+        curve[str(M)] = {"us": round(ms * 1e3, 3), "weight_GBps": round(wb / (ms * 1e-3) / 1e9, 1),
+                         "frac_hbm": round(wb / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    out["qmv_small_m_long_k"] = {"K": K, "N": N, "bits": BITS, "G": G, "curve": curve}
     del ws, base
     torch.cuda.empty_cache()
     return out

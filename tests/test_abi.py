@@ -83,8 +83,12 @@ def test_dispatch_rule():
     assert aq.aq_dispatch(1, 28672, 8192, 32, 3) == aq.AQ_KERNEL_QMV
     for M in (9, 64, 512, 8192):
         assert aq.aq_dispatch(M, 14336, 4096, 64, 4) == aq.AQ_KERNEL_QMM
-    # x staging for QMV would not fit shared memory: QMM takes it
-    assert aq.aq_dispatch(8, 4096, 14336, 64, 4) == aq.AQ_KERNEL_QMM
+    # many tokens over a long K: the decode kernel in token chunks (staged x of a
+    # launch within 120 KB: 4 tokens at K = 14336), not the prefill kernel
+    for M in range(1, 9):
+        assert aq.aq_dispatch(M, 4096, 14336, 64, 4) == aq.AQ_KERNEL_QMV
+    # 3-bit codes have no tensor-core decode; beyond its CUDA-core kernel's shared memory: QMM
+    assert aq.aq_dispatch(8, 200, 14336, 32, 3) == aq.AQ_KERNEL_QMM
     # invalid shapes
     assert aq.aq_dispatch(0, 4096, 4096, 64, 4) == -1
     assert aq.aq_dispatch(1, 4096, 4000, 64, 4) == -1

@@ -526,6 +526,16 @@ def test_qmv_tensor_core_tiles(M, bits, G):
     _matmul_case(M, K, N, bits, G, 9100 + G + bits, "qmv")
 
 
+@pytest.mark.parametrize("M", (5, 6, 7, 8))
+@pytest.mark.parametrize("bits,G", [(4, 64), (2, 32), (8, 128)])
+def test_qmv_many_tokens_long_k(M, bits, G):
+    """Decode with many tokens over a long K (the staged activations would crowd
+    the weight ring out of shared memory) runs the tokens in balanced chunks,
+    one launch each; every token's row matches the oracle."""
+    _matmul_case(M, 14336, 200, bits, G, 9500 + M + bits, "auto")
+    assert aq.aq_dispatch(M, 200, 14336, G, bits) == aq.AQ_KERNEL_QMV
+
+
 def test_qmv_extreme_activation_rows():
     """Rows far outside fp16 range, a row of tiny values, an all-zero row and a
     single 3e38 element: the per-group power-of-two scaling keeps them exact in

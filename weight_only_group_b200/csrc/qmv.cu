@@ -645,8 +645,28 @@ cudaError_t launch_qmv_tc(const uint16_t *x, int64_t M, int64_t K, const uint32_
 
 size_t qmv_required_smem(int64_t M, int64_t K) { return qmv_smem_bytes(static_cast<int>(M), static_cast<int>(K)); }
 
+// Tokens of one tensor-core decode launch at most, by the shared memory their
+// staged activations take (2K + 64 bytes each): past ~120 KB the weight ring
+// left beside them is too shallow to keep HBM busy (measured at K = 14336, N =
+// 4096, 4-bit G64: 653 GB/s at M = 5, against 1281 at M = 4), and past ~200 KB
+// the launch does not fit at all.
+constexpr int64_t kDecodeActBytes = 120 * 1024;
+
+// Launches of a decode over M tokens: one, or balanced chunks of at most
+// kDecodeActBytes of staged activations each (0 when a chunk has no
+// tensor-core plan).  Chunk c is tokens [c * M / n, (c + 1) * M / n).
+int64_t decode_chunks(int64_t M, int64_t N, int64_t K, int G, int bits) {
+  const int64_t per_launch = std::max<int64_t>(1, kDecodeActBytes / (2 * K + 64));
+  if (M <= per_launch) return 1;
+  const int64_t n = (M + per_launch - 1) / per_launch;
+  for (int64_t c = 0; c < n; ++c)
+    if (!qmv_tc_supported((c + 1) * M / n - c * M / n, N, K, G, bits)) return 0;
+  return n;
+}
+
 bool qmv_supported(int64_t M, int64_t N, int64_t K, int G, int bits) {
   if (M < 1 || M > 8) return false;
+  if (decode_chunks(M, N, K, G, bits) > 1) return true;
   if (qmv_tc_supported(M, N, K, G, bits)) return true;
   StreamPlan pl;
   if (plan_stream(M, N, K, G, bits, 148, pl)) return true;
@@ -662,6 +682,18 @@ cudaError_t read_and_clear_qmv_fault(uint32_t *word) {
 
 cudaError_t launch_qmv(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                        const uint16_t *biases, int64_t N, int G, int bits, uint16_t *y, uint32_t flags, cudaStream_t s) {
+  // Many tokens over a long K: run them in balanced chunks, one launch each
+  // (stream-ordered; the weights of the later chunks come mostly from L2).
+  const int64_t chunks = decode_chunks(M, N, K, G, bits);
+  if (chunks > 1) {
+    for (int64_t c = 0; c < chunks; ++c) {
+      const int64_t m0 = c * M / chunks, m1 = (c + 1) * M / chunks;
+      const cudaError_t e =
+          launch_qmv_tc(x + m0 * K, m1 - m0, K, packed, scales, biases, N, G, bits, y + m0 * N, flags, s);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   if (qmv_tc_supported(M, N, K, G, bits))
     return launch_qmv_tc(x, M, K, packed, scales, biases, N, G, bits, y, flags, s);
   switch (bits) {
