@@ -187,7 +187,9 @@ typedef struct {
  * "Mechanics": QMV streams each weight once per decode step; several linears
  * run back to back).  Computes calls[j] for j = 0 .. n-1 (1 <= n <= 4) in
  * order, all with the same M (1..8), G and bits (2, 4 or 8), each with its own
- * N and K, with the arithmetic and accuracy of aq_matmul's tensor-core QMV.
+ * N and K, with the accuracy of aq_matmul's tensor-core QMV (each K chunk's
+ * sums are one work unit here, where aq_matmul may split a chunk in two, so
+ * the two may differ in the last bit of y).
  * Ordering: matmul j reads its x only after every element of matmul j-1's y is
  * written, so calls[j].x_bf16 may be calls[j-1].y_bf16 (a chain of linears);
  * the weights of matmul j stream while matmul j-1 finishes.  No other

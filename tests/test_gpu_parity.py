@@ -962,9 +962,10 @@ SEQ_SHAPES = [(2048, 1024), (1024, 2048), (2048, 512)]  # (K, N) of three indepe
 
 @pytest.mark.parametrize("M,G,bits", [(1, 64, 4), (2, 64, 4), (3, 128, 4), (5, 32, 8), (8, 64, 2)])
 def test_matmul_sequence_equals_single_calls(M, G, bits):
-    """Three matmuls in one launch give, bit for bit, what three aq_matmul
-    calls give (each row's arithmetic is the same), and each is within the
-    matmul tolerance of the oracle."""
+    """Three matmuls in one launch give what three aq_matmul calls give: both
+    within the matmul tolerance of the oracle.  (A sequence takes each K chunk's
+    sums as one work unit; a single call may split a chunk into two units, which
+    changes the fp32 summation order, so the two may differ in the last bit.)"""
     calls, refs = [], []
     for j, (K, N) in enumerate(SEQ_SHAPES):
         p, s, b = quantized(N, K, 9500 + j, True, G, bits)
@@ -978,8 +979,9 @@ def test_matmul_sequence_equals_single_calls(M, G, bits):
     for j, ((x, pg, sg, bg, _), (xb, p, s, b), y) in enumerate(zip(calls, refs, outs)):
         y1 = aq.aq_matmul(x, pg, sg, bg, G, bits)
         torch.cuda.synchronize()
-        assert torch.equal(y.view(torch.int16), y1.view(torch.int16)), f"matmul {j} differs from its single call"
-        _assert_close(y, oracle.matmul(xb, p, s, b, G, bits), f"sequence matmul {j}")
+        y_ref = oracle.matmul(xb, p, s, b, G, bits)
+        _assert_close(y, y_ref, f"sequence matmul {j}")
+        _assert_close(y1, y_ref, f"single call {j}")
 
 
 @pytest.mark.parametrize("M", [1, 4])

@@ -90,7 +90,10 @@ constexpr int kRedBufs = 4;         // tiles whose partial sums can be in flight
 constexpr int kDualSmem = 112 * 1024;   // shared memory of a CTA that shares its SM with the next launch's
 constexpr int kDualConsumers = 8;       // consumer warps of such a CTA
 constexpr int kDualMinStages = 4;
-constexpr int kUnitCodes = 1 << 20;     // codes of a row a work unit covers at least (where the stage allows)
+constexpr int kUnitCodes = 1 << 20;     // codes of a row a work unit covers at most: a whole stage
+#ifndef AQ_QMV_SMALL_UNIT
+#define AQ_QMV_SMALL_UNIT 1024           // codes of a row per work unit where smaller units pay (unit_codes)
+#endif
 constexpr int kMaxStages = 16;
 // Weight stages the producer keeps in flight (issued, not yet landed).  Enough
 // to cover HBM latency at an SM's share of the bandwidth; more only lengthens
@@ -1141,8 +1144,21 @@ static bool place(Plan &pl, int64_t M, int U, int64_t tok_stride, int64_t Gn, in
 // dual: the plan for two CTAs per SM (this kernel's and the next launch's, when
 // that one is a programmatic dependent): at most kDualSmem bytes of shared
 // memory and kDualConsumers consumer warps, at least kDualMinStages stages.
+// Codes of a row per work unit, for M tokens and nch K chunks per tile.  Units
+// smaller than a stage spread a CTA's last stages over more warps (a shorter
+// tail after the stream ends) and balance a CTA's few stages over its
+// consumer warps, at the price of more partial sums per tile.  Measured on
+// B200 (4-bit G64, decode chains): 1024-code units against whole stages of
+// 2048 took the Llama-3-8B decode step from 28.3 to 27.9 us and the small-M
+// curves up by 7-37% (M = 2..8, K = 4096 and 14336), except one token over
+// seven chunks per tile (K = 14336: 11.6 -> 11.9 us), which keeps whole stages.
+static int64_t unit_codes(int64_t M, int64_t nch) {
+  if (M == 1 && nch > 4) return kUnitCodes;
+  return AQ_QMV_SMALL_UNIT;
+}
+
 static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt = 0,
-                      bool dual = false, int stage_target = kStageTarget) {
+                      bool dual = false, int stage_target = kStageTarget, int64_t unit_limit = 0) {
   if (!(bits == 2 || bits == 4 || bits == 8) || !(G == 32 || G == 64 || G == 128)) return false;
   if (M < 1 || M > 8 || N < 1 || K < 1 || K % (8 * G) != 0) return false;
   // mxfp4 scale rows are K/32 bytes: a TMA row stride must be a multiple of 16 bytes
@@ -1193,19 +1209,19 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.job[0].tok_stride = static_cast<int>(2 * K + 64);
   a.zero_stride = static_cast<int>(round_up(U * 64, 128) + 64);
   // work units: fpu folds (a fold: the groups side by side above; nvfp4: twice as
-  // many 16-weight groups) of one stage, at least kUnitCodes codes of a row
-  // where the stage allows.  The kernel is issue-bound, and every unit costs a
-  // partial-sum reduction, so a unit is a whole stage (measured: units of 512
-  // codes were 17% slower on the 33 MB decode launches)
+  // many 16-weight groups) of one stage, at most unit_codes(M, nch) codes of a
+  // row.  Every unit costs a partial-sum reduction (measured: units of 512
+  // codes were 17% slower than whole stages on the 33 MB decode launches)
   // (a fold: the affine format holds 4/MP groups side by side, or one for
   // MP = 8; the block-scaled formats 8/MP)
   const int GS = 8 / MP, SPANS = fmt == 0 ? (MP >= 4 ? 1 : 4 / MP) : fmt == 2 ? GS / 2 : GS;
   const int64_t fold = static_cast<int64_t>(SPANS) * G;  // codes of a row per fold
   // folds per unit: the largest divisor of the stage's folds within kUnitCodes
   const int64_t stage_folds = Kc / fold;
+  const int64_t ucodes = unit_limit > 0 ? unit_limit : unit_codes(M, nch);
   a.job[0].fpu = 1;
   for (int64_t d = 1; d <= stage_folds; ++d)
-    if (stage_folds % d == 0 && fold * d <= kUnitCodes) a.job[0].fpu = static_cast<int>(d);
+    if (stage_folds % d == 0 && fold * d <= ucodes) a.job[0].fpu = static_cast<int>(d);
   a.nper = static_cast<int>(Kc / (fold * a.job[0].fpu));
   a.job[0].parts = static_cast<int>(nch) * a.nper;
   // tiles in flight: the units in progress (one per warp, at most
@@ -1352,8 +1368,8 @@ __device__ unsigned g_seq_bar[kSeqBarSlots][2];
 static bool make_seq_plan(int n, const int64_t *N, const int64_t *K, int64_t M, int G, int bits, int sms, Plan &pl) {
   if (n < 1 || n > kSeqMax) return false;
   Plan pj[kSeqMax];
-  for (int j = 0; j < n; ++j)
-    if (!make_plan(M, N[j], K[j], G, bits, sms, pj[j])) return false;
+  for (int j = 0; j < n; ++j)  // (whole-stage units: one unit size for the whole ring)
+    if (!make_plan(M, N[j], K[j], G, bits, sms, pj[j], 0, false, kStageTarget, kUnitCodes)) return false;
   pl = pj[0];
   Args &a = pl.a;
   a.njobs = n;
