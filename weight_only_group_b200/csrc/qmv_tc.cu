@@ -79,7 +79,7 @@ namespace tc {
 #define AQ_QMV_MAX_CONSUMERS 12
 #endif
 #ifndef AQ_QMV_INFLIGHT
-#define AQ_QMV_INFLIGHT 6
+#define AQ_QMV_INFLIGHT 10
 #endif
 #ifndef AQ_QMV_STAGE_TARGET
 #define AQ_QMV_STAGE_TARGET (16 * 1024)
@@ -98,7 +98,9 @@ constexpr int kMaxStages = 16;
 // Weight stages the producer keeps in flight (issued, not yet landed).  Enough
 // to cover HBM latency at an SM's share of the bandwidth; more only lengthens
 // the queue that every other load of the SM (activations, barrier traffic)
-// waits behind.
+// waits behind.  Measured on B200 (decode step, 4-bit G64): 4 / 6 / 8 / 10 /
+// 12 / 16 stages: 28.6 / 27.35 / 27.3 / 26.8 / 26.8 / 26.8 us (the long-K linear
+// gains; the other shapes and the small-M curves do not move from 6 up).
 constexpr int kInflight = AQ_QMV_INFLIGHT;
 constexpr int kStageTarget = AQ_QMV_STAGE_TARGET;  // packed bytes of one stage we aim for (<= 1 KB per row)
 constexpr int kAcc = 2;                  // independent accumulator chains per digit plane
