@@ -573,7 +573,7 @@ def section_mxfp4(args, aq, torch, dev, stream, peaks):
         tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
         out[f"{name}_qmm_M{M}_K{K}_N{N}"] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1),
                                              "frac_of_burst": round(tf / peaks["bf16_tflops"], 4),
-                                             "kernel": "qmm_kernel (tcgen05 kind::f16, codes dequantized to fp16)"}
+                                             "kernel": "qmm_pair_kernel (CTA pairs, tcgen05 kind::f16, codes dequantized to fp16)"}
         del q
     del w, x, y
     torch.cuda.empty_cache()

@@ -1043,7 +1043,9 @@ def test_matmul_sequence_wait_runs_out_cleanly():
 
 # ----------------------------------------------------------------------------- block-scaled prefill (M > 8)
 
-BS_PREFILL = [(9, 512, 16), (100, 1024, 100), (300, 4096, 600), (130, 2560, 2600)]
+# (K = 768: scale rows of 24 bytes (mxfp4, mxfp8) that do not start on 16-byte
+# boundaries; M > 128 with N % 8 == 0 runs on the CTA-pair kernel)
+BS_PREFILL = [(9, 512, 16), (100, 1024, 100), (300, 4096, 600), (130, 2560, 2600), (40, 768, 64), (200, 768, 264)]
 
 
 @pytest.mark.parametrize("M,K,N", BS_PREFILL)

@@ -28,7 +28,7 @@ bool qmv_tc_supported(int64_t M, int64_t N, int64_t K, int G, int bits);
 constexpr int64_t kQmmGroupMaxE = 256;  // experts of one grouped prefill launch at most
 cudaError_t launch_qmm_block_scaled(int fmt, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                                     const uint8_t *scales, const float *gscale, int64_t N, uint16_t *y, void *ws,
-                                    cudaStream_t s);
+                                    size_t ws_bytes, cudaStream_t s);
 cudaError_t launch_qmm_grouped(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed,
                                const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G, int bits,
                                const int32_t *offsets, uint16_t *y, void *ws, cudaStream_t s);
@@ -219,9 +219,10 @@ cudaError_t ws_alloc(void **p, size_t bytes, cudaStream_t s);
 cudaError_t block_scaled_prefill(int fmt, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                                  const uint8_t *scales, const float *gscale, int64_t N, uint16_t *y, cudaStream_t s) {
   void *ws = nullptr;
-  cudaError_t e = ws_alloc(&ws, aq::qmm_workspace_bytes(M, K), s);
+  const size_t bytes = aq::qmm_workspace_bytes(M, N, K, fmt == 3 ? 8 : 4);  // (with a K split's part, if any)
+  cudaError_t e = ws_alloc(&ws, bytes, s);
   if (e != cudaSuccess) return e;
-  const cudaError_t le = aq::launch_qmm_block_scaled(fmt, x, M, K, packed, scales, gscale, N, y, ws, s);
+  const cudaError_t le = aq::launch_qmm_block_scaled(fmt, x, M, K, packed, scales, gscale, N, y, ws, bytes, s);
   e = cudaFreeAsync(ws, s);
   return le != cudaSuccess ? le : e;
 }

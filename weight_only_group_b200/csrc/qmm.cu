@@ -127,6 +127,22 @@ struct Params {
   uint32_t *arrivals = nullptr;
 };
 
+// Largest byte of a row of n scale bytes (E8M0 and positive E4M3 order like
+// their bits): 16-byte loads where the row allows them, single bytes otherwise
+// (rows of K/32 bytes start on 16-byte boundaries only when K % 512 == 0).
+AQ_DEVICE uint32_t row_max_byte(const uint8_t *row, int n) {
+  uint32_t mx = 0;
+  if ((reinterpret_cast<uintptr_t>(row) & 15u) == 0 && (n & 15) == 0) {
+    for (int i = 0; i < n / 16; ++i) {
+      const uint4 v = ldg_nc16(row + 16 * i);
+      mx = __vmaxu4(mx, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
+    }
+    return max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
+  }
+  for (int i = 0; i < n; ++i) mx = max(mx, static_cast<uint32_t>(__ldg(row + i)));
+  return mx;
+}
+
 // One tile of a launch: its first token row and first W row in the maps, the
 // W row within the weight matrix (or expert), and the end of its token rows.
 struct TileRef {
@@ -306,13 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmm_kernel(const __grid_constant_
       float rowfac = 1.0f;
       if constexpr (FMT != 0) {
         sbrow = prm.bscales + static_cast<int64_t>(row_ok ? tr.wrow + row : 0) * prm.sb_row;
-        uint32_t mx = 0;
-        if (row_ok)
-          for (int i = 0; i < prm.sb_row / 16; ++i) {
-            const uint4 v = ldg_nc16(sbrow + 16 * i);
-            mx = __vmaxu4(mx, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
-          }
-        mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
+        const uint32_t mx = row_ok ? row_max_byte(sbrow, prm.sb_row) : 0u;
         if constexpr (FMT == 2) {
           const float vmax = e4m3_value(mx);
           bexp = vmax > 0.0f ? static_cast<int>((__float_as_uint(vmax) >> 23) & 0xFFu) - 127 + 1 - 13 : 0;
@@ -574,8 +584,9 @@ __host__ __device__ constexpr uint32_t idesc_pair(int bn) {
   return (1u << 4) | (static_cast<uint32_t>(bn >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-// SPLIT: the launch cuts tiles into K parts (Params::ksplit > 1).
-template <int BITS, int BN, bool SPLIT>
+// SPLIT: the launch cuts tiles into K parts (Params::ksplit > 1).  FMT as in
+// qmm_kernel: 0 affine, 1 mxfp4, 2 nvfp4, 3 mxfp8.
+template <int BITS, int BN, bool SPLIT, int FMT = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     qmm_pair_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map,
                     const __grid_constant__ CUtensorMap y_map, Params prm) {
@@ -704,13 +715,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int n = n0 + static_cast<int>(rank) * 128 + row;
       const bool row_ok = n < prm.N;
       const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
+      // Block-scaled formats: this row's power of two 2^-B (from its largest
+      // scale byte; positive E4M3 and E8M0 order like their bits) keeps every
+      // dequantized value within fp16; the epilogue multiplies by 2^B (nvfp4:
+      // and by the tensor scale).
+      const uint8_t *sbrow = nullptr;
+      int bexp = 0;
+      float rowfac = 1.0f;
+      if constexpr (FMT != 0) {
+        sbrow = prm.bscales + static_cast<int64_t>(row_ok ? n : 0) * prm.sb_row;
+        const uint32_t mx = row_ok ? row_max_byte(sbrow, prm.sb_row) : 0u;
+        if constexpr (FMT == 2) {
+          const float vmax = e4m3_value(mx);
+          bexp = vmax > 0.0f ? static_cast<int>((__float_as_uint(vmax) >> 23) & 0xFFu) - 127 + 1 - 13 : 0;
+          rowfac = pow2f_exact(bexp) * __ldg(prm.gscale);
+        } else {
+          bexp = static_cast<int>(mx) - 127 - (FMT == 1 ? 13 : 7);
+          rowfac = pow2f_exact(bexp);
+        }
+      }
       auto load_sb = [&](int kb, uint16_t (&sc)[CH], uint16_t (&bi)[CH]) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          const int g = (kb * C::BK + c * 32) / prm.G;
-          const bool in = row_ok && kb < kb1 && g < prm.Gn;
-          sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
-          bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
+          if constexpr (FMT == 0) {
+            const int g = (kb * C::BK + c * 32) / prm.G;
+            const bool in = row_ok && kb < kb1 && g < prm.Gn;
+            sc[c] = in ? ldg_nc2(prm.scales + g_row + g) : uint16_t(0);
+            bi[c] = in ? ldg_nc2(prm.biases + g_row + g) : uint16_t(0);
+          } else {
+            const int g32 = (kb * C::BK + c * 32) / 32;  // the chunk's 32-code span
+            const bool in = row_ok && kb < kb1 && g32 < prm.K / 32;
+            sc[c] = !in ? uint16_t(0) : FMT == 2 ? ldg_nc2(sbrow + 2 * g32) : static_cast<uint16_t>(sbrow[g32]);
+            bi[c] = 0;
+          }
         }
       };
       // a queue of the next kSbAhead turns' scales, shifted by one each turn
@@ -758,7 +795,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int i = 0; i < BITS; ++i) wv[i] = wrow[c * BITS + i];
           }
           uint32_t packed_cols[16];
-          dequant_chunk_f16<BITS>(wv, sc[c], bi[c], packed_cols);
+          if constexpr (FMT == 0) {
+            dequant_chunk_f16<BITS>(wv, sc[c], bi[c], packed_cols);
+          } else if constexpr (FMT == 1) {
+            const __half2 f = __float2half2_rn(pow2f_exact(static_cast<int>(sc[c]) - 127 - bexp));
+            dequant_chunk_e2m1(reinterpret_cast<const uint32_t(&)[4]>(wv), f, f, packed_cols);
+          } else if constexpr (FMT == 2) {
+            const float p2 = pow2f_exact(-bexp);
+            const __half2 f0 = __float2half2_rn(e4m3_value(sc[c] & 0xFFu) * p2);
+            const __half2 f1 = __float2half2_rn(e4m3_value(sc[c] >> 8) * p2);
+            dequant_chunk_e2m1(reinterpret_cast<const uint32_t(&)[4]>(wv), f0, f1, packed_cols);
+          } else {
+            const __half2 f = __float2half2_rn(pow2f_exact(static_cast<int>(sc[c]) - 127 - bexp + 8));
+            dequant_chunk_e4m3(reinterpret_cast<const uint32_t(&)[8]>(wv), f, packed_cols);
+          }
           tmem_st16(a_tmem + c * 16, packed_cols);
         }
         tmem_st_wait();
@@ -787,7 +837,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float rsi = __shfl_sync(0xffffffffu, rs, i);
-          *reinterpret_cast<__nv_bfloat16 *>(ebox + i * 64 + lane * 2) = __float2bfloat16_rn(v[i] * rsi);
+          const float out = FMT == 0 ? v[i] * rsi : v[i] * rsi * rowfac;  // (rowfac: this lane's W row)
+          *reinterpret_cast<__nv_bfloat16 *>(ebox + i * 64 + lane * 2) = __float2bfloat16_rn(out);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the copy engine reads the box
         __syncwarp();
@@ -1240,10 +1291,13 @@ cudaError_t launch_grouped_t(const uint16_t *x, int64_t T, int64_t K, const uint
   return cudaGetLastError();
 }
 
-template <int BITS, int BN>
+// FMT 0: affine (scales, biases per G codes); 1 mxfp4, 2 nvfp4, 3 mxfp8: the
+// block scales in bscales (rows of K/32 bytes, K/16 for nvfp4) and nvfp4's
+// tensor scale in gscale (device memory).
+template <int BITS, int BN, int FMT = 0>
 cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed, const uint16_t *scales,
                         const uint16_t *biases, int64_t N, int G, uint16_t *y, void *workspace, size_t ws_bytes,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const uint8_t *bscales = nullptr, const float *gscale = nullptr) {
   using C = PairCfg<BITS, BN>;
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -1297,9 +1351,9 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   Params prm;
   prm.offsets = nullptr;
   prm.E = 0;
-  prm.bscales = nullptr;
-  prm.sb_row = 0;
-  prm.gscale = nullptr;
+  prm.bscales = FMT == 0 ? nullptr : bscales;
+  prm.sb_row = FMT == 0 ? 0 : static_cast<int>(FMT == 2 ? K / 16 : K / 32);
+  prm.gscale = FMT == 0 ? nullptr : gscale;
   prm.scales = reinterpret_cast<const __half *>(scales);
   prm.biases = reinterpret_cast<const __half *>(biases);
   prm.row_scale = row_scale;
@@ -1307,11 +1361,11 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   prm.M = static_cast<int>(M);
   prm.N = static_cast<int>(N);
   prm.K = static_cast<int>(K);
-  prm.G = G;
-  prm.Gn = static_cast<int>(K / G);
+  prm.G = FMT == 0 ? G : 32;
+  prm.Gn = static_cast<int>(K / prm.G);
   prm.m_tiles = static_cast<int>((M + BN - 1) / BN);
   prm.n_tiles = static_cast<int>((N + 255) / 256);
-  const int64_t w_bytes = N * K * BITS / 8 + 4 * N * (K / G);
+  const int64_t w_bytes = N * K * BITS / 8 + (FMT == 0 ? 4 * N * (K / G) : static_cast<int64_t>(prm.sb_row) * N);
   prm.n_fastest = (2 * M * K > w_bytes) ? 1 : 0;
 #ifdef AQ_QMM_FORCE_ORDER
   if (AQ_QMM_FORCE_ORDER == 0 || AQ_QMM_FORCE_ORDER == 1) prm.n_fastest = AQ_QMM_FORCE_ORDER;
@@ -1320,14 +1374,14 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   prm.partial = partial;
   prm.arrivals = arrivals;
 
-  auto kern = ksplit > 1 ? qmm_pair_kernel<BITS, BN, true> : qmm_pair_kernel<BITS, BN, false>;
+  auto kern = ksplit > 1 ? qmm_pair_kernel<BITS, BN, true, FMT> : qmm_pair_kernel<BITS, BN, false, FMT>;
   static thread_local int cached_dev = -1;
   static thread_local int sms = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev != cached_dev) {
-    for (auto k : {qmm_pair_kernel<BITS, BN, true>, qmm_pair_kernel<BITS, BN, false>})
+    for (auto k : {qmm_pair_kernel<BITS, BN, true, FMT>, qmm_pair_kernel<BITS, BN, false, FMT>})
       if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)) != cudaSuccess)
         return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -1394,7 +1448,16 @@ cudaError_t launch_bits(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
 // device), 3 mxfp8; token tile 64 / 128 / 256 by M as the affine single CTA.
 cudaError_t launch_qmm_block_scaled(int fmt, const uint16_t *x, int64_t M, int64_t K, const uint32_t *packed,
                                     const uint8_t *scales, const float *gscale, int64_t N, uint16_t *y, void *ws,
-                                    cudaStream_t s) {
+                                    size_t ws_bytes, cudaStream_t s) {
+  // M > 128 (and N % 8 == 0): the CTA pair, as for the affine format
+  if (qmm::pick_shape_is_pair(M, N)) {
+    switch (fmt) {
+      case 1: return qmm::launch_pair<4, 256, 1>(x, M, K, packed, nullptr, nullptr, N, 32, y, ws, ws_bytes, s, scales, gscale);
+      case 2: return qmm::launch_pair<4, 256, 2>(x, M, K, packed, nullptr, nullptr, N, 16, y, ws, ws_bytes, s, scales, gscale);
+      case 3: return qmm::launch_pair<8, 256, 3>(x, M, K, packed, nullptr, nullptr, N, 32, y, ws, ws_bytes, s, scales, gscale);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   const int bn = M <= 64 ? 64 : M <= 128 ? 128 : 256;
 #define AQ_FMT_BN(F)                                                                                               \
   switch (bn) {                                                                                                    \
