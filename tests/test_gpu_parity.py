@@ -199,8 +199,11 @@ def test_quantize_mse_full_size_sampled_rows(G, bits):
 
 # ----------------------------------------------------------------------------- gather matmul, prefill form
 
+# (the last four: segments of more than 192 rows on average, on the CTA-pair kernel)
 @pytest.mark.parametrize("T,E,N,K,G,bits", [(40, 4, 256, 512, 64, 4), (100, 3, 128, 1024, 32, 3),
-                                            (17, 5, 64, 256, 128, 8), (9, 2, 48, 512, 64, 2)])
+                                            (17, 5, 64, 256, 128, 8), (9, 2, 48, 512, 64, 2),
+                                            (700, 3, 264, 512, 64, 4), (600, 2, 520, 1024, 32, 8),
+                                            (650, 3, 256, 1024, 32, 3), (500, 2, 136, 768, 128, 2)])
 def test_gather_grouped_matches_oracle_per_token(T, E, N, K, G, bits):
     ws = [weights(N, K, 600 + e, True) for e in range(E)]
     qs = [oracle.quantize(w, G, bits) for w in ws]
@@ -245,6 +248,32 @@ def test_gather_grouped_mixtral_prefill_bitequal_per_expert():
             ref = aq.aq_matmul(x[rows].contiguous(), P[e], S[e], B[e], 64, 4)
             assert torch.equal(y[rows], ref), e
     torch.cuda.synchronize()
+
+
+def test_gather_grouped_pair_bitequal_per_expert():
+    """Segments of ~512 rows (E = 4, 2048 rows) run on the CTA-pair kernel in one
+    launch; each expert's rows equal aq_matmul of that expert over the same rows
+    (also the CTA pair, same tiles), bit for bit, including the boxes that
+    cross a segment end (stored row by row)."""
+    E, N, K, T = 4, 1024, 1024, 2048
+    packed, scales, biases = [], [], []
+    for e in range(E):
+        w = torch.from_numpy(synth.weights(N, K, 710 + e, True)).cuda()
+        p, s, b = aq.aq_quantize(w, 64, 4)
+        packed.append(p); scales.append(s); biases.append(b)
+        del w
+    P, S, B = torch.stack(packed), torch.stack(scales), torch.stack(biases)
+    rng = np.random.default_rng(11)
+    ex = rng.integers(0, E, T).astype(np.int32)
+    x = _x_gpu(activations_bits(T, K, 711))
+    y = aq.aq_gather_matmul(x, torch.from_numpy(ex).cuda(), P, S, B, 64, 4, grouped=True)
+    for e in range(E):
+        rows = torch.from_numpy(np.nonzero(ex == e)[0]).cuda()
+        assert len(rows) > 128
+        ref = aq.aq_matmul(x[rows].contiguous(), P[e], S[e], B[e], 64, 4)
+        assert torch.equal(y[rows], ref), e
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() == 0
 
 
 # ----------------------------------------------------------------------------- mxfp4 (block-scaled fp4)

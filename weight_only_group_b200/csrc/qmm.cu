@@ -556,6 +556,8 @@ struct PairItem {
 template <bool SPLIT>
 struct PairCursor {
   uint32_t w, P, T, KB, ks;
+  AQ_DEVICE PairCursor(const Params &prm, int pair, int npairs, int KB_, int tiles)
+      : w(pair), P(npairs), T(tiles), KB(KB_), ks(SPLIT ? prm.ksplit : 1) {}
   AQ_DEVICE PairCursor(const Params &prm, int pair, int npairs, int KB_)
       : w(pair), P(npairs), T(prm.m_tiles * prm.n_tiles), KB(KB_), ks(SPLIT ? prm.ksplit : 1) {}
   AQ_DEVICE bool next(PairItem &it) {
@@ -586,7 +588,10 @@ __host__ __device__ constexpr uint32_t idesc_pair(int bn) {
 
 // SPLIT: the launch cuts tiles into K parts (Params::ksplit > 1).  FMT as in
 // qmm_kernel: 0 affine, 1 mxfp4, 2 nvfp4, 3 mxfp8.
-template <int BITS, int BN, bool SPLIT, int FMT = 0>
+// GROUPED (affine, unsplit): the M token rows are E segments with device
+// offsets (Params::offsets), segment e multiplied by expert e (rows e*N .. of
+// the stacked W); token tiles of 256 never straddle a segment.
+template <int BITS, int BN, bool SPLIT, int FMT = 0, bool GROUPED = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     qmm_pair_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap w_map,
                     const __grid_constant__ CUtensorMap y_map, Params prm) {
@@ -606,6 +611,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_rank();
   const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
   const int KB = (prm.K + C::BK - 1) / C::BK;
+  static_assert(!GROUPED || (!SPLIT && FMT == 0), "grouped launches are affine and unsplit");
+  // grouped: [E + 1] segment offsets and [E + 1] prefix sums of their 256-token tiles
+  int *seg = reinterpret_cast<int *>(smem + S * C::STAGE_BYTES + 512 + C::EPI_BYTES);
+  int *mtp = seg + kGroupMaxE + 2;
+  if (GROUPED && threadIdx.x == 64) {  // warp 2 (otherwise idle) reads the segments
+    int run = 0;
+    for (int e = 0; e <= prm.E; ++e) {
+      seg[e] = __ldg(prm.offsets + e);
+      mtp[e] = run;
+      if (e < prm.E) run += (__ldg(prm.offsets + e + 1) - seg[e] + 255) / 256;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -629,6 +646,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // both CTAs' barriers and TMEM exist before either uses the other's
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = GROUPED ? prm.n_tiles * mtp[prm.E] : prm.m_tiles * prm.n_tiles;
+  // Tile origin: first token m0, first W row n0 within the expert (grouped) or
+  // the matrix, the expert's first row of the stacked W, and the end of the
+  // tile's token rows.
+  auto origin = [&](int tile, int &m0, int &n0, int64_t &wbase, int &mend) {
+    if constexpr (GROUPED) {
+      const int nt = tile % prm.n_tiles, mg = tile / prm.n_tiles;
+      int lo = 0, hi = prm.E - 1;  // the segment e with mtp[e] <= mg < mtp[e + 1]
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (mtp[mid] <= mg) lo = mid; else hi = mid - 1;
+      }
+      m0 = seg[lo] + (mg - mtp[lo]) * 256;
+      n0 = nt * 256;
+      wbase = static_cast<int64_t>(lo) * prm.N;
+      mend = seg[lo + 1];
+    } else {
+      tile_origin(prm, tile, BN, 256, m0, n0);
+      wbase = 0;
+      mend = prm.M;
+    }
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer (each CTA)
@@ -637,13 +676,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&w_map)) : "memory");
       uint32_t it = 0;
       bool ok = true;
-      PairCursor<SPLIT> cur(prm, pair, npairs, KB);
+      PairCursor<SPLIT> cur = GROUPED ? PairCursor<SPLIT>(prm, pair, npairs, KB, total_tiles) : PairCursor<SPLIT>(prm, pair, npairs, KB);
       PairItem item;
       while (ok && cur.next(item)) {
-        int m0, n0;
-        tile_origin(prm, item.tile, BN, 256, m0, n0);
+        int m0, n0, mend;
+        int64_t wbase;
+        origin(item.tile, m0, n0, wbase, mend);
         const int xrow = m0 + static_cast<int>(rank) * C::XH;
-        const int wrow = n0 + static_cast<int>(rank) * 128;
+        const int wrow = static_cast<int>(wbase) + n0 + static_cast<int>(rank) * 128;
         for (int kb = item.kb0; kb < item.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t r = it / S;
@@ -667,7 +707,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_pair(BN);
       uint32_t it = 0, t = 0;
       bool ok = true;
-      PairCursor<SPLIT> cur(prm, pair, npairs, KB);
+      PairCursor<SPLIT> cur = GROUPED ? PairCursor<SPLIT>(prm, pair, npairs, KB, total_tiles) : PairCursor<SPLIT>(prm, pair, npairs, KB);
       PairItem item;
       for (; ok && cur.next(item); ++t) {
         const int kb0 = item.kb0;
@@ -704,17 +744,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *ebox = smem + S * C::STAGE_BYTES + 512 + widx * 2048;  // this warp's output box
     uint32_t it0 = 0, t = 0;
     bool ok = true;
-    PairCursor<SPLIT> cur(prm, pair, npairs, KB);
+    PairCursor<SPLIT> cur = GROUPED ? PairCursor<SPLIT>(prm, pair, npairs, KB, total_tiles) : PairCursor<SPLIT>(prm, pair, npairs, KB);
     PairItem item;
     for (; ok && cur.next(item); ++t) {
       const int tile = item.tile, kb0 = item.kb0, kb1 = item.kb1;
-      int m0, n0;
-      tile_origin(prm, tile, BN, 256, m0, n0);
+      int m0, n0, mend;
+      int64_t wbase;
+      origin(tile, m0, n0, wbase, mend);
       const uint32_t itb = it0;  // ring position of this item's first K block
       it0 += static_cast<uint32_t>(kb1 - kb0);
       const int n = n0 + static_cast<int>(rank) * 128 + row;
       const bool row_ok = n < prm.N;
-      const int64_t g_row = static_cast<int64_t>(row_ok ? n : 0) * prm.Gn;
+      const int64_t g_row = (wbase + (row_ok ? n : 0)) * prm.Gn;
       // Block-scaled formats: this row's power of two 2^-B (from its largest
       // scale byte; positive E4M3 and E8M0 order like their bits) keeps every
       // dequantized value within fp16; the epilogue multiplies by 2^B (nvfp4:
@@ -832,6 +873,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // (token-major, the layout of y) and written by one TMA store, which
       // clips rows past N and tokens past M.
       auto emit_box = [&](int col, const float (&v)[32], float rs) {
+        if (GROUPED && m0 + col + 32 > mend) {
+          // the box crosses the end of the segment: plain stores of its rows in
+          // the segment (the tokens past it belong to the next expert)
+          if (m0 + col >= mend) return;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float rsi = __shfl_sync(0xffffffffu, rs, i);
+            if (m0 + col + i < mend && bn0 + lane < prm.N)
+              prm.y[static_cast<int64_t>(m0 + col + i) * prm.N + bn0 + lane] = __float2bfloat16_rn(v[i] * rsi);
+          }
+          return;
+        }
         if (lane == 0) bulk_wait_read<0>();  // the store that last read this box is done with it
         __syncwarp();
 #pragma unroll
@@ -842,7 +895,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the copy engine reads the box
         __syncwarp();
-        if (lane == 0 && bn0 < prm.N && m0 + col < prm.M) {  // (a box wholly past the edges is not stored)
+        if (lane == 0 && bn0 < prm.N && m0 + col < mend) {  // (a box wholly past the edges is not stored)
           tma_store_2d(&y_map, ebox, bn0, m0 + col);
           bulk_commit();
         }
@@ -1393,6 +1446,93 @@ cudaError_t launch_pair(const uint16_t *x, int64_t M, int64_t K, const uint32_t 
   return cudaGetLastError();
 }
 
+// Grouped launch on CTA pairs (see launch_grouped_t): token tiles of 256 rows
+// per segment, W tiles of 256 rows of the segment's expert.
+template <int BITS>
+cudaError_t launch_pair_grouped(const uint16_t *x, int64_t T, int64_t K, const uint32_t *packed,
+                                const uint16_t *scales, const uint16_t *biases, int64_t E, int64_t N, int G,
+                                const int32_t *offsets, uint16_t *y, void *workspace, cudaStream_t stream) {
+  using C = PairCfg<BITS, 256>;
+  constexpr size_t kSmem = C::SMEM_BYTES + kGroupTabBytes;
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+  __half *x16 = reinterpret_cast<__half *>(ws);
+  float *row_scale = reinterpret_cast<float *>(ws + round256(T * K * 2));
+  x_to_f16_rows_kernel<BITS><<<static_cast<unsigned>(T), kPrepThreads, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16 *>(x), static_cast<int>(K), x16, row_scale);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
+  CUtensorMap x_map, w_map, y_map;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(C::XH)};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&x_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const int64_t P = K * BITS / 32;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(P), static_cast<cuuint64_t>(E * N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(P) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(C::BKW), 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&w_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(packed), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(T)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&y_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  Params prm;
+  prm.offsets = offsets;
+  prm.E = static_cast<int>(E);
+  prm.bscales = nullptr;
+  prm.sb_row = 0;
+  prm.gscale = nullptr;
+  prm.scales = reinterpret_cast<const __half *>(scales);
+  prm.biases = reinterpret_cast<const __half *>(biases);
+  prm.row_scale = row_scale;
+  prm.y = reinterpret_cast<__nv_bfloat16 *>(y);
+  prm.M = static_cast<int>(T);
+  prm.N = static_cast<int>(N);
+  prm.K = static_cast<int>(K);
+  prm.G = G;
+  prm.Gn = static_cast<int>(K / G);
+  prm.m_tiles = 0;  // from the offsets, on the device
+  prm.n_tiles = static_cast<int>((N + 255) / 256);
+  prm.n_fastest = 1;
+  prm.ksplit = 1;
+  auto kern = qmm_pair_kernel<BITS, 256, false, 0, true>;
+  static thread_local int cached_dev = -1;
+  static thread_local int sms = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != cached_dev) {
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem))) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cached_dev = dev;
+  }
+  // at most ceil(T / 256) + E token tiles (each segment adds at most one partial tile)
+  const int64_t bound = static_cast<int64_t>(prm.n_tiles) * ((T + 255) / 256 + E);
+  const int pairs = static_cast<int>(std::min<int64_t>(bound, std::max(1, sms / 2)));
+  kern<<<2 * pairs, kThreads, kSmem, stream>>>(x_map, w_map, y_map, prm);
+  return cudaGetLastError();
+}
+
 // Tile shape.  Measured on B200 (4-bit, G = 64, TFLOP/s, pair / one CTA at
 // 256 / one CTA at 128 tokens): M = 512, 2048, 8192 at K = 4096, N = 14336:
 // 532/540/344, 742/744/461, 901/895/510; at K = 14336, N = 4096: 501/383/485,
@@ -1480,6 +1620,15 @@ cudaError_t launch_qmm_grouped(const uint16_t *x, int64_t T, int64_t K, const ui
                                const int32_t *offsets, uint16_t *y, void *ws, cudaStream_t s) {
   if (E < 1 || E > qmm::kGroupMaxE) return cudaErrorInvalidValue;
   const int64_t mean = (T + E - 1) / E;
+  // segments of more than 192 rows on average: CTA pairs (y rows of whole 16-byte units for the output stores)
+  if (mean > 192 && N % 8 == 0) {
+    switch (bits) {
+      case 2: return qmm::launch_pair_grouped<2>(x, T, K, packed, scales, biases, E, N, G, offsets, y, ws, s);
+      case 3: return qmm::launch_pair_grouped<3>(x, T, K, packed, scales, biases, E, N, G, offsets, y, ws, s);
+      case 4: return qmm::launch_pair_grouped<4>(x, T, K, packed, scales, biases, E, N, G, offsets, y, ws, s);
+      default: return qmm::launch_pair_grouped<8>(x, T, K, packed, scales, biases, E, N, G, offsets, y, ws, s);
+    }
+  }
   const int bn = mean <= 96 ? 64 : mean <= 384 ? 128 : 256;
 #define AQ_GROUPED(B, N_)                                                                                          \
   case N_: return qmm::launch_grouped_t<B, N_>(x, T, K, packed, scales, biases, E, N, G, offsets, y, ws, s);
