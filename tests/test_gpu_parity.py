@@ -1100,6 +1100,33 @@ def test_block_scaled_prefill_matches_oracle(M, K, N):
     assert aq.aq_device_fault() == 0
 
 
+def test_block_scaled_prefill_bench_shape_sampled():
+    """mxfp4, nvfp4 and mxfp8 prefill at the benchmarked shape (M = 2048, K = 4096,
+    N = 14336, the CTA-pair kernel as timed): 12 sampled token rows, every
+    column, against the oracle's exact product of those rows."""
+    M, K, N = 2048, 4096, 14336
+    w = weights(N, K, 1210, True)
+    xb = activations_bits(M, K, 1211)
+    x = _x_gpu(xb)
+    rows = sample_rows(M, 12, 1212)
+    sel = torch.from_numpy(rows).cuda()
+    p_ref, s_ref, p, s = _mx_gpu(w)
+    y = aq.aq_mxfp4_matmul(x, p, s)
+    torch.cuda.synchronize()
+    _assert_close(y[sel], oracle.mxfp4_matmul(xb[rows], p_ref, s_ref), "mxfp4 prefill bench shape")
+    del p, s, y
+    p_ref, s_ref, p, s = _mx8_gpu(w)
+    y = aq.aq_mxfp8_matmul(x, p, s)
+    torch.cuda.synchronize()
+    _assert_close(y[sel], oracle.mxfp8_matmul(xb[rows], p_ref, s_ref), "mxfp8 prefill bench shape")
+    del p, s, y
+    p_ref, s_ref, g_ref, p, s, g = _nv_gpu(w)
+    y = aq.aq_nvfp4_matmul(x, p, s, g)
+    torch.cuda.synchronize()
+    _assert_close(y[sel], oracle.nvfp4_matmul(xb[rows], p_ref, s_ref, g_ref), "nvfp4 prefill bench shape")
+    assert aq.aq_device_fault() == 0
+
+
 def test_block_scaled_prefill_special_weights():
     """Zero groups, subnormal and huge block scales and one-signed rows: every
     row's power of two keeps its largest groups exact in fp16."""
