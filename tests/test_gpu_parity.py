@@ -250,6 +250,24 @@ def test_gather_grouped_mixtral_prefill_bitequal_per_expert():
     torch.cuda.synchronize()
 
 
+def test_gather_grouped_bench_shape_sampled():
+    """The MoE prefill point of the benchmark: 8 experts of W[14336, 4096] (4-bit
+    G64), 4096 routed rows, one CTA-pair launch; 16 sampled rows, every column,
+    against the oracle with each row's expert."""
+    E, N, K, T, G, bits = 8, 14336, 4096, 4096, 64, 4
+    parts, (P, S, B) = _stacked_experts(E, N, K, 720, G, bits)  # quantized by the oracle
+    rng = np.random.default_rng(13)
+    ex = rng.integers(0, E, T).astype(np.int32)
+    xb = activations_bits(T, K, 721)
+    y = aq.aq_gather_matmul(_x_gpu(xb), torch.from_numpy(ex).cuda(), P, S, B, G, bits, grouped=True)
+    torch.cuda.synchronize()
+    assert aq.aq_device_fault() == 0
+    for r in sample_rows(T, 16, 722):
+        e = int(ex[r])
+        y_ref = oracle.matmul(xb[r:r + 1], *parts[e], G, bits)
+        _assert_close(y[r:r + 1], y_ref, f"grouped bench shape row {r} (expert {e})")
+
+
 def test_gather_grouped_pair_bitequal_per_expert():
     """Segments of ~512 rows (E = 4, 2048 rows) run on the CTA-pair kernel in one
     launch; each expert's rows equal aq_matmul of that expert over the same rows
@@ -563,6 +581,14 @@ def test_qmv_many_tokens_long_k(M, bits, G):
     one launch each; every token's row matches the oracle."""
     _matmul_case(M, 14336, 200, bits, G, 9500 + M + bits, "auto")
     assert aq.aq_dispatch(M, 200, 14336, G, bits) == aq.AQ_KERNEL_QMV
+
+
+@pytest.mark.parametrize("M", (5, 8))
+def test_qmv_many_tokens_long_k_bench_shape_sampled(M):
+    """The long-K small-M curve's shape (K = 14336, N = 4096, 4-bit G64) at M = 5
+    and 8, run as token chunks: every token row on 400 sampled columns against
+    the oracle."""
+    _matmul_case(M, 14336, 4096, 4, 64, 9600 + M, "auto", full=False, n_rows=M)
 
 
 def test_qmv_extreme_activation_rows():
