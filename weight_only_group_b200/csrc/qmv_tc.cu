@@ -1159,8 +1159,8 @@ static int64_t unit_codes(int64_t M, int64_t nch) {
   return AQ_QMV_SMALL_UNIT;
 }
 
-static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt = 0,
-                      bool dual = false, int stage_target = kStageTarget, int64_t unit_limit = 0) {
+static bool make_plan_uncached(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt,
+                               bool dual, int stage_target, int64_t unit_limit) {
   if (!(bits == 2 || bits == 4 || bits == 8) || !(G == 32 || G == 64 || G == 128)) return false;
   if (M < 1 || M > 8 || N < 1 || K < 1 || K % (8 * G) != 0) return false;
   // mxfp4 scale rows are K/32 bytes: a TMA row stride must be a multiple of 16 bytes
@@ -1232,6 +1232,36 @@ static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms,
   a.wait_cycles = kWaitCycles;
   a.stall = 0;
   return place(pl, M, U, a.job[0].tok_stride, Gn, a.job[0].parts, dual, sms, N);
+}
+
+// A plan is a function of its arguments alone, and one decode call computes the
+// same plan several times (dispatch, validation, the launch): keep the last
+// few per thread.
+static bool make_plan(int64_t M, int64_t N, int64_t K, int G, int bits, int sms, Plan &pl, int fmt = 0,
+                      bool dual = false, int stage_target = kStageTarget, int64_t unit_limit = 0) {
+  struct Entry {
+    int64_t M, N, K, unit_limit;
+    int G, bits, sms, fmt, stage_target;
+    bool dual, used, ok;
+    Plan pl;
+  };
+  constexpr int kEntries = 8;
+  static thread_local Entry cache[kEntries];
+  static thread_local int next = 0;
+  for (Entry &c : cache)
+    if (c.used && c.M == M && c.N == N && c.K == K && c.unit_limit == unit_limit && c.G == G && c.bits == bits &&
+        c.sms == sms && c.fmt == fmt && c.stage_target == stage_target && c.dual == dual) {
+      if (c.ok) pl = c.pl;
+      return c.ok;
+    }
+  Entry &c = cache[next];
+  next = (next + 1) % kEntries;
+  c.M = M; c.N = N; c.K = K; c.unit_limit = unit_limit;
+  c.G = G; c.bits = bits; c.sms = sms; c.fmt = fmt; c.stage_target = stage_target; c.dual = dual;
+  c.ok = make_plan_uncached(M, N, K, G, bits, sms, c.pl, fmt, dual, stage_target, unit_limit);
+  c.used = true;
+  if (c.ok) pl = c.pl;
+  return c.ok;
 }
 using Maps = JobMaps<1>;
 
