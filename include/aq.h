@@ -144,7 +144,10 @@ aq_status aq_dequantize_f32(const uint32_t *packed, const uint16_t *scales, cons
  *    point, rint(x * 2^e) with 2^e the power of two that puts the group's
  *    largest |x| in [2^13, 2^14) (error <= 2^-14 of that largest |x| per
  *    element); group dot products exact in int32, then
- *    y += scale * 2^-e * dot + bias * sum(x) in fp32.  Other shapes and 3-bit
+ *    y += scale * 2^-e * dot + bias * sum(x) in fp32.  Where the staged
+ *    activations of all M tokens would take more than 120 KB of shared memory
+ *    ((2K + 64) bytes per token: M > 4 at K = 14336), the tokens run as
+ *    balanced chunks, one launch each, in stream order.  Other shapes and 3-bit
  *    codes: CUDA cores, fp32 arithmetic on the exact codes.
  *  - QMM otherwise: tcgen05 tensor cores on fp16 operands, weights
  *    fp16_rn(fp32_rn(code*scale + bias)), activations scaled per row by an
@@ -259,7 +262,7 @@ aq_status aq_matmul_qmm_static(const uint16_t *x_bf16, int64_t M, int64_t K,
 
 /* aq_matmul with an explicit kernel.  AQ_KERNEL_QMV and AQ_KERNEL_QMV_TCGEN05
  * return AQ_ERR_UNSUPPORTED when M > 8 or the shared-memory staging of x does
- * not fit; AQ_KERNEL_QMM and AQ_KERNEL_QMM_NOWS return AQ_ERR_UNSUPPORTED when
+ * not fit, even in token chunks; AQ_KERNEL_QMM and AQ_KERNEL_QMM_NOWS return AQ_ERR_UNSUPPORTED when
  * K*bits is not a multiple of 128.  AQ_KERNEL_QMM takes its workspace from
  * the library's stream-ordered pool (see Ownership above); AQ_KERNEL_QMM_NOWS
  * allocates nothing (each token row's power-of-two scale is kept, until the
@@ -315,7 +318,9 @@ aq_status aq_gather_matmul(const uint16_t *x_bf16, int64_t T, int64_t K, const u
  * rows are scattered back after the matmul.  With E <= 256 and K*bits a
  * multiple of 128 the matmul is ONE tensor-core launch over every expert's
  * segment, whose tile count the kernel reads from the device-side segment
- * offsets: the call is asynchronous and can be captured in a CUDA graph.
+ * offsets (on CTA pairs with 256-token tiles when the segments average more
+ * than 192 rows, else on single CTAs): the call is asynchronous and can be
+ * captured in a CUDA graph.
  * Otherwise each expert's rows go through aq_matmul's per-shape kernels; the
  * host then reads the E per-expert counts once, so the call synchronizes its
  * stream (and cannot be captured).  Workspace (offsets, positions, x and y in expert order, the QMM
