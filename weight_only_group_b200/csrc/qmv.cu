@@ -508,7 +508,13 @@ static cudaError_t qmv_stream_launch(const uint16_t *x, int64_t K, const uint32_
 
 // Rows per consumer warp per stage: 2 shares each activation read between two
 // rows; wide codes (8-bit) and M > 4 keep one row to stay within registers.
-__host__ __device__ constexpr int stream_rows(int bits, int64_t M) { return (M <= 4 && bits != 8) ? 2 : 1; }
+// W rows a consumer warp takes per stage.  3-bit codes at M <= 2: four
+// (measured on B200, K = 8192, N = 28672, G = 32 / 64 / 128: M = 1 2730 / 2506
+// / 2397 GB/s against 2730 / 2330 / 2200 with two, M = 2 2055 / 1954 / 1827
+// against 1814 / 1917 / 1842).
+__host__ __device__ constexpr int stream_rows(int bits, int64_t M) {
+  return bits == 3 && M <= 2 ? 4 : (M <= 4 && bits != 8) ? 2 : 1;
+}
 template <int BITS, int M>
 struct StreamRows {
   static constexpr int value = stream_rows(BITS, M);
