@@ -623,9 +623,12 @@ def section_qmm(args, aq, torch, dev, stream, peaks):
         reps = max(2, args.qmm_reps * 8192 // (4 * M))
         ms = timed_graph(torch, stream, lambda i: aq.aq_matmul(x, p, s, b, G, BITS, out=y), 2, reps)
         tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        # the K split runs exactly when the workspace holds more than the activations' part
+        act_bytes = -(-M * K * 2 // 256) * 256 + -(-M * 4 // 256) * 256
         out[f"M{M}_K{K}_N{N}"] = {"TFLOP/s": round(tf, 1), "us": round(ms * 1e3, 2),
                                   "frac_of_burst": round(tf / peaks["bf16_tflops"], 4),
-                                  "frac_of_sustained": round(tf / peaks["bf16_tflops_sustained"], 4)}
+                                  "frac_of_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                                  "k_split": aq.aq_matmul_workspace_bytes(M, N, K, G, BITS) > act_bytes}
         del x, y
     wcache.clear()
     torch.cuda.empty_cache()
